@@ -1,0 +1,305 @@
+"""Pins for the CPU oracle (no GPU).
+
+The oracle is checked against things other than itself:
+  * closed forms derived independently with SO(3) Bloch-vector rotations
+    (L = 0, theta = 0, Rz-only, L = 1, L = 2);
+  * a dense brute-force simulator built here from scipy's matrix exponential and
+    numpy kron products (n <= 5), with gradients by the exact parameter-shift rule;
+  * parameter shift and central finite differences of the oracle's own forward
+    pass against its adjoint gradient (the adjoint code path is separate);
+  * invariants: norm, |E| <= 1, the backward walk returning |0...0>, and the
+    exact zeros of the light cone of Z0;
+  * bf16 rounding against torch's float32 -> bfloat16 conversion.
+
+The method: Kawase, "Fast and memory-efficient classical simulation of quantum
+machine learning via forward and backward gate fusion" -- Deep-dive blog §1.2
+(E(theta), adjoint gradient, lambda recursion) and §2.1 (HEA of Rx, Ry, Rz + CZ).
+"""
+import numpy as np
+import pytest
+import scipy.linalg
+
+import oracle
+from adjoint_gradients_b200.inputs import WORKLOADS, make_inputs, random_case
+
+# ----------------------------------------------------------------------------- helpers
+
+PAULI = {
+    0: np.array([[0, 1], [1, 0]], dtype=complex),
+    1: np.array([[0, -1j], [1j, 0]], dtype=complex),
+    2: np.array([[1, 0], [0, -1]], dtype=complex),
+}
+
+
+def dense_rot(p, t):
+    return scipy.linalg.expm(-0.5j * t * PAULI[p])
+
+
+def dense_on(u, q, n):
+    """Full 2^n operator of a one-qubit u on qubit q (qubit 0 = least significant bit)."""
+    return np.kron(np.eye(1 << (n - 1 - q)), np.kron(u, np.eye(1 << q)))
+
+
+def dense_cz(q1, q2, n):
+    idx = np.arange(1 << n)
+    both = ((idx >> q1) & 1) & ((idx >> q2) & 1)
+    return np.diag(np.where(both == 1, -1.0, 1.0)).astype(complex)
+
+
+def dense_state(x, theta):
+    n = x.shape[0]
+    psi = np.zeros(1 << n, dtype=complex)
+    psi[0] = 1
+    for q in range(n):
+        psi = dense_on(dense_rot(1, x[q]), q, n) @ psi
+    for l in range(theta.shape[0]):
+        for q in range(n):
+            for a in range(3):
+                psi = dense_on(dense_rot(a, theta[l, q, a]), q, n) @ psi
+        for q in range(n - 1):
+            psi = dense_cz(q, q + 1, n) @ psi
+    return psi
+
+
+def dense_E(x, theta):
+    n = x.shape[0]
+    psi = dense_state(x, theta)
+    return float(np.real(np.conj(psi) @ (dense_on(PAULI[2], 0, n) @ psi)))
+
+
+def bloch_rx(v, a):
+    x, y, z = v
+    return np.array([x, y * np.cos(a) - z * np.sin(a), y * np.sin(a) + z * np.cos(a)])
+
+
+def bloch_ry(v, b):
+    x, y, z = v
+    return np.array([x * np.cos(b) + z * np.sin(b), y, -x * np.sin(b) + z * np.cos(b)])
+
+
+def bloch_rz(v, c):
+    x, y, z = v
+    return np.array([x * np.cos(c) - y * np.sin(c), x * np.sin(c) + y * np.cos(c), z])
+
+
+def bloch_layer(v, ang):
+    return bloch_rz(bloch_ry(bloch_rx(v, ang[0]), ang[1]), ang[2])
+
+
+def closed_form_E(x, theta):
+    """<Z0> for L <= 2 by Bloch vectors: the CZ(0,1) of layer 0 dephases qubit 0's
+    x and y components by <Z1>; no other CZ changes qubit 0's reduced state, and
+    the last CZ ladder commutes with Z0."""
+    L = theta.shape[0]
+    v0 = np.array([np.sin(x[0]), 0.0, np.cos(x[0])])
+    if L == 0:
+        return v0[2]
+    v0 = bloch_layer(v0, theta[0, 0])
+    if L == 1:
+        return v0[2]
+    assert L == 2
+    z1 = 1.0
+    if x.shape[0] > 1:
+        z1 = bloch_layer(np.array([np.sin(x[1]), 0.0, np.cos(x[1])]), theta[0, 1])[2]
+    v0 = np.array([v0[0] * z1, v0[1] * z1, v0[2]])
+    return bloch_layer(v0, theta[1, 0])[2]
+
+
+def shift_grad_E(fwd, x, theta):
+    """Parameter-shift dE_b/dtheta for every parameter: [B][L][n][3] (exact for exp(-itP/2))."""
+    B = x.shape[0]
+    out = np.zeros((B,) + theta.shape)
+    for idx in np.ndindex(theta.shape):
+        tp = theta.copy()
+        tm = theta.copy()
+        tp[idx] += np.pi / 2
+        tm[idx] -= np.pi / 2
+        out[(slice(None),) + idx] = 0.5 * (fwd(x, tp) - fwd(x, tm))
+    return out
+
+
+# ----------------------------------------------------------------------------- closed forms
+
+
+@pytest.mark.parametrize("n", [1, 2, 5, 9])
+def test_no_layers_is_cos_x0(n):
+    x, _, _ = random_case(11 + n, 6, n, 0)
+    E = oracle.forward(x, np.zeros((0, n, 3)))
+    np.testing.assert_allclose(E, np.cos(x[:, 0]), atol=1e-14)
+
+
+@pytest.mark.parametrize("n,L", [(3, 1), (6, 4), (10, 3)])
+def test_zero_angles_is_cos_x0(n, L):
+    x, _, _ = random_case(21 + n, 5, n, L)
+    E = oracle.forward(x, np.zeros((L, n, 3)))
+    np.testing.assert_allclose(E, np.cos(x[:, 0]), atol=1e-13)
+
+
+@pytest.mark.parametrize("n,L", [(4, 2), (7, 5)])
+def test_rz_only_is_cos_x0_and_rz_grads_vanish(n, L):
+    x, theta, _ = random_case(31 + n, 4, n, L)
+    theta[..., 0] = 0.0
+    theta[..., 1] = 0.0
+    E = oracle.forward(x, theta)
+    np.testing.assert_allclose(E, np.cos(x[:, 0]), atol=1e-13)
+    grad, _ = oracle.adjoint(x, theta, np.ones(4))
+    np.testing.assert_allclose(grad[..., 2], 0.0, atol=1e-13)
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 8])
+def test_one_layer_closed_form(n):
+    x, theta, _ = random_case(41 + n, 5, n, 1)
+    E = oracle.forward(x, theta)
+    a, b = theta[0, 0, 0], theta[0, 0, 1]
+    x0 = x[:, 0]
+    np.testing.assert_allclose(E, np.cos(x0) * np.cos(a) * np.cos(b) - np.sin(x0) * np.sin(b), atol=1e-13)
+    # gradient seeded with g_b = 1 for one sample at a time
+    for bi in range(x.shape[0]):
+        g = np.zeros(x.shape[0])
+        g[bi] = 1.0
+        grad, _ = oracle.adjoint(x, theta, g)
+        want = np.zeros_like(theta)
+        want[0, 0, 0] = -np.sin(a) * np.cos(b) * np.cos(x0[bi])
+        want[0, 0, 1] = -np.cos(a) * np.sin(b) * np.cos(x0[bi]) - np.cos(b) * np.sin(x0[bi])
+        np.testing.assert_allclose(grad, want, atol=1e-13)
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 6])
+def test_two_layer_closed_form(n):
+    x, theta, _ = random_case(51 + n, 6, n, 2)
+    E = oracle.forward(x, theta)
+    want = np.array([closed_form_E(x[b], theta) for b in range(x.shape[0])])
+    np.testing.assert_allclose(E, want, atol=1e-13)
+
+
+def test_rotation_conventions():
+    # Ry(t)|0>: <Z> = cos t (encoding with one qubit, no layers) ...
+    t = np.array([[0.3], [1.1], [2.9]])
+    np.testing.assert_allclose(oracle.forward(t, np.zeros((0, 1, 3))), np.cos(t[:, 0]), atol=1e-15)
+    # ... and Rx(a) after encoding x=0 gives <Z> = cos a; Ry(b) gives cos b.
+    th = np.zeros((1, 1, 3))
+    th[0, 0, 0] = 0.7
+    np.testing.assert_allclose(oracle.forward(np.zeros((1, 1)), th), [np.cos(0.7)], atol=1e-15)
+    # Ry(pi/2)|0> then Ry(b): <Z> = cos(pi/2 + b) = -sin b pins the sign of Ry.
+    th = np.zeros((1, 1, 3))
+    th[0, 0, 1] = 0.4
+    np.testing.assert_allclose(oracle.forward(np.full((1, 1), np.pi / 2), th), [-np.sin(0.4)], atol=1e-15)
+    # Rx(a) on Ry(pi/2)|0> = |+>: X axis is invariant under Rx, so <Z> = 0 for any a.
+    th = np.zeros((1, 1, 3))
+    th[0, 0, 0] = 1.3
+    np.testing.assert_allclose(oracle.forward(np.full((1, 1), np.pi / 2), th), [0.0], atol=1e-15)
+
+
+# ----------------------------------------------------------------------------- brute force
+
+
+@pytest.mark.parametrize("n,L,seed", [(1, 2, 1), (2, 3, 2), (3, 2, 3), (4, 2, 4), (5, 3, 5)])
+def test_dense_brute_force_state_energy_gradient(n, L, seed):
+    x, theta, y = random_case(seed, 3, n, L)
+    E, psi = oracle.forward(x, theta, want_state=True)
+    for b in range(3):
+        ref = dense_state(x[b], theta)
+        np.testing.assert_allclose(psi[b], ref, atol=1e-12)
+        assert abs(E[b] - dense_E(x[b], theta)) < 1e-12
+    g = oracle.loss_seed(E, y)
+    grad, E2 = oracle.adjoint(x, theta, g)
+    np.testing.assert_allclose(E2, E, atol=1e-14)
+    dense_fwd = lambda xx, tt: np.array([dense_E(xx[b], tt) for b in range(xx.shape[0])])
+    want = np.einsum("b,b...->...", g, shift_grad_E(dense_fwd, x, theta))
+    np.testing.assert_allclose(grad, want, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- parameter shift / FD
+
+
+def test_parameter_shift_tiny_workload():
+    w = WORKLOADS["tiny_4q_L2"]
+    x, theta, y = make_inputs(w)
+    grad, E = oracle.adjoint(x, theta, np.zeros(w.B))
+    g = oracle.loss_seed(E, y)
+    grad, _ = oracle.adjoint(x, theta, g)
+    want = np.einsum("b,b...->...", g, shift_grad_E(oracle.forward, x, theta))
+    np.testing.assert_allclose(grad, want, atol=1e-10)
+    assert w.params == 24 and grad.size == 24
+
+
+def test_parameter_shift_12q_workload_all_params():
+    w = WORKLOADS["hea_12q_L10"]
+    x, theta, y = make_inputs(w)
+    x = x[:2]  # two samples, every one of the 360 parameters
+    E = oracle.forward(x, theta)
+    g = oracle.loss_seed(E, y[:2])
+    grad, _ = oracle.adjoint(x, theta, g)
+    want = np.einsum("b,b...->...", g, shift_grad_E(oracle.forward, x, theta))
+    np.testing.assert_allclose(grad, want, atol=1e-10)
+
+
+def test_central_finite_difference_of_mean_loss():
+    x, theta, y = random_case(77, 4, 6, 4)
+
+    def loss(t):
+        return np.mean((oracle.forward(x, t) - y) ** 2)
+
+    E = oracle.forward(x, theta)
+    grad, _ = oracle.adjoint(x, theta, oracle.loss_seed(E, y))
+    h = 1e-5
+    rng = np.random.default_rng(5)
+    for _ in range(20):
+        idx = tuple(rng.integers(0, s) for s in theta.shape)
+        tp, tm = theta.copy(), theta.copy()
+        tp[idx] += h
+        tm[idx] -= h
+        fd = (loss(tp) - loss(tm)) / (2 * h)
+        assert abs(fd - grad[idx]) < 1e-8, (idx, fd, grad[idx])
+
+
+# ----------------------------------------------------------------------------- invariants
+
+
+def test_norm_bounds_and_return_to_zero_state():
+    x, theta, _ = random_case(91, 3, 9, 6)
+    E, psi = oracle.forward(x, theta, want_state=True)
+    np.testing.assert_allclose(np.sum(np.abs(psi) ** 2, axis=1), 1.0, atol=1e-13)
+    assert np.all(np.abs(E) <= 1.0 + 1e-14)
+    _, _, psi0 = oracle.adjoint(x, theta, np.ones(3), want_state=True)
+    ref = np.zeros_like(psi0)
+    ref[:, 0] = 1.0
+    np.testing.assert_allclose(psi0, ref, atol=1e-12)
+
+
+@pytest.mark.parametrize("n,L", [(6, 3), (8, 5), (5, 9)])
+def test_light_cone_zeros(n, L):
+    """A rotation in layer l (0-based) on qubit q cannot reach Z0 if q > L-1-l, and
+    the Rz on the edge qubit q = L-1-l only meets Z from the CZ spread.  These
+    gradients are zero in exact arithmetic; the fp64 walk leaves ~1e-17."""
+    x, theta, _ = random_case(101 + n, 3, n, L)
+    grad, _ = oracle.adjoint(x, theta, np.array([0.3, -1.0, 0.7]))
+    for l in range(L):
+        edge = L - 1 - l
+        for q in range(n):
+            if q > edge:
+                np.testing.assert_allclose(grad[l, q], 0.0, atol=1e-14)
+            elif q == edge:
+                assert abs(grad[l, q, 2]) < 1e-14
+                assert np.max(np.abs(grad[l, q, :2])) > 1e-6
+
+
+def test_bf16_rounding_matches_torch():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(9)
+    vals = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32),
+        (rng.standard_normal(2000) * 1e-39).astype(np.float32),  # subnormals
+        np.array([0.0, -0.0, 1.0, -1.0, np.inf, -np.inf, 3.4028235e38, -3.4028235e38,
+                  1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, 1.0 + 2.0 ** -9, 1.0 - 2.0 ** -9], dtype=np.float32),
+    ])
+    # exact halfway cases: low 16 bits == 0x8000
+    halves = (rng.integers(0, 2 ** 15, 500, dtype=np.uint32) << 16 | 0x8000).astype(np.uint32).view(np.float32)
+    vals = np.concatenate([vals, halves[np.isfinite(halves)]])
+    ours = oracle.bf16_round(vals)
+    ref = torch.from_numpy(vals).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(ours, ref)
+    nan = oracle.bf16_round(np.array([np.nan], dtype=np.float32))
+    assert (nan[0] & 0x7F80) == 0x7F80 and (nan[0] & 0x7F) != 0
+    back = oracle.bf16_widen(ours)
+    np.testing.assert_array_equal(oracle.bf16_round(back), ours)
