@@ -1,0 +1,507 @@
+// api.cu -- the C ABI of libqml (declared in include/qml.h).
+//
+// Host-side only: argument checks, the pass schedule, the workspace layout,
+// and the order of kernel launches.  Every arithmetic step of the forward and
+// backward paths runs in the kernels of kernels.cu.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "kernels.cuh"
+#include "plan.hpp"
+#include "qml.h"
+
+using namespace qml;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
+
+struct Layout {
+  size_t status, passes, phases, ops, slot_pass, slot_index;
+  size_t coef_fwd, coef_inv, enc, dummy, exp_partial, partials, ckpt;
+  size_t base_total;
+  // host-step extras
+  size_t h_psi, h_lam, h_x, h_theta, h_y, h_E, h_g, h_loss, h_grad;
+  size_t host_total;
+};
+
+class DeviceGuard {
+ public:
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&old_) != cudaSuccess) old_ = -1;
+    if (old_ != dev) cudaSetDevice(dev);
+    dev_ = dev;
+  }
+  ~DeviceGuard() {
+    if (old_ >= 0 && old_ != dev_) cudaSetDevice(old_);
+  }
+
+ private:
+  int old_ = -1, dev_ = 0;
+};
+
+}  // namespace
+
+struct qml_ctx {
+  qml_config cfg{};
+  int device = 0;
+  Plan plan;
+  std::vector<DevPass> dpass;
+  std::vector<DevPhase> dphase;
+  std::vector<DevOp> dop;
+  int prog_bytes = 0;
+  size_t smem = 0;
+  bool probed = false, dev_ok = false;
+  int sms = 148, grid_fwd = 0, grid_bwd = 0;
+  char* ws = nullptr;
+  size_t ws_bytes = 0;
+  Layout lay{};
+  std::vector<int> ckpt_batch;  // batch last written to each slot, -1 = never
+  long long N = 0;
+};
+
+namespace {
+
+int prog_bytes_of(const qml_ctx* c) {
+  int mx = 0;
+  for (const DevPass& p : c->dpass) {
+    int b = (int)((sizeof(DevPass) + 15) & ~size_t(15)) + p.nphases * (int)sizeof(DevPhase) +
+            p.nops * (int)sizeof(DevOp);
+    mx = std::max(mx, b);
+  }
+  return (mx + 15) & ~15;
+}
+
+// Probe the device once: shared-memory opt-in, occupancy, persistent grid size.
+void ensure_device(qml_ctx* c) {
+  if (c->probed) return;
+  c->probed = true;
+  c->smem = pass_smem_bytes(c->prog_bytes, c->plan.max_slots);
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, c->device) != cudaSuccess) {
+    cudaGetLastError();
+    c->dev_ok = false;
+    c->grid_fwd = c->sms * 3;
+    c->grid_bwd = c->sms * 2;
+    return;
+  }
+  DeviceGuard g(c->device);
+  c->sms = prop.multiProcessorCount;
+  int of = 0, ob = 0;
+  if (set_pass_smem_attr(c->smem) != cudaSuccess || pass_occupancy(false, c->smem, &of) != cudaSuccess ||
+      pass_occupancy(true, c->smem, &ob) != cudaSuccess || of < 1 || ob < 1) {
+    cudaGetLastError();
+    c->dev_ok = false;
+    c->grid_fwd = c->sms * 3;
+    c->grid_bwd = c->sms * 2;
+    return;
+  }
+  c->grid_fwd = c->sms * of;
+  c->grid_bwd = c->sms * ob;
+  c->dev_ok = true;
+}
+
+void compute_layout(qml_ctx* c) {
+  const int n = c->cfg.n_qubits, L = c->cfg.n_layers, Bm = c->cfg.max_batch;
+  const long long N = 1ll << n;
+  const size_t U = (size_t)(Bm + 1) / 2;
+  Layout& l = c->lay;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o = align_up(o + bytes);
+    return at;
+  };
+  l.status = take(64);
+  l.passes = take(sizeof(DevPass) * c->dpass.size());
+  l.phases = take(sizeof(DevPhase) * c->dphase.size());
+  l.ops = take(sizeof(DevOp) * std::max<size_t>(1, c->dop.size()));
+  l.slot_pass = take(sizeof(int) * (size_t)L * n);
+  l.slot_index = take(sizeof(int) * (size_t)L * n);
+  l.coef_fwd = take(sizeof(float4) * 4 * (size_t)L * n);
+  l.coef_inv = take(sizeof(float4) * 4 * (size_t)L * n);
+  l.enc = take(sizeof(float2) * 2 * U * n);
+  l.dummy = take(sizeof(float2) * (size_t)N);
+  l.exp_partial = take(sizeof(double) * expect_partial_count(Bm, n));
+  size_t nparts = 0;
+  for (const DevPass& p : c->dpass) nparts += (size_t)c->grid_bwd * p.nslots * 3;
+  l.partials = take(sizeof(float) * std::max<size_t>(1, nparts));
+  const size_t slot_elem = c->cfg.storage == QML_STORE_BF16 ? 4 : 8;
+  l.ckpt = take(slot_elem * (size_t)c->plan.n_ckpt * Bm * (size_t)N + 16);
+  l.base_total = o;
+  l.h_psi = take(sizeof(float2) * (size_t)Bm * N);
+  l.h_lam = take(sizeof(float2) * (size_t)Bm * N);
+  l.h_x = take(sizeof(float) * (size_t)Bm * n);
+  l.h_theta = take(sizeof(float) * (size_t)L * n * 3);
+  l.h_y = take(sizeof(float) * (size_t)Bm);
+  l.h_E = take(sizeof(float) * (size_t)Bm);
+  l.h_g = take(sizeof(float) * (size_t)Bm);
+  l.h_loss = take(sizeof(float) * 4);
+  l.h_grad = take(sizeof(float) * (size_t)L * n * 3);
+  l.host_total = o;
+  // gradient partial offsets per pass
+  long long off = 0;
+  for (DevPass& p : c->dpass) {
+    p.partial_off = off;
+    off += (long long)c->grid_bwd * p.nslots * 3;
+  }
+}
+
+bool misaligned(const void* p, size_t a) { return ((uintptr_t)p) % a != 0; }
+
+qml_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QML_OK : QML_ERR_CUDA; }
+
+template <class T>
+T* at(qml_ctx* c, size_t off) {
+  return reinterpret_cast<T*>(c->ws + off);
+}
+
+qml_status check_ready(qml_ctx* c, int B) {
+  if (!c) return QML_ERR_INVALID_ARG;
+  if (B < 1 || B > c->cfg.max_batch) return QML_ERR_INVALID_ARG;
+  if (!c->ws) return QML_ERR_WORKSPACE;
+  if (!c->dev_ok) return QML_ERR_CUDA;
+  return QML_OK;
+}
+
+qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, float2* psi,
+                       float* expect, cudaStream_t s) {
+  const int n = c->cfg.n_qubits, L = c->cfg.n_layers;
+  cudaError_t e = launch_prep_coef(theta, L, n, at<float4>(c, c->lay.coef_fwd), at<float4>(c, c->lay.coef_inv), s);
+  if (e != cudaSuccess) return QML_ERR_CUDA;
+  e = launch_prep_enc(x, B, n, at<float2>(c, c->lay.enc), s);
+  if (e != cudaSuccess) return QML_ERR_CUDA;
+  PassArgs a{};
+  a.passes = at<DevPass>(c, c->lay.passes);
+  a.phases = at<DevPhase>(c, c->lay.phases);
+  a.ops = at<DevOp>(c, c->lay.ops);
+  a.n = n;
+  a.B = B;
+  a.U = (B + 1) / 2;
+  a.N = c->N;
+  a.buf0 = psi;
+  a.buf1 = nullptr;
+  a.dummy = at<float2>(c, c->lay.dummy);
+  a.coef = at<float4>(c, c->lay.coef_fwd);
+  a.enc = at<float2>(c, c->lay.enc);
+  a.g = nullptr;
+  a.ckpt = c->ws + c->lay.ckpt;
+  a.storage = c->cfg.storage == QML_STORE_BF16 ? 1 : 0;
+  a.bmax = c->cfg.max_batch;
+  a.partials = nullptr;
+  a.status = at<unsigned>(c, c->lay.status);
+  a.smem_prog = c->prog_bytes;
+  for (size_t p = 0; p < c->dpass.size(); ++p) {
+    const DevPass& dp = c->dpass[p];
+    const long long units_per_tile = 1ll << dp.unit_bits;
+    a.pass_idx = (int)p;
+    a.n_tiles = (int)(((a.U + units_per_tile - 1) / units_per_tile) << dp.n_out);
+    e = launch_pass(false, a, c->grid_fwd, c->smem, s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+    if (dp.ckpt >= 0) c->ckpt_batch[dp.ckpt] = B;
+  }
+  if (expect) {
+    e = launch_expect(psi, B, n, at<double>(c, c->lay.exp_partial), expect, at<unsigned>(c, c->lay.status), s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+  }
+  return QML_OK;
+}
+
+qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, float2* psi,
+                        float2* lam, const float* g, float* grad, cudaStream_t s) {
+  (void)x;
+  const int n = c->cfg.n_qubits, L = c->cfg.n_layers;
+  for (int m = 0; m < c->plan.n_ckpt; ++m)
+    if (c->ckpt_batch[m] != B) return QML_ERR_CKPT_MISMATCH;
+  cudaError_t e = launch_prep_coef(theta, L, n, at<float4>(c, c->lay.coef_fwd), at<float4>(c, c->lay.coef_inv), s);
+  if (e != cudaSuccess) return QML_ERR_CUDA;
+  PassArgs a{};
+  a.passes = at<DevPass>(c, c->lay.passes);
+  a.phases = at<DevPhase>(c, c->lay.phases);
+  a.ops = at<DevOp>(c, c->lay.ops);
+  a.n = n;
+  a.B = B;
+  a.U = B;
+  a.N = c->N;
+  a.buf0 = psi;
+  a.buf1 = lam;
+  a.dummy = nullptr;
+  a.coef = at<float4>(c, c->lay.coef_inv);
+  a.enc = nullptr;
+  a.g = g;
+  a.ckpt = c->ws + c->lay.ckpt;
+  a.storage = c->cfg.storage == QML_STORE_BF16 ? 1 : 0;
+  a.bmax = c->cfg.max_batch;
+  a.partials = at<float>(c, c->lay.partials);
+  a.status = at<unsigned>(c, c->lay.status);
+  a.smem_prog = c->prog_bytes;
+  for (int p = (int)c->dpass.size() - 1; p >= 0; --p) {
+    const DevPass& dp = c->dpass[p];
+    const long long units_per_tile = 1ll << dp.unit_bits;
+    a.pass_idx = p;
+    a.n_tiles = (int)(((a.U + units_per_tile - 1) / units_per_tile) << dp.n_out);
+    e = launch_pass(true, a, c->grid_bwd, c->smem, s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+  }
+  e = launch_grad_reduce(at<DevPass>(c, c->lay.passes), at<int>(c, c->lay.slot_pass),
+                         at<int>(c, c->lay.slot_index), at<float>(c, c->lay.partials), c->grid_bwd,
+                         theta, L, n, grad, at<unsigned>(c, c->lay.status), s);
+  return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int qml_abi_version(void) { return 1; }
+
+const char* qml_status_str(qml_status s) {
+  switch (s) {
+    case QML_OK: return "ok";
+    case QML_ERR_INVALID_ARG: return "invalid argument";
+    case QML_ERR_UNSUPPORTED: return "unsupported configuration";
+    case QML_ERR_WORKSPACE: return "workspace missing or too small";
+    case QML_ERR_CUDA: return "CUDA runtime error";
+    case QML_ERR_CKPT_MISMATCH: return "checkpoint slot mismatch";
+    case QML_ERR_NUMERIC: return "non-finite value produced";
+    case QML_ERR_BOUNDS: return "device bounds check failed";
+    case QML_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+qml_status qml_create(const qml_config* cfg, int device, qml_ctx** out) {
+  if (!out) return QML_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!cfg) return QML_ERR_INVALID_ARG;
+  if (cfg->n_qubits < 1 || cfg->n_qubits > 30) return QML_ERR_INVALID_ARG;
+  if (cfg->n_layers < 1 || cfg->n_layers > 100000) return QML_ERR_INVALID_ARG;
+  if (cfg->max_batch < 1 || cfg->max_batch > (1 << 20)) return QML_ERR_INVALID_ARG;
+  if (cfg->ckpt_block < 0) return QML_ERR_INVALID_ARG;
+  if (cfg->storage != QML_STORE_FP32 && cfg->storage != QML_STORE_BF16) return QML_ERR_INVALID_ARG;
+  if (device < 0) return QML_ERR_INVALID_ARG;
+  qml_ctx* c = new (std::nothrow) qml_ctx();
+  if (!c) return QML_ERR_INVALID_ARG;
+  c->cfg = *cfg;
+  c->device = device;
+  c->N = 1ll << cfg->n_qubits;
+  std::string err = make_plan(cfg->n_qubits, cfg->n_layers, cfg->ckpt_block, &c->plan);
+  if (!err.empty()) {
+    delete c;
+    return QML_ERR_UNSUPPORTED;
+  }
+  flatten_plan(c->plan, &c->dpass, &c->dphase, &c->dop);
+  c->prog_bytes = prog_bytes_of(c);
+  c->ckpt_batch.assign(c->plan.n_ckpt, -1);
+  *out = c;
+  return QML_OK;
+}
+
+qml_status qml_destroy(qml_ctx* ctx) {
+  if (!ctx) return QML_ERR_INVALID_ARG;
+  delete ctx;
+  return QML_OK;
+}
+
+size_t qml_workspace_bytes(const qml_ctx* cctx, int B) {
+  qml_ctx* c = const_cast<qml_ctx*>(cctx);
+  if (!c || B < 1 || B > c->cfg.max_batch) return 0;
+  ensure_device(c);
+  compute_layout(c);
+  return c->lay.base_total;
+}
+
+size_t qml_host_workspace_bytes(const qml_ctx* cctx, int B) {
+  qml_ctx* c = const_cast<qml_ctx*>(cctx);
+  if (!c || B < 1 || B > c->cfg.max_batch) return 0;
+  ensure_device(c);
+  compute_layout(c);
+  return c->lay.host_total;
+}
+
+qml_status qml_set_workspace(qml_ctx* c, void* ws, size_t bytes, void* stream) {
+  if (!c || !ws) return QML_ERR_INVALID_ARG;
+  if (misaligned(ws, kAlign)) return QML_ERR_INVALID_ARG;
+  ensure_device(c);
+  if (!c->dev_ok) return QML_ERR_CUDA;
+  compute_layout(c);
+  if (bytes < c->lay.base_total) return QML_ERR_WORKSPACE;
+  DeviceGuard g(c->device);
+  c->ws = static_cast<char*>(ws);
+  c->ws_bytes = bytes;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::vector<int> sp(c->plan.slot_pass.begin(), c->plan.slot_pass.end());
+  std::vector<int> si(c->plan.slot_index.begin(), c->plan.slot_index.end());
+  cudaError_t e = cudaMemsetAsync(c->ws + c->lay.status, 0, 64, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(c->ws + c->lay.passes, c->dpass.data(), sizeof(DevPass) * c->dpass.size(),
+                        cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(c->ws + c->lay.phases, c->dphase.data(), sizeof(DevPhase) * c->dphase.size(),
+                        cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && !c->dop.empty())
+    e = cudaMemcpyAsync(c->ws + c->lay.ops, c->dop.data(), sizeof(DevOp) * c->dop.size(),
+                        cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(c->ws + c->lay.slot_pass, sp.data(), sizeof(int) * sp.size(), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(c->ws + c->lay.slot_index, si.data(), sizeof(int) * si.size(), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->ws + c->lay.dummy, 0, sizeof(float2) * (size_t)c->N, s);
+  // the host vectors above are pageable: the copies complete before return
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  std::fill(c->ckpt_batch.begin(), c->ckpt_batch.end(), -1);
+  if (e != cudaSuccess) {
+    c->ws = nullptr;
+    return QML_ERR_CUDA;
+  }
+  return QML_OK;
+}
+
+qml_status qml_init_state_encode(qml_ctx* c, const float* x, int B, float* psi, void* stream) {
+  qml_status st = check_ready(c, B);
+  if (st != QML_OK) return st;
+  if (!x || !psi || misaligned(psi, 8)) return QML_ERR_INVALID_ARG;
+  DeviceGuard g(c->device);
+  return cuda_status(launch_encode(x, B, c->cfg.n_qubits, reinterpret_cast<float2*>(psi),
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+qml_status qml_forward_expect(qml_ctx* c, const float* theta, const float* x, int B, float* psi,
+                              float* expect, void* stream) {
+  qml_status st = check_ready(c, B);
+  if (st != QML_OK) return st;
+  if (!theta || !x || !psi || !expect || misaligned(psi, 8)) return QML_ERR_INVALID_ARG;
+  DeviceGuard g(c->device);
+  return run_forward(c, theta, x, B, reinterpret_cast<float2*>(psi), expect, static_cast<cudaStream_t>(stream));
+}
+
+qml_status qml_backward_adjoint(qml_ctx* c, const float* theta, const float* x, int B, float* psi,
+                                float* lambda, const float* dLdE, float* grad, void* stream) {
+  qml_status st = check_ready(c, B);
+  if (st != QML_OK) return st;
+  if (!theta || !psi || !lambda || !dLdE || !grad || misaligned(psi, 8) || misaligned(lambda, 8))
+    return QML_ERR_INVALID_ARG;
+  if (psi == lambda) return QML_ERR_INVALID_ARG;
+  DeviceGuard g(c->device);
+  return run_backward(c, theta, x, B, reinterpret_cast<float2*>(psi), reinterpret_cast<float2*>(lambda),
+                      dLdE, grad, static_cast<cudaStream_t>(stream));
+}
+
+qml_status qml_loss_seed(qml_ctx* c, const float* expect, const float* y, int B, float* g_out,
+                         float* loss, void* stream) {
+  qml_status st = check_ready(c, B);
+  if (st != QML_OK) return st;
+  if (!expect || !y) return QML_ERR_INVALID_ARG;
+  DeviceGuard g(c->device);
+  return cuda_status(launch_loss_seed(expect, y, B, g_out, loss, static_cast<cudaStream_t>(stream)));
+}
+
+int qml_num_ckpt_slots(const qml_ctx* c) { return c ? c->plan.n_ckpt : -1; }
+
+static qml_status ckpt_common(qml_ctx* c, int slot, const void* psi, int B) {
+  qml_status st = check_ready(c, B);
+  if (st != QML_OK) return st;
+  if (!psi || misaligned(psi, 8)) return QML_ERR_INVALID_ARG;
+  if (slot < 0 || slot >= c->plan.n_ckpt) return QML_ERR_INVALID_ARG;
+  return QML_OK;
+}
+
+qml_status qml_ckpt_save(qml_ctx* c, int slot, const float* psi, int B, void* stream) {
+  qml_status st = ckpt_common(c, slot, psi, B);
+  if (st != QML_OK) return st;
+  DeviceGuard g(c->device);
+  const size_t elem = c->cfg.storage == QML_STORE_BF16 ? 4 : 8;
+  void* dst = c->ws + c->lay.ckpt + elem * (size_t)slot * c->cfg.max_batch * (size_t)c->N;
+  cudaError_t e = launch_ckpt_copy(true, reinterpret_cast<const float2*>(psi), nullptr, dst,
+                                   c->cfg.storage == QML_STORE_BF16 ? 1 : 0, (long long)B * c->N,
+                                   static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return QML_ERR_CUDA;
+  c->ckpt_batch[slot] = B;
+  return QML_OK;
+}
+
+qml_status qml_ckpt_restore(qml_ctx* c, int slot, float* psi, int B, void* stream) {
+  qml_status st = ckpt_common(c, slot, psi, B);
+  if (st != QML_OK) return st;
+  if (c->ckpt_batch[slot] != B) return QML_ERR_CKPT_MISMATCH;
+  DeviceGuard g(c->device);
+  const size_t elem = c->cfg.storage == QML_STORE_BF16 ? 4 : 8;
+  void* src = c->ws + c->lay.ckpt + elem * (size_t)slot * c->cfg.max_batch * (size_t)c->N;
+  return cuda_status(launch_ckpt_copy(false, nullptr, reinterpret_cast<float2*>(psi), src,
+                                      c->cfg.storage == QML_STORE_BF16 ? 1 : 0, (long long)B * c->N,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+qml_status qml_expect_z0(qml_ctx* c, const float* psi, int B, float* expect, void* stream) {
+  qml_status st = check_ready(c, B);
+  if (st != QML_OK) return st;
+  if (!psi || !expect || misaligned(psi, 8)) return QML_ERR_INVALID_ARG;
+  DeviceGuard g(c->device);
+  return cuda_status(launch_expect(reinterpret_cast<const float2*>(psi), B, c->cfg.n_qubits,
+                                   at<double>(c, c->lay.exp_partial), expect,
+                                   at<unsigned>(c, c->lay.status), static_cast<cudaStream_t>(stream)));
+}
+
+qml_status qml_step_host(qml_ctx* c, const float* x_h, const float* theta_h, const float* y_h, int B,
+                         float* expect_h, float* loss_h, float* grad_h, void* stream) {
+  qml_status st = check_ready(c, B);
+  if (st != QML_OK) return st;
+  if (!x_h || !theta_h || !y_h || !grad_h) return QML_ERR_INVALID_ARG;
+  if (c->ws_bytes < c->lay.host_total) return QML_ERR_WORKSPACE;
+  DeviceGuard g(c->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int n = c->cfg.n_qubits, L = c->cfg.n_layers;
+  const Layout& l = c->lay;
+  cudaError_t e = cudaMemcpyAsync(c->ws + l.h_x, x_h, sizeof(float) * (size_t)B * n, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(c->ws + l.h_theta, theta_h, sizeof(float) * (size_t)L * n * 3, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->ws + l.h_y, y_h, sizeof(float) * (size_t)B, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return QML_ERR_CUDA;
+  float2* psi = at<float2>(c, l.h_psi);
+  float2* lam = at<float2>(c, l.h_lam);
+  st = run_forward(c, at<float>(c, l.h_theta), at<float>(c, l.h_x), B, psi, at<float>(c, l.h_E), s);
+  if (st != QML_OK) return st;
+  e = launch_loss_seed(at<float>(c, l.h_E), at<float>(c, l.h_y), B, at<float>(c, l.h_g), at<float>(c, l.h_loss), s);
+  if (e != cudaSuccess) return QML_ERR_CUDA;
+  st = run_backward(c, at<float>(c, l.h_theta), at<float>(c, l.h_x), B, psi, lam, at<float>(c, l.h_g),
+                    at<float>(c, l.h_grad), s);
+  if (st != QML_OK) return st;
+  e = cudaMemcpyAsync(grad_h, c->ws + l.h_grad, sizeof(float) * (size_t)L * n * 3, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && expect_h)
+    e = cudaMemcpyAsync(expect_h, c->ws + l.h_E, sizeof(float) * (size_t)B, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && loss_h) e = cudaMemcpyAsync(loss_h, c->ws + l.h_loss, sizeof(float), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return cuda_status(e);
+}
+
+qml_status qml_sync(qml_ctx* c, void* stream) {
+  if (!c) return QML_ERR_INVALID_ARG;
+  if (!c->ws) return QML_ERR_WORKSPACE;
+  DeviceGuard g(c->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned word = 0;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemcpy(&word, c->ws + c->lay.status, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(c->ws + c->lay.status, 0, sizeof(word));
+  if (e != cudaSuccess) return QML_ERR_CUDA;
+  for (int code = 1; code < 32; ++code)
+    if (word & (1u << code)) return static_cast<qml_status>(code);
+  return QML_OK;
+}
+
+int qml_debug_schedule(const qml_ctx* c, int* out, int cap) {
+  if (!c) return -1;
+  std::vector<int> v = describe_plan(c->plan);
+  if (out)
+    for (int i = 0; i < cap && i < (int)v.size(); ++i) out[i] = v[i];
+  return (int)v.size();
+}
+
+}  // extern "C"

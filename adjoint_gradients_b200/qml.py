@@ -1,0 +1,257 @@
+"""ctypes binding of libqml (include/qml.h).
+
+Argument marshalling only: torch tensors provide device memory and streams, every
+step of the simulation runs in the library's CUDA kernels.  If the compiled
+library is missing this module raises immediately; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqml.so")
+
+QML_OK = 0
+STATUS_NAMES = {
+    0: "QML_OK", 1: "QML_ERR_INVALID_ARG", 2: "QML_ERR_UNSUPPORTED", 3: "QML_ERR_WORKSPACE",
+    4: "QML_ERR_CUDA", 5: "QML_ERR_CKPT_MISMATCH", 6: "QML_ERR_NUMERIC", 7: "QML_ERR_BOUNDS",
+    8: "QML_ERR_TIMEOUT",
+}
+STORAGE = {"fp32": 0, "bf16": 1}
+
+# every function include/qml.h declares
+EXPORTS = [
+    "qml_abi_version", "qml_status_str", "qml_create", "qml_destroy", "qml_workspace_bytes",
+    "qml_set_workspace", "qml_init_state_encode", "qml_forward_expect", "qml_backward_adjoint",
+    "qml_loss_seed", "qml_ckpt_save", "qml_ckpt_restore", "qml_num_ckpt_slots", "qml_expect_z0",
+    "qml_host_workspace_bytes", "qml_step_host", "qml_sync", "qml_debug_schedule",
+]
+
+
+class QmlError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {STATUS_NAMES.get(code, code)}")
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [("n_qubits", ctypes.c_int), ("n_layers", ctypes.c_int), ("max_batch", ctypes.c_int),
+                ("ckpt_block", ctypes.c_int), ("storage", ctypes.c_int)]
+
+
+_lib = None
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libqml.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libqml.so not found at {path}: run `python -m adjoint_gradients_b200.build`")
+    lib = ctypes.CDLL(path)
+    sig = {
+        "qml_abi_version": ([], _i),
+        "qml_status_str": ([_i], ctypes.c_char_p),
+        "qml_create": ([ctypes.POINTER(_Config), _i, ctypes.POINTER(_vp)], _i),
+        "qml_destroy": ([_vp], _i),
+        "qml_workspace_bytes": ([_vp, _i], ctypes.c_size_t),
+        "qml_host_workspace_bytes": ([_vp, _i], ctypes.c_size_t),
+        "qml_set_workspace": ([_vp, _vp, ctypes.c_size_t, _vp], _i),
+        "qml_init_state_encode": ([_vp, _vp, _i, _vp, _vp], _i),
+        "qml_forward_expect": ([_vp, _vp, _vp, _i, _vp, _vp, _vp], _i),
+        "qml_backward_adjoint": ([_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp], _i),
+        "qml_loss_seed": ([_vp, _vp, _vp, _i, _vp, _vp, _vp], _i),
+        "qml_ckpt_save": ([_vp, _i, _vp, _i, _vp], _i),
+        "qml_ckpt_restore": ([_vp, _i, _vp, _i, _vp], _i),
+        "qml_num_ckpt_slots": ([_vp], _i),
+        "qml_expect_z0": ([_vp, _vp, _i, _vp, _vp], _i),
+        "qml_step_host": ([_vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp], _i),
+        "qml_sync": ([_vp, _vp], _i),
+        "qml_debug_schedule": ([_vp, ctypes.POINTER(_i), _i], _i),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = lib
+    return lib
+
+
+def _check(code: int, what: str):
+    if code != QML_OK:
+        raise QmlError(code, what)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream_handle(stream) -> int | None:
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+@dataclass
+class StepResult:
+    expect: object
+    loss: object
+    grad: object
+
+
+class Context:
+    """One circuit shape (n qubits, L layers) on one CUDA device.
+
+    Complex states are torch float32 tensors of shape [B, 2^n, 2] (re, im), or
+    complex64 tensors of shape [B, 2^n].
+    """
+
+    def __init__(self, n_qubits: int, n_layers: int, max_batch: int, ckpt_block: int = 0,
+                 storage: str = "fp32", device: int = 0, host_step: bool = False, workspace=True):
+        self.lib = load_library()
+        self.n, self.L, self.max_batch = n_qubits, n_layers, max_batch
+        self.ckpt_block, self.storage, self.device = ckpt_block, storage, device
+        cfg = _Config(n_qubits, n_layers, max_batch, ckpt_block, STORAGE[storage])
+        h = _vp()
+        _check(self.lib.qml_create(ctypes.byref(cfg), device, ctypes.byref(h)), "qml_create")
+        self._h = h
+        self.ws = None
+        if workspace:
+            self.allocate_workspace(host_step=host_step)
+
+    # ----------------------------------------------------------------- admin
+    def close(self):
+        if getattr(self, "_h", None):
+            self.lib.qml_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def workspace_bytes(self, host_step: bool = False) -> int:
+        f = self.lib.qml_host_workspace_bytes if host_step else self.lib.qml_workspace_bytes
+        return int(f(self._h, self.max_batch))
+
+    def allocate_workspace(self, host_step: bool = False, stream=None):
+        import torch
+
+        nbytes = self.workspace_bytes(host_step)
+        self.ws = torch.empty(nbytes + 256, dtype=torch.uint8, device=f"cuda:{self.device}")
+        base = self.ws.data_ptr()
+        aligned = (base + 255) // 256 * 256
+        _check(self.lib.qml_set_workspace(self._h, aligned, nbytes, _stream_handle(stream)), "qml_set_workspace")
+
+    @property
+    def num_ckpt_slots(self) -> int:
+        return int(self.lib.qml_num_ckpt_slots(self._h))
+
+    def debug_schedule(self) -> list[int]:
+        need = self.lib.qml_debug_schedule(self._h, None, 0)
+        buf = (ctypes.c_int * need)()
+        self.lib.qml_debug_schedule(self._h, buf, need)
+        return list(buf)
+
+    def sync(self, stream=None):
+        _check(self.lib.qml_sync(self._h, _stream_handle(stream)), "qml_sync (device status)")
+
+    # ------------------------------------------------------------- compute
+    def new_state(self, B: int):
+        import torch
+
+        return torch.empty((B, 1 << self.n, 2), dtype=torch.float32, device=f"cuda:{self.device}")
+
+    @staticmethod
+    def _state_ptr(t):
+        import torch
+
+        if t.dtype == torch.complex64:
+            t = torch.view_as_real(t)
+        if t.dtype != torch.float32 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError("state must be a contiguous CUDA float32 [B, 2^n, 2] or complex64 tensor")
+        return t.data_ptr()
+
+    def encode(self, x, psi=None, stream=None):
+        B = x.shape[0]
+        psi = self.new_state(B) if psi is None else psi
+        _check(self.lib.qml_init_state_encode(self._h, _ptr(x), B, self._state_ptr(psi), _stream_handle(stream)),
+               "qml_init_state_encode")
+        return psi
+
+    def forward(self, theta, x, psi=None, expect=None, stream=None):
+        import torch
+
+        B = x.shape[0]
+        psi = self.new_state(B) if psi is None else psi
+        expect = torch.empty(B, dtype=torch.float32, device=x.device) if expect is None else expect
+        _check(self.lib.qml_forward_expect(self._h, _ptr(theta), _ptr(x), B, self._state_ptr(psi), _ptr(expect),
+                                           _stream_handle(stream)), "qml_forward_expect")
+        return psi, expect
+
+    def backward(self, theta, x, psi, lam, dLdE, grad=None, stream=None):
+        import torch
+
+        B = x.shape[0]
+        grad = torch.empty((self.L, self.n, 3), dtype=torch.float32, device=x.device) if grad is None else grad
+        _check(self.lib.qml_backward_adjoint(self._h, _ptr(theta), _ptr(x), B, self._state_ptr(psi),
+                                             self._state_ptr(lam), _ptr(dLdE), _ptr(grad), _stream_handle(stream)),
+               "qml_backward_adjoint")
+        return grad
+
+    def loss_seed(self, expect, y, stream=None):
+        import torch
+
+        B = expect.shape[0]
+        g = torch.empty(B, dtype=torch.float32, device=expect.device)
+        loss = torch.empty(1, dtype=torch.float32, device=expect.device)
+        _check(self.lib.qml_loss_seed(self._h, _ptr(expect), _ptr(y), B, _ptr(g), _ptr(loss), _stream_handle(stream)),
+               "qml_loss_seed")
+        return g, loss
+
+    def expect_z0(self, psi, expect=None, stream=None):
+        import torch
+
+        B = psi.shape[0]
+        expect = torch.empty(B, dtype=torch.float32, device=psi.device) if expect is None else expect
+        _check(self.lib.qml_expect_z0(self._h, self._state_ptr(psi), B, _ptr(expect), _stream_handle(stream)),
+               "qml_expect_z0")
+        return expect
+
+    def ckpt_save(self, slot: int, psi, stream=None):
+        _check(self.lib.qml_ckpt_save(self._h, slot, self._state_ptr(psi), psi.shape[0], _stream_handle(stream)),
+               "qml_ckpt_save")
+
+    def ckpt_restore(self, slot: int, psi, stream=None):
+        _check(self.lib.qml_ckpt_restore(self._h, slot, self._state_ptr(psi), psi.shape[0], _stream_handle(stream)),
+               "qml_ckpt_restore")
+
+    def step_host(self, x: np.ndarray, theta: np.ndarray, y: np.ndarray, out: StepResult | None = None,
+                  stream=None) -> StepResult:
+        """Forward + loss + backward from (preferably pinned) host arrays."""
+        B = x.shape[0]
+        if out is None:
+            out = StepResult(np.empty(B, np.float32), np.empty(1, np.float32),
+                             np.empty((self.L, self.n, 3), np.float32))
+
+        def hp(a):
+            if hasattr(a, "data_ptr"):
+                return a.data_ptr()
+            assert a.dtype == np.float32 and a.flags.c_contiguous
+            return a.ctypes.data
+
+        _check(self.lib.qml_step_host(self._h, hp(x), hp(theta), hp(y), B, hp(out.expect), hp(out.loss),
+                                      hp(out.grad), _stream_handle(stream)), "qml_step_host")
+        return out

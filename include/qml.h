@@ -1,0 +1,196 @@
+/*
+ * qml.h -- C ABI of libqml: batched state-vector simulation of a
+ * hardware-efficient ansatz (HEA) with a fused forward pass that ends in <Z0>
+ * and a fused adjoint backward pass that yields every parameter gradient, on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method follows the five web summaries of Kawase, "Fast and
+ * memory-efficient classical simulation of quantum machine learning via
+ * forward and backward gate fusion" (arXiv 2603.02804).  Citations below name
+ * the page and its section:
+ *   [Deep-dive]  blog "深度解析：正向与反向门融合驱动的高效量子机器学习仿真"
+ *                (hugo-pages-80e.pages.dev), sections 1.2, 1.3, 1.4, 2.1, 2.3, 3.2
+ *   [Gist-EN]    gist.science "Fast and memory-efficient classical simulation
+ *                of quantum machine learning via forward and backward gate
+ *                fusion", Technical Summary sections 2 and 4
+ *   [Gist-ES]    gist.science/es, Resumen tecnico section 2
+ *
+ * Circuit (qubit q = bit q of the amplitude index, R_P(t) = exp(-i t P/2)):
+ *   |0...0>  ->  Ry(x[b][q]) on every qubit (angle encoding)
+ *   for l in 0..L-1:  Rx(theta[l][q][0]) Ry(theta[l][q][1]) Rz(theta[l][q][2])
+ *                     on every qubit q, then CZ(q, q+1) for q = 0..n-2
+ *   E[b] = <psi_b| Z0 |psi_b>
+ *
+ * Conventions for every call:
+ *   - Complex arrays are interleaved (re, im) float32 pairs, 8-byte aligned;
+ *     state vectors are [B][2^n] complex, i.e. B * 2^n * 2 floats.
+ *   - Every pointer named *_dev is device memory owned by the caller; the
+ *     library never allocates device memory itself (no cudaMalloc, no
+ *     allocating library routine).  *_host pointers are host memory (pinned
+ *     memory makes the copies asynchronous).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy stream).
+ *   - Calls are asynchronous on `stream` unless stated otherwise.  Argument
+ *     errors are returned synchronously and nothing is launched.  Device-side
+ *     problems (a non-finite expectation value, a failed bounds check) are
+ *     latched in a status word inside the workspace and returned by the next
+ *     qml_sync().
+ *   - No call aborts, traps or throws across the ABI.
+ *   - A context is not thread-safe; concurrent calls on one context race.
+ */
+#ifndef QML_H
+#define QML_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define QML_API __attribute__((visibility("default")))
+#else
+#define QML_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QML_OK = 0,
+  QML_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, size out of range */
+  QML_ERR_UNSUPPORTED = 2,  /* configuration outside what the kernels handle */
+  QML_ERR_WORKSPACE = 3,    /* no workspace set, or too small for this batch */
+  QML_ERR_CUDA = 4,         /* a CUDA runtime call failed */
+  QML_ERR_CKPT_MISMATCH = 5,/* checkpoint slot / batch / storage mismatch */
+  QML_ERR_NUMERIC = 6,      /* a non-finite value was produced */
+  QML_ERR_BOUNDS = 7,       /* a device-side bounds check failed */
+  QML_ERR_TIMEOUT = 8       /* reserved: a bounded device wait gave up */
+} qml_status;
+
+/* Storage format of checkpoint slots: fp32 (re, im) pairs, or the
+ * memory-save mode's bfloat16 pairs (round to nearest even; compute stays
+ * fp32).  [Gist-EN] Technical Summary sec. 2 "Memory-Saving Mode";
+ * [Deep-dive] sec. 2.3. */
+typedef enum { QML_STORE_FP32 = 0, QML_STORE_BF16 = 1 } qml_storage;
+
+typedef struct {
+  int n_qubits;       /* 1 .. 30 */
+  int n_layers;       /* 1 .. 100000 */
+  int max_batch;      /* largest B any call will use, >= 1 */
+  int ckpt_block;     /* layers per checkpoint block (0 = no checkpoints);
+                         the pages find 10-20 best, [Deep-dive] sec. 2.3 */
+  qml_storage storage;
+} qml_config;
+
+typedef struct qml_ctx qml_ctx; /* opaque, host-side metadata only */
+
+/* Version of the ABI (currently 1). */
+QML_API int qml_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+QML_API const char* qml_status_str(qml_status s);
+
+/* Create a context for one circuit shape on CUDA device `device`.  Builds the
+ * host-side pass schedule; touches no device memory.  *out is NULL on error. */
+QML_API qml_status qml_create(const qml_config* cfg, int device, qml_ctx** out);
+
+/* Destroy a context.  The caller frees the workspace afterwards. */
+QML_API qml_status qml_destroy(qml_ctx* ctx);
+
+/* Device workspace bytes that calls with batch B need: the pass schedule,
+ * gate-coefficient tables, checkpoint slots for max_batch samples, reduction
+ * partials and the status word.  Returns 0 for B out of range. */
+QML_API size_t qml_workspace_bytes(const qml_ctx* ctx, int B);
+
+/* Hand the context a caller-owned device workspace (256-byte aligned,
+ * qml_workspace_bytes(ctx, max_batch) bytes).  The schedule is uploaded on
+ * `stream`; the status word is cleared. */
+QML_API qml_status qml_set_workspace(qml_ctx* ctx, void* ws_dev, size_t bytes, void* stream);
+
+/* Angle encoding only: psi_dev[b] = (x) Ry(x[b][q])|0>, the product state the
+ * forward pass starts from ([Deep-dive] sec. 1.2: psi in C^{2^n}).
+ *   x_dev    [B][n] float32
+ *   psi_dev  [B][2^n] complex64, written */
+QML_API qml_status qml_init_state_encode(qml_ctx* ctx, const float* x_dev, int B, float* psi_dev,
+                                 void* stream);
+
+/* Fused forward pass.  Builds the encoded state, applies every layer in
+ * passes that each read and write the state once ([Deep-dive] sec. 1.4 item
+ * 1; [Gist-EN] sec. 2 "Forward Path Gate Fusion"), writes checkpoint slots at
+ * block boundaries, and reduces E = <psi|Z0|psi> ([Deep-dive] sec. 1.2,
+ * E(theta); sec. 3.2, matrix-free expectation).
+ *   theta_dev  [L][n][3] float32 (Rx, Ry, Rz angle per qubit per layer)
+ *   x_dev      [B][n] float32 encoding angles
+ *   psi_dev    [B][2^n] complex64, out: final state
+ *   expect_dev [B] float32, out */
+QML_API qml_status qml_forward_expect(qml_ctx* ctx, const float* theta_dev, const float* x_dev, int B,
+                              float* psi_dev, float* expect_dev, void* stream);
+
+/* Fused adjoint backward pass.  Starting from the final state and
+ * lambda = dL/dE[b] * Z0 psi, walks the passes in reverse; inside each pass
+ * it rebuilds psi_{j-1} = U_j^dagger psi_j on chip alongside
+ * lambda_{j-1} = U_j^dagger lambda_j and accumulates
+ * dL/dtheta_j = 2 Re<lambda_j| dU_j/dtheta_j |psi_{j-1}>
+ * ([Deep-dive] sec. 1.2 adjoint-gradient equation and lambda recursion,
+ * sec. 1.4 item 2; [Gist-EN] sec. 2 "Backward Path Gate Fusion").  At each
+ * checkpoint boundary psi is reloaded from its slot.  Gradients are reduced in
+ * a fixed order (deterministic).
+ *   psi_dev     [B][2^n] complex64: in, the final state from
+ *               qml_forward_expect; clobbered (used as working memory)
+ *   lambda_dev  [B][2^n] complex64 working memory, clobbered
+ *   dLdE_dev    [B] float32, dL/dE per sample
+ *   grad_dev    [L][n][3] float32, out (overwritten): sum_b dL/dE[b] dE[b]/dtheta */
+QML_API qml_status qml_backward_adjoint(qml_ctx* ctx, const float* theta_dev, const float* x_dev, int B,
+                                float* psi_dev, float* lambda_dev, const float* dLdE_dev,
+                                float* grad_dev, void* stream);
+
+/* Loss seed for L = mean_b (E[b] - y[b])^2: g[b] = 2 (E[b] - y[b]) / B and
+ * loss = L (one float).  Any of g_dev / loss_dev may be NULL. */
+QML_API qml_status qml_loss_seed(qml_ctx* ctx, const float* expect_dev, const float* y_dev, int B,
+                         float* g_dev, float* loss_dev, void* stream);
+
+/* Store psi (standard layout) into checkpoint slot `slot` (0 ..
+ * qml_num_ckpt_slots-1) in the context's storage format, or restore it.  A
+ * restore from a slot last written with a different batch size or by nothing
+ * returns QML_ERR_CKPT_MISMATCH.  ([Gist-EN] sec. 2 "Gradient Checkpointing
+ * Integration": only block-boundary states are stored.) */
+QML_API qml_status qml_ckpt_save(qml_ctx* ctx, int slot, const float* psi_dev, int B, void* stream);
+QML_API qml_status qml_ckpt_restore(qml_ctx* ctx, int slot, float* psi_dev, int B, void* stream);
+
+/* Number of checkpoint slots the schedule uses (ceil(L / ckpt_block) - 1). */
+QML_API int qml_num_ckpt_slots(const qml_ctx* ctx);
+
+/* Standalone Z0 expectation of B states: E[b] = sum_i |psi_b(i)|^2 (+1 if
+ * bit 0 of i is 0, else -1).  [Deep-dive] sec. 3.2 (matrix-free Pauli
+ * expectation, Z part). */
+QML_API qml_status qml_expect_z0(qml_ctx* ctx, const float* psi_dev, int B, float* expect_dev,
+                         void* stream);
+
+/* One full training step through HOST buffers: copies x, theta and y from
+ * host to device, runs qml_forward_expect, qml_loss_seed and
+ * qml_backward_adjoint, and copies E, the loss and the gradient back.  Needs
+ * the larger workspace of qml_host_workspace_bytes (it also holds psi, lambda
+ * and the staged inputs).  Synchronises `stream` before returning.
+ *   x_host [B][n], theta_host [L][n][3], y_host [B]      (in)
+ *   expect_host [B], loss_host [1], grad_host [L][n][3]  (out; may be NULL
+ *   except grad_host) */
+QML_API size_t qml_host_workspace_bytes(const qml_ctx* ctx, int B);
+QML_API qml_status qml_step_host(qml_ctx* ctx, const float* x_host, const float* theta_host,
+                         const float* y_host, int B, float* expect_host, float* loss_host,
+                         float* grad_host, void* stream);
+
+/* Synchronise `stream` and return the first device-side error latched since
+ * the last qml_sync / qml_set_workspace (then clear it). */
+QML_API qml_status qml_sync(qml_ctx* ctx, void* stream);
+
+/* Schedule introspection (host only, no device work): the pass plan as a flat
+ * int array, for tests of the scheduler.  Writes at most `cap` ints into
+ * `out` and returns the number needed.  Layout: [n_passes, then per pass:
+ * geometry id, n_ops, then per op 4 ints (kind, a, b, c)].  Op kinds:
+ * 1 = register-layout exchange (a = from phase, b = to phase),
+ * 2 = rotate (a = layer, b = qubit mask over the whole register, c = unused),
+ * 3 = CZ ladder (a = layer), 4 = encode. */
+QML_API int qml_debug_schedule(const qml_ctx* ctx, int* out, int cap);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QML_H */
