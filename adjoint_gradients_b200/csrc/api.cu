@@ -59,12 +59,22 @@ struct qml_ctx {
   int prog_bytes = 0;
   size_t smem = 0;
   bool probed = false, dev_ok = false;
+  bool slow = false;  // the plan puts a batch-unit bit in registers (n < 5)
   int sms = 148, grid_fwd = 0, grid_bwd = 0;
   char* ws = nullptr;
   size_t ws_bytes = 0;
   Layout lay{};
   std::vector<int> ckpt_batch;  // batch last written to each slot, -1 = never
   long long N = 0;
+  long long launches = 0;
+  bool timing = false;
+  struct Span {
+    cudaEvent_t a, b;
+    bool bwd;
+    int passes;
+  };
+  std::vector<Span> spans;
+  std::vector<cudaEvent_t> spare;
 };
 
 namespace {
@@ -95,8 +105,8 @@ void ensure_device(qml_ctx* c) {
   DeviceGuard g(c->device);
   c->sms = prop.multiProcessorCount;
   int of = 0, ob = 0;
-  if (set_pass_smem_attr(c->smem) != cudaSuccess || pass_occupancy(false, c->smem, &of) != cudaSuccess ||
-      pass_occupancy(true, c->smem, &ob) != cudaSuccess || of < 1 || ob < 1) {
+  if (set_pass_smem_attr(c->smem) != cudaSuccess || pass_occupancy(false, c->slow, c->smem, &of) != cudaSuccess ||
+      pass_occupancy(true, c->slow, c->smem, &ob) != cudaSuccess || of < 1 || ob < 1) {
     cudaGetLastError();
     c->dev_ok = false;
     c->grid_fwd = c->sms * 3;
@@ -154,6 +164,32 @@ void compute_layout(qml_ctx* c) {
   }
 }
 
+cudaEvent_t take_event(qml_ctx* c) {
+  if (!c->spare.empty()) {
+    cudaEvent_t e = c->spare.back();
+    c->spare.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Record the start of a run of pass launches; returns false if timing is off.
+bool span_begin(qml_ctx* c, cudaStream_t s, qml_ctx::Span* sp, bool bwd) {
+  if (!c->timing) return false;
+  sp->a = take_event(c);
+  sp->b = take_event(c);
+  sp->bwd = bwd;
+  sp->passes = (int)c->dpass.size();
+  if (!sp->a || !sp->b) return false;
+  return cudaEventRecord(sp->a, s) == cudaSuccess;
+}
+
+void span_end(qml_ctx* c, cudaStream_t s, qml_ctx::Span* sp) {
+  if (cudaEventRecord(sp->b, s) == cudaSuccess) c->spans.push_back(*sp);
+}
+
 bool misaligned(const void* p, size_t a) { return ((uintptr_t)p) % a != 0; }
 
 qml_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QML_OK : QML_ERR_CUDA; }
@@ -198,16 +234,22 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
   a.partials = nullptr;
   a.status = at<unsigned>(c, c->lay.status);
   a.smem_prog = c->prog_bytes;
+  c->launches += 2;
+  qml_ctx::Span sp{};
+  const bool timed = span_begin(c, s, &sp, false);
   for (size_t p = 0; p < c->dpass.size(); ++p) {
     const DevPass& dp = c->dpass[p];
     const long long units_per_tile = 1ll << dp.unit_bits;
     a.pass_idx = (int)p;
     a.n_tiles = (int)(((a.U + units_per_tile - 1) / units_per_tile) << dp.n_out);
-    e = launch_pass(false, a, c->grid_fwd, c->smem, s);
+    e = launch_pass(false, c->slow, a, c->grid_fwd, c->smem, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
+    ++c->launches;
     if (dp.ckpt >= 0) c->ckpt_batch[dp.ckpt] = B;
   }
+  if (timed) span_end(c, s, &sp);
   if (expect) {
+    c->launches += 2;
     e = launch_expect(psi, B, n, at<double>(c, c->lay.exp_partial), expect, at<unsigned>(c, c->lay.status), s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
   }
@@ -242,14 +284,21 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
   a.partials = at<float>(c, c->lay.partials);
   a.status = at<unsigned>(c, c->lay.status);
   a.smem_prog = c->prog_bytes;
+  e = launch_bwd_init(psi, lam, g, B, n, s);
+  if (e != cudaSuccess) return QML_ERR_CUDA;
+  c->launches += 3;  // coefficient prep, lambda init, gradient reduce
+  qml_ctx::Span sp{};
+  const bool timed = span_begin(c, s, &sp, true);
   for (int p = (int)c->dpass.size() - 1; p >= 0; --p) {
     const DevPass& dp = c->dpass[p];
     const long long units_per_tile = 1ll << dp.unit_bits;
     a.pass_idx = p;
     a.n_tiles = (int)(((a.U + units_per_tile - 1) / units_per_tile) << dp.n_out);
-    e = launch_pass(true, a, c->grid_bwd, c->smem, s);
+    e = launch_pass(true, c->slow, a, c->grid_bwd, c->smem, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
+    ++c->launches;
   }
+  if (timed) span_end(c, s, &sp);
   e = launch_grad_reduce(at<DevPass>(c, c->lay.passes), at<int>(c, c->lay.slot_pass),
                          at<int>(c, c->lay.slot_index), at<float>(c, c->lay.partials), c->grid_bwd,
                          theta, L, n, grad, at<unsigned>(c, c->lay.status), s);
@@ -299,6 +348,8 @@ qml_status qml_create(const qml_config* cfg, int device, qml_ctx** out) {
   }
   flatten_plan(c->plan, &c->dpass, &c->dphase, &c->dop);
   c->prog_bytes = prog_bytes_of(c);
+  for (const DevPhase& ph : c->dphase)
+    if (ph.has_reg_unit) c->slow = true;
   c->ckpt_batch.assign(c->plan.n_ckpt, -1);
   *out = c;
   return QML_OK;
@@ -306,6 +357,11 @@ qml_status qml_create(const qml_config* cfg, int device, qml_ctx** out) {
 
 qml_status qml_destroy(qml_ctx* ctx) {
   if (!ctx) return QML_ERR_INVALID_ARG;
+  for (auto& sp : ctx->spans) {
+    cudaEventDestroy(sp.a);
+    cudaEventDestroy(sp.b);
+  }
+  for (cudaEvent_t e : ctx->spare) cudaEventDestroy(e);
   delete ctx;
   return QML_OK;
 }
@@ -400,6 +456,7 @@ qml_status qml_loss_seed(qml_ctx* c, const float* expect, const float* y, int B,
   if (st != QML_OK) return st;
   if (!expect || !y) return QML_ERR_INVALID_ARG;
   DeviceGuard g(c->device);
+  ++c->launches;
   return cuda_status(launch_loss_seed(expect, y, B, g_out, loss, static_cast<cudaStream_t>(stream)));
 }
 
@@ -469,6 +526,7 @@ qml_status qml_step_host(qml_ctx* c, const float* x_h, const float* theta_h, con
   st = run_forward(c, at<float>(c, l.h_theta), at<float>(c, l.h_x), B, psi, at<float>(c, l.h_E), s);
   if (st != QML_OK) return st;
   e = launch_loss_seed(at<float>(c, l.h_E), at<float>(c, l.h_y), B, at<float>(c, l.h_g), at<float>(c, l.h_loss), s);
+  ++c->launches;
   if (e != cudaSuccess) return QML_ERR_CUDA;
   st = run_backward(c, at<float>(c, l.h_theta), at<float>(c, l.h_x), B, psi, lam, at<float>(c, l.h_g),
                     at<float>(c, l.h_grad), s);
@@ -495,6 +553,35 @@ qml_status qml_sync(qml_ctx* c, void* stream) {
     if (word & (1u << code)) return static_cast<qml_status>(code);
   return QML_OK;
 }
+
+qml_status qml_enable_timing(qml_ctx* c, int enable) {
+  if (!c) return QML_ERR_INVALID_ARG;
+  c->timing = enable != 0;
+  return QML_OK;
+}
+
+qml_status qml_read_timing(qml_ctx* c, double* fwd_ms, long long* fwd_n, double* bwd_ms, long long* bwd_n) {
+  if (!c) return QML_ERR_INVALID_ARG;
+  DeviceGuard g(c->device);
+  double f = 0.0, b = 0.0;
+  long long nf = 0, nb = 0;
+  qml_status st = QML_OK;
+  for (auto& sp : c->spans) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(sp.b) != cudaSuccess || cudaEventElapsedTime(&ms, sp.a, sp.b) != cudaSuccess) st = QML_ERR_CUDA;
+    if (sp.bwd) { b += ms; nb += sp.passes; } else { f += ms; nf += sp.passes; }
+    c->spare.push_back(sp.a);
+    c->spare.push_back(sp.b);
+  }
+  c->spans.clear();
+  if (fwd_ms) *fwd_ms = f;
+  if (fwd_n) *fwd_n = nf;
+  if (bwd_ms) *bwd_ms = b;
+  if (bwd_n) *bwd_n = nb;
+  return st;
+}
+
+long long qml_launch_count(const qml_ctx* c) { return c ? c->launches : -1; }
 
 int qml_debug_schedule(const qml_ctx* c, int* out, int cap) {
   if (!c) return -1;

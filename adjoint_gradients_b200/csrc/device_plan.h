@@ -7,8 +7,8 @@
 namespace qml {
 
 constexpr int kTileBits = 12;  // positions per tile = 4096
-constexpr int kRegBits = 5;    // positions per thread = 32
-constexpr int kThrBits = 7;    // threads per block = 128
+constexpr int kRegBits = 4;    // positions per thread = 16
+constexpr int kThrBits = 8;    // threads per block = 256
 constexpr int kPos = 1 << kRegBits;
 constexpr int kThreads = 1 << kThrBits;
 constexpr int kTilePos = 1 << kTileBits;

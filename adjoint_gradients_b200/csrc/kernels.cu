@@ -115,12 +115,12 @@ __device__ __forceinline__ float3 rot_bwd(float2 (&re)[kPos], float2 (&im)[kPos]
 
 __device__ __forceinline__ void rot_fwd_k(int k, float2 (&re)[kPos], float2 (&im)[kPos],
                                           const Coef& c) {
+  static_assert(kRegBits == 4, "dispatch below covers four register bits");
   switch (k) {
     case 0: rot_fwd<0>(re, im, c); break;
     case 1: rot_fwd<1>(re, im, c); break;
     case 2: rot_fwd<2>(re, im, c); break;
-    case 3: rot_fwd<3>(re, im, c); break;
-    default: rot_fwd<4>(re, im, c); break;
+    default: rot_fwd<3>(re, im, c); break;
   }
 }
 
@@ -130,8 +130,7 @@ __device__ __forceinline__ float3 rot_bwd_k(int k, float2 (&re)[kPos], float2 (&
     case 0: return rot_bwd<0>(re, im, c);
     case 1: return rot_bwd<1>(re, im, c);
     case 2: return rot_bwd<2>(re, im, c);
-    case 3: return rot_bwd<3>(re, im, c);
-    default: return rot_bwd<4>(re, im, c);
+    default: return rot_bwd<3>(re, im, c);
   }
 }
 
@@ -224,7 +223,7 @@ __device__ __forceinline__ void apply_cz(float2 (&re)[kPos], float2 (&im)[kPos],
   const uint32_t qa = __popc(aq & (aq >> 1)) & 1u;
   const uint32_t m = (aq << 1) ^ (aq >> 1);
   uint32_t w = ph.cz_reg ^ (qa ? 0xffffffffu : 0u);
-  const uint32_t pat[kRegBits] = {0xAAAAAAAAu, 0xCCCCCCCCu, 0xF0F0F0F0u, 0xFF00FF00u, 0xFFFF0000u};
+  const uint32_t pat[5] = {0xAAAAAAAAu, 0xCCCCCCCCu, 0xF0F0F0F0u, 0xFF00FF00u, 0xFFFF0000u};
 #pragma unroll
   for (int k = 0; k < kRegBits; ++k)
     if (ph.reg_q[k] >= 0 && ((m >> ph.reg_q[k]) & 1u)) w ^= pat[k];
@@ -234,6 +233,32 @@ __device__ __forceinline__ void apply_cz(float2 (&re)[kPos], float2 (&im)[kPos],
     flip(re[j], sb);
     flip(im[j], sb);
   }
+}
+
+// Value of register position j for a runtime j (slow paths for n < 5 only).
+__device__ __forceinline__ float2 sel(const float2 (&v)[kPos], int j) {
+  float2 r = v[0];
+#pragma unroll
+  for (int k = 1; k < kPos; ++k)
+    if (k == j) r = v[k];
+  return r;
+}
+
+__device__ __forceinline__ void put(float2 (&v)[kPos], int j, float2 x) {
+#pragma unroll
+  for (int k = 0; k < kPos; ++k)
+    if (k == j) v[k] = x;
+}
+
+// Register position j's batch unit and qubit index, for a runtime j.
+__device__ __forceinline__ void pos_of(const RegMaps& m, const ThreadCtx& tc, int j, uint32_t* u,
+                                       uint32_t* i) {
+  uint32_t uu = tc.ut, ii = tc.aq;
+#pragma unroll
+  for (int k = 0; k < kRegBits; ++k)
+    if (j & (1 << k)) { uu += m.u[k]; ii |= m.q[k]; }
+  *u = uu;
+  *i = ii;
 }
 
 // ------------------------------------------------------------------ planes
@@ -249,11 +274,11 @@ struct Planes {
   }
 };
 
-template <bool BWD>
+template <bool BWD, bool SLOW>
 __device__ void load_planes(const PassArgs& a, const DevPhase& ph, const ThreadCtx& tc,
                             float2 (&re)[kPos], float2 (&im)[kPos]) {
   const RegMaps m = reg_maps(ph);
-  if (!ph.has_reg_unit) {
+  if constexpr (!SLOW) {
     if (tc.ut < (uint32_t)a.U) {
       const float2* p0 = Planes<BWD>::p0(a, tc.ut) + tc.aq;
       const float2* p1 = Planes<BWD>::p1(a, tc.ut) + tc.aq;
@@ -268,25 +293,26 @@ __device__ void load_planes(const PassArgs& a, const DevPhase& ph, const ThreadC
       for (int j = 0; j < kPos; ++j) re[j] = im[j] = make_float2(0.f, 0.f);
     }
   } else {
-#pragma unroll
+#pragma unroll 1
     for (int j = 0; j < kPos; ++j) {
-      const uint32_t u = tc.ut + REG_COMBINE(m.u, j, +=);
-      const uint32_t i = tc.aq | REG_COMBINE(m.q, j, |=);
+      uint32_t u, i;
+      pos_of(m, tc, j, &u, &i);
+      float2 r = make_float2(0.f, 0.f), v = r;
       if (u < (uint32_t)a.U) {
-        re[j] = Planes<BWD>::p0(a, u)[i];
-        im[j] = Planes<BWD>::p1(a, u)[i];
-      } else {
-        re[j] = im[j] = make_float2(0.f, 0.f);
+        r = Planes<BWD>::p0(a, u)[i];
+        v = Planes<BWD>::p1(a, u)[i];
       }
+      put(re, j, r);
+      put(im, j, v);
     }
   }
 }
 
-template <bool BWD>
+template <bool BWD, bool SLOW>
 __device__ void store_planes(const PassArgs& a, const DevPhase& ph, const ThreadCtx& tc,
                              const float2 (&re)[kPos], const float2 (&im)[kPos]) {
   const RegMaps m = reg_maps(ph);
-  if (!ph.has_reg_unit) {
+  if constexpr (!SLOW) {
     if (tc.ut < (uint32_t)a.U) {
       float2* p0 = Planes<BWD>::p0(a, tc.ut) + tc.aq;
       float2* p1 = Planes<BWD>::p1(a, tc.ut) + tc.aq;
@@ -298,86 +324,148 @@ __device__ void store_planes(const PassArgs& a, const DevPhase& ph, const Thread
       }
     }
   } else {
-#pragma unroll
+#pragma unroll 1
     for (int j = 0; j < kPos; ++j) {
-      const uint32_t u = tc.ut + REG_COMBINE(m.u, j, +=);
-      const uint32_t i = tc.aq | REG_COMBINE(m.q, j, |=);
+      uint32_t u, i;
+      pos_of(m, tc, j, &u, &i);
       if (u < (uint32_t)a.U) {
-        Planes<BWD>::p0(a, u)[i] = re[j];
-        Planes<BWD>::p1(a, u)[i] = im[j];
+        Planes<BWD>::p0(a, u)[i] = sel(re, j);
+        Planes<BWD>::p1(a, u)[i] = sel(im, j);
       }
     }
   }
 }
 
 // Forward, last pass: write the standard (re, im) layout of both samples.
+template <bool SLOW>
 __device__ void store_standard_fwd(const PassArgs& a, const DevPhase& ph, const ThreadCtx& tc,
                                    const float2 (&re)[kPos], const float2 (&im)[kPos]) {
   const RegMaps m = reg_maps(ph);
+  if constexpr (!SLOW) {
+    const uint32_t u = tc.ut;
+    if (u >= (uint32_t)a.U) return;
+    float2* s0 = a.buf0 + (size_t)(2 * u) * a.N + tc.aq;
+    float2* s1 = s0 + a.N;
+    const bool has1 = 2 * u + 1 < (uint32_t)a.B;
 #pragma unroll
-  for (int j = 0; j < kPos; ++j) {
-    const uint32_t u = tc.ut + REG_COMBINE(m.u, j, +=);
-    const uint32_t i = tc.aq | REG_COMBINE(m.q, j, |=);
-    if (u < (uint32_t)a.U) {
-      a.buf0[(size_t)(2 * u) * a.N + i] = make_float2(re[j].x, im[j].x);
-      if (2 * u + 1 < (uint32_t)a.B) a.buf0[(size_t)(2 * u + 1) * a.N + i] = make_float2(re[j].y, im[j].y);
+    for (int j = 0; j < kPos; ++j) {
+      const uint32_t b = REG_COMBINE(m.q, j, |=);
+      s0[b] = make_float2(re[j].x, im[j].x);
+      if (has1) s1[b] = make_float2(re[j].y, im[j].y);
     }
+  } else {
+#pragma unroll 1
+  for (int j = 0; j < kPos; ++j) {
+    uint32_t u = tc.ut, i = tc.aq;
+    for (int k = 0; k < kRegBits; ++k)
+      if (j & (1 << k)) { u += m.u[k]; i |= m.q[k]; }
+    if (u < (uint32_t)a.U) {
+      const float2 r = sel(re, j), v = sel(im, j);
+      a.buf0[(size_t)(2 * u) * a.N + i] = make_float2(r.x, v.x);
+      if (2 * u + 1 < (uint32_t)a.B) a.buf0[(size_t)(2 * u + 1) * a.N + i] = make_float2(r.y, v.y);
+    }
+  }
   }
 }
 
 // Forward: checkpoint slot (standard layout, fp32 or bf16 round-to-nearest-even).
+template <bool SLOW>
 __device__ void store_ckpt_fwd(const PassArgs& a, int slot, const DevPhase& ph,
                                const ThreadCtx& tc, const float2 (&re)[kPos],
                                const float2 (&im)[kPos], int bmax) {
   const RegMaps m = reg_maps(ph);
+  if constexpr (!SLOW) {
+    const uint32_t u = tc.ut;
+    if (u >= (uint32_t)a.U) return;
+    const size_t e0 = ((size_t)slot * bmax + 2 * u) * a.N + tc.aq;
+    const bool has1 = 2 * u + 1 < (uint32_t)a.B;
+    if (a.storage == 0) {
+      float2* s0 = reinterpret_cast<float2*>(a.ckpt) + e0;
+      float2* s1 = s0 + a.N;
 #pragma unroll
+      for (int j = 0; j < kPos; ++j) {
+        const uint32_t b = REG_COMBINE(m.q, j, |=);
+        s0[b] = make_float2(re[j].x, im[j].x);
+        if (has1) s1[b] = make_float2(re[j].y, im[j].y);
+      }
+    } else {
+      __nv_bfloat162* s0 = reinterpret_cast<__nv_bfloat162*>(a.ckpt) + e0;
+      __nv_bfloat162* s1 = s0 + a.N;
+#pragma unroll
+      for (int j = 0; j < kPos; ++j) {
+        const uint32_t b = REG_COMBINE(m.q, j, |=);
+        s0[b] = __floats2bfloat162_rn(re[j].x, im[j].x);
+        if (has1) s1[b] = __floats2bfloat162_rn(re[j].y, im[j].y);
+      }
+    }
+  } else {
+#pragma unroll 1
   for (int j = 0; j < kPos; ++j) {
-    const uint32_t u = tc.ut + REG_COMBINE(m.u, j, +=);
-    const uint32_t i = tc.aq | REG_COMBINE(m.q, j, |=);
+    uint32_t u = tc.ut, i = tc.aq;
+    for (int k = 0; k < kRegBits; ++k)
+      if (j & (1 << k)) { u += m.u[k]; i |= m.q[k]; }
     if (u >= (uint32_t)a.U) continue;
+    const float2 r = sel(re, j), v = sel(im, j);
     const size_t e0 = ((size_t)slot * bmax + 2 * u) * a.N + i;
-    const size_t e1 = e0 + a.N;
     const bool has1 = 2 * u + 1 < (uint32_t)a.B;
     if (a.storage == 0) {
       float2* s = reinterpret_cast<float2*>(a.ckpt);
-      s[e0] = make_float2(re[j].x, im[j].x);
-      if (has1) s[e1] = make_float2(re[j].y, im[j].y);
+      s[e0] = make_float2(r.x, v.x);
+      if (has1) s[e0 + a.N] = make_float2(r.y, v.y);
     } else {
       __nv_bfloat162* s = reinterpret_cast<__nv_bfloat162*>(a.ckpt);
-      s[e0] = __floats2bfloat162_rn(re[j].x, im[j].x);
-      if (has1) s[e1] = __floats2bfloat162_rn(re[j].y, im[j].y);
+      s[e0] = __floats2bfloat162_rn(r.x, v.x);
+      if (has1) s[e0 + a.N] = __floats2bfloat162_rn(r.y, v.y);
     }
+  }
   }
 }
 
 // Backward: replace the psi lanes by the checkpointed state of slot `slot`.
+template <bool SLOW>
 __device__ void restore_ckpt_bwd(const PassArgs& a, int slot, const DevPhase& ph,
                                  const ThreadCtx& tc, float2 (&re)[kPos], float2 (&im)[kPos],
                                  int bmax) {
   const RegMaps m = reg_maps(ph);
+  if constexpr (!SLOW) {
+    const uint32_t u = tc.ut;
+    if (u >= (uint32_t)a.U) return;
+    const size_t e = ((size_t)slot * bmax + u) * a.N + tc.aq;
 #pragma unroll
+    for (int j = 0; j < kPos; ++j) {
+      const uint32_t b = REG_COMBINE(m.q, j, |=);
+      float2 v;
+      if (a.storage == 0) v = reinterpret_cast<const float2*>(a.ckpt)[e + b];
+      else v = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(a.ckpt)[e + b]);
+      re[j].x = v.x;
+      im[j].x = v.y;
+    }
+  } else {
+#pragma unroll 1
   for (int j = 0; j < kPos; ++j) {
-    const uint32_t u = tc.ut + REG_COMBINE(m.u, j, +=);
-    const uint32_t i = tc.aq | REG_COMBINE(m.q, j, |=);
+    uint32_t u, i;
+    pos_of(m, tc, j, &u, &i);
     if (u >= (uint32_t)a.U) continue;
     const size_t e = ((size_t)slot * bmax + u) * a.N + i;
     float2 v;
-    if (a.storage == 0) {
-      v = reinterpret_cast<const float2*>(a.ckpt)[e];
-    } else {
-      v = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(a.ckpt)[e]);
-    }
-    re[j].x = v.x;
-    im[j].x = v.y;
+    if (a.storage == 0) v = reinterpret_cast<const float2*>(a.ckpt)[e];
+    else v = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(a.ckpt)[e]);
+    float2 r = sel(re, j), w = sel(im, j);
+    r.x = v.x;
+    w.x = v.y;
+    put(re, j, r);
+    put(im, j, w);
+  }
   }
 }
 
 // Forward: the angle-encoded product state prod_q (cos, sin)(x_q/2)[bit q].
+template <bool SLOW>
 __device__ void gen_state(const PassArgs& a, const DevPhase& ph, const ThreadCtx& tc,
                           float2 (&re)[kPos], float2 (&im)[kPos]) {
   const RegMaps m = reg_maps(ph);
   const int n = a.n;
-  if (!ph.has_reg_unit) {
+  if constexpr (!SLOW) {
     if (tc.ut >= (uint32_t)a.U) {
 #pragma unroll
       for (int j = 0; j < kPos; ++j) re[j] = im[j] = make_float2(0.f, 0.f);
@@ -406,46 +494,26 @@ __device__ void gen_state(const PassArgs& a, const DevPhase& ph, const ThreadCtx
       im[j] = make_float2(0.f, 0.f);
     }
   } else {
-#pragma unroll
+#pragma unroll 1
     for (int j = 0; j < kPos; ++j) {
-      const uint32_t u = tc.ut + REG_COMBINE(m.u, j, +=);
-      const uint32_t i = tc.aq | REG_COMBINE(m.q, j, |=);
+      uint32_t u, i;
+      pos_of(m, tc, j, &u, &i);
       float2 v = make_float2(0.f, 0.f);
       if (u < (uint32_t)a.U) {
         const float2* e = a.enc + (size_t)u * n * 2;
         v = make_float2(1.f, 1.f);
         for (int q = 0; q < n; ++q) v = __fmul2_rn(v, __ldg(&e[2 * q + ((i >> q) & 1u)]));
       }
-      re[j] = v;
-      im[j] = make_float2(0.f, 0.f);
-    }
-  }
-}
-
-// Backward, first pass: psi from the standard layout, lambda = dL/dE * Z0 psi.
-__device__ void load_standard_init_lambda(const PassArgs& a, const DevPhase& ph,
-                                          const ThreadCtx& tc, float2 (&re)[kPos],
-                                          float2 (&im)[kPos]) {
-  const RegMaps m = reg_maps(ph);
-#pragma unroll
-  for (int j = 0; j < kPos; ++j) {
-    const uint32_t u = tc.ut + REG_COMBINE(m.u, j, +=);
-    const uint32_t i = tc.aq | REG_COMBINE(m.q, j, |=);
-    if (u < (uint32_t)a.U) {
-      const float2 v = a.buf0[(size_t)u * a.N + i];
-      const float gs = (i & 1u) ? -__ldg(&a.g[u]) : __ldg(&a.g[u]);
-      re[j] = make_float2(v.x, gs * v.x);
-      im[j] = make_float2(v.y, gs * v.y);
-    } else {
-      re[j] = im[j] = make_float2(0.f, 0.f);
+      put(re, j, v);
+      put(im, j, make_float2(0.f, 0.f));
     }
   }
 }
 
 // ----------------------------------------------------------- the pass kernel
 
-template <bool BWD>
-__global__ void __launch_bounds__(kThreads, BWD ? 2 : 3) pass_kernel(const PassArgs a) {
+template <bool BWD, bool SLOW>
+__global__ void __launch_bounds__(kThreads, 2) pass_kernel(const PassArgs a) {
   const int bmax = a.bmax;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   float4* tile = reinterpret_cast<float4*>(smem_raw);
@@ -472,10 +540,11 @@ __global__ void __launch_bounds__(kThreads, BWD ? 2 : 3) pass_kernel(const PassA
     int* dso = reinterpret_cast<int*>(OPS);
     for (int i = tid; i < P->nops * 4; i += kThreads) dso[i] = so[i];
   }
-  float* acc = reinterpret_cast<float*>(prog + a.smem_prog);  // [4 warps][nslots*3]
+  constexpr int kWarps = kThreads / 32;
+  float* acc = reinterpret_cast<float*>(prog + a.smem_prog);  // [warps][nslots*3]
   const int nacc = P->nslots * 3;
   if (BWD)
-    for (int i = tid; i < 4 * nacc; i += kThreads) acc[i] = 0.f;
+    for (int i = tid; i < kWarps * nacc; i += kThreads) acc[i] = 0.f;
   __syncthreads();
 
   const int n_out = P->n_out;
@@ -494,12 +563,11 @@ __global__ void __launch_bounds__(kThreads, BWD ? 2 : 3) pass_kernel(const PassA
     {
       const ThreadCtx tc = thread_ctx(PH[cur], tid, base_q, unit_base);
       if (!BWD) {
-        if (P->gen) gen_state(a, PH[cur], tc, re, im);
-        else load_planes<false>(a, PH[cur], tc, re, im);
+        if (P->gen) gen_state<SLOW>(a, PH[cur], tc, re, im);
+        else load_planes<false, SLOW>(a, PH[cur], tc, re, im);
       } else {
-        if (P->last) load_standard_init_lambda(a, PH[cur], tc, re, im);
-        else load_planes<true>(a, PH[cur], tc, re, im);
-        if (P->ckpt >= 0) restore_ckpt_bwd(a, P->ckpt, PH[cur], tc, re, im, bmax);
+        load_planes<true, SLOW>(a, PH[cur], tc, re, im);
+        if (P->ckpt >= 0) restore_ckpt_bwd<SLOW>(a, P->ckpt, PH[cur], tc, re, im, bmax);
       }
     }
 
@@ -522,9 +590,9 @@ __global__ void __launch_bounds__(kThreads, BWD ? 2 : 3) pass_kernel(const PassA
         }
       }
       const ThreadCtx tc = thread_ctx(PH[cur], tid, base_q, unit_base);
-      if (P->ckpt >= 0) store_ckpt_fwd(a, P->ckpt, PH[cur], tc, re, im, bmax);
-      if (P->last) store_standard_fwd(a, PH[cur], tc, re, im);
-      else store_planes<false>(a, PH[cur], tc, re, im);
+      if (P->ckpt >= 0) store_ckpt_fwd<SLOW>(a, P->ckpt, PH[cur], tc, re, im, bmax);
+      if (P->last) store_standard_fwd<SLOW>(a, PH[cur], tc, re, im);
+      else store_planes<false, SLOW>(a, PH[cur], tc, re, im);
     } else {
       for (int oi = P->nops - 1; oi >= 0; --oi) {
         const DevOp op = OPS[oi];
@@ -555,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, BWD ? 2 : 3) pass_kernel(const PassA
       }
       if (!P->gen) {
         const ThreadCtx tc = thread_ctx(PH[cur], tid, base_q, unit_base);
-        store_planes<true>(a, PH[cur], tc, re, im);
+        store_planes<true, SLOW>(a, PH[cur], tc, re, im);
       }
     }
   }
@@ -563,7 +631,12 @@ __global__ void __launch_bounds__(kThreads, BWD ? 2 : 3) pass_kernel(const PassA
   if (BWD) {
     __syncthreads();
     float* out = a.partials + P->partial_off + (size_t)blockIdx.x * nacc;
-    for (int i = tid; i < nacc; i += kThreads) out[i] = acc[i] + acc[nacc + i] + acc[2 * nacc + i] + acc[3 * nacc + i];
+    for (int i = tid; i < nacc; i += kThreads) {
+      float v = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) v += acc[w * nacc + i];
+      out[i] = v;
+    }
   }
 }
 
@@ -696,6 +769,21 @@ __global__ void loss_seed_kernel(const float* E, const float* y, int B, float* g
   if (threadIdx.x == 0 && loss) *loss = (float)(red[0] / B);
 }
 
+// Start of the adjoint walk: lambda = dL/dE[b] Z0 psi, written together with
+// psi into the plane layout the backward passes use: plane 0 (the psi buffer,
+// in place) holds (Re psi, Re lambda), plane 1 (the lambda buffer) holds
+// (Im psi, Im lambda).
+__global__ void bwd_init_kernel(float2* psi, float2* lam, const float* g, int B, int n) {
+  const long long N = 1ll << n;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)B * N) return;
+  const int b = (int)(idx >> n);
+  const float gs = (idx & 1) ? -__ldg(&g[b]) : __ldg(&g[b]);
+  const float2 v = psi[idx];
+  psi[idx] = make_float2(v.x, gs * v.x);
+  lam[idx] = make_float2(v.y, gs * v.y);
+}
+
 // Encoded product state, standard layout, one thread per amplitude.
 __global__ void encode_kernel(const float* x, int B, int n, float2* psi) {
   const long long N = 1ll << n;
@@ -728,24 +816,34 @@ __global__ void ckpt_copy_kernel(bool save, const float2* in, float2* out, void*
 }  // namespace
 
 size_t pass_smem_bytes(int prog_bytes, int max_slots) {
-  return (size_t)kTilePos * sizeof(float4) + (size_t)prog_bytes + (size_t)4 * max_slots * 3 * sizeof(float);
+  return (size_t)kTilePos * sizeof(float4) + (size_t)prog_bytes + (size_t)(kThreads / 32) * max_slots * 3 * sizeof(float);
 }
 
 cudaError_t set_pass_smem_attr(size_t smem) {
-  cudaError_t e = cudaFuncSetAttribute(pass_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(pass_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const int v = (int)smem;
+  cudaError_t e = cudaFuncSetAttribute(pass_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, v);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(pass_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, v);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(pass_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, v);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(pass_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, v);
+  return e;
 }
 
-cudaError_t pass_occupancy(bool backward, size_t smem, int* blocks_per_sm) {
+cudaError_t pass_occupancy(bool backward, bool slow, size_t smem, int* blocks_per_sm) {
   if (backward)
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true>, kThreads, smem);
-  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false>, kThreads, smem);
+    return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, true>, kThreads, smem)
+                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, false>, kThreads, smem);
+  return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, true>, kThreads, smem)
+              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, false>, kThreads, smem);
 }
 
-cudaError_t launch_pass(bool backward, const PassArgs& a, int grid, size_t smem, cudaStream_t s) {
-  if (backward) pass_kernel<true><<<grid, kThreads, smem, s>>>(a);
-  else pass_kernel<false><<<grid, kThreads, smem, s>>>(a);
+cudaError_t launch_pass(bool backward, bool slow, const PassArgs& a, int grid, size_t smem, cudaStream_t s) {
+  if (backward) {
+    if (slow) pass_kernel<true, true><<<grid, kThreads, smem, s>>>(a);
+    else pass_kernel<true, false><<<grid, kThreads, smem, s>>>(a);
+  } else {
+    if (slow) pass_kernel<false, true><<<grid, kThreads, smem, s>>>(a);
+    else pass_kernel<false, false><<<grid, kThreads, smem, s>>>(a);
+  }
   return cudaGetLastError();
 }
 
@@ -799,6 +897,12 @@ cudaError_t launch_encode(const float* x, int B, int n, float2* psi, cudaStream_
   const long long tot = (long long)B << n;
   const long long blocks = (tot + 255) / 256;
   encode_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, B, n, psi);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_init(float2* psi, float2* lam, const float* g, int B, int n, cudaStream_t s) {
+  const long long tot = (long long)B << n;
+  bwd_init_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(psi, lam, g, B, n);
   return cudaGetLastError();
 }
 

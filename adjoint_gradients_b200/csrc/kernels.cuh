@@ -33,9 +33,11 @@ struct PassArgs {
 
 size_t pass_smem_bytes(int prog_bytes, int max_slots);
 
-cudaError_t launch_pass(bool backward, const PassArgs& a, int grid, size_t smem, cudaStream_t s);
+// `slow`: some register bit indexes a batch unit (only when n < 5); the
+// generic per-position code then replaces the single-unit fast path.
+cudaError_t launch_pass(bool backward, bool slow, const PassArgs& a, int grid, size_t smem, cudaStream_t s);
 cudaError_t set_pass_smem_attr(size_t smem);
-cudaError_t pass_occupancy(bool backward, size_t smem, int* blocks_per_sm);
+cudaError_t pass_occupancy(bool backward, bool slow, size_t smem, int* blocks_per_sm);
 
 cudaError_t launch_prep_coef(const float* theta, int L, int n, float4* coef_fwd, float4* coef_inv,
                              cudaStream_t s);
@@ -48,6 +50,7 @@ cudaError_t launch_grad_reduce(const DevPass* passes, const int* slot_pass, cons
                                float* grad, unsigned* status, cudaStream_t s);
 cudaError_t launch_loss_seed(const float* E, const float* y, int B, float* g, float* loss,
                              cudaStream_t s);
+cudaError_t launch_bwd_init(float2* psi, float2* lam, const float* g, int B, int n, cudaStream_t s);
 cudaError_t launch_encode(const float* x, int B, int n, float2* psi, cudaStream_t s);
 cudaError_t launch_ckpt_copy(bool save, const float2* psi_in, float2* psi_out, void* slot,
                              int storage, long long count, cudaStream_t s);

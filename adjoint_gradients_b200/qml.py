@@ -29,6 +29,7 @@ EXPORTS = [
     "qml_set_workspace", "qml_init_state_encode", "qml_forward_expect", "qml_backward_adjoint",
     "qml_loss_seed", "qml_ckpt_save", "qml_ckpt_restore", "qml_num_ckpt_slots", "qml_expect_z0",
     "qml_host_workspace_bytes", "qml_step_host", "qml_sync", "qml_debug_schedule",
+    "qml_enable_timing", "qml_read_timing", "qml_launch_count",
 ]
 
 
@@ -75,6 +76,10 @@ def load_library(path: str = LIB_PATH):
         "qml_step_host": ([_vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp], _i),
         "qml_sync": ([_vp, _vp], _i),
         "qml_debug_schedule": ([_vp, ctypes.POINTER(_i), _i], _i),
+        "qml_enable_timing": ([_vp, _i], _i),
+        "qml_read_timing": ([_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong),
+                             ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)], _i),
+        "qml_launch_count": ([_vp], ctypes.c_longlong),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -164,6 +169,21 @@ class Context:
         buf = (ctypes.c_int * need)()
         self.lib.qml_debug_schedule(self._h, buf, need)
         return list(buf)
+
+    def enable_timing(self, on: bool = True):
+        _check(self.lib.qml_enable_timing(self._h, 1 if on else 0), "qml_enable_timing")
+
+    def read_timing(self):
+        """(fwd pass ms, fwd pass launches, bwd pass ms, bwd pass launches) since the last read."""
+        fm, bm = ctypes.c_double(), ctypes.c_double()
+        fn, bn = ctypes.c_longlong(), ctypes.c_longlong()
+        _check(self.lib.qml_read_timing(self._h, ctypes.byref(fm), ctypes.byref(fn), ctypes.byref(bm),
+                                        ctypes.byref(bn)), "qml_read_timing")
+        return fm.value, fn.value, bm.value, bn.value
+
+    @property
+    def launch_count(self) -> int:
+        return int(self.lib.qml_launch_count(self._h))
 
     def sync(self, stream=None):
         _check(self.lib.qml_sync(self._h, _stream_handle(stream)), "qml_sync (device status)")

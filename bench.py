@@ -1,0 +1,393 @@
+#!/usr/bin/env python
+"""Benchmark of the fused HEA forward + adjoint-gradient path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload hea_20q_L100]
+
+One step = one training step on one synthetic batch: the fused forward pass
+(encoding, every layer, checkpoint slots, <Z0>), the loss seed, and the fused
+adjoint backward pass (every gradient).  Inputs are resident in HBM before the
+timed region; the 512 MiB working state of the default workload is larger than
+L2, so no flush is needed between steps.  For N > 1 every rank runs its own
+batch (weak scaling) and the gradients are summed with one NCCL all-reduce per
+step, as data-parallel training does.
+
+--impl reference times the CPU oracle (complex128, gate by gate) on the host
+cores instead: there is no other runnable implementation of this method.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from adjoint_gradients_b200.inputs import WORKLOADS, draw_theta, draw_x, draw_y  # noqa: E402
+
+METRIC = "HEA samples/sec (fwd + adjoint grad), 20q; achieved HBM GB/s vs B200 peak"
+UNIT = "samples/s"
+# FP32 ALU roofline: 148 SMs x 128 FP32 lanes x 2 flop (FMA) x 1965 MHz max SM clock.
+SMS, FP32_LANES, SM_MAX_MHZ = 148, 128, 1965.0
+ALU_PEAK_TFLOPS = SMS * FP32_LANES * 2 * SM_MAX_MHZ * 1e6 / 1e12
+FMA_FWD_PER_ROT = 8   # per amplitude: one fused SU(2) on a pair = 16 FMA / 2 amplitudes
+FMA_BWD_PER_ROT = 22  # per amplitude: U^dagger on psi (8) and lambda (8) + three Im<l|P|p> terms (6)
+CPU_SAMPLE_LAYERS = 16  # oracle sample depth (cost is linear in depth)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d.get("hbm_gbs", 6650.0)), "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------- clocks
+
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+                "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                "clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = max(mx, float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[4:8]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- helpers
+
+def algorithmic_counts(ctx, w, B):
+    """Per-pass algorithmic FMAs and HBM bytes of the forward and backward pass kernels."""
+    sched = ctx.debug_schedule()
+    P = sched[0]
+    N = 1 << w.n
+    amp = B * N
+    # bytes per amplitude moved by each pass, from the schedule flags
+    i = 1
+    fwd_bytes = bwd_bytes = 0
+    slot_b = 4 if w.storage == "bf16" else 8
+    for _ in range(P):
+        set_id, gen, last, ck, nops = sched[i:i + 5]
+        i += 5 + 4 * nops
+        fwd_bytes += (0 if gen else 8) + 8 + (slot_b if ck >= 0 else 0)
+        rd = 8 if last else 16
+        wr = 0 if gen else 16
+        bwd_bytes += rd + wr + (slot_b if ck >= 0 else 0)
+    rots = w.n * w.L
+    return {
+        "passes": P,
+        "fwd_fma": FMA_FWD_PER_ROT * rots * amp,
+        "bwd_fma": FMA_BWD_PER_ROT * rots * amp,
+        "fwd_bytes": fwd_bytes * amp,
+        "bwd_bytes": bwd_bytes * amp,
+    }
+
+
+def oracle_sample(w, layers, rank=0):
+    """Time the oracle (forward + adjoint) on one sample of the workload at reduced depth."""
+    import oracle
+
+    x = draw_x(w.index, 1, w.n)
+    theta = draw_theta(w.index, w.L, w.n)[:layers]
+    y = draw_y(w.index, 1)
+    t0 = time.perf_counter()
+    E = oracle.forward(x, theta)
+    oracle.adjoint(x, theta, oracle.loss_seed(E, y))
+    return time.perf_counter() - t0, oracle.num_threads()
+
+
+def cpu_baseline(w):
+    t, cores = oracle_sample(w, CPU_SAMPLE_LAYERS)
+    per_sample = t * w.L / CPU_SAMPLE_LAYERS
+    return {
+        "value": 1.0 / per_sample, "unit": UNIT, "cores": cores, "kind": "oracle",
+        "sample": (f"1 sample of {w.name} at {CPU_SAMPLE_LAYERS} of {w.L} layers "
+                   f"({t:.1f} s), scaled x{w.L / CPU_SAMPLE_LAYERS:g} to full depth"),
+    }
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def physical_gpu(local):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        try:
+            return int(vis.split(",")[local])
+        except (ValueError, IndexError):
+            return local
+    return local
+
+
+# ---------------------------------------------------------------------------- arms
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    w = WORKLOADS[args.workload]
+    if rank != 0:
+        return 0
+    layers = max(1, min(w.L, args.ref_layers))
+    for _ in range(args.warmup):
+        oracle_sample(w, layers)
+    times = []
+    cores = 1
+    for _ in range(args.steps):
+        t, cores = oracle_sample(w, layers)
+        times.append(t)
+    per_step = float(np.mean(times))
+    per_sample = per_step * w.L / layers
+    value = 1.0 / per_sample
+    sample = f"1 sample of {w.name} at {layers} of {w.L} layers per step, scaled x{w.L / layers:g} to full depth"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, w.B),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, B):
+    return {
+        "workload": w.name, "n_qubits": w.n, "layers": w.L, "batch_per_gpu": B, "params": w.params,
+        "ckpt_block": w.ckpt_block, "ckpt_storage": w.storage, "state": "complex64 [B][2^n]",
+        "l2": "inputs larger than L2 (working state B*2^n*8 B > 126 MB); no flush",
+        "seeds": {"x": 1000 + w.index, "theta": 2000 + w.index, "y": 3000 + w.index},
+    }
+
+
+def run_ours(args):
+    import torch
+
+    from adjoint_gradients_b200 import qml
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    w = WORKLOADS[args.workload]
+    B = w.B
+    dev = f"cuda:{local}"
+    # each rank draws its own batch; theta is shared
+    x = np.random.default_rng(1000 + w.index + 7919 * rank).uniform(0, np.pi, (B, w.n))
+    y = np.random.default_rng(3000 + w.index + 7919 * rank).integers(0, 2, B) * 2.0 - 1.0
+    theta = draw_theta(w.index, w.L, w.n)
+    xd = torch.tensor(x, dtype=torch.float32, device=dev)
+    yd = torch.tensor(y, dtype=torch.float32, device=dev)
+    td = torch.tensor(theta, dtype=torch.float32, device=dev)
+
+    ctx = qml.Context(w.n, w.L, B, ckpt_block=w.ckpt_block, storage=w.storage, device=local)
+    psi = ctx.new_state(B)
+    lam = ctx.new_state(B)
+    E = torch.empty(B, dtype=torch.float32, device=dev)
+    grad = torch.empty((w.L, w.n, 3), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ctx.forward(td, xd, psi, E)
+        g, _ = ctx.loss_seed(E, yd)
+        ctx.backward(td, xd, psi, lam, g, grad)
+        if dist is not None:
+            dist.all_reduce(grad)
+
+    for _ in range(args.warmup):
+        step()
+    ctx.sync()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clocks = ClockSampler(physical_gpu(local))
+    clocks.start()
+    time.sleep(0.3)
+    ctx.enable_timing(True)
+    ctx.read_timing()
+    launches0 = ctx.launch_count
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    launches = ctx.launch_count - launches0
+    fwd_ms, fwd_n, bwd_ms, bwd_n = ctx.read_timing()
+    ctx.enable_timing(False)
+    clk = clocks.stop()
+    ctx.sync()
+    ms = ev0.elapsed_time(ev1)
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    value = world * B * args.steps / (ms / 1e3)
+
+    # ---- roofline of the dominant kernel (the backward pass kernel)
+    cnt = algorithmic_counts(ctx, w, B)
+    hbm_peak, peak_src = measured_peaks()
+    bwd_avg_s = bwd_ms / 1e3 / max(1, bwd_n)
+    fwd_avg_s = fwd_ms / 1e3 / max(1, fwd_n)
+    P = cnt["passes"]
+    bwd_tflops = 2 * cnt["bwd_fma"] / P / bwd_avg_s / 1e12
+    fwd_tflops = 2 * cnt["fwd_fma"] / P / fwd_avg_s / 1e12
+    bwd_gbs = cnt["bwd_bytes"] / P / bwd_avg_s / 1e9
+    fwd_gbs = cnt["fwd_bytes"] / P / fwd_avg_s / 1e9
+    traffic = None
+    tfile = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tfile):
+        with open(tfile) as f:
+            tr = json.load(f).get(w.name, {})
+        traffic = tr.get("bwd_pass_bytes_per_launch")
+    roofline = {
+        "kernel": "pass_kernel<backward>", "bound": "alu", "achieved": bwd_tflops, "peak": ALU_PEAK_TFLOPS,
+        "unit": "TFLOP/s", "frac": bwd_tflops / ALU_PEAK_TFLOPS, "traffic": traffic,
+        "peak_src": "148 SMs x 128 FP32 lanes x 2 x 1965 MHz (FFMA; packed f32x2 FMA measured at the same rate)",
+        "avg_launch_ms": bwd_avg_s * 1e3, "launches": bwd_n,
+        "hbm_achieved_gbs": bwd_gbs, "hbm_peak_gbs": hbm_peak, "hbm_frac": bwd_gbs / hbm_peak,
+        "hbm_peak_src": peak_src,
+        "forward_kernel": {"achieved_tflops": fwd_tflops, "frac": fwd_tflops / ALU_PEAK_TFLOPS,
+                           "hbm_gbs": fwd_gbs, "hbm_frac": fwd_gbs / hbm_peak, "avg_launch_ms": fwd_avg_s * 1e3},
+    }
+
+    # ---- end to end through host buffers (pinned), same metric
+    e2e = None
+    if not args.no_e2e:
+        ctx_h = qml.Context(w.n, w.L, B, ckpt_block=w.ckpt_block, storage=w.storage, device=local, host_step=True)
+        xh = torch.tensor(x, dtype=torch.float32).pin_memory()
+        th = torch.tensor(theta, dtype=torch.float32).pin_memory()
+        yh = torch.tensor(y, dtype=torch.float32).pin_memory()
+        out = qml.StepResult(torch.empty(B).pin_memory(), torch.empty(1).pin_memory(),
+                             torch.empty((w.L, w.n, 3)).pin_memory())
+        for _ in range(max(1, min(args.warmup, 2))):
+            ctx_h.step_host(xh, th, yh, out)
+        k2 = max(1, args.steps)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(k2):
+            ctx_h.step_host(xh, th, yh, out)
+            if dist is not None:
+                gt = out.grad.to(dev, non_blocking=False)
+                dist.all_reduce(gt)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        if dist is not None:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        h2d = 4 * (B * w.n + w.L * w.n * 3 + B)
+        d2h = 4 * (B + 1 + w.L * w.n * 3)
+        e2e = {"value": world * B * k2 / (ems / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "api": "qml_step_host"}
+        ctx_h.sync()
+        del ctx_h
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {**workload_config(w, B), "parallelism": f"dp{world}" if world > 1 else "single"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="hea_20q_L100", choices=sorted(WORKLOADS))
+    ap.add_argument("--ref-layers", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -180,6 +180,19 @@ QML_API qml_status qml_step_host(qml_ctx* ctx, const float* x_host, const float*
  * the last qml_sync / qml_set_workspace (then clear it). */
 QML_API qml_status qml_sync(qml_ctx* ctx, void* stream);
 
+/* Pass-kernel timing, for benchmarks.  While enabled, every
+ * qml_forward_expect / qml_backward_adjoint call records one CUDA event pair
+ * on its own stream around its pass-kernel launches (events are host-side
+ * handles; no device memory is allocated).  qml_read_timing waits for those
+ * events and returns the summed milliseconds and launch counts since the
+ * previous read (any output pointer may be NULL). */
+QML_API qml_status qml_enable_timing(qml_ctx* ctx, int enable);
+QML_API qml_status qml_read_timing(qml_ctx* ctx, double* fwd_pass_ms, long long* fwd_pass_launches,
+                                   double* bwd_pass_ms, long long* bwd_pass_launches);
+
+/* Number of kernels this context has launched so far (host-side counter). */
+QML_API long long qml_launch_count(const qml_ctx* ctx);
+
 /* Schedule introspection (host only, no device work): the pass plan as a flat
  * int array, for tests of the scheduler.  Writes at most `cap` ints into
  * `out` and returns the number needed.  Layout: [n_passes, then per pass:
