@@ -24,7 +24,7 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 
 struct Layout {
-  size_t status, passes, phases, ops, slot_pass, slot_index;
+  size_t status, passes, slot_pass, slot_index;
   size_t coef_fwd, coef_inv, enc, dummy, exp_partial, partials, ckpt;
   size_t base_total;
   // host-step extras
@@ -54,9 +54,6 @@ struct qml_ctx {
   int device = 0;
   Plan plan;
   std::vector<DevPass> dpass;
-  std::vector<DevPhase> dphase;
-  std::vector<DevOp> dop;
-  int prog_bytes = 0;
   size_t smem = 0;
   bool probed = false, dev_ok = false;
   bool slow = false;  // the plan puts a batch-unit bit in registers (n < 5)
@@ -79,21 +76,11 @@ struct qml_ctx {
 
 namespace {
 
-int prog_bytes_of(const qml_ctx* c) {
-  int mx = 0;
-  for (const DevPass& p : c->dpass) {
-    int b = (int)((sizeof(DevPass) + 15) & ~size_t(15)) + p.nphases * (int)sizeof(DevPhase) +
-            p.nops * (int)sizeof(DevOp);
-    mx = std::max(mx, b);
-  }
-  return (mx + 15) & ~15;
-}
-
 // Probe the device once: shared-memory opt-in, occupancy, persistent grid size.
 void ensure_device(qml_ctx* c) {
   if (c->probed) return;
   c->probed = true;
-  c->smem = pass_smem_bytes(c->prog_bytes, c->plan.max_slots);
+  c->smem = pass_smem_bytes(c->plan.max_slots);
   cudaDeviceProp prop;
   if (cudaGetDeviceProperties(&prop, c->device) != cudaSuccess) {
     cudaGetLastError();
@@ -131,8 +118,6 @@ void compute_layout(qml_ctx* c) {
   };
   l.status = take(64);
   l.passes = take(sizeof(DevPass) * c->dpass.size());
-  l.phases = take(sizeof(DevPhase) * c->dphase.size());
-  l.ops = take(sizeof(DevOp) * std::max<size_t>(1, c->dop.size()));
   l.slot_pass = take(sizeof(int) * (size_t)L * n);
   l.slot_index = take(sizeof(int) * (size_t)L * n);
   l.coef_fwd = take(sizeof(float4) * 4 * (size_t)L * n);
@@ -216,8 +201,6 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
   if (e != cudaSuccess) return QML_ERR_CUDA;
   PassArgs a{};
   a.passes = at<DevPass>(c, c->lay.passes);
-  a.phases = at<DevPhase>(c, c->lay.phases);
-  a.ops = at<DevOp>(c, c->lay.ops);
   a.n = n;
   a.B = B;
   a.U = (B + 1) / 2;
@@ -233,7 +216,6 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
   a.bmax = c->cfg.max_batch;
   a.partials = nullptr;
   a.status = at<unsigned>(c, c->lay.status);
-  a.smem_prog = c->prog_bytes;
   c->launches += 2;
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, false);
@@ -266,8 +248,6 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
   if (e != cudaSuccess) return QML_ERR_CUDA;
   PassArgs a{};
   a.passes = at<DevPass>(c, c->lay.passes);
-  a.phases = at<DevPhase>(c, c->lay.phases);
-  a.ops = at<DevOp>(c, c->lay.ops);
   a.n = n;
   a.B = B;
   a.U = B;
@@ -283,7 +263,6 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
   a.bmax = c->cfg.max_batch;
   a.partials = at<float>(c, c->lay.partials);
   a.status = at<unsigned>(c, c->lay.status);
-  a.smem_prog = c->prog_bytes;
   e = launch_bwd_init(psi, lam, g, B, n, s);
   if (e != cudaSuccess) return QML_ERR_CUDA;
   c->launches += 3;  // coefficient prep, lambda init, gradient reduce
@@ -346,10 +325,9 @@ qml_status qml_create(const qml_config* cfg, int device, qml_ctx** out) {
     delete c;
     return QML_ERR_UNSUPPORTED;
   }
-  flatten_plan(c->plan, &c->dpass, &c->dphase, &c->dop);
-  c->prog_bytes = prog_bytes_of(c);
-  for (const DevPhase& ph : c->dphase)
-    if (ph.has_reg_unit) c->slow = true;
+  flatten_plan(c->plan, &c->dpass);
+  for (const DevPass& dp : c->dpass)
+    if (dp.slow) c->slow = true;
   c->ckpt_batch.assign(c->plan.n_ckpt, -1);
   *out = c;
   return QML_OK;
@@ -398,12 +376,6 @@ qml_status qml_set_workspace(qml_ctx* c, void* ws, size_t bytes, void* stream) {
   cudaError_t e = cudaMemsetAsync(c->ws + c->lay.status, 0, 64, s);
   if (e == cudaSuccess)
     e = cudaMemcpyAsync(c->ws + c->lay.passes, c->dpass.data(), sizeof(DevPass) * c->dpass.size(),
-                        cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess)
-    e = cudaMemcpyAsync(c->ws + c->lay.phases, c->dphase.data(), sizeof(DevPhase) * c->dphase.size(),
-                        cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess && !c->dop.empty())
-    e = cudaMemcpyAsync(c->ws + c->lay.ops, c->dop.data(), sizeof(DevOp) * c->dop.size(),
                         cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess)
     e = cudaMemcpyAsync(c->ws + c->lay.slot_pass, sp.data(), sizeof(int) * sp.size(), cudaMemcpyHostToDevice, s);

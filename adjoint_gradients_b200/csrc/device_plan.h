@@ -1,5 +1,13 @@
 // device_plan.h -- plain-old-data schedule records shared by the host planner
 // and the CUDA kernels.  No CUDA or C++ library types.
+//
+// A tile is 4096 amplitude positions (12 "tile bits") of one batch unit.  Its
+// 256 threads each keep 16 positions in registers.  The register layout is
+// one of three fixed "phases": in phase p the four register-index bits of a
+// thread are tile bits 4p .. 4p+3, and the eight thread-index bits are the
+// other tile bits in increasing order.  A 2x2 gate on a qubit that sits in a
+// phase's register bits needs no communication; changing phase is a
+// shared-memory exchange.  The planner decides which qubit each tile bit is.
 #pragma once
 
 #include <stdint.h>
@@ -9,44 +17,43 @@ namespace qml {
 constexpr int kTileBits = 12;  // positions per tile = 4096
 constexpr int kRegBits = 4;    // positions per thread = 16
 constexpr int kThrBits = 8;    // threads per block = 256
+constexpr int kPhases = 3;     // register layouts
 constexpr int kPos = 1 << kRegBits;
 constexpr int kThreads = 1 << kThrBits;
 constexpr int kTilePos = 1 << kTileBits;
+constexpr int kSmemSlots = kTilePos + (kTilePos >> 4);  // one pad slot per 16
 constexpr int kMaxSet = 10;           // qubits rotated per pass when n > 12
-constexpr int kMaxLayersPerPass = 16; // cap for circuits that fit one tile
+constexpr int kMaxLayersPerPass = 8;  // cap for circuits that fit one tile
 constexpr int kMaxOut = 30;           // out-of-tile qubits
+constexpr int kMaxOps = 64;
+constexpr int kMaxSlots = kMaxLayersPerPass * kTileBits;
 
 enum : int { OP_EXCH = 1, OP_ROT = 2, OP_CZ = 3, OP_GEN = 4 };
 
-// Where the 12 tile bits sit for one register layout.
-struct DevPhase {
-  int reg_q[kRegBits];        // qubit addressed by register-index bit k, or -1
-  int reg_u[kRegBits];        // batch-unit bit addressed by register bit k, or -1
-  int thr_q[kThrBits];        // qubit addressed by thread-index bit k, or -1
-  int thr_u[kThrBits];        // batch-unit bit addressed by thread bit k, or -1
-  uint32_t reg_phys[kRegBits];  // swizzled shared-memory slot of register bit k
-  uint32_t thr_phys[kThrBits];  // swizzled shared-memory slot of thread bit k
-  uint32_t cz_reg;            // bit j: CZ-ladder parity of register part of position j
-  uint32_t z0_reg;            // bit j: qubit-0 bit of register part of position j
-  int has_reg_unit;           // some register bit is a batch-unit bit
-  int pad_;
-};
-
+// OP_EXCH: a = from phase, b = to phase
+// OP_ROT : a = phase, b = register-bit mask, c = layer, d = first slot
+// OP_CZ  : a = phase, c = layer
+// OP_GEN : a = phase
 struct DevOp {
-  int kind, a, b, c;
+  int kind, a, b, c, d;
 };
 
 struct DevPass {
-  int op0, nops;        // ops[op0 .. op0+nops) in forward order
-  int phase0, nphases;  // phases[phase0 .. phase0+nphases)
+  int nops;
   int load_phase, store_phase;
   int gen, last;
-  int ckpt;             // checkpoint slot, or -1
-  int nslots;           // gradient slots
+  int ckpt;             // checkpoint slot written after / read before this pass, or -1
+  int nslots;           // rotated (layer, qubit) pairs = gradient slots
   int n_out;            // qubits outside the tile
   int unit_bits;        // batch-unit bits inside the tile
-  int out_q[kMaxOut];
-  long long partial_off;  // float offset of this pass's gradient partials
+  int slow;             // a load/store/encode phase has a batch-unit register bit
+  int tile_q[kTileBits];  // tile bit -> qubit (>= 0) or -1 - (batch-unit bit)
+  int out_q[kMaxOut];     // out-of-tile qubits, increasing
+  uint32_t cz_reg[kPhases];  // bit j: CZ-ladder parity of the register part of position j
+  int pad_[1];
+  long long partial_off;     // float offset of this pass's gradient partials
+  int slot_lq[kMaxSlots];    // slot -> layer * n + qubit
+  DevOp ops[kMaxOps];        // forward order
 };
 
 }  // namespace qml

@@ -38,8 +38,9 @@ struct Coef {
   float2 ar, ai, nai, br, bi, nbi, nbr;  // broadcast (v, v) pairs
 };
 
+// p points into the block's shared-memory copy of the pass's coefficients.
 __device__ __forceinline__ Coef load_coef(const float4* p) {
-  const float4 f0 = __ldg(p), f1 = __ldg(p + 1), f2 = __ldg(p + 2), f3 = __ldg(p + 3);
+  const float4 f0 = p[0], f1 = p[1], f2 = p[2], f3 = p[3];
   Coef c;
   c.ar = make_float2(f0.x, f0.y);
   c.ai = make_float2(f0.z, f0.w);
@@ -134,12 +135,6 @@ __device__ __forceinline__ float3 rot_bwd_k(int k, float2 (&re)[kPos], float2 (&
   }
 }
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
 __device__ __forceinline__ void flip(float2& v, uint32_t signbit) {
   v.x = __uint_as_float(__float_as_uint(v.x) ^ signbit);
   v.y = __uint_as_float(__float_as_uint(v.y) ^ signbit);
@@ -147,41 +142,61 @@ __device__ __forceinline__ void flip(float2& v, uint32_t signbit) {
 
 // ------------------------------------------------------------ tile geometry
 
-struct ThreadCtx {
-  uint32_t aq;    // qubit-space index of this thread's register position 0
-  uint32_t ut;    // batch unit of register position 0
-  uint32_t slot;  // swizzled shared-memory slot of register position 0
+// Shared-memory slot (16 bytes) of tile position t: one pad slot every 16
+// positions keeps every quarter warp on eight different bank groups in all
+// three register layouts.  phys(a | b) = phys(a) + phys(b) for disjoint bits.
+__host__ __device__ constexpr uint32_t phys(uint32_t t) { return t + (t >> 4); }
+
+__host__ __device__ constexpr size_t align16(size_t v) { return (v + 15) & ~size_t(15); }
+
+// Tile position of (thread tid, register 0) in phase P: the thread bits are the
+// tile bits outside 4P..4P+3, in increasing order.
+template <int P>
+__device__ __forceinline__ uint32_t thr_tpos(uint32_t tid) {
+  if constexpr (P == 0) return tid << 4;
+  else if constexpr (P == 1) return (tid & 15u) | ((tid >> 4) << 8);
+  else return tid;
+}
+
+// Shared-memory slot offset of register position j in phase P (compile time).
+template <int P>
+__host__ __device__ constexpr uint32_t reg_slot(int j) {
+  return phys((uint32_t)j << (4 * P));
+}
+
+// Per-block copy of the pass record plus per-thread layout constants.
+struct BlockCtx {
+  uint32_t qbit[kTileBits];     // tile bit -> 1 << qubit (0 for a unit bit)
+  uint32_t ubit[kTileBits];     // tile bit -> unit increment (0 for a qubit)
 };
 
-__device__ __forceinline__ ThreadCtx thread_ctx(const DevPhase& ph, int tid, uint32_t base_q,
-                                                uint32_t unit_base) {
-  ThreadCtx t;
-  t.aq = base_q;
-  t.ut = unit_base;
-  t.slot = 0;
+// Qubit-space index and batch unit of (thread, register 0) in phase P.
+template <int P>
+__device__ __forceinline__ void thread_pos(const BlockCtx& bc, uint32_t tid, uint32_t* aq, uint32_t* ut) {
+  const uint32_t t = thr_tpos<P>(tid);
+  uint32_t q = 0, u = 0;
 #pragma unroll
-  for (int k = 0; k < kThrBits; ++k)
-    if ((tid >> k) & 1) {
-      if (ph.thr_q[k] >= 0) t.aq |= 1u << ph.thr_q[k];
-      else t.ut += 1u << ph.thr_u[k];
-      t.slot ^= ph.thr_phys[k];
+  for (int b = 0; b < kTileBits; ++b)
+    if ((t >> b) & 1u) {
+      q |= bc.qbit[b];
+      u += bc.ubit[b];
     }
-  return t;
+  *aq = q;
+  *ut = u;
 }
 
 struct RegMaps {
-  uint32_t q[kRegBits];     // qubit bit of register bit k (0 if a unit bit)
-  uint32_t u[kRegBits];     // unit increment of register bit k (0 if a qubit)
-  uint32_t phys[kRegBits];  // shared-memory slot bit(s) of register bit k
+  uint32_t q[kRegBits];  // qubit bit of register bit k (0 if a unit bit)
+  uint32_t u[kRegBits];  // unit increment of register bit k (0 if a qubit)
 };
 
-__device__ __forceinline__ RegMaps reg_maps(const DevPhase& ph) {
+template <int P>
+__device__ __forceinline__ RegMaps reg_maps(const BlockCtx& bc) {
   RegMaps m;
 #pragma unroll
   for (int k = 0; k < kRegBits; ++k) {
-    m.q[k] = ph.reg_q[k] >= 0 ? (1u << ph.reg_q[k]) : 0u;
-    m.u[k] = ph.reg_u[k] >= 0 ? (1u << ph.reg_u[k]) : 0u;
-    m.phys[k] = ph.reg_phys[k];
+    m.q[k] = bc.qbit[P * kRegBits + k];
+    m.u[k] = bc.ubit[P * kRegBits + k];
   }
   return m;
 }
@@ -193,40 +208,47 @@ __device__ __forceinline__ RegMaps reg_maps(const DevPhase& ph) {
     return r_;                                                    \
   }())
 
-__device__ void exchange(float2 (&re)[kPos], float2 (&im)[kPos], float4* tile,
-                         const DevPhase& from, const DevPhase& to, int tid) {
-  const ThreadCtx tf = thread_ctx(from, tid, 0, 0);
-  const ThreadCtx tt = thread_ctx(to, tid, 0, 0);
-  const RegMaps mf = reg_maps(from);
-  const RegMaps mt = reg_maps(to);
+template <int X, int Y>
+__device__ __forceinline__ void exchange_t(float2 (&re)[kPos], float2 (&im)[kPos], float4* tile, uint32_t tid) {
+  const uint32_t sx = phys(thr_tpos<X>(tid));
+  const uint32_t sy = phys(thr_tpos<Y>(tid));
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kPos; ++j) tile[sx + reg_slot<X>(j)] = make_float4(re[j].x, re[j].y, im[j].x, im[j].y);
   __syncthreads();
 #pragma unroll
   for (int j = 0; j < kPos; ++j) {
-    const uint32_t s = tf.slot ^ REG_COMBINE(mf.phys, j, ^=);
-    tile[s] = make_float4(re[j].x, re[j].y, im[j].x, im[j].y);
-  }
-  __syncthreads();
-#pragma unroll
-  for (int j = 0; j < kPos; ++j) {
-    const uint32_t s = tt.slot ^ REG_COMBINE(mt.phys, j, ^=);
-    const float4 v = tile[s];
+    const float4 v = tile[sy + reg_slot<Y>(j)];
     re[j] = make_float2(v.x, v.y);
     im[j] = make_float2(v.z, v.w);
+  }
+}
+
+__device__ __forceinline__ void exchange(int x, int y, float2 (&re)[kPos], float2 (&im)[kPos], float4* tile,
+                                         uint32_t tid) {
+  const int c = x * 3 + y;
+  switch (c) {
+    case 1: exchange_t<0, 1>(re, im, tile, tid); break;
+    case 2: exchange_t<0, 2>(re, im, tile, tid); break;
+    case 3: exchange_t<1, 0>(re, im, tile, tid); break;
+    case 5: exchange_t<1, 2>(re, im, tile, tid); break;
+    case 6: exchange_t<2, 0>(re, im, tile, tid); break;
+    default: exchange_t<2, 1>(re, im, tile, tid); break;
   }
 }
 
 // CZ(q, q+1) for every q: sign (-1)^{sum_q i_q i_{q+1}} of the global index i.
 // With i = a | b (a: thread and out-of-tile bits, b: register bits, disjoint),
 // the exponent is Q(a) + Q(b) + parity(b & ((a << 1) ^ (a >> 1))).
-__device__ __forceinline__ void apply_cz(float2 (&re)[kPos], float2 (&im)[kPos],
-                                         const DevPhase& ph, uint32_t aq) {
+__device__ __forceinline__ void apply_cz(float2 (&re)[kPos], float2 (&im)[kPos], uint32_t cz_reg,
+                                         const uint32_t (&rq)[kRegBits], uint32_t aq) {
   const uint32_t qa = __popc(aq & (aq >> 1)) & 1u;
   const uint32_t m = (aq << 1) ^ (aq >> 1);
-  uint32_t w = ph.cz_reg ^ (qa ? 0xffffffffu : 0u);
-  const uint32_t pat[5] = {0xAAAAAAAAu, 0xCCCCCCCCu, 0xF0F0F0F0u, 0xFF00FF00u, 0xFFFF0000u};
+  uint32_t w = cz_reg ^ (qa ? 0xffffffffu : 0u);
+  const uint32_t pat[4] = {0xAAAAAAAAu, 0xCCCCCCCCu, 0xF0F0F0F0u, 0xFF00FF00u};
 #pragma unroll
   for (int k = 0; k < kRegBits; ++k)
-    if (ph.reg_q[k] >= 0 && ((m >> ph.reg_q[k]) & 1u)) w ^= pat[k];
+    if (m & rq[k]) w ^= pat[k];
 #pragma unroll
   for (int j = 0; j < kPos; ++j) {
     const uint32_t sb = (w << (31 - j)) & 0x80000000u;
@@ -235,30 +257,22 @@ __device__ __forceinline__ void apply_cz(float2 (&re)[kPos], float2 (&im)[kPos],
   }
 }
 
-// Value of register position j for a runtime j (slow paths for n < 5 only).
-__device__ __forceinline__ float2 sel(const float2 (&v)[kPos], int j) {
-  float2 r = v[0];
+// Sum 16 per-lane values over the warp with 16 shuffles: afterwards even lane
+// 2i holds the warp total of value i.
+__device__ __forceinline__ void warp_reduce16(float (&v)[16], int lane) {
 #pragma unroll
-  for (int k = 1; k < kPos; ++k)
-    if (k == j) r = v[k];
-  return r;
-}
-
-__device__ __forceinline__ void put(float2 (&v)[kPos], int j, float2 x) {
+  for (int step = 0; step < 4; ++step) {
+    const int off = 16 >> step;        // 16, 8, 4, 2
+    const int half = 8 >> step;        // values kept after this step
+    const bool hi = (lane & off) != 0;
 #pragma unroll
-  for (int k = 0; k < kPos; ++k)
-    if (k == j) v[k] = x;
-}
-
-// Register position j's batch unit and qubit index, for a runtime j.
-__device__ __forceinline__ void pos_of(const RegMaps& m, const ThreadCtx& tc, int j, uint32_t* u,
-                                       uint32_t* i) {
-  uint32_t uu = tc.ut, ii = tc.aq;
-#pragma unroll
-  for (int k = 0; k < kRegBits; ++k)
-    if (j & (1 << k)) { uu += m.u[k]; ii |= m.q[k]; }
-  *u = uu;
-  *i = ii;
+    for (int i = 0; i < half; ++i) {
+      const float keep = hi ? v[half + i] : v[i];
+      const float send = hi ? v[i] : v[half + i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
 }
 
 // ------------------------------------------------------------------ planes
@@ -274,239 +288,102 @@ struct Planes {
   }
 };
 
-template <bool BWD, bool SLOW>
-__device__ void load_planes(const PassArgs& a, const DevPhase& ph, const ThreadCtx& tc,
-                            float2 (&re)[kPos], float2 (&im)[kPos]) {
-  const RegMaps m = reg_maps(ph);
-  if constexpr (!SLOW) {
-    if (tc.ut < (uint32_t)a.U) {
-      const float2* p0 = Planes<BWD>::p0(a, tc.ut) + tc.aq;
-      const float2* p1 = Planes<BWD>::p1(a, tc.ut) + tc.aq;
-#pragma unroll
-      for (int j = 0; j < kPos; ++j) {
-        const uint32_t b = REG_COMBINE(m.q, j, |=);
-        re[j] = p0[b];
-        im[j] = p1[b];
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < kPos; ++j) re[j] = im[j] = make_float2(0.f, 0.f);
-    }
-  } else {
-#pragma unroll 1
-    for (int j = 0; j < kPos; ++j) {
-      uint32_t u, i;
-      pos_of(m, tc, j, &u, &i);
-      float2 r = make_float2(0.f, 0.f), v = r;
-      if (u < (uint32_t)a.U) {
-        r = Planes<BWD>::p0(a, u)[i];
-        v = Planes<BWD>::p1(a, u)[i];
-      }
-      put(re, j, r);
-      put(im, j, v);
-    }
-  }
-}
+// What a pass does to HBM at its start or end, in the memory layout P.
+enum MemOp { M_LOAD, M_STORE, M_STORE_STD, M_GEN, M_CKPT_STORE, M_CKPT_RESTORE };
 
-template <bool BWD, bool SLOW>
-__device__ void store_planes(const PassArgs& a, const DevPhase& ph, const ThreadCtx& tc,
-                             const float2 (&re)[kPos], const float2 (&im)[kPos]) {
-  const RegMaps m = reg_maps(ph);
-  if constexpr (!SLOW) {
-    if (tc.ut < (uint32_t)a.U) {
-      float2* p0 = Planes<BWD>::p0(a, tc.ut) + tc.aq;
-      float2* p1 = Planes<BWD>::p1(a, tc.ut) + tc.aq;
-#pragma unroll
-      for (int j = 0; j < kPos; ++j) {
-        const uint32_t b = REG_COMBINE(m.q, j, |=);
-        p0[b] = re[j];
-        p1[b] = im[j];
-      }
-    }
-  } else {
-#pragma unroll 1
-    for (int j = 0; j < kPos; ++j) {
-      uint32_t u, i;
-      pos_of(m, tc, j, &u, &i);
-      if (u < (uint32_t)a.U) {
-        Planes<BWD>::p0(a, u)[i] = sel(re, j);
-        Planes<BWD>::p1(a, u)[i] = sel(im, j);
-      }
-    }
-  }
-}
-
-// Forward, last pass: write the standard (re, im) layout of both samples.
-template <bool SLOW>
-__device__ void store_standard_fwd(const PassArgs& a, const DevPhase& ph, const ThreadCtx& tc,
-                                   const float2 (&re)[kPos], const float2 (&im)[kPos]) {
-  const RegMaps m = reg_maps(ph);
-  if constexpr (!SLOW) {
-    const uint32_t u = tc.ut;
-    if (u >= (uint32_t)a.U) return;
-    float2* s0 = a.buf0 + (size_t)(2 * u) * a.N + tc.aq;
-    float2* s1 = s0 + a.N;
-    const bool has1 = 2 * u + 1 < (uint32_t)a.B;
-#pragma unroll
-    for (int j = 0; j < kPos; ++j) {
-      const uint32_t b = REG_COMBINE(m.q, j, |=);
-      s0[b] = make_float2(re[j].x, im[j].x);
-      if (has1) s1[b] = make_float2(re[j].y, im[j].y);
-    }
-  } else {
-#pragma unroll 1
-  for (int j = 0; j < kPos; ++j) {
-    uint32_t u = tc.ut, i = tc.aq;
-    for (int k = 0; k < kRegBits; ++k)
-      if (j & (1 << k)) { u += m.u[k]; i |= m.q[k]; }
-    if (u < (uint32_t)a.U) {
-      const float2 r = sel(re, j), v = sel(im, j);
-      a.buf0[(size_t)(2 * u) * a.N + i] = make_float2(r.x, v.x);
-      if (2 * u + 1 < (uint32_t)a.B) a.buf0[(size_t)(2 * u + 1) * a.N + i] = make_float2(r.y, v.y);
-    }
-  }
-  }
-}
-
-// Forward: checkpoint slot (standard layout, fp32 or bf16 round-to-nearest-even).
-template <bool SLOW>
-__device__ void store_ckpt_fwd(const PassArgs& a, int slot, const DevPhase& ph,
-                               const ThreadCtx& tc, const float2 (&re)[kPos],
-                               const float2 (&im)[kPos], int bmax) {
-  const RegMaps m = reg_maps(ph);
-  if constexpr (!SLOW) {
-    const uint32_t u = tc.ut;
-    if (u >= (uint32_t)a.U) return;
-    const size_t e0 = ((size_t)slot * bmax + 2 * u) * a.N + tc.aq;
-    const bool has1 = 2 * u + 1 < (uint32_t)a.B;
-    if (a.storage == 0) {
-      float2* s0 = reinterpret_cast<float2*>(a.ckpt) + e0;
-      float2* s1 = s0 + a.N;
-#pragma unroll
-      for (int j = 0; j < kPos; ++j) {
-        const uint32_t b = REG_COMBINE(m.q, j, |=);
-        s0[b] = make_float2(re[j].x, im[j].x);
-        if (has1) s1[b] = make_float2(re[j].y, im[j].y);
-      }
-    } else {
-      __nv_bfloat162* s0 = reinterpret_cast<__nv_bfloat162*>(a.ckpt) + e0;
-      __nv_bfloat162* s1 = s0 + a.N;
-#pragma unroll
-      for (int j = 0; j < kPos; ++j) {
-        const uint32_t b = REG_COMBINE(m.q, j, |=);
-        s0[b] = __floats2bfloat162_rn(re[j].x, im[j].x);
-        if (has1) s1[b] = __floats2bfloat162_rn(re[j].y, im[j].y);
-      }
-    }
-  } else {
-#pragma unroll 1
-  for (int j = 0; j < kPos; ++j) {
-    uint32_t u = tc.ut, i = tc.aq;
-    for (int k = 0; k < kRegBits; ++k)
-      if (j & (1 << k)) { u += m.u[k]; i |= m.q[k]; }
-    if (u >= (uint32_t)a.U) continue;
-    const float2 r = sel(re, j), v = sel(im, j);
-    const size_t e0 = ((size_t)slot * bmax + 2 * u) * a.N + i;
-    const bool has1 = 2 * u + 1 < (uint32_t)a.B;
-    if (a.storage == 0) {
-      float2* s = reinterpret_cast<float2*>(a.ckpt);
-      s[e0] = make_float2(r.x, v.x);
-      if (has1) s[e0 + a.N] = make_float2(r.y, v.y);
-    } else {
-      __nv_bfloat162* s = reinterpret_cast<__nv_bfloat162*>(a.ckpt);
-      s[e0] = __floats2bfloat162_rn(r.x, v.x);
-      if (has1) s[e0 + a.N] = __floats2bfloat162_rn(r.y, v.y);
-    }
-  }
-  }
-}
-
-// Backward: replace the psi lanes by the checkpointed state of slot `slot`.
-template <bool SLOW>
-__device__ void restore_ckpt_bwd(const PassArgs& a, int slot, const DevPhase& ph,
-                                 const ThreadCtx& tc, float2 (&re)[kPos], float2 (&im)[kPos],
-                                 int bmax) {
-  const RegMaps m = reg_maps(ph);
-  if constexpr (!SLOW) {
-    const uint32_t u = tc.ut;
-    if (u >= (uint32_t)a.U) return;
-    const size_t e = ((size_t)slot * bmax + u) * a.N + tc.aq;
-#pragma unroll
-    for (int j = 0; j < kPos; ++j) {
-      const uint32_t b = REG_COMBINE(m.q, j, |=);
-      float2 v;
-      if (a.storage == 0) v = reinterpret_cast<const float2*>(a.ckpt)[e + b];
-      else v = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(a.ckpt)[e + b]);
-      re[j].x = v.x;
-      im[j].x = v.y;
-    }
-  } else {
-#pragma unroll 1
-  for (int j = 0; j < kPos; ++j) {
-    uint32_t u, i;
-    pos_of(m, tc, j, &u, &i);
-    if (u >= (uint32_t)a.U) continue;
-    const size_t e = ((size_t)slot * bmax + u) * a.N + i;
-    float2 v;
-    if (a.storage == 0) v = reinterpret_cast<const float2*>(a.ckpt)[e];
-    else v = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(a.ckpt)[e]);
-    float2 r = sel(re, j), w = sel(im, j);
-    r.x = v.x;
-    w.x = v.y;
-    put(re, j, r);
-    put(im, j, w);
-  }
-  }
-}
-
-// Forward: the angle-encoded product state prod_q (cos, sin)(x_q/2)[bit q].
-template <bool SLOW>
-__device__ void gen_state(const PassArgs& a, const DevPhase& ph, const ThreadCtx& tc,
-                          float2 (&re)[kPos], float2 (&im)[kPos]) {
-  const RegMaps m = reg_maps(ph);
+template <bool BWD, bool SLOW, int P, int OP>
+__device__ __forceinline__ void mem_t(const PassArgs& a, const BlockCtx& bc, uint32_t tid, uint32_t base_q,
+                                      uint32_t unit_base, float2 (&re)[kPos], float2 (&im)[kPos], int slot) {
+  uint32_t aq, ut;
+  thread_pos<P>(bc, tid, &aq, &ut);
+  aq |= base_q;
+  ut += unit_base;
+  const RegMaps m = reg_maps<P>(bc);
   const int n = a.n;
-  if constexpr (!SLOW) {
-    if (tc.ut >= (uint32_t)a.U) {
 #pragma unroll
-      for (int j = 0; j < kPos; ++j) re[j] = im[j] = make_float2(0.f, 0.f);
-      return;
-    }
-    const float2* e = a.enc + (size_t)tc.ut * n * 2;
-    uint32_t regq = 0;
-#pragma unroll
-    for (int k = 0; k < kRegBits; ++k) regq |= m.q[k];
-    float2 c = make_float2(1.f, 1.f);
-    for (int q = 0; q < n; ++q)
-      if (!((regq >> q) & 1u)) c = __fmul2_rn(c, __ldg(&e[2 * q + ((tc.aq >> q) & 1u)]));
-    float2 e0[kRegBits], e1[kRegBits];
-#pragma unroll
-    for (int k = 0; k < kRegBits; ++k) {
-      const int q = ph.reg_q[k];
-      e0[k] = __ldg(&e[2 * q]);
-      e1[k] = __ldg(&e[2 * q + 1]);
-    }
-#pragma unroll
-    for (int j = 0; j < kPos; ++j) {
-      float2 v = c;
-#pragma unroll
-      for (int k = 0; k < kRegBits; ++k) v = __fmul2_rn(v, (j & (1 << k)) ? e1[k] : e0[k]);
-      re[j] = v;
-      im[j] = make_float2(0.f, 0.f);
-    }
-  } else {
-#pragma unroll 1
-    for (int j = 0; j < kPos; ++j) {
-      uint32_t u, i;
-      pos_of(m, tc, j, &u, &i);
+  for (int j = 0; j < kPos; ++j) {
+    const uint32_t i = aq | REG_COMBINE(m.q, j, |=);
+    const uint32_t u = SLOW ? ut + REG_COMBINE(m.u, j, +=) : ut;
+    const bool ok = u < (uint32_t)a.U;
+    if constexpr (OP == M_LOAD) {
+      if (ok) {
+        re[j] = Planes<BWD>::p0(a, u)[i];
+        im[j] = Planes<BWD>::p1(a, u)[i];
+      } else {
+        re[j] = im[j] = make_float2(0.f, 0.f);
+      }
+    } else if constexpr (OP == M_STORE) {
+      if (ok) {
+        Planes<BWD>::p0(a, u)[i] = re[j];
+        Planes<BWD>::p1(a, u)[i] = im[j];
+      }
+    } else if constexpr (OP == M_STORE_STD) {  // forward only
+      if (ok) {
+        a.buf0[(size_t)(2 * u) * a.N + i] = make_float2(re[j].x, im[j].x);
+        if (2 * u + 1 < (uint32_t)a.B) a.buf0[(size_t)(2 * u + 1) * a.N + i] = make_float2(re[j].y, im[j].y);
+      }
+    } else if constexpr (OP == M_GEN) {  // forward only: angle-encoded product state
       float2 v = make_float2(0.f, 0.f);
-      if (u < (uint32_t)a.U) {
+      if (ok) {
         const float2* e = a.enc + (size_t)u * n * 2;
         v = make_float2(1.f, 1.f);
         for (int q = 0; q < n; ++q) v = __fmul2_rn(v, __ldg(&e[2 * q + ((i >> q) & 1u)]));
       }
-      put(re, j, v);
-      put(im, j, make_float2(0.f, 0.f));
+      re[j] = v;
+      im[j] = make_float2(0.f, 0.f);
+    } else if constexpr (OP == M_CKPT_STORE) {  // forward only
+      if (ok) {
+        const size_t e0 = ((size_t)slot * a.bmax + 2 * u) * a.N + i;
+        const bool has1 = 2 * u + 1 < (uint32_t)a.B;
+        if (a.storage == 0) {
+          float2* s = reinterpret_cast<float2*>(a.ckpt);
+          s[e0] = make_float2(re[j].x, im[j].x);
+          if (has1) s[e0 + a.N] = make_float2(re[j].y, im[j].y);
+        } else {
+          __nv_bfloat162* s = reinterpret_cast<__nv_bfloat162*>(a.ckpt);
+          s[e0] = __floats2bfloat162_rn(re[j].x, im[j].x);
+          if (has1) s[e0 + a.N] = __floats2bfloat162_rn(re[j].y, im[j].y);
+        }
+      }
+    } else {  // M_CKPT_RESTORE, backward only: psi lanes from the slot
+      if (ok) {
+        const size_t e = ((size_t)slot * a.bmax + u) * a.N + i;
+        float2 v;
+        if (a.storage == 0) v = reinterpret_cast<const float2*>(a.ckpt)[e];
+        else v = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(a.ckpt)[e]);
+        re[j].x = v.x;
+        im[j].x = v.y;
+      }
     }
+  }
+}
+
+template <bool BWD, bool SLOW, int OP>
+__device__ __forceinline__ void mem_op(int phase, const PassArgs& a, const BlockCtx& bc, uint32_t tid,
+                                       uint32_t base_q, uint32_t unit_base, float2 (&re)[kPos],
+                                       float2 (&im)[kPos], int slot = 0) {
+  switch (phase) {
+    case 0: mem_t<BWD, SLOW, 0, OP>(a, bc, tid, base_q, unit_base, re, im, slot); break;
+    case 1: mem_t<BWD, SLOW, 1, OP>(a, bc, tid, base_q, unit_base, re, im, slot); break;
+    default: mem_t<BWD, SLOW, 2, OP>(a, bc, tid, base_q, unit_base, re, im, slot); break;
+  }
+}
+
+template <int P>
+__device__ __forceinline__ void cz_t(float2 (&re)[kPos], float2 (&im)[kPos], const BlockCtx& bc, uint32_t cz_reg,
+                                     uint32_t tid, uint32_t base_q) {
+  uint32_t aq, ut;
+  thread_pos<P>(bc, tid, &aq, &ut);
+  const RegMaps m = reg_maps<P>(bc);
+  apply_cz(re, im, cz_reg, m.q, aq | base_q);
+}
+
+__device__ __forceinline__ void cz_op(int phase, float2 (&re)[kPos], float2 (&im)[kPos], const BlockCtx& bc,
+                                      uint32_t cz_reg, uint32_t tid, uint32_t base_q) {
+  switch (phase) {
+    case 0: cz_t<0>(re, im, bc, cz_reg, tid, base_q); break;
+    case 1: cz_t<1>(re, im, bc, cz_reg, tid, base_q); break;
+    default: cz_t<2>(re, im, bc, cz_reg, tid, base_q); break;
   }
 }
 
@@ -514,42 +391,38 @@ __device__ void gen_state(const PassArgs& a, const DevPhase& ph, const ThreadCtx
 
 template <bool BWD, bool SLOW>
 __global__ void __launch_bounds__(kThreads, 2) pass_kernel(const PassArgs a) {
-  const int bmax = a.bmax;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   float4* tile = reinterpret_cast<float4*>(smem_raw);
-  unsigned char* prog = smem_raw + (size_t)kTilePos * sizeof(float4);
-  DevPass* P = reinterpret_cast<DevPass*>(prog);
-  const DevPass& gp = a.passes[a.pass_idx];
-  DevPhase* PH = reinterpret_cast<DevPhase*>(prog + ((sizeof(DevPass) + 15) & ~size_t(15)));
-  const int tid = threadIdx.x;
+  unsigned char* rest = smem_raw + (size_t)kSmemSlots * sizeof(float4);
+  DevPass* P = reinterpret_cast<DevPass*>(rest);
+  BlockCtx* bc = reinterpret_cast<BlockCtx*>(rest + align16(sizeof(DevPass)));
+  float4* coef = reinterpret_cast<float4*>(rest + align16(sizeof(DevPass)) + align16(sizeof(BlockCtx)));
+  const uint32_t tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  constexpr int kWarps = kThreads / 32;
 
-  // copy the pass program into shared memory
+  // ---- block setup: pass record, tile-bit maps, gate coefficients
   {
-    const int* src = reinterpret_cast<const int*>(&gp);
+    const int* src = reinterpret_cast<const int*>(a.passes + a.pass_idx);
     int* dst = reinterpret_cast<int*>(P);
     for (int i = tid; i < (int)(sizeof(DevPass) / 4); i += kThreads) dst[i] = src[i];
   }
   __syncthreads();
-  DevOp* OPS = reinterpret_cast<DevOp*>(reinterpret_cast<unsigned char*>(PH) +
-                                       sizeof(DevPhase) * P->nphases);
-  {
-    const int* src = reinterpret_cast<const int*>(a.phases + P->phase0);
-    int* dst = reinterpret_cast<int*>(PH);
-    for (int i = tid; i < (int)(P->nphases * sizeof(DevPhase) / 4); i += kThreads) dst[i] = src[i];
-    const int* so = reinterpret_cast<const int*>(a.ops + P->op0);
-    int* dso = reinterpret_cast<int*>(OPS);
-    for (int i = tid; i < P->nops * 4; i += kThreads) dso[i] = so[i];
+  const int nslots = P->nslots;
+  float* acc = reinterpret_cast<float*>(coef + 4 * nslots);  // [warps][nslots*3]
+  const int nacc = nslots * 3;
+  if (tid < kTileBits) {
+    const int q = P->tile_q[tid];
+    bc->qbit[tid] = q >= 0 ? (1u << q) : 0u;
+    bc->ubit[tid] = q >= 0 ? 0u : (1u << (-1 - q));
   }
-  constexpr int kWarps = kThreads / 32;
-  float* acc = reinterpret_cast<float*>(prog + a.smem_prog);  // [warps][nslots*3]
-  const int nacc = P->nslots * 3;
+  for (int i = tid; i < 4 * nslots; i += kThreads) coef[i] = __ldg(a.coef + (size_t)P->slot_lq[i >> 2] * 4 + (i & 3));
   if (BWD)
     for (int i = tid; i < kWarps * nacc; i += kThreads) acc[i] = 0.f;
   __syncthreads();
 
   const int n_out = P->n_out;
-  const int warp = tid >> 5, lane = tid & 31;
-
+  const int nops = P->nops;
   for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x) {
     const uint32_t o = (uint32_t)t & ((1u << n_out) - 1u);
     const uint32_t ug = (uint32_t)t >> n_out;
@@ -559,72 +432,64 @@ __global__ void __launch_bounds__(kThreads, 2) pass_kernel(const PassArgs a) {
     const uint32_t unit_base = ug << P->unit_bits;
 
     float2 re[kPos], im[kPos];
-    int cur = BWD ? P->store_phase : P->load_phase;
-    {
-      const ThreadCtx tc = thread_ctx(PH[cur], tid, base_q, unit_base);
-      if (!BWD) {
-        if (P->gen) gen_state<SLOW>(a, PH[cur], tc, re, im);
-        else load_planes<false, SLOW>(a, PH[cur], tc, re, im);
-      } else {
-        load_planes<true, SLOW>(a, PH[cur], tc, re, im);
-        if (P->ckpt >= 0) restore_ckpt_bwd<SLOW>(a, P->ckpt, PH[cur], tc, re, im, bmax);
-      }
-    }
-
     if (!BWD) {
-      for (int oi = 0; oi < P->nops; ++oi) {
-        const DevOp op = OPS[oi];
+      if (P->gen) mem_op<false, SLOW, M_GEN>(P->load_phase, a, *bc, tid, base_q, unit_base, re, im);
+      else mem_op<false, SLOW, M_LOAD>(P->load_phase, a, *bc, tid, base_q, unit_base, re, im);
+      for (int oi = 0; oi < nops; ++oi) {
+        const DevOp op = P->ops[oi];
         if (op.kind == OP_EXCH) {
-          exchange(re, im, tile, PH[op.a], PH[op.b], tid);
-          cur = op.b;
+          exchange(op.a, op.b, re, im, tile, tid);
         } else if (op.kind == OP_ROT) {
+          int slot = op.d;
+#pragma unroll
           for (int k = 0; k < kRegBits; ++k)
             if ((op.b >> k) & 1) {
-              const int q = PH[cur].reg_q[k];
-              const Coef c = load_coef(a.coef + ((size_t)op.a * a.n + q) * 4);
+              const Coef c = load_coef(coef + 4 * slot++);
               rot_fwd_k(k, re, im, c);
             }
         } else if (op.kind == OP_CZ) {
-          const ThreadCtx tc = thread_ctx(PH[cur], tid, base_q, unit_base);
-          apply_cz(re, im, PH[cur], tc.aq);
+          cz_op(op.a, re, im, *bc, P->cz_reg[op.a], tid, base_q);
         }
       }
-      const ThreadCtx tc = thread_ctx(PH[cur], tid, base_q, unit_base);
-      if (P->ckpt >= 0) store_ckpt_fwd<SLOW>(a, P->ckpt, PH[cur], tc, re, im, bmax);
-      if (P->last) store_standard_fwd<SLOW>(a, PH[cur], tc, re, im);
-      else store_planes<false, SLOW>(a, PH[cur], tc, re, im);
+      if (P->ckpt >= 0) mem_op<false, SLOW, M_CKPT_STORE>(P->store_phase, a, *bc, tid, base_q, unit_base, re, im, P->ckpt);
+      if (P->last) mem_op<false, SLOW, M_STORE_STD>(P->store_phase, a, *bc, tid, base_q, unit_base, re, im);
+      else mem_op<false, SLOW, M_STORE>(P->store_phase, a, *bc, tid, base_q, unit_base, re, im);
     } else {
-      for (int oi = P->nops - 1; oi >= 0; --oi) {
-        const DevOp op = OPS[oi];
+      mem_op<true, SLOW, M_LOAD>(P->store_phase, a, *bc, tid, base_q, unit_base, re, im);
+      if (P->ckpt >= 0) mem_op<true, SLOW, M_CKPT_RESTORE>(P->store_phase, a, *bc, tid, base_q, unit_base, re, im, P->ckpt);
+      for (int oi = nops - 1; oi >= 0; --oi) {
+        const DevOp op = P->ops[oi];
         if (op.kind == OP_EXCH) {
-          exchange(re, im, tile, PH[op.b], PH[op.a], tid);
-          cur = op.a;
+          exchange(op.b, op.a, re, im, tile, tid);
         } else if (op.kind == OP_ROT) {
-          for (int k = kRegBits - 1; k >= 0; --k)
+          float s[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) s[i] = 0.f;
+          int slot = op.d;
+          int g = 0;
+#pragma unroll
+          for (int k = 0; k < kRegBits; ++k)
             if ((op.b >> k) & 1) {
-              const int q = PH[cur].reg_q[k];
-              const Coef c = load_coef(a.coef + ((size_t)op.a * a.n + q) * 4);
-              float3 s = rot_bwd_k(k, re, im, c);
-              s.x = warp_sum(s.x);
-              s.y = warp_sum(s.y);
-              s.z = warp_sum(s.z);
-              if (lane == 0) {
-                const int slot = op.c + __popc((unsigned)op.b & ((1u << k) - 1u));
-                float* w = acc + warp * nacc + slot * 3;
-                w[0] += s.x;
-                w[1] += s.y;
-                w[2] += s.z;
-              }
+              const Coef c = load_coef(coef + 4 * slot++);
+              const float3 v = rot_bwd_k(k, re, im, c);
+              // values of gate g sit at 3g .. 3g+2 (g counts the mask bits)
+#pragma unroll
+              for (int gg = 0; gg < kRegBits; ++gg)
+                if (gg == g) {
+                  s[3 * gg] = v.x;
+                  s[3 * gg + 1] = v.y;
+                  s[3 * gg + 2] = v.z;
+                }
+              ++g;
             }
+          warp_reduce16(s, lane);
+          const int vi = lane >> 1;
+          if (!(lane & 1) && vi < 3 * g) acc[warp * nacc + op.d * 3 + vi] += s[0];
         } else if (op.kind == OP_CZ) {
-          const ThreadCtx tc = thread_ctx(PH[cur], tid, base_q, unit_base);
-          apply_cz(re, im, PH[cur], tc.aq);
+          cz_op(op.a, re, im, *bc, P->cz_reg[op.a], tid, base_q);
         }
       }
-      if (!P->gen) {
-        const ThreadCtx tc = thread_ctx(PH[cur], tid, base_q, unit_base);
-        store_planes<true, SLOW>(a, PH[cur], tc, re, im);
-      }
+      if (!P->gen) mem_op<true, SLOW, M_STORE>(P->load_phase, a, *bc, tid, base_q, unit_base, re, im);
     }
   }
 
@@ -815,8 +680,9 @@ __global__ void ckpt_copy_kernel(bool save, const float2* in, float2* out, void*
 
 }  // namespace
 
-size_t pass_smem_bytes(int prog_bytes, int max_slots) {
-  return (size_t)kTilePos * sizeof(float4) + (size_t)prog_bytes + (size_t)(kThreads / 32) * max_slots * 3 * sizeof(float);
+size_t pass_smem_bytes(int max_slots) {
+  return (size_t)kSmemSlots * sizeof(float4) + align16(sizeof(DevPass)) + align16(sizeof(BlockCtx)) +
+         (size_t)max_slots * 4 * sizeof(float4) + (size_t)(kThreads / 32) * max_slots * 3 * sizeof(float);
 }
 
 cudaError_t set_pass_smem_attr(size_t smem) {

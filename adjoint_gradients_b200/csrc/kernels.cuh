@@ -11,8 +11,6 @@ namespace qml {
 // Arguments of one pass launch (forward or backward).
 struct PassArgs {
   const DevPass* passes;
-  const DevPhase* phases;
-  const DevOp* ops;
   int pass_idx;
   int n, B, U;           // qubits, samples, batch units (forward: ceil(B/2); backward: B)
   long long N;           // 2^n
@@ -28,10 +26,9 @@ struct PassArgs {
   int bmax;              // samples per checkpoint slot (slot stride)
   float* partials;       // backward gradient partials
   unsigned* status;
-  int smem_prog;         // bytes reserved for the pass program in shared memory
 };
 
-size_t pass_smem_bytes(int prog_bytes, int max_slots);
+size_t pass_smem_bytes(int max_slots);
 
 // `slow`: some register bit indexes a batch unit (only when n < 5); the
 // generic per-position code then replaces the single-unit fast path.

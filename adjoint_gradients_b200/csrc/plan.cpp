@@ -2,7 +2,6 @@
 #include "plan.hpp"
 
 #include <algorithm>
-#include <cstdio>
 
 namespace qml {
 namespace {
@@ -14,65 +13,31 @@ struct Task {
   int set;
 };
 
-int popcount32(uint32_t v) { return __builtin_popcount(v); }
-
-// GF(2)^3: are a, b, c a basis?
-bool basis3(uint32_t a, uint32_t b, uint32_t c) {
-  if (!a || !b || a == b) return false;
-  return c && c != a && c != b && c != (a ^ b);
+// Tile bits that are thread-index bits in phase p, in increasing order.
+void thread_tbits(int p, int out[kThrBits]) {
+  int h = 0;
+  for (int t = 0; t < kTileBits; ++t)
+    if (t / kRegBits != p) out[h++] = t;
 }
 
-// Choose, per tile bit >= 3, the 3-bit column that is XORed into the low three
-// bits of the shared-memory slot, so that in every phase the eight lanes of a
-// quarter warp (thread bits 0..2) hit eight different 16-byte bank groups.
-bool choose_swizzle(HostPass* ps) {
-  uint32_t col[kTileBits];
-  uint64_t rng = 0x9E3779B97F4A7C15ull;
-  for (int attempt = 0; attempt < 4096; ++attempt) {
-    for (int t = 0; t < kTileBits; ++t) col[t] = t < 3 ? (1u << t) : 0xFFu;  // 0xFF = unassigned
-    bool ok = true;
-    for (const HostPhase& ph : ps->phases) {
-      uint32_t v[3];
-      for (int k = 0; k < 3; ++k) {
-        int t = ph.thr_tbit[k];
-        if (col[t] == 0xFFu) {
-          // pick a value; first attempt is greedy, later attempts random
-          uint32_t pick = 0;
-          for (uint32_t cand = 1; cand < 8; ++cand) {
-            uint32_t c = attempt == 0 ? cand : (uint32_t)(1 + ((rng >> 33) % 7));
-            rng = rng * 6364136223846793005ull + 1442695040888963407ull;
-            bool clash = false;
-            for (int m = 0; m < k; ++m)
-              if (c == v[m] || (k == 2 && c == (v[0] ^ v[1]))) clash = true;
-            if (!clash) { pick = c; break; }
-          }
-          if (!pick) pick = 1;
-          col[t] = pick;
-        }
-        v[k] = col[t];
-      }
-      if (!basis3(v[0], v[1], v[2])) { ok = false; break; }
-    }
-    if (ok) {
-      for (int t = 0; t < kTileBits; ++t) ps->swz_col[t] = (t < 3) ? 0u : (col[t] == 0xFFu ? 0u : col[t]);
-      return true;
-    }
-    rng ^= (uint64_t)attempt * 0xD1B54A32D192ED03ull;
-  }
-  return false;
-}
-
-uint32_t phys_of_bit(const HostPass& ps, int t) { return (1u << t) ^ ps.swz_col[t]; }
-
-// How many leading lanes address consecutive low qubits 0, 1, 2, ... (a
-// measure of how contiguous a warp's global access is in this phase).
-int coalesce_score(const HostPass& ps, const HostPhase& ph) {
+// How many leading lanes of phase p address consecutive low qubits 0, 1, 2, ...
+// (the longer, the more contiguous a warp's global access).
+int coalesce_score(const HostPass& ps, int p) {
+  int tb[kThrBits];
+  thread_tbits(p, tb);
   int s = 0;
   for (int k = 0; k < 5; ++k) {
-    if (ps.tile_q[ph.thr_tbit[k]] != k) break;
+    if (ps.tile_q[tb[k]] != k) break;
     ++s;
   }
   return s;
+}
+
+// Phase p's register bits are all qubits (no batch-unit bit).
+bool phase_fast(const HostPass& ps, int p) {
+  for (int k = 0; k < kRegBits; ++k)
+    if (ps.tile_q[p * kRegBits + k] < 0) return false;
+  return true;
 }
 
 }  // namespace
@@ -91,10 +56,11 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
     p.sets.push_back({});
     for (int q = 0; q < n; ++q) p.sets[0].push_back(q);
   } else {
-    int s = (n + kMaxSet - 1) / kMaxSet;
-    int base = n / s, extra = n % s, q = 0;
+    const int s = (n + kMaxSet - 1) / kMaxSet;
+    const int base = n / s, extra = n % s;
+    int q = 0;
     for (int i = 0; i < s; ++i) {
-      int sz = base + (i < extra ? 1 : 0);
+      const int sz = base + (i < extra ? 1 : 0);
       std::vector<int> set;
       for (int k = 0; k < sz; ++k) set.push_back(q++);
       p.sets.push_back(set);
@@ -102,9 +68,7 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
   }
   p.n_sets = (int)p.sets.size();
   const int S = p.n_sets;
-
-  int n_blocks = (ckpt_block > 0) ? (L + ckpt_block - 1) / ckpt_block : 1;
-  p.n_ckpt = (ckpt_block > 0) ? n_blocks - 1 : 0;
+  p.n_ckpt = (ckpt_block > 0) ? (L + ckpt_block - 1) / ckpt_block - 1 : 0;
 
   // ---- task list: encode, then per layer the sets in boustrophedon order, then CZ
   std::vector<Task> tasks;
@@ -114,7 +78,9 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
     tasks.push_back({T_CZ, l, -1});
   }
 
-  // ---- group tasks into passes
+  // ---- group tasks into passes: a new pass starts when the rotated set
+  // changes, when a single-tile pass is full, or after a checkpoint boundary
+  // of a single-tile circuit (so that its slot is a clean layer boundary)
   struct Proto {
     int set = -1;
     std::vector<Task> t;
@@ -125,9 +91,7 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
   for (const Task& tk : tasks) {
     Proto* cur = &protos.back();
     if (tk.kind == T_ROT) {
-      bool need_new = false;
-      if (cur->set >= 0 && cur->set != tk.set) need_new = true;
-      if (S == 1 && cur->rots >= kMaxLayersPerPass) need_new = true;
+      bool need_new = (cur->set >= 0 && cur->set != tk.set) || (S == 1 && cur->rots >= kMaxLayersPerPass);
       if (need_new) {
         protos.emplace_back();
         cur = &protos.back();
@@ -137,16 +101,10 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
     }
     cur->t.push_back(tk);
     if (tk.kind == T_CZ && ckpt_block > 0) {
-      int l = tk.layer;
+      const int l = tk.layer;
       if ((l + 1) % ckpt_block == 0 && l + 1 < L) {
-        int m = (l + 1) / ckpt_block;  // slot m-1 holds the state after layer m*b-1
-        if (S == 1) {
-          // single-tile circuits: cut the pass here so the slot is a layer boundary
-          cur->ckpt = m - 1;
-          protos.emplace_back();
-        } else {
-          cur->ckpt = m - 1;  // written after the pass that holds this CZ
-        }
+        cur->ckpt = (l + 1) / ckpt_block - 1;  // slot m-1 holds the state after layer m*b-1
+        if (S == 1) protos.emplace_back();
       }
     }
   }
@@ -159,137 +117,104 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
     const Proto& pr = protos[pi];
     HostPass ps;
     ps.set_id = pr.set;
-    ps.gen = false;
     ps.last = (pi + 1 == protos.size());
     ps.ckpt = pr.ckpt;
-    ps.nslots = 0;
+    ps.gen = false;
+    for (const Task& tk : pr.t)
+      if (tk.kind == T_GEN) ps.gen = true;
 
-    // tile bits
-    std::vector<int> tq;
+    // ---- tile bits
+    std::vector<bool> rotated_q(n, false);
     if (S == 1) {
-      for (int q = 0; q < n; ++q) tq.push_back(q);
+      for (int q = 0; q < n; ++q) rotated_q[q] = true;
       ps.unit_bits = kTileBits - n;
       for (int t = 0; t < kTileBits; ++t) ps.tile_q[t] = t < n ? t : -1 - (t - n);
     } else {
-      const std::vector<int>& set = p.sets[pr.set >= 0 ? pr.set : 0];
+      const std::vector<int>& set = p.sets[pr.set];
       std::vector<bool> in(n, false);
-      for (int q : set) in[q] = true;
-      tq = set;
+      std::vector<int> tq = set;
+      for (int q : set) in[q] = rotated_q[q] = true;
       for (int q = 0; q < n && (int)tq.size() < kTileBits; ++q)
-        if (!in[q]) { tq.push_back(q); in[q] = true; }
+        if (!in[q]) {
+          tq.push_back(q);
+          in[q] = true;
+        }
       std::sort(tq.begin(), tq.end());
       for (int q = 0; q < n; ++q)
         if (!in[q]) ps.out_q.push_back(q);
       ps.unit_bits = 0;
       for (int t = 0; t < kTileBits; ++t) ps.tile_q[t] = tq[t];
     }
-    std::vector<int> q2t(n, -1);
-    for (int t = 0; t < kTileBits; ++t)
-      if (ps.tile_q[t] >= 0) q2t[ps.tile_q[t]] = t;
+    if ((int)ps.out_q.size() > kMaxOut) return "internal: too many out-of-tile qubits";
 
-    // register groups: the rotated qubits in chunks of five
-    std::vector<int> rot_q = (S == 1) ? p.sets[0] : p.sets[pr.set >= 0 ? pr.set : 0];
-    std::vector<std::vector<int>> groups;  // tile bits
-    for (size_t i = 0; i < rot_q.size(); i += kRegBits) {
-      std::vector<int> g;
-      for (size_t k = i; k < rot_q.size() && k < i + kRegBits; ++k) g.push_back(q2t[rot_q[k]]);
-      groups.push_back(g);
-    }
-    std::vector<bool> rotated_tbit(kTileBits, false);
-    for (auto& g : groups)
-      for (int t : g) rotated_tbit[t] = true;
-    for (auto& g : groups) {
-      HostPhase ph;
-      std::vector<bool> used(kTileBits, false);
-      for (int t : g) used[t] = true;
-      std::vector<int> regs = g;
-      // pad: highest passive qubit bits, then highest other qubit bits, then unit bits
-      for (int pass_kind = 0; pass_kind < 3 && (int)regs.size() < kRegBits; ++pass_kind) {
-        for (int t = kTileBits - 1; t >= 0 && (int)regs.size() < kRegBits; --t) {
-          if (used[t]) continue;
-          bool is_q = ps.tile_q[t] >= 0;
-          bool ok = (pass_kind == 0 && is_q && !rotated_tbit[t]) || (pass_kind == 1 && is_q) ||
-                    (pass_kind == 2 && !is_q);
-          if (ok) { regs.push_back(t); used[t] = true; }
-        }
+    // ---- rotated register bits per phase, and the phase that touches HBM
+    int mask[kPhases];
+    std::vector<int> active;
+    for (int g = 0; g < kPhases; ++g) {
+      mask[g] = 0;
+      for (int k = 0; k < kRegBits; ++k) {
+        const int q = ps.tile_q[g * kRegBits + k];
+        if (q >= 0 && rotated_q[q]) mask[g] |= 1 << k;
       }
-      for (int k = 0; k < kRegBits; ++k) ph.reg_tbit[k] = regs[k];
-      int h = 0;
-      for (int t = 0; t < kTileBits; ++t)
-        if (!used[t]) ph.thr_tbit[h++] = t;
-      ps.phases.push_back(ph);
+      if (mask[g]) active.push_back(g);
     }
-    const int G = (int)groups.size();
-    // best group for global access
-    int best = 0, best_score = -1;
-    for (int g = 0; g < G; ++g) {
-      int sc = coalesce_score(ps, ps.phases[g]);
-      if (sc > best_score) { best_score = sc; best = g; }
-    }
+    int mem = -1, best = -1;
+    for (int g = kPhases - 1; g >= 0; --g)
+      if (phase_fast(ps, g) && coalesce_score(ps, g) > best) {
+        best = coalesce_score(ps, g);
+        mem = g;
+      }
+    ps.slow = mem < 0;
+    if (mem < 0) mem = 0;
+    ps.load_phase = mem;
+
+    // group order of the first rotation: start in the memory phase when
+    // loading; when encoding, choose the direction that ends in it
     std::vector<int> order;
-    order.push_back(best);
-    for (int g = 0; g < G; ++g)
-      if (g != best) order.push_back(g);
-
-    bool has_gen = false;
-    for (const Task& tk : pr.t)
-      if (tk.kind == T_GEN) has_gen = true;
-    ps.gen = has_gen;
-    int nrot = pr.rots;
-    // direction of the first rotation: loading passes start in the best
-    // layout; encoding passes choose the direction that ends in it
-    bool forward_dir = true;
-    if (has_gen) forward_dir = (nrot % 2 == 0);
-
-    int cur = -1;
-    bool gen_emitted = false;
+    if (std::find(active.begin(), active.end(), mem) != active.end()) order.push_back(mem);
+    for (int g : active)
+      if (g != mem) order.push_back(g);
+    const bool ends_at_mem_if_forward = (pr.rots % 2 == 0);
+    bool dir = true;
+    if (ps.gen) dir = ends_at_mem_if_forward;
+    int cur = mem;
+    if (ps.gen) {
+      // encode directly in the first group's layout when that layout is fast
+      std::vector<int> first = order;
+      if (!dir) std::reverse(first.begin(), first.end());
+      if (phase_fast(ps, first[0])) cur = first[0];
+      ps.load_phase = cur;
+      ps.ops.push_back({OP_GEN, cur, 0, 0, 0});
+    }
     int rot_i = 0;
-    auto emit_exch = [&](int to) {
-      if (cur >= 0 && cur != to) ps.ops.push_back({OP_EXCH, cur, to, 0});
-      cur = to;
-    };
     for (const Task& tk : pr.t) {
-      if (tk.kind == T_GEN) continue;  // emitted lazily once the layout is known
       if (tk.kind == T_ROT) {
-        bool dir = (rot_i % 2 == 0) ? forward_dir : !forward_dir;
-        ++rot_i;
         std::vector<int> ord = order;
-        if (!dir) std::reverse(ord.begin(), ord.end());
+        const bool d = (rot_i++ % 2 == 0) ? dir : !dir;
+        if (!d) std::reverse(ord.begin(), ord.end());
         for (int g : ord) {
-          if (cur < 0) {
-            cur = g;
-            if (has_gen && !gen_emitted) {
-              ps.ops.push_back({OP_GEN, 0, 0, 0});
-              gen_emitted = true;
-            }
-            ps.load_phase = g;
-          }
-          emit_exch(g);
-          uint32_t mask = 0;
-          const HostPhase& ph = ps.phases[g];
+          if (g != cur) ps.ops.push_back({OP_EXCH, cur, g, 0, 0});
+          cur = g;
+          const int slot0 = (int)ps.slot_lq.size();
           for (int k = 0; k < kRegBits; ++k)
-            for (int t : groups[g])
-              if (ph.reg_tbit[k] == t) mask |= 1u << k;
-          int slot0 = ps.nslots;
-          for (int k = 0; k < kRegBits; ++k)
-            if (mask & (1u << k)) {
-              int q = ps.tile_q[ph.reg_tbit[k]];
-              size_t idx = (size_t)tk.layer * n + q;
+            if (mask[g] & (1 << k)) {
+              const int q = ps.tile_q[g * kRegBits + k];
+              const size_t idx = (size_t)tk.layer * n + q;
               p.slot_pass[idx] = (int)pi;
-              p.slot_index[idx] = ps.nslots++;
+              p.slot_index[idx] = (int)ps.slot_lq.size();
+              ps.slot_lq.push_back(tk.layer * n + q);
             }
-          ps.ops.push_back({OP_ROT, tk.layer, (int)mask, slot0});
+          ps.ops.push_back({OP_ROT, g, mask[g], tk.layer, slot0});
         }
       } else if (tk.kind == T_CZ) {
-        if (cur < 0) return "internal: CZ before any rotation in a pass";
-        ps.ops.push_back({OP_CZ, tk.layer, 0, 0});
+        ps.ops.push_back({OP_CZ, cur, 0, tk.layer, 0});
       }
     }
-    if (cur < 0) return "internal: pass without rotations";
-    if (coalesce_score(ps, ps.phases[cur]) < best_score) emit_exch(best);
-    ps.store_phase = cur;
-    if (!choose_swizzle(&ps)) return "internal: no bank-conflict-free swizzle found";
-    p.max_slots = std::max(p.max_slots, ps.nslots);
+    if (cur != mem) ps.ops.push_back({OP_EXCH, cur, mem, 0, 0});
+    ps.store_phase = mem;
+    if ((int)ps.ops.size() > kMaxOps) return "internal: too many ops in a pass";
+    if ((int)ps.slot_lq.size() > kMaxSlots) return "internal: too many gradient slots in a pass";
+    p.max_slots = std::max(p.max_slots, (int)ps.slot_lq.size());
     p.passes.push_back(ps);
   }
   for (size_t i = 0; i < p.slot_pass.size(); ++i)
@@ -298,60 +223,45 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
   return "";
 }
 
-void flatten_plan(const Plan& p, std::vector<DevPass>* passes, std::vector<DevPhase>* phases,
-                  std::vector<DevOp>* ops) {
+void flatten_plan(const Plan& p, std::vector<DevPass>* passes) {
   passes->clear();
-  phases->clear();
-  ops->clear();
   for (const HostPass& ps : p.passes) {
     DevPass d{};
-    d.op0 = (int)ops->size();
     d.nops = (int)ps.ops.size();
-    d.phase0 = (int)phases->size();
-    d.nphases = (int)ps.phases.size();
     d.load_phase = ps.load_phase;
     d.store_phase = ps.store_phase;
     d.gen = ps.gen ? 1 : 0;
     d.last = ps.last ? 1 : 0;
     d.ckpt = ps.ckpt;
-    d.nslots = ps.nslots;
+    d.nslots = (int)ps.slot_lq.size();
     d.n_out = (int)ps.out_q.size();
     d.unit_bits = ps.unit_bits;
+    d.slow = ps.slow ? 1 : 0;
+    for (int t = 0; t < kTileBits; ++t) d.tile_q[t] = ps.tile_q[t];
     for (int i = 0; i < kMaxOut; ++i) d.out_q[i] = i < d.n_out ? ps.out_q[i] : -1;
-    d.partial_off = 0;
-    passes->push_back(d);
-    for (const HostOp& o : ps.ops) ops->push_back({o.kind, o.a, o.b, o.c});
-    for (const HostPhase& ph : ps.phases) {
-      DevPhase dp{};
-      dp.has_reg_unit = 0;
-      uint32_t qbit[kRegBits];
-      for (int k = 0; k < kRegBits; ++k) {
-        int t = ph.reg_tbit[k];
-        int q = ps.tile_q[t];
-        dp.reg_q[k] = q >= 0 ? q : -1;
-        dp.reg_u[k] = q >= 0 ? -1 : (-1 - q);
-        if (q < 0) dp.has_reg_unit = 1;
-        dp.reg_phys[k] = phys_of_bit(ps, t);
-        qbit[k] = q >= 0 ? (1u << q) : 0u;
-      }
-      for (int k = 0; k < kThrBits; ++k) {
-        int t = ph.thr_tbit[k];
-        int q = ps.tile_q[t];
-        dp.thr_q[k] = q >= 0 ? q : -1;
-        dp.thr_u[k] = q >= 0 ? -1 : (-1 - q);
-        dp.thr_phys[k] = phys_of_bit(ps, t);
-      }
-      dp.cz_reg = 0;
-      dp.z0_reg = 0;
+    for (int g = 0; g < kPhases; ++g) {
+      uint32_t w = 0;
       for (int j = 0; j < kPos; ++j) {
         uint32_t b = 0;
-        for (int k = 0; k < kRegBits; ++k)
-          if (j & (1 << k)) b |= qbit[k];
-        if (popcount32(b & (b >> 1)) & 1) dp.cz_reg |= 1u << j;
-        if (b & 1u) dp.z0_reg |= 1u << j;
+        for (int k = 0; k < kRegBits; ++k) {
+          const int q = ps.tile_q[g * kRegBits + k];
+          if ((j >> k) & 1 && q >= 0) b |= 1u << q;
+        }
+        if (__builtin_popcount(b & (b >> 1)) & 1) w |= 1u << j;
       }
-      phases->push_back(dp);
+      d.cz_reg[g] = w;
     }
+    d.partial_off = 0;
+    for (int s = 0; s < kMaxSlots; ++s) d.slot_lq[s] = s < d.nslots ? ps.slot_lq[s] : 0;
+    for (int o = 0; o < kMaxOps; ++o) {
+      if (o < d.nops) {
+        const HostOp& h = ps.ops[o];
+        d.ops[o] = {h.kind, h.a, h.b, h.c, h.d};
+      } else {
+        d.ops[o] = {0, 0, 0, 0, 0};
+      }
+    }
+    passes->push_back(d);
   }
 }
 
@@ -364,23 +274,24 @@ std::vector<int> describe_plan(const Plan& p) {
     v.push_back(ps.last ? 1 : 0);
     v.push_back(ps.ckpt);
     v.push_back((int)ps.ops.size());
-    int cur = ps.load_phase;  // the layout the first data op runs in
     for (const HostOp& o : ps.ops) {
-      int b = o.b;
-      if (o.kind == OP_EXCH) cur = o.b;
-      if (o.kind == OP_ROT) {
+      int a = o.a, b = 0, c = 0;
+      if (o.kind == OP_EXCH) {
+        b = o.b;
+      } else if (o.kind == OP_ROT) {
+        a = o.c;  // layer
         uint32_t qm = 0;
         for (int k = 0; k < kRegBits; ++k)
-          if (o.b & (1 << k)) {
-            const int q = ps.tile_q[ps.phases[cur].reg_tbit[k]];
-            if (q >= 0) qm |= 1u << q;
-          }
+          if (o.b & (1 << k)) qm |= 1u << ps.tile_q[o.a * kRegBits + k];
         b = (int)qm;
+        c = o.d;
+      } else if (o.kind == OP_CZ) {
+        a = o.c;  // layer
       }
       v.push_back(o.kind);
-      v.push_back(o.a);
+      v.push_back(a);
       v.push_back(b);
-      v.push_back(o.c);
+      v.push_back(c);
     }
   }
   return v;

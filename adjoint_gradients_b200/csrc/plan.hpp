@@ -7,14 +7,12 @@
 // gist.science Technical Summary (sec. 2, "Forward Path Gate Fusion").  The
 // backward pass runs the same passes in reverse (sec. 1.4, item 2).
 //
-// A pass owns a 12-bit tile: 4096 amplitude positions of one batch unit whose
-// out-of-tile index bits are fixed.  Qubits are split into sets of at most ten
-// that are rotated together; a pass rotates one set and carries enough of the
-// lowest remaining qubits as "passive" tile bits to keep HBM accesses
-// contiguous.  Inside a pass, 128 threads hold 32 positions each in registers.
-// A "phase" says which five tile bits index a thread's registers (the qubits a
-// 2x2 gate can be applied to without communication) and which seven index the
-// thread; changing phase is a shared-memory exchange.
+// Qubits are split into sets of at most ten that are rotated together.  A
+// pass owns 12 tile bits: the rotated set plus enough of the lowest other
+// qubits ("passive" bits) to keep HBM accesses contiguous; for n <= 12 the
+// tile is the whole state plus batch-unit bits.  Tile bits are assigned to
+// qubits in increasing order, so the three fixed register groups (tile bits
+// 0-3, 4-7, 8-11; see device_plan.h) each hold up to four rotated qubits.
 #pragma once
 
 #include <cstdint>
@@ -25,32 +23,22 @@
 
 namespace qml {
 
-struct HostPhase {
-  int reg_tbit[kRegBits];  // tile bit addressed by register-index bit k
-  int thr_tbit[kThrBits];  // tile bit addressed by thread-index bit k (0..4 = lane)
-};
-
 struct HostOp {
-  int kind;   // OP_EXCH / OP_ROT / OP_CZ / OP_GEN
-  int a, b, c;
-  // OP_EXCH: a = from phase, b = to phase (local indices)
-  // OP_ROT : a = layer, b = register-bit mask, c = first gradient slot
-  // OP_CZ  : a = layer
+  int kind, a, b, c, d;  // as DevOp
 };
 
 struct HostPass {
-  int set_id;                 // which qubit set is rotated (-1: none)
+  int set_id;                 // which qubit set is rotated
   int tile_q[kTileBits];      // tile bit -> qubit, or -1 - k for batch-unit bit k
   std::vector<int> out_q;     // qubits outside the tile, increasing
   int unit_bits;              // batch-unit bits inside the tile (n < 12)
-  std::vector<HostPhase> phases;
   std::vector<HostOp> ops;    // forward order
   int load_phase, store_phase;
   bool gen;                   // forward: encode instead of loading
   bool last;                  // forward: last pass (stores the standard layout)
   int ckpt;                   // checkpoint slot written after this pass, or -1
-  int nslots;                 // gradient slots (one per rotated (layer, qubit))
-  uint32_t swz_col[kTileBits];  // shared-memory swizzle column of each tile bit
+  std::vector<int> slot_lq;   // gradient slot -> layer * n + qubit
+  bool slow;
 };
 
 struct Plan {
@@ -67,9 +55,8 @@ struct Plan {
 // Build the schedule.  Returns an empty string on success, else an error.
 std::string make_plan(int n, int L, int ckpt_block, Plan* out);
 
-// Flatten to the device representation (phases / ops / passes arrays).
-void flatten_plan(const Plan& p, std::vector<DevPass>* passes, std::vector<DevPhase>* phases,
-                  std::vector<DevOp>* ops);
+// Flatten to the device representation.
+void flatten_plan(const Plan& p, std::vector<DevPass>* passes);
 
 // Layout of qml_debug_schedule (see qml.h).
 std::vector<int> describe_plan(const Plan& p);

@@ -377,13 +377,24 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="hea_20q_L100", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="hea_20q_L100", choices=sorted(WORKLOADS) + ["custom"])
     ap.add_argument("--ref-layers", type=int, default=2)
+    ap.add_argument("--case", default=None,
+                    help="n,L,B[,ckpt_block[,storage]]: a custom shape with the workload's seeds (for profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.case:
+        from adjoint_gradients_b200.inputs import Workload
+
+        f = args.case.split(",")
+        n, L, B = int(f[0]), int(f[1]), int(f[2])
+        ck = int(f[3]) if len(f) > 3 else 0
+        st = f[4] if len(f) > 4 else "fp32"
+        WORKLOADS["custom"] = Workload(WORKLOADS[args.workload].index, f"custom_{n}q_L{L}_B{B}", n, L, B, ck, st)
+        args.workload = "custom"
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

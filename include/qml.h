@@ -196,10 +196,11 @@ QML_API long long qml_launch_count(const qml_ctx* ctx);
 /* Schedule introspection (host only, no device work): the pass plan as a flat
  * int array, for tests of the scheduler.  Writes at most `cap` ints into
  * `out` and returns the number needed.  Layout: [n_passes, then per pass:
- * geometry id, n_ops, then per op 4 ints (kind, a, b, c)].  Op kinds:
- * 1 = register-layout exchange (a = from phase, b = to phase),
- * 2 = rotate (a = layer, b = qubit mask over the whole register, c = unused),
- * 3 = CZ ladder (a = layer), 4 = encode. */
+ * rotated-set id, encodes (0/1), last (0/1), checkpoint slot (-1 = none),
+ * n_ops, then per op 4 ints (kind, a, b, c)].  Op kinds:
+ * 1 = register-layout exchange (a = from layout, b = to layout),
+ * 2 = rotate (a = layer, b = bit mask of the rotated qubits, c = first slot),
+ * 3 = CZ ladder (a = layer), 4 = encode (a = layout). */
 QML_API int qml_debug_schedule(const qml_ctx* ctx, int* out, int cap);
 
 #ifdef __cplusplus
