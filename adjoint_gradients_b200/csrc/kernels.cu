@@ -53,27 +53,27 @@ __device__ __forceinline__ Coef load_coef(const float4* p) {
 }
 
 // (x, y) <- [[a, b], [-conj b, conj a]] (x, y) on two lanes at once.
+// Term order: every x term comes first, so x is dead before the last term of
+// each output, and the final terms read only the y value that is overwritten
+// by, or already consumed before, the instruction that writes them.  The
+// results can then land in the registers of (x, y) without extra moves.
 __device__ __forceinline__ void su2(float2& xr, float2& xi, float2& yr, float2& yi, const Coef& c) {
   float2 o0r = __fmul2_rn(c.ar, xr);
-  o0r = __ffma2_rn(c.nai, xi, o0r);
-  o0r = __ffma2_rn(c.br, yr, o0r);
-  o0r = __ffma2_rn(c.nbi, yi, o0r);
   float2 o0i = __fmul2_rn(c.ar, xi);
-  o0i = __ffma2_rn(c.ai, xr, o0i);
-  o0i = __ffma2_rn(c.br, yi, o0i);
-  o0i = __ffma2_rn(c.bi, yr, o0i);
   float2 o1r = __fmul2_rn(c.nbr, xr);
-  o1r = __ffma2_rn(c.nbi, xi, o1r);
-  o1r = __ffma2_rn(c.ar, yr, o1r);
-  o1r = __ffma2_rn(c.ai, yi, o1r);
   float2 o1i = __fmul2_rn(c.nbr, xi);
+  o0r = __ffma2_rn(c.nai, xi, o0r);
+  o0i = __ffma2_rn(c.ai, xr, o0i);
+  o1r = __ffma2_rn(c.nbi, xi, o1r);
   o1i = __ffma2_rn(c.bi, xr, o1i);
-  o1i = __ffma2_rn(c.ar, yi, o1i);
+  o0r = __ffma2_rn(c.br, yr, o0r);
+  o0i = __ffma2_rn(c.br, yi, o0i);
+  o1r = __ffma2_rn(c.ai, yi, o1r);
   o1i = __ffma2_rn(c.nai, yr, o1i);
-  xr = o0r;
-  xi = o0i;
-  yr = o1r;
-  yi = o1i;
+  xr = __ffma2_rn(c.nbi, yi, o0r);
+  xi = __ffma2_rn(c.bi, yr, o0i);
+  yr = __ffma2_rn(c.ar, yr, o1r);
+  yi = __ffma2_rn(c.ar, yi, o1i);
 }
 
 template <int K>
