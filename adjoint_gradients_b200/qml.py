@@ -29,7 +29,7 @@ EXPORTS = [
     "qml_set_workspace", "qml_init_state_encode", "qml_forward_expect", "qml_backward_adjoint",
     "qml_loss_seed", "qml_ckpt_save", "qml_ckpt_restore", "qml_num_ckpt_slots", "qml_expect_z0",
     "qml_host_workspace_bytes", "qml_step_host", "qml_sync", "qml_debug_schedule",
-    "qml_enable_timing", "qml_read_timing", "qml_launch_count",
+    "qml_enable_timing", "qml_read_timing", "qml_launch_count", "qml_expect_z0_static",
 ]
 
 
@@ -80,6 +80,7 @@ def load_library(path: str = LIB_PATH):
         "qml_read_timing": ([_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong),
                              ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)], _i),
         "qml_launch_count": ([_vp], ctypes.c_longlong),
+        "qml_expect_z0_static": ([_vp, _i, _i, _vp, _vp], _i),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)

@@ -163,6 +163,32 @@ QML_API int qml_num_ckpt_slots(const qml_ctx* ctx);
 QML_API qml_status qml_expect_z0(qml_ctx* ctx, const float* psi_dev, int B, float* expect_dev,
                          void* stream);
 
+/* Allocation-free Z0 expectation, for callers that may not allocate device
+ * memory at all (for example a plugin inside an application whose framework
+ * owns all device memory through its own pool, or a loop in which an
+ * allocation that may synchronise the device is not allowed).  It needs no
+ * context and no workspace: the partial sums of its two-stage reduction live
+ * in a fixed array compiled into the library (32768 doubles = 256 KiB, held
+ * on every GPU that loads the library until the process exits).  It computes
+ * exactly what qml_expect_z0 computes; the paper has no counterpart of this
+ * entry point.
+ *   psi_dev    [B][2^n] complex64 on the current device (8-byte aligned)
+ *   expect_dev [B] float32, out
+ * Limits and behaviour:
+ *   - B * ceil(2^n / 65536) must not exceed 32768 (e.g. B <= 2048 at n = 20,
+ *     B <= 4 at n = 29); larger calls return QML_ERR_WORKSPACE and launch
+ *     nothing.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current and caches it; make
+ *     that first call before any stream capture.
+ *   - All calls on a device share the one array.  Each call overwrites every
+ *     partial it later reads, so stale contents are never used, but calls
+ *     whose kernels overlap on the GPU (different streams, no ordering) race
+ *     on it.
+ *   - No cudaMalloc, cudaFree or allocating library routine is called. */
+QML_API qml_status qml_expect_z0_static(const float* psi_dev, int n_qubits, int B, float* expect_dev,
+                                        void* stream);
+
 /* One full training step through HOST buffers: copies x, theta and y from
  * host to device, runs qml_forward_expect, qml_loss_seed and
  * qml_backward_adjoint, and copies E, the loss and the gradient back.  Needs
