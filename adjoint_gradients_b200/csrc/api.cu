@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <new>
@@ -57,6 +58,7 @@ struct qml_ctx {
   size_t smem = 0;
   bool probed = false, dev_ok = false;
   bool slow = false;  // the plan puts a batch-unit bit in registers (n < 5)
+  int region = 0;     // constant-memory coefficient region
   int sms = 148, grid_fwd = 0, grid_bwd = 0;
   char* ws = nullptr;
   size_t ws_bytes = 0;
@@ -120,8 +122,8 @@ void compute_layout(qml_ctx* c) {
   l.passes = take(sizeof(DevPass) * c->dpass.size());
   l.slot_pass = take(sizeof(int) * (size_t)L * n);
   l.slot_index = take(sizeof(int) * (size_t)L * n);
-  l.coef_fwd = take(sizeof(float4) * 4 * (size_t)L * n);
-  l.coef_inv = take(sizeof(float4) * 4 * (size_t)L * n);
+  l.coef_fwd = take(sizeof(float4) * 4 * (size_t)kMaxSlots * c->dpass.size());
+  l.coef_inv = take(sizeof(float4) * 4 * (size_t)kMaxSlots * c->dpass.size());
   l.enc = take(sizeof(float2) * 2 * U * n);
   l.dummy = take(sizeof(float2) * (size_t)N);
   l.exp_partial = take(sizeof(double) * expect_partial_count(Bm, n));
@@ -194,13 +196,15 @@ qml_status check_ready(qml_ctx* c, int B) {
 
 qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, float2* psi,
                        float* expect, cudaStream_t s) {
-  const int n = c->cfg.n_qubits, L = c->cfg.n_layers;
-  cudaError_t e = launch_prep_coef(theta, L, n, at<float4>(c, c->lay.coef_fwd), at<float4>(c, c->lay.coef_inv), s);
+  const int n = c->cfg.n_qubits;
+  const int P = (int)c->dpass.size();
+  float4* cf = at<float4>(c, c->lay.coef_fwd);
+  cudaError_t e = launch_prep_pass_coef(at<DevPass>(c, c->lay.passes), P, theta, cf, at<float4>(c, c->lay.coef_inv), s);
   if (e != cudaSuccess) return QML_ERR_CUDA;
   e = launch_prep_enc(x, B, n, at<float2>(c, c->lay.enc), s);
   if (e != cudaSuccess) return QML_ERR_CUDA;
   PassArgs a{};
-  a.passes = at<DevPass>(c, c->lay.passes);
+  a.region = c->region;
   a.n = n;
   a.B = B;
   a.U = (B + 1) / 2;
@@ -208,7 +212,6 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
   a.buf0 = psi;
   a.buf1 = nullptr;
   a.dummy = at<float2>(c, c->lay.dummy);
-  a.coef = at<float4>(c, c->lay.coef_fwd);
   a.enc = at<float2>(c, c->lay.enc);
   a.g = nullptr;
   a.ckpt = c->ws + c->lay.ckpt;
@@ -219,12 +222,13 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
   c->launches += 2;
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, false);
-  for (size_t p = 0; p < c->dpass.size(); ++p) {
+  for (int p = 0; p < P; ++p) {
     const DevPass& dp = c->dpass[p];
     const long long units_per_tile = 1ll << dp.unit_bits;
-    a.pass_idx = (int)p;
     a.n_tiles = (int)(((a.U + units_per_tile - 1) / units_per_tile) << dp.n_out);
-    e = launch_pass(false, c->slow, a, c->grid_fwd, c->smem, s);
+    e = copy_pass_coef(c->region, cf + (size_t)p * kMaxSlots * 4, dp.nslots, s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+    e = launch_pass(false, a, dp, c->grid_fwd, c->smem, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
     ++c->launches;
     if (dp.ckpt >= 0) c->ckpt_batch[dp.ckpt] = B;
@@ -242,12 +246,16 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
                         float2* lam, const float* g, float* grad, cudaStream_t s) {
   (void)x;
   const int n = c->cfg.n_qubits, L = c->cfg.n_layers;
+  const int P = (int)c->dpass.size();
   for (int m = 0; m < c->plan.n_ckpt; ++m)
     if (c->ckpt_batch[m] != B) return QML_ERR_CKPT_MISMATCH;
-  cudaError_t e = launch_prep_coef(theta, L, n, at<float4>(c, c->lay.coef_fwd), at<float4>(c, c->lay.coef_inv), s);
+  float4* ci = at<float4>(c, c->lay.coef_inv);
+  cudaError_t e = launch_prep_pass_coef(at<DevPass>(c, c->lay.passes), P, theta, at<float4>(c, c->lay.coef_fwd), ci, s);
+  if (e != cudaSuccess) return QML_ERR_CUDA;
+  e = launch_bwd_init(psi, lam, g, B, n, s);
   if (e != cudaSuccess) return QML_ERR_CUDA;
   PassArgs a{};
-  a.passes = at<DevPass>(c, c->lay.passes);
+  a.region = c->region;
   a.n = n;
   a.B = B;
   a.U = B;
@@ -255,7 +263,6 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
   a.buf0 = psi;
   a.buf1 = lam;
   a.dummy = nullptr;
-  a.coef = at<float4>(c, c->lay.coef_inv);
   a.enc = nullptr;
   a.g = g;
   a.ckpt = c->ws + c->lay.ckpt;
@@ -263,17 +270,16 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
   a.bmax = c->cfg.max_batch;
   a.partials = at<float>(c, c->lay.partials);
   a.status = at<unsigned>(c, c->lay.status);
-  e = launch_bwd_init(psi, lam, g, B, n, s);
-  if (e != cudaSuccess) return QML_ERR_CUDA;
   c->launches += 3;  // coefficient prep, lambda init, gradient reduce
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, true);
-  for (int p = (int)c->dpass.size() - 1; p >= 0; --p) {
+  for (int p = P - 1; p >= 0; --p) {
     const DevPass& dp = c->dpass[p];
     const long long units_per_tile = 1ll << dp.unit_bits;
-    a.pass_idx = p;
     a.n_tiles = (int)(((a.U + units_per_tile - 1) / units_per_tile) << dp.n_out);
-    e = launch_pass(true, c->slow, a, c->grid_bwd, c->smem, s);
+    e = copy_pass_coef(c->region, ci + (size_t)p * kMaxSlots * 4, dp.nslots, s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+    e = launch_pass(true, a, dp, c->grid_bwd, c->smem, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
     ++c->launches;
   }
@@ -326,6 +332,8 @@ qml_status qml_create(const qml_config* cfg, int device, qml_ctx** out) {
     return QML_ERR_UNSUPPORTED;
   }
   flatten_plan(c->plan, &c->dpass);
+  static std::atomic<int> next_region{0};
+  c->region = next_region.fetch_add(1) % kCoefRegions;
   for (const DevPass& dp : c->dpass)
     if (dp.slow) c->slow = true;
   c->ckpt_batch.assign(c->plan.n_ckpt, -1);

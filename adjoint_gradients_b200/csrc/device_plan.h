@@ -2,12 +2,15 @@
 // and the CUDA kernels.  No CUDA or C++ library types.
 //
 // A tile is 4096 amplitude positions (12 "tile bits") of one batch unit.  Its
-// 256 threads each keep 16 positions in registers.  The register layout is
-// one of three fixed "phases": in phase p the four register-index bits of a
-// thread are tile bits 4p .. 4p+3, and the eight thread-index bits are the
-// other tile bits in increasing order.  A 2x2 gate on a qubit that sits in a
-// phase's register bits needs no communication; changing phase is a
-// shared-memory exchange.  The planner decides which qubit each tile bit is.
+// 128 threads each keep 32 positions in registers.  The register layout is
+// one of three fixed "phases"; in each phase the five register-index bits of
+// a thread are five fixed tile bits:
+//   phase 0: tile bits 0-4      phase 1: tile bits 5-9
+//   phase 2: tile bits 10, 11, 0, 1, 2   (only for circuits of 11-12 qubits)
+// and the seven thread-index bits are the remaining tile bits in a fixed
+// order.  A 2x2 gate on a qubit that sits in a phase's register bits needs no
+// communication; changing phase is a shared-memory exchange.  The planner
+// decides which qubit each tile bit is.
 #pragma once
 
 #include <stdint.h>
@@ -15,18 +18,19 @@
 namespace qml {
 
 constexpr int kTileBits = 12;  // positions per tile = 4096
-constexpr int kRegBits = 4;    // positions per thread = 16
-constexpr int kThrBits = 8;    // threads per block = 256
+constexpr int kRegBits = 5;    // positions per thread = 32
+constexpr int kThrBits = 7;    // threads per block = 128
 constexpr int kPhases = 3;     // register layouts
 constexpr int kPos = 1 << kRegBits;
 constexpr int kThreads = 1 << kThrBits;
 constexpr int kTilePos = 1 << kTileBits;
-constexpr int kSmemSlots = kTilePos + (kTilePos >> 4);  // one pad slot per 16
+constexpr int kSmemSlots = kTilePos + (kTilePos >> 5);  // slot(t) = t + t / 32
 constexpr int kMaxSet = 10;           // qubits rotated per pass when n > 12
-constexpr int kMaxLayersPerPass = 8;  // cap for circuits that fit one tile
+constexpr int kMaxLayersPerPass = 2;  // cap for circuits that fit one tile
 constexpr int kMaxOut = 30;           // out-of-tile qubits
-constexpr int kMaxOps = 64;
-constexpr int kMaxSlots = kMaxLayersPerPass * kTileBits;
+constexpr int kMaxOps = 24;
+constexpr int kMaxSlots = kMaxLayersPerPass * kTileBits;  // rotations per pass
+constexpr int kCoefRegions = 40;      // per-context regions of constant memory
 
 enum : int { OP_EXCH = 1, OP_ROT = 2, OP_CZ = 3, OP_GEN = 4 };
 
@@ -46,11 +50,11 @@ struct DevPass {
   int nslots;           // rotated (layer, qubit) pairs = gradient slots
   int n_out;            // qubits outside the tile
   int unit_bits;        // batch-unit bits inside the tile
-  int slow;             // a load/store/encode phase has a batch-unit register bit
+  int slow;             // a memory phase has a batch-unit register bit (n < 5)
+  int variant;          // 0: phase-1 lanes are tile bits 0-4; 1: tile bits 0,1,2,10,11
   int tile_q[kTileBits];  // tile bit -> qubit (>= 0) or -1 - (batch-unit bit)
   int out_q[kMaxOut];     // out-of-tile qubits, increasing
   uint32_t cz_reg[kPhases];  // bit j: CZ-ladder parity of the register part of position j
-  int pad_[1];
   long long partial_off;     // float offset of this pass's gradient partials
   int slot_lq[kMaxSlots];    // slot -> layer * n + qubit
   DevOp ops[kMaxOps];        // forward order

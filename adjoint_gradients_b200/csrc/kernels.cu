@@ -28,6 +28,13 @@
 #include "kernels.cuh"
 
 namespace qml {
+
+// Gate coefficients of the current pass, per context region: for slot s,
+// four float4 = broadcast pairs (ar, ai, -ai, br, bi, -bi, -br, 0).  Read
+// through the constant cache with warp-uniform indices, they feed the packed
+// FMAs from uniform registers instead of the vector register file.
+__constant__ float4 c_coef[kCoefRegions][kMaxSlots][4];
+
 namespace {
 
 constexpr unsigned kErrNumeric = 1u << 6;  // bit (QML_ERR_NUMERIC)
@@ -38,9 +45,9 @@ struct Coef {
   float2 ar, ai, nai, br, bi, nbi, nbr;  // broadcast (v, v) pairs
 };
 
-// p points into the block's shared-memory copy of the pass's coefficients.
-__device__ __forceinline__ Coef load_coef(const float4* p) {
-  const float4 f0 = p[0], f1 = p[1], f2 = p[2], f3 = p[3];
+__device__ __forceinline__ Coef const_coef(int region, int slot) {
+  const float4 f0 = c_coef[region][slot][0], f1 = c_coef[region][slot][1];
+  const float4 f2 = c_coef[region][slot][2], f3 = c_coef[region][slot][3];
   Coef c;
   c.ar = make_float2(f0.x, f0.y);
   c.ai = make_float2(f0.z, f0.w);
@@ -114,25 +121,43 @@ __device__ __forceinline__ float3 rot_bwd(float2 (&re)[kPos], float2 (&im)[kPos]
   return make_float3(sx, sy, sz);
 }
 
-__device__ __forceinline__ void rot_fwd_k(int k, float2 (&re)[kPos], float2 (&im)[kPos],
-                                          const Coef& c) {
-  static_assert(kRegBits == 4, "dispatch below covers four register bits");
+__device__ __forceinline__ void rot_fwd_k(int k, float2 (&re)[kPos], float2 (&im)[kPos], const Coef& c) {
+  static_assert(kRegBits == 5, "dispatch below covers five register bits");
   switch (k) {
     case 0: rot_fwd<0>(re, im, c); break;
     case 1: rot_fwd<1>(re, im, c); break;
     case 2: rot_fwd<2>(re, im, c); break;
-    default: rot_fwd<3>(re, im, c); break;
+    case 3: rot_fwd<3>(re, im, c); break;
+    default: rot_fwd<4>(re, im, c); break;
   }
 }
 
-__device__ __forceinline__ float3 rot_bwd_k(int k, float2 (&re)[kPos], float2 (&im)[kPos],
-                                            const Coef& c) {
+__device__ __forceinline__ float3 rot_bwd_k(int k, float2 (&re)[kPos], float2 (&im)[kPos], const Coef& c) {
   switch (k) {
     case 0: return rot_bwd<0>(re, im, c);
     case 1: return rot_bwd<1>(re, im, c);
     case 2: return rot_bwd<2>(re, im, c);
-    default: return rot_bwd<3>(re, im, c);
+    case 3: return rot_bwd<3>(re, im, c);
+    default: return rot_bwd<4>(re, im, c);
   }
+}
+
+// Sum (a, b, c) over the warp with six shuffles; afterwards lanes 0, 8 and 16
+// hold the totals of a, b and c.
+__device__ __forceinline__ float warp_reduce3(float a, float b, float c, int lane) {
+  // 4 values (a, b, c, 0) over 32 lanes: halve the value count at offsets 16 and 8
+  const bool h16 = (lane & 16) != 0;
+  float k0 = h16 ? c : a, k1 = h16 ? 0.f : b;
+  const float s0 = h16 ? a : c, s1 = h16 ? b : 0.f;
+  k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+  k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+  const bool h8 = (lane & 8) != 0;
+  float v = h8 ? k1 : k0;
+  v += __shfl_xor_sync(0xffffffffu, h8 ? k0 : k1, 8);
+  v += __shfl_xor_sync(0xffffffffu, v, 4);
+  v += __shfl_xor_sync(0xffffffffu, v, 2);
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  return v;  // value index (lane >> 3): 0 = a, 1 = b, 2 = c, 3 = pad
 }
 
 __device__ __forceinline__ void flip(float2& v, uint32_t signbit) {
@@ -142,44 +167,63 @@ __device__ __forceinline__ void flip(float2& v, uint32_t signbit) {
 
 // ------------------------------------------------------------ tile geometry
 
-// Shared-memory slot (16 bytes) of tile position t: one pad slot every 16
-// positions keeps every quarter warp on eight different bank groups in all
-// three register layouts.  phys(a | b) = phys(a) + phys(b) for disjoint bits.
-__host__ __device__ constexpr uint32_t phys(uint32_t t) { return t + (t >> 4); }
+// Shared-memory slot (16 bytes) of tile position t: one pad slot every 32
+// positions.  slot(a | b) = slot(a) + slot(b) for disjoint bits, so register
+// offsets are compile-time constants, and in every layout below the eight
+// lanes of a quarter warp hit eight different bank groups.
+__host__ __device__ constexpr uint32_t wbit(int b) { return b < 5 ? (1u << b) : (1u << b) + (1u << (b - 5)); }
 
-__host__ __device__ constexpr size_t align16(size_t v) { return (v + 15) & ~size_t(15); }
-
-// Tile position of (thread tid, register 0) in phase P: the thread bits are the
-// tile bits outside 4P..4P+3, in increasing order.
+// Tile bit addressed by register-index bit k in phase P.
 template <int P>
-__device__ __forceinline__ uint32_t thr_tpos(uint32_t tid) {
-  if constexpr (P == 0) return tid << 4;
-  else if constexpr (P == 1) return (tid & 15u) | ((tid >> 4) << 8);
-  else return tid;
+__host__ __device__ constexpr int reg_tbit(int k) {
+  return P == 0 ? k : P == 1 ? 5 + k : (k < 2 ? 10 + k : k - 2);
 }
 
-// Shared-memory slot offset of register position j in phase P (compile time).
+// Tile bit addressed by thread-index bit m in phase P (V: layout variant).
+template <int P, int V>
+__host__ __device__ constexpr int thr_tbit(int m) {
+  if (P == 0) return 5 + m;  // 5..11
+  if (P == 1) {
+    if (V == 0) return m < 5 ? m : 5 + m;  // 0,1,2,3,4,10,11
+    constexpr int o[7] = {0, 1, 2, 10, 11, 3, 4};
+    return o[m];
+  }
+  constexpr int o2[7] = {5, 6, 7, 3, 4, 8, 9};
+  return o2[m];
+}
+
 template <int P>
 __host__ __device__ constexpr uint32_t reg_slot(int j) {
-  return phys((uint32_t)j << (4 * P));
+  uint32_t s = 0;
+  for (int k = 0; k < kRegBits; ++k)
+    if ((j >> k) & 1) s += wbit(reg_tbit<P>(k));
+  return s;
 }
 
-// Per-block copy of the pass record plus per-thread layout constants.
+template <int P, int V>
+__device__ __forceinline__ uint32_t thr_slot(uint32_t tid) {
+  uint32_t s = 0;
+#pragma unroll
+  for (int m = 0; m < kThrBits; ++m)
+    if ((tid >> m) & 1u) s += wbit(thr_tbit<P, V>(m));
+  return s;
+}
+
+// Per-block tile-bit maps of the pass.
 struct BlockCtx {
-  uint32_t qbit[kTileBits];     // tile bit -> 1 << qubit (0 for a unit bit)
-  uint32_t ubit[kTileBits];     // tile bit -> unit increment (0 for a qubit)
+  uint32_t qbit[kTileBits];  // tile bit -> 1 << qubit (0 for a unit bit)
+  uint32_t ubit[kTileBits];  // tile bit -> unit increment (0 for a qubit)
 };
 
 // Qubit-space index and batch unit of (thread, register 0) in phase P.
-template <int P>
+template <int P, int V>
 __device__ __forceinline__ void thread_pos(const BlockCtx& bc, uint32_t tid, uint32_t* aq, uint32_t* ut) {
-  const uint32_t t = thr_tpos<P>(tid);
   uint32_t q = 0, u = 0;
 #pragma unroll
-  for (int b = 0; b < kTileBits; ++b)
-    if ((t >> b) & 1u) {
-      q |= bc.qbit[b];
-      u += bc.ubit[b];
+  for (int m = 0; m < kThrBits; ++m)
+    if ((tid >> m) & 1u) {
+      q |= bc.qbit[thr_tbit<P, V>(m)];
+      u += bc.ubit[thr_tbit<P, V>(m)];
     }
   *aq = q;
   *ut = u;
@@ -195,8 +239,8 @@ __device__ __forceinline__ RegMaps reg_maps(const BlockCtx& bc) {
   RegMaps m;
 #pragma unroll
   for (int k = 0; k < kRegBits; ++k) {
-    m.q[k] = bc.qbit[P * kRegBits + k];
-    m.u[k] = bc.ubit[P * kRegBits + k];
+    m.q[k] = bc.qbit[reg_tbit<P>(k)];
+    m.u[k] = bc.ubit[reg_tbit<P>(k)];
   }
   return m;
 }
@@ -208,10 +252,10 @@ __device__ __forceinline__ RegMaps reg_maps(const BlockCtx& bc) {
     return r_;                                                    \
   }())
 
-template <int X, int Y>
+template <int X, int Y, int V>
 __device__ __forceinline__ void exchange_t(float2 (&re)[kPos], float2 (&im)[kPos], float4* tile, uint32_t tid) {
-  const uint32_t sx = phys(thr_tpos<X>(tid));
-  const uint32_t sy = phys(thr_tpos<Y>(tid));
+  const uint32_t sx = thr_slot<X, V>(tid);
+  const uint32_t sy = thr_slot<Y, V>(tid);
   __syncthreads();
 #pragma unroll
   for (int j = 0; j < kPos; ++j) tile[sx + reg_slot<X>(j)] = make_float4(re[j].x, re[j].y, im[j].x, im[j].y);
@@ -224,16 +268,16 @@ __device__ __forceinline__ void exchange_t(float2 (&re)[kPos], float2 (&im)[kPos
   }
 }
 
+template <int V>
 __device__ __forceinline__ void exchange(int x, int y, float2 (&re)[kPos], float2 (&im)[kPos], float4* tile,
                                          uint32_t tid) {
-  const int c = x * 3 + y;
-  switch (c) {
-    case 1: exchange_t<0, 1>(re, im, tile, tid); break;
-    case 2: exchange_t<0, 2>(re, im, tile, tid); break;
-    case 3: exchange_t<1, 0>(re, im, tile, tid); break;
-    case 5: exchange_t<1, 2>(re, im, tile, tid); break;
-    case 6: exchange_t<2, 0>(re, im, tile, tid); break;
-    default: exchange_t<2, 1>(re, im, tile, tid); break;
+  switch (x * 3 + y) {
+    case 1: exchange_t<0, 1, V>(re, im, tile, tid); break;
+    case 2: exchange_t<0, 2, V>(re, im, tile, tid); break;
+    case 3: exchange_t<1, 0, V>(re, im, tile, tid); break;
+    case 5: exchange_t<1, 2, V>(re, im, tile, tid); break;
+    case 6: exchange_t<2, 0, V>(re, im, tile, tid); break;
+    default: exchange_t<2, 1, V>(re, im, tile, tid); break;
   }
 }
 
@@ -245,7 +289,7 @@ __device__ __forceinline__ void apply_cz(float2 (&re)[kPos], float2 (&im)[kPos],
   const uint32_t qa = __popc(aq & (aq >> 1)) & 1u;
   const uint32_t m = (aq << 1) ^ (aq >> 1);
   uint32_t w = cz_reg ^ (qa ? 0xffffffffu : 0u);
-  const uint32_t pat[4] = {0xAAAAAAAAu, 0xCCCCCCCCu, 0xF0F0F0F0u, 0xFF00FF00u};
+  const uint32_t pat[5] = {0xAAAAAAAAu, 0xCCCCCCCCu, 0xF0F0F0F0u, 0xFF00FF00u, 0xFFFF0000u};
 #pragma unroll
   for (int k = 0; k < kRegBits; ++k)
     if (m & rq[k]) w ^= pat[k];
@@ -255,24 +299,6 @@ __device__ __forceinline__ void apply_cz(float2 (&re)[kPos], float2 (&im)[kPos],
     flip(re[j], sb);
     flip(im[j], sb);
   }
-}
-
-// Sum 16 per-lane values over the warp with 16 shuffles: afterwards even lane
-// 2i holds the warp total of value i.
-__device__ __forceinline__ void warp_reduce16(float (&v)[16], int lane) {
-#pragma unroll
-  for (int step = 0; step < 4; ++step) {
-    const int off = 16 >> step;        // 16, 8, 4, 2
-    const int half = 8 >> step;        // values kept after this step
-    const bool hi = (lane & off) != 0;
-#pragma unroll
-    for (int i = 0; i < half; ++i) {
-      const float keep = hi ? v[half + i] : v[i];
-      const float send = hi ? v[i] : v[half + i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-    }
-  }
-  v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
 }
 
 // ------------------------------------------------------------------ planes
@@ -291,11 +317,11 @@ struct Planes {
 // What a pass does to HBM at its start or end, in the memory layout P.
 enum MemOp { M_LOAD, M_STORE, M_STORE_STD, M_GEN, M_CKPT_STORE, M_CKPT_RESTORE };
 
-template <bool BWD, bool SLOW, int P, int OP>
+template <bool BWD, bool SLOW, int P, int V, int OP>
 __device__ __forceinline__ void mem_t(const PassArgs& a, const BlockCtx& bc, uint32_t tid, uint32_t base_q,
                                       uint32_t unit_base, float2 (&re)[kPos], float2 (&im)[kPos], int slot) {
   uint32_t aq, ut;
-  thread_pos<P>(bc, tid, &aq, &ut);
+  thread_pos<P, V>(bc, tid, &aq, &ut);
   aq |= base_q;
   ut += unit_base;
   const RegMaps m = reg_maps<P>(bc);
@@ -358,144 +384,118 @@ __device__ __forceinline__ void mem_t(const PassArgs& a, const BlockCtx& bc, uin
   }
 }
 
-template <bool BWD, bool SLOW, int OP>
+template <bool BWD, bool SLOW, int V, int OP>
 __device__ __forceinline__ void mem_op(int phase, const PassArgs& a, const BlockCtx& bc, uint32_t tid,
                                        uint32_t base_q, uint32_t unit_base, float2 (&re)[kPos],
                                        float2 (&im)[kPos], int slot = 0) {
-  switch (phase) {
-    case 0: mem_t<BWD, SLOW, 0, OP>(a, bc, tid, base_q, unit_base, re, im, slot); break;
-    case 1: mem_t<BWD, SLOW, 1, OP>(a, bc, tid, base_q, unit_base, re, im, slot); break;
-    default: mem_t<BWD, SLOW, 2, OP>(a, bc, tid, base_q, unit_base, re, im, slot); break;
-  }
+  // memory ops run in phase 0 or 1 (the planner never picks phase 2)
+  if (phase == 0) mem_t<BWD, SLOW, 0, V, OP>(a, bc, tid, base_q, unit_base, re, im, slot);
+  else mem_t<BWD, SLOW, 1, V, OP>(a, bc, tid, base_q, unit_base, re, im, slot);
 }
 
-template <int P>
+template <int P, int V>
 __device__ __forceinline__ void cz_t(float2 (&re)[kPos], float2 (&im)[kPos], const BlockCtx& bc, uint32_t cz_reg,
                                      uint32_t tid, uint32_t base_q) {
   uint32_t aq, ut;
-  thread_pos<P>(bc, tid, &aq, &ut);
+  thread_pos<P, V>(bc, tid, &aq, &ut);
   const RegMaps m = reg_maps<P>(bc);
   apply_cz(re, im, cz_reg, m.q, aq | base_q);
 }
 
+template <int V>
 __device__ __forceinline__ void cz_op(int phase, float2 (&re)[kPos], float2 (&im)[kPos], const BlockCtx& bc,
                                       uint32_t cz_reg, uint32_t tid, uint32_t base_q) {
   switch (phase) {
-    case 0: cz_t<0>(re, im, bc, cz_reg, tid, base_q); break;
-    case 1: cz_t<1>(re, im, bc, cz_reg, tid, base_q); break;
-    default: cz_t<2>(re, im, bc, cz_reg, tid, base_q); break;
+    case 0: cz_t<0, V>(re, im, bc, cz_reg, tid, base_q); break;
+    case 1: cz_t<1, V>(re, im, bc, cz_reg, tid, base_q); break;
+    default: cz_t<2, V>(re, im, bc, cz_reg, tid, base_q); break;
   }
 }
 
 // ----------------------------------------------------------- the pass kernel
+//
+// One launch runs one pass over every tile of the batch (persistent blocks,
+// tiles assigned round-robin).  The pass record arrives as a kernel parameter
+// so that its ops and slot numbers are uniform across the warp.
 
-template <bool BWD, bool SLOW>
-__global__ void __launch_bounds__(kThreads, 2) pass_kernel(const PassArgs a) {
+template <bool BWD, bool SLOW, int V>
+__global__ void __launch_bounds__(kThreads, 2) pass_kernel(const PassArgs a, const __grid_constant__ DevPass P) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   float4* tile = reinterpret_cast<float4*>(smem_raw);
-  unsigned char* rest = smem_raw + (size_t)kSmemSlots * sizeof(float4);
-  DevPass* P = reinterpret_cast<DevPass*>(rest);
-  BlockCtx* bc = reinterpret_cast<BlockCtx*>(rest + align16(sizeof(DevPass)));
-  float4* coef = reinterpret_cast<float4*>(rest + align16(sizeof(DevPass)) + align16(sizeof(BlockCtx)));
+  BlockCtx* bc = reinterpret_cast<BlockCtx*>(smem_raw + (size_t)kSmemSlots * sizeof(float4));
+  float* acc = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(bc) + sizeof(BlockCtx));  // [warps][nslots*3]
   const uint32_t tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   constexpr int kWarps = kThreads / 32;
+  const int region = a.region;
+  const int nacc = P.nslots * 3;
 
-  // ---- block setup: pass record, tile-bit maps, gate coefficients
-  {
-    const int* src = reinterpret_cast<const int*>(a.passes + a.pass_idx);
-    int* dst = reinterpret_cast<int*>(P);
-    for (int i = tid; i < (int)(sizeof(DevPass) / 4); i += kThreads) dst[i] = src[i];
-  }
-  __syncthreads();
-  const int nslots = P->nslots;
-  float* acc = reinterpret_cast<float*>(coef + 4 * nslots);  // [warps][nslots*3]
-  const int nacc = nslots * 3;
   if (tid < kTileBits) {
-    const int q = P->tile_q[tid];
+    const int q = P.tile_q[tid];
     bc->qbit[tid] = q >= 0 ? (1u << q) : 0u;
     bc->ubit[tid] = q >= 0 ? 0u : (1u << (-1 - q));
   }
-  for (int i = tid; i < 4 * nslots; i += kThreads) coef[i] = __ldg(a.coef + (size_t)P->slot_lq[i >> 2] * 4 + (i & 3));
   if (BWD)
     for (int i = tid; i < kWarps * nacc; i += kThreads) acc[i] = 0.f;
   __syncthreads();
 
-  const int n_out = P->n_out;
-  const int nops = P->nops;
+  const int n_out = P.n_out;
   for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x) {
     const uint32_t o = (uint32_t)t & ((1u << n_out) - 1u);
     const uint32_t ug = (uint32_t)t >> n_out;
     uint32_t base_q = 0;
     for (int k = 0; k < n_out; ++k)
-      if ((o >> k) & 1u) base_q |= 1u << P->out_q[k];
-    const uint32_t unit_base = ug << P->unit_bits;
+      if ((o >> k) & 1u) base_q |= 1u << P.out_q[k];
+    const uint32_t unit_base = ug << P.unit_bits;
 
     float2 re[kPos], im[kPos];
     if (!BWD) {
-      if (P->gen) mem_op<false, SLOW, M_GEN>(P->load_phase, a, *bc, tid, base_q, unit_base, re, im);
-      else mem_op<false, SLOW, M_LOAD>(P->load_phase, a, *bc, tid, base_q, unit_base, re, im);
-      for (int oi = 0; oi < nops; ++oi) {
-        const DevOp op = P->ops[oi];
+      if (P.gen) mem_op<false, SLOW, V, M_GEN>(P.load_phase, a, *bc, tid, base_q, unit_base, re, im);
+      else mem_op<false, SLOW, V, M_LOAD>(P.load_phase, a, *bc, tid, base_q, unit_base, re, im);
+      for (int oi = 0; oi < P.nops; ++oi) {
+        const DevOp op = P.ops[oi];
         if (op.kind == OP_EXCH) {
-          exchange(op.a, op.b, re, im, tile, tid);
+          exchange<V>(op.a, op.b, re, im, tile, tid);
         } else if (op.kind == OP_ROT) {
           int slot = op.d;
 #pragma unroll
           for (int k = 0; k < kRegBits; ++k)
-            if ((op.b >> k) & 1) {
-              const Coef c = load_coef(coef + 4 * slot++);
-              rot_fwd_k(k, re, im, c);
-            }
+            if ((op.b >> k) & 1) rot_fwd_k(k, re, im, const_coef(region, slot++));
         } else if (op.kind == OP_CZ) {
-          cz_op(op.a, re, im, *bc, P->cz_reg[op.a], tid, base_q);
+          cz_op<V>(op.a, re, im, *bc, P.cz_reg[op.a], tid, base_q);
         }
       }
-      if (P->ckpt >= 0) mem_op<false, SLOW, M_CKPT_STORE>(P->store_phase, a, *bc, tid, base_q, unit_base, re, im, P->ckpt);
-      if (P->last) mem_op<false, SLOW, M_STORE_STD>(P->store_phase, a, *bc, tid, base_q, unit_base, re, im);
-      else mem_op<false, SLOW, M_STORE>(P->store_phase, a, *bc, tid, base_q, unit_base, re, im);
+      if (P.ckpt >= 0) mem_op<false, SLOW, V, M_CKPT_STORE>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im, P.ckpt);
+      if (P.last) mem_op<false, SLOW, V, M_STORE_STD>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im);
+      else mem_op<false, SLOW, V, M_STORE>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im);
     } else {
-      mem_op<true, SLOW, M_LOAD>(P->store_phase, a, *bc, tid, base_q, unit_base, re, im);
-      if (P->ckpt >= 0) mem_op<true, SLOW, M_CKPT_RESTORE>(P->store_phase, a, *bc, tid, base_q, unit_base, re, im, P->ckpt);
-      for (int oi = nops - 1; oi >= 0; --oi) {
-        const DevOp op = P->ops[oi];
+      mem_op<true, SLOW, V, M_LOAD>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im);
+      if (P.ckpt >= 0) mem_op<true, SLOW, V, M_CKPT_RESTORE>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im, P.ckpt);
+      for (int oi = P.nops - 1; oi >= 0; --oi) {
+        const DevOp op = P.ops[oi];
         if (op.kind == OP_EXCH) {
-          exchange(op.b, op.a, re, im, tile, tid);
+          exchange<V>(op.b, op.a, re, im, tile, tid);
         } else if (op.kind == OP_ROT) {
-          float s[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) s[i] = 0.f;
           int slot = op.d;
-          int g = 0;
 #pragma unroll
           for (int k = 0; k < kRegBits; ++k)
             if ((op.b >> k) & 1) {
-              const Coef c = load_coef(coef + 4 * slot++);
-              const float3 v = rot_bwd_k(k, re, im, c);
-              // values of gate g sit at 3g .. 3g+2 (g counts the mask bits)
-#pragma unroll
-              for (int gg = 0; gg < kRegBits; ++gg)
-                if (gg == g) {
-                  s[3 * gg] = v.x;
-                  s[3 * gg + 1] = v.y;
-                  s[3 * gg + 2] = v.z;
-                }
-              ++g;
+              const float3 v = rot_bwd_k(k, re, im, const_coef(region, slot));
+              const float r = warp_reduce3(v.x, v.y, v.z, lane);
+              if ((lane & 7) == 0 && lane < 24) acc[warp * nacc + slot * 3 + (lane >> 3)] += r;
+              ++slot;
             }
-          warp_reduce16(s, lane);
-          const int vi = lane >> 1;
-          if (!(lane & 1) && vi < 3 * g) acc[warp * nacc + op.d * 3 + vi] += s[0];
         } else if (op.kind == OP_CZ) {
-          cz_op(op.a, re, im, *bc, P->cz_reg[op.a], tid, base_q);
+          cz_op<V>(op.a, re, im, *bc, P.cz_reg[op.a], tid, base_q);
         }
       }
-      if (!P->gen) mem_op<true, SLOW, M_STORE>(P->load_phase, a, *bc, tid, base_q, unit_base, re, im);
+      if (!P.gen) mem_op<true, SLOW, V, M_STORE>(P.load_phase, a, *bc, tid, base_q, unit_base, re, im);
     }
   }
 
   if (BWD) {
     __syncthreads();
-    float* out = a.partials + P->partial_off + (size_t)blockIdx.x * nacc;
+    float* out = a.partials + P.partial_off + (size_t)blockIdx.x * nacc;
     for (int i = tid; i < nacc; i += kThreads) {
       float v = 0.f;
 #pragma unroll
@@ -507,31 +507,39 @@ __global__ void __launch_bounds__(kThreads, 2) pass_kernel(const PassArgs a) {
 
 // ----------------------------------------------------------------- helpers
 
-// Gate coefficients of U = Rz(g) Ry(b) Rx(a) = [[A, B], [-conj B, conj A]] in
-// fp64, rounded to fp32 broadcast pairs, and of U^dagger = [[conj A, -B], ...].
-__global__ void prep_coef_kernel(const float* theta, int L, int n, float4* cf, float4* ci) {
+// Gate coefficients of every pass slot: U = Rz(g) Ry(b) Rx(a) =
+// [[A, B], [-conj B, conj A]] computed in fp64 and rounded to fp32 broadcast
+// pairs, and U^dagger = [[conj A, -B], ...] for the backward passes.
+// Output: [pass][kMaxSlots][4] float4 per direction.
+__global__ void prep_pass_coef_kernel(const DevPass* passes, int n_passes, const float* theta, float4* cf,
+                                      float4* ci) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= L * n) return;
-  const double al = theta[idx * 3 + 0], be = theta[idx * 3 + 1], ga = theta[idx * 3 + 2];
+  if (idx >= n_passes * kMaxSlots) return;
+  const int p = idx / kMaxSlots, s = idx % kMaxSlots;
+  if (s >= passes[p].nslots) return;
+  const int lq = passes[p].slot_lq[s];
+  const double al = theta[lq * 3 + 0], be = theta[lq * 3 + 1], ga = theta[lq * 3 + 2];
   double sa, ca, sb, cb, sg, cg;
   sincos(0.5 * al, &sa, &ca);
   sincos(0.5 * be, &sb, &cb);
   sincos(0.5 * ga, &sg, &cg);
-  // e^{-i g/2} = cg - i sg
-  const double p_re = cb * ca, p_im = sb * sa;     // (Ry Rx)[0][0]
-  const double q_re = -sb * ca, q_im = -cb * sa;   // (Ry Rx)[0][1]
+  // (Ry Rx)[0][0] = cb ca + i sb sa, (Ry Rx)[0][1] = -sb ca - i cb sa; row 0 of Rz is e^{-i g/2}
+  const double p_re = cb * ca, p_im = sb * sa;
+  const double q_re = -sb * ca, q_im = -cb * sa;
   const double ar = cg * p_re + sg * p_im, ai = cg * p_im - sg * p_re;
   const double br = cg * q_re + sg * q_im, bi = cg * q_im - sg * q_re;
   const float far = (float)ar, fai = (float)ai, fbr = (float)br, fbi = (float)bi;
-  cf[idx * 4 + 0] = make_float4(far, far, fai, fai);
-  cf[idx * 4 + 1] = make_float4(-fai, -fai, fbr, fbr);
-  cf[idx * 4 + 2] = make_float4(fbi, fbi, -fbi, -fbi);
-  cf[idx * 4 + 3] = make_float4(-fbr, -fbr, 0.f, 0.f);
+  float4* f = cf + (size_t)idx * 4;
+  f[0] = make_float4(far, far, fai, fai);
+  f[1] = make_float4(-fai, -fai, fbr, fbr);
+  f[2] = make_float4(fbi, fbi, -fbi, -fbi);
+  f[3] = make_float4(-fbr, -fbr, 0.f, 0.f);
   // U^dagger: A' = conj A, B' = -B
-  ci[idx * 4 + 0] = make_float4(far, far, -fai, -fai);
-  ci[idx * 4 + 1] = make_float4(fai, fai, -fbr, -fbr);
-  ci[idx * 4 + 2] = make_float4(-fbi, -fbi, fbi, fbi);
-  ci[idx * 4 + 3] = make_float4(fbr, fbr, 0.f, 0.f);
+  float4* g = ci + (size_t)idx * 4;
+  g[0] = make_float4(far, far, -fai, -fai);
+  g[1] = make_float4(fai, fai, -fbr, -fbr);
+  g[2] = make_float4(-fbi, -fbi, fbi, fbi);
+  g[3] = make_float4(fbr, fbr, 0.f, 0.f);
 }
 
 // (cos, sin)(x/2) for the two samples of each forward unit.
@@ -681,42 +689,55 @@ __global__ void ckpt_copy_kernel(bool save, const float2* in, float2* out, void*
 }  // namespace
 
 size_t pass_smem_bytes(int max_slots) {
-  return (size_t)kSmemSlots * sizeof(float4) + align16(sizeof(DevPass)) + align16(sizeof(BlockCtx)) +
-         (size_t)max_slots * 4 * sizeof(float4) + (size_t)(kThreads / 32) * max_slots * 3 * sizeof(float);
+  return (size_t)kSmemSlots * sizeof(float4) + sizeof(BlockCtx) + (size_t)(kThreads / 32) * max_slots * 3 * sizeof(float);
 }
 
+#define QML_FOR_EACH_PASS_KERNEL(X) \
+  X(false, false, 0) X(true, false, 0) X(false, true, 0) X(true, true, 0) X(false, false, 1) X(true, false, 1)
+
 cudaError_t set_pass_smem_attr(size_t smem) {
-  const int v = (int)smem;
-  cudaError_t e = cudaFuncSetAttribute(pass_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, v);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(pass_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, v);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(pass_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, v);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(pass_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, v);
+  cudaError_t e = cudaSuccess;
+#define QML_SET_ATTR(B, S, V)                                                                                    \
+  if (e == cudaSuccess)                                                                                          \
+    e = cudaFuncSetAttribute(pass_kernel<B, S, V>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  QML_FOR_EACH_PASS_KERNEL(QML_SET_ATTR)
+#undef QML_SET_ATTR
   return e;
 }
 
 cudaError_t pass_occupancy(bool backward, bool slow, size_t smem, int* blocks_per_sm) {
   if (backward)
-    return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, true>, kThreads, smem)
-                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, false>, kThreads, smem);
-  return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, true>, kThreads, smem)
-              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, false>, kThreads, smem);
+    return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, true, 0>, kThreads, smem)
+                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, false, 0>, kThreads, smem);
+  return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, true, 0>, kThreads, smem)
+              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, false, 0>, kThreads, smem);
 }
 
-cudaError_t launch_pass(bool backward, bool slow, const PassArgs& a, int grid, size_t smem, cudaStream_t s) {
-  if (backward) {
-    if (slow) pass_kernel<true, true><<<grid, kThreads, smem, s>>>(a);
-    else pass_kernel<true, false><<<grid, kThreads, smem, s>>>(a);
+cudaError_t launch_pass(bool backward, const PassArgs& a, const DevPass& p, int grid, size_t smem, cudaStream_t s) {
+  const bool slow = p.slow != 0;
+  if (p.variant == 1) {
+    if (backward) pass_kernel<true, false, 1><<<grid, kThreads, smem, s>>>(a, p);
+    else pass_kernel<false, false, 1><<<grid, kThreads, smem, s>>>(a, p);
+  } else if (slow) {
+    if (backward) pass_kernel<true, true, 0><<<grid, kThreads, smem, s>>>(a, p);
+    else pass_kernel<false, true, 0><<<grid, kThreads, smem, s>>>(a, p);
   } else {
-    if (slow) pass_kernel<false, true><<<grid, kThreads, smem, s>>>(a);
-    else pass_kernel<false, false><<<grid, kThreads, smem, s>>>(a);
+    if (backward) pass_kernel<true, false, 0><<<grid, kThreads, smem, s>>>(a, p);
+    else pass_kernel<false, false, 0><<<grid, kThreads, smem, s>>>(a, p);
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_prep_coef(const float* theta, int L, int n, float4* cf, float4* ci,
-                             cudaStream_t s) {
-  const int tot = L * n;
-  prep_coef_kernel<<<(tot + 127) / 128, 128, 0, s>>>(theta, L, n, cf, ci);
+cudaError_t copy_pass_coef(int region, const float4* src, int nslots, cudaStream_t s) {
+  if (nslots <= 0) return cudaSuccess;
+  const size_t off = (size_t)region * kMaxSlots * 4 * sizeof(float4);
+  return cudaMemcpyToSymbolAsync(c_coef, src, (size_t)nslots * 4 * sizeof(float4), off, cudaMemcpyDeviceToDevice, s);
+}
+
+cudaError_t launch_prep_pass_coef(const DevPass* passes, int n_passes, const float* theta, float4* cf, float4* ci,
+                                  cudaStream_t s) {
+  const int tot = n_passes * kMaxSlots;
+  prep_pass_coef_kernel<<<(tot + 127) / 128, 128, 0, s>>>(passes, n_passes, theta, cf, ci);
   return cudaGetLastError();
 }
 

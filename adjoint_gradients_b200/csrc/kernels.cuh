@@ -10,15 +10,13 @@ namespace qml {
 
 // Arguments of one pass launch (forward or backward).
 struct PassArgs {
-  const DevPass* passes;
-  int pass_idx;
+  int region;            // constant-memory coefficient region of the context
   int n, B, U;           // qubits, samples, batch units (forward: ceil(B/2); backward: B)
   long long N;           // 2^n
   int n_tiles;           // tiles in this pass
   float2* buf0;          // forward: psi; backward: psi (plane 0)
   float2* buf1;          // backward: lambda (plane 1)
   float2* dummy;         // forward: partner plane of the last unit when B is odd
-  const float4* coef;    // [L*n][4] broadcast gate coefficients (forward U, or U^dagger)
   const float2* enc;     // forward: [U][n][2] (cos, sin)(x/2) pairs
   const float* g;        // backward: dL/dE [B]
   void* ckpt;            // checkpoint slots
@@ -30,14 +28,17 @@ struct PassArgs {
 
 size_t pass_smem_bytes(int max_slots);
 
-// `slow`: some register bit indexes a batch unit (only when n < 5); the
-// generic per-position code then replaces the single-unit fast path.
-cudaError_t launch_pass(bool backward, bool slow, const PassArgs& a, int grid, size_t smem, cudaStream_t s);
+// Launch one pass; the kernel instance follows the pass's layout variant and
+// whether a memory layout has a batch-unit register bit (only when n < 5).
+cudaError_t launch_pass(bool backward, const PassArgs& a, const DevPass& p, int grid, size_t smem, cudaStream_t s);
+// Copy one pass's gate coefficients ([nslots][4] float4, device memory) into
+// the context's constant-memory region, in stream order.
+cudaError_t copy_pass_coef(int region, const float4* src, int nslots, cudaStream_t s);
+cudaError_t launch_prep_pass_coef(const DevPass* passes, int n_passes, const float* theta, float4* cf, float4* ci,
+                                  cudaStream_t s);
 cudaError_t set_pass_smem_attr(size_t smem);
 cudaError_t pass_occupancy(bool backward, bool slow, size_t smem, int* blocks_per_sm);
 
-cudaError_t launch_prep_coef(const float* theta, int L, int n, float4* coef_fwd, float4* coef_inv,
-                             cudaStream_t s);
 cudaError_t launch_prep_enc(const float* x, int B, int n, float2* enc, cudaStream_t s);
 cudaError_t launch_expect(const float2* psi, int B, int n, double* partial, float* E,
                           unsigned* status, cudaStream_t s);

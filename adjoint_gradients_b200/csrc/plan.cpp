@@ -13,30 +13,17 @@ struct Task {
   int set;
 };
 
-// Tile bits that are thread-index bits in phase p, in increasing order.
-void thread_tbits(int p, int out[kThrBits]) {
-  int h = 0;
-  for (int t = 0; t < kTileBits; ++t)
-    if (t / kRegBits != p) out[h++] = t;
-}
-
-// How many leading lanes of phase p address consecutive low qubits 0, 1, 2, ...
-// (the longer, the more contiguous a warp's global access).
-int coalesce_score(const HostPass& ps, int p) {
-  int tb[kThrBits];
-  thread_tbits(p, tb);
-  int s = 0;
-  for (int k = 0; k < 5; ++k) {
-    if (ps.tile_q[tb[k]] != k) break;
-    ++s;
-  }
-  return s;
+// Tile bit addressed by register-index bit k in phase p (mirrors the kernels).
+int reg_tbit(int p, int k) {
+  if (p == 0) return k;
+  if (p == 1) return 5 + k;
+  return k < 2 ? 10 + k : k - 2;
 }
 
 // Phase p's register bits are all qubits (no batch-unit bit).
 bool phase_fast(const HostPass& ps, int p) {
   for (int k = 0; k < kRegBits; ++k)
-    if (ps.tile_q[p * kRegBits + k] < 0) return false;
+    if (ps.tile_q[reg_tbit(p, k)] < 0) return false;
   return true;
 }
 
@@ -127,45 +114,55 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
     std::vector<bool> rotated_q(n, false);
     if (S == 1) {
       for (int q = 0; q < n; ++q) rotated_q[q] = true;
+      ps.variant = 0;
       ps.unit_bits = kTileBits - n;
       for (int t = 0; t < kTileBits; ++t) ps.tile_q[t] = t < n ? t : -1 - (t - n);
     } else {
+      // rotated qubits on tile bits 0 .. |R|-1; the lowest other qubits are
+      // passive tile bits.  If the set starts at qubit 0, phase 1's lanes
+      // (tile bits 0-4) are qubits 0-4 (variant 0).  Otherwise the two lowest
+      // passive qubits go to tile bits 10 and 11, which are lanes of phase 1 in
+      // variant 1, so a warp touches runs of four consecutive amplitudes.
       const std::vector<int>& set = p.sets[pr.set];
       std::vector<bool> in(n, false);
-      std::vector<int> tq = set;
       for (int q : set) in[q] = rotated_q[q] = true;
-      for (int q = 0; q < n && (int)tq.size() < kTileBits; ++q)
+      std::vector<int> passive;
+      for (int q = 0; q < n && (int)(set.size() + passive.size()) < kTileBits; ++q)
         if (!in[q]) {
-          tq.push_back(q);
+          passive.push_back(q);
           in[q] = true;
         }
-      std::sort(tq.begin(), tq.end());
       for (int q = 0; q < n; ++q)
         if (!in[q]) ps.out_q.push_back(q);
       ps.unit_bits = 0;
-      for (int t = 0; t < kTileBits; ++t) ps.tile_q[t] = tq[t];
+      ps.variant = set[0] == 0 ? 0 : 1;
+      for (int t = 0; t < (int)set.size(); ++t) ps.tile_q[t] = set[t];
+      if (ps.variant == 0) {
+        for (size_t i = 0; i < passive.size(); ++i) ps.tile_q[set.size() + i] = passive[i];
+      } else {
+        ps.tile_q[10] = passive[0];
+        ps.tile_q[11] = passive[1];
+        for (size_t i = 2; i < passive.size(); ++i) ps.tile_q[set.size() + i - 2] = passive[i];
+      }
     }
     if ((int)ps.out_q.size() > kMaxOut) return "internal: too many out-of-tile qubits";
 
-    // ---- rotated register bits per phase, and the phase that touches HBM
+    // ---- rotated qubits per register group (tile bits 0-4, 5-9, 10-11), and
+    // the phase that touches HBM: phase 1 when its register bits are all
+    // qubits (its lanes are the contiguous tile bits), else phase 0
     int mask[kPhases];
     std::vector<int> active;
     for (int g = 0; g < kPhases; ++g) {
       mask[g] = 0;
-      for (int k = 0; k < kRegBits; ++k) {
-        const int q = ps.tile_q[g * kRegBits + k];
+      const int nk = g == 2 ? 2 : kRegBits;
+      for (int k = 0; k < nk; ++k) {
+        const int q = ps.tile_q[reg_tbit(g, k)];
         if (q >= 0 && rotated_q[q]) mask[g] |= 1 << k;
       }
       if (mask[g]) active.push_back(g);
     }
-    int mem = -1, best = -1;
-    for (int g = kPhases - 1; g >= 0; --g)
-      if (phase_fast(ps, g) && coalesce_score(ps, g) > best) {
-        best = coalesce_score(ps, g);
-        mem = g;
-      }
-    ps.slow = mem < 0;
-    if (mem < 0) mem = 0;
+    int mem = phase_fast(ps, 1) ? 1 : 0;
+    ps.slow = !phase_fast(ps, mem);
     ps.load_phase = mem;
 
     // group order of the first rotation: start in the memory phase when
@@ -182,7 +179,7 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
       // encode directly in the first group's layout when that layout is fast
       std::vector<int> first = order;
       if (!dir) std::reverse(first.begin(), first.end());
-      if (phase_fast(ps, first[0])) cur = first[0];
+      if (first[0] != 2 && phase_fast(ps, first[0])) cur = first[0];  // memory ops use phase 0 or 1
       ps.load_phase = cur;
       ps.ops.push_back({OP_GEN, cur, 0, 0, 0});
     }
@@ -198,7 +195,7 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
           const int slot0 = (int)ps.slot_lq.size();
           for (int k = 0; k < kRegBits; ++k)
             if (mask[g] & (1 << k)) {
-              const int q = ps.tile_q[g * kRegBits + k];
+              const int q = ps.tile_q[reg_tbit(g, k)];
               const size_t idx = (size_t)tk.layer * n + q;
               p.slot_pass[idx] = (int)pi;
               p.slot_index[idx] = (int)ps.slot_lq.size();
@@ -237,6 +234,7 @@ void flatten_plan(const Plan& p, std::vector<DevPass>* passes) {
     d.n_out = (int)ps.out_q.size();
     d.unit_bits = ps.unit_bits;
     d.slow = ps.slow ? 1 : 0;
+    d.variant = ps.variant;
     for (int t = 0; t < kTileBits; ++t) d.tile_q[t] = ps.tile_q[t];
     for (int i = 0; i < kMaxOut; ++i) d.out_q[i] = i < d.n_out ? ps.out_q[i] : -1;
     for (int g = 0; g < kPhases; ++g) {
@@ -244,7 +242,7 @@ void flatten_plan(const Plan& p, std::vector<DevPass>* passes) {
       for (int j = 0; j < kPos; ++j) {
         uint32_t b = 0;
         for (int k = 0; k < kRegBits; ++k) {
-          const int q = ps.tile_q[g * kRegBits + k];
+          const int q = ps.tile_q[reg_tbit(g, k)];
           if ((j >> k) & 1 && q >= 0) b |= 1u << q;
         }
         if (__builtin_popcount(b & (b >> 1)) & 1) w |= 1u << j;
@@ -282,7 +280,7 @@ std::vector<int> describe_plan(const Plan& p) {
         a = o.c;  // layer
         uint32_t qm = 0;
         for (int k = 0; k < kRegBits; ++k)
-          if (o.b & (1 << k)) qm |= 1u << ps.tile_q[o.a * kRegBits + k];
+          if (o.b & (1 << k)) qm |= 1u << ps.tile_q[reg_tbit(o.a, k)];
         b = (int)qm;
         c = o.d;
       } else if (o.kind == OP_CZ) {

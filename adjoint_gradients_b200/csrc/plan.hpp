@@ -10,9 +10,10 @@
 // Qubits are split into sets of at most ten that are rotated together.  A
 // pass owns 12 tile bits: the rotated set plus enough of the lowest other
 // qubits ("passive" bits) to keep HBM accesses contiguous; for n <= 12 the
-// tile is the whole state plus batch-unit bits.  Tile bits are assigned to
-// qubits in increasing order, so the three fixed register groups (tile bits
-// 0-3, 4-7, 8-11; see device_plan.h) each hold up to four rotated qubits.
+// tile is the whole state plus batch-unit bits.  The rotated qubits sit on
+// tile bits 0-9, so the two register groups of five (tile bits 0-4 and 5-9,
+// see device_plan.h) hold them all; circuits of 11-12 qubits also use the
+// third group (tile bits 10-11).
 #pragma once
 
 #include <cstdint>
@@ -39,6 +40,7 @@ struct HostPass {
   int ckpt;                   // checkpoint slot written after this pass, or -1
   std::vector<int> slot_lq;   // gradient slot -> layer * n + qubit
   bool slow;
+  int variant;                // see DevPass::variant
 };
 
 struct Plan {

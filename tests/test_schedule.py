@@ -77,9 +77,9 @@ def test_schedule_replays_the_circuit(n, L, ck):
 
 
 def test_pass_counts_match_the_design():
-    # n <= 12: one pass per 8 layers; n = 20: L + 1 passes (two qubit sets);
+    # n <= 12: one pass per 2 layers; n = 20: L + 1 passes (two qubit sets);
     # n = 29: 2L + 1 passes (three sets, boustrophedon)
-    assert parse(qml.Context(12, 10, 4, workspace=False).debug_schedule()).__len__() == 2
+    assert len(parse(qml.Context(12, 10, 4, workspace=False).debug_schedule())) == 5
     assert len(parse(qml.Context(20, 100, 4, workspace=False).debug_schedule())) == 101
     assert len(parse(qml.Context(29, 20, 4, workspace=False).debug_schedule())) == 41
 
