@@ -52,6 +52,7 @@ struct DevPass {
   int unit_bits;        // batch-unit bits inside the tile
   int slow;             // a memory phase has a batch-unit register bit (n < 5)
   int variant;          // 0: phase-1 lanes are tile bits 0-4; 1: tile bits 0,1,2,10,11
+  int pf_fwd, pf_bwd;   // op index after which the next tile is prefetched (-1: right after loading)
   int tile_q[kTileBits];  // tile bit -> qubit (>= 0) or -1 - (batch-unit bit)
   int out_q[kMaxOut];     // out-of-tile qubits, increasing
   uint32_t cz_reg[kPhases];  // bit j: CZ-ladder parity of the register part of position j

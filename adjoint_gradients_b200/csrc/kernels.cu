@@ -90,35 +90,33 @@ __device__ __forceinline__ void rot_fwd(float2 (&re)[kPos], float2 (&im)[kPos], 
     if (!(j & (1 << K))) su2(re[j], im[j], re[j | (1 << K)], im[j | (1 << K)], c);
 }
 
+__device__ __forceinline__ float2 swap2(float2 v) { return make_float2(v.y, v.x); }
+
 // Gradient terms of one qubit at the state just after its fused rotation, then
 // U^dagger on psi and lambda.  With psi in lane x and lambda in lane y:
 //   s_z = Im<lambda|Z|psi>, s_x = Im<lambda|X|psi>, s_y = Im<lambda|Y|psi>.
 // 2 Re<lambda|(-i/2) P|psi> = Im<lambda|P|psi>, so these are the gradients of
 // the three rotation angles up to a known rotation (applied in grad_reduce).
+// The products lambda * psi are formed as packed products of a pair with a
+// lane-swapped pair, e.g. (p0r, l0r) * (l0i, p0i) = (p0r l0i, l0r p0i), whose
+// lane difference is Im(conj(l0) p0); the differences are taken at the end.
 template <int K>
 __device__ __forceinline__ float3 rot_bwd(float2 (&re)[kPos], float2 (&im)[kPos], const Coef& c) {
-  float sx = 0.f, sy = 0.f, sz = 0.f;
+  float2 ax = make_float2(0.f, 0.f), ay = ax, az0 = ax, az1 = ax;
 #pragma unroll
   for (int j = 0; j < kPos; ++j) {
     if (j & (1 << K)) continue;
     const int jj = j | (1 << K);
-    const float p0r = re[j].x, l0r = re[j].y, p0i = im[j].x, l0i = im[j].y;
-    const float p1r = re[jj].x, l1r = re[jj].y, p1i = im[jj].x, l1i = im[jj].y;
-    sz = fmaf(l0r, p0i, sz);
-    sz = fmaf(-l0i, p0r, sz);
-    sz = fmaf(-l1r, p1i, sz);
-    sz = fmaf(l1i, p1r, sz);
-    sx = fmaf(l0r, p1i, sx);
-    sx = fmaf(-l0i, p1r, sx);
-    sx = fmaf(l1r, p0i, sx);
-    sx = fmaf(-l1i, p0r, sx);
-    sy = fmaf(-l0r, p1r, sy);
-    sy = fmaf(-l0i, p1i, sy);
-    sy = fmaf(l1r, p0r, sy);
-    sy = fmaf(l1i, p0i, sy);
+    const float2 si0 = swap2(im[j]), si1 = swap2(im[jj]), sr1 = swap2(re[jj]);
+    az0 = __ffma2_rn(re[j], si0, az0);   // y - x: Im(conj l0 p0)
+    az1 = __ffma2_rn(re[jj], si1, az1);  // y - x: Im(conj l1 p1)
+    ax = __ffma2_rn(re[j], si1, ax);     // y - x: l0r p1i - p0r l1i
+    ax = __ffma2_rn(re[jj], si0, ax);    // y - x: l1r p0i - p1r l0i
+    ay = __ffma2_rn(re[j], sr1, ay);     // x - y: p0r l1r - l0r p1r
+    ay = __ffma2_rn(im[j], si1, ay);     // x - y: p0i l1i - l0i p1i
     su2(re[j], im[j], re[jj], im[jj], c);
   }
-  return make_float3(sx, sy, sz);
+  return make_float3(ax.y - ax.x, ay.x - ay.y, (az0.y - az0.x) - (az1.y - az1.x));
 }
 
 __device__ __forceinline__ void rot_fwd_k(int k, float2 (&re)[kPos], float2 (&im)[kPos], const Coef& c) {
@@ -393,6 +391,71 @@ __device__ __forceinline__ void mem_op(int phase, const PassArgs& a, const Block
   else mem_t<BWD, SLOW, 1, V, OP>(a, bc, tid, base_q, unit_base, re, im, slot);
 }
 
+// Prefetch of the block's next tile: each thread copies its own positions of
+// the load layout P into the shared-memory slots it will read them from, with
+// cp.async (zero fill for batch units past the end).
+template <bool BWD, int P, int V>
+__device__ __forceinline__ void prefetch_t(const PassArgs& a, const BlockCtx& bc, uint32_t tid, uint32_t base_q,
+                                           uint32_t unit_base, float4* tile) {
+  uint32_t aq, ut;
+  thread_pos<P, V>(bc, tid, &aq, &ut);
+  aq |= base_q;
+  ut += unit_base;
+  const RegMaps m = reg_maps<P>(bc);
+  const bool ok = ut < (uint32_t)a.U;
+  const float2* p0 = Planes<BWD>::p0(a, ok ? ut : 0u) + (ok ? aq : 0u);
+  const float2* p1 = Planes<BWD>::p1(a, ok ? ut : 0u) + (ok ? aq : 0u);
+  const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(tile) + thr_slot<P, V>(tid) * 16u;
+  const int nbytes = ok ? 8 : 0;
+#pragma unroll
+  for (int j = 0; j < kPos; ++j) {
+    const uint32_t b = ok ? REG_COMBINE(m.q, j, |=) : 0u;
+    const uint32_t dst = sbase + reg_slot<P>(j) * 16u;
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(p0 + b), "r"(nbytes) : "memory");
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst + 8u), "l"(p1 + b), "r"(nbytes) : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <bool BWD, int V>
+__device__ __forceinline__ void prefetch_op(int phase, const PassArgs& a, const BlockCtx& bc, uint32_t tid,
+                                            uint32_t base_q, uint32_t unit_base, float4* tile) {
+  if (phase == 0) prefetch_t<BWD, 0, V>(a, bc, tid, base_q, unit_base, tile);
+  else prefetch_t<BWD, 1, V>(a, bc, tid, base_q, unit_base, tile);
+}
+
+// Registers of layout P from the thread's own prefetched slots.
+template <int P, int V>
+__device__ __forceinline__ void load_prefetched_t(float2 (&re)[kPos], float2 (&im)[kPos], const float4* tile,
+                                                  uint32_t tid) {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  const uint32_t s0 = thr_slot<P, V>(tid);
+#pragma unroll
+  for (int j = 0; j < kPos; ++j) {
+    const float4 v = tile[s0 + reg_slot<P>(j)];
+    re[j] = make_float2(v.x, v.y);
+    im[j] = make_float2(v.z, v.w);
+  }
+}
+
+template <int V>
+__device__ __forceinline__ void load_prefetched(int phase, float2 (&re)[kPos], float2 (&im)[kPos], const float4* tile,
+                                                uint32_t tid) {
+  if (phase == 0) load_prefetched_t<0, V>(re, im, tile, tid);
+  else load_prefetched_t<1, V>(re, im, tile, tid);
+}
+
+// Out-of-tile qubit bits and first batch unit of tile t.
+__device__ __forceinline__ void tile_base(const DevPass& P, int t, uint32_t* base_q, uint32_t* unit_base) {
+  const int n_out = P.n_out;
+  const uint32_t o = (uint32_t)t & ((1u << n_out) - 1u);
+  uint32_t bq = 0;
+  for (int k = 0; k < n_out; ++k)
+    if ((o >> k) & 1u) bq |= 1u << P.out_q[k];
+  *base_q = bq;
+  *unit_base = ((uint32_t)t >> n_out) << P.unit_bits;
+}
+
 template <int P, int V>
 __device__ __forceinline__ void cz_t(float2 (&re)[kPos], float2 (&im)[kPos], const BlockCtx& bc, uint32_t cz_reg,
                                      uint32_t tid, uint32_t base_q) {
@@ -439,19 +502,31 @@ __global__ void __launch_bounds__(kThreads, 2) pass_kernel(const PassArgs a, con
     for (int i = tid; i < kWarps * nacc; i += kThreads) acc[i] = 0.f;
   __syncthreads();
 
-  const int n_out = P.n_out;
+  // Loads of the next tile are prefetched into shared memory once the tile
+  // buffer is free (after the pass's last exchange), so their latency hides
+  // behind the last register phase.  Encoding passes and n < 5 load nothing / directly.
+  const bool can_pf = !SLOW && (BWD || !P.gen);
+  const int mem_ph = BWD ? P.store_phase : P.load_phase;
+  const int pf_at = BWD ? P.pf_bwd : P.pf_fwd;  // op index after which to prefetch (-1: after the load)
+  bool have_pf = false;
   for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x) {
-    const uint32_t o = (uint32_t)t & ((1u << n_out) - 1u);
-    const uint32_t ug = (uint32_t)t >> n_out;
-    uint32_t base_q = 0;
-    for (int k = 0; k < n_out; ++k)
-      if ((o >> k) & 1u) base_q |= 1u << P.out_q[k];
-    const uint32_t unit_base = ug << P.unit_bits;
+    uint32_t base_q, unit_base;
+    tile_base(P, t, &base_q, &unit_base);
+    const int tn = t + (int)gridDim.x;
+    const bool pf_next = can_pf && tn < a.n_tiles;
+    auto prefetch_next = [&]() {
+      uint32_t bq, ub;
+      tile_base(P, tn, &bq, &ub);
+      __syncthreads();  // every thread is done reading the tile buffer
+      prefetch_op<BWD, V>(mem_ph, a, *bc, tid, bq, ub, tile);
+    };
 
     float2 re[kPos], im[kPos];
     if (!BWD) {
       if (P.gen) mem_op<false, SLOW, V, M_GEN>(P.load_phase, a, *bc, tid, base_q, unit_base, re, im);
+      else if (have_pf) load_prefetched<V>(P.load_phase, re, im, tile, tid);
       else mem_op<false, SLOW, V, M_LOAD>(P.load_phase, a, *bc, tid, base_q, unit_base, re, im);
+      if (pf_next && pf_at < 0) prefetch_next();
       for (int oi = 0; oi < P.nops; ++oi) {
         const DevOp op = P.ops[oi];
         if (op.kind == OP_EXCH) {
@@ -464,13 +539,16 @@ __global__ void __launch_bounds__(kThreads, 2) pass_kernel(const PassArgs a, con
         } else if (op.kind == OP_CZ) {
           cz_op<V>(op.a, re, im, *bc, P.cz_reg[op.a], tid, base_q);
         }
+        if (pf_next && oi == pf_at) prefetch_next();
       }
       if (P.ckpt >= 0) mem_op<false, SLOW, V, M_CKPT_STORE>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im, P.ckpt);
       if (P.last) mem_op<false, SLOW, V, M_STORE_STD>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im);
       else mem_op<false, SLOW, V, M_STORE>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im);
     } else {
-      mem_op<true, SLOW, V, M_LOAD>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im);
+      if (have_pf) load_prefetched<V>(P.store_phase, re, im, tile, tid);
+      else mem_op<true, SLOW, V, M_LOAD>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im);
       if (P.ckpt >= 0) mem_op<true, SLOW, V, M_CKPT_RESTORE>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im, P.ckpt);
+      if (pf_next && pf_at < 0) prefetch_next();
       for (int oi = P.nops - 1; oi >= 0; --oi) {
         const DevOp op = P.ops[oi];
         if (op.kind == OP_EXCH) {
@@ -488,9 +566,11 @@ __global__ void __launch_bounds__(kThreads, 2) pass_kernel(const PassArgs a, con
         } else if (op.kind == OP_CZ) {
           cz_op<V>(op.a, re, im, *bc, P.cz_reg[op.a], tid, base_q);
         }
+        if (pf_next && oi == pf_at) prefetch_next();
       }
       if (!P.gen) mem_op<true, SLOW, V, M_STORE>(P.load_phase, a, *bc, tid, base_q, unit_base, re, im);
     }
+    have_pf = pf_next;
   }
 
   if (BWD) {

@@ -235,6 +235,13 @@ void flatten_plan(const Plan& p, std::vector<DevPass>* passes) {
     d.unit_bits = ps.unit_bits;
     d.slow = ps.slow ? 1 : 0;
     d.variant = ps.variant;
+    // forward: after the last exchange; backward (ops run in reverse): after the first
+    d.pf_fwd = d.pf_bwd = -1;
+    for (int o = 0; o < (int)ps.ops.size(); ++o)
+      if (ps.ops[o].kind == OP_EXCH) {
+        d.pf_fwd = o;
+        if (d.pf_bwd < 0) d.pf_bwd = o;
+      }
     for (int t = 0; t < kTileBits; ++t) d.tile_q[t] = ps.tile_q[t];
     for (int i = 0; i < kMaxOut; ++i) d.out_q[i] = i < d.n_out ? ps.out_q[i] : -1;
     for (int g = 0; g < kPhases; ++g) {
