@@ -74,6 +74,16 @@ struct qml_ctx {
   };
   std::vector<Span> spans;
   std::vector<cudaEvent_t> spare;
+  // tensor maps of the passes that load by tensor copies, keyed by the view
+  // of the tile and by the buffers they were encoded for
+  struct MapEntry {
+    int pass;  // a pass with this view
+    bool backward;
+    int B;
+    const void *buf0, *buf1;
+    PassMaps maps;
+  };
+  std::vector<MapEntry> maps;
 };
 
 namespace {
@@ -194,6 +204,28 @@ qml_status check_ready(qml_ctx* c, int B) {
   return QML_OK;
 }
 
+bool same_tma_view(const DevPass& x, const DevPass& y) {
+  return std::memcmp(x.tma_kind, y.tma_kind, sizeof(x.tma_kind)) == 0 &&
+         std::memcmp(x.tma_qlo, y.tma_qlo, sizeof(x.tma_qlo)) == 0 &&
+         std::memcmp(x.tma_bits, y.tma_bits, sizeof(x.tma_bits)) == 0;
+}
+
+// Tensor maps for pass p over (buf0, buf1), encoded once per view and buffers.
+const PassMaps* pass_maps(qml_ctx* c, int p, bool backward, int B, const void* buf0, const void* buf1) {
+  static const PassMaps none{};
+  const DevPass& dp = c->dpass[p];
+  if (!dp.tma) return &none;
+  for (const qml_ctx::MapEntry& m : c->maps)
+    if (m.backward == backward && m.B == B && m.buf0 == buf0 && m.buf1 == buf1 && same_tma_view(c->dpass[m.pass], dp))
+      return &m.maps;
+  qml_ctx::MapEntry m{};
+  m.pass = p, m.backward = backward, m.B = B, m.buf0 = buf0, m.buf1 = buf1;
+  if (encode_pass_maps(dp, c->cfg.n_qubits, B, backward, buf0, buf1, &m.maps) != cudaSuccess) return nullptr;
+  if (c->maps.size() >= 64) c->maps.clear();
+  c->maps.push_back(m);
+  return &c->maps.back().maps;
+}
+
 qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, float2* psi,
                        float* expect, cudaStream_t s) {
   const int n = c->cfg.n_qubits;
@@ -228,7 +260,9 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
     a.n_tiles = (int)(((a.U + units_per_tile - 1) / units_per_tile) << dp.n_out);
     e = copy_pass_coef(c->region, cf + (size_t)p * kMaxSlots * 4, dp.nslots, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
-    e = launch_pass(false, a, dp, c->grid_fwd, c->smem, s);
+    const PassMaps* maps = pass_maps(c, p, false, B, psi, a.dummy);
+    if (!maps) return QML_ERR_CUDA;
+    e = launch_pass(false, a, dp, *maps, c->grid_fwd, c->smem, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
     ++c->launches;
     if (dp.ckpt >= 0) c->ckpt_batch[dp.ckpt] = B;
@@ -279,7 +313,9 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
     a.n_tiles = (int)(((a.U + units_per_tile - 1) / units_per_tile) << dp.n_out);
     e = copy_pass_coef(c->region, ci + (size_t)p * kMaxSlots * 4, dp.nslots, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
-    e = launch_pass(true, a, dp, c->grid_bwd, c->smem, s);
+    const PassMaps* maps = pass_maps(c, p, true, B, psi, lam);
+    if (!maps) return QML_ERR_CUDA;
+    e = launch_pass(true, a, dp, *maps, c->grid_bwd, c->smem, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
     ++c->launches;
   }
@@ -413,7 +449,7 @@ qml_status qml_forward_expect(qml_ctx* c, const float* theta, const float* x, in
                               float* expect, void* stream) {
   qml_status st = check_ready(c, B);
   if (st != QML_OK) return st;
-  if (!theta || !x || !psi || !expect || misaligned(psi, 8)) return QML_ERR_INVALID_ARG;
+  if (!theta || !x || !psi || !expect || misaligned(psi, 16)) return QML_ERR_INVALID_ARG;
   DeviceGuard g(c->device);
   return run_forward(c, theta, x, B, reinterpret_cast<float2*>(psi), expect, static_cast<cudaStream_t>(stream));
 }
@@ -422,7 +458,7 @@ qml_status qml_backward_adjoint(qml_ctx* c, const float* theta, const float* x, 
                                 float* lambda, const float* dLdE, float* grad, void* stream) {
   qml_status st = check_ready(c, B);
   if (st != QML_OK) return st;
-  if (!theta || !psi || !lambda || !dLdE || !grad || misaligned(psi, 8) || misaligned(lambda, 8))
+  if (!theta || !psi || !lambda || !dLdE || !grad || misaligned(psi, 16) || misaligned(lambda, 16))
     return QML_ERR_INVALID_ARG;
   if (psi == lambda) return QML_ERR_INVALID_ARG;
   DeviceGuard g(c->device);
@@ -566,6 +602,28 @@ long long qml_launch_count(const qml_ctx* c) { return c ? c->launches : -1; }
 int qml_debug_schedule(const qml_ctx* c, int* out, int cap) {
   if (!c) return -1;
   std::vector<int> v = describe_plan(c->plan);
+  if (out)
+    for (int i = 0; i < cap && i < (int)v.size(); ++i) out[i] = v[i];
+  return (int)v.size();
+}
+
+int qml_debug_tile_view(const qml_ctx* c, int pass, int* out, int cap) {
+  if (!c || pass < 0 || pass >= (int)c->dpass.size()) return -1;
+  const DevPass& d = c->dpass[pass];
+  std::vector<int> v;
+  v.push_back(d.tma);
+  for (int i = 0; i < kTmaRank; ++i) {
+    v.push_back(d.tma_kind[i]);
+    v.push_back(d.tma_qlo[i]);
+    v.push_back(d.tma_bits[i]);
+    v.push_back(d.tma_shift[i]);
+  }
+  for (int b = 0; b < kTileBits; ++b) {
+    v.push_back(d.tile_q[b]);
+    v.push_back(d.sstride[b]);
+  }
+  v.push_back(d.n_out);
+  for (int i = 0; i < d.n_out; ++i) v.push_back(d.out_q[i]);
   if (out)
     for (int i = 0; i < cap && i < (int)v.size(); ++i) out[i] = v[i];
   return (int)v.size();

@@ -23,6 +23,9 @@ constexpr int kThrBits = 7;    // threads per block = 128
 constexpr int kPhases = 3;     // register layouts
 constexpr int kPos = 1 << kRegBits;
 constexpr int kThreads = 1 << kThrBits;
+// Resident pass blocks per SM: 3 x 128 threads x 168 registers fill the
+// register file, 3 x ~69 KB of tile buffer fit the shared memory.
+constexpr int kBlocksPerSm = 3;
 constexpr int kTilePos = 1 << kTileBits;
 constexpr int kSmemSlots = kTilePos + (kTilePos >> 5);  // slot(t) = t + t / 32
 constexpr int kMaxSet = 10;           // qubits rotated per pass when n > 12
@@ -33,6 +36,17 @@ constexpr int kMaxSlots = kMaxLayersPerPass * kTileBits;  // rotations per pass
 constexpr int kCoefRegions = 40;      // per-context regions of constant memory
 
 enum : int { OP_EXCH = 1, OP_ROT = 2, OP_CZ = 3, OP_GEN = 4 };
+
+// Tensor-copy (TMA) view of a pass's tile, used when n > 12: the state
+// [B][2^n] is seen as a rank-5 tensor whose dimensions are runs of qubits
+// (in increasing qubit order) plus the sample index.  A run of in-tile qubits
+// is copied whole (box = 2^bits, at most 8 bits per dimension); a run of
+// out-of-tile qubits is fixed per tile (box 1, coordinate = those bits of the
+// tile's out-of-tile index); the sample dimension has box 1, merged with the
+// highest qubit run when that run is out of the tile.  Unused dimensions have
+// size 1.
+constexpr int kTmaRank = 5;
+enum : int { TD_PAD = 0, TD_IN = 1, TD_OUT = 2, TD_SAMPLE = 3, TD_OUT_SAMPLE = 4 };
 
 // OP_EXCH: a = from phase, b = to phase
 // OP_ROT : a = phase, b = register-bit mask, c = layer, d = first slot
@@ -53,6 +67,12 @@ struct DevPass {
   int slow;             // a memory phase has a batch-unit register bit (n < 5)
   int variant;          // 0: phase-1 lanes are tile bits 0-4; 1: tile bits 0,1,2,10,11
   int pf_fwd, pf_bwd;   // op index after which the next tile is prefetched (-1: right after loading)
+  int tma;              // 1: tiles are loaded by tensor copies (see kTmaRank)
+  int tma_kind[kTmaRank];
+  int tma_qlo[kTmaRank];    // lowest qubit of the run (TD_IN, TD_OUT, TD_OUT_SAMPLE)
+  int tma_bits[kTmaRank];   // qubits in the run
+  int tma_shift[kTmaRank];  // TD_OUT, TD_OUT_SAMPLE: first bit of the run in the out-of-tile index
+  int sstride[kTileBits];   // element offset in the copied tile of each tile bit (plane 1 at +4096)
   int tile_q[kTileBits];  // tile bit -> qubit (>= 0) or -1 - (batch-unit bit)
   int out_q[kMaxOut];     // out-of-tile qubits, increasing
   uint32_t cz_reg[kPhases];  // bit j: CZ-ladder parity of the register part of position j

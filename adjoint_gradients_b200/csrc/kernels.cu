@@ -23,7 +23,11 @@
 // the re pairs and plane 1 the im pairs, each as [2^n] float2 at the same
 // byte positions the standard (re, im) layout uses, so converting between
 // layouts is always in place.
+#include <cuda.h>
 #include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
 
 #include "kernels.cuh"
 
@@ -38,6 +42,11 @@ __constant__ float4 c_coef[kCoefRegions][kMaxSlots][4];
 namespace {
 
 constexpr unsigned kErrNumeric = 1u << 6;  // bit (QML_ERR_NUMERIC)
+constexpr unsigned kErrBounds = 1u << 7;   // bit (QML_ERR_BOUNDS)
+constexpr unsigned kErrTimeout = 1u << 8;  // bit (QML_ERR_TIMEOUT)
+// Polls of an mbarrier before a wait is declared failed (each poll may
+// suspend the thread briefly, so this bounds the wait to well under a second).
+constexpr uint32_t kWaitLimit = 1u << 22;
 
 // ---------------------------------------------------------------- gate math
 
@@ -211,6 +220,9 @@ __device__ __forceinline__ uint32_t thr_slot(uint32_t tid) {
 struct BlockCtx {
   uint32_t qbit[kTileBits];  // tile bit -> 1 << qubit (0 for a unit bit)
   uint32_t ubit[kTileBits];  // tile bit -> unit increment (0 for a qubit)
+  unsigned long long mbar;   // completion barrier of the tile's tensor copies
+  int tma_c[2][kTmaRank];    // tensor coordinates of the next tile's copies
+  int tma_sel;               // plane 1 of the next tile comes through tm1
 };
 
 // Qubit-space index and batch unit of (thread, register 0) in phase P.
@@ -445,6 +457,127 @@ __device__ __forceinline__ void load_prefetched(int phase, float2 (&re)[kPos], f
   else load_prefetched_t<1, V>(re, im, tile, tid);
 }
 
+
+// ------------------------------------------------ tensor-copy (TMA) tile loads
+//
+// With a tensor map per plane buffer, one thread loads a whole tile (both
+// planes, 64 KB) into the shared tile buffer with two bulk tensor copies that
+// signal an mbarrier; no other thread issues a memory instruction for it.  The
+// copied layout is the tensor's dimension order (see kTmaRank); sstride gives
+// each tile bit's element offset in it, plane 1 sits 4096 elements after
+// plane 0.
+
+// Tensor coordinates of both planes of tile `tile` (computed by the issuing
+// thread ahead of time, so that the issue point needs few registers).  In the
+// forward pass plane 1 of unit u is sample 2u+1; when that sample does not
+// exist (odd B, last unit) the plane lives in the one-sample partner buffer,
+// whose map is tm1, at sample 0.
+__device__ __forceinline__ void tma_coords(const DevPass& P, bool bwd, int B, int tile, int (&c)[2][kTmaRank],
+                                           int* sel) {
+  const uint32_t o = (uint32_t)tile & ((1u << P.n_out) - 1u);
+  const uint32_t u = (uint32_t)tile >> P.n_out;
+  const bool partner = !bwd && 2u * u + 1u >= (uint32_t)B;
+  *sel = bwd || partner;
+#pragma unroll
+  for (int p = 0; p < 2; ++p) {
+    const uint32_t smp = bwd ? u : (p == 1 && partner) ? 0u : 2u * u + (uint32_t)p;
+#pragma unroll
+    for (int d = 0; d < kTmaRank; ++d) {
+      const int k = P.tma_kind[d];
+      const uint32_t ob = (o >> P.tma_shift[d]) & ((1u << P.tma_bits[d]) - 1u);
+      c[p][d] = k == TD_OUT ? (int)ob : k == TD_SAMPLE ? (int)smp : k == TD_OUT_SAMPLE ? (int)(ob | (smp << P.tma_bits[d])) : 0;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_tile(const CUtensorMap* m0, const CUtensorMap* m1, int sel,
+                                              const int (&c)[2][kTmaRank], uint32_t dst, uint32_t mbar) {
+  // the shared buffer was last written through the generic proxy (exchanges)
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(kTilePos * 16) : "memory");
+#pragma unroll
+  for (int p = 0; p < 2; ++p) {
+    const CUtensorMap* m = (p == 1 && sel) ? m1 : m0;
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, "
+        "%6}], [%7];" ::"r"(dst + (uint32_t)p * (kTilePos * 8)),
+        "l"(m), "r"(c[p][0]), "r"(c[p][1]), "r"(c[p][2]), "r"(c[p][3]), "r"(c[p][4]), "r"(mbar)
+        : "memory");
+  }
+}
+
+// Bounded wait for the phase with the given parity; false if it never came.
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(mbar), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+
+// Registers of layout P from the copied tile.
+template <int P, int V>
+__device__ __forceinline__ void load_tma_t(float2 (&re)[kPos], float2 (&im)[kPos], const float2* buf,
+                                           const DevPass& Pp, uint32_t tid) {
+  uint32_t s0 = 0;
+#pragma unroll
+  for (int m = 0; m < kThrBits; ++m)
+    if ((tid >> m) & 1u) s0 += (uint32_t)Pp.sstride[thr_tbit<P, V>(m)];
+  uint32_t r[kRegBits];
+#pragma unroll
+  for (int k = 0; k < kRegBits; ++k) r[k] = (uint32_t)Pp.sstride[reg_tbit<P>(k)];
+#pragma unroll
+  for (int j = 0; j < kPos; ++j) {
+    const uint32_t off = s0 + REG_COMBINE(r, j, +=);
+    re[j] = buf[off];
+    im[j] = buf[off + kTilePos];
+  }
+}
+
+// Backward checkpoint restore on the copied tile: replace the psi lanes of
+// this thread's positions (layout P) with the slot's values, before the tile
+// is read into registers (so no state registers are live here).
+template <int P, int V>
+__device__ __forceinline__ void restore_tma_t(const PassArgs& a, const BlockCtx& bc, const DevPass& Pp, uint32_t tid,
+                                              uint32_t base_q, uint32_t unit_base, float2* buf, int slot) {
+  uint32_t aq, ut;
+  thread_pos<P, V>(bc, tid, &aq, &ut);
+  aq |= base_q;
+  ut += unit_base;
+  if (ut >= (uint32_t)a.U) return;
+  uint32_t s0 = 0;
+#pragma unroll
+  for (int m = 0; m < kThrBits; ++m)
+    if ((tid >> m) & 1u) s0 += (uint32_t)Pp.sstride[thr_tbit<P, V>(m)];
+  const RegMaps m = reg_maps<P>(bc);
+  const size_t e0 = ((size_t)slot * a.bmax + ut) * a.N;
+#pragma unroll 4
+  for (int j = 0; j < kPos; ++j) {
+    uint32_t off = s0;
+#pragma unroll
+    for (int k = 0; k < kRegBits; ++k)
+      if ((j >> k) & 1) off += (uint32_t)Pp.sstride[reg_tbit<P>(k)];
+    const size_t e = e0 + (aq | REG_COMBINE(m.q, j, |=));
+    float2 v;
+    if (a.storage == 0) v = reinterpret_cast<const float2*>(a.ckpt)[e];
+    else v = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(a.ckpt)[e]);
+    buf[off].x = v.x;
+    buf[off + kTilePos].x = v.y;
+  }
+}
+
+template <int V>
+__device__ __forceinline__ void load_tma(int phase, float2 (&re)[kPos], float2 (&im)[kPos], const float2* buf,
+                                         const DevPass& Pp, uint32_t tid) {
+  if (phase == 0) load_tma_t<0, V>(re, im, buf, Pp, tid);
+  else load_tma_t<1, V>(re, im, buf, Pp, tid);
+}
+
 // Out-of-tile qubit bits and first batch unit of tile t.
 __device__ __forceinline__ void tile_base(const DevPass& P, int t, uint32_t* base_q, uint32_t* unit_base) {
   const int n_out = P.n_out;
@@ -480,10 +613,18 @@ __device__ __forceinline__ void cz_op(int phase, float2 (&re)[kPos], float2 (&im
 // One launch runs one pass over every tile of the batch (persistent blocks,
 // tiles assigned round-robin).  The pass record arrives as a kernel parameter
 // so that its ops and slot numbers are uniform across the warp.
+//
+// MODE 0: a memory layout has a batch-unit register bit (n < 5), generic
+// addressing.  MODE 1: tiles are loaded by the threads (the next tile with
+// cp.async).  MODE 2: tiles are loaded by tensor copies through tm0 / tm1.
 
-template <bool BWD, bool SLOW, int V>
-__global__ void __launch_bounds__(kThreads, 2) pass_kernel(const PassArgs a, const __grid_constant__ DevPass P) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+template <bool BWD, int MODE, int V>
+__global__ void __launch_bounds__(kThreads, kBlocksPerSm)
+    pass_kernel(const PassArgs a, const __grid_constant__ DevPass P, const __grid_constant__ CUtensorMap tm0,
+                const __grid_constant__ CUtensorMap tm1) {
+  constexpr bool SLOW = MODE == 0;
+  constexpr bool TMA = MODE == 2;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
   float4* tile = reinterpret_cast<float4*>(smem_raw);
   BlockCtx* bc = reinterpret_cast<BlockCtx*>(smem_raw + (size_t)kSmemSlots * sizeof(float4));
   float* acc = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(bc) + sizeof(BlockCtx));  // [warps][nslots*3]
@@ -492,6 +633,9 @@ __global__ void __launch_bounds__(kThreads, 2) pass_kernel(const PassArgs a, con
   constexpr int kWarps = kThreads / 32;
   const int region = a.region;
   const int nacc = P.nslots * 3;
+  const bool loads = BWD || !P.gen;  // the forward's encoding pass reads nothing
+  const uint32_t tile_s = (uint32_t)__cvta_generic_to_shared(tile);
+  const uint32_t mbar = (uint32_t)__cvta_generic_to_shared(&bc->mbar);
 
   if (tid < kTileBits) {
     const int q = P.tile_q[tid];
@@ -500,12 +644,28 @@ __global__ void __launch_bounds__(kThreads, 2) pass_kernel(const PassArgs a, con
   }
   if (BWD)
     for (int i = tid; i < kWarps * nacc; i += kThreads) acc[i] = 0.f;
+  if (TMA) {
+    if ((tile_s & 127u) != 0) {  // tensor copies need a 128-byte aligned destination
+      if (tid == 0) atomicOr(a.status, kErrBounds);
+      return;
+    }
+    if (tid == 0) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(mbar) : "memory");
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+  }
   __syncthreads();
+  if (TMA && loads && tid == 0 && (int)blockIdx.x < a.n_tiles) {
+    tma_coords(P, BWD, a.B, blockIdx.x, bc->tma_c, &bc->tma_sel);
+    tma_load_tile(&tm0, &tm1, bc->tma_sel, bc->tma_c, tile_s, mbar);
+  }
+  uint32_t parity = 0;
 
-  // Loads of the next tile are prefetched into shared memory once the tile
-  // buffer is free (after the pass's last exchange), so their latency hides
-  // behind the last register phase.  Encoding passes and n < 5 load nothing / directly.
-  const bool can_pf = !SLOW && (BWD || !P.gen);
+  // The next tile is fetched into the shared tile buffer once the buffer is
+  // free (after the pass's last exchange), so its latency hides behind the last
+  // register phase.  n < 5 loads directly.
+  const bool can_pf = !SLOW && loads;
   const int mem_ph = BWD ? P.store_phase : P.load_phase;
   const int pf_at = BWD ? P.pf_bwd : P.pf_fwd;  // op index after which to prefetch (-1: after the load)
   bool have_pf = false;
@@ -515,16 +675,41 @@ __global__ void __launch_bounds__(kThreads, 2) pass_kernel(const PassArgs a, con
     const int tn = t + (int)gridDim.x;
     const bool pf_next = can_pf && tn < a.n_tiles;
     auto prefetch_next = [&]() {
-      uint32_t bq, ub;
-      tile_base(P, tn, &bq, &ub);
-      __syncthreads();  // every thread is done reading the tile buffer
-      prefetch_op<BWD, V>(mem_ph, a, *bc, tid, bq, ub, tile);
+      __syncthreads();  // every thread is done with the tile buffer
+      if (TMA) {
+        if (tid == 0) tma_load_tile(&tm0, &tm1, bc->tma_sel, bc->tma_c, tile_s, mbar);
+      } else {
+        uint32_t bq, ub;
+        tile_base(P, tn, &bq, &ub);
+        prefetch_op<BWD, V>(mem_ph, a, *bc, tid, bq, ub, tile);
+      }
     };
 
+    if (TMA && pf_next && tid == 0) tma_coords(P, BWD, a.B, tn, bc->tma_c, &bc->tma_sel);
     float2 re[kPos], im[kPos];
+    if (TMA && loads) {
+      const uint32_t ph = parity;
+      parity ^= 1u;
+      const bool ok = mbar_wait(mbar, ph);
+      if (__syncthreads_or(!ok)) {
+        // the copy never completed: report, give it one more bounded wait, stop
+        if (tid == 0) {
+          atomicOr(a.status, kErrTimeout);
+          mbar_wait(mbar, ph);
+        }
+        return;
+      }
+      float2* tb = reinterpret_cast<float2*>(tile);
+      if (BWD && P.ckpt >= 0) {
+        if (mem_ph == 0) restore_tma_t<0, V>(a, *bc, P, tid, base_q, unit_base, tb, P.ckpt);
+        else restore_tma_t<1, V>(a, *bc, P, tid, base_q, unit_base, tb, P.ckpt);
+      }
+      load_tma<V>(mem_ph, re, im, tb, P, tid);
+    }
     if (!BWD) {
       if (P.gen) mem_op<false, SLOW, V, M_GEN>(P.load_phase, a, *bc, tid, base_q, unit_base, re, im);
-      else if (have_pf) load_prefetched<V>(P.load_phase, re, im, tile, tid);
+      else if (TMA) {
+      } else if (have_pf) load_prefetched<V>(P.load_phase, re, im, tile, tid);
       else mem_op<false, SLOW, V, M_LOAD>(P.load_phase, a, *bc, tid, base_q, unit_base, re, im);
       if (pf_next && pf_at < 0) prefetch_next();
       for (int oi = 0; oi < P.nops; ++oi) {
@@ -545,9 +730,10 @@ __global__ void __launch_bounds__(kThreads, 2) pass_kernel(const PassArgs a, con
       if (P.last) mem_op<false, SLOW, V, M_STORE_STD>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im);
       else mem_op<false, SLOW, V, M_STORE>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im);
     } else {
-      if (have_pf) load_prefetched<V>(P.store_phase, re, im, tile, tid);
+      if (TMA) {
+      } else if (have_pf) load_prefetched<V>(P.store_phase, re, im, tile, tid);
       else mem_op<true, SLOW, V, M_LOAD>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im);
-      if (P.ckpt >= 0) mem_op<true, SLOW, V, M_CKPT_RESTORE>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im, P.ckpt);
+      if (!TMA && P.ckpt >= 0) mem_op<true, SLOW, V, M_CKPT_RESTORE>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im, P.ckpt);
       if (pf_next && pf_at < 0) prefetch_next();
       for (int oi = P.nops - 1; oi >= 0; --oi) {
         const DevOp op = P.ops[oi];
@@ -773,13 +959,16 @@ size_t pass_smem_bytes(int max_slots) {
 }
 
 #define QML_FOR_EACH_PASS_KERNEL(X) \
-  X(false, false, 0) X(true, false, 0) X(false, true, 0) X(true, true, 0) X(false, false, 1) X(true, false, 1)
+  X(false, 0, 0) X(true, 0, 0) X(false, 1, 0) X(true, 1, 0) X(false, 1, 1) X(true, 1, 1) X(false, 2, 0) X(true, 2, 0) \
+  X(false, 2, 1) X(true, 2, 1)
 
 cudaError_t set_pass_smem_attr(size_t smem) {
   cudaError_t e = cudaSuccess;
 #define QML_SET_ATTR(B, S, V)                                                                                    \
   if (e == cudaSuccess)                                                                                          \
-    e = cudaFuncSetAttribute(pass_kernel<B, S, V>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(pass_kernel<B, S, V>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+  if (e == cudaSuccess)                                                                                          \
+    e = cudaFuncSetAttribute(pass_kernel<B, S, V>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   QML_FOR_EACH_PASS_KERNEL(QML_SET_ATTR)
 #undef QML_SET_ATTR
   return e;
@@ -787,25 +976,84 @@ cudaError_t set_pass_smem_attr(size_t smem) {
 
 cudaError_t pass_occupancy(bool backward, bool slow, size_t smem, int* blocks_per_sm) {
   if (backward)
-    return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, true, 0>, kThreads, smem)
-                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, false, 0>, kThreads, smem);
-  return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, true, 0>, kThreads, smem)
-              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, false, 0>, kThreads, smem);
+    return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, 0, 0>, kThreads, smem)
+                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, 2, 1>, kThreads, smem);
+  return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, 0, 0>, kThreads, smem)
+              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, 2, 1>, kThreads, smem);
 }
 
-cudaError_t launch_pass(bool backward, const PassArgs& a, const DevPass& p, int grid, size_t smem, cudaStream_t s) {
-  const bool slow = p.slow != 0;
-  if (p.variant == 1) {
-    if (backward) pass_kernel<true, false, 1><<<grid, kThreads, smem, s>>>(a, p);
-    else pass_kernel<false, false, 1><<<grid, kThreads, smem, s>>>(a, p);
-  } else if (slow) {
-    if (backward) pass_kernel<true, true, 0><<<grid, kThreads, smem, s>>>(a, p);
-    else pass_kernel<false, true, 0><<<grid, kThreads, smem, s>>>(a, p);
-  } else {
-    if (backward) pass_kernel<true, false, 0><<<grid, kThreads, smem, s>>>(a, p);
-    else pass_kernel<false, false, 0><<<grid, kThreads, smem, s>>>(a, p);
+cudaError_t launch_pass(bool backward, const PassArgs& a, const DevPass& p, const PassMaps& maps, int grid,
+                        size_t smem, cudaStream_t s) {
+  const int mode = p.slow ? 0 : p.tma ? 2 : 1;
+  const CUtensorMap& m0 = *reinterpret_cast<const CUtensorMap*>(maps.m0);
+  const CUtensorMap& m1 = *reinterpret_cast<const CUtensorMap*>(maps.m1);
+#define QML_LAUNCH(B, M, V)                                                                 \
+  if (backward == B && mode == M && p.variant == V) {                                       \
+    pass_kernel<B, M, V><<<grid, kThreads, smem, s>>>(a, p, m0, m1);                        \
+    return cudaGetLastError();                                                              \
   }
-  return cudaGetLastError();
+  QML_FOR_EACH_PASS_KERNEL(QML_LAUNCH)
+#undef QML_LAUNCH
+  return cudaErrorInvalidValue;
+}
+
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+bool g_encode_probed = false;
+}  // namespace
+
+cudaError_t encode_pass_maps(const DevPass& p, int n, int B, bool backward, const void* buf0, const void* buf1,
+                             PassMaps* maps) {
+  // forward: buf1 is the one-sample partner buffer of an odd batch's last unit
+  const int samples[2] = {B, backward ? B : 1};
+  std::memset(maps, 0, sizeof(*maps));
+  if (!p.tma) return cudaSuccess;
+  if (!g_encode_probed) {
+    g_encode_probed = true;
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    cudaGetLastError();
+  }
+  if (!g_encode_tiled) return cudaErrorNotSupported;
+  void* bases[2] = {const_cast<void*>(buf0), const_cast<void*>(buf1)};
+  void* outs[2] = {maps->m0, maps->m1};
+  if (p.tma_kind[0] != TD_IN || p.tma_qlo[0] != 0) return cudaErrorInvalidValue;
+  for (int i = 0; i < 2; ++i) {
+    if (!bases[i] || (reinterpret_cast<uintptr_t>(bases[i]) & 15u)) return cudaErrorInvalidValue;
+    cuuint64_t dims[kTmaRank], strides[kTmaRank];
+    cuuint32_t box[kTmaRank], estr[kTmaRank];
+    const cuuint64_t esz = sizeof(float2);
+    for (int d = 0; d < kTmaRank; ++d) {
+      const int k = p.tma_kind[d];
+      estr[d] = 1;
+      if (k == TD_IN || k == TD_OUT) {
+        dims[d] = 1ull << p.tma_bits[d];
+        strides[d] = esz << p.tma_qlo[d];
+        box[d] = k == TD_IN ? (cuuint32_t)(1u << p.tma_bits[d]) : 1u;
+      } else if (k == TD_SAMPLE) {
+        dims[d] = (cuuint64_t)samples[i];
+        strides[d] = esz << n;
+        box[d] = 1;
+      } else if (k == TD_OUT_SAMPLE) {
+        dims[d] = (cuuint64_t)samples[i] << p.tma_bits[d];
+        strides[d] = esz << p.tma_qlo[d];
+        box[d] = 1;
+      } else {  // padding
+        dims[d] = 1;
+        strides[d] = d > 0 ? strides[d - 1] * dims[d - 1] : esz;
+        box[d] = 1;
+      }
+    }
+    CUresult r = g_encode_tiled(reinterpret_cast<CUtensorMap*>(outs[i]), CU_TENSOR_MAP_DATA_TYPE_FLOAT64, kTmaRank,
+                                bases[i], dims, strides + 1, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t copy_pass_coef(int region, const float4* src, int nslots, cudaStream_t s) {

@@ -28,9 +28,22 @@ struct PassArgs {
 
 size_t pass_smem_bytes(int max_slots);
 
+// Tensor maps (CUtensorMap, 128 bytes each) of a pass whose tiles are loaded
+// by tensor copies.  Backward: m0 over psi (plane 0), m1 over lambda (plane 1).
+// Forward: m0 over psi (planes 0 and 1 of unit u at samples 2u, 2u+1), m1 over
+// the one-sample partner buffer that holds plane 1 of an odd batch's last unit.
+struct PassMaps {
+  alignas(64) unsigned char m0[128];
+  alignas(64) unsigned char m1[128];
+};
+// Encode the maps of pass p over (buf0, buf1) (no-op when !p.tma).
+cudaError_t encode_pass_maps(const DevPass& p, int n, int B, bool backward, const void* buf0, const void* buf1,
+                             PassMaps* maps);
+
 // Launch one pass; the kernel instance follows the pass's layout variant and
-// whether a memory layout has a batch-unit register bit (only when n < 5).
-cudaError_t launch_pass(bool backward, const PassArgs& a, const DevPass& p, int grid, size_t smem, cudaStream_t s);
+// how its tiles are loaded (n < 5: generic; tensor copies when p.tma).
+cudaError_t launch_pass(bool backward, const PassArgs& a, const DevPass& p, const PassMaps& maps, int grid,
+                        size_t smem, cudaStream_t s);
 // Copy one pass's gate coefficients ([nslots][4] float4, device memory) into
 // the context's constant-memory region, in stream order.
 cudaError_t copy_pass_coef(int region, const float4* src, int nslots, cudaStream_t s);

@@ -27,6 +27,53 @@ bool phase_fast(const HostPass& ps, int p) {
   return true;
 }
 
+
+// Tensor-copy view of the tile (see kTmaRank).  Multi-set plans only: their
+// tiles hold no batch-unit bit, qubit 0 is always in the tile (rotated or
+// passive), and at least two low qubits are, so the innermost run is >= 32 B.
+void set_tma_view(int n, const HostPass& ps, DevPass* d) {
+  d->tma = 0;
+  for (int i = 0; i < kTmaRank; ++i) d->tma_kind[i] = TD_PAD, d->tma_qlo[i] = d->tma_bits[i] = d->tma_shift[i] = 0;
+  for (int b = 0; b < kTileBits; ++b) d->sstride[b] = 0;
+  if (n <= kTileBits || ps.slow || ps.unit_bits != 0) return;
+  std::vector<int> tbit_of_q(n, -1);
+  for (int b = 0; b < kTileBits; ++b)
+    if (ps.tile_q[b] >= 0) tbit_of_q[ps.tile_q[b]] = b;
+  if (tbit_of_q[0] < 0 || tbit_of_q[1] < 0) return;
+  int rank = 0, out_seen = 0;
+  long long box = 1;  // elements of the box below the current dimension
+  int q = 0;
+  while (q < n) {
+    const bool in = tbit_of_q[q] >= 0;
+    int e = q;
+    while (e < n && (tbit_of_q[e] >= 0) == in) ++e;
+    if (in) {
+      for (int lo = q; lo < e; lo += 8) {
+        const int bits = std::min(8, e - lo);
+        if (rank == kTmaRank) return;
+        d->tma_kind[rank] = TD_IN, d->tma_qlo[rank] = lo, d->tma_bits[rank] = bits;
+        for (int k = 0; k < bits; ++k) d->sstride[tbit_of_q[lo + k]] = (int)(box << k);
+        box <<= bits;
+        ++rank;
+      }
+    } else {
+      if (rank == kTmaRank) return;
+      d->tma_kind[rank] = e == n ? TD_OUT_SAMPLE : TD_OUT;
+      d->tma_qlo[rank] = q, d->tma_bits[rank] = e - q, d->tma_shift[rank] = out_seen;
+      out_seen += e - q;
+      ++rank;
+    }
+    q = e;
+  }
+  if (tbit_of_q[n - 1] >= 0) {  // highest qubit in the tile: a separate sample dimension
+    if (rank == kTmaRank) return;
+    d->tma_kind[rank] = TD_SAMPLE;
+    ++rank;
+  }
+  if (box != kTilePos) return;
+  d->tma = 1;
+}
+
 }  // namespace
 
 std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
@@ -243,6 +290,7 @@ void flatten_plan(const Plan& p, std::vector<DevPass>* passes) {
         if (d.pf_bwd < 0) d.pf_bwd = o;
       }
     for (int t = 0; t < kTileBits; ++t) d.tile_q[t] = ps.tile_q[t];
+    set_tma_view(p.n, ps, &d);
     for (int i = 0; i < kMaxOut; ++i) d.out_q[i] = i < d.n_out ? ps.out_q[i] : -1;
     for (int g = 0; g < kPhases; ++g) {
       uint32_t w = 0;

@@ -30,6 +30,7 @@ EXPORTS = [
     "qml_loss_seed", "qml_ckpt_save", "qml_ckpt_restore", "qml_num_ckpt_slots", "qml_expect_z0",
     "qml_host_workspace_bytes", "qml_step_host", "qml_sync", "qml_debug_schedule",
     "qml_enable_timing", "qml_read_timing", "qml_launch_count", "qml_expect_z0_static",
+    "qml_debug_tile_view",
 ]
 
 
@@ -81,6 +82,7 @@ def load_library(path: str = LIB_PATH):
                              ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)], _i),
         "qml_launch_count": ([_vp], ctypes.c_longlong),
         "qml_expect_z0_static": ([_vp, _i, _i, _vp, _vp], _i),
+        "qml_debug_tile_view": ([_vp, _i, ctypes.POINTER(_i), _i], _i),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -170,6 +172,21 @@ class Context:
         buf = (ctypes.c_int * need)()
         self.lib.qml_debug_schedule(self._h, buf, need)
         return list(buf)
+
+    def debug_tile_view(self, pass_index: int) -> dict:
+        """Memory view of one pass (see qml_debug_tile_view in include/qml.h)."""
+        need = self.lib.qml_debug_tile_view(self._h, pass_index, None, 0)
+        if need < 0:
+            raise IndexError(pass_index)
+        buf = (ctypes.c_int * need)()
+        self.lib.qml_debug_tile_view(self._h, pass_index, buf, need)
+        v = list(buf)
+        dims = [dict(kind=v[1 + 4 * d], qlo=v[2 + 4 * d], bits=v[3 + 4 * d], shift=v[4 + 4 * d]) for d in range(5)]
+        i = 21
+        tile_q = [v[i + 2 * b] for b in range(12)]
+        sstride = [v[i + 2 * b + 1] for b in range(12)]
+        n_out = v[i + 24]
+        return dict(tma=v[0], dims=dims, tile_q=tile_q, sstride=sstride, out_q=v[i + 25:i + 25 + n_out])
 
     def enable_timing(self, on: bool = True):
         _check(self.lib.qml_enable_timing(self._h, 1 if on else 0), "qml_enable_timing")

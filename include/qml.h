@@ -118,7 +118,8 @@ QML_API qml_status qml_init_state_encode(qml_ctx* ctx, const float* x_dev, int B
  * E(theta); sec. 3.2, matrix-free expectation).
  *   theta_dev  [L][n][3] float32 (Rx, Ry, Rz angle per qubit per layer)
  *   x_dev      [B][n] float32 encoding angles
- *   psi_dev    [B][2^n] complex64, out: final state
+ *   psi_dev    [B][2^n] complex64, out: final state (16-byte aligned: for
+ *              n > 12 the passes load their tiles with tensor copies)
  *   expect_dev [B] float32, out */
 QML_API qml_status qml_forward_expect(qml_ctx* ctx, const float* theta_dev, const float* x_dev, int B,
                               float* psi_dev, float* expect_dev, void* stream);
@@ -135,6 +136,7 @@ QML_API qml_status qml_forward_expect(qml_ctx* ctx, const float* theta_dev, cons
  *   psi_dev     [B][2^n] complex64: in, the final state from
  *               qml_forward_expect; clobbered (used as working memory)
  *   lambda_dev  [B][2^n] complex64 working memory, clobbered
+ *   (psi_dev and lambda_dev 16-byte aligned, as for the forward pass)
  *   dLdE_dev    [B] float32, dL/dE per sample
  *   grad_dev    [L][n][3] float32, out (overwritten): sum_b dL/dE[b] dE[b]/dtheta */
 QML_API qml_status qml_backward_adjoint(qml_ctx* ctx, const float* theta_dev, const float* x_dev, int B,
@@ -228,6 +230,16 @@ QML_API long long qml_launch_count(const qml_ctx* ctx);
  * 2 = rotate (a = layer, b = bit mask of the rotated qubits, c = first slot),
  * 3 = CZ ladder (a = layer), 4 = encode (a = layout). */
 QML_API int qml_debug_schedule(const qml_ctx* ctx, int* out, int cap);
+
+/* Debugging aid: the memory view of pass `pass` (0-based, forward order),
+ * written like qml_debug_schedule (returns the number of ints, -1 on a bad
+ * argument).  Layout: [tensor-copy loads (0/1), then 5 dimensions x
+ * (kind, lowest qubit, qubits, first bit in the out-of-tile index), then 12
+ * tile bits x (qubit or -1 - unit bit, element offset in the copied tile),
+ * then n_out, then the out-of-tile qubits].  Dimension kinds: 0 unused,
+ * 1 in-tile qubits (copied whole), 2 out-of-tile qubits (fixed per tile),
+ * 3 sample, 4 out-of-tile qubits merged with the sample index above them. */
+QML_API int qml_debug_tile_view(const qml_ctx* ctx, int pass, int* out, int cap);
 
 #ifdef __cplusplus
 }
