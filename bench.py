@@ -357,12 +357,17 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w)
 
+    cfg = {**workload_config(w, B), "parallelism": f"dp{world}" if world > 1 else "single",
+           "peak_hbm_bytes": int(torch.cuda.max_memory_allocated(dev))}
+    if w.samples_per_epoch:
+        cfg["s_per_epoch"] = w.samples_per_epoch / (value / world)
+        cfg["epoch"] = f"{w.samples_per_epoch} samples per GPU at the measured samples/s (mini-batch {B})"
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {**workload_config(w, B), "parallelism": f"dp{world}" if world > 1 else "single"},
+            "config": cfg,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
             "clocks": clk,
         }
