@@ -607,6 +607,8 @@ int qml_debug_schedule(const qml_ctx* c, int* out, int cap) {
   return (int)v.size();
 }
 
+int qml_debug_layouts(int* out, int cap) { return debug_layouts(out, out ? cap : 0); }
+
 int qml_debug_tile_view(const qml_ctx* c, int pass, int* out, int cap) {
   if (!c || pass < 0 || pass >= (int)c->dpass.size()) return -1;
   const DevPass& d = c->dpass[pass];

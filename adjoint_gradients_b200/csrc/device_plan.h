@@ -8,7 +8,7 @@
 //   phase 0: tile bits 0-4      phase 1: tile bits 5-9
 //   phase 2: tile bits 10, 11, 0, 1, 2   (only for circuits of 11-12 qubits)
 // and the seven thread-index bits are the remaining tile bits in a fixed
-// order.  A 2x2 gate on a qubit that sits in a phase's register bits needs no
+// order (phase 1 has two orders, the layout variants V0 and V1).  A 2x2 gate on a qubit that sits in a phase's register bits needs no
 // communication; changing phase is a shared-memory exchange.  The planner
 // decides which qubit each tile bit is.
 #pragma once
@@ -27,7 +27,7 @@ constexpr int kThreads = 1 << kThrBits;
 // register file, 3 x ~69 KB of tile buffer fit the shared memory.
 constexpr int kBlocksPerSm = 3;
 constexpr int kTilePos = 1 << kTileBits;
-constexpr int kSmemSlots = kTilePos + (kTilePos >> 5);  // slot(t) = t + t / 32
+constexpr int kSmemSlots = kTilePos + (kTilePos >> 5) + 8;  // exchange slots (see wbit in the kernels)
 constexpr int kMaxSet = 10;           // qubits rotated per pass when n > 12
 constexpr int kMaxLayersPerPass = 2;  // cap for circuits that fit one tile
 constexpr int kMaxOut = 30;           // out-of-tile qubits

@@ -174,11 +174,15 @@ __device__ __forceinline__ void flip(float2& v, uint32_t signbit) {
 
 // ------------------------------------------------------------ tile geometry
 
-// Shared-memory slot (16 bytes) of tile position t: one pad slot every 32
-// positions.  slot(a | b) = slot(a) + slot(b) for disjoint bits, so register
-// offsets are compile-time constants, and in every layout below the eight
-// lanes of a quarter warp hit eight different bank groups.
-__host__ __device__ constexpr uint32_t wbit(int b) { return b < 5 ? (1u << b) : (1u << b) + (1u << (b - 5)); }
+// Shared-memory slot (16 bytes) of tile position t: slot(t) = sum over the set
+// bits b of t of wbit(b), i.e. t plus one pad slot every 32 positions plus a
+// small offset for tile bits 10 and 11.  The map is injective and additive
+// over disjoint bits, so register offsets are compile-time constants, and in
+// every layout below the eight lanes of a quarter warp (one 128-byte
+// wavefront of 16-byte accesses) hit eight different bank groups.
+__host__ __device__ constexpr uint32_t wbit(int b) {
+  return b < 5 ? (1u << b) : (1u << b) + (1u << (b - 5)) + (b == 10 ? 2u : b == 11 ? 4u : 0u);
+}
 
 // Tile bit addressed by register-index bit k in phase P.
 template <int P>
@@ -191,8 +195,8 @@ template <int P, int V>
 __host__ __device__ constexpr int thr_tbit(int m) {
   if (P == 0) return 5 + m;  // 5..11
   if (P == 1) {
-    if (V == 0) return m < 5 ? m : 5 + m;  // 0,1,2,3,4,10,11
-    constexpr int o[7] = {0, 1, 2, 10, 11, 3, 4};
+    if (V == 0) return m < 5 ? m : 5 + m;  // 0,1,2,3,4,10,11; V1: 10,11,0,1,2,3,4
+    constexpr int o[7] = {10, 11, 0, 1, 2, 3, 4};
     return o[m];
   }
   constexpr int o2[7] = {5, 6, 7, 3, 4, 8, 9};
@@ -972,6 +976,21 @@ cudaError_t set_pass_smem_attr(size_t smem) {
   QML_FOR_EACH_PASS_KERNEL(QML_SET_ATTR)
 #undef QML_SET_ATTR
   return e;
+}
+
+int debug_layouts(int* out, int cap) {
+  int v[2 * 3 * 12 + kTileBits + 1];
+  int k = 0;
+  for (int P = 0; P < kPhases; ++P)
+    for (int V = 0; V < 2; ++V) {
+      for (int m = 0; m < kThrBits; ++m)
+        v[k++] = P == 0 ? thr_tbit<0, 0>(m) : P == 1 ? (V ? thr_tbit<1, 1>(m) : thr_tbit<1, 0>(m)) : thr_tbit<2, 0>(m);
+      for (int r = 0; r < kRegBits; ++r) v[k++] = P == 0 ? reg_tbit<0>(r) : P == 1 ? reg_tbit<1>(r) : reg_tbit<2>(r);
+    }
+  for (int b = 0; b < kTileBits; ++b) v[k++] = (int)wbit(b);
+  v[k++] = kSmemSlots;
+  for (int i = 0; i < k && i < cap; ++i) out[i] = v[i];
+  return k;
 }
 
 cudaError_t pass_occupancy(bool backward, bool slow, size_t smem, int* blocks_per_sm) {

@@ -28,6 +28,11 @@ struct PassArgs {
 
 size_t pass_smem_bytes(int max_slots);
 
+// Register layouts for tests: per (phase, variant) the tile bit of each of the
+// 7 thread-index bits and 5 register-index bits, then the 12 slot weights and
+// the slot count.  Returns the number of ints.
+int debug_layouts(int* out, int cap);
+
 // Tensor maps (CUtensorMap, 128 bytes each) of a pass whose tiles are loaded
 // by tensor copies.  Backward: m0 over psi (plane 0), m1 over lambda (plane 1).
 // Forward: m0 over psi (planes 0 and 1 of unit u at samples 2u, 2u+1), m1 over

@@ -165,11 +165,13 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
       ps.unit_bits = kTileBits - n;
       for (int t = 0; t < kTileBits; ++t) ps.tile_q[t] = t < n ? t : -1 - (t - n);
     } else {
-      // rotated qubits on tile bits 0 .. |R|-1; the lowest other qubits are
-      // passive tile bits.  If the set starts at qubit 0, phase 1's lanes
-      // (tile bits 0-4) are qubits 0-4 (variant 0).  Otherwise the two lowest
-      // passive qubits go to tile bits 10 and 11, which are lanes of phase 1 in
-      // variant 1, so a warp touches runs of four consecutive amplitudes.
+      // The lowest other qubits are passive tile bits.  If the set starts at
+      // qubit 0 (variant 0), the set sits on tile bits 0 .. |R|-1 and phase
+      // 1's lanes (tile bits 0-4) are qubits 0-4.  Otherwise (variant 1) the
+      // two lowest passive qubits go to tile bits 10 and 11 and the others to
+      // tile bits 0, 1, ..., then the set: phase 1's lanes are tile bits 10,
+      // 11, 0, 1, 2 in lane order, so a half warp covers the lowest in-tile
+      // qubits (contiguous HBM runs, contiguous elements of a copied tile).
       const std::vector<int>& set = p.sets[pr.set];
       std::vector<bool> in(n, false);
       for (int q : set) in[q] = rotated_q[q] = true;
@@ -183,13 +185,15 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
         if (!in[q]) ps.out_q.push_back(q);
       ps.unit_bits = 0;
       ps.variant = set[0] == 0 ? 0 : 1;
-      for (int t = 0; t < (int)set.size(); ++t) ps.tile_q[t] = set[t];
       if (ps.variant == 0) {
+        for (int t = 0; t < (int)set.size(); ++t) ps.tile_q[t] = set[t];
         for (size_t i = 0; i < passive.size(); ++i) ps.tile_q[set.size() + i] = passive[i];
       } else {
         ps.tile_q[10] = passive[0];
         ps.tile_q[11] = passive[1];
-        for (size_t i = 2; i < passive.size(); ++i) ps.tile_q[set.size() + i - 2] = passive[i];
+        const int extra = (int)passive.size() - 2;
+        for (int i = 0; i < extra; ++i) ps.tile_q[i] = passive[2 + i];
+        for (int t = 0; t < (int)set.size(); ++t) ps.tile_q[extra + t] = set[t];
       }
     }
     if ((int)ps.out_q.size() > kMaxOut) return "internal: too many out-of-tile qubits";

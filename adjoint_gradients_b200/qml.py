@@ -30,8 +30,24 @@ EXPORTS = [
     "qml_loss_seed", "qml_ckpt_save", "qml_ckpt_restore", "qml_num_ckpt_slots", "qml_expect_z0",
     "qml_host_workspace_bytes", "qml_step_host", "qml_sync", "qml_debug_schedule",
     "qml_enable_timing", "qml_read_timing", "qml_launch_count", "qml_expect_z0_static",
-    "qml_debug_tile_view",
+    "qml_debug_tile_view", "qml_debug_layouts",
 ]
+
+
+def debug_layouts() -> dict:
+    """The kernels' register layouts (see qml_debug_layouts in include/qml.h)."""
+    lib = load_library()
+    need = lib.qml_debug_layouts(None, 0)
+    buf = (ctypes.c_int * need)()
+    lib.qml_debug_layouts(buf, need)
+    v = list(buf)
+    lay = {}
+    k = 0
+    for P in range(3):
+        for V in range(2):
+            lay[(P, V)] = (v[k:k + 7], v[k + 7:k + 12])
+            k += 12
+    return dict(layouts=lay, weights=v[k:k + 12], slots=v[k + 12])
 
 
 class QmlError(RuntimeError):
@@ -83,6 +99,7 @@ def load_library(path: str = LIB_PATH):
         "qml_launch_count": ([_vp], ctypes.c_longlong),
         "qml_expect_z0_static": ([_vp, _i, _i, _vp, _vp], _i),
         "qml_debug_tile_view": ([_vp, _i, ctypes.POINTER(_i), _i], _i),
+        "qml_debug_layouts": ([ctypes.POINTER(_i), _i], _i),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)

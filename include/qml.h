@@ -241,6 +241,14 @@ QML_API int qml_debug_schedule(const qml_ctx* ctx, int* out, int cap);
  * 3 sample, 4 out-of-tile qubits merged with the sample index above them. */
 QML_API int qml_debug_tile_view(const qml_ctx* ctx, int pass, int* out, int cap);
 
+/* Debugging aid: the kernels' register layouts, written like
+ * qml_debug_schedule.  Layout: for phase 0..2 and layout variant 0..1, the
+ * tile bit of each of the 7 thread-index bits then of each of the 5
+ * register-index bits; then the 12 shared-memory slot weights of the tile
+ * bits (slot of a position = sum of the weights of its set bits); then the
+ * number of slots. */
+QML_API int qml_debug_layouts(int* out, int cap);
+
 #ifdef __cplusplus
 }
 #endif
