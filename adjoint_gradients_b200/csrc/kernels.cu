@@ -139,14 +139,60 @@ __device__ __forceinline__ void rot_fwd_k(int k, float2 (&re)[kPos], float2 (&im
   }
 }
 
-__device__ __forceinline__ float3 rot_bwd_k(int k, float2 (&re)[kPos], float2 (&im)[kPos], const Coef& c) {
-  switch (k) {
-    case 0: return rot_bwd<0>(re, im, c);
-    case 1: return rot_bwd<1>(re, im, c);
-    case 2: return rot_bwd<2>(re, im, c);
-    case 3: return rot_bwd<3>(re, im, c);
-    default: return rot_bwd<4>(re, im, c);
+// rot_bwd<K> that also finishes the warp sum of the previous qubit's terms
+// (pv): the shuffle steps of warp_reduce3 are spread over the pair loop so
+// that their latency hides behind this qubit's FMAs.  *r_prev receives the
+// sum as warp_reduce3 returns it.
+template <int K>
+__device__ __forceinline__ float3 rot_bwd_red(float2 (&re)[kPos], float2 (&im)[kPos], const Coef& c, float3 pv,
+                                              int lane, float* r_prev) {
+  const bool h16 = (lane & 16) != 0, h8 = (lane & 8) != 0;
+  float k0 = h16 ? pv.z : pv.x, k1 = h16 ? 0.f : pv.y;
+  const float s0 = h16 ? pv.x : pv.z, s1 = h16 ? pv.y : 0.f;
+  float v = 0.f;
+  float2 ax = make_float2(0.f, 0.f), ay = ax, az0 = ax, az1 = ax;
+#pragma unroll
+  for (int j = 0; j < kPos; ++j) {
+    if (j & (1 << K)) continue;
+    const int pi = (j & ((1 << K) - 1)) | ((j >> (K + 1)) << K);  // pair index 0..15
+    if (pi == 0) {
+      k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+      k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+    } else if (pi == 3) {
+      v = h8 ? k1 : k0;
+      v += __shfl_xor_sync(0xffffffffu, h8 ? k0 : k1, 8);
+    } else if (pi == 6) {
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+    } else if (pi == 9) {
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+    } else if (pi == 12) {
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+    }
+    const int jj = j | (1 << K);
+    const float2 si0 = swap2(im[j]), si1 = swap2(im[jj]), sr1 = swap2(re[jj]);
+    az0 = __ffma2_rn(re[j], si0, az0);
+    az1 = __ffma2_rn(re[jj], si1, az1);
+    ax = __ffma2_rn(re[j], si1, ax);
+    ax = __ffma2_rn(re[jj], si0, ax);
+    ay = __ffma2_rn(re[j], sr1, ay);
+    ay = __ffma2_rn(im[j], si1, ay);
+    su2(re[j], im[j], re[jj], im[jj], c);
   }
+  *r_prev = v;
+  return make_float3(ax.y - ax.x, ay.x - ay.y, (az0.y - az0.x) - (az1.y - az1.x));
+}
+
+__device__ __forceinline__ float3 rot_bwd_red_k(int k, float2 (&re)[kPos], float2 (&im)[kPos], const Coef& c,
+                                                float3 pv, int lane, float* r_prev) {
+  switch (k) {
+    case 0: return rot_bwd_red<0>(re, im, c, pv, lane, r_prev);
+    case 1: return rot_bwd_red<1>(re, im, c, pv, lane, r_prev);
+    case 2: return rot_bwd_red<2>(re, im, c, pv, lane, r_prev);
+    case 3: return rot_bwd_red<3>(re, im, c, pv, lane, r_prev);
+    default: return rot_bwd_red<4>(re, im, c, pv, lane, r_prev);
+  }
+}
+
 }
 
 // Sum (a, b, c) over the warp with six shuffles; afterwards lanes 0, 8 and 16
@@ -744,15 +790,22 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
         if (op.kind == OP_EXCH) {
           exchange<V>(op.b, op.a, re, im, tile, tid);
         } else if (op.kind == OP_ROT) {
-          int slot = op.d;
+          // each rotation finishes the warp sum of the previous one
+          int slot = op.d, pslot = -1;
+          float3 pend = make_float3(0.f, 0.f, 0.f);
 #pragma unroll
           for (int k = 0; k < kRegBits; ++k)
             if ((op.b >> k) & 1) {
-              const float3 v = rot_bwd_k(k, re, im, const_coef(region, slot));
-              const float r = warp_reduce3(v.x, v.y, v.z, lane);
-              if ((lane & 7) == 0 && lane < 24) acc[warp * nacc + slot * 3 + (lane >> 3)] += r;
-              ++slot;
+              float r;
+              const float3 v = rot_bwd_red_k(k, re, im, const_coef(region, slot), pend, lane, &r);
+              if (pslot >= 0 && (lane & 7) == 0 && lane < 24) acc[warp * nacc + pslot * 3 + (lane >> 3)] += r;
+              pend = v;
+              pslot = slot++;
             }
+          if (pslot >= 0) {
+            const float r = warp_reduce3(pend.x, pend.y, pend.z, lane);
+            if ((lane & 7) == 0 && lane < 24) acc[warp * nacc + pslot * 3 + (lane >> 3)] += r;
+          }
         } else if (op.kind == OP_CZ) {
           cz_op<V>(op.a, re, im, *bc, P.cz_reg[op.a], tid, base_q);
         }
