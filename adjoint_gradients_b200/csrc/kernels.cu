@@ -193,8 +193,6 @@ __device__ __forceinline__ float3 rot_bwd_red_k(int k, float2 (&re)[kPos], float
   }
 }
 
-}
-
 // Sum (a, b, c) over the warp with six shuffles; afterwards lanes 0, 8 and 16
 // hold the totals of a, b and c.
 __device__ __forceinline__ float warp_reduce3(float a, float b, float c, int lane) {
