@@ -43,6 +43,17 @@ FMA_BWD_PER_ROT = 22  # per amplitude: U^dagger on psi (8) and lambda (8) + thre
 CPU_SAMPLE_LAYERS = 16  # oracle sample depth (cost is linear in depth)
 
 
+def kernel_sources_digest():
+    """sha256 over the sources of the pass kernels (ties recorded counters to a build)."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for rel in ("kernels.cu", "device_plan.h", "plan.cpp"):
+        with open(os.path.join(ROOT, "adjoint_gradients_b200", "csrc", rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -305,7 +316,9 @@ def run_ours(args):
     if os.path.exists(tfile):
         with open(tfile) as f:
             tr = json.load(f).get(w.name, {})
-        traffic = tr.get("bwd_pass_bytes_per_launch")
+        # counters taken on another build of the kernels do not count
+        if tr.get("kernel_sources_sha256") == kernel_sources_digest():
+            traffic = tr.get("bwd_pass_bytes_per_launch")
     roofline = {
         "kernel": "pass_kernel<backward>", "bound": "alu", "achieved": bwd_tflops, "peak": ALU_PEAK_TFLOPS,
         "unit": "TFLOP/s", "frac": bwd_tflops / ALU_PEAK_TFLOPS, "traffic": traffic,
