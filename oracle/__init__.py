@@ -9,7 +9,8 @@ Every function follows the definitions printed on the summaries of Kawase,
 "Fast and memory-efficient classical simulation of quantum machine learning via
 forward and backward gate fusion" (arXiv 2603.02804):
 
-* ``forward``  -- E(theta) = <psi_M|Z0|psi_M>  (Deep-dive blog, §1.2, the E(theta) equation)
+* ``forward``  -- E(theta) = <psi_M|O|psi_M>  (Deep-dive blog, §1.2, the E(theta) equation)
+  with O = Z0, or a sum of Pauli strings (``observable``)
 * ``adjoint``  -- dL/dtheta_j = 2 Re<lambda_j|dU_j/dtheta_j|psi_{j-1}>,
   lambda_{j-1} = U_j^dagger lambda_j  (Deep-dive blog, §1.2, adjoint-gradient equation
   and the lambda recursion; the factor 2 is the derivative of <psi|O|psi>)
@@ -49,6 +50,10 @@ def _load():
         lib.oracle_forward.restype = ctypes.c_int
         lib.oracle_adjoint.argtypes = [ctypes.c_int] * 3 + [_dp] * 6
         lib.oracle_adjoint.restype = ctypes.c_int
+        lib.oracle_forward_obs.argtypes = [ctypes.c_int] * 3 + [_dp] * 2 + [ctypes.c_int, ctypes.c_char_p] + [_dp] * 3
+        lib.oracle_forward_obs.restype = ctypes.c_int
+        lib.oracle_adjoint_obs.argtypes = [ctypes.c_int] * 3 + [_dp] * 2 + [ctypes.c_int, ctypes.c_char_p] + [_dp] * 5
+        lib.oracle_adjoint_obs.restype = ctypes.c_int
         lib.oracle_bf16_round.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t]
         lib.oracle_bf16_widen.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t]
         lib.oracle_num_threads.restype = ctypes.c_int
@@ -76,21 +81,37 @@ def num_threads() -> int:
     return int(_load().oracle_num_threads())
 
 
-def forward(x, theta, want_state: bool = False):
-    """<Z0> per sample, and optionally the final states ``[B][2^n]`` complex128."""
+def _observable(observable, n):
+    """(term count, Pauli letters, coefficients) of [(coef, "XIZ...")]: letter q of a
+    string acts on qubit q."""
+    if observable is None:
+        return 0, None, None
+    letters, coef = [], []
+    for c, word in observable:
+        if len(word) != n or any(ch not in "IXYZ" for ch in word):
+            raise ValueError(f"Pauli string {word!r} must have {n} letters from IXYZ")
+        letters.append(word)
+        coef.append(float(c))
+    return len(coef), "".join(letters).encode(), np.ascontiguousarray(coef, dtype=np.float64)
+
+
+def forward(x, theta, want_state: bool = False, observable=None):
+    """<O> per sample (O = Z0, or the Pauli sum ``observable`` = [(coef, word)]), and
+    optionally the final states ``[B][2^n]`` complex128."""
     x, theta, B, n, L = _prep(x, theta)
     E = np.zeros(B, dtype=np.float64)
     psi = np.zeros((B, 1 << n, 2), dtype=np.float64) if want_state else None
-    rc = _load().oracle_forward(n, L, B, _ptr(x), _ptr(theta), _ptr(E), _ptr(psi))
+    k, words, coef = _observable(observable, n)
+    rc = _load().oracle_forward_obs(n, L, B, _ptr(x), _ptr(theta), k, words, _ptr(coef), _ptr(E), _ptr(psi))
     if rc != 0:
-        raise RuntimeError("oracle_forward failed")
+        raise RuntimeError("oracle_forward_obs failed")
     if want_state:
         return E, psi[..., 0] + 1j * psi[..., 1]
     return E
 
 
-def adjoint(x, theta, g, want_state: bool = False):
-    """sum_b g_b dE_b/dtheta as ``[L][n][3]``, <Z0> per sample, and optionally the
+def adjoint(x, theta, g, want_state: bool = False, observable=None):
+    """sum_b g_b dE_b/dtheta as ``[L][n][3]``, <O> per sample, and optionally the
     state after walking the circuit back to its start (must be |0...0>)."""
     x, theta, B, n, L = _prep(x, theta)
     g = np.ascontiguousarray(g, dtype=np.float64)
@@ -99,9 +120,11 @@ def adjoint(x, theta, g, want_state: bool = False):
     grad = np.zeros((L, n, 3), dtype=np.float64)
     E = np.zeros(B, dtype=np.float64)
     psi0 = np.zeros((B, 1 << n, 2), dtype=np.float64) if want_state else None
-    rc = _load().oracle_adjoint(n, L, B, _ptr(x), _ptr(theta), _ptr(g), _ptr(grad), _ptr(E), _ptr(psi0))
+    k, words, coef = _observable(observable, n)
+    rc = _load().oracle_adjoint_obs(n, L, B, _ptr(x), _ptr(theta), k, words, _ptr(coef), _ptr(g), _ptr(grad),
+                                    _ptr(E), _ptr(psi0))
     if rc != 0:
-        raise RuntimeError("oracle_adjoint failed")
+        raise RuntimeError("oracle_adjoint_obs failed")
     if want_state:
         return grad, E, psi0[..., 0] + 1j * psi0[..., 1]
     return grad, E

@@ -170,6 +170,42 @@ static double expect_z0(const cplx* psi, int n) {
   return e;
 }
 
+/*
+ * Observable H = sum_k coef[k] P_k, P_k a tensor product of one-qubit Paulis:
+ * character paulis[k*n + q] in {'I','X','Y','Z'} is the factor on qubit q.
+ * This is the general observable O of E(theta) = <psi|O|psi> ([Deep-dive]
+ * sec. 1.2); the Pauli strings are applied as explicit 2x2 matrices, one qubit
+ * at a time.  out <- H psi, using tmp as scratch.  Returns -1 on a bad letter.
+ */
+static int pauli_index(char c) {
+  return c == 'X' ? PX : c == 'Y' ? PY : c == 'Z' ? PZ : c == 'I' ? -1 : -2;
+}
+
+static int apply_observable(const cplx* psi, cplx* out, cplx* tmp, int n, int nterms, const char* paulis,
+                            const double* coef) {
+  const size_t N = (size_t)1 << n;
+  for (size_t i = 0; i < N; ++i) out[i] = 0;
+  for (int k = 0; k < nterms; ++k) {
+    memcpy(tmp, psi, sizeof(cplx) * N);
+    for (int q = 0; q < n; ++q) {
+      int p = pauli_index(paulis[(size_t)k * n + q]);
+      if (p == -2) return -1;
+      if (p >= 0) apply_1q(tmp, n, q, pauli(p));
+    }
+    for (size_t i = 0; i < N; ++i) out[i] += coef[k] * tmp[i];
+  }
+  return 0;
+}
+
+/* Re <a|b> */
+static double re_inner(const cplx* a, const cplx* b, int n) {
+  const size_t N = (size_t)1 << n;
+  double e = 0.0;
+#pragma omp parallel for schedule(static) reduction(+ : e) if (n >= PAR_AMP_MIN_QUBITS)
+  for (size_t i = 0; i < N; ++i) e += creal(conj(a[i]) * b[i]);
+  return e;
+}
+
 /* ----------------------------------------------------------------- circuit */
 
 /* Number of gates: n encoding rotations + L * (3n rotations + (n-1) CZ). */
@@ -212,7 +248,7 @@ static void zero_state(cplx* psi, int n) {
 
 /* ----------------------------------------------------------------- exports */
 
-int oracle_version(void) { return 1; }
+int oracle_version(void) { return 2; }
 
 int oracle_num_threads(void) {
 #ifdef _OPENMP
@@ -225,16 +261,17 @@ int oracle_num_threads(void) {
 static int bad_args(int n, int L, int B) { return n < 1 || n > 30 || L < 0 || B < 0; }
 
 /*
- * Forward pass for B samples.
+ * Forward pass for B samples with observable H (nterms > 0; see
+ * apply_observable) or Z0 (nterms == 0).
  *   x      [B][n]     encoding angles
  *   theta  [L][n][3]  rotation angles (Rx, Ry, Rz per qubit per layer)
- *   expect [B]        out: <Z0> of the final state            (may be NULL)
+ *   expect [B]        out: <H> of the final state             (may be NULL)
  *   psi    [B][2^n][2] out: final state as (re, im) doubles    (may be NULL)
  * Returns 0, or -1 on bad arguments / allocation failure.
  */
-int oracle_forward(int n, int L, int B, const double* x, const double* theta, double* expect,
-                   double* psi_out) {
-  if (bad_args(n, L, B)) return -1;
+int oracle_forward_obs(int n, int L, int B, const double* x, const double* theta, int nterms, const char* paulis,
+                       const double* coef, double* expect, double* psi_out) {
+  if (bad_args(n, L, B) || nterms < 0 || (nterms > 0 && (!paulis || !coef))) return -1;
   const size_t N = (size_t)1 << n;
   const long ng = circuit_len(n, L);
   int err = 0;
@@ -243,39 +280,58 @@ int oracle_forward(int n, int L, int B, const double* x, const double* theta, do
   for (int b = 0; b < B; ++b) {
     gate* g = (gate*)malloc(sizeof(gate) * (size_t)ng);
     cplx* psi = (cplx*)malloc(sizeof(cplx) * N);
-    if (!g || !psi) {
+    cplx* hp = nterms ? (cplx*)malloc(sizeof(cplx) * N) : NULL;
+    cplx* tmp = nterms ? (cplx*)malloc(sizeof(cplx) * N) : NULL;
+    if (!g || !psi || (nterms && (!hp || !tmp))) {
       err |= 1;
     } else {
       build_circuit(g, n, L, x + (size_t)b * n, theta);
       zero_state(psi, n);
       for (long k = 0; k < ng; ++k) apply_gate(psi, n, &g[k], 0);
-      if (expect) expect[b] = expect_z0(psi, n);
+      if (expect) {
+        if (!nterms) {
+          expect[b] = expect_z0(psi, n);
+        } else if (apply_observable(psi, hp, tmp, n, nterms, paulis, coef)) {
+          err |= 1;
+        } else {
+          expect[b] = re_inner(psi, hp, n);
+        }
+      }
       if (psi_out) memcpy(psi_out + (size_t)b * N * 2, psi, sizeof(cplx) * N);
     }
     free(g);
     free(psi);
+    free(hp);
+    free(tmp);
   }
   return err ? -1 : 0;
 }
 
+/* Forward pass with the Z0 observable. */
+int oracle_forward(int n, int L, int B, const double* x, const double* theta, double* expect,
+                   double* psi_out) {
+  return oracle_forward_obs(n, L, B, x, theta, 0, NULL, NULL, expect, psi_out);
+}
+
 /*
- * Adjoint-method gradient for B samples.
+ * Adjoint-method gradient for B samples with observable H (nterms > 0) or Z0
+ * (nterms == 0).
  *   g      [B]        dL/dE_b, the loss seed per sample
  *   grad   [L][n][3]  out: sum_b g_b dE_b/dtheta (overwritten)
- *   expect [B]        out: <Z0> per sample (may be NULL)
+ *   expect [B]        out: <H> per sample (may be NULL)
  *   psi0   [B][2^n][2] out: the state after walking the whole circuit back
  *                     to the start, which must be |0...0> (may be NULL)
  *
- * Per sample: run the circuit forward to psi_M, set lambda = g_b Z0 psi_M,
+ * Per sample: run the circuit forward to psi_M, set lambda = g_b H psi_M,
  * then walk the gates in reverse.  For a rotation U_j:
  *     psi    <- U_j^dagger psi                     (psi is now psi_{j-1})
  *     grad_j += 2 Re <lambda| dU_j/dtheta |psi>    (lambda is still lambda_j)
  *     lambda <- U_j^dagger lambda                  (lambda_{j-1})
  * and for CZ both states are multiplied by CZ.
  */
-int oracle_adjoint(int n, int L, int B, const double* x, const double* theta, const double* gseed,
-                   double* grad, double* expect, double* psi0_out) {
-  if (bad_args(n, L, B)) return -1;
+int oracle_adjoint_obs(int n, int L, int B, const double* x, const double* theta, int nterms, const char* paulis,
+                       const double* coef, const double* gseed, double* grad, double* expect, double* psi0_out) {
+  if (bad_args(n, L, B) || nterms < 0 || (nterms > 0 && (!paulis || !coef))) return -1;
   const size_t N = (size_t)1 << n;
   const long ng = circuit_len(n, L);
   const long P = (long)L * n * 3;
@@ -288,17 +344,25 @@ int oracle_adjoint(int n, int L, int B, const double* x, const double* theta, co
     gate* g = (gate*)malloc(sizeof(gate) * (size_t)ng);
     cplx* psi = (cplx*)malloc(sizeof(cplx) * N);
     cplx* lam = (cplx*)malloc(sizeof(cplx) * N);
-    if (!g || !psi || !lam) {
+    cplx* tmp = nterms ? (cplx*)malloc(sizeof(cplx) * N) : NULL;
+    if (!g || !psi || !lam || (nterms && !tmp)) {
       err |= 1;
     } else {
       double* gb = per + (size_t)b * P;
       build_circuit(g, n, L, x + (size_t)b * n, theta);
       zero_state(psi, n);
       for (long k = 0; k < ng; ++k) apply_gate(psi, n, &g[k], 0);
-      if (expect) expect[b] = expect_z0(psi, n);
-      /* lambda_M = dL/dE * Z0 psi_M  (the derivative of <psi|Z0|psi> w.r.t. <psi|) */
-      for (size_t i = 0; i < N; ++i) lam[i] = gseed[b] * ((i & 1) ? -psi[i] : psi[i]);
-      for (long k = ng - 1; k >= 0; --k) {
+      /* lambda_M = dL/dE * H psi_M  (the derivative of <psi|H|psi> w.r.t. <psi|) */
+      if (!nterms) {
+        if (expect) expect[b] = expect_z0(psi, n);
+        for (size_t i = 0; i < N; ++i) lam[i] = gseed[b] * ((i & 1) ? -psi[i] : psi[i]);
+      } else if (apply_observable(psi, lam, tmp, n, nterms, paulis, coef)) {
+        err |= 1;
+      } else {
+        if (expect) expect[b] = re_inner(psi, lam, n);
+        for (size_t i = 0; i < N; ++i) lam[i] *= gseed[b];
+      }
+      for (long k = ng - 1; k >= 0 && !err; --k) {
         const gate* gk = &g[k];
         if (gk->kind == G_CZ) {
           apply_cz(psi, n, gk->q, gk->q2);
@@ -318,6 +382,7 @@ int oracle_adjoint(int n, int L, int B, const double* x, const double* theta, co
     free(g);
     free(psi);
     free(lam);
+    free(tmp);
   }
   if (!err) {
     /* sum over samples in a fixed order */
@@ -329,6 +394,12 @@ int oracle_adjoint(int n, int L, int B, const double* x, const double* theta, co
   }
   free(per);
   return err ? -1 : 0;
+}
+
+/* Adjoint gradient with the Z0 observable. */
+int oracle_adjoint(int n, int L, int B, const double* x, const double* theta, const double* gseed,
+                   double* grad, double* expect, double* psi0_out) {
+  return oracle_adjoint_obs(n, L, B, x, theta, 0, NULL, NULL, gseed, grad, expect, psi0_out);
 }
 
 /*

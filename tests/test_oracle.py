@@ -303,3 +303,110 @@ def test_bf16_rounding_matches_torch():
     assert (nan[0] & 0x7F80) == 0x7F80 and (nan[0] & 0x7F) != 0
     back = oracle.bf16_widen(ours)
     np.testing.assert_array_equal(oracle.bf16_round(back), ours)
+
+
+# ----------------------------------------------------------------------------- Pauli-sum observables
+#
+# E = <psi|O|psi> for a general observable O (Deep-dive blog §1.2) taken as a sum
+# of Pauli strings; lambda_M = dL/dE * O psi_M.  Letter q of a string acts on
+# qubit q.
+
+PAULI_OF = {"X": PAULI[0], "Y": PAULI[1], "Z": PAULI[2]}
+
+
+def dense_observable(obs, n):
+    H = np.zeros((1 << n, 1 << n), dtype=complex)
+    for c, word in obs:
+        M = np.eye(1 << n, dtype=complex)
+        for q, ch in enumerate(word):
+            if ch != "I":
+                M = dense_on(PAULI_OF[ch], q, n) @ M
+        H += c * M
+    return H
+
+
+def random_observable(rng, n, terms):
+    obs = []
+    for _ in range(terms):
+        word = "".join(rng.choice(list("IXYZ"), size=n))
+        obs.append((float(rng.normal()), word))
+    return obs
+
+
+def test_observable_z0_reproduces_the_default():
+    x, theta, y = random_case(11, 3, 5, 3)
+    obs = [(1.0, "ZIIII")]
+    np.testing.assert_allclose(oracle.forward(x, theta, observable=obs), oracle.forward(x, theta), atol=1e-14)
+    g = np.array([0.4, -1.1, 0.25])
+    ga, Ea = oracle.adjoint(x, theta, g, observable=obs)
+    gb, Eb = oracle.adjoint(x, theta, g)
+    np.testing.assert_allclose(ga, gb, atol=1e-14)
+    np.testing.assert_allclose(Ea, Eb, atol=1e-14)
+
+
+def test_observable_product_state_closed_forms():
+    """L = 0: qubit q is Ry(x_q)|0>, Bloch vector (sin x_q, 0, cos x_q), and the
+    qubits are uncorrelated, so a Pauli string's value is the product of the
+    per-qubit components."""
+    x = np.array([[0.3, 1.1, 2.0, 0.7]])
+    th = np.zeros((0, 4, 3))
+    bloch = {"I": np.ones(4), "X": np.sin(x[0]), "Y": np.zeros(4), "Z": np.cos(x[0])}
+    for word in ["XIII", "IYII", "IIZI", "ZZII", "XIZI", "IXXZ", "YIIX", "ZXZX", "IIII"]:
+        want = np.prod([bloch[ch][q] for q, ch in enumerate(word)])
+        got = oracle.forward(x, th, observable=[(1.0, word)])[0]
+        assert abs(got - want) < 1e-14, word
+
+
+@pytest.mark.parametrize("n,L,seed", [(1, 2, 21), (2, 2, 22), (3, 3, 23), (4, 2, 24), (5, 2, 25)])
+def test_observable_dense_brute_force(n, L, seed):
+    rng = np.random.default_rng(seed)
+    x, theta, y = random_case(seed, 2, n, L)
+    obs = random_observable(rng, n, 4)
+    H = dense_observable(obs, n)
+    assert np.allclose(H, H.conj().T)
+
+    def dense_fwd(xx, tt):
+        out = []
+        for b in range(xx.shape[0]):
+            psi = dense_state(xx[b], tt)
+            out.append(float(np.real(np.conj(psi) @ (H @ psi))))
+        return np.array(out)
+
+    E = oracle.forward(x, theta, observable=obs)
+    np.testing.assert_allclose(E, dense_fwd(x, theta), atol=1e-12)
+    g = oracle.loss_seed(E, y)
+    grad, E2 = oracle.adjoint(x, theta, g, observable=obs)
+    np.testing.assert_allclose(E2, E, atol=1e-13)
+    want = np.einsum("b,b...->...", g, shift_grad_E(dense_fwd, x, theta))
+    np.testing.assert_allclose(grad, want, atol=1e-11)
+
+
+def test_observable_is_linear():
+    rng = np.random.default_rng(31)
+    x, theta, _ = random_case(31, 3, 6, 3)
+    o1, o2 = random_observable(rng, 6, 3), random_observable(rng, 6, 2)
+    both = o1 + [(2.0 * c, w) for c, w in o2]
+    E1, E2, E12 = (oracle.forward(x, theta, observable=o) for o in (o1, o2, both))
+    np.testing.assert_allclose(E12, E1 + 2.0 * E2, atol=1e-13)
+    g = np.array([0.3, -0.8, 1.2])
+    G1, G2, G12 = (oracle.adjoint(x, theta, g, observable=o)[0] for o in (o1, o2, both))
+    np.testing.assert_allclose(G12, G1 + 2.0 * G2, atol=1e-12)
+
+
+def test_observable_parameter_shift():
+    rng = np.random.default_rng(41)
+    x, theta, y = random_case(41, 2, 7, 2)
+    obs = random_observable(rng, 7, 6) + [(0.5, "XXIIIIZ")]
+    E = oracle.forward(x, theta, observable=obs)
+    g = oracle.loss_seed(E, y)
+    grad, _ = oracle.adjoint(x, theta, g, observable=obs)
+    fwd = lambda xx, tt: oracle.forward(xx, tt, observable=obs)
+    want = np.einsum("b,b...->...", g, shift_grad_E(fwd, x, theta))
+    np.testing.assert_allclose(grad, want, atol=1e-10)
+
+
+def test_observable_rejects_bad_words():
+    x, theta, _ = random_case(1, 1, 3, 1)
+    for bad in [[(1.0, "ZZ")], [(1.0, "ZQI")]]:
+        with pytest.raises(ValueError):
+            oracle.forward(x, theta, observable=bad)
