@@ -26,7 +26,7 @@ size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 
 struct Layout {
   size_t status, passes, slot_pass, slot_index;
-  size_t coef_fwd, coef_inv, enc, dummy, exp_partial, partials, ckpt;
+  size_t coef_fwd, coef_inv, enc, dummy, exp_partial, partials, obs_groups, obs_terms, ckpt;
   size_t base_total;
   // host-step extras
   size_t h_psi, h_lam, h_x, h_theta, h_y, h_E, h_g, h_loss, h_grad;
@@ -84,6 +84,10 @@ struct qml_ctx {
     PassMaps maps;
   };
   std::vector<MapEntry> maps;
+  // observable (empty: Z0); uploaded to the workspace before its next use
+  std::vector<ObsGroup> obs_groups;
+  std::vector<ObsTerm> obs_terms;
+  bool obs_dirty = false;
 };
 
 namespace {
@@ -140,6 +144,8 @@ void compute_layout(qml_ctx* c) {
   size_t nparts = 0;
   for (const DevPass& p : c->dpass) nparts += (size_t)c->grid_bwd * p.nslots * 3;
   l.partials = take(sizeof(float) * std::max<size_t>(1, nparts));
+  l.obs_groups = take(sizeof(ObsGroup) * QML_MAX_OBS_TERMS);
+  l.obs_terms = take(sizeof(ObsTerm) * QML_MAX_OBS_TERMS);
   const size_t slot_elem = c->cfg.storage == QML_STORE_BF16 ? 4 : 8;
   l.ckpt = take(slot_elem * (size_t)c->plan.n_ckpt * Bm * (size_t)N + 16);
   l.base_total = o;
@@ -226,6 +232,33 @@ const PassMaps* pass_maps(qml_ctx* c, int p, bool backward, int B, const void* b
   return &c->maps.back().maps;
 }
 
+// Copy the observable's terms into the workspace if they changed since the
+// last upload (a copy from pageable host memory: it may wait for the stream).
+cudaError_t upload_observable(qml_ctx* c, cudaStream_t s) {
+  if (!c->obs_dirty || c->obs_terms.empty()) {
+    c->obs_dirty = false;
+    return cudaSuccess;
+  }
+  cudaError_t e = cudaMemcpyAsync(c->ws + c->lay.obs_groups, c->obs_groups.data(),
+                                  sizeof(ObsGroup) * c->obs_groups.size(), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(c->ws + c->lay.obs_terms, c->obs_terms.data(), sizeof(ObsTerm) * c->obs_terms.size(),
+                        cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) c->obs_dirty = false;
+  return e;
+}
+
+cudaError_t launch_expectation(qml_ctx* c, const float2* psi, int B, float* expect, cudaStream_t s) {
+  const int n = c->cfg.n_qubits;
+  if (c->obs_terms.empty())
+    return launch_expect(psi, B, n, at<double>(c, c->lay.exp_partial), expect, at<unsigned>(c, c->lay.status), s);
+  cudaError_t e = upload_observable(c, s);
+  if (e != cudaSuccess) return e;
+  return launch_obs_expect(psi, B, n, at<ObsGroup>(c, c->lay.obs_groups), (int)c->obs_groups.size(),
+                           at<ObsTerm>(c, c->lay.obs_terms), at<double>(c, c->lay.exp_partial), expect,
+                           at<unsigned>(c, c->lay.status), s);
+}
+
 qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, float2* psi,
                        float* expect, cudaStream_t s) {
   const int n = c->cfg.n_qubits;
@@ -270,7 +303,7 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
   if (timed) span_end(c, s, &sp);
   if (expect) {
     c->launches += 2;
-    e = launch_expect(psi, B, n, at<double>(c, c->lay.exp_partial), expect, at<unsigned>(c, c->lay.status), s);
+    e = launch_expectation(c, psi, B, expect, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
   }
   return QML_OK;
@@ -286,7 +319,14 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
   float4* ci = at<float4>(c, c->lay.coef_inv);
   cudaError_t e = launch_prep_pass_coef(at<DevPass>(c, c->lay.passes), P, theta, at<float4>(c, c->lay.coef_fwd), ci, s);
   if (e != cudaSuccess) return QML_ERR_CUDA;
-  e = launch_bwd_init(psi, lam, g, B, n, s);
+  if (c->obs_terms.empty()) {
+    e = launch_bwd_init(psi, lam, g, B, n, s);
+  } else {
+    e = upload_observable(c, s);
+    if (e == cudaSuccess)
+      e = launch_obs_bwd_init(psi, lam, g, B, n, at<ObsGroup>(c, c->lay.obs_groups), (int)c->obs_groups.size(),
+                              at<ObsTerm>(c, c->lay.obs_terms), s);
+  }
   if (e != cudaSuccess) return QML_ERR_CUDA;
   PassArgs a{};
   a.region = c->region;
@@ -520,6 +560,54 @@ qml_status qml_expect_z0(qml_ctx* c, const float* psi, int B, float* expect, voi
   return cuda_status(launch_expect(reinterpret_cast<const float2*>(psi), B, c->cfg.n_qubits,
                                    at<double>(c, c->lay.exp_partial), expect,
                                    at<unsigned>(c, c->lay.status), static_cast<cudaStream_t>(stream)));
+}
+
+qml_status qml_set_observable(qml_ctx* c, int n_terms, const char* paulis, const double* coeffs) {
+  if (!c || n_terms < 0 || n_terms > QML_MAX_OBS_TERMS) return QML_ERR_INVALID_ARG;
+  if (n_terms > 0 && (!paulis || !coeffs)) return QML_ERR_INVALID_ARG;
+  const int n = c->cfg.n_qubits;
+  struct Term {
+    uint32_t x, z;
+    int ny;
+    double c;
+  };
+  std::vector<Term> t((size_t)n_terms);
+  for (int k = 0; k < n_terms; ++k) {
+    Term& tk = t[(size_t)k];
+    tk.x = tk.z = 0;
+    tk.ny = 0;
+    tk.c = coeffs[k];
+    if (!(tk.c == tk.c) || tk.c - tk.c != 0.0) return QML_ERR_INVALID_ARG;  // NaN or infinite
+    for (int q = 0; q < n; ++q) {
+      const char ch = paulis[(size_t)k * n + q];
+      if (ch == 'X' || ch == 'Y') tk.x |= 1u << q;
+      if (ch == 'Z' || ch == 'Y') tk.z |= 1u << q;
+      if (ch == 'Y') ++tk.ny;
+      if (ch != 'I' && ch != 'X' && ch != 'Y' && ch != 'Z') return QML_ERR_INVALID_ARG;
+    }
+  }
+  std::stable_sort(t.begin(), t.end(), [](const Term& a, const Term& b) { return a.x < b.x; });
+  c->obs_terms.clear();
+  c->obs_groups.clear();
+  for (const Term& tk : t) {
+    if (c->obs_groups.empty() || c->obs_groups.back().x != tk.x)
+      c->obs_groups.push_back({tk.x, (int)c->obs_terms.size(), 0, 0});
+    c->obs_groups.back().count++;
+    c->obs_terms.push_back({tk.z, tk.ny, tk.c});
+  }
+  c->obs_dirty = true;
+  return QML_OK;
+}
+
+int qml_observable_terms(const qml_ctx* c) { return c ? (int)c->obs_terms.size() : -1; }
+
+qml_status qml_expect_observable(qml_ctx* c, const float* psi, int B, float* expect, void* stream) {
+  qml_status st = check_ready(c, B);
+  if (st != QML_OK) return st;
+  if (!psi || !expect || misaligned(psi, 8)) return QML_ERR_INVALID_ARG;
+  DeviceGuard g(c->device);
+  return cuda_status(launch_expectation(c, reinterpret_cast<const float2*>(psi), B, expect,
+                                        static_cast<cudaStream_t>(stream)));
 }
 
 qml_status qml_step_host(qml_ctx* c, const float* x_h, const float* theta_h, const float* y_h, int B,

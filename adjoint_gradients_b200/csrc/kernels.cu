@@ -967,6 +967,93 @@ __global__ void loss_seed_kernel(const float* E, const float* y, int B, float* g
 // psi into the plane layout the backward passes use: plane 0 (the psi buffer,
 // in place) holds (Re psi, Re lambda), plane 1 (the lambda buffer) holds
 // (Im psi, Im lambda).
+// ---------------------------------------------- observables: sums of Pauli strings
+//
+// O = sum_k c_k P_k with P_k = i^ny X^x Z^z (x: qubits carrying X or Y, z:
+// qubits carrying Z or Y, ny: the number of Y), so that
+//   (P psi)(j) = i^ny (-1)^popcount((j ^ x) & z) psi(j ^ x),
+//   <psi|P|psi> = sum_j conj(psi(j)) (P psi)(j).
+// Terms are grouped by x, so each group reads psi(j ^ x) once.  The general
+// observable of E(theta) = <psi|O|psi> ([Deep-dive] sec. 1.2), evaluated
+// matrix-free by bit flips ([Deep-dive] sec. 3.2, the expectation listing).
+
+// sum over the group's terms of c_k i^ny (-1)^popcount(m & z_k), m = j ^ x
+__device__ __forceinline__ double2 obs_weight(const ObsTerm* t, int count, uint32_t m) {
+  double wr = 0.0, wi = 0.0;
+  for (int k = 0; k < count; ++k) {
+    const double c = (__popc(m & t[k].z) & 1) ? -t[k].c : t[k].c;
+    switch (t[k].ny & 3) {
+      case 0: wr += c; break;
+      case 1: wi += c; break;
+      case 2: wr -= c; break;
+      default: wi -= c; break;
+    }
+  }
+  return make_double2(wr, wi);
+}
+
+__global__ void obs_expect_partial_kernel(const float2* psi, int n, const ObsGroup* groups, int ngroups,
+                                          const ObsTerm* terms, double* partial) {
+  const long long N = 1ll << n;
+  const int chunks = (int)((N + (1ll << kExpChunkLog) - 1) >> kExpChunkLog);
+  const int b = blockIdx.y, c = blockIdx.x;
+  const long long lo = (long long)c << kExpChunkLog;
+  const long long hi = min(N, lo + (1ll << kExpChunkLog));
+  const float2* p = psi + (size_t)b * N;
+  double s = 0.0;
+  for (int gi = 0; gi < ngroups; ++gi) {
+    const ObsGroup G = groups[gi];
+    for (long long j = lo + threadIdx.x; j < hi; j += kExpThreads) {
+      const uint32_t m = (uint32_t)j ^ G.x;
+      const float2 a = p[j], q = p[m];
+      // conj(a) * q
+      const double wr = (double)a.x * q.x + (double)a.y * q.y;
+      const double wi = (double)a.x * q.y - (double)a.y * q.x;
+      const double2 d = obs_weight(terms + G.first, G.count, m);
+      s += wr * d.x - wi * d.y;
+    }
+  }
+  __shared__ double red[kExpThreads];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = kExpThreads / 2; w; w >>= 1) {
+    if ((int)threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) partial[(size_t)b * chunks + c] = red[0];
+}
+
+// lambda = g_b O psi in the standard layout (psi and lambda are different buffers)
+__global__ void obs_lambda_kernel(const float2* psi, float2* lam, const float* g, int B, int n,
+                                  const ObsGroup* groups, int ngroups, const ObsTerm* terms) {
+  const long long N = 1ll << n;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)B * N) return;
+  const int b = (int)(idx >> n);
+  const uint32_t j = (uint32_t)(idx & (N - 1));
+  const float2* p = psi + (size_t)b * N;
+  double ar = 0.0, ai = 0.0;
+  for (int gi = 0; gi < ngroups; ++gi) {
+    const ObsGroup G = groups[gi];
+    const uint32_t m = j ^ G.x;
+    const float2 q = p[m];
+    const double2 d = obs_weight(terms + G.first, G.count, m);
+    ar += d.x * q.x - d.y * q.y;
+    ai += d.x * q.y + d.y * q.x;
+  }
+  const double gs = (double)__ldg(&g[b]);
+  lam[idx] = make_float2((float)(gs * ar), (float)(gs * ai));
+}
+
+// psi, lambda (standard layout) -> the backward planes, in place, position by position
+__global__ void planes_kernel(float2* psi, float2* lam, long long count) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= count) return;
+  const float2 v = psi[idx], l = lam[idx];
+  psi[idx] = make_float2(v.x, l.x);
+  lam[idx] = make_float2(v.y, l.y);
+}
+
 __global__ void bwd_init_kernel(float2* psi, float2* lam, const float* g, int B, int n) {
   const long long N = 1ll << n;
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -1182,6 +1269,29 @@ cudaError_t launch_encode(const float* x, int B, int n, float2* psi, cudaStream_
   const long long tot = (long long)B << n;
   const long long blocks = (tot + 255) / 256;
   encode_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, B, n, psi);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_obs_expect(const float2* psi, int B, int n, const ObsGroup* groups, int ngroups,
+                              const ObsTerm* terms, double* partial, float* E, unsigned* status, cudaStream_t s) {
+  const long long N = 1ll << n;
+  const int chunks = (int)((N + (1ll << kExpChunkLog) - 1) >> kExpChunkLog);
+  dim3 grid(chunks, B);
+  obs_expect_partial_kernel<<<grid, kExpThreads, 0, s>>>(psi, n, groups, ngroups, terms, partial);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  expect_final_kernel<<<(B + 127) / 128, 128, 0, s>>>(partial, chunks, B, E, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_obs_bwd_init(float2* psi, float2* lam, const float* g, int B, int n, const ObsGroup* groups,
+                                int ngroups, const ObsTerm* terms, cudaStream_t s) {
+  const long long tot = (long long)B << n;
+  const unsigned blocks = (unsigned)((tot + 255) / 256);
+  obs_lambda_kernel<<<blocks, 256, 0, s>>>(psi, lam, g, B, n, groups, ngroups, terms);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  planes_kernel<<<blocks, 256, 0, s>>>(psi, lam, tot);
   return cudaGetLastError();
 }
 

@@ -67,6 +67,24 @@ cudaError_t launch_grad_reduce(const DevPass* passes, const int* slot_pass, cons
 cudaError_t launch_loss_seed(const float* E, const float* y, int B, float* g, float* loss,
                              cudaStream_t s);
 cudaError_t launch_bwd_init(float2* psi, float2* lam, const float* g, int B, int n, cudaStream_t s);
+
+// Observables O = sum_k c_k i^ny X^x Z^z, terms grouped by x (see kernels.cu).
+struct ObsTerm {
+  uint32_t z;  // qubits carrying Z or Y
+  int ny;      // number of Y factors
+  double c;    // coefficient
+};
+struct ObsGroup {
+  uint32_t x;  // qubits carrying X or Y, shared by the group's terms
+  int first, count;
+  int pad;
+};
+// E[b] = <psi_b|O|psi_b> (partial: expect_partial_count(B, n) doubles).
+cudaError_t launch_obs_expect(const float2* psi, int B, int n, const ObsGroup* groups, int ngroups,
+                              const ObsTerm* terms, double* partial, float* E, unsigned* status, cudaStream_t s);
+// lambda = g_b O psi, then psi and lambda into the backward planes (in place).
+cudaError_t launch_obs_bwd_init(float2* psi, float2* lam, const float* g, int B, int n, const ObsGroup* groups,
+                                int ngroups, const ObsTerm* terms, cudaStream_t s);
 cudaError_t launch_encode(const float* x, int B, int n, float2* psi, cudaStream_t s);
 cudaError_t launch_ckpt_copy(bool save, const float2* psi_in, float2* psi_out, void* slot,
                              int storage, long long count, cudaStream_t s);

@@ -30,7 +30,8 @@ EXPORTS = [
     "qml_loss_seed", "qml_ckpt_save", "qml_ckpt_restore", "qml_num_ckpt_slots", "qml_expect_z0",
     "qml_host_workspace_bytes", "qml_step_host", "qml_sync", "qml_debug_schedule",
     "qml_enable_timing", "qml_read_timing", "qml_launch_count", "qml_expect_z0_static",
-    "qml_debug_tile_view", "qml_debug_layouts",
+    "qml_debug_tile_view", "qml_debug_layouts", "qml_set_observable", "qml_observable_terms",
+    "qml_expect_observable",
 ]
 
 
@@ -100,6 +101,9 @@ def load_library(path: str = LIB_PATH):
         "qml_expect_z0_static": ([_vp, _i, _i, _vp, _vp], _i),
         "qml_debug_tile_view": ([_vp, _i, ctypes.POINTER(_i), _i], _i),
         "qml_debug_layouts": ([ctypes.POINTER(_i), _i], _i),
+        "qml_set_observable": ([_vp, _i, ctypes.c_char_p, ctypes.POINTER(ctypes.c_double)], _i),
+        "qml_observable_terms": ([_vp], _i),
+        "qml_expect_observable": ([_vp, _vp, _i, _vp, _vp], _i),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -189,6 +193,29 @@ class Context:
         buf = (ctypes.c_int * need)()
         self.lib.qml_debug_schedule(self._h, buf, need)
         return list(buf)
+
+    def set_observable(self, observable=None):
+        """Observable for the following calls: None (Z0) or [(coef, word)], where
+        letter q of `word` (one of I, X, Y, Z) acts on qubit q."""
+        if not observable:
+            _check(self.lib.qml_set_observable(self._h, 0, None, None), "qml_set_observable")
+            return
+        words = "".join(w for _, w in observable).encode()
+        coef = (ctypes.c_double * len(observable))(*[float(c) for c, _ in observable])
+        _check(self.lib.qml_set_observable(self._h, len(observable), words, coef), "qml_set_observable")
+
+    @property
+    def observable_terms(self) -> int:
+        return int(self.lib.qml_observable_terms(self._h))
+
+    def expect_observable(self, psi, expect=None, stream=None):
+        import torch
+
+        B = psi.shape[0]
+        expect = torch.empty(B, dtype=torch.float32, device=psi.device) if expect is None else expect
+        _check(self.lib.qml_expect_observable(self._h, self._state_ptr(psi), B, _ptr(expect),
+                                              _stream_handle(stream)), "qml_expect_observable")
+        return expect
 
     def debug_tile_view(self, pass_index: int) -> dict:
         """Memory view of one pass (see qml_debug_tile_view in include/qml.h)."""

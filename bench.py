@@ -225,6 +225,22 @@ def workload_config(w, B):
     }
 
 
+def observable_terms(name, n):
+    """[(coef, word)] for --observable (letter q acts on qubit q), or None for Z0."""
+    if name == "z0":
+        return None
+    out = []
+    for q in range(n - 1):
+        w = ["I"] * n
+        w[q] = w[q + 1] = "Z"
+        out.append((1.0, "".join(w)))
+    for q in range(n):
+        w = ["I"] * n
+        w[q] = "X"
+        out.append((0.9, "".join(w)))
+    return out
+
+
 def run_ours(args):
     import torch
 
@@ -251,6 +267,8 @@ def run_ours(args):
     td = torch.tensor(theta, dtype=torch.float32, device=dev)
 
     ctx = qml.Context(w.n, w.L, B, ckpt_block=w.ckpt_block, storage=w.storage, device=local)
+    obs = observable_terms(args.observable, w.n)
+    ctx.set_observable(obs)
     psi = ctx.new_state(B)
     lam = ctx.new_state(B)
     E = torch.empty(B, dtype=torch.float32, device=dev)
@@ -334,6 +352,7 @@ def run_ours(args):
     e2e = None
     if not args.no_e2e:
         ctx_h = qml.Context(w.n, w.L, B, ckpt_block=w.ckpt_block, storage=w.storage, device=local, host_step=True)
+        ctx_h.set_observable(obs)
         xh = torch.tensor(x, dtype=torch.float32).pin_memory()
         th = torch.tensor(theta, dtype=torch.float32).pin_memory()
         yh = torch.tensor(y, dtype=torch.float32).pin_memory()
@@ -371,6 +390,7 @@ def run_ours(args):
         cpu = cpu_baseline(w)
 
     cfg = {**workload_config(w, B), "parallelism": f"dp{world}" if world > 1 else "single",
+           "observable": "Z0" if obs is None else f"{args.observable} ({len(obs)} Pauli strings)",
            "peak_hbm_bytes": int(torch.cuda.max_memory_allocated(dev))}
     if w.samples_per_epoch:
         cfg["s_per_epoch"] = w.samples_per_epoch / (value / world)
@@ -401,6 +421,8 @@ def main():
     ap.add_argument("--ref-layers", type=int, default=2)
     ap.add_argument("--case", default=None,
                     help="n,L,B[,ckpt_block[,storage]]: a custom shape with the workload's seeds (for profiling)")
+    ap.add_argument("--observable", default="z0", choices=["z0", "tfim"],
+                    help="z0: <Z0> (the workloads' readout); tfim: sum_q Z_q Z_q+1 + 0.9 sum_q X_q")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -165,6 +165,34 @@ QML_API int qml_num_ckpt_slots(const qml_ctx* ctx);
 QML_API qml_status qml_expect_z0(qml_ctx* ctx, const float* psi_dev, int B, float* expect_dev,
                          void* stream);
 
+/* Largest number of Pauli-string terms an observable may have. */
+#define QML_MAX_OBS_TERMS 4096
+
+/* Observable for the following forward, backward and expectation calls:
+ * O = sum_k coeffs[k] P_k, a sum of Pauli strings (the general observable O
+ * of E(theta) = <psi|O|psi> and lambda_M = dL/dE O psi_M, [Deep-dive] sec.
+ * 1.2; evaluated matrix-free by bit flips, [Deep-dive] sec. 3.2, the
+ * expectation listing).
+ *   n_terms  0 .. QML_MAX_OBS_TERMS; 0 restores the default O = Z0
+ *   paulis   host, n_terms * n_qubits characters (no terminator): character
+ *            k * n_qubits + q is the factor of term k on qubit q, one of
+ *            'I', 'X', 'Y', 'Z'
+ *   coeffs   host, n_terms finite real coefficients
+ * The context keeps a copy; the terms reach the device workspace at the next
+ * call that needs them (a copy from pageable memory on that call's stream,
+ * which may wait for the stream: make that call before capturing a graph).
+ * Returns QML_ERR_INVALID_ARG on a bad letter, a non-finite coefficient or a
+ * bad count; the previous observable then stays in force. */
+QML_API qml_status qml_set_observable(qml_ctx* ctx, int n_terms, const char* paulis, const double* coeffs);
+
+/* Number of terms of the observable in force (0 = the default Z0). */
+QML_API int qml_observable_terms(const qml_ctx* ctx);
+
+/* Standalone expectation of the observable in force: E[b] = <psi_b|O|psi_b>
+ * for B states in the standard layout (fp64 partial sums, deterministic). */
+QML_API qml_status qml_expect_observable(qml_ctx* ctx, const float* psi_dev, int B, float* expect_dev,
+                                         void* stream);
+
 /* Allocation-free Z0 expectation, for callers that may not allocate device
  * memory at all (for example a plugin inside an application whose framework
  * owns all device memory through its own pool, or a loop in which an

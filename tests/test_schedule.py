@@ -114,3 +114,20 @@ def test_calls_without_workspace_fail_cleanly():
     assert lib.qml_status_str(5) == b"checkpoint slot mismatch"
     assert lib.qml_abi_version() == 1
     assert ctx.workspace_bytes() > 0 and ctx.workspace_bytes(host_step=True) > ctx.workspace_bytes()
+
+
+def test_set_observable_validates_and_counts():
+    ctx = qml.Context(3, 2, 4, workspace=False)
+    assert ctx.observable_terms == 0
+    ctx.set_observable([(1.0, "XIZ"), (-0.5, "YYI"), (0.25, "XZZ")])
+    assert ctx.observable_terms == 3
+    lib = ctx.lib
+    c = (ctypes.c_double * 2)(1.0, 2.0)
+    assert lib.qml_set_observable(ctx._h, 2, b"XIZQII", c) == 1       # bad letter
+    assert lib.qml_set_observable(ctx._h, -1, None, None) == 1
+    assert lib.qml_set_observable(ctx._h, 4097, b"I" * 3 * 4097, (ctypes.c_double * 4097)()) == 1
+    nan = (ctypes.c_double * 1)(float("nan"))
+    assert lib.qml_set_observable(ctx._h, 1, b"ZII", nan) == 1
+    assert ctx.observable_terms == 3   # a rejected call keeps the previous observable
+    ctx.set_observable(None)
+    assert ctx.observable_terms == 0
