@@ -410,3 +410,17 @@ def test_observable_rejects_bad_words():
     for bad in [[(1.0, "ZZ")], [(1.0, "ZQI")]]:
         with pytest.raises(ValueError):
             oracle.forward(x, theta, observable=bad)
+
+
+@pytest.mark.parametrize("n,L", [(1, 3), (2, 4), (6, 5)])
+def test_zero_angles_gradient_closed_form(n, L):
+    """theta = 0: only layer l's Ry on qubit 0 has a derivative, -sin x0 dephased
+    by <Z1> = cos x1 for an odd number of preceding CZ(0, 1) (CZ^2 = I)."""
+    x, _, _ = random_case(60 + n, 3, n, 1)
+    grad, E = oracle.adjoint(x, np.zeros((L, n, 3)), np.ones(3))
+    want = np.zeros((L, n, 3))
+    for l in range(L):
+        f = np.cos(x[:, 1]) ** (l % 2) if n > 1 else 1.0
+        want[l, 0, 1] = np.sum(-np.sin(x[:, 0]) * f)
+    np.testing.assert_allclose(grad, want, atol=1e-13)
+    np.testing.assert_allclose(E, np.cos(x[:, 0]), atol=1e-14)
