@@ -209,15 +209,21 @@ static double re_inner(const cplx* a, const cplx* b, int n) {
 /* ----------------------------------------------------------------- circuit */
 
 /* Number of gates: n encoding rotations + L * (3n rotations + (n-1) CZ). */
-static long circuit_len(int n, int L) { return (long)n + (long)L * (3 * (long)n + (n - 1)); }
+/* Entangler of every layer: CZ on each bond (a, b) of a list, in list order.
+ * bonds == NULL means the open chain CZ(q, q+1), q = 0 .. n-2. */
+static int n_bonds_of(int n, int nbonds, const int* bonds) { return bonds ? nbonds : n - 1; }
+
+static long circuit_len(int n, int L, int nb) { return (long)n + (long)L * (3 * (long)n + nb); }
 
 /* The circuit as a flat, ordered gate list for one sample. */
-static void build_circuit(gate* g, int n, int L, const double* x, const double* theta) {
+static void build_circuit(gate* g, int n, int L, const double* x, const double* theta, int nbonds,
+                          const int* bonds) {
   long k = 0;
   for (int q = 0; q < n; ++q) { /* angle encoding Ry(x_q)|0> */
     gate e = {G_ROT, PY, q, -1, x[q], -1};
     g[k++] = e;
   }
+  const int nb = n_bonds_of(n, nbonds, bonds);
   for (int l = 0; l < L; ++l) {
     for (int q = 0; q < n; ++q)
       for (int a = 0; a < 3; ++a) { /* Rx, then Ry, then Rz */
@@ -225,11 +231,21 @@ static void build_circuit(gate* g, int n, int L, const double* x, const double* 
         gate r = {G_ROT, a, q, -1, theta[pi], pi};
         g[k++] = r;
       }
-    for (int q = 0; q + 1 < n; ++q) { /* CZ ladder */
-      gate c = {G_CZ, 0, q, q + 1, 0.0, -1};
+    for (int e = 0; e < nb; ++e) { /* CZ entangler */
+      gate c = {G_CZ, 0, bonds ? bonds[2 * e] : e, bonds ? bonds[2 * e + 1] : e + 1, 0.0, -1};
       g[k++] = c;
     }
   }
+}
+
+static int bad_bonds(int n, int nbonds, const int* bonds) {
+  if (!bonds) return 0;
+  if (nbonds < 0) return 1;
+  for (int e = 0; e < nbonds; ++e) {
+    int a = bonds[2 * e], b = bonds[2 * e + 1];
+    if (a < 0 || b < 0 || a >= n || b >= n || a == b) return 1;
+  }
+  return 0;
 }
 
 static void apply_gate(cplx* psi, int n, const gate* g, int inverse) {
@@ -248,7 +264,7 @@ static void zero_state(cplx* psi, int n) {
 
 /* ----------------------------------------------------------------- exports */
 
-int oracle_version(void) { return 2; }
+int oracle_version(void) { return 3; }
 
 int oracle_num_threads(void) {
 #ifdef _OPENMP
@@ -269,11 +285,11 @@ static int bad_args(int n, int L, int B) { return n < 1 || n > 30 || L < 0 || B 
  *   psi    [B][2^n][2] out: final state as (re, im) doubles    (may be NULL)
  * Returns 0, or -1 on bad arguments / allocation failure.
  */
-int oracle_forward_obs(int n, int L, int B, const double* x, const double* theta, int nterms, const char* paulis,
-                       const double* coef, double* expect, double* psi_out) {
-  if (bad_args(n, L, B) || nterms < 0 || (nterms > 0 && (!paulis || !coef))) return -1;
+int oracle_forward_gen(int n, int L, int B, const double* x, const double* theta, int nbonds, const int* bonds,
+                       int nterms, const char* paulis, const double* coef, double* expect, double* psi_out) {
+  if (bad_args(n, L, B) || nterms < 0 || (nterms > 0 && (!paulis || !coef)) || bad_bonds(n, nbonds, bonds)) return -1;
   const size_t N = (size_t)1 << n;
-  const long ng = circuit_len(n, L);
+  const long ng = circuit_len(n, L, n_bonds_of(n, nbonds, bonds));
   int err = 0;
   const int outer = n < PAR_AMP_MIN_QUBITS;
 #pragma omp parallel for schedule(dynamic, 1) if (outer) reduction(| : err)
@@ -285,7 +301,7 @@ int oracle_forward_obs(int n, int L, int B, const double* x, const double* theta
     if (!g || !psi || (nterms && (!hp || !tmp))) {
       err |= 1;
     } else {
-      build_circuit(g, n, L, x + (size_t)b * n, theta);
+      build_circuit(g, n, L, x + (size_t)b * n, theta, nbonds, bonds);
       zero_state(psi, n);
       for (long k = 0; k < ng; ++k) apply_gate(psi, n, &g[k], 0);
       if (expect) {
@@ -307,10 +323,16 @@ int oracle_forward_obs(int n, int L, int B, const double* x, const double* theta
   return err ? -1 : 0;
 }
 
-/* Forward pass with the Z0 observable. */
+/* Forward pass with the CZ chain and an observable. */
+int oracle_forward_obs(int n, int L, int B, const double* x, const double* theta, int nterms, const char* paulis,
+                       const double* coef, double* expect, double* psi_out) {
+  return oracle_forward_gen(n, L, B, x, theta, 0, NULL, nterms, paulis, coef, expect, psi_out);
+}
+
+/* Forward pass with the CZ chain and the Z0 observable. */
 int oracle_forward(int n, int L, int B, const double* x, const double* theta, double* expect,
                    double* psi_out) {
-  return oracle_forward_obs(n, L, B, x, theta, 0, NULL, NULL, expect, psi_out);
+  return oracle_forward_gen(n, L, B, x, theta, 0, NULL, 0, NULL, NULL, expect, psi_out);
 }
 
 /*
@@ -329,11 +351,12 @@ int oracle_forward(int n, int L, int B, const double* x, const double* theta, do
  *     lambda <- U_j^dagger lambda                  (lambda_{j-1})
  * and for CZ both states are multiplied by CZ.
  */
-int oracle_adjoint_obs(int n, int L, int B, const double* x, const double* theta, int nterms, const char* paulis,
-                       const double* coef, const double* gseed, double* grad, double* expect, double* psi0_out) {
-  if (bad_args(n, L, B) || nterms < 0 || (nterms > 0 && (!paulis || !coef))) return -1;
+int oracle_adjoint_gen(int n, int L, int B, const double* x, const double* theta, int nbonds, const int* bonds,
+                       int nterms, const char* paulis, const double* coef, const double* gseed, double* grad,
+                       double* expect, double* psi0_out) {
+  if (bad_args(n, L, B) || nterms < 0 || (nterms > 0 && (!paulis || !coef)) || bad_bonds(n, nbonds, bonds)) return -1;
   const size_t N = (size_t)1 << n;
-  const long ng = circuit_len(n, L);
+  const long ng = circuit_len(n, L, n_bonds_of(n, nbonds, bonds));
   const long P = (long)L * n * 3;
   int err = 0;
   double* per = (double*)calloc((size_t)(B > 0 ? B : 1) * (size_t)(P > 0 ? P : 1), sizeof(double));
@@ -349,7 +372,7 @@ int oracle_adjoint_obs(int n, int L, int B, const double* x, const double* theta
       err |= 1;
     } else {
       double* gb = per + (size_t)b * P;
-      build_circuit(g, n, L, x + (size_t)b * n, theta);
+      build_circuit(g, n, L, x + (size_t)b * n, theta, nbonds, bonds);
       zero_state(psi, n);
       for (long k = 0; k < ng; ++k) apply_gate(psi, n, &g[k], 0);
       /* lambda_M = dL/dE * H psi_M  (the derivative of <psi|H|psi> w.r.t. <psi|) */
@@ -396,10 +419,16 @@ int oracle_adjoint_obs(int n, int L, int B, const double* x, const double* theta
   return err ? -1 : 0;
 }
 
-/* Adjoint gradient with the Z0 observable. */
+/* Adjoint gradient with the CZ chain and an observable. */
+int oracle_adjoint_obs(int n, int L, int B, const double* x, const double* theta, int nterms, const char* paulis,
+                       const double* coef, const double* gseed, double* grad, double* expect, double* psi0_out) {
+  return oracle_adjoint_gen(n, L, B, x, theta, 0, NULL, nterms, paulis, coef, gseed, grad, expect, psi0_out);
+}
+
+/* Adjoint gradient with the CZ chain and the Z0 observable. */
 int oracle_adjoint(int n, int L, int B, const double* x, const double* theta, const double* gseed,
                    double* grad, double* expect, double* psi0_out) {
-  return oracle_adjoint_obs(n, L, B, x, theta, 0, NULL, NULL, gseed, grad, expect, psi0_out);
+  return oracle_adjoint_gen(n, L, B, x, theta, 0, NULL, 0, NULL, NULL, gseed, grad, expect, psi0_out);
 }
 
 /*

@@ -424,3 +424,84 @@ def test_zero_angles_gradient_closed_form(n, L):
         want[l, 0, 1] = np.sum(-np.sin(x[:, 0]) * f)
     np.testing.assert_allclose(grad, want, atol=1e-13)
     np.testing.assert_allclose(E, np.cos(x[:, 0]), atol=1e-14)
+
+
+# ----------------------------------------------------------------------------- entanglers
+#
+# Every layer ends with CZ on each bond of a list (the default is the chain
+# (q, q+1)); CZ gates are diagonal, so any bond graph keeps the fused-pass
+# structure.
+
+
+def dense_state_bonds(x, theta, bonds):
+    n = x.shape[0]
+    psi = np.zeros(1 << n, dtype=complex)
+    psi[0] = 1
+    for q in range(n):
+        psi = dense_on(dense_rot(1, x[q]), q, n) @ psi
+    for l in range(theta.shape[0]):
+        for q in range(n):
+            for a in range(3):
+                psi = dense_on(dense_rot(a, theta[l, q, a]), q, n) @ psi
+        for a, b in bonds:
+            psi = dense_cz(a, b, n) @ psi
+    return psi
+
+
+def random_bonds(rng, n, count):
+    pairs = [(a, b) for a in range(n) for b in range(a + 1, n)]
+    idx = rng.choice(len(pairs), size=min(count, len(pairs)), replace=False)
+    return [tuple(int(v) for v in (pairs[i] if rng.random() < 0.5 else pairs[i][::-1])) for i in idx]
+
+
+def test_explicit_chain_equals_the_default():
+    x, theta, _ = random_case(5, 3, 6, 3)
+    chain = [(q, q + 1) for q in range(5)]
+    np.testing.assert_allclose(oracle.forward(x, theta, bonds=chain), oracle.forward(x, theta), atol=1e-15)
+    g = np.array([0.2, 0.5, -0.9])
+    np.testing.assert_allclose(oracle.adjoint(x, theta, g, bonds=chain)[0], oracle.adjoint(x, theta, g)[0],
+                               atol=1e-15)
+
+
+@pytest.mark.parametrize("n,L,seed", [(2, 3, 71), (3, 2, 72), (4, 3, 73), (5, 2, 74)])
+def test_random_bond_graph_dense_brute_force(n, L, seed):
+    rng = np.random.default_rng(seed)
+    bonds = random_bonds(rng, n, n + 1)
+    x, theta, y = random_case(seed, 2, n, L)
+    Z0 = dense_on(PAULI[2], 0, n)
+
+    def dense_fwd(xx, tt):
+        return np.array([float(np.real(np.conj(p) @ (Z0 @ p)))
+                         for p in (dense_state_bonds(xx[b], tt, bonds) for b in range(xx.shape[0]))])
+
+    E = oracle.forward(x, theta, bonds=bonds)
+    np.testing.assert_allclose(E, dense_fwd(x, theta), atol=1e-12)
+    g = oracle.loss_seed(E, y)
+    grad, _ = oracle.adjoint(x, theta, g, bonds=bonds)
+    want = np.einsum("b,b...->...", g, shift_grad_E(dense_fwd, x, theta))
+    np.testing.assert_allclose(grad, want, atol=1e-11)
+
+
+def test_no_entangler_is_a_product_of_bloch_rotations():
+    x, theta, _ = random_case(9, 2, 4, 5)
+    E = oracle.forward(x, theta, bonds=[])
+    for b in range(2):
+        v = np.array([np.sin(x[b, 0]), 0.0, np.cos(x[b, 0])])
+        for l in range(5):
+            v = bloch_layer(v, theta[l, 0])
+        assert abs(E[b] - v[2]) < 1e-13
+
+
+@pytest.mark.parametrize("n,L", [(4, 3), (6, 4)])
+def test_ring_zero_angle_gradient_closed_form(n, L):
+    """theta = 0 with a ring (chain plus CZ(n-1, 0)): qubit 0's Bloch x component
+    is dephased by cos x1 cos x_{n-1} once per odd number of preceding layers."""
+    ring = [(q, q + 1) for q in range(n - 1)] + [(n - 1, 0)]
+    x, _, _ = random_case(80 + n, 3, n, 1)
+    grad, E = oracle.adjoint(x, np.zeros((L, n, 3)), np.ones(3), bonds=ring)
+    want = np.zeros((L, n, 3))
+    for l in range(L):
+        f = (np.cos(x[:, 1]) * np.cos(x[:, n - 1])) ** (l % 2)
+        want[l, 0, 1] = np.sum(-np.sin(x[:, 0]) * f)
+    np.testing.assert_allclose(grad, want, atol=1e-13)
+    np.testing.assert_allclose(E, np.cos(x[:, 0]), atol=1e-14)
