@@ -88,6 +88,10 @@ struct qml_ctx {
   std::vector<ObsGroup> obs_groups;
   std::vector<ObsTerm> obs_terms;
   bool obs_dirty = false;
+  // entangler of every layer (CZ bonds); chain = the default (q, q+1) ladder
+  Bonds bonds;
+  bool chain = true;
+  uint32_t nbhi[kMaxQubits] = {0};
 };
 
 namespace {
@@ -284,6 +288,8 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
   a.bmax = c->cfg.max_batch;
   a.partials = nullptr;
   a.status = at<unsigned>(c, c->lay.status);
+  a.cz_chain = c->chain ? 1 : 0;
+  for (int q = 0; q < kMaxQubits; ++q) a.cz_nbhi[q] = c->nbhi[q];
   c->launches += 2;
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, false);
@@ -344,6 +350,8 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
   a.bmax = c->cfg.max_batch;
   a.partials = at<float>(c, c->lay.partials);
   a.status = at<unsigned>(c, c->lay.status);
+  a.cz_chain = c->chain ? 1 : 0;
+  for (int q = 0; q < kMaxQubits; ++q) a.cz_nbhi[q] = c->nbhi[q];
   c->launches += 3;  // coefficient prep, lambda init, gradient reduce
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, true);
@@ -408,6 +416,9 @@ qml_status qml_create(const qml_config* cfg, int device, qml_ctx** out) {
     return QML_ERR_UNSUPPORTED;
   }
   flatten_plan(c->plan, &c->dpass);
+  c->bonds = chain_bonds(cfg->n_qubits);
+  set_pass_entangler(c->plan, c->bonds, &c->dpass);
+  for (const auto& e : c->bonds) c->nbhi[std::min(e.first, e.second)] ^= 1u << std::max(e.first, e.second);
   static std::atomic<int> next_region{0};
   c->region = next_region.fetch_add(1) % kCoefRegions;
   for (const DevPass& dp : c->dpass)
@@ -598,6 +609,27 @@ qml_status qml_set_observable(qml_ctx* c, int n_terms, const char* paulis, const
   c->obs_dirty = true;
   return QML_OK;
 }
+
+qml_status qml_set_entangler(qml_ctx* c, int n_bonds, const int* bonds) {
+  if (!c || n_bonds < 0 || n_bonds > QML_MAX_BONDS || (n_bonds > 0 && !bonds)) return QML_ERR_INVALID_ARG;
+  const int n = c->cfg.n_qubits;
+  Bonds b;
+  for (int e = 0; e < n_bonds; ++e) {
+    const int x = bonds[2 * e], y = bonds[2 * e + 1];
+    if (x < 0 || y < 0 || x >= n || y >= n || x == y) return QML_ERR_INVALID_ARG;
+    b.push_back({x, y});
+  }
+  uint32_t hi[kMaxQubits] = {0}, chain_hi[kMaxQubits] = {0};
+  for (const auto& e : b) hi[std::min(e.first, e.second)] ^= 1u << std::max(e.first, e.second);
+  for (int q = 0; q + 1 < n; ++q) chain_hi[q] = 1u << (q + 1);
+  c->bonds = b;
+  c->chain = std::memcmp(hi, chain_hi, sizeof(hi)) == 0;
+  std::memcpy(c->nbhi, hi, sizeof(hi));
+  set_pass_entangler(c->plan, c->bonds, &c->dpass);
+  return QML_OK;
+}
+
+int qml_entangler_bonds(const qml_ctx* c) { return c ? (int)c->bonds.size() : -1; }
 
 int qml_observable_terms(const qml_ctx* c) { return c ? (int)c->obs_terms.size() : -1; }
 

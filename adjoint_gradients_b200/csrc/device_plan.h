@@ -31,6 +31,7 @@ constexpr int kSmemSlots = kTilePos + (kTilePos >> 5) + 8;  // exchange slots (s
 constexpr int kMaxSet = 10;           // qubits rotated per pass when n > 12
 constexpr int kMaxLayersPerPass = 2;  // cap for circuits that fit one tile
 constexpr int kMaxOut = 30;           // out-of-tile qubits
+constexpr int kMaxQubits = 30;
 constexpr int kMaxOps = 24;
 constexpr int kMaxSlots = kMaxLayersPerPass * kTileBits;  // rotations per pass
 constexpr int kCoefRegions = 40;      // per-context regions of constant memory
@@ -75,7 +76,8 @@ struct DevPass {
   int sstride[kTileBits];   // element offset in the copied tile of each tile bit (plane 1 at +4096)
   int tile_q[kTileBits];  // tile bit -> qubit (>= 0) or -1 - (batch-unit bit)
   int out_q[kMaxOut];     // out-of-tile qubits, increasing
-  uint32_t cz_reg[kPhases];  // bit j: CZ-ladder parity of the register part of position j
+  uint32_t cz_reg[kPhases];  // bit j: entangler parity of the register part of position j
+  uint32_t cz_nb[kPhases][kRegBits];  // CZ neighbours (qubit mask) of each register bit's qubit
   long long partial_off;     // float offset of this pass's gradient partials
   int slot_lq[kMaxSlots];    // slot -> layer * n + qubit
   DevOp ops[kMaxOps];        // forward order

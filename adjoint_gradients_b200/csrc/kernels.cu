@@ -339,18 +339,30 @@ __device__ __forceinline__ void exchange(int x, int y, float2 (&re)[kPos], float
   }
 }
 
-// CZ(q, q+1) for every q: sign (-1)^{sum_q i_q i_{q+1}} of the global index i.
-// With i = a | b (a: thread and out-of-tile bits, b: register bits, disjoint),
-// the exponent is Q(a) + Q(b) + parity(b & ((a << 1) ^ (a >> 1))).
+// CZ on every bond (a, b) of the entangler: sign (-1)^{sum over bonds of i_a i_b}
+// of the global index i.  With i = A | R (A: thread and out-of-tile bits, R:
+// register bits, disjoint) the exponent is S(A) + S(R) + sum over register
+// bits k set in R of parity(A & nb(q_k)), nb(q) = q's neighbours.  S(R) is the
+// per-phase table cz_reg; for the chain S(A) = parity(A & (A >> 1)).
 __device__ __forceinline__ void apply_cz(float2 (&re)[kPos], float2 (&im)[kPos], uint32_t cz_reg,
-                                         const uint32_t (&rq)[kRegBits], uint32_t aq) {
-  const uint32_t qa = __popc(aq & (aq >> 1)) & 1u;
-  const uint32_t m = (aq << 1) ^ (aq >> 1);
+                                         const uint32_t (&nb)[kRegBits], uint32_t aq, const PassArgs& a) {
+  uint32_t qa;
+  if (a.cz_chain) {
+    qa = __popc(aq & (aq >> 1)) & 1u;
+  } else {
+    uint32_t s = 0, rem = aq;
+    while (rem) {
+      const int q = __ffs(rem) - 1;
+      rem &= rem - 1u;
+      s ^= (uint32_t)__popc(aq & a.cz_nbhi[q]);
+    }
+    qa = s & 1u;
+  }
   uint32_t w = cz_reg ^ (qa ? 0xffffffffu : 0u);
   const uint32_t pat[5] = {0xAAAAAAAAu, 0xCCCCCCCCu, 0xF0F0F0F0u, 0xFF00FF00u, 0xFFFF0000u};
 #pragma unroll
   for (int k = 0; k < kRegBits; ++k)
-    if (m & rq[k]) w ^= pat[k];
+    if (__popc(aq & nb[k]) & 1) w ^= pat[k];
 #pragma unroll
   for (int j = 0; j < kPos; ++j) {
     const uint32_t sb = (w << (31 - j)) & 0x80000000u;
@@ -638,21 +650,23 @@ __device__ __forceinline__ void tile_base(const DevPass& P, int t, uint32_t* bas
 }
 
 template <int P, int V>
-__device__ __forceinline__ void cz_t(float2 (&re)[kPos], float2 (&im)[kPos], const BlockCtx& bc, uint32_t cz_reg,
-                                     uint32_t tid, uint32_t base_q) {
+__device__ __forceinline__ void cz_t(float2 (&re)[kPos], float2 (&im)[kPos], const BlockCtx& bc, const DevPass& Pp,
+                                     uint32_t tid, uint32_t base_q, const PassArgs& a) {
   uint32_t aq, ut;
   thread_pos<P, V>(bc, tid, &aq, &ut);
-  const RegMaps m = reg_maps<P>(bc);
-  apply_cz(re, im, cz_reg, m.q, aq | base_q);
+  uint32_t nb[kRegBits];
+#pragma unroll
+  for (int k = 0; k < kRegBits; ++k) nb[k] = Pp.cz_nb[P][k];
+  apply_cz(re, im, Pp.cz_reg[P], nb, aq | base_q, a);
 }
 
 template <int V>
 __device__ __forceinline__ void cz_op(int phase, float2 (&re)[kPos], float2 (&im)[kPos], const BlockCtx& bc,
-                                      uint32_t cz_reg, uint32_t tid, uint32_t base_q) {
+                                      const DevPass& Pp, uint32_t tid, uint32_t base_q, const PassArgs& a) {
   switch (phase) {
-    case 0: cz_t<0, V>(re, im, bc, cz_reg, tid, base_q); break;
-    case 1: cz_t<1, V>(re, im, bc, cz_reg, tid, base_q); break;
-    default: cz_t<2, V>(re, im, bc, cz_reg, tid, base_q); break;
+    case 0: cz_t<0, V>(re, im, bc, Pp, tid, base_q, a); break;
+    case 1: cz_t<1, V>(re, im, bc, Pp, tid, base_q, a); break;
+    default: cz_t<2, V>(re, im, bc, Pp, tid, base_q, a); break;
   }
 }
 
@@ -770,7 +784,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
           for (int k = 0; k < kRegBits; ++k)
             if ((op.b >> k) & 1) rot_fwd_k(k, re, im, const_coef(region, slot++));
         } else if (op.kind == OP_CZ) {
-          cz_op<V>(op.a, re, im, *bc, P.cz_reg[op.a], tid, base_q);
+          cz_op<V>(op.a, re, im, *bc, P, tid, base_q, a);
         }
         if (pf_next && oi == pf_at) prefetch_next();
       }
@@ -805,7 +819,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
             if ((lane & 7) == 0 && lane < 24) acc[warp * nacc + pslot * 3 + (lane >> 3)] += r;
           }
         } else if (op.kind == OP_CZ) {
-          cz_op<V>(op.a, re, im, *bc, P.cz_reg[op.a], tid, base_q);
+          cz_op<V>(op.a, re, im, *bc, P, tid, base_q, a);
         }
         if (pf_next && oi == pf_at) prefetch_next();
       }

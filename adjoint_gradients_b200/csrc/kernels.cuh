@@ -24,6 +24,8 @@ struct PassArgs {
   int bmax;              // samples per checkpoint slot (slot stride)
   float* partials;       // backward gradient partials
   unsigned* status;
+  int cz_chain;          // the entangler is the chain (q, q+1): closed-form parity
+  uint32_t cz_nbhi[kMaxQubits];  // CZ neighbours of each qubit above it (qubit mask)
 };
 
 size_t pass_smem_bytes(int max_slots);

@@ -296,18 +296,6 @@ void flatten_plan(const Plan& p, std::vector<DevPass>* passes) {
     for (int t = 0; t < kTileBits; ++t) d.tile_q[t] = ps.tile_q[t];
     set_tma_view(p.n, ps, &d);
     for (int i = 0; i < kMaxOut; ++i) d.out_q[i] = i < d.n_out ? ps.out_q[i] : -1;
-    for (int g = 0; g < kPhases; ++g) {
-      uint32_t w = 0;
-      for (int j = 0; j < kPos; ++j) {
-        uint32_t b = 0;
-        for (int k = 0; k < kRegBits; ++k) {
-          const int q = ps.tile_q[reg_tbit(g, k)];
-          if ((j >> k) & 1 && q >= 0) b |= 1u << q;
-        }
-        if (__builtin_popcount(b & (b >> 1)) & 1) w |= 1u << j;
-      }
-      d.cz_reg[g] = w;
-    }
     d.partial_off = 0;
     for (int s = 0; s < kMaxSlots; ++s) d.slot_lq[s] = s < d.nslots ? ps.slot_lq[s] : 0;
     for (int o = 0; o < kMaxOps; ++o) {
@@ -319,6 +307,43 @@ void flatten_plan(const Plan& p, std::vector<DevPass>* passes) {
       }
     }
     passes->push_back(d);
+  }
+}
+
+Bonds chain_bonds(int n) {
+  Bonds b;
+  for (int q = 0; q + 1 < n; ++q) b.push_back({q, q + 1});
+  return b;
+}
+
+void set_pass_entangler(const Plan& p, const Bonds& bonds, std::vector<DevPass>* passes) {
+  uint32_t nb[32] = {0};
+  for (const auto& e : bonds) {
+    nb[e.first] ^= 1u << e.second;  // a bond listed twice cancels (CZ^2 = I)
+    nb[e.second] ^= 1u << e.first;
+  }
+  for (size_t pi = 0; pi < p.passes.size(); ++pi) {
+    const HostPass& ps = p.passes[pi];
+    DevPass& d = (*passes)[pi];
+    for (int g = 0; g < kPhases; ++g) {
+      // parity of sum over bonds of i_a i_b for each register part j of a position
+      uint32_t w = 0;
+      for (int j = 0; j < kPos; ++j) {
+        uint32_t b = 0;
+        for (int k = 0; k < kRegBits; ++k) {
+          const int q = ps.tile_q[reg_tbit(g, k)];
+          if ((j >> k) & 1 && q >= 0) b |= 1u << q;
+        }
+        int s = 0;
+        for (const auto& e : bonds) s ^= (int)((b >> e.first) & (b >> e.second) & 1u);
+        if (s) w |= 1u << j;
+      }
+      d.cz_reg[g] = w;
+      for (int k = 0; k < kRegBits; ++k) {
+        const int q = ps.tile_q[reg_tbit(g, k)];
+        d.cz_nb[g][k] = q >= 0 ? nb[q] : 0u;
+      }
+    }
   }
 }
 

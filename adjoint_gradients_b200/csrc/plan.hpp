@@ -18,6 +18,7 @@
 
 #include <cstdint>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "device_plan.h"
@@ -57,8 +58,16 @@ struct Plan {
 // Build the schedule.  Returns an empty string on success, else an error.
 std::string make_plan(int n, int L, int ckpt_block, Plan* out);
 
+// Entangler of every layer: CZ on each bond (a, b).  The default is the
+// chain (q, q+1), q = 0 .. n-2.
+using Bonds = std::vector<std::pair<int, int>>;
+Bonds chain_bonds(int n);
+
 // Flatten to the device representation.
 void flatten_plan(const Plan& p, std::vector<DevPass>* passes);
+
+// Entangler tables of each pass (cz_reg, cz_nb) for the bond list.
+void set_pass_entangler(const Plan& p, const Bonds& bonds, std::vector<DevPass>* passes);
 
 // Layout of qml_debug_schedule (see qml.h).
 std::vector<int> describe_plan(const Plan& p);

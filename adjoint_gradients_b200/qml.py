@@ -31,7 +31,7 @@ EXPORTS = [
     "qml_host_workspace_bytes", "qml_step_host", "qml_sync", "qml_debug_schedule",
     "qml_enable_timing", "qml_read_timing", "qml_launch_count", "qml_expect_z0_static",
     "qml_debug_tile_view", "qml_debug_layouts", "qml_set_observable", "qml_observable_terms",
-    "qml_expect_observable",
+    "qml_expect_observable", "qml_set_entangler", "qml_entangler_bonds",
 ]
 
 
@@ -104,6 +104,8 @@ def load_library(path: str = LIB_PATH):
         "qml_set_observable": ([_vp, _i, ctypes.c_char_p, ctypes.POINTER(ctypes.c_double)], _i),
         "qml_observable_terms": ([_vp], _i),
         "qml_expect_observable": ([_vp, _vp, _i, _vp, _vp], _i),
+        "qml_set_entangler": ([_vp, _i, ctypes.POINTER(_i)], _i),
+        "qml_entangler_bonds": ([_vp], _i),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -203,6 +205,18 @@ class Context:
         words = "".join(w for _, w in observable).encode()
         coef = (ctypes.c_double * len(observable))(*[float(c) for c, _ in observable])
         _check(self.lib.qml_set_observable(self._h, len(observable), words, coef), "qml_set_observable")
+
+    def set_entangler(self, bonds=None):
+        """CZ bonds [(a, b), ...] ending every layer; None restores the chain (q, q+1)."""
+        if bonds is None:
+            bonds = [(q, q + 1) for q in range(self.n - 1)]
+        flat = [int(v) for e in bonds for v in e]
+        arr = (ctypes.c_int * max(1, len(flat)))(*flat)
+        _check(self.lib.qml_set_entangler(self._h, len(bonds), arr), "qml_set_entangler")
+
+    @property
+    def entangler_bonds(self) -> int:
+        return int(self.lib.qml_entangler_bonds(self._h))
 
     @property
     def observable_terms(self) -> int:

@@ -241,6 +241,12 @@ def observable_terms(name, n):
     return out
 
 
+def entangler_bonds(name, n):
+    """CZ bonds for --entangler."""
+    chain = [(q, q + 1) for q in range(n - 1)]
+    return {"chain": chain, "ring": chain + [(n - 1, 0)], "none": []}[name]
+
+
 def run_ours(args):
     import torch
 
@@ -269,6 +275,8 @@ def run_ours(args):
     ctx = qml.Context(w.n, w.L, B, ckpt_block=w.ckpt_block, storage=w.storage, device=local)
     obs = observable_terms(args.observable, w.n)
     ctx.set_observable(obs)
+    bonds = entangler_bonds(args.entangler, w.n)
+    ctx.set_entangler(bonds)
     psi = ctx.new_state(B)
     lam = ctx.new_state(B)
     E = torch.empty(B, dtype=torch.float32, device=dev)
@@ -353,6 +361,7 @@ def run_ours(args):
     if not args.no_e2e:
         ctx_h = qml.Context(w.n, w.L, B, ckpt_block=w.ckpt_block, storage=w.storage, device=local, host_step=True)
         ctx_h.set_observable(obs)
+        ctx_h.set_entangler(bonds)
         xh = torch.tensor(x, dtype=torch.float32).pin_memory()
         th = torch.tensor(theta, dtype=torch.float32).pin_memory()
         yh = torch.tensor(y, dtype=torch.float32).pin_memory()
@@ -391,6 +400,7 @@ def run_ours(args):
 
     cfg = {**workload_config(w, B), "parallelism": f"dp{world}" if world > 1 else "single",
            "observable": "Z0" if obs is None else f"{args.observable} ({len(obs)} Pauli strings)",
+           "entangler": f"CZ {args.entangler} ({len(bonds)} bonds)",
            "peak_hbm_bytes": int(torch.cuda.max_memory_allocated(dev))}
     if w.samples_per_epoch:
         cfg["s_per_epoch"] = w.samples_per_epoch / (value / world)
@@ -423,6 +433,8 @@ def main():
                     help="n,L,B[,ckpt_block[,storage]]: a custom shape with the workload's seeds (for profiling)")
     ap.add_argument("--observable", default="z0", choices=["z0", "tfim"],
                     help="z0: <Z0> (the workloads' readout); tfim: sum_q Z_q Z_q+1 + 0.9 sum_q X_q")
+    ap.add_argument("--entangler", default="chain", choices=["chain", "ring", "none"],
+                    help="CZ bonds ending every layer: chain (q, q+1) as in the workloads, ring, or none")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -165,6 +165,23 @@ QML_API int qml_num_ckpt_slots(const qml_ctx* ctx);
 QML_API qml_status qml_expect_z0(qml_ctx* ctx, const float* psi_dev, int B, float* expect_dev,
                          void* stream);
 
+/* Largest number of CZ bonds in an entangler. */
+#define QML_MAX_BONDS 1024
+
+/* Entangler for the following forward and backward calls: every layer ends
+ * with CZ(bonds[2e], bonds[2e+1]) for e = 0 .. n_bonds-1 (host array of
+ * n_bonds pairs of distinct qubits).  The default after qml_create is the
+ * chain CZ(q, q+1), q = 0 .. n-2 ([Deep-dive] sec. 2.1 names CZ entanglers;
+ * the chain is this build's reading).  CZ gates are diagonal, so any bond
+ * graph (ring, all-to-all, brick, none: n_bonds = 0) runs through the same
+ * fused passes; a bond listed twice cancels (CZ^2 = I).  Returns
+ * QML_ERR_INVALID_ARG on a bad pair or count (the previous entangler then
+ * stays in force).  Set it before the forward pass whose backward it serves. */
+QML_API qml_status qml_set_entangler(qml_ctx* ctx, int n_bonds, const int* bonds);
+
+/* Number of bonds of the entangler in force. */
+QML_API int qml_entangler_bonds(const qml_ctx* ctx);
+
 /* Largest number of Pauli-string terms an observable may have. */
 #define QML_MAX_OBS_TERMS 4096
 

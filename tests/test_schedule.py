@@ -131,3 +131,20 @@ def test_set_observable_validates_and_counts():
     assert ctx.observable_terms == 3   # a rejected call keeps the previous observable
     ctx.set_observable(None)
     assert ctx.observable_terms == 0
+
+
+def test_set_entangler_validates_and_counts():
+    ctx = qml.Context(5, 2, 4, workspace=False)
+    assert ctx.entangler_bonds == 4  # the chain
+    ctx.set_entangler([(0, 2), (4, 1), (3, 0)])
+    assert ctx.entangler_bonds == 3
+    lib = ctx.lib
+    for bad in [[(0, 0)], [(0, 5)], [(-1, 2)]]:
+        flat = (ctypes.c_int * 2)(*bad[0])
+        assert lib.qml_set_entangler(ctx._h, 1, flat) == 1
+    assert lib.qml_set_entangler(ctx._h, -1, None) == 1
+    assert ctx.entangler_bonds == 3
+    ctx.set_entangler([])
+    assert ctx.entangler_bonds == 0
+    ctx.set_entangler(None)
+    assert ctx.entangler_bonds == 4
