@@ -90,8 +90,7 @@ struct qml_ctx {
   bool obs_dirty = false;
   // entangler of every layer (CZ bonds); chain = the default (q, q+1) ladder
   Bonds bonds;
-  bool chain = true;
-  uint32_t nbhi[kMaxQubits] = {0};
+  uint32_t nb[kMaxQubits] = {0}, nbhi[kMaxQubits] = {0};
 };
 
 namespace {
@@ -263,6 +262,16 @@ cudaError_t launch_expectation(qml_ctx* c, const float2* psi, int B, float* expe
                            at<unsigned>(c, c->lay.status), s);
 }
 
+// Neighbour masks of the entangler (a bond listed twice cancels).
+void set_bond_masks(qml_ctx* c) {
+  for (int q = 0; q < kMaxQubits; ++q) c->nb[q] = c->nbhi[q] = 0;
+  for (const auto& e : c->bonds) {
+    c->nb[e.first] ^= 1u << e.second;
+    c->nb[e.second] ^= 1u << e.first;
+    c->nbhi[std::min(e.first, e.second)] ^= 1u << std::max(e.first, e.second);
+  }
+}
+
 qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, float2* psi,
                        float* expect, cudaStream_t s) {
   const int n = c->cfg.n_qubits;
@@ -288,8 +297,7 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
   a.bmax = c->cfg.max_batch;
   a.partials = nullptr;
   a.status = at<unsigned>(c, c->lay.status);
-  a.cz_chain = c->chain ? 1 : 0;
-  for (int q = 0; q < kMaxQubits; ++q) a.cz_nbhi[q] = c->nbhi[q];
+  for (int q = 0; q < kMaxQubits; ++q) a.cz_nb[q] = c->nb[q], a.cz_nbhi[q] = c->nbhi[q];
   c->launches += 2;
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, false);
@@ -350,8 +358,7 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
   a.bmax = c->cfg.max_batch;
   a.partials = at<float>(c, c->lay.partials);
   a.status = at<unsigned>(c, c->lay.status);
-  a.cz_chain = c->chain ? 1 : 0;
-  for (int q = 0; q < kMaxQubits; ++q) a.cz_nbhi[q] = c->nbhi[q];
+  for (int q = 0; q < kMaxQubits; ++q) a.cz_nb[q] = c->nb[q], a.cz_nbhi[q] = c->nbhi[q];
   c->launches += 3;  // coefficient prep, lambda init, gradient reduce
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, true);
@@ -418,7 +425,7 @@ qml_status qml_create(const qml_config* cfg, int device, qml_ctx** out) {
   flatten_plan(c->plan, &c->dpass);
   c->bonds = chain_bonds(cfg->n_qubits);
   set_pass_entangler(c->plan, c->bonds, &c->dpass);
-  for (const auto& e : c->bonds) c->nbhi[std::min(e.first, e.second)] ^= 1u << std::max(e.first, e.second);
+  set_bond_masks(c);
   static std::atomic<int> next_region{0};
   c->region = next_region.fetch_add(1) % kCoefRegions;
   for (const DevPass& dp : c->dpass)
@@ -619,12 +626,8 @@ qml_status qml_set_entangler(qml_ctx* c, int n_bonds, const int* bonds) {
     if (x < 0 || y < 0 || x >= n || y >= n || x == y) return QML_ERR_INVALID_ARG;
     b.push_back({x, y});
   }
-  uint32_t hi[kMaxQubits] = {0}, chain_hi[kMaxQubits] = {0};
-  for (const auto& e : b) hi[std::min(e.first, e.second)] ^= 1u << std::max(e.first, e.second);
-  for (int q = 0; q + 1 < n; ++q) chain_hi[q] = 1u << (q + 1);
   c->bonds = b;
-  c->chain = std::memcmp(hi, chain_hi, sizeof(hi)) == 0;
-  std::memcpy(c->nbhi, hi, sizeof(hi));
+  set_bond_masks(c);
   set_pass_entangler(c->plan, c->bonds, &c->dpass);
   return QML_OK;
 }

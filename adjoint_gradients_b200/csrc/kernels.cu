@@ -271,6 +271,8 @@ struct BlockCtx {
   unsigned long long mbar;   // completion barrier of the tile's tensor copies
   int tma_c[2][kTmaRank];    // tensor coordinates of the next tile's copies
   int tma_sel;               // plane 1 of the next tile comes through tm1
+  uint32_t cz_w[kPhases][kThreads];  // per layout and thread: entangler terms of the thread bits
+  uint32_t cz_n[kPhases][kThreads];  // per layout and thread: xor of the thread bits' neighbours
 };
 
 // Qubit-space index and batch unit of (thread, register 0) in phase P.
@@ -339,36 +341,40 @@ __device__ __forceinline__ void exchange(int x, int y, float2 (&re)[kPos], float
   }
 }
 
-// CZ on every bond (a, b) of the entangler: sign (-1)^{sum over bonds of i_a i_b}
-// of the global index i.  With i = A | R (A: thread and out-of-tile bits, R:
-// register bits, disjoint) the exponent is S(A) + S(R) + sum over register
-// bits k set in R of parity(A & nb(q_k)), nb(q) = q's neighbours.  S(R) is the
-// per-phase table cz_reg; for the chain S(A) = parity(A & (A >> 1)).
-__device__ __forceinline__ void apply_cz(float2 (&re)[kPos], float2 (&im)[kPos], uint32_t cz_reg,
-                                         const uint32_t (&nb)[kRegBits], uint32_t aq, const PassArgs& a) {
-  uint32_t qa;
-  if (a.cz_chain) {
-    qa = __popc(aq & (aq >> 1)) & 1u;
-  } else {
-    uint32_t s = 0, rem = aq;
-    while (rem) {
-      const int q = __ffs(rem) - 1;
-      rem &= rem - 1u;
-      s ^= (uint32_t)__popc(aq & a.cz_nbhi[q]);
-    }
-    qa = s & 1u;
-  }
-  uint32_t w = cz_reg ^ (qa ? 0xffffffffu : 0u);
+// CZ on every bond (a, b) of the entangler: sign (-1)^{S(i)}, S(i) = sum over
+// bonds of i_a i_b, of the global index i.  Split i = T | O | R (thread bits,
+// out-of-tile bits, register bits; disjoint).  S is a quadratic form, so
+//   S(i) = S(T) + S(O) + S(R) + parity(O & N(T)) + sum_k R_k [parity(T & nb(q_k))
+//          + parity(O & nb(q_k))],
+// N(T) = xor of the neighbour masks of T's qubits, nb(q) = q's neighbours.
+// Per thread and layout the terms in T alone are one 32-bit word over the
+// register index (with the per-pass table S(R)), kept in shared memory; S(O)
+// is computed once per tile.
+__device__ __forceinline__ void apply_cz(float2 (&re)[kPos], float2 (&im)[kPos], uint32_t w_t, uint32_t n_t,
+                                         const uint32_t (&nb)[kRegBits], uint32_t base_q, uint32_t s_o) {
+  const uint32_t qo = (s_o ^ (uint32_t)__popc(base_q & n_t)) & 1u;
+  uint32_t w = w_t ^ (qo ? 0xffffffffu : 0u);
   const uint32_t pat[5] = {0xAAAAAAAAu, 0xCCCCCCCCu, 0xF0F0F0F0u, 0xFF00FF00u, 0xFFFF0000u};
 #pragma unroll
   for (int k = 0; k < kRegBits; ++k)
-    if (__popc(aq & nb[k]) & 1) w ^= pat[k];
+    if (__popc(base_q & nb[k]) & 1) w ^= pat[k];
 #pragma unroll
   for (int j = 0; j < kPos; ++j) {
     const uint32_t sb = (w << (31 - j)) & 0x80000000u;
     flip(re[j], sb);
     flip(im[j], sb);
   }
+}
+
+// S(A) = sum over bonds within the qubit mask A (nbhi: neighbours above).
+__device__ __forceinline__ uint32_t bond_parity(uint32_t aq, const PassArgs& a) {
+  uint32_t s = 0, rem = aq;
+  while (rem) {
+    const int q = __ffs(rem) - 1;
+    rem &= rem - 1u;
+    s ^= (uint32_t)__popc(aq & a.cz_nbhi[q]);
+  }
+  return s & 1u;
 }
 
 // ------------------------------------------------------------------ planes
@@ -651,23 +657,37 @@ __device__ __forceinline__ void tile_base(const DevPass& P, int t, uint32_t* bas
 
 template <int P, int V>
 __device__ __forceinline__ void cz_t(float2 (&re)[kPos], float2 (&im)[kPos], const BlockCtx& bc, const DevPass& Pp,
-                                     uint32_t tid, uint32_t base_q, const PassArgs& a) {
-  uint32_t aq, ut;
-  thread_pos<P, V>(bc, tid, &aq, &ut);
+                                     uint32_t tid, uint32_t base_q, uint32_t s_o) {
   uint32_t nb[kRegBits];
 #pragma unroll
   for (int k = 0; k < kRegBits; ++k) nb[k] = Pp.cz_nb[P][k];
-  apply_cz(re, im, Pp.cz_reg[P], nb, aq | base_q, a);
+  apply_cz(re, im, bc.cz_w[P][tid], bc.cz_n[P][tid], nb, base_q, s_o);
 }
 
 template <int V>
 __device__ __forceinline__ void cz_op(int phase, float2 (&re)[kPos], float2 (&im)[kPos], const BlockCtx& bc,
-                                      const DevPass& Pp, uint32_t tid, uint32_t base_q, const PassArgs& a) {
+                                      const DevPass& Pp, uint32_t tid, uint32_t base_q, uint32_t s_o) {
   switch (phase) {
-    case 0: cz_t<0, V>(re, im, bc, Pp, tid, base_q, a); break;
-    case 1: cz_t<1, V>(re, im, bc, Pp, tid, base_q, a); break;
-    default: cz_t<2, V>(re, im, bc, Pp, tid, base_q, a); break;
+    case 0: cz_t<0, V>(re, im, bc, Pp, tid, base_q, s_o); break;
+    case 1: cz_t<1, V>(re, im, bc, Pp, tid, base_q, s_o); break;
+    default: cz_t<2, V>(re, im, bc, Pp, tid, base_q, s_o); break;
   }
+}
+
+// Entangler terms of this thread's fixed bits in layout P (see apply_cz).
+template <int P, int V>
+__device__ __forceinline__ void cz_thread_terms(BlockCtx& bc, const DevPass& Pp, const PassArgs& a, uint32_t tid) {
+  uint32_t tq, ut;
+  thread_pos<P, V>(bc, tid, &tq, &ut);
+  uint32_t n_t = 0;
+  for (uint32_t rem = tq; rem; rem &= rem - 1u) n_t ^= a.cz_nb[__ffs(rem) - 1];
+  uint32_t w = Pp.cz_reg[P] ^ (bond_parity(tq, a) ? 0xffffffffu : 0u);
+  const uint32_t pat[5] = {0xAAAAAAAAu, 0xCCCCCCCCu, 0xF0F0F0F0u, 0xFF00FF00u, 0xFFFF0000u};
+#pragma unroll
+  for (int k = 0; k < kRegBits; ++k)
+    if (__popc(tq & Pp.cz_nb[P][k]) & 1) w ^= pat[k];
+  bc.cz_w[P][tid] = w;
+  bc.cz_n[P][tid] = n_t;
 }
 
 // ----------------------------------------------------------- the pass kernel
@@ -718,6 +738,9 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     }
   }
   __syncthreads();
+  cz_thread_terms<0, V>(*bc, P, a, tid);
+  cz_thread_terms<1, V>(*bc, P, a, tid);
+  cz_thread_terms<2, V>(*bc, P, a, tid);
   if (TMA && loads && tid == 0 && (int)blockIdx.x < a.n_tiles) {
     tma_coords(P, BWD, a.B, blockIdx.x, bc->tma_c, &bc->tma_sel);
     tma_load_tile(&tm0, &tm1, bc->tma_sel, bc->tma_c, tile_s, mbar);
@@ -734,6 +757,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x) {
     uint32_t base_q, unit_base;
     tile_base(P, t, &base_q, &unit_base);
+    const uint32_t s_o = bond_parity(base_q, a);  // entangler terms of the out-of-tile bits
     const int tn = t + (int)gridDim.x;
     const bool pf_next = can_pf && tn < a.n_tiles;
     auto prefetch_next = [&]() {
@@ -784,7 +808,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
           for (int k = 0; k < kRegBits; ++k)
             if ((op.b >> k) & 1) rot_fwd_k(k, re, im, const_coef(region, slot++));
         } else if (op.kind == OP_CZ) {
-          cz_op<V>(op.a, re, im, *bc, P, tid, base_q, a);
+          cz_op<V>(op.a, re, im, *bc, P, tid, base_q, s_o);
         }
         if (pf_next && oi == pf_at) prefetch_next();
       }
@@ -819,7 +843,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
             if ((lane & 7) == 0 && lane < 24) acc[warp * nacc + pslot * 3 + (lane >> 3)] += r;
           }
         } else if (op.kind == OP_CZ) {
-          cz_op<V>(op.a, re, im, *bc, P, tid, base_q, a);
+          cz_op<V>(op.a, re, im, *bc, P, tid, base_q, s_o);
         }
         if (pf_next && oi == pf_at) prefetch_next();
       }

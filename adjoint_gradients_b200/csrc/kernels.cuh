@@ -24,7 +24,7 @@ struct PassArgs {
   int bmax;              // samples per checkpoint slot (slot stride)
   float* partials;       // backward gradient partials
   unsigned* status;
-  int cz_chain;          // the entangler is the chain (q, q+1): closed-form parity
+  uint32_t cz_nb[kMaxQubits];    // CZ neighbours of each qubit (qubit mask)
   uint32_t cz_nbhi[kMaxQubits];  // CZ neighbours of each qubit above it (qubit mask)
 };
 
