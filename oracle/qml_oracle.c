@@ -213,11 +213,17 @@ static double re_inner(const cplx* a, const cplx* b, int n) {
  * bonds == NULL means the open chain CZ(q, q+1), q = 0 .. n-2. */
 static int n_bonds_of(int n, int nbonds, const int* bonds) { return bonds ? nbonds : n - 1; }
 
-static long circuit_len(int n, int L, int nb) { return (long)n + (long)L * (3 * (long)n + nb); }
+/* Gate count: the encoding, then per layer (the encoding again when data is
+ * re-uploaded) 3n rotations and the entangler's CZ gates. */
+static long circuit_len(int n, int L, int nb, int reupload) {
+  return (long)n + (long)L * ((reupload ? 4 : 3) * (long)n + nb);
+}
 
-/* The circuit as a flat, ordered gate list for one sample. */
+/* The circuit as a flat, ordered gate list for one sample.  With reupload,
+ * every layer starts with the angle encoding Ry(x_q) on every qubit again
+ * (data re-uploading); those gates carry no parameter. */
 static void build_circuit(gate* g, int n, int L, const double* x, const double* theta, int nbonds,
-                          const int* bonds) {
+                          const int* bonds, int reupload) {
   long k = 0;
   for (int q = 0; q < n; ++q) { /* angle encoding Ry(x_q)|0> */
     gate e = {G_ROT, PY, q, -1, x[q], -1};
@@ -225,6 +231,11 @@ static void build_circuit(gate* g, int n, int L, const double* x, const double* 
   }
   const int nb = n_bonds_of(n, nbonds, bonds);
   for (int l = 0; l < L; ++l) {
+    if (reupload)
+      for (int q = 0; q < n; ++q) {
+        gate e = {G_ROT, PY, q, -1, x[q], -1};
+        g[k++] = e;
+      }
     for (int q = 0; q < n; ++q)
       for (int a = 0; a < 3; ++a) { /* Rx, then Ry, then Rz */
         long pi = ((long)l * n + q) * 3 + a;
@@ -264,7 +275,7 @@ static void zero_state(cplx* psi, int n) {
 
 /* ----------------------------------------------------------------- exports */
 
-int oracle_version(void) { return 3; }
+int oracle_version(void) { return 4; }
 
 int oracle_num_threads(void) {
 #ifdef _OPENMP
@@ -285,11 +296,12 @@ static int bad_args(int n, int L, int B) { return n < 1 || n > 30 || L < 0 || B 
  *   psi    [B][2^n][2] out: final state as (re, im) doubles    (may be NULL)
  * Returns 0, or -1 on bad arguments / allocation failure.
  */
-int oracle_forward_gen(int n, int L, int B, const double* x, const double* theta, int nbonds, const int* bonds,
-                       int nterms, const char* paulis, const double* coef, double* expect, double* psi_out) {
+int oracle_forward_gen(int n, int L, int B, const double* x, const double* theta, int reupload, int nbonds,
+                       const int* bonds, int nterms, const char* paulis, const double* coef, double* expect,
+                       double* psi_out) {
   if (bad_args(n, L, B) || nterms < 0 || (nterms > 0 && (!paulis || !coef)) || bad_bonds(n, nbonds, bonds)) return -1;
   const size_t N = (size_t)1 << n;
-  const long ng = circuit_len(n, L, n_bonds_of(n, nbonds, bonds));
+  const long ng = circuit_len(n, L, n_bonds_of(n, nbonds, bonds), reupload);
   int err = 0;
   const int outer = n < PAR_AMP_MIN_QUBITS;
 #pragma omp parallel for schedule(dynamic, 1) if (outer) reduction(| : err)
@@ -301,7 +313,7 @@ int oracle_forward_gen(int n, int L, int B, const double* x, const double* theta
     if (!g || !psi || (nterms && (!hp || !tmp))) {
       err |= 1;
     } else {
-      build_circuit(g, n, L, x + (size_t)b * n, theta, nbonds, bonds);
+      build_circuit(g, n, L, x + (size_t)b * n, theta, nbonds, bonds, reupload);
       zero_state(psi, n);
       for (long k = 0; k < ng; ++k) apply_gate(psi, n, &g[k], 0);
       if (expect) {
@@ -326,13 +338,13 @@ int oracle_forward_gen(int n, int L, int B, const double* x, const double* theta
 /* Forward pass with the CZ chain and an observable. */
 int oracle_forward_obs(int n, int L, int B, const double* x, const double* theta, int nterms, const char* paulis,
                        const double* coef, double* expect, double* psi_out) {
-  return oracle_forward_gen(n, L, B, x, theta, 0, NULL, nterms, paulis, coef, expect, psi_out);
+  return oracle_forward_gen(n, L, B, x, theta, 0, 0, NULL, nterms, paulis, coef, expect, psi_out);
 }
 
 /* Forward pass with the CZ chain and the Z0 observable. */
 int oracle_forward(int n, int L, int B, const double* x, const double* theta, double* expect,
                    double* psi_out) {
-  return oracle_forward_gen(n, L, B, x, theta, 0, NULL, 0, NULL, NULL, expect, psi_out);
+  return oracle_forward_gen(n, L, B, x, theta, 0, 0, NULL, 0, NULL, NULL, expect, psi_out);
 }
 
 /*
@@ -351,12 +363,12 @@ int oracle_forward(int n, int L, int B, const double* x, const double* theta, do
  *     lambda <- U_j^dagger lambda                  (lambda_{j-1})
  * and for CZ both states are multiplied by CZ.
  */
-int oracle_adjoint_gen(int n, int L, int B, const double* x, const double* theta, int nbonds, const int* bonds,
-                       int nterms, const char* paulis, const double* coef, const double* gseed, double* grad,
-                       double* expect, double* psi0_out) {
+int oracle_adjoint_gen(int n, int L, int B, const double* x, const double* theta, int reupload, int nbonds,
+                       const int* bonds, int nterms, const char* paulis, const double* coef, const double* gseed,
+                       double* grad, double* expect, double* psi0_out) {
   if (bad_args(n, L, B) || nterms < 0 || (nterms > 0 && (!paulis || !coef)) || bad_bonds(n, nbonds, bonds)) return -1;
   const size_t N = (size_t)1 << n;
-  const long ng = circuit_len(n, L, n_bonds_of(n, nbonds, bonds));
+  const long ng = circuit_len(n, L, n_bonds_of(n, nbonds, bonds), reupload);
   const long P = (long)L * n * 3;
   int err = 0;
   double* per = (double*)calloc((size_t)(B > 0 ? B : 1) * (size_t)(P > 0 ? P : 1), sizeof(double));
@@ -372,7 +384,7 @@ int oracle_adjoint_gen(int n, int L, int B, const double* x, const double* theta
       err |= 1;
     } else {
       double* gb = per + (size_t)b * P;
-      build_circuit(g, n, L, x + (size_t)b * n, theta, nbonds, bonds);
+      build_circuit(g, n, L, x + (size_t)b * n, theta, nbonds, bonds, reupload);
       zero_state(psi, n);
       for (long k = 0; k < ng; ++k) apply_gate(psi, n, &g[k], 0);
       /* lambda_M = dL/dE * H psi_M  (the derivative of <psi|H|psi> w.r.t. <psi|) */
@@ -422,13 +434,13 @@ int oracle_adjoint_gen(int n, int L, int B, const double* x, const double* theta
 /* Adjoint gradient with the CZ chain and an observable. */
 int oracle_adjoint_obs(int n, int L, int B, const double* x, const double* theta, int nterms, const char* paulis,
                        const double* coef, const double* gseed, double* grad, double* expect, double* psi0_out) {
-  return oracle_adjoint_gen(n, L, B, x, theta, 0, NULL, nterms, paulis, coef, gseed, grad, expect, psi0_out);
+  return oracle_adjoint_gen(n, L, B, x, theta, 0, 0, NULL, nterms, paulis, coef, gseed, grad, expect, psi0_out);
 }
 
 /* Adjoint gradient with the CZ chain and the Z0 observable. */
 int oracle_adjoint(int n, int L, int B, const double* x, const double* theta, const double* gseed,
                    double* grad, double* expect, double* psi0_out) {
-  return oracle_adjoint_gen(n, L, B, x, theta, 0, NULL, 0, NULL, NULL, gseed, grad, expect, psi0_out);
+  return oracle_adjoint_gen(n, L, B, x, theta, 0, 0, NULL, 0, NULL, NULL, gseed, grad, expect, psi0_out);
 }
 
 /*

@@ -505,3 +505,57 @@ def test_ring_zero_angle_gradient_closed_form(n, L):
         want[l, 0, 1] = np.sum(-np.sin(x[:, 0]) * f)
     np.testing.assert_allclose(grad, want, atol=1e-13)
     np.testing.assert_allclose(E, np.cos(x[:, 0]), atol=1e-14)
+
+
+# ----------------------------------------------------------------------------- data re-uploading
+#
+# Every layer starts with the angle encoding Ry(x_q) on every qubit again.
+
+
+def dense_state_reupload(x, theta):
+    n = x.shape[0]
+    psi = np.zeros(1 << n, dtype=complex)
+    psi[0] = 1
+    enc = lambda p: [p := dense_on(dense_rot(1, x[q]), q, n) @ p for q in range(n)][-1]
+    psi = enc(psi)
+    for l in range(theta.shape[0]):
+        psi = enc(psi)
+        for q in range(n):
+            for a in range(3):
+                psi = dense_on(dense_rot(a, theta[l, q, a]), q, n) @ psi
+        for q in range(n - 1):
+            psi = dense_cz(q, q + 1, n) @ psi
+    return psi
+
+
+def test_reupload_one_layer_closed_form():
+    """One layer: qubit 0 sees Ry(x0) twice = Ry(2 x0), then Rx(a) Ry(b)."""
+    x, theta, _ = random_case(17, 4, 5, 1)
+    a, b = theta[0, 0, 0], theta[0, 0, 1]
+    want = np.cos(2 * x[:, 0]) * np.cos(a) * np.cos(b) - np.sin(2 * x[:, 0]) * np.sin(b)
+    np.testing.assert_allclose(oracle.forward(x, theta, reupload=True), want, atol=1e-14)
+
+
+@pytest.mark.parametrize("n,L,seed", [(1, 3, 91), (3, 2, 92), (4, 3, 93)])
+def test_reupload_dense_brute_force(n, L, seed):
+    x, theta, y = random_case(seed, 2, n, L)
+    Z0 = dense_on(PAULI[2], 0, n)
+
+    def dense_fwd(xx, tt):
+        return np.array([float(np.real(np.conj(p) @ (Z0 @ p)))
+                         for p in (dense_state_reupload(xx[b], tt) for b in range(xx.shape[0]))])
+
+    E = oracle.forward(x, theta, reupload=True)
+    np.testing.assert_allclose(E, dense_fwd(x, theta), atol=1e-12)
+    g = oracle.loss_seed(E, y)
+    grad, _ = oracle.adjoint(x, theta, g, reupload=True)
+    want = np.einsum("b,b...->...", g, shift_grad_E(dense_fwd, x, theta))
+    np.testing.assert_allclose(grad, want, atol=1e-11)
+
+
+def test_reupload_returns_to_the_zero_state():
+    x, theta, _ = random_case(19, 2, 7, 4)
+    _, _, psi0 = oracle.adjoint(x, theta, np.ones(2), want_state=True, reupload=True)
+    ref = np.zeros_like(psi0)
+    ref[:, 0] = 1.0
+    np.testing.assert_allclose(psi0, ref, atol=1e-12)
