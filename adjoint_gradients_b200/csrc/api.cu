@@ -91,6 +91,7 @@ struct qml_ctx {
   // entangler of every layer (CZ bonds); chain = the default (q, q+1) ladder
   Bonds bonds;
   uint32_t nb[kMaxQubits] = {0}, nbhi[kMaxQubits] = {0};
+  bool reupload = false;  // every layer starts with the encoding again
 };
 
 namespace {
@@ -298,6 +299,7 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
   a.partials = nullptr;
   a.status = at<unsigned>(c, c->lay.status);
   for (int q = 0; q < kMaxQubits; ++q) a.cz_nb[q] = c->nb[q], a.cz_nbhi[q] = c->nbhi[q];
+  a.reupload = c->reupload ? 1 : 0;
   c->launches += 2;
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, false);
@@ -325,7 +327,6 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
 
 qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, float2* psi,
                         float2* lam, const float* g, float* grad, cudaStream_t s) {
-  (void)x;
   const int n = c->cfg.n_qubits, L = c->cfg.n_layers;
   const int P = (int)c->dpass.size();
   for (int m = 0; m < c->plan.n_ckpt; ++m)
@@ -342,6 +343,10 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
                               at<ObsTerm>(c, c->lay.obs_terms), s);
   }
   if (e != cudaSuccess) return QML_ERR_CUDA;
+  if (c->reupload) {  // per-sample encoding angles for un-applying the re-uploaded encodings
+    e = launch_prep_enc(x, B, n, at<float2>(c, c->lay.enc), s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+  }
   PassArgs a{};
   a.region = c->region;
   a.n = n;
@@ -351,7 +356,7 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
   a.buf0 = psi;
   a.buf1 = lam;
   a.dummy = nullptr;
-  a.enc = nullptr;
+  a.enc = at<float2>(c, c->lay.enc);
   a.g = g;
   a.ckpt = c->ws + c->lay.ckpt;
   a.storage = c->cfg.storage == QML_STORE_BF16 ? 1 : 0;
@@ -359,6 +364,7 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
   a.partials = at<float>(c, c->lay.partials);
   a.status = at<unsigned>(c, c->lay.status);
   for (int q = 0; q < kMaxQubits; ++q) a.cz_nb[q] = c->nb[q], a.cz_nbhi[q] = c->nbhi[q];
+  a.reupload = c->reupload ? 1 : 0;
   c->launches += 3;  // coefficient prep, lambda init, gradient reduce
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, true);
@@ -519,6 +525,7 @@ qml_status qml_backward_adjoint(qml_ctx* c, const float* theta, const float* x, 
   if (!theta || !psi || !lambda || !dLdE || !grad || misaligned(psi, 16) || misaligned(lambda, 16))
     return QML_ERR_INVALID_ARG;
   if (psi == lambda) return QML_ERR_INVALID_ARG;
+  if (c->reupload && !x) return QML_ERR_INVALID_ARG;  // the re-uploaded encodings need x
   DeviceGuard g(c->device);
   return run_backward(c, theta, x, B, reinterpret_cast<float2*>(psi), reinterpret_cast<float2*>(lambda),
                       dLdE, grad, static_cast<cudaStream_t>(stream));
@@ -631,6 +638,15 @@ qml_status qml_set_entangler(qml_ctx* c, int n_bonds, const int* bonds) {
   set_pass_entangler(c->plan, c->bonds, &c->dpass);
   return QML_OK;
 }
+
+qml_status qml_set_reupload(qml_ctx* c, int on) {
+  if (!c) return QML_ERR_INVALID_ARG;
+  if (on && c->slow) return QML_ERR_UNSUPPORTED;  // n < 5: register layouts with batch-unit bits
+  c->reupload = on != 0;
+  return QML_OK;
+}
+
+int qml_reupload(const qml_ctx* c) { return c ? (c->reupload ? 1 : 0) : -1; }
 
 int qml_entangler_bonds(const qml_ctx* c) { return c ? (int)c->bonds.size() : -1; }
 

@@ -193,6 +193,70 @@ __device__ __forceinline__ float3 rot_bwd_red_k(int k, float2 (&re)[kPos], float
   }
 }
 
+// Data re-uploading: Ry(x_q) (forward) or Ry(-x_q) (backward) on qubit K's
+// register pairs, with per-sample angles.  Forward lanes are two samples, so
+// the (cos, sin)(x/2) pairs are per lane; backward lanes are psi and lambda of
+// one sample, so both lanes take that sample's values.
+template <bool BWD>
+__device__ __forceinline__ void enc_coef(const PassArgs& a, uint32_t unit, int q, float2* c, float2* s) {
+  if (!BWD) {
+    const float2* e = a.enc + ((size_t)unit * a.n + q) * 2;
+    *c = __ldg(&e[0]);
+    *s = __ldg(&e[1]);
+  } else {
+    const float2* e = a.enc + ((size_t)(unit >> 1) * a.n + q) * 2;
+    const float2 c2 = __ldg(&e[0]), s2 = __ldg(&e[1]);
+    const float cv = (unit & 1u) ? c2.y : c2.x, sv = (unit & 1u) ? s2.y : s2.x;
+    *c = make_float2(cv, cv);
+    *s = make_float2(sv, sv);
+  }
+}
+
+template <bool BWD>
+__device__ __forceinline__ void enc_pair(float2& r0, float2& i0, float2& r1, float2& i1, float2 c, float2 s) {
+  const float2 ns = make_float2(-s.x, -s.y);
+  const float2 a0 = BWD ? s : ns, a1 = BWD ? ns : s;
+  const float2 nr0 = __ffma2_rn(a0, r1, __fmul2_rn(c, r0));
+  const float2 ni0 = __ffma2_rn(a0, i1, __fmul2_rn(c, i0));
+  const float2 nr1 = __ffma2_rn(a1, r0, __fmul2_rn(c, r1));
+  const float2 ni1 = __ffma2_rn(a1, i0, __fmul2_rn(c, i1));
+  r0 = nr0, i0 = ni0, r1 = nr1, i1 = ni1;
+}
+
+// unit: the thread's batch unit; mu[k]: unit increment of register bit k (0
+// unless a register bit is a batch-unit bit, which happens only for n < 10)
+template <bool BWD, int K>
+__device__ __forceinline__ void enc_rot(float2 (&re)[kPos], float2 (&im)[kPos], const PassArgs& a, int q,
+                                        uint32_t unit, const uint32_t (&mu)[kRegBits]) {
+  const bool uni = (mu[0] | mu[1] | mu[2] | mu[3] | mu[4]) == 0u;
+  float2 c, s;
+  if (uni) enc_coef<BWD>(a, unit, q, &c, &s);
+#pragma unroll
+  for (int j = 0; j < kPos; ++j) {
+    if (j & (1 << K)) continue;
+    if (!uni) {
+      uint32_t du = 0;
+#pragma unroll
+      for (int k = 0; k < kRegBits; ++k)
+        if ((j >> k) & 1) du += mu[k];
+      enc_coef<BWD>(a, unit + du, q, &c, &s);
+    }
+    enc_pair<BWD>(re[j], im[j], re[j | (1 << K)], im[j | (1 << K)], c, s);
+  }
+}
+
+template <bool BWD>
+__device__ __forceinline__ void enc_rot_k(int k, float2 (&re)[kPos], float2 (&im)[kPos], const PassArgs& a, int q,
+                                          uint32_t unit, const uint32_t (&mu)[kRegBits]) {
+  switch (k) {
+    case 0: enc_rot<BWD, 0>(re, im, a, q, unit, mu); break;
+    case 1: enc_rot<BWD, 1>(re, im, a, q, unit, mu); break;
+    case 2: enc_rot<BWD, 2>(re, im, a, q, unit, mu); break;
+    case 3: enc_rot<BWD, 3>(re, im, a, q, unit, mu); break;
+    default: enc_rot<BWD, 4>(re, im, a, q, unit, mu); break;
+  }
+}
+
 // Sum (a, b, c) over the warp with six shuffles; afterwards lanes 0, 8 and 16
 // hold the totals of a, b and c.
 __device__ __forceinline__ float warp_reduce3(float a, float b, float c, int lane) {
@@ -674,6 +738,32 @@ __device__ __forceinline__ void cz_op(int phase, float2 (&re)[kPos], float2 (&im
   }
 }
 
+// The thread's batch unit, the register bits' unit increments and qubits in
+// layout P (for data re-uploading).
+template <int P, int V>
+__device__ __forceinline__ void unit_maps_t(const BlockCtx& bc, uint32_t tid, uint32_t unit_base, uint32_t* unit,
+                                            uint32_t (&mu)[kRegBits], int (&rq)[kRegBits]) {
+  uint32_t aq, ut;
+  thread_pos<P, V>(bc, tid, &aq, &ut);
+  *unit = unit_base + ut;
+#pragma unroll
+  for (int k = 0; k < kRegBits; ++k) {
+    mu[k] = bc.ubit[reg_tbit<P>(k)];
+    const uint32_t qb = bc.qbit[reg_tbit<P>(k)];
+    rq[k] = qb ? __ffs(qb) - 1 : -1;
+  }
+}
+
+template <int V>
+__device__ __forceinline__ void unit_maps(int phase, const BlockCtx& bc, uint32_t tid, uint32_t unit_base,
+                                          uint32_t* unit, uint32_t (&mu)[kRegBits], int (&rq)[kRegBits]) {
+  switch (phase) {
+    case 0: unit_maps_t<0, V>(bc, tid, unit_base, unit, mu, rq); break;
+    case 1: unit_maps_t<1, V>(bc, tid, unit_base, unit, mu, rq); break;
+    default: unit_maps_t<2, V>(bc, tid, unit_base, unit, mu, rq); break;
+  }
+}
+
 // Entangler terms of this thread's fixed bits in layout P (see apply_cz).
 template <int P, int V>
 __device__ __forceinline__ void cz_thread_terms(BlockCtx& bc, const DevPass& Pp, const PassArgs& a, uint32_t tid) {
@@ -699,8 +789,9 @@ __device__ __forceinline__ void cz_thread_terms(BlockCtx& bc, const DevPass& Pp,
 // MODE 0: a memory layout has a batch-unit register bit (n < 5), generic
 // addressing.  MODE 1: tiles are loaded by the threads (the next tile with
 // cp.async).  MODE 2: tiles are loaded by tensor copies through tm0 / tm1.
+// RE: data re-uploading (every layer starts with the encoding again).
 
-template <bool BWD, int MODE, int V>
+template <bool BWD, int MODE, int V, bool RE>
 __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     pass_kernel(const PassArgs a, const __grid_constant__ DevPass P, const __grid_constant__ CUtensorMap tm0,
                 const __grid_constant__ CUtensorMap tm1) {
@@ -804,6 +895,14 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
           exchange<V>(op.a, op.b, re, im, tile, tid);
         } else if (op.kind == OP_ROT) {
           int slot = op.d;
+          if (RE) {  // the encoding again before the layer's rotations
+            uint32_t unit, mu[kRegBits];
+            int rq[kRegBits];
+            unit_maps<V>(op.a, *bc, tid, unit_base, &unit, mu, rq);
+#pragma unroll
+            for (int k = 0; k < kRegBits; ++k)
+              if ((op.b >> k) & 1) enc_rot_k<false>(k, re, im, a, rq[k], unit, mu);
+          }
 #pragma unroll
           for (int k = 0; k < kRegBits; ++k)
             if ((op.b >> k) & 1) rot_fwd_k(k, re, im, const_coef(region, slot++));
@@ -841,6 +940,14 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
           if (pslot >= 0) {
             const float r = warp_reduce3(pend.x, pend.y, pend.z, lane);
             if ((lane & 7) == 0 && lane < 24) acc[warp * nacc + pslot * 3 + (lane >> 3)] += r;
+          }
+          if (RE) {  // un-apply the layer's encoding
+            uint32_t unit, mu[kRegBits];
+            int rq[kRegBits];
+            unit_maps<V>(op.a, *bc, tid, unit_base, &unit, mu, rq);
+#pragma unroll
+            for (int k = 0; k < kRegBits; ++k)
+              if ((op.b >> k) & 1) enc_rot_k<true>(k, re, im, a, rq[k], unit, mu);
           }
         } else if (op.kind == OP_CZ) {
           cz_op<V>(op.a, re, im, *bc, P, tid, base_q, s_o);
@@ -1138,17 +1245,19 @@ size_t pass_smem_bytes(int max_slots) {
   return (size_t)kSmemSlots * sizeof(float4) + sizeof(BlockCtx) + (size_t)(kThreads / 32) * max_slots * 3 * sizeof(float);
 }
 
-#define QML_FOR_EACH_PASS_KERNEL(X) \
-  X(false, 0, 0) X(true, 0, 0) X(false, 1, 0) X(true, 1, 0) X(false, 1, 1) X(true, 1, 1) X(false, 2, 0) X(true, 2, 0) \
-  X(false, 2, 1) X(true, 2, 1)
+#define QML_FOR_EACH_PASS_KERNEL(X)                                                                          \
+  X(false, 0, 0, false) X(true, 0, 0, false) X(false, 1, 0, false) X(true, 1, 0, false) X(false, 1, 1, false)     \
+  X(true, 1, 1, false) X(false, 2, 0, false) X(true, 2, 0, false) X(false, 2, 1, false) X(true, 2, 1, false)      \
+  X(false, 1, 0, true) X(true, 1, 0, true) X(false, 1, 1, true) X(true, 1, 1, true) X(false, 2, 0, true)          \
+  X(true, 2, 0, true) X(false, 2, 1, true) X(true, 2, 1, true)
 
 cudaError_t set_pass_smem_attr(size_t smem) {
   cudaError_t e = cudaSuccess;
-#define QML_SET_ATTR(B, S, V)                                                                                    \
+#define QML_SET_ATTR(B, S, V, R)                                                                                 \
   if (e == cudaSuccess)                                                                                          \
-    e = cudaFuncSetAttribute(pass_kernel<B, S, V>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+    e = cudaFuncSetAttribute(pass_kernel<B, S, V, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
   if (e == cudaSuccess)                                                                                          \
-    e = cudaFuncSetAttribute(pass_kernel<B, S, V>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    e = cudaFuncSetAttribute(pass_kernel<B, S, V, R>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   QML_FOR_EACH_PASS_KERNEL(QML_SET_ATTR)
 #undef QML_SET_ATTR
   return e;
@@ -1171,10 +1280,10 @@ int debug_layouts(int* out, int cap) {
 
 cudaError_t pass_occupancy(bool backward, bool slow, size_t smem, int* blocks_per_sm) {
   if (backward)
-    return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, 0, 0>, kThreads, smem)
-                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, 2, 1>, kThreads, smem);
-  return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, 0, 0>, kThreads, smem)
-              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, 2, 1>, kThreads, smem);
+    return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, 0, 0, false>, kThreads, smem)
+                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, 2, 1, false>, kThreads, smem);
+  return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, 0, 0, false>, kThreads, smem)
+              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, 2, 1, false>, kThreads, smem);
 }
 
 cudaError_t launch_pass(bool backward, const PassArgs& a, const DevPass& p, const PassMaps& maps, int grid,
@@ -1182,9 +1291,10 @@ cudaError_t launch_pass(bool backward, const PassArgs& a, const DevPass& p, cons
   const int mode = p.slow ? 0 : p.tma ? 2 : 1;
   const CUtensorMap& m0 = *reinterpret_cast<const CUtensorMap*>(maps.m0);
   const CUtensorMap& m1 = *reinterpret_cast<const CUtensorMap*>(maps.m1);
-#define QML_LAUNCH(B, M, V)                                                                 \
-  if (backward == B && mode == M && p.variant == V) {                                       \
-    pass_kernel<B, M, V><<<grid, kThreads, smem, s>>>(a, p, m0, m1);                        \
+  const bool re = a.reupload != 0;
+#define QML_LAUNCH(B, M, V, R)                                                              \
+  if (backward == B && mode == M && p.variant == V && re == R) {                            \
+    pass_kernel<B, M, V, R><<<grid, kThreads, smem, s>>>(a, p, m0, m1);                     \
     return cudaGetLastError();                                                              \
   }
   QML_FOR_EACH_PASS_KERNEL(QML_LAUNCH)

@@ -17,13 +17,14 @@ struct PassArgs {
   float2* buf0;          // forward: psi; backward: psi (plane 0)
   float2* buf1;          // backward: lambda (plane 1)
   float2* dummy;         // forward: partner plane of the last unit when B is odd
-  const float2* enc;     // forward: [U][n][2] (cos, sin)(x/2) pairs
+  const float2* enc;     // [U][n][2] (cos, sin)(x/2) of the unit's two samples (lane pairs)
   const float* g;        // backward: dL/dE [B]
   void* ckpt;            // checkpoint slots
   int storage;           // 0 fp32, 1 bf16
   int bmax;              // samples per checkpoint slot (slot stride)
   float* partials;       // backward gradient partials
   unsigned* status;
+  int reupload;          // every layer starts with the encoding Ry(x_q) again
   uint32_t cz_nb[kMaxQubits];    // CZ neighbours of each qubit (qubit mask)
   uint32_t cz_nbhi[kMaxQubits];  // CZ neighbours of each qubit above it (qubit mask)
 };

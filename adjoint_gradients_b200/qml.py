@@ -31,7 +31,7 @@ EXPORTS = [
     "qml_host_workspace_bytes", "qml_step_host", "qml_sync", "qml_debug_schedule",
     "qml_enable_timing", "qml_read_timing", "qml_launch_count", "qml_expect_z0_static",
     "qml_debug_tile_view", "qml_debug_layouts", "qml_set_observable", "qml_observable_terms",
-    "qml_expect_observable", "qml_set_entangler", "qml_entangler_bonds",
+    "qml_expect_observable", "qml_set_entangler", "qml_entangler_bonds", "qml_set_reupload", "qml_reupload",
 ]
 
 
@@ -106,6 +106,8 @@ def load_library(path: str = LIB_PATH):
         "qml_expect_observable": ([_vp, _vp, _i, _vp, _vp], _i),
         "qml_set_entangler": ([_vp, _i, ctypes.POINTER(_i)], _i),
         "qml_entangler_bonds": ([_vp], _i),
+        "qml_set_reupload": ([_vp, _i], _i),
+        "qml_reupload": ([_vp], _i),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -213,6 +215,14 @@ class Context:
         flat = [int(v) for e in bonds for v in e]
         arr = (ctypes.c_int * max(1, len(flat)))(*flat)
         _check(self.lib.qml_set_entangler(self._h, len(bonds), arr), "qml_set_entangler")
+
+    def set_reupload(self, on: bool = True):
+        """Data re-uploading: every layer starts with the encoding Ry(x_q) again."""
+        _check(self.lib.qml_set_reupload(self._h, 1 if on else 0), "qml_set_reupload")
+
+    @property
+    def reupload(self) -> bool:
+        return bool(self.lib.qml_reupload(self._h))
 
     @property
     def entangler_bonds(self) -> int:

@@ -277,6 +277,7 @@ def run_ours(args):
     ctx.set_observable(obs)
     bonds = entangler_bonds(args.entangler, w.n)
     ctx.set_entangler(bonds)
+    ctx.set_reupload(args.reupload)
     psi = ctx.new_state(B)
     lam = ctx.new_state(B)
     E = torch.empty(B, dtype=torch.float32, device=dev)
@@ -362,6 +363,7 @@ def run_ours(args):
         ctx_h = qml.Context(w.n, w.L, B, ckpt_block=w.ckpt_block, storage=w.storage, device=local, host_step=True)
         ctx_h.set_observable(obs)
         ctx_h.set_entangler(bonds)
+        ctx_h.set_reupload(args.reupload)
         xh = torch.tensor(x, dtype=torch.float32).pin_memory()
         th = torch.tensor(theta, dtype=torch.float32).pin_memory()
         yh = torch.tensor(y, dtype=torch.float32).pin_memory()
@@ -401,6 +403,7 @@ def run_ours(args):
     cfg = {**workload_config(w, B), "parallelism": f"dp{world}" if world > 1 else "single",
            "observable": "Z0" if obs is None else f"{args.observable} ({len(obs)} Pauli strings)",
            "entangler": f"CZ {args.entangler} ({len(bonds)} bonds)",
+           "reupload": bool(args.reupload),
            "peak_hbm_bytes": int(torch.cuda.max_memory_allocated(dev))}
     if w.samples_per_epoch:
         cfg["s_per_epoch"] = w.samples_per_epoch / (value / world)
@@ -435,6 +438,7 @@ def main():
                     help="z0: <Z0> (the workloads' readout); tfim: sum_q Z_q Z_q+1 + 0.9 sum_q X_q")
     ap.add_argument("--entangler", default="chain", choices=["chain", "ring", "none"],
                     help="CZ bonds ending every layer: chain (q, q+1) as in the workloads, ring, or none")
+    ap.add_argument("--reupload", action="store_true", help="data re-uploading: the encoding again in every layer")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -182,6 +182,14 @@ QML_API qml_status qml_set_entangler(qml_ctx* ctx, int n_bonds, const int* bonds
 /* Number of bonds of the entangler in force. */
 QML_API int qml_entangler_bonds(const qml_ctx* ctx);
 
+/* Data re-uploading for the following forward and backward calls: with
+ * on != 0 every layer starts with the angle encoding Ry(x[b][q]) on every
+ * qubit again (no parameters; its inverse is un-applied in the backward pass,
+ * which then needs x_dev).  Off after qml_create.  QML_ERR_UNSUPPORTED for
+ * n_qubits < 5.  Set it before the forward pass whose backward it serves. */
+QML_API qml_status qml_set_reupload(qml_ctx* ctx, int on);
+QML_API int qml_reupload(const qml_ctx* ctx);
+
 /* Largest number of Pauli-string terms an observable may have. */
 #define QML_MAX_OBS_TERMS 4096
 

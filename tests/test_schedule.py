@@ -148,3 +148,14 @@ def test_set_entangler_validates_and_counts():
     assert ctx.entangler_bonds == 0
     ctx.set_entangler(None)
     assert ctx.entangler_bonds == 4
+
+
+def test_set_reupload_flags():
+    ctx = qml.Context(6, 2, 4, workspace=False)
+    assert not ctx.reupload
+    ctx.set_reupload(True)
+    assert ctx.reupload
+    ctx.set_reupload(False)
+    assert not ctx.reupload
+    small = qml.Context(3, 2, 4, workspace=False)
+    assert small.lib.qml_set_reupload(small._h, 1) == 2  # QML_ERR_UNSUPPORTED below 5 qubits
