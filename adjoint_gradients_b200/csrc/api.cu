@@ -224,7 +224,7 @@ bool same_tma_view(const DevPass& x, const DevPass& y) {
 const PassMaps* pass_maps(qml_ctx* c, int p, bool backward, int B, const void* buf0, const void* buf1) {
   static const PassMaps none{};
   const DevPass& dp = c->dpass[p];
-  if (!dp.tma) return &none;
+  if (!dp.tma || !buf0) return &none;
   for (const qml_ctx::MapEntry& m : c->maps)
     if (m.backward == backward && m.B == B && m.buf0 == buf0 && m.buf1 == buf1 && same_tma_view(c->dpass[m.pass], dp))
       return &m.maps;
@@ -273,6 +273,25 @@ void set_bond_masks(qml_ctx* c) {
   }
 }
 
+// Conversion between the standard order and the working-state order of the
+// plan (addr_of); both move only the lowest index bits, within chunks.
+cudaError_t convert_layout(qml_ctx* c, float2* buf, int B, bool to_working, cudaStream_t s) {
+  const int n = c->cfg.n_qubits;
+  int cb = 0;
+  for (int q = 0; q < n; ++q)
+    if (c->plan.addr_of[q] != q) cb = std::max(cb, std::max(q, c->plan.addr_of[q]) + 1);
+  if (cb == 0) return cudaSuccess;
+  ++c->launches;
+  int to[kTileBits];
+  for (int b = 0; b < cb; ++b) {
+    if (to_working) to[b] = c->plan.addr_of[b];  // standard bit b -> its address bit
+    else
+      for (int q = 0; q < cb; ++q)
+        if (c->plan.addr_of[q] == b) to[b] = q;  // address bit b -> its qubit
+  }
+  return launch_permute_bits(buf, (long long)B << n, cb, to, c->sms * 8, s);
+}
+
 qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, float2* psi,
                        float* expect, cudaStream_t s) {
   const int n = c->cfg.n_qubits;
@@ -317,6 +336,8 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
     if (dp.ckpt >= 0) c->ckpt_batch[dp.ckpt] = B;
   }
   if (timed) span_end(c, s, &sp);
+  e = convert_layout(c, psi, B, false, s);  // working-state order -> standard order
+  if (e != cudaSuccess) return QML_ERR_CUDA;
   if (expect) {
     c->launches += 2;
     e = launch_expectation(c, psi, B, expect, s);
@@ -342,6 +363,9 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
       e = launch_obs_bwd_init(psi, lam, g, B, n, at<ObsGroup>(c, c->lay.obs_groups), (int)c->obs_groups.size(),
                               at<ObsTerm>(c, c->lay.obs_terms), s);
   }
+  if (e != cudaSuccess) return QML_ERR_CUDA;
+  e = convert_layout(c, psi, B, true, s);  // both backward planes: standard -> working-state order
+  if (e == cudaSuccess) e = convert_layout(c, lam, B, true, s);
   if (e != cudaSuccess) return QML_ERR_CUDA;
   if (c->reupload) {  // per-sample encoding angles for un-applying the re-uploaded encodings
     e = launch_prep_enc(x, B, n, at<float2>(c, c->lay.enc), s);
@@ -765,6 +789,9 @@ int qml_debug_tile_view(const qml_ctx* c, int pass, int* out, int cap) {
   }
   v.push_back(d.n_out);
   for (int i = 0; i < d.n_out; ++i) v.push_back(d.out_q[i]);
+  for (int b = 0; b < kTileBits; ++b) v.push_back(d.tile_abit[b] ? __builtin_ctz(d.tile_abit[b]) : -1);
+  for (int i = 0; i < d.n_out; ++i) v.push_back(__builtin_ctz(d.out_abit[i]));
+  v.push_back(d.variant);
   if (out)
     for (int i = 0; i < cap && i < (int)v.size(); ++i) out[i] = v[i];
   return (int)v.size();

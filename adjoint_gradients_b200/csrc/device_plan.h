@@ -39,8 +39,8 @@ constexpr int kCoefRegions = 40;      // per-context regions of constant memory
 enum : int { OP_EXCH = 1, OP_ROT = 2, OP_CZ = 3, OP_GEN = 4 };
 
 // Tensor-copy (TMA) view of a pass's tile, used when n > 12: the state
-// [B][2^n] is seen as a rank-5 tensor whose dimensions are runs of qubits
-// (in increasing qubit order) plus the sample index.  A run of in-tile qubits
+// [B][2^n] (working-state address order) is seen as a rank-5 tensor whose
+// dimensions are runs of address bits plus the sample index.  A run of in-tile qubits
 // is copied whole (box = 2^bits, at most 8 bits per dimension); a run of
 // out-of-tile qubits is fixed per tile (box 1, coordinate = those bits of the
 // tile's out-of-tile index); the sample dimension has box 1, merged with the
@@ -70,12 +70,14 @@ struct DevPass {
   int pf_fwd, pf_bwd;   // op index after which the next tile is prefetched (-1: right after loading)
   int tma;              // 1: tiles are loaded by tensor copies (see kTmaRank)
   int tma_kind[kTmaRank];
-  int tma_qlo[kTmaRank];    // lowest qubit of the run (TD_IN, TD_OUT, TD_OUT_SAMPLE)
-  int tma_bits[kTmaRank];   // qubits in the run
+  int tma_qlo[kTmaRank];    // lowest address bit of the run (TD_IN, TD_OUT, TD_OUT_SAMPLE)
+  int tma_bits[kTmaRank];   // address bits in the run
   int tma_shift[kTmaRank];  // TD_OUT, TD_OUT_SAMPLE: first bit of the run in the out-of-tile index
   int sstride[kTileBits];   // element offset in the copied tile of each tile bit (plane 1 at +4096)
   int tile_q[kTileBits];  // tile bit -> qubit (>= 0) or -1 - (batch-unit bit)
-  int out_q[kMaxOut];     // out-of-tile qubits, increasing
+  int out_q[kMaxOut];     // out-of-tile qubits, in increasing address order
+  uint32_t tile_abit[kTileBits];  // tile bit -> its address bit in the working state (0: unit bit)
+  uint32_t out_abit[kMaxOut];     // out-of-tile qubit -> its address bit
   uint32_t cz_reg[kPhases];  // bit j: entangler parity of the register part of position j
   uint32_t cz_nb[kPhases][kRegBits];  // CZ neighbours (qubit mask) of each register bit's qubit
   long long partial_off;     // float offset of this pass's gradient partials

@@ -332,6 +332,7 @@ __device__ __forceinline__ uint32_t thr_slot(uint32_t tid) {
 struct BlockCtx {
   uint32_t qbit[kTileBits];  // tile bit -> 1 << qubit (0 for a unit bit)
   uint32_t ubit[kTileBits];  // tile bit -> unit increment (0 for a qubit)
+  uint32_t abit[kTileBits];  // tile bit -> its address bit in the working state (0 for a unit bit)
   unsigned long long mbar;   // completion barrier of the tile's tensor copies
   int tma_c[2][kTmaRank];    // tensor coordinates of the next tile's copies
   int tma_sel;               // plane 1 of the next tile comes through tm1
@@ -356,7 +357,18 @@ __device__ __forceinline__ void thread_pos(const BlockCtx& bc, uint32_t tid, uin
 struct RegMaps {
   uint32_t q[kRegBits];  // qubit bit of register bit k (0 if a unit bit)
   uint32_t u[kRegBits];  // unit increment of register bit k (0 if a qubit)
+  uint32_t a[kRegBits];  // working-state address bit of register bit k (0 if a unit bit)
 };
+
+// Working-state address bits of this thread's fixed tile bits in layout P.
+template <int P, int V>
+__device__ __forceinline__ uint32_t thread_addr(const BlockCtx& bc, uint32_t tid) {
+  uint32_t x = 0;
+#pragma unroll
+  for (int m = 0; m < kThrBits; ++m)
+    if ((tid >> m) & 1u) x |= bc.abit[thr_tbit<P, V>(m)];
+  return x;
+}
 
 template <int P>
 __device__ __forceinline__ RegMaps reg_maps(const BlockCtx& bc) {
@@ -365,6 +377,7 @@ __device__ __forceinline__ RegMaps reg_maps(const BlockCtx& bc) {
   for (int k = 0; k < kRegBits; ++k) {
     m.q[k] = bc.qbit[reg_tbit<P>(k)];
     m.u[k] = bc.ubit[reg_tbit<P>(k)];
+    m.a[k] = bc.abit[reg_tbit<P>(k)];
   }
   return m;
 }
@@ -457,18 +470,26 @@ struct Planes {
 // What a pass does to HBM at its start or end, in the memory layout P.
 enum MemOp { M_LOAD, M_STORE, M_STORE_STD, M_GEN, M_CKPT_STORE, M_CKPT_RESTORE };
 
+// The state in the buffers is stored at working-state addresses
+// (DevPass::tile_abit / out_abit; the identity unless the plan has three or
+// more qubit sets, in which case separate kernels convert it from and to the
+// standard order at the ends of the pass chain).  The encoding and the
+// checkpoint slots use the standard index, i.e. the qubit bits.
 template <bool BWD, bool SLOW, int P, int V, int OP>
 __device__ __forceinline__ void mem_t(const PassArgs& a, const BlockCtx& bc, uint32_t tid, uint32_t base_q,
-                                      uint32_t unit_base, float2 (&re)[kPos], float2 (&im)[kPos], int slot) {
+                                      uint32_t base_a, uint32_t unit_base, float2 (&re)[kPos], float2 (&im)[kPos],
+                                      int slot) {
   uint32_t aq, ut;
   thread_pos<P, V>(bc, tid, &aq, &ut);
-  aq |= base_q;
+  constexpr bool std_index = !(OP == M_LOAD || OP == M_STORE || OP == M_STORE_STD);
+  if (std_index) aq |= base_q;
+  else aq = thread_addr<P, V>(bc, tid) | base_a;
   ut += unit_base;
   const RegMaps m = reg_maps<P>(bc);
   const int n = a.n;
 #pragma unroll
   for (int j = 0; j < kPos; ++j) {
-    const uint32_t i = aq | REG_COMBINE(m.q, j, |=);
+    const uint32_t i = aq | (std_index ? REG_COMBINE(m.q, j, |=) : REG_COMBINE(m.a, j, |=));
     const uint32_t u = SLOW ? ut + REG_COMBINE(m.u, j, +=) : ut;
     const bool ok = u < (uint32_t)a.U;
     if constexpr (OP == M_LOAD) {
@@ -526,11 +547,11 @@ __device__ __forceinline__ void mem_t(const PassArgs& a, const BlockCtx& bc, uin
 
 template <bool BWD, bool SLOW, int V, int OP>
 __device__ __forceinline__ void mem_op(int phase, const PassArgs& a, const BlockCtx& bc, uint32_t tid,
-                                       uint32_t base_q, uint32_t unit_base, float2 (&re)[kPos],
+                                       uint32_t base_q, uint32_t base_a, uint32_t unit_base, float2 (&re)[kPos],
                                        float2 (&im)[kPos], int slot = 0) {
   // memory ops run in phase 0 or 1 (the planner never picks phase 2)
-  if (phase == 0) mem_t<BWD, SLOW, 0, V, OP>(a, bc, tid, base_q, unit_base, re, im, slot);
-  else mem_t<BWD, SLOW, 1, V, OP>(a, bc, tid, base_q, unit_base, re, im, slot);
+  if (phase == 0) mem_t<BWD, SLOW, 0, V, OP>(a, bc, tid, base_q, base_a, unit_base, re, im, slot);
+  else mem_t<BWD, SLOW, 1, V, OP>(a, bc, tid, base_q, base_a, unit_base, re, im, slot);
 }
 
 // Prefetch of the block's next tile: each thread copies its own positions of
@@ -538,12 +559,14 @@ __device__ __forceinline__ void mem_op(int phase, const PassArgs& a, const Block
 // cp.async (zero fill for batch units past the end).
 template <bool BWD, int P, int V>
 __device__ __forceinline__ void prefetch_t(const PassArgs& a, const BlockCtx& bc, uint32_t tid, uint32_t base_q,
-                                           uint32_t unit_base, float4* tile) {
+                                           uint32_t base_a, uint32_t unit_base, float4* tile) {
   uint32_t aq, ut;
   thread_pos<P, V>(bc, tid, &aq, &ut);
-  aq |= base_q;
+  aq = thread_addr<P, V>(bc, tid) | base_a;
   ut += unit_base;
-  const RegMaps m = reg_maps<P>(bc);
+  RegMaps m = reg_maps<P>(bc);
+#pragma unroll
+  for (int k = 0; k < kRegBits; ++k) m.q[k] = m.a[k];
   const bool ok = ut < (uint32_t)a.U;
   const float2* p0 = Planes<BWD>::p0(a, ok ? ut : 0u) + (ok ? aq : 0u);
   const float2* p1 = Planes<BWD>::p1(a, ok ? ut : 0u) + (ok ? aq : 0u);
@@ -561,9 +584,9 @@ __device__ __forceinline__ void prefetch_t(const PassArgs& a, const BlockCtx& bc
 
 template <bool BWD, int V>
 __device__ __forceinline__ void prefetch_op(int phase, const PassArgs& a, const BlockCtx& bc, uint32_t tid,
-                                            uint32_t base_q, uint32_t unit_base, float4* tile) {
-  if (phase == 0) prefetch_t<BWD, 0, V>(a, bc, tid, base_q, unit_base, tile);
-  else prefetch_t<BWD, 1, V>(a, bc, tid, base_q, unit_base, tile);
+                                            uint32_t base_q, uint32_t base_a, uint32_t unit_base, float4* tile) {
+  if (phase == 0) prefetch_t<BWD, 0, V>(a, bc, tid, base_q, base_a, unit_base, tile);
+  else prefetch_t<BWD, 1, V>(a, bc, tid, base_q, base_a, unit_base, tile);
 }
 
 // Registers of layout P from the thread's own prefetched slots.
@@ -709,13 +732,16 @@ __device__ __forceinline__ void load_tma(int phase, float2 (&re)[kPos], float2 (
 }
 
 // Out-of-tile qubit bits and first batch unit of tile t.
-__device__ __forceinline__ void tile_base(const DevPass& P, int t, uint32_t* base_q, uint32_t* unit_base) {
+// (out-of-tile bits as qubit bits and as working-state address bits)
+__device__ __forceinline__ void tile_base(const DevPass& P, int t, uint32_t* base_q, uint32_t* base_a,
+                                          uint32_t* unit_base) {
   const int n_out = P.n_out;
   const uint32_t o = (uint32_t)t & ((1u << n_out) - 1u);
-  uint32_t bq = 0;
+  uint32_t bq = 0, ba = 0;
   for (int k = 0; k < n_out; ++k)
-    if ((o >> k) & 1u) bq |= 1u << P.out_q[k];
+    if ((o >> k) & 1u) bq |= 1u << P.out_q[k], ba |= P.out_abit[k];
   *base_q = bq;
+  *base_a = ba;
   *unit_base = ((uint32_t)t >> n_out) << P.unit_bits;
 }
 
@@ -814,6 +840,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     const int q = P.tile_q[tid];
     bc->qbit[tid] = q >= 0 ? (1u << q) : 0u;
     bc->ubit[tid] = q >= 0 ? 0u : (1u << (-1 - q));
+    bc->abit[tid] = P.tile_abit[tid];
   }
   if (BWD)
     for (int i = tid; i < kWarps * nacc; i += kThreads) acc[i] = 0.f;
@@ -846,8 +873,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   const int pf_at = BWD ? P.pf_bwd : P.pf_fwd;  // op index after which to prefetch (-1: after the load)
   bool have_pf = false;
   for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x) {
-    uint32_t base_q, unit_base;
-    tile_base(P, t, &base_q, &unit_base);
+    uint32_t base_q, base_a, unit_base;
+    tile_base(P, t, &base_q, &base_a, &unit_base);
     const uint32_t s_o = bond_parity(base_q, a);  // entangler terms of the out-of-tile bits
     const int tn = t + (int)gridDim.x;
     const bool pf_next = can_pf && tn < a.n_tiles;
@@ -856,9 +883,9 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
       if (TMA) {
         if (tid == 0) tma_load_tile(&tm0, &tm1, bc->tma_sel, bc->tma_c, tile_s, mbar);
       } else {
-        uint32_t bq, ub;
-        tile_base(P, tn, &bq, &ub);
-        prefetch_op<BWD, V>(mem_ph, a, *bc, tid, bq, ub, tile);
+        uint32_t bq, ba, ub;
+        tile_base(P, tn, &bq, &ba, &ub);
+        prefetch_op<BWD, V>(mem_ph, a, *bc, tid, bq, ba, ub, tile);
       }
     };
 
@@ -884,10 +911,10 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
       load_tma<V>(mem_ph, re, im, tb, P, tid);
     }
     if (!BWD) {
-      if (P.gen) mem_op<false, SLOW, V, M_GEN>(P.load_phase, a, *bc, tid, base_q, unit_base, re, im);
+      if (P.gen) mem_op<false, SLOW, V, M_GEN>(P.load_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
       else if (TMA) {
       } else if (have_pf) load_prefetched<V>(P.load_phase, re, im, tile, tid);
-      else mem_op<false, SLOW, V, M_LOAD>(P.load_phase, a, *bc, tid, base_q, unit_base, re, im);
+      else mem_op<false, SLOW, V, M_LOAD>(P.load_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
       if (pf_next && pf_at < 0) prefetch_next();
       for (int oi = 0; oi < P.nops; ++oi) {
         const DevOp op = P.ops[oi];
@@ -911,14 +938,14 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
         }
         if (pf_next && oi == pf_at) prefetch_next();
       }
-      if (P.ckpt >= 0) mem_op<false, SLOW, V, M_CKPT_STORE>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im, P.ckpt);
-      if (P.last) mem_op<false, SLOW, V, M_STORE_STD>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im);
-      else mem_op<false, SLOW, V, M_STORE>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im);
+      if (P.ckpt >= 0) mem_op<false, SLOW, V, M_CKPT_STORE>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im, P.ckpt);
+      if (P.last) mem_op<false, SLOW, V, M_STORE_STD>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
+      else mem_op<false, SLOW, V, M_STORE>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
     } else {
       if (TMA) {
       } else if (have_pf) load_prefetched<V>(P.store_phase, re, im, tile, tid);
-      else mem_op<true, SLOW, V, M_LOAD>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im);
-      if (!TMA && P.ckpt >= 0) mem_op<true, SLOW, V, M_CKPT_RESTORE>(P.store_phase, a, *bc, tid, base_q, unit_base, re, im, P.ckpt);
+      else mem_op<true, SLOW, V, M_LOAD>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
+      if (!TMA && P.ckpt >= 0) mem_op<true, SLOW, V, M_CKPT_RESTORE>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im, P.ckpt);
       if (pf_next && pf_at < 0) prefetch_next();
       for (int oi = P.nops - 1; oi >= 0; --oi) {
         const DevOp op = P.ops[oi];
@@ -954,7 +981,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
         }
         if (pf_next && oi == pf_at) prefetch_next();
       }
-      if (!P.gen) mem_op<true, SLOW, V, M_STORE>(P.load_phase, a, *bc, tid, base_q, unit_base, re, im);
+      if (!P.gen) mem_op<true, SLOW, V, M_STORE>(P.load_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
     }
     have_pf = pf_next;
   }
@@ -1199,6 +1226,31 @@ __global__ void planes_kernel(float2* psi, float2* lam, long long count) {
   lam[idx] = make_float2(v.y, l.y);
 }
 
+// In-place permutation of the low index bits of every aligned chunk of
+// 2^cb elements: element j of a chunk moves to position sum_b j_b << to[b].
+// A chunk maps onto itself, so one block per chunk makes it race-free.
+struct BitPerm {
+  int cb;
+  int to[kTileBits];
+};
+
+__global__ void permute_bits_kernel(float2* buf, long long chunks, const BitPerm perm) {
+  extern __shared__ float2 chunk[];
+  const int size = 1 << perm.cb;
+  for (long long c = blockIdx.x; c < chunks; c += gridDim.x) {
+    float2* base = buf + (size_t)c * size;
+    for (int j = threadIdx.x; j < size; j += blockDim.x) chunk[j] = base[j];
+    __syncthreads();
+    for (int j = threadIdx.x; j < size; j += blockDim.x) {
+      // the element that lands at j comes from src with j = sum_b src_b << to[b]
+      int src = 0;
+      for (int b = 0; b < perm.cb; ++b) src |= ((j >> perm.to[b]) & 1) << b;
+      base[j] = chunk[src];
+    }
+    __syncthreads();
+  }
+}
+
 __global__ void bwd_init_kernel(float2* psi, float2* lam, const float* g, int B, int n) {
   const long long N = 1ll << n;
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -1440,6 +1492,15 @@ cudaError_t launch_obs_bwd_init(float2* psi, float2* lam, const float* g, int B,
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   planes_kernel<<<blocks, 256, 0, s>>>(psi, lam, tot);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_bits(float2* buf, long long count, int cb, const int* to, int grid, cudaStream_t s) {
+  BitPerm perm{};
+  perm.cb = cb;
+  for (int b = 0; b < cb; ++b) perm.to[b] = to[b];
+  const long long chunks = count >> cb;
+  permute_bits_kernel<<<grid, 256, sizeof(float2) << cb, s>>>(buf, chunks, perm);
   return cudaGetLastError();
 }
 

@@ -71,6 +71,11 @@ cudaError_t launch_loss_seed(const float* E, const float* y, int B, float* g, fl
                              cudaStream_t s);
 cudaError_t launch_bwd_init(float2* psi, float2* lam, const float* g, int B, int n, cudaStream_t s);
 
+// In place, for every aligned chunk of 2^cb elements of buf (count elements):
+// element j moves to sum_b j_b << to[b] (a permutation of the low cb index
+// bits, cb <= 12).
+cudaError_t launch_permute_bits(float2* buf, long long count, int cb, const int* to, int grid, cudaStream_t s);
+
 // Observables O = sum_k c_k i^ny X^x Z^z, terms grouped by x (see kernels.cu).
 struct ObsTerm {
   uint32_t z;  // qubits carrying Z or Y

@@ -28,31 +28,32 @@ bool phase_fast(const HostPass& ps, int p) {
 }
 
 
-// Tensor-copy view of the tile (see kTmaRank).  Multi-set plans only: their
-// tiles hold no batch-unit bit, qubit 0 is always in the tile (rotated or
-// passive), and at least two low qubits are, so the innermost run is >= 32 B.
-void set_tma_view(int n, const HostPass& ps, DevPass* d) {
+// Tensor-copy view of the tile (see kTmaRank) over the address bits of the
+// working-state layout (addr_of).  Multi-set plans only: their tiles hold no
+// batch-unit bit, address bits 0 and 1 are always in the tile, so the
+// innermost run is >= 32 B.
+void set_tma_view(int n, const HostPass& ps, const std::vector<int>& addr_of, DevPass* d) {
   d->tma = 0;
   for (int i = 0; i < kTmaRank; ++i) d->tma_kind[i] = TD_PAD, d->tma_qlo[i] = d->tma_bits[i] = d->tma_shift[i] = 0;
   for (int b = 0; b < kTileBits; ++b) d->sstride[b] = 0;
   if (n <= kTileBits || ps.slow || ps.unit_bits != 0) return;
-  std::vector<int> tbit_of_q(n, -1);
+  std::vector<int> tbit_of_a(n, -1);  // address bit -> tile bit
   for (int b = 0; b < kTileBits; ++b)
-    if (ps.tile_q[b] >= 0) tbit_of_q[ps.tile_q[b]] = b;
-  if (tbit_of_q[0] < 0 || tbit_of_q[1] < 0) return;
+    if (ps.tile_q[b] >= 0) tbit_of_a[addr_of[ps.tile_q[b]]] = b;
+  if (tbit_of_a[0] < 0 || tbit_of_a[1] < 0) return;
   int rank = 0, out_seen = 0;
   long long box = 1;  // elements of the box below the current dimension
   int q = 0;
   while (q < n) {
-    const bool in = tbit_of_q[q] >= 0;
+    const bool in = tbit_of_a[q] >= 0;
     int e = q;
-    while (e < n && (tbit_of_q[e] >= 0) == in) ++e;
+    while (e < n && (tbit_of_a[e] >= 0) == in) ++e;
     if (in) {
       for (int lo = q; lo < e; lo += 8) {
         const int bits = std::min(8, e - lo);
         if (rank == kTmaRank) return;
         d->tma_kind[rank] = TD_IN, d->tma_qlo[rank] = lo, d->tma_bits[rank] = bits;
-        for (int k = 0; k < bits; ++k) d->sstride[tbit_of_q[lo + k]] = (int)(box << k);
+        for (int k = 0; k < bits; ++k) d->sstride[tbit_of_a[lo + k]] = (int)(box << k);
         box <<= bits;
         ++rank;
       }
@@ -65,7 +66,7 @@ void set_tma_view(int n, const HostPass& ps, DevPass* d) {
     }
     q = e;
   }
-  if (tbit_of_q[n - 1] >= 0) {  // highest qubit in the tile: a separate sample dimension
+  if (tbit_of_a[n - 1] >= 0) {  // highest address bit in the tile: a separate sample dimension
     if (rank == kTmaRank) return;
     d->tma_kind[rank] = TD_SAMPLE;
     ++rank;
@@ -102,6 +103,23 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
   }
   p.n_sets = (int)p.sets.size();
   const int S = p.n_sets;
+  // ---- working-state address bits: identity, except that plans with three
+  // or more sets move the second set's first two qubits to address bits 2
+  // and 3 (every set's tile then covers address bits 0-3 or 0-2: HBM runs of
+  // >= 64 B instead of 32 B); the layout is converted to and from the
+  // standard one by a separate kernel at the ends of the pass chain
+  p.addr_of.resize(n);
+  {
+    std::vector<int> order;
+    if (S >= 3) {
+      order = {0, 1, p.sets[1][0], p.sets[1][1]};
+      for (int q = 0; q < n; ++q)
+        if (std::find(order.begin(), order.end(), q) == order.end()) order.push_back(q);
+    } else {
+      for (int q = 0; q < n; ++q) order.push_back(q);
+    }
+    for (int a = 0; a < n; ++a) p.addr_of[order[a]] = a;
+  }
   p.n_ckpt = (ckpt_block > 0) ? (L + ckpt_block - 1) / ckpt_block - 1 : 0;
 
   // ---- task list: encode, then per layer the sets in boustrophedon order, then CZ
@@ -165,35 +183,46 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
       ps.unit_bits = kTileBits - n;
       for (int t = 0; t < kTileBits; ++t) ps.tile_q[t] = t < n ? t : -1 - (t - n);
     } else {
-      // The lowest other qubits are passive tile bits.  If the set starts at
-      // qubit 0 (variant 0), the set sits on tile bits 0 .. |R|-1 and phase
-      // 1's lanes (tile bits 0-4) are qubits 0-4.  Otherwise (variant 1) the
-      // two lowest passive qubits go to tile bits 10 and 11 and the others to
-      // tile bits 0, 1, ..., then the set: phase 1's lanes are tile bits 10,
-      // 11, 0, 1, 2 in lane order, so a half warp covers the lowest in-tile
-      // qubits (contiguous HBM runs, contiguous elements of a copied tile).
+      // The passive tile bits are the other qubits with the lowest address
+      // bits; the out-of-tile qubits are listed in address order.
       const std::vector<int>& set = p.sets[pr.set];
       std::vector<bool> in(n, false);
       for (int q : set) in[q] = rotated_q[q] = true;
+      std::vector<int> by_addr(n);
+      for (int q = 0; q < n; ++q) by_addr[p.addr_of[q]] = q;
       std::vector<int> passive;
-      for (int q = 0; q < n && (int)(set.size() + passive.size()) < kTileBits; ++q)
+      for (int a = 0; a < n && (int)(set.size() + passive.size()) < kTileBits; ++a) {
+        const int q = by_addr[a];
         if (!in[q]) {
           passive.push_back(q);
           in[q] = true;
         }
-      for (int q = 0; q < n; ++q)
-        if (!in[q]) ps.out_q.push_back(q);
+      }
+      for (int a = 0; a < n; ++a)
+        if (!in[by_addr[a]]) ps.out_q.push_back(by_addr[a]);
       ps.unit_bits = 0;
-      ps.variant = set[0] == 0 ? 0 : 1;
-      if (ps.variant == 0) {
+      const bool identity = S < 3;
+      if (identity && set[0] == 0) {
+        // variant 0: the set on tile bits 0 .. |R|-1, passive after; phase
+        // 1's lanes (tile bits 0-4) are qubits 0-4
+        ps.variant = 0;
         for (int t = 0; t < (int)set.size(); ++t) ps.tile_q[t] = set[t];
         for (size_t i = 0; i < passive.size(); ++i) ps.tile_q[set.size() + i] = passive[i];
       } else {
+        // variant 1: the two lowest-address passive qubits on tile bits 10
+        // and 11 (never rotated: register bits only in phase 2), the other
+        // in-tile qubits on tile bits 0 .. 9 in address order.  Phase 1's
+        // lanes are tile bits 10, 11, 0, 1, 2 in lane order, so a warp
+        // covers the five lowest in-tile addresses (long HBM runs; a half
+        // warp reads contiguous elements of a copied tile).
+        ps.variant = 1;
         ps.tile_q[10] = passive[0];
         ps.tile_q[11] = passive[1];
-        const int extra = (int)passive.size() - 2;
-        for (int i = 0; i < extra; ++i) ps.tile_q[i] = passive[2 + i];
-        for (int t = 0; t < (int)set.size(); ++t) ps.tile_q[extra + t] = set[t];
+        int t = 0;
+        for (int a = 0; a < n; ++a) {
+          const int q = by_addr[a];
+          if (in[q] && q != passive[0] && q != passive[1]) ps.tile_q[t++] = q;
+        }
       }
     }
     if ((int)ps.out_q.size() > kMaxOut) return "internal: too many out-of-tile qubits";
@@ -294,7 +323,9 @@ void flatten_plan(const Plan& p, std::vector<DevPass>* passes) {
         if (d.pf_bwd < 0) d.pf_bwd = o;
       }
     for (int t = 0; t < kTileBits; ++t) d.tile_q[t] = ps.tile_q[t];
-    set_tma_view(p.n, ps, &d);
+    set_tma_view(p.n, ps, p.addr_of, &d);
+    for (int b = 0; b < kTileBits; ++b) d.tile_abit[b] = ps.tile_q[b] >= 0 ? 1u << p.addr_of[ps.tile_q[b]] : 0u;
+    for (int i = 0; i < kMaxOut; ++i) d.out_abit[i] = i < d.n_out ? 1u << p.addr_of[ps.out_q[i]] : 0u;
     for (int i = 0; i < kMaxOut; ++i) d.out_q[i] = i < d.n_out ? ps.out_q[i] : -1;
     d.partial_off = 0;
     for (int s = 0; s < kMaxSlots; ++s) d.slot_lq[s] = s < d.nslots ? ps.slot_lq[s] : 0;

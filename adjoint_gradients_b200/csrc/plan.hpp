@@ -47,6 +47,11 @@ struct HostPass {
 struct Plan {
   int n = 0, L = 0, ckpt_block = 0;
   int n_sets = 0;
+  // Address bit of each qubit in the working state between passes (HBM
+  // layout; the standard layout is addr_of[q] = q).  Multi-set plans put the
+  // first two qubits of the second set at address bits 2 and 3, so that every
+  // set's tile is a run of >= 4 consecutive addresses plus these.
+  std::vector<int> addr_of;
   std::vector<std::vector<int>> sets;
   std::vector<HostPass> passes;
   std::vector<int> slot_pass;   // [L*n] -> pass of (layer, qubit)

@@ -254,7 +254,9 @@ class Context:
         tile_q = [v[i + 2 * b] for b in range(12)]
         sstride = [v[i + 2 * b + 1] for b in range(12)]
         n_out = v[i + 24]
-        return dict(tma=v[0], dims=dims, tile_q=tile_q, sstride=sstride, out_q=v[i + 25:i + 25 + n_out])
+        j = i + 25 + n_out
+        return dict(tma=v[0], dims=dims, tile_q=tile_q, sstride=sstride, out_q=v[i + 25:j],
+                    tile_addr=v[j:j + 12], out_addr=v[j + 12:j + 12 + n_out], variant=v[j + 12 + n_out])
 
     def enable_timing(self, on: bool = True):
         _check(self.lib.qml_enable_timing(self._h, 1 if on else 0), "qml_enable_timing")

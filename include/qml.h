@@ -289,9 +289,12 @@ QML_API int qml_debug_schedule(const qml_ctx* ctx, int* out, int cap);
  * argument).  Layout: [tensor-copy loads (0/1), then 5 dimensions x
  * (kind, lowest qubit, qubits, first bit in the out-of-tile index), then 12
  * tile bits x (qubit or -1 - unit bit, element offset in the copied tile),
- * then n_out, then the out-of-tile qubits].  Dimension kinds: 0 unused,
- * 1 in-tile qubits (copied whole), 2 out-of-tile qubits (fixed per tile),
- * 3 sample, 4 out-of-tile qubits merged with the sample index above them. */
+ * then n_out, then the out-of-tile qubits (in address order), then the
+ * working-state address bit of each tile bit (-1 for a unit bit) and of each
+ * out-of-tile qubit, then the register-layout variant].  Dimension kinds: 0
+ * unused, 1 in-tile address bits (copied whole), 2 out-of-tile address bits
+ * (fixed per tile), 3 sample, 4 out-of-tile address bits merged with the
+ * sample index above them.  The lowest address bit of a run is given. */
 QML_API int qml_debug_tile_view(const qml_ctx* ctx, int pass, int* out, int cap);
 
 /* Debugging aid: the kernels' register layouts, written like

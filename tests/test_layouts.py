@@ -46,8 +46,7 @@ def test_copied_tile_reads_have_no_bank_conflicts(n):
     for p in range(ctx.debug_schedule()[0]):
         v = ctx.debug_tile_view(p)
         assert v["tma"] == 1
-        variant = 1 if v["tile_q"][10] == 0 else 0
-        thr = lay[(1, variant)][0]
+        thr = lay[(1, v["variant"])][0]
         for h in range(2):
             banks = set()
             for lane in range(16 * h, 16 * h + 16):

@@ -1,13 +1,16 @@
 """CPU check of the tensor-copy view of each pass (no GPU).
 
 For circuits above 12 qubits a pass loads each tile with bulk tensor copies:
-the state [B][2^n] is viewed as a rank-5 tensor whose dimensions are runs of
-qubits and the sample index.  For every such pass this test recomputes, from
-the view the library reports, the element each copied box position comes
-from (the coordinate rule the kernel uses, restated here) and checks that
-  * the box is exactly the tile: position p of the tile (tile bits -> qubits,
-    out-of-tile bits from the tile index) lands at box offset sum_b p_b *
+the working state [B][2^n] (qubits stored at permuted address bits) is viewed
+as a rank-5 tensor whose dimensions are runs of address bits and the sample
+index.  For every such pass this test recomputes, from the view the library
+reports, the element each copied box position comes from (the coordinate
+rule the kernel uses, restated here) and checks that
+  * the box is exactly the tile: position p of the tile (tile bits -> address
+    bits, out-of-tile bits from the tile index) lands at box offset sum_b p_b *
     sstride[b], and that offset map is a bijection onto [0, 4096);
+  * the address bits are a permutation of the qubits, and every set's tile
+    covers address bits 0 and 1 (runs of >= 32 bytes);
   * the innermost dimension starts at qubit 0 and spans >= 16 bytes, and every
     other dimension's stride is a multiple of 16 bytes (tensor-copy rules).
 """
@@ -54,7 +57,10 @@ def test_tensor_copy_view_is_the_tile(n, L):
         v = ctx.debug_tile_view(p)
         assert v["tma"] == 1, f"pass {p} of n={n} has no tensor-copy view"
         tq, ss, out_q = v["tile_q"], v["sstride"], v["out_q"]
+        ta, oa = v["tile_addr"], v["out_addr"]
         assert all(q >= 0 for q in tq) and sorted(tq + out_q) == list(range(n))
+        assert sorted(ta + oa) == list(range(n)) and 0 in ta and 1 in ta
+        assert oa == sorted(oa), "out-of-tile qubits must be listed in address order"
         d0 = v["dims"][0]
         assert d0["kind"] == TD_IN and d0["qlo"] == 0 and (8 << d0["bits"]) >= 16
         for d in v["dims"][1:]:
@@ -66,12 +72,12 @@ def test_tensor_copy_view_is_the_tile(n, L):
         for b in range(12):
             bit = (pos >> b) & 1
             off += bit * ss[b]
-            amp += bit << tq[b]
+            amp += bit << ta[b]
         assert sorted(off.tolist()) == list(range(4096)), "offsets are not a bijection"
         n_out = len(out_q)
         for t in rng.integers(0, (B << n_out), size=6):
             o, u = int(t) & ((1 << n_out) - 1), int(t) >> n_out
-            base = sum(((o >> k) & 1) << q for k, q in enumerate(out_q))
+            base = sum(((o >> k) & 1) << a for k, a in enumerate(oa))
             sample = min(u, B - 1)
             got = box_elements(v, n, B, sample, o)
             want = np.empty(4096, dtype=np.int64)
