@@ -92,6 +92,7 @@ struct qml_ctx {
   Bonds bonds;
   uint32_t nb[kMaxQubits] = {0}, nbhi[kMaxQubits] = {0};
   bool reupload = false;  // every layer starts with the encoding again
+  bool f64 = false;       // fp64 compute mode (qml_create_f64)
 };
 
 namespace {
@@ -100,6 +101,23 @@ namespace {
 void ensure_device(qml_ctx* c) {
   if (c->probed) return;
   c->probed = true;
+  if (c->f64) {
+    cudaDeviceProp prop;
+    int bf = 0, bb = 0;
+    DeviceGuard g(c->device);
+    if (cudaGetDeviceProperties(&prop, c->device) != cudaSuccess || pass64_setup(&bf, &bb) != cudaSuccess ||
+        bf < 1 || bb < 1) {
+      cudaGetLastError();
+      c->dev_ok = false;
+      c->grid_fwd = c->grid_bwd = c->sms;
+      return;
+    }
+    c->sms = prop.multiProcessorCount;
+    c->grid_fwd = c->sms * bf;
+    c->grid_bwd = c->sms * bb;
+    c->dev_ok = true;
+    return;
+  }
   c->smem = pass_smem_bytes(c->plan.max_slots);
   cudaDeviceProp prop;
   if (cudaGetDeviceProperties(&prop, c->device) != cudaSuccess) {
@@ -125,6 +143,11 @@ void ensure_device(qml_ctx* c) {
   c->dev_ok = true;
 }
 
+// Bytes per amplitude of a checkpoint slot.
+size_t slot_bytes(const qml_ctx* c) {
+  return c->cfg.storage == QML_STORE_FP64 ? 16 : c->cfg.storage == QML_STORE_BF16 ? 4 : 8;
+}
+
 void compute_layout(qml_ctx* c) {
   const int n = c->cfg.n_qubits, L = c->cfg.n_layers, Bm = c->cfg.max_batch;
   const long long N = 1ll << n;
@@ -144,24 +167,25 @@ void compute_layout(qml_ctx* c) {
   l.coef_inv = take(sizeof(float4) * 4 * (size_t)kMaxSlots * c->dpass.size());
   l.enc = take(sizeof(float2) * 2 * U * n);
   l.dummy = take(sizeof(float2) * (size_t)N);
-  l.exp_partial = take(sizeof(double) * expect_partial_count(Bm, n));
+  l.exp_partial = take(sizeof(double) * (c->f64 ? expect64_partial_count(Bm, n) : expect_partial_count(Bm, n)));
   size_t nparts = 0;
   for (const DevPass& p : c->dpass) nparts += (size_t)c->grid_bwd * p.nslots * 3;
-  l.partials = take(sizeof(float) * std::max<size_t>(1, nparts));
+  l.partials = take((c->f64 ? sizeof(double) : sizeof(float)) * std::max<size_t>(1, nparts));
   l.obs_groups = take(sizeof(ObsGroup) * QML_MAX_OBS_TERMS);
   l.obs_terms = take(sizeof(ObsTerm) * QML_MAX_OBS_TERMS);
-  const size_t slot_elem = c->cfg.storage == QML_STORE_BF16 ? 4 : 8;
+  const size_t slot_elem = slot_bytes(c);
   l.ckpt = take(slot_elem * (size_t)c->plan.n_ckpt * Bm * (size_t)N + 16);
   l.base_total = o;
-  l.h_psi = take(sizeof(float2) * (size_t)Bm * N);
-  l.h_lam = take(sizeof(float2) * (size_t)Bm * N);
-  l.h_x = take(sizeof(float) * (size_t)Bm * n);
-  l.h_theta = take(sizeof(float) * (size_t)L * n * 3);
-  l.h_y = take(sizeof(float) * (size_t)Bm);
-  l.h_E = take(sizeof(float) * (size_t)Bm);
-  l.h_g = take(sizeof(float) * (size_t)Bm);
-  l.h_loss = take(sizeof(float) * 4);
-  l.h_grad = take(sizeof(float) * (size_t)L * n * 3);
+  const size_t fe = c->f64 ? sizeof(double) : sizeof(float);  // real element of the host-step buffers
+  l.h_psi = take(2 * fe * (size_t)Bm * N);
+  l.h_lam = take(2 * fe * (size_t)Bm * N);
+  l.h_x = take(fe * (size_t)Bm * n);
+  l.h_theta = take(fe * (size_t)L * n * 3);
+  l.h_y = take(fe * (size_t)Bm);
+  l.h_E = take(fe * (size_t)Bm);
+  l.h_g = take(fe * (size_t)Bm);
+  l.h_loss = take(fe * 4);
+  l.h_grad = take(fe * (size_t)L * n * 3);
   l.host_total = o;
   // gradient partial offsets per pass
   long long off = 0;
@@ -206,8 +230,11 @@ T* at(qml_ctx* c, size_t off) {
   return reinterpret_cast<T*>(c->ws + off);
 }
 
-qml_status check_ready(qml_ctx* c, int B) {
+// Readiness of a context for a call with batch B; f64 is the precision the
+// call is made for (a context computes in one precision only).
+qml_status check_ready(qml_ctx* c, int B, bool f64 = false) {
   if (!c) return QML_ERR_INVALID_ARG;
+  if (c->f64 != f64) return QML_ERR_UNSUPPORTED;
   if (B < 1 || B > c->cfg.max_batch) return QML_ERR_INVALID_ARG;
   if (!c->ws) return QML_ERR_WORKSPACE;
   if (!c->dev_ok) return QML_ERR_CUDA;
@@ -289,7 +316,7 @@ cudaError_t convert_layout(qml_ctx* c, float2* buf, int B, bool to_working, cuda
       for (int q = 0; q < cb; ++q)
         if (c->plan.addr_of[q] == b) to[b] = q;  // address bit b -> its qubit
   }
-  return launch_permute_bits(buf, (long long)B << n, cb, to, c->sms * 8, s);
+  return launch_permute_bits(buf, (long long)B << n, cb, to, c->sms, s);
 }
 
 qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, float2* psi,
@@ -411,6 +438,70 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
   return cuda_status(e);
 }
 
+Pass64Args pass64_args(qml_ctx* c, const double* theta, const double* x, int B, double2* psi, double2* lam) {
+  Pass64Args a{};
+  const int n = c->cfg.n_qubits;
+  a.n = n;
+  a.B = B;
+  a.T = std::min(n, kTileBits);
+  a.n_tiles = (long long)B << (n - a.T);
+  a.theta = theta;
+  a.x = x;
+  a.psi = psi;
+  a.lam = lam;
+  a.ckpt = c->ws + c->lay.ckpt;
+  a.storage = c->cfg.storage == QML_STORE_FP64 ? 2 : c->cfg.storage == QML_STORE_BF16 ? 1 : 0;
+  a.slot_elems = (long long)c->cfg.max_batch * c->N;
+  a.partials = at<double>(c, c->lay.partials);
+  a.status = at<unsigned>(c, c->lay.status);
+  a.reupload = c->reupload ? 1 : 0;
+  for (int q = 0; q < kMaxQubits; ++q) a.nb[q] = c->nb[q], a.nbhi[q] = c->nbhi[q];
+  return a;
+}
+
+qml_status run_forward64(qml_ctx* c, const double* theta, const double* x, int B, double2* psi, double* expect,
+                         cudaStream_t s) {
+  const Pass64Args a = pass64_args(c, theta, x, B, psi, nullptr);
+  qml_ctx::Span sp{};
+  const bool timed = span_begin(c, s, &sp, false);
+  for (int p = 0; p < (int)c->dpass.size(); ++p) {
+    const DevPass& dp = c->dpass[p];
+    if (launch_pass64(false, a, dp, (int)std::min<long long>(c->grid_fwd, a.n_tiles), s) != cudaSuccess)
+      return QML_ERR_CUDA;
+    ++c->launches;
+    if (dp.ckpt >= 0) c->ckpt_batch[dp.ckpt] = B;
+  }
+  if (timed) span_end(c, s, &sp);
+  if (expect) {
+    c->launches += 2;
+    if (launch_expect64(psi, B, c->cfg.n_qubits, at<double>(c, c->lay.exp_partial), expect,
+                        at<unsigned>(c, c->lay.status), s) != cudaSuccess)
+      return QML_ERR_CUDA;
+  }
+  return QML_OK;
+}
+
+qml_status run_backward64(qml_ctx* c, const double* theta, const double* x, int B, double2* psi, double2* lam,
+                          const double* g, double* grad, cudaStream_t s) {
+  const int n = c->cfg.n_qubits, L = c->cfg.n_layers;
+  for (int m = 0; m < c->plan.n_ckpt; ++m)
+    if (c->ckpt_batch[m] != B) return QML_ERR_CKPT_MISMATCH;
+  if (launch_bwd_init64(psi, lam, g, B, n, s) != cudaSuccess) return QML_ERR_CUDA;
+  const Pass64Args a = pass64_args(c, theta, x, B, psi, lam);
+  c->launches += 2;  // lambda init, gradient reduce
+  qml_ctx::Span sp{};
+  const bool timed = span_begin(c, s, &sp, true);
+  // every block writes its partials, so the grid is the one the layout counted
+  for (int p = (int)c->dpass.size() - 1; p >= 0; --p) {
+    if (launch_pass64(true, a, c->dpass[p], c->grid_bwd, s) != cudaSuccess) return QML_ERR_CUDA;
+    ++c->launches;
+  }
+  if (timed) span_end(c, s, &sp);
+  return cuda_status(launch_grad_reduce64(at<DevPass>(c, c->lay.passes), at<int>(c, c->lay.slot_pass),
+                                          at<int>(c, c->lay.slot_index), at<double>(c, c->lay.partials),
+                                          c->grid_bwd, theta, L, n, grad, at<unsigned>(c, c->lay.status), s));
+}
+
 }  // namespace
 
 extern "C" {
@@ -432,7 +523,23 @@ const char* qml_status_str(qml_status s) {
   return "unknown status";
 }
 
+static qml_status create_ctx(const qml_config* cfg, int device, bool f64, qml_ctx** out);
+
 qml_status qml_create(const qml_config* cfg, int device, qml_ctx** out) {
+  if (cfg && cfg->storage == QML_STORE_FP64) {  // fp64 slots only for fp64 contexts
+    if (out) *out = nullptr;
+    return QML_ERR_INVALID_ARG;
+  }
+  return create_ctx(cfg, device, false, out);
+}
+
+qml_status qml_create_f64(const qml_config* cfg, int device, qml_ctx** out) {
+  return create_ctx(cfg, device, true, out);
+}
+
+int qml_precision(const qml_ctx* c) { return c ? (c->f64 ? 64 : 32) : -1; }
+
+static qml_status create_ctx(const qml_config* cfg, int device, bool f64, qml_ctx** out) {
   if (!out) return QML_ERR_INVALID_ARG;
   *out = nullptr;
   if (!cfg) return QML_ERR_INVALID_ARG;
@@ -440,11 +547,13 @@ qml_status qml_create(const qml_config* cfg, int device, qml_ctx** out) {
   if (cfg->n_layers < 1 || cfg->n_layers > 100000) return QML_ERR_INVALID_ARG;
   if (cfg->max_batch < 1 || cfg->max_batch > (1 << 20)) return QML_ERR_INVALID_ARG;
   if (cfg->ckpt_block < 0) return QML_ERR_INVALID_ARG;
-  if (cfg->storage != QML_STORE_FP32 && cfg->storage != QML_STORE_BF16) return QML_ERR_INVALID_ARG;
+  if (cfg->storage != QML_STORE_FP32 && cfg->storage != QML_STORE_BF16 && cfg->storage != QML_STORE_FP64)
+    return QML_ERR_INVALID_ARG;
   if (device < 0) return QML_ERR_INVALID_ARG;
   qml_ctx* c = new (std::nothrow) qml_ctx();
   if (!c) return QML_ERR_INVALID_ARG;
   c->cfg = *cfg;
+  c->f64 = f64;
   c->device = device;
   c->N = 1ll << cfg->n_qubits;
   std::string err = make_plan(cfg->n_qubits, cfg->n_layers, cfg->ckpt_block, &c->plan);
@@ -665,7 +774,7 @@ qml_status qml_set_entangler(qml_ctx* c, int n_bonds, const int* bonds) {
 
 qml_status qml_set_reupload(qml_ctx* c, int on) {
   if (!c) return QML_ERR_INVALID_ARG;
-  if (on && c->slow) return QML_ERR_UNSUPPORTED;  // n < 5: register layouts with batch-unit bits
+  if (on && c->slow && !c->f64) return QML_ERR_UNSUPPORTED;  // fp32, n < 5: batch-unit register bits
   c->reupload = on != 0;
   return QML_OK;
 }
@@ -795,6 +904,81 @@ int qml_debug_tile_view(const qml_ctx* c, int pass, int* out, int cap) {
   if (out)
     for (int i = 0; i < cap && i < (int)v.size(); ++i) out[i] = v[i];
   return (int)v.size();
+}
+
+
+// ------------------------------------------------------------ fp64 mode
+
+qml_status qml_forward_expect_f64(qml_ctx* c, const double* theta, const double* x, int B, double* psi,
+                                  double* expect, void* stream) {
+  qml_status st = check_ready(c, B, true);
+  if (st != QML_OK) return st;
+  if (!theta || !x || !psi || !expect || misaligned(psi, 16)) return QML_ERR_INVALID_ARG;
+  if (!c->obs_terms.empty()) return QML_ERR_UNSUPPORTED;  // fp64 mode reads out Z0
+  DeviceGuard g(c->device);
+  return run_forward64(c, theta, x, B, reinterpret_cast<double2*>(psi), expect, static_cast<cudaStream_t>(stream));
+}
+
+qml_status qml_backward_adjoint_f64(qml_ctx* c, const double* theta, const double* x, int B, double* psi,
+                                    double* lambda, const double* dLdE, double* grad, void* stream) {
+  qml_status st = check_ready(c, B, true);
+  if (st != QML_OK) return st;
+  if (!theta || !psi || !lambda || !dLdE || !grad || misaligned(psi, 16) || misaligned(lambda, 16))
+    return QML_ERR_INVALID_ARG;
+  if (psi == lambda) return QML_ERR_INVALID_ARG;
+  if (c->reupload && !x) return QML_ERR_INVALID_ARG;
+  if (!c->obs_terms.empty()) return QML_ERR_UNSUPPORTED;
+  DeviceGuard g(c->device);
+  return run_backward64(c, theta, x, B, reinterpret_cast<double2*>(psi), reinterpret_cast<double2*>(lambda),
+                        dLdE, grad, static_cast<cudaStream_t>(stream));
+}
+
+qml_status qml_loss_seed_f64(qml_ctx* c, const double* expect, const double* y, int B, double* g_out,
+                             double* loss, void* stream) {
+  qml_status st = check_ready(c, B, true);
+  if (st != QML_OK) return st;
+  if (!expect || !y) return QML_ERR_INVALID_ARG;
+  DeviceGuard g(c->device);
+  ++c->launches;
+  return cuda_status(launch_loss_seed64(expect, y, B, g_out, loss, static_cast<cudaStream_t>(stream)));
+}
+
+qml_status qml_step_host_f64(qml_ctx* c, const double* x_h, const double* theta_h, const double* y_h, int B,
+                             double* expect_h, double* loss_h, double* grad_h, void* stream) {
+  qml_status st = check_ready(c, B, true);
+  if (st != QML_OK) return st;
+  if (!x_h || !theta_h || !y_h || !grad_h) return QML_ERR_INVALID_ARG;
+  if (c->ws_bytes < c->lay.host_total) return QML_ERR_WORKSPACE;
+  if (!c->obs_terms.empty()) return QML_ERR_UNSUPPORTED;
+  DeviceGuard g(c->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int n = c->cfg.n_qubits, L = c->cfg.n_layers;
+  const Layout& l = c->lay;
+  const size_t P = (size_t)L * n * 3;
+  cudaError_t e = cudaMemcpyAsync(c->ws + l.h_x, x_h, sizeof(double) * (size_t)B * n, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->ws + l.h_theta, theta_h, sizeof(double) * P, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->ws + l.h_y, y_h, sizeof(double) * (size_t)B, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return QML_ERR_CUDA;
+  double* x = at<double>(c, l.h_x);
+  double* th = at<double>(c, l.h_theta);
+  double2* psi = at<double2>(c, l.h_psi);
+  double2* lam = at<double2>(c, l.h_lam);
+  double* E = at<double>(c, l.h_E);
+  double* gv = at<double>(c, l.h_g);
+  double* loss = at<double>(c, l.h_loss);
+  double* grad = at<double>(c, l.h_grad);
+  st = run_forward64(c, th, x, B, psi, E, s);
+  if (st != QML_OK) return st;
+  ++c->launches;
+  if (launch_loss_seed64(E, at<double>(c, l.h_y), B, gv, loss, s) != cudaSuccess) return QML_ERR_CUDA;
+  st = run_backward64(c, th, x, B, psi, lam, gv, grad, s);
+  if (st != QML_OK) return st;
+  e = cudaMemcpyAsync(grad_h, grad, sizeof(double) * P, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && expect_h)
+    e = cudaMemcpyAsync(expect_h, E, sizeof(double) * (size_t)B, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && loss_h) e = cudaMemcpyAsync(loss_h, loss, sizeof(double), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return cuda_status(e);
 }
 
 }  // extern "C"

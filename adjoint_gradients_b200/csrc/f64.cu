@@ -1,0 +1,491 @@
+// f64.cu -- fp64 compute mode: the same fused forward and adjoint backward
+// passes with complex128 state vectors (re, im doubles) and fp64 arithmetic.
+//
+// The method is the one of kernels.cu (forward gate fusion, backward gate
+// fusion that rebuilds psi next to lambda, CZ entanglers as index-parity
+// signs; Kawase, "Fast and memory-efficient classical simulation of quantum
+// machine learning via forward and backward gate fusion", [Deep-dive] sec. 1.2
+// and 1.4, sec. 3.2).  The pages state that the simulator runs in double as
+// well as single precision ([Gist-EN] Technical Summary sec. 2 and 4).
+//
+// Layout and schedule.  The passes of the fp32 schedule are reused unchanged:
+// a pass owns the 2^T (T = min(n, 12)) positions of a tile, the tile's qubits
+// are the ones the schedule gives it, and the ops are the same rotations and
+// CZ layers.  The state stays in the standard index order throughout.  A
+// block keeps one sample's tile in shared memory (psi, and lambda in the
+// backward: 72 KB per plane with one pad element per eight), and a rotation
+// op is applied in chunks of up to three qubits: each thread takes the eight
+// positions of one chunk group into registers, applies the chunk's 2x2
+// unitaries (and, backward, accumulates the three Im<lambda|P|psi> terms of
+// each qubit first), and writes them back.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "kernels.cuh"
+
+namespace qml {
+
+namespace {
+
+constexpr unsigned kErrNumeric = 1u << 6;  // QML_ERR_NUMERIC
+constexpr unsigned kErrBounds = 1u << 7;   // QML_ERR_BOUNDS
+
+constexpr int kW = kF64Warps;
+constexpr int kT = kF64Threads;
+constexpr int kPad = kTilePos + (kTilePos >> 3);  // shared positions of one plane
+
+__device__ __forceinline__ int padp(int p) { return p + (p >> 3); }
+
+// Per-block schedule data, built at kernel start.
+struct Ctx64 {
+  int T, n_out;
+  int tq[kTileBits];      // position bit -> qubit (ascending)
+  int oq[kMaxQubits];     // out-of-tile qubits (ascending)
+  int pos_of_q[kMaxQubits];
+  uint32_t off_lo[64], off_hi[64];  // index offset of position bits 0-5 / 6-11
+  uint32_t s_off[kTilePos / 32];    // entangler parity of the in-tile part of each position
+  double4 coef[kMaxSlots];          // (ar, ai, br, bi): U forward, U^dagger backward
+  double cs[kMaxQubits], sn[kMaxQubits];  // (cos, sin)(x/2) of the tile's sample
+};
+
+size_t f64_smem_bytes(bool bwd) {
+  size_t b = sizeof(double2) * (size_t)kPad * (bwd ? 2 : 1) + sizeof(Ctx64);
+  if (bwd) b += sizeof(double) * (size_t)kW * kMaxSlots * 3;
+  return b;
+}
+
+// (x, y) <- (a x + b y, -conj(b) x + conj(a) y), u = (ar, ai, br, bi)
+__device__ __forceinline__ void su2_64(double2& x, double2& y, const double4& u) {
+  const double xr = x.x, xi = x.y, yr = y.x, yi = y.y;
+  x.x = fma(u.x, xr, fma(-u.y, xi, fma(u.z, yr, -u.w * yi)));
+  x.y = fma(u.x, xi, fma(u.y, xr, fma(u.z, yi, u.w * yr)));
+  y.x = fma(-u.z, xr, fma(-u.w, xi, fma(u.x, yr, u.y * yi)));
+  y.y = fma(-u.z, xi, fma(u.w, xr, fma(u.x, yi, -u.y * yr)));
+}
+
+// Re-uploading folded into the rotation (one sample per tile): U Ry(x)
+// forward, Ry(-x) U^dagger backward (u holding U^dagger); (c, s) = (cos,
+// sin)(x/2).  U Ry(x): a' = a c + b s, b' = b c - a s.  Ry(-x) U^dagger:
+// a' = a c - conj(b) s, b' = b c + conj(a) s.
+template <bool BWD>
+__device__ __forceinline__ double4 reup64(double4 u, double c, double s) {
+  if (!BWD) return make_double4(u.x * c + u.z * s, u.y * c + u.w * s, u.z * c - u.x * s, u.w * c - u.y * s);
+  return make_double4(u.x * c - u.z * s, u.y * c + u.w * s, u.z * c + u.x * s, u.w * c - u.y * s);
+}
+
+template <typename T>
+__device__ __forceinline__ T warp_sum(T v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ double2 slot_load(const Pass64Args& a, int slot, size_t g) {
+  const size_t i = (size_t)slot * a.slot_elems + g;
+  if (a.storage == 2) return reinterpret_cast<const double2*>(a.ckpt)[i];
+  if (a.storage == 1) {
+    const __nv_bfloat162 v = reinterpret_cast<const __nv_bfloat162*>(a.ckpt)[i];
+    return make_double2((double)__bfloat162float(v.x), (double)__bfloat162float(v.y));
+  }
+  const float2 v = reinterpret_cast<const float2*>(a.ckpt)[i];
+  return make_double2((double)v.x, (double)v.y);
+}
+
+__device__ __forceinline__ void slot_store(const Pass64Args& a, int slot, size_t g, double2 v) {
+  const size_t i = (size_t)slot * a.slot_elems + g;
+  if (a.storage == 2) {
+    reinterpret_cast<double2*>(a.ckpt)[i] = v;
+  } else if (a.storage == 1) {
+    __nv_bfloat162 h;
+    h.x = __float2bfloat16_rn((float)v.x);  // fp64 -> fp32 -> bf16, both round to nearest even
+    h.y = __float2bfloat16_rn((float)v.y);
+    reinterpret_cast<__nv_bfloat162*>(a.ckpt)[i] = h;
+  } else {
+    reinterpret_cast<float2*>(a.ckpt)[i] = make_float2((float)v.x, (float)v.y);
+  }
+}
+
+// One rotation chunk of K qubits (slots s0 .. s0+K-1) over the tile.
+template <bool BWD, int K>
+__device__ void rot_chunk(const Pass64Args& a, const DevPass& P, const Ctx64& cx, double2* tp, double2* tl,
+                          double* acc, int s0, int warp, int lane) {
+  int pb[K], srt[K];
+  double4 u[K];
+#pragma unroll
+  for (int i = 0; i < K; ++i) {
+    const int q = P.slot_lq[s0 + i] % a.n;
+    pb[i] = cx.pos_of_q[q];
+    u[i] = cx.coef[s0 + i];
+    if (a.reupload) u[i] = reup64<BWD>(u[i], cx.cs[q], cx.sn[q]);
+    srt[i] = pb[i];
+  }
+#pragma unroll
+  for (int i = 1; i < K; ++i)  // ascending, for inserting the chunk bits
+#pragma unroll
+    for (int j = K - 1; j >= i; --j)
+      if (srt[j - 1] > srt[j]) {
+        const int t = srt[j];
+        srt[j] = srt[j - 1];
+        srt[j - 1] = t;
+      }
+  double sx[K], sy[K], sz[K];
+#pragma unroll
+  for (int i = 0; i < K; ++i) sx[i] = sy[i] = sz[i] = 0.0;
+  const int G = (1 << cx.T) >> K;
+  for (int g = threadIdx.x; g < G; g += kT) {
+    int p0 = g;
+#pragma unroll
+    for (int i = 0; i < K; ++i) p0 = ((p0 >> srt[i]) << (srt[i] + 1)) | (p0 & ((1 << srt[i]) - 1));
+    int pos[1 << K];
+    double2 v[1 << K], w[1 << K];
+#pragma unroll
+    for (int j = 0; j < (1 << K); ++j) {
+      int p = p0;
+#pragma unroll
+      for (int i = 0; i < K; ++i)
+        if ((j >> i) & 1) p |= 1 << pb[i];
+      pos[j] = padp(p);
+      v[j] = tp[pos[j]];
+      if (BWD) w[j] = tl[pos[j]];
+    }
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+#pragma unroll
+      for (int j = 0; j < (1 << K); ++j) {
+        if ((j >> i) & 1) continue;
+        const int jj = j | (1 << i);
+        if (BWD) {
+          // terms at the state just after this qubit's rotation (psi = v, lambda = w)
+          const double2 p0v = v[j], p1v = v[jj], l0 = w[j], l1 = w[jj];
+          sx[i] += l0.x * p1v.y - l0.y * p1v.x + l1.x * p0v.y - l1.y * p0v.x;  // Im(conj l0 p1 + conj l1 p0)
+          sy[i] += l1.x * p0v.x + l1.y * p0v.y - l0.x * p1v.x - l0.y * p1v.y;  // Re(conj l1 p0 - conj l0 p1)
+          sz[i] += l0.x * p0v.y - l0.y * p0v.x - l1.x * p1v.y + l1.y * p1v.x;  // Im(conj l0 p0 - conj l1 p1)
+          su2_64(w[j], w[jj], u[i]);
+        }
+        su2_64(v[j], v[jj], u[i]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < (1 << K); ++j) {
+      tp[pos[j]] = v[j];
+      if (BWD) tl[pos[j]] = w[j];
+    }
+  }
+  if (BWD) {
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+      const double rx = warp_sum(sx[i]), ry = warp_sum(sy[i]), rz = warp_sum(sz[i]);
+      if (lane == 0) {
+        double* d = acc + ((size_t)warp * kMaxSlots + s0 + i) * 3;
+        d[0] += rx;
+        d[1] += ry;
+        d[2] += rz;
+      }
+    }
+  }
+}
+
+template <bool BWD>
+__global__ void __launch_bounds__(kT) pass64_kernel(const Pass64Args a, const __grid_constant__ DevPass P) {
+  extern __shared__ __align__(16) unsigned char smem64[];
+  double2* tp = reinterpret_cast<double2*>(smem64);
+  double2* tl = tp + kPad;
+  Ctx64& cx = *reinterpret_cast<Ctx64*>(smem64 + sizeof(double2) * kPad * (BWD ? 2 : 1));
+  double* acc = reinterpret_cast<double*>(reinterpret_cast<unsigned char*>(&cx) + sizeof(Ctx64));
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n = a.n;
+
+  if (tid == 0) {
+    uint32_t inmask = 0;
+    for (int b = 0; b < kTileBits; ++b)
+      if (P.tile_q[b] >= 0 && P.tile_q[b] < n) inmask |= 1u << P.tile_q[b];
+    int T = 0, no = 0;
+    for (int q = 0; q < n; ++q) {
+      cx.pos_of_q[q] = -1;
+      if ((inmask >> q) & 1u) {
+        cx.pos_of_q[q] = T;
+        cx.tq[T++] = q;
+      } else {
+        cx.oq[no++] = q;
+      }
+    }
+    cx.T = T;
+    cx.n_out = no;
+  }
+  // gate coefficients of the pass's slots: U = Rz Ry Rx, in fp64
+  for (int s = tid; s < P.nslots; s += kT) {
+    const int lq = P.slot_lq[s];
+    double sa, ca, sb, cb, sg, cg;
+    sincos(0.5 * a.theta[lq * 3 + 0], &sa, &ca);
+    sincos(0.5 * a.theta[lq * 3 + 1], &sb, &cb);
+    sincos(0.5 * a.theta[lq * 3 + 2], &sg, &cg);
+    // (Ry Rx)[0][0] = cb ca + i sb sa, (Ry Rx)[0][1] = -sb ca - i cb sa; Rz row 0 is e^{-i g/2}
+    const double p_re = cb * ca, p_im = sb * sa, q_re = -sb * ca, q_im = -cb * sa;
+    const double ar = cg * p_re + sg * p_im, ai = cg * p_im - sg * p_re;
+    const double br = cg * q_re + sg * q_im, bi = cg * q_im - sg * q_re;
+    cx.coef[s] = BWD ? make_double4(ar, -ai, -br, -bi) : make_double4(ar, ai, br, bi);  // U^dagger: (conj a, -b)
+  }
+  if (BWD)
+    for (int i = tid; i < kW * kMaxSlots * 3; i += kT) acc[i] = 0.0;
+  __syncthreads();
+  const int T = cx.T, P2 = 1 << T, no = cx.n_out;
+  if (T != a.T) {  // the schedule and the host disagree on the tile: touch nothing
+    if (tid == 0) atomicOr(a.status, kErrBounds);
+    return;
+  }
+  for (int i = tid; i < 64; i += kT) {
+    uint32_t lo = 0, hi = 0;
+    for (int k = 0; k < 6; ++k)
+      if ((i >> k) & 1) {
+        if (k < T) lo |= 1u << cx.tq[k];
+        if (k + 6 < T) hi |= 1u << cx.tq[k + 6];
+      }
+    cx.off_lo[i] = lo;
+    cx.off_hi[i] = hi;
+  }
+  __syncthreads();
+  // entangler parity of the in-tile part of every position
+  for (int v0 = warp * 32; v0 < kTilePos; v0 += kT) {
+    const int v = v0 + lane;
+    const uint32_t i = cx.off_lo[v & 63] | cx.off_hi[(v >> 6) & 63];
+    uint32_t par = 0;
+    for (uint32_t r = i; r; r &= r - 1u) par ^= (uint32_t)__popc(i & a.nbhi[__ffs(r) - 1]);
+    const uint32_t bits = __ballot_sync(0xffffffffu, v < P2 && (par & 1u));
+    if (lane == 0) cx.s_off[v0 >> 5] = bits;
+  }
+  __syncthreads();
+
+  const bool enc = (!BWD && P.gen) || a.reupload;
+  for (long long t = blockIdx.x; t < a.n_tiles; t += gridDim.x) {
+    const int b = (int)(t >> no);
+    const uint32_t o = (uint32_t)(t & ((1ll << no) - 1));
+    uint32_t base = 0;
+    for (int k = 0; k < no; ++k)
+      if ((o >> k) & 1u) base |= 1u << cx.oq[k];
+    const size_t gbase = ((size_t)b << n) + base;
+    if (enc) {
+      for (int q = tid; q < n; q += kT) sincos(0.5 * a.x[(size_t)b * n + q], &cx.sn[q], &cx.cs[q]);
+      __syncthreads();
+    }
+    // entangler parity of the out-of-tile part and of its bonds into the tile
+    uint32_t s_base = 0, cm = 0;
+    for (uint32_t r = base; r; r &= r - 1u) s_base ^= (uint32_t)__popc(base & a.nbhi[__ffs(r) - 1]);
+    for (int k = 0; k < T; ++k) cm |= ((uint32_t)__popc(base & a.nb[cx.tq[k]]) & 1u) << k;
+    s_base &= 1u;
+
+    for (int v = tid; v < P2; v += kT) {
+      const uint32_t idx = cx.off_lo[v & 63] | cx.off_hi[(v >> 6) & 63];
+      const size_t g = gbase + idx;
+      double2 pv;
+      if (!BWD && P.gen) {
+        const uint32_t i = base | idx;
+        double r = 1.0;
+        for (int q = 0; q < n; ++q) r *= ((i >> q) & 1u) ? cx.sn[q] : cx.cs[q];
+        pv = make_double2(r, 0.0);
+      } else if (BWD && P.ckpt >= 0) {
+        pv = slot_load(a, P.ckpt, g);  // the checkpoint replaces the uncomputed state
+      } else {
+        pv = a.psi[g];
+      }
+      tp[padp(v)] = pv;
+      if (BWD) tl[padp(v)] = a.lam[g];
+    }
+    __syncthreads();
+
+    for (int k = 0; k < P.nops; ++k) {
+      const DevOp op = P.ops[BWD ? P.nops - 1 - k : k];
+      if (op.kind == OP_ROT) {
+        const int m = __popc((unsigned)op.b);
+        for (int c0 = 0; c0 < m; c0 += 3) {
+          const int kk = min(3, m - c0);
+          if (kk == 3) rot_chunk<BWD, 3>(a, P, cx, tp, tl, acc, op.d + c0, warp, lane);
+          else if (kk == 2) rot_chunk<BWD, 2>(a, P, cx, tp, tl, acc, op.d + c0, warp, lane);
+          else rot_chunk<BWD, 1>(a, P, cx, tp, tl, acc, op.d + c0, warp, lane);
+          __syncthreads();
+        }
+      } else if (op.kind == OP_CZ) {
+        for (int v = tid; v < P2; v += kT) {
+          const uint32_t par = s_base ^ ((cx.s_off[v >> 5] >> (v & 31)) & 1u) ^ ((uint32_t)__popc(v & cm) & 1u);
+          if (par) {
+            const int p = padp(v);
+            tp[p] = make_double2(-tp[p].x, -tp[p].y);
+            if (BWD) tl[p] = make_double2(-tl[p].x, -tl[p].y);
+          }
+        }
+        __syncthreads();
+      }
+    }
+
+    if (!BWD || !P.gen) {
+      for (int v = tid; v < P2; v += kT) {
+        const size_t g = gbase + (cx.off_lo[v & 63] | cx.off_hi[(v >> 6) & 63]);
+        const double2 pv = tp[padp(v)];
+        if (!BWD && P.ckpt >= 0) slot_store(a, P.ckpt, g, pv);
+        a.psi[g] = pv;
+        if (BWD) a.lam[g] = tl[padp(v)];
+      }
+    }
+    __syncthreads();  // the tile buffers are reused by the next tile
+  }
+  if (BWD) {
+    const int nacc = P.nslots * 3;
+    for (int i = tid; i < nacc; i += kT) {
+      double s = 0.0;
+      for (int w = 0; w < kW; ++w) s += acc[((size_t)w * kMaxSlots) * 3 + i];  // fixed warp order
+      a.partials[P.partial_off + (long long)blockIdx.x * nacc + i] = s;
+    }
+  }
+}
+
+// lambda = g[b] Z0 psi (separate buffer; psi unchanged).
+__global__ void bwd_init64_kernel(const double2* psi, double2* lam, const double* g, int n, long long tot) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= tot) return;
+  const double gs = (idx & 1) ? -g[idx >> n] : g[idx >> n];
+  const double2 v = psi[idx];
+  lam[idx] = make_double2(gs * v.x, gs * v.y);
+}
+
+constexpr int kExp64Threads = 256;
+constexpr int kExp64ChunkLog = 16;
+
+__global__ void expect64_partial_kernel(const double2* psi, int n, double* partial) {
+  const long long N = 1ll << n;
+  const int chunks = (int)((N + (1ll << kExp64ChunkLog) - 1) >> kExp64ChunkLog);
+  const int b = blockIdx.y, c = blockIdx.x;
+  const long long lo = (long long)c << kExp64ChunkLog;
+  const long long hi = min(N, lo + (1ll << kExp64ChunkLog));
+  const double2* p = psi + (size_t)b * N;
+  double s = 0.0;
+  for (long long i = lo + threadIdx.x; i < hi; i += kExp64Threads) {
+    const double2 v = p[i];
+    const double m = v.x * v.x + v.y * v.y;
+    s += (i & 1) ? -m : m;
+  }
+  __shared__ double red[kExp64Threads];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = kExp64Threads / 2; w; w >>= 1) {
+    if ((int)threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) partial[(size_t)b * chunks + c] = red[0];
+}
+
+__global__ void expect64_final_kernel(const double* partial, int chunks, int B, double* E, unsigned* status) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  double s = 0.0;
+  for (int c = 0; c < chunks; ++c) s += partial[(size_t)b * chunks + c];
+  E[b] = s;
+  if (!isfinite(s) && status) atomicOr(status, kErrNumeric);
+}
+
+__global__ void grad_reduce64_kernel(const DevPass* passes, const int* slot_pass, const int* slot_index,
+                                     const double* partials, int grid, const double* theta, int L, int n,
+                                     double* grad, unsigned* status) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= L * n) return;
+  const int p = slot_pass[idx], s = slot_index[idx];
+  const DevPass& ps = passes[p];
+  const int stride = ps.nslots * 3;
+  const double* base = partials + ps.partial_off + s * 3;
+  double sx = 0.0, sy = 0.0, sz = 0.0;
+  for (int c = 0; c < grid; ++c) {
+    sx += base[(size_t)c * stride + 0];
+    sy += base[(size_t)c * stride + 1];
+    sz += base[(size_t)c * stride + 2];
+  }
+  // (s_x, s_y, s_z) are Im<lambda|P|psi> at the rotation's output; the angle
+  // gradients take X and Y back through the Rz and Ry that follow them
+  double sb, cb, sg, cg;
+  sincos(theta[idx * 3 + 1], &sb, &cb);
+  sincos(theta[idx * 3 + 2], &sg, &cg);
+  const double gz = sz;
+  const double gy = cg * sy - sg * sx;
+  const double gx = cb * (cg * sx + sg * sy) - sb * sz;
+  grad[idx * 3 + 0] = gx;
+  grad[idx * 3 + 1] = gy;
+  grad[idx * 3 + 2] = gz;
+  if (!(isfinite(gx) && isfinite(gy) && isfinite(gz)) && status) atomicOr(status, kErrNumeric);
+}
+
+// g[b] = 2 (E[b] - y[b]) / B, loss = mean (E - y)^2 (fixed-order sum).
+__global__ void loss_seed64_kernel(const double* E, const double* y, int B, double* g, double* loss) {
+  __shared__ double red[256];
+  double s = 0.0;
+  for (int b = threadIdx.x; b < B; b += 256) {
+    const double d = E[b] - y[b];
+    if (g) g[b] = 2.0 * d / B;
+    s += d * d;
+  }
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = 128; w; w >>= 1) {
+    if ((int)threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0 && loss) loss[0] = red[0] / B;
+}
+
+}  // namespace
+
+size_t pass64_smem_bytes(bool backward) { return f64_smem_bytes(backward); }
+
+cudaError_t pass64_setup(int* blocks_fwd, int* blocks_bwd) {
+  cudaError_t e = cudaFuncSetAttribute(pass64_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)f64_smem_bytes(false));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(pass64_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)f64_smem_bytes(true));
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_fwd, pass64_kernel<false>, kT, f64_smem_bytes(false));
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_bwd, pass64_kernel<true>, kT, f64_smem_bytes(true));
+  return e;
+}
+
+cudaError_t launch_pass64(bool backward, const Pass64Args& a, const DevPass& p, int grid, cudaStream_t s) {
+  if (backward) pass64_kernel<true><<<grid, kT, f64_smem_bytes(true), s>>>(a, p);
+  else pass64_kernel<false><<<grid, kT, f64_smem_bytes(false), s>>>(a, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_init64(const double2* psi, double2* lam, const double* g, int B, int n, cudaStream_t s) {
+  const long long tot = (long long)B << n;
+  bwd_init64_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(psi, lam, g, n, tot);
+  return cudaGetLastError();
+}
+
+size_t expect64_partial_count(int B, int n) {
+  const long long N = 1ll << n;
+  return (size_t)B * (size_t)((N + (1ll << kExp64ChunkLog) - 1) >> kExp64ChunkLog);
+}
+
+cudaError_t launch_expect64(const double2* psi, int B, int n, double* partial, double* E, unsigned* status,
+                            cudaStream_t s) {
+  const long long N = 1ll << n;
+  const int chunks = (int)((N + (1ll << kExp64ChunkLog) - 1) >> kExp64ChunkLog);
+  expect64_partial_kernel<<<dim3(chunks, B), kExp64Threads, 0, s>>>(psi, n, partial);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  expect64_final_kernel<<<(B + 127) / 128, 128, 0, s>>>(partial, chunks, B, E, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_grad_reduce64(const DevPass* passes, const int* slot_pass, const int* slot_index,
+                                 const double* partials, int grid, const double* theta, int L, int n, double* grad,
+                                 unsigned* status, cudaStream_t s) {
+  const int tot = L * n;
+  grad_reduce64_kernel<<<(tot + 127) / 128, 128, 0, s>>>(passes, slot_pass, slot_index, partials, grid, theta, L,
+                                                          n, grad, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_loss_seed64(const double* E, const double* y, int B, double* g, double* loss, cudaStream_t s) {
+  loss_seed64_kernel<<<1, 256, 0, s>>>(E, y, B, g, loss);
+  return cudaGetLastError();
+}
+
+}  // namespace qml

@@ -92,14 +92,33 @@ __device__ __forceinline__ void su2(float2& xr, float2& xi, float2& yr, float2& 
   yi = __ffma2_rn(c.ar, yi, o1i);
 }
 
-template <int K>
-__device__ __forceinline__ void rot_fwd(float2 (&re)[kPos], float2 (&im)[kPos], const Coef& c) {
+// cf(j) gives the coefficients for register pair (j, j | 1 << K).
+template <int K, class CF>
+__device__ __forceinline__ void rot_fwd(float2 (&re)[kPos], float2 (&im)[kPos], const CF& cf) {
 #pragma unroll
   for (int j = 0; j < kPos; ++j)
-    if (!(j & (1 << K))) su2(re[j], im[j], re[j | (1 << K)], im[j | (1 << K)], c);
+    if (!(j & (1 << K))) su2(re[j], im[j], re[j | (1 << K)], im[j | (1 << K)], cf(j));
 }
 
+// The same coefficients for every register pair.
+struct SameCoef {
+  Coef c;
+  __device__ __forceinline__ Coef operator()(int) const { return c; }
+};
+
 __device__ __forceinline__ float2 swap2(float2 v) { return make_float2(v.y, v.x); }
+
+template <class CF>
+__device__ __forceinline__ void rot_fwd_k(int k, float2 (&re)[kPos], float2 (&im)[kPos], const CF& cf) {
+  static_assert(kRegBits == 5, "dispatch below covers five register bits");
+  switch (k) {
+    case 0: rot_fwd<0>(re, im, cf); break;
+    case 1: rot_fwd<1>(re, im, cf); break;
+    case 2: rot_fwd<2>(re, im, cf); break;
+    case 3: rot_fwd<3>(re, im, cf); break;
+    default: rot_fwd<4>(re, im, cf); break;
+  }
+}
 
 // Gradient terms of one qubit at the state just after its fused rotation, then
 // U^dagger on psi and lambda.  With psi in lane x and lambda in lane y:
@@ -109,42 +128,13 @@ __device__ __forceinline__ float2 swap2(float2 v) { return make_float2(v.y, v.x)
 // The products lambda * psi are formed as packed products of a pair with a
 // lane-swapped pair, e.g. (p0r, l0r) * (l0i, p0i) = (p0r l0i, l0r p0i), whose
 // lane difference is Im(conj(l0) p0); the differences are taken at the end.
-template <int K>
-__device__ __forceinline__ float3 rot_bwd(float2 (&re)[kPos], float2 (&im)[kPos], const Coef& c) {
-  float2 ax = make_float2(0.f, 0.f), ay = ax, az0 = ax, az1 = ax;
-#pragma unroll
-  for (int j = 0; j < kPos; ++j) {
-    if (j & (1 << K)) continue;
-    const int jj = j | (1 << K);
-    const float2 si0 = swap2(im[j]), si1 = swap2(im[jj]), sr1 = swap2(re[jj]);
-    az0 = __ffma2_rn(re[j], si0, az0);   // y - x: Im(conj l0 p0)
-    az1 = __ffma2_rn(re[jj], si1, az1);  // y - x: Im(conj l1 p1)
-    ax = __ffma2_rn(re[j], si1, ax);     // y - x: l0r p1i - p0r l1i
-    ax = __ffma2_rn(re[jj], si0, ax);    // y - x: l1r p0i - p1r l0i
-    ay = __ffma2_rn(re[j], sr1, ay);     // x - y: p0r l1r - l0r p1r
-    ay = __ffma2_rn(im[j], si1, ay);     // x - y: p0i l1i - l0i p1i
-    su2(re[j], im[j], re[jj], im[jj], c);
-  }
-  return make_float3(ax.y - ax.x, ay.x - ay.y, (az0.y - az0.x) - (az1.y - az1.x));
-}
-
-__device__ __forceinline__ void rot_fwd_k(int k, float2 (&re)[kPos], float2 (&im)[kPos], const Coef& c) {
-  static_assert(kRegBits == 5, "dispatch below covers five register bits");
-  switch (k) {
-    case 0: rot_fwd<0>(re, im, c); break;
-    case 1: rot_fwd<1>(re, im, c); break;
-    case 2: rot_fwd<2>(re, im, c); break;
-    case 3: rot_fwd<3>(re, im, c); break;
-    default: rot_fwd<4>(re, im, c); break;
-  }
-}
-
-// rot_bwd<K> that also finishes the warp sum of the previous qubit's terms
+// The same call also finishes the warp sum of the previous qubit's terms
 // (pv): the shuffle steps of warp_reduce3 are spread over the pair loop so
 // that their latency hides behind this qubit's FMAs.  *r_prev receives the
-// sum as warp_reduce3 returns it.
-template <int K>
-__device__ __forceinline__ float3 rot_bwd_red(float2 (&re)[kPos], float2 (&im)[kPos], const Coef& c, float3 pv,
+// sum as warp_reduce3 returns it.  cf(j) gives the coefficients of U^dagger
+// for register pair (j, j | 1 << K).
+template <int K, class CF>
+__device__ __forceinline__ float3 rot_bwd_red(float2 (&re)[kPos], float2 (&im)[kPos], const CF& cf, float3 pv,
                                               int lane, float* r_prev) {
   const bool h16 = (lane & 16) != 0, h8 = (lane & 8) != 0;
   float k0 = h16 ? pv.z : pv.x, k1 = h16 ? 0.f : pv.y;
@@ -170,26 +160,27 @@ __device__ __forceinline__ float3 rot_bwd_red(float2 (&re)[kPos], float2 (&im)[k
     }
     const int jj = j | (1 << K);
     const float2 si0 = swap2(im[j]), si1 = swap2(im[jj]), sr1 = swap2(re[jj]);
-    az0 = __ffma2_rn(re[j], si0, az0);
-    az1 = __ffma2_rn(re[jj], si1, az1);
-    ax = __ffma2_rn(re[j], si1, ax);
-    ax = __ffma2_rn(re[jj], si0, ax);
-    ay = __ffma2_rn(re[j], sr1, ay);
-    ay = __ffma2_rn(im[j], si1, ay);
-    su2(re[j], im[j], re[jj], im[jj], c);
+    az0 = __ffma2_rn(re[j], si0, az0);   // y - x: Im(conj l0 p0)
+    az1 = __ffma2_rn(re[jj], si1, az1);  // y - x: Im(conj l1 p1)
+    ax = __ffma2_rn(re[j], si1, ax);     // y - x: l0r p1i - p0r l1i
+    ax = __ffma2_rn(re[jj], si0, ax);    // y - x: l1r p0i - p1r l0i
+    ay = __ffma2_rn(re[j], sr1, ay);     // x - y: p0r l1r - l0r p1r
+    ay = __ffma2_rn(im[j], si1, ay);     // x - y: p0i l1i - l0i p1i
+    su2(re[j], im[j], re[jj], im[jj], cf(j));
   }
   *r_prev = v;
   return make_float3(ax.y - ax.x, ay.x - ay.y, (az0.y - az0.x) - (az1.y - az1.x));
 }
 
-__device__ __forceinline__ float3 rot_bwd_red_k(int k, float2 (&re)[kPos], float2 (&im)[kPos], const Coef& c,
+template <class CF>
+__device__ __forceinline__ float3 rot_bwd_red_k(int k, float2 (&re)[kPos], float2 (&im)[kPos], const CF& cf,
                                                 float3 pv, int lane, float* r_prev) {
   switch (k) {
-    case 0: return rot_bwd_red<0>(re, im, c, pv, lane, r_prev);
-    case 1: return rot_bwd_red<1>(re, im, c, pv, lane, r_prev);
-    case 2: return rot_bwd_red<2>(re, im, c, pv, lane, r_prev);
-    case 3: return rot_bwd_red<3>(re, im, c, pv, lane, r_prev);
-    default: return rot_bwd_red<4>(re, im, c, pv, lane, r_prev);
+    case 0: return rot_bwd_red<0>(re, im, cf, pv, lane, r_prev);
+    case 1: return rot_bwd_red<1>(re, im, cf, pv, lane, r_prev);
+    case 2: return rot_bwd_red<2>(re, im, cf, pv, lane, r_prev);
+    case 3: return rot_bwd_red<3>(re, im, cf, pv, lane, r_prev);
+    default: return rot_bwd_red<4>(re, im, cf, pv, lane, r_prev);
   }
 }
 
@@ -212,50 +203,56 @@ __device__ __forceinline__ void enc_coef(const PassArgs& a, uint32_t unit, int q
   }
 }
 
+// Data re-uploading folded into the layer's rotation: the SU(2) coefficients
+// of U Ry(x) (forward, c holding U) or of Ry(-x) U^dagger (backward, c holding
+// U^dagger), with (cs, sn) = (cos, sin)(x/2) per lane.  With U = [[a, b],
+// [-conj b, conj a]]: U Ry(x) has a' = a cs + b sn, b' = b cs - a sn, and
+// Ry(-x) U^dagger has a' = a cs - conj(b) sn, b' = b cs + conj(a) sn.
 template <bool BWD>
-__device__ __forceinline__ void enc_pair(float2& r0, float2& i0, float2& r1, float2& i1, float2 c, float2 s) {
-  const float2 ns = make_float2(-s.x, -s.y);
-  const float2 a0 = BWD ? s : ns, a1 = BWD ? ns : s;
-  const float2 nr0 = __ffma2_rn(a0, r1, __fmul2_rn(c, r0));
-  const float2 ni0 = __ffma2_rn(a0, i1, __fmul2_rn(c, i0));
-  const float2 nr1 = __ffma2_rn(a1, r0, __fmul2_rn(c, r1));
-  const float2 ni1 = __ffma2_rn(a1, i0, __fmul2_rn(c, i1));
-  r0 = nr0, i0 = ni0, r1 = nr1, i1 = ni1;
+__device__ __forceinline__ Coef reup_coef(const Coef& c, float2 cs, float2 sn) {
+  const float2 nsn = make_float2(-sn.x, -sn.y);
+  Coef m;
+  if (!BWD) {
+    m.ar = __ffma2_rn(c.br, sn, __fmul2_rn(c.ar, cs));
+    m.ai = __ffma2_rn(c.bi, sn, __fmul2_rn(c.ai, cs));
+    m.nai = __ffma2_rn(c.nbi, sn, __fmul2_rn(c.nai, cs));
+    m.br = __ffma2_rn(c.ar, nsn, __fmul2_rn(c.br, cs));
+    m.bi = __ffma2_rn(c.nai, sn, __fmul2_rn(c.bi, cs));
+    m.nbi = __ffma2_rn(c.ai, sn, __fmul2_rn(c.nbi, cs));
+    m.nbr = __ffma2_rn(c.ar, sn, __fmul2_rn(c.nbr, cs));
+  } else {
+    m.ar = __ffma2_rn(c.nbr, sn, __fmul2_rn(c.ar, cs));
+    m.ai = __ffma2_rn(c.bi, sn, __fmul2_rn(c.ai, cs));
+    m.nai = __ffma2_rn(c.nbi, sn, __fmul2_rn(c.nai, cs));
+    m.br = __ffma2_rn(c.ar, sn, __fmul2_rn(c.br, cs));
+    m.bi = __ffma2_rn(c.nai, sn, __fmul2_rn(c.bi, cs));
+    m.nbi = __ffma2_rn(c.ai, sn, __fmul2_rn(c.nbi, cs));
+    m.nbr = __ffma2_rn(c.ar, nsn, __fmul2_rn(c.nbr, cs));
+  }
+  return m;
 }
 
-// unit: the thread's batch unit; mu[k]: unit increment of register bit k (0
-// unless a register bit is a batch-unit bit, which happens only for n < 10)
-template <bool BWD, int K>
-__device__ __forceinline__ void enc_rot(float2 (&re)[kPos], float2 (&im)[kPos], const PassArgs& a, int q,
-                                        uint32_t unit, const uint32_t (&mu)[kRegBits]) {
-  const bool uni = (mu[0] | mu[1] | mu[2] | mu[3] | mu[4]) == 0u;
-  float2 c, s;
-  if (uni) enc_coef<BWD>(a, unit, q, &c, &s);
-#pragma unroll
-  for (int j = 0; j < kPos; ++j) {
-    if (j & (1 << K)) continue;
-    if (!uni) {
-      uint32_t du = 0;
-#pragma unroll
-      for (int k = 0; k < kRegBits; ++k)
-        if ((j >> k) & 1) du += mu[k];
-      enc_coef<BWD>(a, unit + du, q, &c, &s);
-    }
-    enc_pair<BWD>(re[j], im[j], re[j | (1 << K)], im[j | (1 << K)], c, s);
-  }
-}
-
+// U Ry(x) (forward) or Ry(-x) U^dagger (backward) per register pair, for
+// register bits that also span batch units: pair j takes the coefficients of
+// its own unit (unit plus the mu[k] of its set bits; mu[k] is 0 unless
+// register bit k is a batch-unit bit, which happens only for n < 10).
 template <bool BWD>
-__device__ __forceinline__ void enc_rot_k(int k, float2 (&re)[kPos], float2 (&im)[kPos], const PassArgs& a, int q,
-                                          uint32_t unit, const uint32_t (&mu)[kRegBits]) {
-  switch (k) {
-    case 0: enc_rot<BWD, 0>(re, im, a, q, unit, mu); break;
-    case 1: enc_rot<BWD, 1>(re, im, a, q, unit, mu); break;
-    case 2: enc_rot<BWD, 2>(re, im, a, q, unit, mu); break;
-    case 3: enc_rot<BWD, 3>(re, im, a, q, unit, mu); break;
-    default: enc_rot<BWD, 4>(re, im, a, q, unit, mu); break;
+struct ReupPairCoef {
+  Coef c;
+  const PassArgs& a;
+  int q;
+  uint32_t unit;
+  const uint32_t (&mu)[kRegBits];
+  __device__ __forceinline__ Coef operator()(int j) const {
+    uint32_t du = 0;
+#pragma unroll
+    for (int k = 0; k < kRegBits; ++k)
+      if ((j >> k) & 1) du += mu[k];
+    float2 cs, sn;
+    enc_coef<BWD>(a, unit + du, q, &cs, &sn);
+    return reup_coef<BWD>(c, cs, sn);
   }
-}
+};
 
 // Sum (a, b, c) over the warp with six shuffles; afterwards lanes 0, 8 and 16
 // hold the totals of a, b and c.
@@ -815,9 +812,13 @@ __device__ __forceinline__ void cz_thread_terms(BlockCtx& bc, const DevPass& Pp,
 // MODE 0: a memory layout has a batch-unit register bit (n < 5), generic
 // addressing.  MODE 1: tiles are loaded by the threads (the next tile with
 // cp.async).  MODE 2: tiles are loaded by tensor copies through tm0 / tm1.
-// RE: data re-uploading (every layer starts with the encoding again).
+// RE: data re-uploading (every layer starts with the encoding again), folded
+// into the layer's rotations.  RE 1: the tile holds no batch-unit bit, so each
+// thread's amplitudes belong to one batch unit and each rotation takes one set
+// of coefficients.  RE 2: tiles with batch-unit bits (n < 12), coefficients
+// per register pair.
 
-template <bool BWD, int MODE, int V, bool RE>
+template <bool BWD, int MODE, int V, int RE>
 __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     pass_kernel(const PassArgs a, const __grid_constant__ DevPass P, const __grid_constant__ CUtensorMap tm0,
                 const __grid_constant__ CUtensorMap tm1) {
@@ -922,17 +923,27 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
           exchange<V>(op.a, op.b, re, im, tile, tid);
         } else if (op.kind == OP_ROT) {
           int slot = op.d;
-          if (RE) {  // the encoding again before the layer's rotations
+          if (RE != 0) {  // the encoding again, folded into the layer's rotations
             uint32_t unit, mu[kRegBits];
             int rq[kRegBits];
             unit_maps<V>(op.a, *bc, tid, unit_base, &unit, mu, rq);
 #pragma unroll
             for (int k = 0; k < kRegBits; ++k)
-              if ((op.b >> k) & 1) enc_rot_k<false>(k, re, im, a, rq[k], unit, mu);
-          }
+              if ((op.b >> k) & 1) {
+                const Coef c = const_coef(region, slot++);
+                if (RE == 1) {
+                  float2 cs, sn;
+                  enc_coef<false>(a, unit, rq[k], &cs, &sn);
+                  rot_fwd_k(k, re, im, SameCoef{reup_coef<false>(c, cs, sn)});
+                } else {
+                  rot_fwd_k(k, re, im, ReupPairCoef<false>{c, a, rq[k], unit, mu});
+                }
+              }
+          } else {
 #pragma unroll
-          for (int k = 0; k < kRegBits; ++k)
-            if ((op.b >> k) & 1) rot_fwd_k(k, re, im, const_coef(region, slot++));
+            for (int k = 0; k < kRegBits; ++k)
+              if ((op.b >> k) & 1) rot_fwd_k(k, re, im, SameCoef{const_coef(region, slot++)});
+          }
         } else if (op.kind == OP_CZ) {
           cz_op<V>(op.a, re, im, *bc, P, tid, base_q, s_o);
         }
@@ -955,11 +966,25 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
           // each rotation finishes the warp sum of the previous one
           int slot = op.d, pslot = -1;
           float3 pend = make_float3(0.f, 0.f, 0.f);
+          // re-uploading: Ry(-x) of the layer's encoding joins U^dagger
+          uint32_t unit = 0, mu[kRegBits] = {0u, 0u, 0u, 0u, 0u};
+          int rq[kRegBits] = {0, 0, 0, 0, 0};
+          if (RE != 0) unit_maps<V>(op.a, *bc, tid, unit_base, &unit, mu, rq);
 #pragma unroll
           for (int k = 0; k < kRegBits; ++k)
             if ((op.b >> k) & 1) {
               float r;
-              const float3 v = rot_bwd_red_k(k, re, im, const_coef(region, slot), pend, lane, &r);
+              float3 v;
+              const Coef c = const_coef(region, slot);
+              if (RE == 0) {
+                v = rot_bwd_red_k(k, re, im, SameCoef{c}, pend, lane, &r);
+              } else if (RE == 1) {
+                float2 cs, sn;
+                enc_coef<true>(a, unit, rq[k], &cs, &sn);
+                v = rot_bwd_red_k(k, re, im, SameCoef{reup_coef<true>(c, cs, sn)}, pend, lane, &r);
+              } else {
+                v = rot_bwd_red_k(k, re, im, ReupPairCoef<true>{c, a, rq[k], unit, mu}, pend, lane, &r);
+              }
               if (pslot >= 0 && (lane & 7) == 0 && lane < 24) acc[warp * nacc + pslot * 3 + (lane >> 3)] += r;
               pend = v;
               pslot = slot++;
@@ -967,14 +992,6 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
           if (pslot >= 0) {
             const float r = warp_reduce3(pend.x, pend.y, pend.z, lane);
             if ((lane & 7) == 0 && lane < 24) acc[warp * nacc + pslot * 3 + (lane >> 3)] += r;
-          }
-          if (RE) {  // un-apply the layer's encoding
-            uint32_t unit, mu[kRegBits];
-            int rq[kRegBits];
-            unit_maps<V>(op.a, *bc, tid, unit_base, &unit, mu, rq);
-#pragma unroll
-            for (int k = 0; k < kRegBits; ++k)
-              if ((op.b >> k) & 1) enc_rot_k<true>(k, re, im, a, rq[k], unit, mu);
           }
         } else if (op.kind == OP_CZ) {
           cz_op<V>(op.a, re, im, *bc, P, tid, base_q, s_o);
@@ -1226,31 +1243,6 @@ __global__ void planes_kernel(float2* psi, float2* lam, long long count) {
   lam[idx] = make_float2(v.y, l.y);
 }
 
-// In-place permutation of the low index bits of every aligned chunk of
-// 2^cb elements: element j of a chunk moves to position sum_b j_b << to[b].
-// A chunk maps onto itself, so one block per chunk makes it race-free.
-struct BitPerm {
-  int cb;
-  int to[kTileBits];
-};
-
-__global__ void permute_bits_kernel(float2* buf, long long chunks, const BitPerm perm) {
-  extern __shared__ float2 chunk[];
-  const int size = 1 << perm.cb;
-  for (long long c = blockIdx.x; c < chunks; c += gridDim.x) {
-    float2* base = buf + (size_t)c * size;
-    for (int j = threadIdx.x; j < size; j += blockDim.x) chunk[j] = base[j];
-    __syncthreads();
-    for (int j = threadIdx.x; j < size; j += blockDim.x) {
-      // the element that lands at j comes from src with j = sum_b src_b << to[b]
-      int src = 0;
-      for (int b = 0; b < perm.cb; ++b) src |= ((j >> perm.to[b]) & 1) << b;
-      base[j] = chunk[src];
-    }
-    __syncthreads();
-  }
-}
-
 __global__ void bwd_init_kernel(float2* psi, float2* lam, const float* g, int B, int n) {
   const long long N = 1ll << n;
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -1298,10 +1290,10 @@ size_t pass_smem_bytes(int max_slots) {
 }
 
 #define QML_FOR_EACH_PASS_KERNEL(X)                                                                          \
-  X(false, 0, 0, false) X(true, 0, 0, false) X(false, 1, 0, false) X(true, 1, 0, false) X(false, 1, 1, false)     \
-  X(true, 1, 1, false) X(false, 2, 0, false) X(true, 2, 0, false) X(false, 2, 1, false) X(true, 2, 1, false)      \
-  X(false, 1, 0, true) X(true, 1, 0, true) X(false, 1, 1, true) X(true, 1, 1, true) X(false, 2, 0, true)          \
-  X(true, 2, 0, true) X(false, 2, 1, true) X(true, 2, 1, true)
+  X(false, 0, 0, 0) X(true, 0, 0, 0) X(false, 1, 0, 0) X(true, 1, 0, 0) X(false, 1, 1, 0) X(true, 1, 1, 0)         \
+  X(false, 2, 0, 0) X(true, 2, 0, 0) X(false, 2, 1, 0) X(true, 2, 1, 0) X(false, 1, 0, 1) X(true, 1, 0, 1)         \
+  X(false, 1, 1, 1) X(true, 1, 1, 1) X(false, 2, 0, 1) X(true, 2, 0, 1) X(false, 2, 1, 1) X(true, 2, 1, 1)         \
+  X(false, 1, 0, 2) X(true, 1, 0, 2) X(false, 1, 1, 2) X(true, 1, 1, 2)
 
 cudaError_t set_pass_smem_attr(size_t smem) {
   cudaError_t e = cudaSuccess;
@@ -1332,10 +1324,10 @@ int debug_layouts(int* out, int cap) {
 
 cudaError_t pass_occupancy(bool backward, bool slow, size_t smem, int* blocks_per_sm) {
   if (backward)
-    return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, 0, 0, false>, kThreads, smem)
-                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, 2, 1, false>, kThreads, smem);
-  return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, 0, 0, false>, kThreads, smem)
-              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, 2, 1, false>, kThreads, smem);
+    return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, 0, 0, 0>, kThreads, smem)
+                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, 2, 1, 0>, kThreads, smem);
+  return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, 0, 0, 0>, kThreads, smem)
+              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, 2, 1, 0>, kThreads, smem);
 }
 
 cudaError_t launch_pass(bool backward, const PassArgs& a, const DevPass& p, const PassMaps& maps, int grid,
@@ -1343,7 +1335,13 @@ cudaError_t launch_pass(bool backward, const PassArgs& a, const DevPass& p, cons
   const int mode = p.slow ? 0 : p.tma ? 2 : 1;
   const CUtensorMap& m0 = *reinterpret_cast<const CUtensorMap*>(maps.m0);
   const CUtensorMap& m1 = *reinterpret_cast<const CUtensorMap*>(maps.m1);
-  const bool re = a.reupload != 0;
+  // re-uploading: RE 2 where the tile holds a batch-unit bit, else RE 1
+  int re = 0;
+  if (a.reupload) {
+    re = 1;
+    for (int b = 0; b < kTileBits; ++b)
+      if (p.tile_q[b] < 0) re = 2;
+  }
 #define QML_LAUNCH(B, M, V, R)                                                              \
   if (backward == B && mode == M && p.variant == V && re == R) {                            \
     pass_kernel<B, M, V, R><<<grid, kThreads, smem, s>>>(a, p, m0, m1);                     \
@@ -1492,15 +1490,6 @@ cudaError_t launch_obs_bwd_init(float2* psi, float2* lam, const float* g, int B,
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   planes_kernel<<<blocks, 256, 0, s>>>(psi, lam, tot);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_permute_bits(float2* buf, long long count, int cb, const int* to, int grid, cudaStream_t s) {
-  BitPerm perm{};
-  perm.cb = cb;
-  for (int b = 0; b < cb; ++b) perm.to[b] = to[b];
-  const long long chunks = count >> cb;
-  permute_bits_kernel<<<grid, 256, sizeof(float2) << cb, s>>>(buf, chunks, perm);
   return cudaGetLastError();
 }
 

@@ -73,8 +73,9 @@ cudaError_t launch_bwd_init(float2* psi, float2* lam, const float* g, int B, int
 
 // In place, for every aligned chunk of 2^cb elements of buf (count elements):
 // element j moves to sum_b j_b << to[b] (a permutation of the low cb index
-// bits, cb <= 12).
-cudaError_t launch_permute_bits(float2* buf, long long count, int cb, const int* to, int grid, cudaStream_t s);
+// bits, cb <= 12).  count must be a multiple of 4096 and buf 16-byte aligned
+// (cudaErrorInvalidValue otherwise); the grid is sized from sms.
+cudaError_t launch_permute_bits(float2* buf, long long count, int cb, const int* to, int sms, cudaStream_t s);
 
 // Observables O = sum_k c_k i^ny X^x Z^z, terms grouped by x (see kernels.cu).
 struct ObsTerm {
@@ -96,5 +97,41 @@ cudaError_t launch_obs_bwd_init(float2* psi, float2* lam, const float* g, int B,
 cudaError_t launch_encode(const float* x, int B, int n, float2* psi, cudaStream_t s);
 cudaError_t launch_ckpt_copy(bool save, const float2* psi_in, float2* psi_out, void* slot,
                              int storage, long long count, cudaStream_t s);
+
+// ---------------------------------------------------------------- fp64 mode
+constexpr int kF64Threads = 512;  // threads of an fp64 pass block
+constexpr int kF64Warps = kF64Threads / 32;
+
+// Arguments of one fp64 pass launch (f64.cu).  One block keeps one sample's
+// tile; the state is in the standard index order.
+struct Pass64Args {
+  int n, B, T;            // qubits, samples, tile qubits (min(n, 12))
+  long long n_tiles;      // B << (n - T)
+  const double* theta;    // [L][n][3]
+  const double* x;        // [B][n]
+  double2* psi;           // [B][2^n]
+  double2* lam;           // backward: [B][2^n]
+  void* ckpt;             // checkpoint slots
+  int storage;            // 0 fp32, 1 bf16, 2 fp64 slots
+  long long slot_elems;   // elements per slot (max_batch << n)
+  double* partials;       // backward gradient partials
+  unsigned* status;
+  int reupload;           // every layer starts with the encoding Ry(x_q) again
+  uint32_t nb[kMaxQubits];    // CZ neighbours of each qubit (qubit mask)
+  uint32_t nbhi[kMaxQubits];  // CZ neighbours of each qubit above it
+};
+
+size_t pass64_smem_bytes(bool backward);
+// Shared-memory opt-in of the fp64 pass kernels and their resident blocks per SM.
+cudaError_t pass64_setup(int* blocks_fwd, int* blocks_bwd);
+cudaError_t launch_pass64(bool backward, const Pass64Args& a, const DevPass& p, int grid, cudaStream_t s);
+cudaError_t launch_bwd_init64(const double2* psi, double2* lam, const double* g, int B, int n, cudaStream_t s);
+size_t expect64_partial_count(int B, int n);
+cudaError_t launch_expect64(const double2* psi, int B, int n, double* partial, double* E, unsigned* status,
+                            cudaStream_t s);
+cudaError_t launch_grad_reduce64(const DevPass* passes, const int* slot_pass, const int* slot_index,
+                                 const double* partials, int grid, const double* theta, int L, int n, double* grad,
+                                 unsigned* status, cudaStream_t s);
+cudaError_t launch_loss_seed64(const double* E, const double* y, int B, double* g, double* loss, cudaStream_t s);
 
 }  // namespace qml

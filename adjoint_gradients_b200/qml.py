@@ -21,7 +21,8 @@ STATUS_NAMES = {
     4: "QML_ERR_CUDA", 5: "QML_ERR_CKPT_MISMATCH", 6: "QML_ERR_NUMERIC", 7: "QML_ERR_BOUNDS",
     8: "QML_ERR_TIMEOUT",
 }
-STORAGE = {"fp32": 0, "bf16": 1}
+STORAGE = {"fp32": 0, "bf16": 1, "fp64": 2}
+PRECISION = ("fp32", "fp64")
 
 # every function include/qml.h declares
 EXPORTS = [
@@ -32,6 +33,8 @@ EXPORTS = [
     "qml_enable_timing", "qml_read_timing", "qml_launch_count", "qml_expect_z0_static",
     "qml_debug_tile_view", "qml_debug_layouts", "qml_set_observable", "qml_observable_terms",
     "qml_expect_observable", "qml_set_entangler", "qml_entangler_bonds", "qml_set_reupload", "qml_reupload",
+    "qml_create_f64", "qml_precision", "qml_forward_expect_f64", "qml_backward_adjoint_f64", "qml_loss_seed_f64",
+    "qml_step_host_f64",
 ]
 
 
@@ -108,6 +111,12 @@ def load_library(path: str = LIB_PATH):
         "qml_entangler_bonds": ([_vp], _i),
         "qml_set_reupload": ([_vp, _i], _i),
         "qml_reupload": ([_vp], _i),
+        "qml_create_f64": ([ctypes.POINTER(_Config), _i, ctypes.POINTER(_vp)], _i),
+        "qml_precision": ([_vp], _i),
+        "qml_forward_expect_f64": ([_vp, _vp, _vp, _i, _vp, _vp, _vp], _i),
+        "qml_backward_adjoint_f64": ([_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp], _i),
+        "qml_loss_seed_f64": ([_vp, _vp, _vp, _i, _vp, _vp, _vp], _i),
+        "qml_step_host_f64": ([_vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp], _i),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -147,17 +156,24 @@ class Context:
     """One circuit shape (n qubits, L layers) on one CUDA device.
 
     Complex states are torch float32 tensors of shape [B, 2^n, 2] (re, im), or
-    complex64 tensors of shape [B, 2^n].
+    complex64 tensors of shape [B, 2^n]; with precision="fp64" float64
+    [B, 2^n, 2] or complex128 [B, 2^n], and float64 inputs and outputs.
     """
 
     def __init__(self, n_qubits: int, n_layers: int, max_batch: int, ckpt_block: int = 0,
-                 storage: str = "fp32", device: int = 0, host_step: bool = False, workspace=True):
+                 storage: str = "fp32", device: int = 0, host_step: bool = False, workspace=True,
+                 precision: str = "fp32"):
+        if precision not in PRECISION:
+            raise ValueError(f"precision must be one of {PRECISION}")
         self.lib = load_library()
         self.n, self.L, self.max_batch = n_qubits, n_layers, max_batch
         self.ckpt_block, self.storage, self.device = ckpt_block, storage, device
+        self.precision = precision
+        self.f64 = precision == "fp64"
         cfg = _Config(n_qubits, n_layers, max_batch, ckpt_block, STORAGE[storage])
         h = _vp()
-        _check(self.lib.qml_create(ctypes.byref(cfg), device, ctypes.byref(h)), "qml_create")
+        create = self.lib.qml_create_f64 if self.f64 else self.lib.qml_create
+        _check(create(ctypes.byref(cfg), device, ctypes.byref(h)), "qml_create_f64" if self.f64 else "qml_create")
         self._h = h
         self.ws = None
         if workspace:
@@ -277,19 +293,25 @@ class Context:
         _check(self.lib.qml_sync(self._h, _stream_handle(stream)), "qml_sync (device status)")
 
     # ------------------------------------------------------------- compute
+    @property
+    def real_dtype(self):
+        import torch
+
+        return torch.float64 if self.f64 else torch.float32
+
     def new_state(self, B: int):
         import torch
 
-        return torch.empty((B, 1 << self.n, 2), dtype=torch.float32, device=f"cuda:{self.device}")
+        return torch.empty((B, 1 << self.n, 2), dtype=self.real_dtype, device=f"cuda:{self.device}")
 
-    @staticmethod
-    def _state_ptr(t):
+    def _state_ptr(self, t):
         import torch
 
-        if t.dtype == torch.complex64:
+        if t.dtype in (torch.complex64, torch.complex128):
             t = torch.view_as_real(t)
-        if t.dtype != torch.float32 or not t.is_contiguous() or not t.is_cuda:
-            raise ValueError("state must be a contiguous CUDA float32 [B, 2^n, 2] or complex64 tensor")
+        if t.dtype != self.real_dtype or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"state must be a contiguous CUDA {self.real_dtype} [B, 2^n, 2] tensor "
+                             "(or its complex view)")
         return t.data_ptr()
 
     def encode(self, x, psi=None, stream=None):
@@ -304,29 +326,30 @@ class Context:
 
         B = x.shape[0]
         psi = self.new_state(B) if psi is None else psi
-        expect = torch.empty(B, dtype=torch.float32, device=x.device) if expect is None else expect
-        _check(self.lib.qml_forward_expect(self._h, _ptr(theta), _ptr(x), B, self._state_ptr(psi), _ptr(expect),
-                                           _stream_handle(stream)), "qml_forward_expect")
+        expect = torch.empty(B, dtype=self.real_dtype, device=x.device) if expect is None else expect
+        f = self.lib.qml_forward_expect_f64 if self.f64 else self.lib.qml_forward_expect
+        _check(f(self._h, _ptr(theta), _ptr(x), B, self._state_ptr(psi), _ptr(expect), _stream_handle(stream)),
+               "qml_forward_expect")
         return psi, expect
 
     def backward(self, theta, x, psi, lam, dLdE, grad=None, stream=None):
         import torch
 
         B = x.shape[0]
-        grad = torch.empty((self.L, self.n, 3), dtype=torch.float32, device=x.device) if grad is None else grad
-        _check(self.lib.qml_backward_adjoint(self._h, _ptr(theta), _ptr(x), B, self._state_ptr(psi),
-                                             self._state_ptr(lam), _ptr(dLdE), _ptr(grad), _stream_handle(stream)),
-               "qml_backward_adjoint")
+        grad = torch.empty((self.L, self.n, 3), dtype=self.real_dtype, device=x.device) if grad is None else grad
+        f = self.lib.qml_backward_adjoint_f64 if self.f64 else self.lib.qml_backward_adjoint
+        _check(f(self._h, _ptr(theta), _ptr(x), B, self._state_ptr(psi), self._state_ptr(lam), _ptr(dLdE),
+                 _ptr(grad), _stream_handle(stream)), "qml_backward_adjoint")
         return grad
 
     def loss_seed(self, expect, y, stream=None):
         import torch
 
         B = expect.shape[0]
-        g = torch.empty(B, dtype=torch.float32, device=expect.device)
-        loss = torch.empty(1, dtype=torch.float32, device=expect.device)
-        _check(self.lib.qml_loss_seed(self._h, _ptr(expect), _ptr(y), B, _ptr(g), _ptr(loss), _stream_handle(stream)),
-               "qml_loss_seed")
+        g = torch.empty(B, dtype=self.real_dtype, device=expect.device)
+        loss = torch.empty(1, dtype=self.real_dtype, device=expect.device)
+        f = self.lib.qml_loss_seed_f64 if self.f64 else self.lib.qml_loss_seed
+        _check(f(self._h, _ptr(expect), _ptr(y), B, _ptr(g), _ptr(loss), _stream_handle(stream)), "qml_loss_seed")
         return g, loss
 
     def expect_z0(self, psi, expect=None, stream=None):
@@ -350,16 +373,21 @@ class Context:
                   stream=None) -> StepResult:
         """Forward + loss + backward from (preferably pinned) host arrays."""
         B = x.shape[0]
+        dt = np.float64 if self.f64 else np.float32
         if out is None:
-            out = StepResult(np.empty(B, np.float32), np.empty(1, np.float32),
-                             np.empty((self.L, self.n, 3), np.float32))
+            out = StepResult(np.empty(B, dt), np.empty(1, dt), np.empty((self.L, self.n, 3), dt))
 
         def hp(a):
             if hasattr(a, "data_ptr"):
                 return a.data_ptr()
-            assert a.dtype == np.float32 and a.flags.c_contiguous
+            assert a.dtype == dt and a.flags.c_contiguous
             return a.ctypes.data
 
-        _check(self.lib.qml_step_host(self._h, hp(x), hp(theta), hp(y), B, hp(out.expect), hp(out.loss),
-                                      hp(out.grad), _stream_handle(stream)), "qml_step_host")
+        f = self.lib.qml_step_host_f64 if self.f64 else self.lib.qml_step_host
+        _check(f(self._h, hp(x), hp(theta), hp(y), B, hp(out.expect), hp(out.loss), hp(out.grad),
+                 _stream_handle(stream)), "qml_step_host")
         return out
+
+    @property
+    def precision_bits(self) -> int:
+        return int(self.lib.qml_precision(self._h))

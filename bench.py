@@ -38,6 +38,8 @@ UNIT = "samples/s"
 # FP32 ALU roofline: 148 SMs x 128 FP32 lanes x 2 flop (FMA) x 1965 MHz max SM clock.
 SMS, FP32_LANES, SM_MAX_MHZ = 148, 128, 1965.0
 ALU_PEAK_TFLOPS = SMS * FP32_LANES * 2 * SM_MAX_MHZ * 1e6 / 1e12
+FP64_LANES = 64       # FP64 FMA lanes per SM (B200 data sheet: 40 TFLOP/s FP64 at boost)
+ALU64_PEAK_TFLOPS = SMS * FP64_LANES * 2 * SM_MAX_MHZ * 1e6 / 1e12
 FMA_FWD_PER_ROT = 8   # per amplitude: one fused SU(2) on a pair = 16 FMA / 2 amplitudes
 FMA_BWD_PER_ROT = 22  # per amplitude: U^dagger on psi (8) and lambda (8) + three Im<l|P|p> terms (6)
 CPU_SAMPLE_LAYERS = 16  # oracle sample depth (cost is linear in depth)
@@ -117,7 +119,7 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------- helpers
 
-def algorithmic_counts(ctx, w, B):
+def algorithmic_counts(ctx, w, B, f64=False):
     """Per-pass algorithmic FMAs and HBM bytes of the forward and backward pass kernels."""
     sched = ctx.debug_schedule()
     P = sched[0]
@@ -126,11 +128,15 @@ def algorithmic_counts(ctx, w, B):
     # bytes per amplitude moved by each pass, from the schedule flags
     i = 1
     fwd_bytes = bwd_bytes = 0
-    slot_b = 4 if w.storage == "bf16" else 8
+    slot_b = {"bf16": 4, "fp32": 8, "fp64": 16}[w.storage]
+    c = 16 if f64 else 8  # one complex amplitude
     for _ in range(P):
         set_id, gen, last, ck, nops = sched[i:i + 5]
         i += 5 + 4 * nops
-        fwd_bytes += (0 if gen else 8) + 8 + (slot_b if ck >= 0 else 0)
+        fwd_bytes += (0 if gen else c) + c + (slot_b if ck >= 0 else 0)
+        if f64:  # psi and lambda read (the slot replaces psi at a boundary) and written
+            bwd_bytes += 2 * c + (slot_b - c if ck >= 0 else 0) + (0 if gen else 2 * c)
+            continue
         rd = 8 if last else 16
         wr = 0 if gen else 16
         bwd_bytes += rd + wr + (slot_b if ck >= 0 else 0)
@@ -218,11 +224,12 @@ def run_reference(args):
     return 0
 
 
-def workload_config(w, B):
+def workload_config(w, B, f64=False):
     return {
         "workload": w.name, "n_qubits": w.n, "layers": w.L, "batch_per_gpu": B, "params": w.params,
-        "ckpt_block": w.ckpt_block, "ckpt_storage": w.storage, "state": "complex64 [B][2^n]",
-        "l2": "inputs larger than L2 (working state B*2^n*8 B > 126 MB); no flush",
+        "ckpt_block": w.ckpt_block, "ckpt_storage": w.storage,
+        "state": "complex128 [B][2^n]" if f64 else "complex64 [B][2^n]",
+        "l2": (f"inputs larger than L2 (working state B*2^n*{16 if f64 else 8} B > 126 MB); no flush"),
         "seeds": {"x": 1000 + w.index, "theta": 2000 + w.index, "y": 3000 + w.index},
     }
 
@@ -264,17 +271,24 @@ def run_ours(args):
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     w = WORKLOADS[args.workload]
+    f64 = args.precision == "fp64"
+    if f64:  # fp64 mode keeps its checkpoint slots exact
+        import dataclasses
+
+        w = dataclasses.replace(w, storage="fp64")
+    fdt = torch.float64 if f64 else torch.float32
     B = w.B
     dev = f"cuda:{local}"
     # each rank draws its own batch; theta is shared
     x = np.random.default_rng(1000 + w.index + 7919 * rank).uniform(0, np.pi, (B, w.n))
     y = np.random.default_rng(3000 + w.index + 7919 * rank).integers(0, 2, B) * 2.0 - 1.0
     theta = draw_theta(w.index, w.L, w.n)
-    xd = torch.tensor(x, dtype=torch.float32, device=dev)
-    yd = torch.tensor(y, dtype=torch.float32, device=dev)
-    td = torch.tensor(theta, dtype=torch.float32, device=dev)
+    xd = torch.tensor(x, dtype=fdt, device=dev)
+    yd = torch.tensor(y, dtype=fdt, device=dev)
+    td = torch.tensor(theta, dtype=fdt, device=dev)
 
-    ctx = qml.Context(w.n, w.L, B, ckpt_block=w.ckpt_block, storage=w.storage, device=local)
+    ctx = qml.Context(w.n, w.L, B, ckpt_block=w.ckpt_block, storage=w.storage, device=local,
+                      precision=args.precision)
     obs = observable_terms(args.observable, w.n)
     ctx.set_observable(obs)
     bonds = entangler_bonds(args.entangler, w.n)
@@ -282,8 +296,8 @@ def run_ours(args):
     ctx.set_reupload(args.reupload)
     psi = ctx.new_state(B)
     lam = ctx.new_state(B)
-    E = torch.empty(B, dtype=torch.float32, device=dev)
-    grad = torch.empty((w.L, w.n, 3), dtype=torch.float32, device=dev)
+    E = torch.empty(B, dtype=fdt, device=dev)
+    grad = torch.empty((w.L, w.n, 3), dtype=fdt, device=dev)
     stream = torch.cuda.current_stream()
 
     from adjoint_gradients_b200 import dp
@@ -331,8 +345,9 @@ def run_ours(args):
     value = world * B * args.steps / (ms / 1e3)
 
     # ---- roofline of the dominant kernel (the backward pass kernel)
-    cnt = algorithmic_counts(ctx, w, B)
+    cnt = algorithmic_counts(ctx, w, B, f64)
     hbm_peak, peak_src = measured_peaks()
+    alu_peak = ALU64_PEAK_TFLOPS if f64 else ALU_PEAK_TFLOPS
     bwd_avg_s = bwd_ms / 1e3 / max(1, bwd_n)
     fwd_avg_s = fwd_ms / 1e3 / max(1, fwd_n)
     P = cnt["passes"]
@@ -346,31 +361,34 @@ def run_ours(args):
         with open(tfile) as f:
             tr = json.load(f).get(w.name, {})
         # counters taken on another build of the kernels do not count
-        if tr.get("kernel_sources_sha256") == kernel_sources_digest():
+        if tr.get("kernel_sources_sha256") == kernel_sources_digest() and not f64:
             traffic = tr.get("bwd_pass_bytes_per_launch")
     roofline = {
-        "kernel": "pass_kernel<backward>", "bound": "alu", "achieved": bwd_tflops, "peak": ALU_PEAK_TFLOPS,
-        "unit": "TFLOP/s", "frac": bwd_tflops / ALU_PEAK_TFLOPS, "traffic": traffic,
-        "peak_src": "148 SMs x 128 FP32 lanes x 2 x 1965 MHz (FFMA; packed f32x2 FMA measured at the same rate)",
+        "kernel": "pass64_kernel<backward>" if f64 else "pass_kernel<backward>", "bound": "alu",
+        "achieved": bwd_tflops, "peak": alu_peak,
+        "unit": "TFLOP/s", "frac": bwd_tflops / alu_peak, "traffic": traffic,
+        "peak_src": ("148 SMs x 64 FP64 lanes x 2 x 1965 MHz (DFMA; derived from unit counts)" if f64 else
+                     "148 SMs x 128 FP32 lanes x 2 x 1965 MHz (FFMA; packed f32x2 FMA measured at the same rate)"),
         "avg_launch_ms": bwd_avg_s * 1e3, "launches": bwd_n,
         "hbm_achieved_gbs": bwd_gbs, "hbm_peak_gbs": hbm_peak, "hbm_frac": bwd_gbs / hbm_peak,
         "hbm_peak_src": peak_src,
-        "forward_kernel": {"achieved_tflops": fwd_tflops, "frac": fwd_tflops / ALU_PEAK_TFLOPS,
+        "forward_kernel": {"achieved_tflops": fwd_tflops, "frac": fwd_tflops / alu_peak,
                            "hbm_gbs": fwd_gbs, "hbm_frac": fwd_gbs / hbm_peak, "avg_launch_ms": fwd_avg_s * 1e3},
     }
 
     # ---- end to end through host buffers (pinned), same metric
     e2e = None
     if not args.no_e2e:
-        ctx_h = qml.Context(w.n, w.L, B, ckpt_block=w.ckpt_block, storage=w.storage, device=local, host_step=True)
+        ctx_h = qml.Context(w.n, w.L, B, ckpt_block=w.ckpt_block, storage=w.storage, device=local, host_step=True,
+                            precision=args.precision)
         ctx_h.set_observable(obs)
         ctx_h.set_entangler(bonds)
         ctx_h.set_reupload(args.reupload)
-        xh = torch.tensor(x, dtype=torch.float32).pin_memory()
-        th = torch.tensor(theta, dtype=torch.float32).pin_memory()
-        yh = torch.tensor(y, dtype=torch.float32).pin_memory()
-        out = qml.StepResult(torch.empty(B).pin_memory(), torch.empty(1).pin_memory(),
-                             torch.empty((w.L, w.n, 3)).pin_memory())
+        xh = torch.tensor(x, dtype=fdt).pin_memory()
+        th = torch.tensor(theta, dtype=fdt).pin_memory()
+        yh = torch.tensor(y, dtype=fdt).pin_memory()
+        out = qml.StepResult(torch.empty(B, dtype=fdt).pin_memory(), torch.empty(1, dtype=fdt).pin_memory(),
+                             torch.empty((w.L, w.n, 3), dtype=fdt).pin_memory())
         for _ in range(max(1, min(args.warmup, 2))):
             ctx_h.step_host(xh, th, yh, out)
         k2 = max(1, args.steps)
@@ -391,8 +409,9 @@ def run_ours(args):
             t = torch.tensor([ems], device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             ems = float(t.item())
-        h2d = 4 * (B * w.n + w.L * w.n * 3 + B)
-        d2h = 4 * (B + 1 + w.L * w.n * 3)
+        fb = 8 if f64 else 4
+        h2d = fb * (B * w.n + w.L * w.n * 3 + B)
+        d2h = fb * (B + 1 + w.L * w.n * 3)
         e2e = {"value": world * B * k2 / (ems / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "api": "qml_step_host"}
         ctx_h.sync()
@@ -402,7 +421,7 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w)
 
-    cfg = {**workload_config(w, B), "parallelism": f"dp{world}" if world > 1 else "single",
+    cfg = {**workload_config(w, B, f64), "parallelism": f"dp{world}" if world > 1 else "single",
            "observable": "Z0" if obs is None else f"{args.observable} ({len(obs)} Pauli strings)",
            "entangler": f"CZ {args.entangler} ({len(bonds)} bonds)",
            "reupload": bool(args.reupload),
@@ -414,7 +433,7 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64" if f64 else "f32", "data": "synthetic",
             "config": cfg,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
             "clocks": clk,
@@ -441,6 +460,8 @@ def main():
     ap.add_argument("--entangler", default="chain", choices=["chain", "ring", "none"],
                     help="CZ bonds ending every layer: chain (q, q+1) as in the workloads, ring, or none")
     ap.add_argument("--reupload", action="store_true", help="data re-uploading: the encoding again in every layer")
+    ap.add_argument("--precision", default="fp32", choices=["fp32", "fp64"],
+                    help="arithmetic of the path: fp32, or fp64 (complex128 state, exact checkpoint slots)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

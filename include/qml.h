@@ -66,9 +66,9 @@ typedef enum {
 
 /* Storage format of checkpoint slots: fp32 (re, im) pairs, or the
  * memory-save mode's bfloat16 pairs (round to nearest even; compute stays
- * fp32).  [Gist-EN] Technical Summary sec. 2 "Memory-Saving Mode";
- * [Deep-dive] sec. 2.3. */
-typedef enum { QML_STORE_FP32 = 0, QML_STORE_BF16 = 1 } qml_storage;
+ * fp32 or fp64).  [Gist-EN] Technical Summary sec. 2 "Memory-Saving Mode";
+ * [Deep-dive] sec. 2.3.  fp64 pairs only for contexts of qml_create_f64. */
+typedef enum { QML_STORE_FP32 = 0, QML_STORE_BF16 = 1, QML_STORE_FP64 = 2 } qml_storage;
 
 typedef struct {
   int n_qubits;       /* 1 .. 30 */
@@ -304,6 +304,56 @@ QML_API int qml_debug_tile_view(const qml_ctx* ctx, int pass, int* out, int cap)
  * bits (slot of a position = sum of the weights of its set bits); then the
  * number of slots. */
 QML_API int qml_debug_layouts(int* out, int cap);
+
+/* ------------------------------------------------------------------------
+ * fp64 compute mode.  The pages state that the simulator runs in double as
+ * well as single precision ([Gist-EN] Technical Summary sec. 2 and 4).  A
+ * context made by qml_create_f64 runs the same schedule of fused forward and
+ * adjoint backward passes with complex128 state vectors and fp64 arithmetic;
+ * its inputs and outputs are float64 and its state vectors are [B][2^n]
+ * (re, im) double pairs, 16-byte aligned.  Checkpoint slots take the
+ * config's storage: QML_STORE_FP64 keeps them exact, QML_STORE_FP32 /
+ * QML_STORE_BF16 round them (the backward pass then restarts from the
+ * rounded state at each slot).  Entanglers (qml_set_entangler) and data
+ * re-uploading (qml_set_reupload, any n) apply; the observable is Z0 (a
+ * Pauli-sum observable makes the calls below return QML_ERR_UNSUPPORTED).
+ * The fp32 calls (qml_forward_expect, qml_backward_adjoint, qml_loss_seed,
+ * qml_step_host, qml_init_state_encode, qml_ckpt_save / _restore,
+ * qml_expect_z0, qml_expect_observable) return QML_ERR_UNSUPPORTED on an
+ * fp64 context, and the calls below on an fp32 one.  Workspace, entangler,
+ * timing and sync calls are shared.
+ * ------------------------------------------------------------------------ */
+
+/* Create an fp64 context (same arguments and errors as qml_create). */
+QML_API qml_status qml_create_f64(const qml_config* cfg, int device, qml_ctx** out);
+
+/* 32 or 64: the arithmetic precision of a context (-1 for NULL). */
+QML_API int qml_precision(const qml_ctx* ctx);
+
+/* As qml_forward_expect, in fp64.
+ *   theta_dev [L][n][3] float64, x_dev [B][n] float64
+ *   psi_dev   [B][2^n] complex128, out: final state (16-byte aligned)
+ *   expect_dev [B] float64, out */
+QML_API qml_status qml_forward_expect_f64(qml_ctx* ctx, const double* theta_dev, const double* x_dev, int B,
+                                          double* psi_dev, double* expect_dev, void* stream);
+
+/* As qml_backward_adjoint, in fp64 (psi_dev and lambda_dev complex128,
+ * 16-byte aligned, both clobbered; dLdE_dev [B] and grad_dev [L][n][3]
+ * float64).  Gradients are reduced in a fixed order (deterministic). */
+QML_API qml_status qml_backward_adjoint_f64(qml_ctx* ctx, const double* theta_dev, const double* x_dev, int B,
+                                            double* psi_dev, double* lambda_dev, const double* dLdE_dev,
+                                            double* grad_dev, void* stream);
+
+/* As qml_loss_seed, in fp64. */
+QML_API qml_status qml_loss_seed_f64(qml_ctx* ctx, const double* expect_dev, const double* y_dev, int B,
+                                     double* g_dev, double* loss_dev, void* stream);
+
+/* As qml_step_host, in fp64 (host arrays of doubles; the workspace of
+ * qml_host_workspace_bytes, which for an fp64 context sizes the staged
+ * buffers in doubles). */
+QML_API qml_status qml_step_host_f64(qml_ctx* ctx, const double* x_host, const double* theta_host,
+                                     const double* y_host, int B, double* expect_host, double* loss_host,
+                                     double* grad_host, void* stream);
 
 #ifdef __cplusplus
 }
