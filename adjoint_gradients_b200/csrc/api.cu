@@ -93,6 +93,8 @@ struct qml_ctx {
   uint32_t nb[kMaxQubits] = {0}, nbhi[kMaxQubits] = {0};
   bool reupload = false;  // every layer starts with the encoding again
   bool f64 = false;       // fp64 compute mode (qml_create_f64)
+  std::vector<uint32_t> f64_mask;  // fp64: tile qubits of each pass
+  int f64_tmax = 0;                // fp64: largest tile (qubits)
 };
 
 namespace {
@@ -105,7 +107,8 @@ void ensure_device(qml_ctx* c) {
     cudaDeviceProp prop;
     int bf = 0, bb = 0;
     DeviceGuard g(c->device);
-    if (cudaGetDeviceProperties(&prop, c->device) != cudaSuccess || pass64_setup(&bf, &bb) != cudaSuccess ||
+    if (cudaGetDeviceProperties(&prop, c->device) != cudaSuccess ||
+        pass64_setup(c->f64_tmax, &bf, &bb) != cudaSuccess ||
         bf < 1 || bb < 1) {
       cudaGetLastError();
       c->dev_ok = false;
@@ -438,13 +441,31 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
   return cuda_status(e);
 }
 
+// fp64 tiles: the schedule's tile qubits, less the highest qubit the pass
+// does not rotate when the tile has 12 (2^11-position tiles let two blocks
+// share an SM; a passive qubit can leave the tile because CZ is diagonal).
+void set_f64_tiles(qml_ctx* c) {
+  const int n = c->cfg.n_qubits;
+  c->f64_mask.clear();
+  c->f64_tmax = 1;
+  for (const DevPass& dp : c->dpass) {
+    uint32_t m = 0, rot = 0;
+    for (int b = 0; b < kTileBits; ++b)
+      if (dp.tile_q[b] >= 0 && dp.tile_q[b] < n) m |= 1u << dp.tile_q[b];
+    for (int s = 0; s < dp.nslots; ++s) rot |= 1u << (dp.slot_lq[s] % n);
+    const uint32_t passive = m & ~rot;
+    if (__builtin_popcount(m) == kTileBits && passive) m &= ~(1u << (31 - __builtin_clz(passive)));
+    c->f64_mask.push_back(m);
+    c->f64_tmax = std::max(c->f64_tmax, __builtin_popcount(m));
+  }
+}
+
 Pass64Args pass64_args(qml_ctx* c, const double* theta, const double* x, int B, double2* psi, double2* lam) {
   Pass64Args a{};
   const int n = c->cfg.n_qubits;
   a.n = n;
   a.B = B;
-  a.T = std::min(n, kTileBits);
-  a.n_tiles = (long long)B << (n - a.T);
+  a.tmax = c->f64_tmax;
   a.theta = theta;
   a.x = x;
   a.psi = psi;
@@ -459,13 +480,20 @@ Pass64Args pass64_args(qml_ctx* c, const double* theta, const double* x, int B, 
   return a;
 }
 
+void set_pass_tile(const qml_ctx* c, int p, int B, Pass64Args* a) {
+  a->tile_mask = c->f64_mask[p];
+  a->T = __builtin_popcount(a->tile_mask);
+  a->n_tiles = (long long)B << (c->cfg.n_qubits - a->T);
+}
+
 qml_status run_forward64(qml_ctx* c, const double* theta, const double* x, int B, double2* psi, double* expect,
                          cudaStream_t s) {
-  const Pass64Args a = pass64_args(c, theta, x, B, psi, nullptr);
+  Pass64Args a = pass64_args(c, theta, x, B, psi, nullptr);
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, false);
   for (int p = 0; p < (int)c->dpass.size(); ++p) {
     const DevPass& dp = c->dpass[p];
+    set_pass_tile(c, p, B, &a);
     if (launch_pass64(false, a, dp, (int)std::min<long long>(c->grid_fwd, a.n_tiles), s) != cudaSuccess)
       return QML_ERR_CUDA;
     ++c->launches;
@@ -487,12 +515,13 @@ qml_status run_backward64(qml_ctx* c, const double* theta, const double* x, int 
   for (int m = 0; m < c->plan.n_ckpt; ++m)
     if (c->ckpt_batch[m] != B) return QML_ERR_CKPT_MISMATCH;
   if (launch_bwd_init64(psi, lam, g, B, n, s) != cudaSuccess) return QML_ERR_CUDA;
-  const Pass64Args a = pass64_args(c, theta, x, B, psi, lam);
+  Pass64Args a = pass64_args(c, theta, x, B, psi, lam);
   c->launches += 2;  // lambda init, gradient reduce
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, true);
   // every block writes its partials, so the grid is the one the layout counted
   for (int p = (int)c->dpass.size() - 1; p >= 0; --p) {
+    set_pass_tile(c, p, B, &a);
     if (launch_pass64(true, a, c->dpass[p], c->grid_bwd, s) != cudaSuccess) return QML_ERR_CUDA;
     ++c->launches;
   }
@@ -570,6 +599,7 @@ static qml_status create_ctx(const qml_config* cfg, int device, bool f64, qml_ct
   for (const DevPass& dp : c->dpass)
     if (dp.slow) c->slow = true;
   c->ckpt_batch.assign(c->plan.n_ckpt, -1);
+  if (f64) set_f64_tiles(c);
   *out = c;
   return QML_OK;
 }

@@ -8,12 +8,13 @@
 // and 1.4, sec. 3.2).  The pages state that the simulator runs in double as
 // well as single precision ([Gist-EN] Technical Summary sec. 2 and 4).
 //
-// Layout and schedule.  The passes of the fp32 schedule are reused unchanged:
-// a pass owns the 2^T (T = min(n, 12)) positions of a tile, the tile's qubits
-// are the ones the schedule gives it, and the ops are the same rotations and
-// CZ layers.  The state stays in the standard index order throughout.  A
+// Layout and schedule.  The passes of the fp32 schedule are reused: the ops
+// are the same rotations and CZ layers, and a pass's tile holds the qubits
+// the schedule gives it, less one qubit that the pass does not rotate when the
+// schedule's tile has 12 (so a tile is at most 2^11 positions and two blocks
+// fit on an SM).  The state stays in the standard index order throughout.  A
 // block keeps one sample's tile in shared memory (psi, and lambda in the
-// backward: 72 KB per plane with one pad element per eight), and a rotation
+// backward: 36 KB per plane with one pad element per eight), and a rotation
 // op is applied in chunks of up to three qubits: each thread takes the eight
 // positions of one chunk group into registers, applies the chunk's 2x2
 // unitaries (and, backward, accumulates the three Im<lambda|P|psi> terms of
@@ -33,9 +34,10 @@ constexpr unsigned kErrBounds = 1u << 7;   // QML_ERR_BOUNDS
 
 constexpr int kW = kF64Warps;
 constexpr int kT = kF64Threads;
-constexpr int kPad = kTilePos + (kTilePos >> 3);  // shared positions of one plane
 
 __device__ __forceinline__ int padp(int p) { return p + (p >> 3); }
+// shared positions of one plane for tiles of up to 2^tmax positions
+constexpr int plane_slots(int tmax) { return (1 << tmax) + ((1 << tmax) >> 3); }
 
 // Per-block schedule data, built at kernel start.
 struct Ctx64 {
@@ -49,8 +51,8 @@ struct Ctx64 {
   double cs[kMaxQubits], sn[kMaxQubits];  // (cos, sin)(x/2) of the tile's sample
 };
 
-size_t f64_smem_bytes(bool bwd) {
-  size_t b = sizeof(double2) * (size_t)kPad * (bwd ? 2 : 1) + sizeof(Ctx64);
+size_t f64_smem_bytes(bool bwd, int tmax) {
+  size_t b = sizeof(double2) * (size_t)plane_slots(tmax) * (bwd ? 2 : 1) + sizeof(Ctx64);
   if (bwd) b += sizeof(double) * (size_t)kW * kMaxSlots * 3;
   return b;
 }
@@ -137,17 +139,19 @@ __device__ void rot_chunk(const Pass64Args& a, const DevPass& P, const Ctx64& cx
     int p0 = g;
 #pragma unroll
     for (int i = 0; i < K; ++i) p0 = ((p0 >> srt[i]) << (srt[i] + 1)) | (p0 & ((1 << srt[i]) - 1));
-    int pos[1 << K];
-    double2 v[1 << K], w[1 << K];
-#pragma unroll
-    for (int j = 0; j < (1 << K); ++j) {
+    // position of register j: p0 plus the chunk bits set in j
+    auto pos = [&](int j) {
       int p = p0;
 #pragma unroll
       for (int i = 0; i < K; ++i)
         if ((j >> i) & 1) p |= 1 << pb[i];
-      pos[j] = padp(p);
-      v[j] = tp[pos[j]];
-      if (BWD) w[j] = tl[pos[j]];
+      return padp(p);
+    };
+    double2 v[1 << K], w[1 << K];
+#pragma unroll
+    for (int j = 0; j < (1 << K); ++j) {
+      v[j] = tp[pos(j)];
+      if (BWD) w[j] = tl[pos(j)];
     }
 #pragma unroll
     for (int i = 0; i < K; ++i) {
@@ -168,8 +172,8 @@ __device__ void rot_chunk(const Pass64Args& a, const DevPass& P, const Ctx64& cx
     }
 #pragma unroll
     for (int j = 0; j < (1 << K); ++j) {
-      tp[pos[j]] = v[j];
-      if (BWD) tl[pos[j]] = w[j];
+      tp[pos(j)] = v[j];
+      if (BWD) tl[pos(j)] = w[j];
     }
   }
   if (BWD) {
@@ -187,19 +191,18 @@ __device__ void rot_chunk(const Pass64Args& a, const DevPass& P, const Ctx64& cx
 }
 
 template <bool BWD>
-__global__ void __launch_bounds__(kT) pass64_kernel(const Pass64Args a, const __grid_constant__ DevPass P) {
+__global__ void __launch_bounds__(kT, 2) pass64_kernel(const Pass64Args a, const __grid_constant__ DevPass P) {
   extern __shared__ __align__(16) unsigned char smem64[];
   double2* tp = reinterpret_cast<double2*>(smem64);
-  double2* tl = tp + kPad;
-  Ctx64& cx = *reinterpret_cast<Ctx64*>(smem64 + sizeof(double2) * kPad * (BWD ? 2 : 1));
+  const int plane = plane_slots(a.tmax);
+  double2* tl = tp + plane;
+  Ctx64& cx = *reinterpret_cast<Ctx64*>(smem64 + sizeof(double2) * plane * (BWD ? 2 : 1));
   double* acc = reinterpret_cast<double*>(reinterpret_cast<unsigned char*>(&cx) + sizeof(Ctx64));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n = a.n;
 
   if (tid == 0) {
-    uint32_t inmask = 0;
-    for (int b = 0; b < kTileBits; ++b)
-      if (P.tile_q[b] >= 0 && P.tile_q[b] < n) inmask |= 1u << P.tile_q[b];
+    const uint32_t inmask = a.tile_mask;  // this pass's tile qubits
     int T = 0, no = 0;
     for (int q = 0; q < n; ++q) {
       cx.pos_of_q[q] = -1;
@@ -230,7 +233,7 @@ __global__ void __launch_bounds__(kT) pass64_kernel(const Pass64Args a, const __
     for (int i = tid; i < kW * kMaxSlots * 3; i += kT) acc[i] = 0.0;
   __syncthreads();
   const int T = cx.T, P2 = 1 << T, no = cx.n_out;
-  if (T != a.T) {  // the schedule and the host disagree on the tile: touch nothing
+  if (T != a.T || T > a.tmax) {  // the host's tile does not fit: touch nothing
     if (tid == 0) atomicOr(a.status, kErrBounds);
     return;
   }
@@ -431,24 +434,27 @@ __global__ void loss_seed64_kernel(const double* E, const double* y, int B, doub
 
 }  // namespace
 
-size_t pass64_smem_bytes(bool backward) { return f64_smem_bytes(backward); }
+size_t pass64_smem_bytes(bool backward, int tmax) { return f64_smem_bytes(backward, tmax); }
 
-cudaError_t pass64_setup(int* blocks_fwd, int* blocks_bwd) {
+cudaError_t pass64_setup(int tmax, int* blocks_fwd, int* blocks_bwd) {
   cudaError_t e = cudaFuncSetAttribute(pass64_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)f64_smem_bytes(false));
+                                       (int)f64_smem_bytes(false, kTileBits));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(pass64_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)f64_smem_bytes(true));
+                             (int)f64_smem_bytes(true, kTileBits));
   if (e == cudaSuccess)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_fwd, pass64_kernel<false>, kT, f64_smem_bytes(false));
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_fwd, pass64_kernel<false>, kT,
+                                                      f64_smem_bytes(false, tmax));
   if (e == cudaSuccess)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_bwd, pass64_kernel<true>, kT, f64_smem_bytes(true));
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_bwd, pass64_kernel<true>, kT,
+                                                      f64_smem_bytes(true, tmax));
   return e;
 }
 
 cudaError_t launch_pass64(bool backward, const Pass64Args& a, const DevPass& p, int grid, cudaStream_t s) {
-  if (backward) pass64_kernel<true><<<grid, kT, f64_smem_bytes(true), s>>>(a, p);
-  else pass64_kernel<false><<<grid, kT, f64_smem_bytes(false), s>>>(a, p);
+  if (a.tmax < a.T || a.tmax > kTileBits) return cudaErrorInvalidValue;
+  if (backward) pass64_kernel<true><<<grid, kT, f64_smem_bytes(true, a.tmax), s>>>(a, p);
+  else pass64_kernel<false><<<grid, kT, f64_smem_bytes(false, a.tmax), s>>>(a, p);
   return cudaGetLastError();
 }
 

@@ -99,13 +99,15 @@ cudaError_t launch_ckpt_copy(bool save, const float2* psi_in, float2* psi_out, v
                              int storage, long long count, cudaStream_t s);
 
 // ---------------------------------------------------------------- fp64 mode
-constexpr int kF64Threads = 512;  // threads of an fp64 pass block
+constexpr int kF64Threads = 256;  // threads of an fp64 pass block
 constexpr int kF64Warps = kF64Threads / 32;
 
 // Arguments of one fp64 pass launch (f64.cu).  One block keeps one sample's
 // tile; the state is in the standard index order.
 struct Pass64Args {
-  int n, B, T;            // qubits, samples, tile qubits (min(n, 12))
+  int n, B, T;            // qubits, samples, tile qubits of this pass
+  int tmax;               // largest T of the context's passes (shared-memory size)
+  uint32_t tile_mask;     // this pass's tile qubits
   long long n_tiles;      // B << (n - T)
   const double* theta;    // [L][n][3]
   const double* x;        // [B][n]
@@ -121,9 +123,10 @@ struct Pass64Args {
   uint32_t nbhi[kMaxQubits];  // CZ neighbours of each qubit above it
 };
 
-size_t pass64_smem_bytes(bool backward);
-// Shared-memory opt-in of the fp64 pass kernels and their resident blocks per SM.
-cudaError_t pass64_setup(int* blocks_fwd, int* blocks_bwd);
+size_t pass64_smem_bytes(bool backward, int tmax);
+// Shared-memory opt-in of the fp64 pass kernels and their resident blocks per
+// SM for tiles of up to 2^tmax positions.
+cudaError_t pass64_setup(int tmax, int* blocks_fwd, int* blocks_bwd);
 cudaError_t launch_pass64(bool backward, const Pass64Args& a, const DevPass& p, int grid, cudaStream_t s);
 cudaError_t launch_bwd_init64(const double2* psi, double2* lam, const double* g, int B, int n, cudaStream_t s);
 size_t expect64_partial_count(int B, int n);
