@@ -61,6 +61,12 @@ def _load():
         lib.oracle_adjoint_gen.argtypes = ([ctypes.c_int] * 3 + [_dp] * 2 + [ctypes.c_int, ctypes.c_int, _ip,
                                            ctypes.c_int, ctypes.c_char_p] + [_dp] * 5)
         lib.oracle_adjoint_gen.restype = ctypes.c_int
+        lib.oracle_forward_ent.argtypes = ([ctypes.c_int] * 3 + [_dp] * 2 + [ctypes.c_int] * 3 + [_ip,
+                                           ctypes.c_int, ctypes.c_char_p] + [_dp] * 3)
+        lib.oracle_forward_ent.restype = ctypes.c_int
+        lib.oracle_adjoint_ent.argtypes = ([ctypes.c_int] * 3 + [_dp] * 2 + [ctypes.c_int] * 3 + [_ip,
+                                           ctypes.c_int, ctypes.c_char_p] + [_dp] * 5)
+        lib.oracle_adjoint_ent.restype = ctypes.c_int
         lib.oracle_bf16_round.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t]
         lib.oracle_bf16_widen.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t]
         lib.oracle_num_threads.restype = ctypes.c_int
@@ -110,26 +116,32 @@ def _bonds(bonds):
     return arr.shape[0], arr, arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
 
 
-def forward(x, theta, want_state: bool = False, observable=None, bonds=None, reupload: bool = False):
+_ENTANGLERS = {"cz": 0, "cnot": 1}
+
+
+def forward(x, theta, want_state: bool = False, observable=None, bonds=None, reupload: bool = False,
+            entangler: str = "cz"):
     """<O> per sample (O = Z0, or the Pauli sum ``observable`` = [(coef, word)]), and
-    optionally the final states ``[B][2^n]`` complex128.  ``bonds``: the CZ pairs
-    of every layer's entangler, applied in list order (None: the chain q, q+1).
+    optionally the final states ``[B][2^n]`` complex128.  ``bonds``: the pairs
+    of every layer's entangler, applied in list order (None: the chain q, q+1);
+    ``entangler``: "cz", or "cnot" (each pair is (control, target)).
     ``reupload``: every layer starts with the encoding Ry(x_q) again."""
     x, theta, B, n, L = _prep(x, theta)
     E = np.zeros(B, dtype=np.float64)
     psi = np.zeros((B, 1 << n, 2), dtype=np.float64) if want_state else None
     k, words, coef = _observable(observable, n)
     nb, keep, bp = _bonds(bonds)
-    rc = _load().oracle_forward_gen(n, L, B, _ptr(x), _ptr(theta), int(reupload), nb, bp, k, words, _ptr(coef),
-                                    _ptr(E), _ptr(psi))
+    rc = _load().oracle_forward_ent(n, L, B, _ptr(x), _ptr(theta), int(reupload), _ENTANGLERS[entangler], nb, bp,
+                                    k, words, _ptr(coef), _ptr(E), _ptr(psi))
     if rc != 0:
-        raise RuntimeError("oracle_forward_gen failed")
+        raise RuntimeError("oracle_forward_ent failed")
     if want_state:
         return E, psi[..., 0] + 1j * psi[..., 1]
     return E
 
 
-def adjoint(x, theta, g, want_state: bool = False, observable=None, bonds=None, reupload: bool = False):
+def adjoint(x, theta, g, want_state: bool = False, observable=None, bonds=None, reupload: bool = False,
+            entangler: str = "cz"):
     """sum_b g_b dE_b/dtheta as ``[L][n][3]``, <O> per sample, and optionally the
     state after walking the circuit back to its start (must be |0...0>)."""
     x, theta, B, n, L = _prep(x, theta)
@@ -141,10 +153,10 @@ def adjoint(x, theta, g, want_state: bool = False, observable=None, bonds=None, 
     psi0 = np.zeros((B, 1 << n, 2), dtype=np.float64) if want_state else None
     k, words, coef = _observable(observable, n)
     nb, keep, bp = _bonds(bonds)
-    rc = _load().oracle_adjoint_gen(n, L, B, _ptr(x), _ptr(theta), int(reupload), nb, bp, k, words, _ptr(coef),
-                                    _ptr(g), _ptr(grad), _ptr(E), _ptr(psi0))
+    rc = _load().oracle_adjoint_ent(n, L, B, _ptr(x), _ptr(theta), int(reupload), _ENTANGLERS[entangler], nb, bp,
+                                    k, words, _ptr(coef), _ptr(g), _ptr(grad), _ptr(E), _ptr(psi0))
     if rc != 0:
-        raise RuntimeError("oracle_adjoint_gen failed")
+        raise RuntimeError("oracle_adjoint_ent failed")
     if want_state:
         return grad, E, psi0[..., 0] + 1j * psi0[..., 1]
     return grad, E

@@ -26,7 +26,10 @@
  * the design notes of the repository):
  *   - R_P(t) = exp(-i t P / 2) for P in {X, Y, Z};
  *   - a layer is Rx(theta[l][q][0]), Ry(theta[l][q][1]), Rz(theta[l][q][2])
- *     on every qubit q, then CZ(q, q+1) for q = 0 .. n-2 (open chain);
+ *     on every qubit q, then CZ(q, q+1) for q = 0 .. n-2 (open chain); other
+ *     bond lists, and CNOT(control, target) instead of CZ on each bond (the
+ *     pages name CNOT gates as the other entangler they fuse, [Deep-dive]
+ *     sec. 3.2), are options;
  *   - the input x is angle-encoded once, Ry(x_q) on |0...0>, before layer 0;
  *   - qubit q is bit q of the amplitude index (qubit 0 = least significant);
  *   - the observable is Z on qubit 0;
@@ -51,7 +54,9 @@
 typedef double complex cplx;
 
 enum { PX = 0, PY = 1, PZ = 2 };
-enum { G_ROT = 0, G_CZ = 1 };
+enum { G_ROT = 0, G_CZ = 1, G_CNOT = 2 };
+/* Entangler kinds: CZ on each bond, or CNOT(control, target) on each bond. */
+enum { ENT_CZ = 0, ENT_CNOT = 1 };
 
 typedef struct {
   cplx m[2][2];
@@ -59,9 +64,9 @@ typedef struct {
 
 /* One gate of the circuit, in the order it is applied. */
 typedef struct {
-  int kind;    /* G_ROT or G_CZ */
+  int kind;    /* G_ROT, G_CZ or G_CNOT */
   int pauli;   /* PX, PY, PZ for G_ROT */
-  int q, q2;   /* target qubit; second qubit for CZ */
+  int q, q2;   /* target qubit; second qubit for CZ; control (q) and target (q2) for CNOT */
   double angle;
   long param;  /* index into theta[L][n][3], or -1 for a fixed (encoding) gate */
 } gate;
@@ -138,6 +143,21 @@ static void apply_cz(cplx* psi, int n, int q1, int q2) {
 #pragma omp parallel for schedule(static) if (n >= PAR_AMP_MIN_QUBITS)
   for (size_t i = 0; i < N; ++i)
     if ((i & m) == m) psi[i] = -psi[i];
+}
+
+/* psi <- CNOT(c, t) psi: where bit c is set, the amplitudes with bit t = 0
+ * and bit t = 1 trade places (X on the target, controlled by c). */
+static void apply_cnot(cplx* psi, int n, int c, int t) {
+  const size_t half = (size_t)1 << (n - 1);
+  const size_t tbit = (size_t)1 << t, cbit = (size_t)1 << c;
+#pragma omp parallel for schedule(static) if (n >= PAR_AMP_MIN_QUBITS)
+  for (size_t k = 0; k < half; ++k) {
+    size_t i0 = ((k >> t) << (t + 1)) | (k & (tbit - 1));
+    if (!(i0 & cbit)) continue;
+    cplx a = psi[i0];
+    psi[i0] = psi[i0 | tbit];
+    psi[i0 | tbit] = a;
+  }
 }
 
 /* <lambda| (d acting on qubit q) |phi>, summed pair by pair (no temporary). */
@@ -223,7 +243,7 @@ static long circuit_len(int n, int L, int nb, int reupload) {
  * every layer starts with the angle encoding Ry(x_q) on every qubit again
  * (data re-uploading); those gates carry no parameter. */
 static void build_circuit(gate* g, int n, int L, const double* x, const double* theta, int nbonds,
-                          const int* bonds, int reupload) {
+                          const int* bonds, int reupload, int ent) {
   long k = 0;
   for (int q = 0; q < n; ++q) { /* angle encoding Ry(x_q)|0> */
     gate e = {G_ROT, PY, q, -1, x[q], -1};
@@ -242,8 +262,9 @@ static void build_circuit(gate* g, int n, int L, const double* x, const double* 
         gate r = {G_ROT, a, q, -1, theta[pi], pi};
         g[k++] = r;
       }
-    for (int e = 0; e < nb; ++e) { /* CZ entangler */
-      gate c = {G_CZ, 0, bonds ? bonds[2 * e] : e, bonds ? bonds[2 * e + 1] : e + 1, 0.0, -1};
+    for (int e = 0; e < nb; ++e) { /* entangler: CZ or CNOT(control, target) per bond, in list order */
+      gate c = {ent == ENT_CNOT ? G_CNOT : G_CZ, 0, bonds ? bonds[2 * e] : e, bonds ? bonds[2 * e + 1] : e + 1,
+                0.0, -1};
       g[k++] = c;
     }
   }
@@ -262,6 +283,8 @@ static int bad_bonds(int n, int nbonds, const int* bonds) {
 static void apply_gate(cplx* psi, int n, const gate* g, int inverse) {
   if (g->kind == G_CZ) {
     apply_cz(psi, n, g->q, g->q2); /* CZ is its own inverse */
+  } else if (g->kind == G_CNOT) {
+    apply_cnot(psi, n, g->q, g->q2); /* so is CNOT */
   } else {
     mat2 u = rotation(g->pauli, g->angle);
     apply_1q(psi, n, g->q, inverse ? dagger(u) : u);
@@ -275,7 +298,7 @@ static void zero_state(cplx* psi, int n) {
 
 /* ----------------------------------------------------------------- exports */
 
-int oracle_version(void) { return 4; }
+int oracle_version(void) { return 5; }
 
 int oracle_num_threads(void) {
 #ifdef _OPENMP
@@ -296,10 +319,11 @@ static int bad_args(int n, int L, int B) { return n < 1 || n > 30 || L < 0 || B 
  *   psi    [B][2^n][2] out: final state as (re, im) doubles    (may be NULL)
  * Returns 0, or -1 on bad arguments / allocation failure.
  */
-int oracle_forward_gen(int n, int L, int B, const double* x, const double* theta, int reupload, int nbonds,
-                       const int* bonds, int nterms, const char* paulis, const double* coef, double* expect,
-                       double* psi_out) {
+int oracle_forward_ent(int n, int L, int B, const double* x, const double* theta, int reupload, int ent,
+                       int nbonds, const int* bonds, int nterms, const char* paulis, const double* coef,
+                       double* expect, double* psi_out) {
   if (bad_args(n, L, B) || nterms < 0 || (nterms > 0 && (!paulis || !coef)) || bad_bonds(n, nbonds, bonds)) return -1;
+  if (ent != ENT_CZ && ent != ENT_CNOT) return -1;
   const size_t N = (size_t)1 << n;
   const long ng = circuit_len(n, L, n_bonds_of(n, nbonds, bonds), reupload);
   int err = 0;
@@ -313,7 +337,7 @@ int oracle_forward_gen(int n, int L, int B, const double* x, const double* theta
     if (!g || !psi || (nterms && (!hp || !tmp))) {
       err |= 1;
     } else {
-      build_circuit(g, n, L, x + (size_t)b * n, theta, nbonds, bonds, reupload);
+      build_circuit(g, n, L, x + (size_t)b * n, theta, nbonds, bonds, reupload, ent);
       zero_state(psi, n);
       for (long k = 0; k < ng; ++k) apply_gate(psi, n, &g[k], 0);
       if (expect) {
@@ -333,6 +357,14 @@ int oracle_forward_gen(int n, int L, int B, const double* x, const double* theta
     free(tmp);
   }
   return err ? -1 : 0;
+}
+
+/* Forward pass with CZ entanglers. */
+int oracle_forward_gen(int n, int L, int B, const double* x, const double* theta, int reupload, int nbonds,
+                       const int* bonds, int nterms, const char* paulis, const double* coef, double* expect,
+                       double* psi_out) {
+  return oracle_forward_ent(n, L, B, x, theta, reupload, ENT_CZ, nbonds, bonds, nterms, paulis, coef, expect,
+                            psi_out);
 }
 
 /* Forward pass with the CZ chain and an observable. */
@@ -363,10 +395,11 @@ int oracle_forward(int n, int L, int B, const double* x, const double* theta, do
  *     lambda <- U_j^dagger lambda                  (lambda_{j-1})
  * and for CZ both states are multiplied by CZ.
  */
-int oracle_adjoint_gen(int n, int L, int B, const double* x, const double* theta, int reupload, int nbonds,
-                       const int* bonds, int nterms, const char* paulis, const double* coef, const double* gseed,
-                       double* grad, double* expect, double* psi0_out) {
+int oracle_adjoint_ent(int n, int L, int B, const double* x, const double* theta, int reupload, int ent,
+                       int nbonds, const int* bonds, int nterms, const char* paulis, const double* coef,
+                       const double* gseed, double* grad, double* expect, double* psi0_out) {
   if (bad_args(n, L, B) || nterms < 0 || (nterms > 0 && (!paulis || !coef)) || bad_bonds(n, nbonds, bonds)) return -1;
+  if (ent != ENT_CZ && ent != ENT_CNOT) return -1;
   const size_t N = (size_t)1 << n;
   const long ng = circuit_len(n, L, n_bonds_of(n, nbonds, bonds), reupload);
   const long P = (long)L * n * 3;
@@ -384,7 +417,7 @@ int oracle_adjoint_gen(int n, int L, int B, const double* x, const double* theta
       err |= 1;
     } else {
       double* gb = per + (size_t)b * P;
-      build_circuit(g, n, L, x + (size_t)b * n, theta, nbonds, bonds, reupload);
+      build_circuit(g, n, L, x + (size_t)b * n, theta, nbonds, bonds, reupload, ent);
       zero_state(psi, n);
       for (long k = 0; k < ng; ++k) apply_gate(psi, n, &g[k], 0);
       /* lambda_M = dL/dE * H psi_M  (the derivative of <psi|H|psi> w.r.t. <psi|) */
@@ -402,6 +435,11 @@ int oracle_adjoint_gen(int n, int L, int B, const double* x, const double* theta
         if (gk->kind == G_CZ) {
           apply_cz(psi, n, gk->q, gk->q2);
           apply_cz(lam, n, gk->q, gk->q2);
+          continue;
+        }
+        if (gk->kind == G_CNOT) {
+          apply_cnot(psi, n, gk->q, gk->q2);
+          apply_cnot(lam, n, gk->q, gk->q2);
           continue;
         }
         mat2 ud = dagger(rotation(gk->pauli, gk->angle));
@@ -429,6 +467,14 @@ int oracle_adjoint_gen(int n, int L, int B, const double* x, const double* theta
   }
   free(per);
   return err ? -1 : 0;
+}
+
+/* Adjoint gradient with CZ entanglers. */
+int oracle_adjoint_gen(int n, int L, int B, const double* x, const double* theta, int reupload, int nbonds,
+                       const int* bonds, int nterms, const char* paulis, const double* coef, const double* gseed,
+                       double* grad, double* expect, double* psi0_out) {
+  return oracle_adjoint_ent(n, L, B, x, theta, reupload, ENT_CZ, nbonds, bonds, nterms, paulis, coef, gseed, grad,
+                            expect, psi0_out);
 }
 
 /* Adjoint gradient with the CZ chain and an observable. */

@@ -559,3 +559,95 @@ def test_reupload_returns_to_the_zero_state():
     ref = np.zeros_like(psi0)
     ref[:, 0] = 1.0
     np.testing.assert_allclose(psi0, ref, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# CNOT entanglers: every layer ends with CNOT(control, target) on each pair of
+# a list, in list order (the pages name CNOT gates as the other entangler their
+# kernels fuse).  Pinned by a dense CNOT built from projectors, by the exact
+# action on computational basis states (a CNOT ladder maps bit k to the XOR of
+# bits 0..k) and by the parameter-shift rule.
+
+
+def dense_cnot(c, t, n):
+    """|0><0|_c (x) I + |1><1|_c (x) X_t, as a 2^n matrix."""
+    p0 = np.array([[1, 0], [0, 0]], dtype=complex)
+    p1 = np.array([[0, 0], [0, 1]], dtype=complex)
+    return dense_on(p0, c, n) + dense_on(p1, c, n) @ dense_on(PAULI[0], t, n)
+
+
+def dense_state_cnot(x, theta, pairs):
+    n = x.shape[0]
+    psi = np.zeros(1 << n, dtype=complex)
+    psi[0] = 1
+    for q in range(n):
+        psi = dense_on(dense_rot(1, x[q]), q, n) @ psi
+    for l in range(theta.shape[0]):
+        for q in range(n):
+            for a in range(3):
+                psi = dense_on(dense_rot(a, theta[l, q, a]), q, n) @ psi
+        for c, t in pairs:
+            psi = dense_cnot(c, t, n) @ psi
+    return psi
+
+
+@pytest.mark.parametrize("n,L,seed,kind", [(2, 3, 81, "ladder"), (3, 2, 82, "ladder"), (4, 3, 83, "ring"),
+                                           (5, 2, 84, "random")])
+def test_cnot_dense_brute_force(n, L, seed, kind):
+    rng = np.random.default_rng(seed)
+    if kind == "ladder":
+        pairs = [(q, q + 1) for q in range(n - 1)]
+    elif kind == "ring":
+        pairs = [(q, (q + 1) % n) for q in range(n)]
+    else:
+        pairs = random_bonds(rng, n, n + 1)
+    x, theta, y = random_case(seed, 2, n, L)
+    Z0 = dense_on(PAULI[2], 0, n)
+
+    def dense_fwd(xx, tt):
+        return np.array([float(np.real(np.conj(p) @ (Z0 @ p)))
+                         for p in (dense_state_cnot(xx[b], tt, pairs) for b in range(xx.shape[0]))])
+
+    E, psi = oracle.forward(x, theta, want_state=True, bonds=pairs, entangler="cnot")
+    np.testing.assert_allclose(psi[0], dense_state_cnot(x[0], theta, pairs), atol=1e-12)
+    np.testing.assert_allclose(E, dense_fwd(x, theta), atol=1e-12)
+    g = oracle.loss_seed(E, y)
+    grad, _ = oracle.adjoint(x, theta, g, bonds=pairs, entangler="cnot")
+    want = np.einsum("b,b...->...", g, shift_grad_E(dense_fwd, x, theta))
+    np.testing.assert_allclose(grad, want, atol=1e-11)
+
+
+@pytest.mark.parametrize("n,L", [(3, 1), (5, 2), (7, 3)])
+def test_cnot_ladder_on_basis_states(n, L):
+    """x in {0, pi} encodes a basis state (Ry(pi)|0> = |1>); with theta = 0 each
+    ladder layer replaces bit k by the XOR of bits 0..k."""
+    rng = np.random.default_rng(90 + n)
+    bits = rng.integers(0, 2, size=(4, n))
+    x = bits * np.pi
+    theta = np.zeros((L, n, 3))
+    pairs = [(q, q + 1) for q in range(n - 1)]
+    _, psi = oracle.forward(x, theta, want_state=True, bonds=pairs, entangler="cnot")
+    for b in range(4):
+        v = list(bits[b])
+        for _ in range(L):
+            v = [int(np.bitwise_xor.reduce(v[:k + 1])) for k in range(n)]
+        want = sum(bit << k for k, bit in enumerate(v))
+        assert abs(abs(psi[b, want]) - 1.0) < 1e-12
+        assert np.sum(np.abs(psi[b]) ** 2) - abs(psi[b, want]) ** 2 < 1e-24
+
+
+def test_cnot_control_and_target_are_not_interchangeable():
+    """CNOT(0, 1) on |01> (qubit 0 set) gives |11>; CNOT(1, 0) leaves it."""
+    x = np.array([[np.pi, 0.0]])
+    theta = np.zeros((1, 2, 3))
+    _, a = oracle.forward(x, theta, want_state=True, bonds=[(0, 1)], entangler="cnot")
+    _, b = oracle.forward(x, theta, want_state=True, bonds=[(1, 0)], entangler="cnot")
+    assert abs(abs(a[0, 3]) - 1) < 1e-12 and abs(abs(b[0, 1]) - 1) < 1e-12
+
+
+def test_cnot_returns_to_the_zero_state():
+    x, theta, y = random_case(95, 3, 6, 4)
+    pairs = [(q, q + 1) for q in range(5)]
+    E = oracle.forward(x, theta, bonds=pairs, entangler="cnot")
+    _, _, psi0 = oracle.adjoint(x, theta, oracle.loss_seed(E, y), want_state=True, bonds=pairs, entangler="cnot")
+    assert np.max(np.abs(psi0[:, 0] - 1)) < 1e-12 and np.max(np.abs(psi0[:, 1:])) < 1e-12
