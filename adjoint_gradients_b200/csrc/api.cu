@@ -27,6 +27,7 @@ size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 struct Layout {
   size_t status, passes, slot_pass, slot_index;
   size_t coef_fwd, coef_inv, enc, dummy, exp_partial, partials, obs_groups, obs_terms, ckpt;
+  size_t scratch, dummy2, sub_passes, sub_slot_pass, sub_slot_index;  // CNOT entanglers only
   size_t base_total;
   // host-step extras
   size_t h_psi, h_lam, h_x, h_theta, h_y, h_E, h_g, h_loss, h_grad;
@@ -77,7 +78,7 @@ struct qml_ctx {
   // tensor maps of the passes that load by tensor copies, keyed by the view
   // of the tile and by the buffers they were encoded for
   struct MapEntry {
-    int pass;  // a pass with this view
+    DevPass view;  // a pass with this view
     bool backward;
     int B;
     const void *buf0, *buf1;
@@ -92,6 +93,15 @@ struct qml_ctx {
   Bonds bonds;
   uint32_t nb[kMaxQubits] = {0}, nbhi[kMaxQubits] = {0};
   bool reupload = false;  // every layer starts with the encoding again
+  // CNOT entanglers (qml_set_entangler_cnot): every layer's rotations run as
+  // the passes of a one-layer schedule (sub[v], v = 2 * encodes + stores the
+  // standard layout), and the layer's CNOT list as a gather between buffers
+  bool cnot = false;
+  std::vector<std::pair<int, int>> cnot_pairs;
+  LinMap cnot_fwd{}, cnot_bwd{};  // M^-1 (apply) and M (un-apply) of a layer's CNOT list
+  Plan plan1;
+  std::vector<DevPass> sub[4];
+  bool sub_uploaded = false;
   bool f64 = false;       // fp64 compute mode (qml_create_f64)
   std::vector<uint32_t> f64_mask;  // fp64: tile qubits of each pass
   int f64_tmax = 0;                // fp64: largest tile (qubits)
@@ -178,6 +188,13 @@ void compute_layout(qml_ctx* c) {
   l.obs_terms = take(sizeof(ObsTerm) * QML_MAX_OBS_TERMS);
   const size_t slot_elem = slot_bytes(c);
   l.ckpt = take(slot_elem * (size_t)c->plan.n_ckpt * Bm * (size_t)N + 16);
+  if (c->cnot) {  // second state buffer and partner plane for the gathers, the one-layer schedules
+    l.scratch = take(sizeof(float2) * (size_t)Bm * N);
+    l.dummy2 = take(sizeof(float2) * (size_t)N);
+    l.sub_passes = take(sizeof(DevPass) * 4 * c->sub[0].size());
+    l.sub_slot_pass = take(sizeof(int) * (size_t)n);
+    l.sub_slot_index = take(sizeof(int) * (size_t)n);
+  }
   l.base_total = o;
   const size_t fe = c->f64 ? sizeof(double) : sizeof(float);  // real element of the host-step buffers
   l.h_psi = take(2 * fe * (size_t)Bm * N);
@@ -196,6 +213,15 @@ void compute_layout(qml_ctx* c) {
     p.partial_off = off;
     off += (long long)c->grid_bwd * p.nslots * 3;
   }
+  // one-layer schedules: one layer's partials at a time, in the same area
+  for (auto& v : c->sub) {
+    long long o2 = 0;
+    for (DevPass& p : v) {
+      p.partial_off = o2;
+      o2 += (long long)c->grid_bwd * p.nslots * 3;
+    }
+  }
+  c->sub_uploaded = false;
 }
 
 cudaEvent_t take_event(qml_ctx* c) {
@@ -251,19 +277,23 @@ bool same_tma_view(const DevPass& x, const DevPass& y) {
 }
 
 // Tensor maps for pass p over (buf0, buf1), encoded once per view and buffers.
-const PassMaps* pass_maps(qml_ctx* c, int p, bool backward, int B, const void* buf0, const void* buf1) {
+const PassMaps* pass_maps_for(qml_ctx* c, const DevPass& dp, bool backward, int B, const void* buf0,
+                              const void* buf1) {
   static const PassMaps none{};
-  const DevPass& dp = c->dpass[p];
   if (!dp.tma || !buf0) return &none;
   for (const qml_ctx::MapEntry& m : c->maps)
-    if (m.backward == backward && m.B == B && m.buf0 == buf0 && m.buf1 == buf1 && same_tma_view(c->dpass[m.pass], dp))
+    if (m.backward == backward && m.B == B && m.buf0 == buf0 && m.buf1 == buf1 && same_tma_view(m.view, dp))
       return &m.maps;
   qml_ctx::MapEntry m{};
-  m.pass = p, m.backward = backward, m.B = B, m.buf0 = buf0, m.buf1 = buf1;
+  m.view = dp, m.backward = backward, m.B = B, m.buf0 = buf0, m.buf1 = buf1;
   if (encode_pass_maps(dp, c->cfg.n_qubits, B, backward, buf0, buf1, &m.maps) != cudaSuccess) return nullptr;
   if (c->maps.size() >= 64) c->maps.clear();
   c->maps.push_back(m);
   return &c->maps.back().maps;
+}
+
+const PassMaps* pass_maps(qml_ctx* c, int p, bool backward, int B, const void* buf0, const void* buf1) {
+  return pass_maps_for(c, c->dpass[p], backward, B, buf0, buf1);
 }
 
 // Copy the observable's terms into the workspace if they changed since the
@@ -322,8 +352,208 @@ cudaError_t convert_layout(qml_ctx* c, float2* buf, int B, bool to_working, cuda
   return launch_permute_bits(buf, (long long)B << n, cb, to, c->sms, s);
 }
 
+// ------------------------------------------------------------ CNOT entanglers
+
+// Upload the one-layer schedules (pageable host memory: the copy may wait
+// for the stream) once per workspace layout.
+cudaError_t upload_sub(qml_ctx* c, cudaStream_t s) {
+  if (c->sub_uploaded) return cudaSuccess;
+  const size_t P1 = c->sub[0].size();
+  cudaError_t e = cudaSuccess;
+  for (int v = 0; v < 4 && e == cudaSuccess; ++v)
+    e = cudaMemcpyAsync(c->ws + c->lay.sub_passes + sizeof(DevPass) * P1 * v, c->sub[v].data(),
+                        sizeof(DevPass) * P1, cudaMemcpyHostToDevice, s);
+  std::vector<int> sp(c->plan1.slot_pass.begin(), c->plan1.slot_pass.end());
+  std::vector<int> si(c->plan1.slot_index.begin(), c->plan1.slot_index.end());
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(c->ws + c->lay.sub_slot_pass, sp.data(), sizeof(int) * sp.size(), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(c->ws + c->lay.sub_slot_index, si.data(), sizeof(int) * si.size(), cudaMemcpyHostToDevice,
+                        s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);  // the host vectors above are temporaries
+  if (e == cudaSuccess) c->sub_uploaded = true;
+  return e;
+}
+
+// Schedule variant of layer l: the first layer encodes, the last one leaves
+// the standard layout.
+int sub_variant(int l, int L) { return (l == 0 ? 2 : 0) + (l == L - 1 ? 1 : 0); }
+
+qml_status run_forward_cnot(qml_ctx* c, const float* theta, const float* x, int B, float2* psi, float* expect,
+                            cudaStream_t s) {
+  const int n = c->cfg.n_qubits, L = c->cfg.n_layers, cb = c->cfg.ckpt_block;
+  if (c->ws_bytes < c->lay.base_total) return QML_ERR_WORKSPACE;
+  cudaError_t e = upload_sub(c, s);
+  if (e != cudaSuccess) return QML_ERR_CUDA;
+  const int P1 = (int)c->sub[0].size();
+  float4* cf = at<float4>(c, c->lay.coef_fwd);
+  float4* ci = at<float4>(c, c->lay.coef_inv);
+  e = launch_prep_enc(x, B, n, at<float2>(c, c->lay.enc), s);
+  if (e != cudaSuccess) return QML_ERR_CUDA;
+  PassArgs a{};
+  a.region = c->region;
+  a.n = n;
+  a.B = B;
+  a.U = (B + 1) / 2;
+  a.N = c->N;
+  a.enc = at<float2>(c, c->lay.enc);
+  a.ckpt = c->ws + c->lay.ckpt;
+  a.storage = c->cfg.storage == QML_STORE_BF16 ? 1 : 0;
+  a.bmax = c->cfg.max_batch;
+  a.status = at<unsigned>(c, c->lay.status);
+  a.reupload = c->reupload ? 1 : 0;  // CZ neighbour masks stay zero: no CZ in this mode
+  float2* cur = psi;
+  float2* other = at<float2>(c, c->lay.scratch);
+  float2* part = at<float2>(c, c->lay.dummy);  // partner plane of an odd batch's last unit
+  float2* part_other = at<float2>(c, c->lay.dummy2);
+  c->launches += 1;
+  for (int l = 0; l < L; ++l) {
+    const int v = sub_variant(l, L);
+    const DevPass* dsub = at<DevPass>(c, c->lay.sub_passes) + (size_t)P1 * v;
+    e = launch_prep_pass_coef(dsub, P1, theta + (size_t)l * n * 3, cf, ci, s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+    ++c->launches;
+    qml_ctx::Span sp{};
+    const bool timed = span_begin(c, s, &sp, false);
+    for (int p = 0; p < P1; ++p) {
+      const DevPass& dp = c->sub[v][p];
+      a.n_tiles = (int)(((a.U + (1ll << dp.unit_bits) - 1) >> dp.unit_bits) << dp.n_out);
+      a.buf0 = cur;
+      a.dummy = part;
+      e = copy_pass_coef(c->region, cf + (size_t)p * kMaxSlots * 4, dp.nslots, s);
+      if (e != cudaSuccess) return QML_ERR_CUDA;
+      const PassMaps* maps = pass_maps_for(c, dp, false, B, cur, part);
+      if (!maps) return QML_ERR_CUDA;
+      e = launch_pass(false, a, dp, *maps, c->grid_fwd, c->smem, s);
+      if (e != cudaSuccess) return QML_ERR_CUDA;
+      ++c->launches;
+    }
+    if (timed) {
+      sp.passes = P1;
+      span_end(c, s, &sp);
+    }
+    // the layer's CNOT list: psi'(j) = psi(M^-1 j), on every plane
+    e = launch_gather_bits(cur, other, n, B, c->cnot_fwd, c->sms, s);
+    if (e == cudaSuccess && (B & 1) && l + 1 < L) e = launch_gather_bits(part, part_other, n, 1, c->cnot_fwd, c->sms, s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+    c->launches += (B & 1) && l + 1 < L ? 2 : 1;
+    std::swap(cur, other);
+    std::swap(part, part_other);
+    if (cb > 0 && (l + 1) % cb == 0 && l + 1 < L) {  // slot m holds the state after layer (m + 1) b - 1
+      const int m = (l + 1) / cb - 1;
+      void* slot = c->ws + c->lay.ckpt + slot_bytes(c) * (size_t)m * c->cfg.max_batch * (size_t)c->N;
+      e = launch_slot_from_planes(cur, part, slot, a.storage, B, n, c->sms, s);
+      if (e != cudaSuccess) return QML_ERR_CUDA;
+      ++c->launches;
+      c->ckpt_batch[m] = B;
+    }
+  }
+  if (cur != psi) {
+    e = cudaMemcpyAsync(psi, cur, sizeof(float2) * (size_t)B * c->N, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+  }
+  if (expect) {
+    c->launches += 2;
+    e = launch_expectation(c, psi, B, expect, s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+  }
+  return QML_OK;
+}
+
+qml_status run_backward_cnot(qml_ctx* c, const float* theta, const float* x, int B, float2* psi, float2* lam,
+                             const float* g, float* grad, cudaStream_t s) {
+  const int n = c->cfg.n_qubits, L = c->cfg.n_layers, cb = c->cfg.ckpt_block;
+  if (c->ws_bytes < c->lay.base_total) return QML_ERR_WORKSPACE;
+  for (int m = 0; m < c->plan.n_ckpt; ++m)
+    if (c->ckpt_batch[m] != B) return QML_ERR_CKPT_MISMATCH;
+  cudaError_t e = upload_sub(c, s);
+  if (e != cudaSuccess) return QML_ERR_CUDA;
+  const int P1 = (int)c->sub[0].size();
+  float4* cf = at<float4>(c, c->lay.coef_fwd);
+  float4* ci = at<float4>(c, c->lay.coef_inv);
+  if (c->obs_terms.empty()) {
+    e = launch_bwd_init(psi, lam, g, B, n, s);
+  } else {
+    e = upload_observable(c, s);
+    if (e == cudaSuccess)
+      e = launch_obs_bwd_init(psi, lam, g, B, n, at<ObsGroup>(c, c->lay.obs_groups), (int)c->obs_groups.size(),
+                              at<ObsTerm>(c, c->lay.obs_terms), s);
+  }
+  if (e != cudaSuccess) return QML_ERR_CUDA;
+  if (c->reupload) {
+    e = launch_prep_enc(x, B, n, at<float2>(c, c->lay.enc), s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+  }
+  PassArgs a{};
+  a.region = c->region;
+  a.n = n;
+  a.B = B;
+  a.U = B;
+  a.N = c->N;
+  a.enc = at<float2>(c, c->lay.enc);
+  a.g = g;
+  a.ckpt = c->ws + c->lay.ckpt;
+  a.storage = c->cfg.storage == QML_STORE_BF16 ? 1 : 0;
+  a.bmax = c->cfg.max_batch;
+  a.partials = at<float>(c, c->lay.partials);
+  a.status = at<unsigned>(c, c->lay.status);
+  a.reupload = c->reupload ? 1 : 0;
+  float2* b0 = psi;  // plane 0: (Re psi, Re lambda)
+  float2* b1 = lam;  // plane 1: (Im psi, Im lambda)
+  float2* sc = at<float2>(c, c->lay.scratch);
+  c->launches += 1;
+  for (int l = L - 1; l >= 0; --l) {
+    if (cb > 0 && (l + 1) % cb == 0 && l + 1 < L) {  // the stored state after layer l replaces the uncomputed one
+      const int m = (l + 1) / cb - 1;
+      const void* slot = c->ws + c->lay.ckpt + slot_bytes(c) * (size_t)m * c->cfg.max_batch * (size_t)c->N;
+      e = launch_restore_planes(b0, b1, slot, a.storage, (long long)B * c->N, c->sms, s);
+      if (e != cudaSuccess) return QML_ERR_CUDA;
+      ++c->launches;
+    }
+    // un-apply the layer's CNOT list: psi(b) = psi'(M b), on both planes
+    e = launch_gather_bits(b0, sc, n, B, c->cnot_bwd, c->sms, s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+    std::swap(b0, sc);
+    e = launch_gather_bits(b1, sc, n, B, c->cnot_bwd, c->sms, s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+    std::swap(b1, sc);
+    c->launches += 2;
+    const int v = sub_variant(l, L);
+    const DevPass* dsub = at<DevPass>(c, c->lay.sub_passes) + (size_t)P1 * v;
+    e = launch_prep_pass_coef(dsub, P1, theta + (size_t)l * n * 3, cf, ci, s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+    ++c->launches;
+    qml_ctx::Span sp{};
+    const bool timed = span_begin(c, s, &sp, true);
+    for (int p = P1 - 1; p >= 0; --p) {
+      const DevPass& dp = c->sub[v][p];
+      a.n_tiles = (int)(((a.U + (1ll << dp.unit_bits) - 1) >> dp.unit_bits) << dp.n_out);
+      a.buf0 = b0;
+      a.buf1 = b1;
+      e = copy_pass_coef(c->region, ci + (size_t)p * kMaxSlots * 4, dp.nslots, s);
+      if (e != cudaSuccess) return QML_ERR_CUDA;
+      const PassMaps* maps = pass_maps_for(c, dp, true, B, b0, b1);
+      if (!maps) return QML_ERR_CUDA;
+      e = launch_pass(true, a, dp, *maps, c->grid_bwd, c->smem, s);
+      if (e != cudaSuccess) return QML_ERR_CUDA;
+      ++c->launches;
+    }
+    if (timed) {
+      sp.passes = P1;
+      span_end(c, s, &sp);
+    }
+    e = launch_grad_reduce(dsub, at<int>(c, c->lay.sub_slot_pass), at<int>(c, c->lay.sub_slot_index),
+                           at<float>(c, c->lay.partials), c->grid_bwd, theta + (size_t)l * n * 3, 1, n,
+                           grad + (size_t)l * n * 3, at<unsigned>(c, c->lay.status), s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+    ++c->launches;
+  }
+  return QML_OK;
+}
+
 qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, float2* psi,
                        float* expect, cudaStream_t s) {
+  if (c->cnot) return run_forward_cnot(c, theta, x, B, psi, expect, s);
   const int n = c->cfg.n_qubits;
   const int P = (int)c->dpass.size();
   float4* cf = at<float4>(c, c->lay.coef_fwd);
@@ -378,6 +608,7 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
 
 qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, float2* psi,
                         float2* lam, const float* g, float* grad, cudaStream_t s) {
+  if (c->cnot) return run_backward_cnot(c, theta, x, B, psi, lam, g, grad, s);
   const int n = c->cfg.n_qubits, L = c->cfg.n_layers;
   const int P = (int)c->dpass.size();
   for (int m = 0; m < c->plan.n_ckpt; ++m)
@@ -799,8 +1030,49 @@ qml_status qml_set_entangler(qml_ctx* c, int n_bonds, const int* bonds) {
   c->bonds = b;
   set_bond_masks(c);
   set_pass_entangler(c->plan, c->bonds, &c->dpass);
+  c->cnot = false;
+  c->cnot_pairs.clear();
   return QML_OK;
 }
+
+qml_status qml_set_entangler_cnot(qml_ctx* c, int n_pairs, const int* pairs) {
+  if (!c || n_pairs < 1 || n_pairs > QML_MAX_BONDS || !pairs) return QML_ERR_INVALID_ARG;
+  const int n = c->cfg.n_qubits;
+  std::vector<std::pair<int, int>> v;
+  for (int e = 0; e < n_pairs; ++e) {
+    const int ct = pairs[2 * e], tg = pairs[2 * e + 1];
+    if (ct < 0 || tg < 0 || ct >= n || tg >= n || ct == tg) return QML_ERR_INVALID_ARG;
+    v.push_back({ct, tg});
+  }
+  if (c->f64 || c->plan.n_sets > 2) return QML_ERR_UNSUPPORTED;  // fp32, up to two qubit sets (n <= 20)
+  Plan p1;
+  if (!make_plan(n, 1, 0, &p1).empty()) return QML_ERR_UNSUPPORTED;
+  std::vector<DevPass> d;
+  flatten_plan(p1, &d);
+  set_pass_entangler(p1, Bonds{}, &d);  // the one-layer passes keep no CZ
+  for (int var = 0; var < 4; ++var) {
+    c->sub[var] = d;
+    const bool encodes = (var & 2) != 0, standard = (var & 1) != 0;
+    if (!encodes) c->sub[var][0].gen = 0;  // later layers load the previous layer's state
+    if (!standard) c->sub[var].back().last = 0;
+  }
+  // the layer's CNOT list as a map of index bits: M (in list order) and M^-1
+  for (int k = 0; k < n; ++k) {
+    uint32_t fwd = 1u << k, inv = 1u << k;
+    for (const auto& e : v) fwd ^= ((fwd >> e.first) & 1u) << e.second;
+    for (auto it = v.rbegin(); it != v.rend(); ++it) inv ^= ((inv >> it->first) & 1u) << it->second;
+    c->cnot_bwd.col[k] = fwd;
+    c->cnot_fwd.col[k] = inv;
+  }
+  for (int k = n; k < kMaxQubits; ++k) c->cnot_bwd.col[k] = c->cnot_fwd.col[k] = 0;
+  c->plan1 = p1;
+  c->cnot_pairs = v;
+  c->cnot = true;
+  compute_layout(c);  // the gathers need a second state buffer in the workspace
+  return QML_OK;
+}
+
+int qml_entangler_kind(const qml_ctx* c) { return c ? (c->cnot ? 1 : 0) : -1; }
 
 qml_status qml_set_reupload(qml_ctx* c, int on) {
   if (!c) return QML_ERR_INVALID_ARG;
@@ -811,7 +1083,9 @@ qml_status qml_set_reupload(qml_ctx* c, int on) {
 
 int qml_reupload(const qml_ctx* c) { return c ? (c->reupload ? 1 : 0) : -1; }
 
-int qml_entangler_bonds(const qml_ctx* c) { return c ? (int)c->bonds.size() : -1; }
+int qml_entangler_bonds(const qml_ctx* c) {
+  return c ? (int)(c->cnot ? c->cnot_pairs.size() : c->bonds.size()) : -1;
+}
 
 int qml_observable_terms(const qml_ctx* c) { return c ? (int)c->obs_terms.size() : -1; }
 

@@ -1,0 +1,108 @@
+// entangle.cu -- CNOT entanglers.
+//
+// A layer's CNOT list (CNOT(c, t): bit t of the index flips where bit c is
+// set; the pages name CNOT gates as the other entangler their kernels fuse by
+// recomputing indices with shifts and masks, [Deep-dive] sec. 3.2) is, as a
+// whole, a linear map M of the index bits over GF(2): the layer sends the
+// amplitude at index b to index M b.  Applying it is therefore a gather,
+// psi'(j) = psi(M^-1 j), and un-applying it the gather psi(b) = psi'(M b).
+// The map is given by the images of single bits (col[k] = image of 2^k).
+// A CNOT moves amplitudes across any tile boundary, so the gather is its own
+// pass between the fused rotation passes, out of place into a second buffer.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "kernels.cuh"
+
+namespace qml {
+
+namespace {
+
+// dst[b][j] = src[b][m(j)] for every sample b, with m(j) = XOR of col[k] over
+// the set bits k of j.  Writes are coalesced; for ladders and rings the
+// sources of a warp stay within a few 32-byte sectors.
+__global__ void gather_bits_kernel(const float2* __restrict__ src, float2* __restrict__ dst, int n,
+                                   long long total, const LinMap m) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  const uint32_t mask = (uint32_t)((1ull << n) - 1);
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += stride) {
+    const uint32_t j = (uint32_t)e & mask;
+    uint32_t s = 0;
+    for (uint32_t r = j; r; r &= r - 1u) s ^= m.col[__ffs(r) - 1];
+    dst[e] = __ldg(&src[(e & ~(long long)mask) | s]);
+  }
+}
+
+// The psi lanes of the backward planes from a checkpoint slot (standard
+// layout): plane0[i].x = Re slot[i], plane1[i].x = Im slot[i].
+__global__ void restore_planes_kernel(float2* plane0, float2* plane1, const void* slot, int storage,
+                                      long long count) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += stride) {
+    float re, im;
+    if (storage == 1) {
+      const __nv_bfloat162 v = reinterpret_cast<const __nv_bfloat162*>(slot)[i];
+      re = __bfloat162float(v.x);
+      im = __bfloat162float(v.y);
+    } else {
+      const float2 v = reinterpret_cast<const float2*>(slot)[i];
+      re = v.x;
+      im = v.y;
+    }
+    plane0[i].x = re;
+    plane1[i].x = im;
+  }
+}
+
+// A checkpoint slot (standard layout, sample-major) from the forward pass's
+// working layout: unit u = samples 2u, 2u+1 keeps (Re psi_2u, Re psi_2u+1) at
+// sample 2u's positions and (Im psi_2u, Im psi_2u+1) at sample 2u+1's (or in
+// `partner` for an odd batch's last unit).
+__global__ void slot_from_planes_kernel(const float2* buf, const float2* partner, void* slot, int storage, int B,
+                                        int n) {
+  const long long N = 1ll << n, count = (long long)B << n;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < count; e += stride) {
+    const int b = (int)(e >> n);
+    const long long i = e & (N - 1);
+    const int u = b >> 1;
+    const float2 p0 = buf[(size_t)(2 * u) * N + i];
+    const float2 p1 = (2 * u + 1 < B) ? buf[(size_t)(2 * u + 1) * N + i] : partner[i];
+    const float re = (b & 1) ? p0.y : p0.x, im = (b & 1) ? p1.y : p1.x;
+    if (storage == 1) reinterpret_cast<__nv_bfloat162*>(slot)[e] = __floats2bfloat162_rn(re, im);
+    else reinterpret_cast<float2*>(slot)[e] = make_float2(re, im);
+  }
+}
+
+unsigned grid_for(long long count, int sms) {
+  const long long blocks = (count + 255) / 256;
+  return (unsigned)std::min<long long>(blocks, (long long)sms * 16);
+}
+
+}  // namespace
+
+cudaError_t launch_gather_bits(const float2* src, float2* dst, int n, int B, const LinMap& m, int sms,
+                               cudaStream_t s) {
+  const long long total = (long long)B << n;
+  if (total == 0) return cudaSuccess;
+  gather_bits_kernel<<<grid_for(total, sms), 256, 0, s>>>(src, dst, n, total, m);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_slot_from_planes(const float2* buf, const float2* partner, void* slot, int storage, int B, int n,
+                                   int sms, cudaStream_t s) {
+  const long long count = (long long)B << n;
+  if (count == 0) return cudaSuccess;
+  slot_from_planes_kernel<<<grid_for(count, sms), 256, 0, s>>>(buf, partner, slot, storage, B, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_restore_planes(float2* plane0, float2* plane1, const void* slot, int storage, long long count,
+                                  int sms, cudaStream_t s) {
+  if (count == 0) return cudaSuccess;
+  restore_planes_kernel<<<grid_for(count, sms), 256, 0, s>>>(plane0, plane1, slot, storage, count);
+  return cudaGetLastError();
+}
+
+}  // namespace qml

@@ -98,6 +98,22 @@ cudaError_t launch_encode(const float* x, int B, int n, float2* psi, cudaStream_
 cudaError_t launch_ckpt_copy(bool save, const float2* psi_in, float2* psi_out, void* slot,
                              int storage, long long count, cudaStream_t s);
 
+// ---------------------------------------------------------- CNOT entanglers
+// A linear map of the index bits over GF(2): col[k] is the image of bit k.
+struct LinMap {
+  uint32_t col[kMaxQubits];
+};
+// dst[b][j] = src[b][m(j)] for b < B, j < 2^n (m linear: XOR of col over j's bits).
+cudaError_t launch_gather_bits(const float2* src, float2* dst, int n, int B, const LinMap& m, int sms,
+                               cudaStream_t s);
+// Checkpoint slot (standard layout, storage 0 fp32 / 1 bf16) from the forward
+// pass's working layout in buf (and partner: an odd batch's last unit).
+cudaError_t launch_slot_from_planes(const float2* buf, const float2* partner, void* slot, int storage, int B, int n,
+                                   int sms, cudaStream_t s);
+// psi lanes of the backward planes from a checkpoint slot (storage 0 fp32, 1 bf16).
+cudaError_t launch_restore_planes(float2* plane0, float2* plane1, const void* slot, int storage, long long count,
+                                  int sms, cudaStream_t s);
+
 // ---------------------------------------------------------------- fp64 mode
 constexpr int kF64Threads = 256;  // threads of an fp64 pass block
 constexpr int kF64Warps = kF64Threads / 32;

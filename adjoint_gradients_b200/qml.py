@@ -34,7 +34,7 @@ EXPORTS = [
     "qml_debug_tile_view", "qml_debug_layouts", "qml_set_observable", "qml_observable_terms",
     "qml_expect_observable", "qml_set_entangler", "qml_entangler_bonds", "qml_set_reupload", "qml_reupload",
     "qml_create_f64", "qml_precision", "qml_forward_expect_f64", "qml_backward_adjoint_f64", "qml_loss_seed_f64",
-    "qml_step_host_f64",
+    "qml_step_host_f64", "qml_set_entangler_cnot", "qml_entangler_kind",
 ]
 
 
@@ -117,6 +117,8 @@ def load_library(path: str = LIB_PATH):
         "qml_backward_adjoint_f64": ([_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp], _i),
         "qml_loss_seed_f64": ([_vp, _vp, _vp, _i, _vp, _vp, _vp], _i),
         "qml_step_host_f64": ([_vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp], _i),
+        "qml_set_entangler_cnot": ([_vp, _i, ctypes.POINTER(_i)], _i),
+        "qml_entangler_kind": ([_vp], _i),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -176,6 +178,7 @@ class Context:
         _check(create(ctypes.byref(cfg), device, ctypes.byref(h)), "qml_create_f64" if self.f64 else "qml_create")
         self._h = h
         self.ws = None
+        self._host_step = host_step
         if workspace:
             self.allocate_workspace(host_step=host_step)
 
@@ -198,6 +201,7 @@ class Context:
     def allocate_workspace(self, host_step: bool = False, stream=None):
         import torch
 
+        self._host_step = host_step
         nbytes = self.workspace_bytes(host_step)
         self.ws = torch.empty(nbytes + 256, dtype=torch.uint8, device=f"cuda:{self.device}")
         base = self.ws.data_ptr()
@@ -224,13 +228,27 @@ class Context:
         coef = (ctypes.c_double * len(observable))(*[float(c) for c, _ in observable])
         _check(self.lib.qml_set_observable(self._h, len(observable), words, coef), "qml_set_observable")
 
-    def set_entangler(self, bonds=None):
-        """CZ bonds [(a, b), ...] ending every layer; None restores the chain (q, q+1)."""
+    def set_entangler(self, bonds=None, kind: str = "cz"):
+        """Pairs [(a, b), ...] ending every layer; None means the chain (q, q+1).
+        kind "cz": CZ on each pair; "cnot": CNOT(control a, target b) on each
+        pair in list order (needs a second state buffer: the workspace is
+        re-allocated when it is too small)."""
         if bonds is None:
             bonds = [(q, q + 1) for q in range(self.n - 1)]
         flat = [int(v) for e in bonds for v in e]
         arr = (ctypes.c_int * max(1, len(flat)))(*flat)
-        _check(self.lib.qml_set_entangler(self._h, len(bonds), arr), "qml_set_entangler")
+        if kind == "cz":
+            _check(self.lib.qml_set_entangler(self._h, len(bonds), arr), "qml_set_entangler")
+        elif kind == "cnot":
+            _check(self.lib.qml_set_entangler_cnot(self._h, len(bonds), arr), "qml_set_entangler_cnot")
+            if self.ws is not None and self.ws.numel() - 256 < self.workspace_bytes(self._host_step):
+                self.allocate_workspace(host_step=self._host_step)
+        else:
+            raise ValueError("kind must be 'cz' or 'cnot'")
+
+    @property
+    def entangler_kind(self) -> str:
+        return "cnot" if self.lib.qml_entangler_kind(self._h) == 1 else "cz"
 
     def set_reupload(self, on: bool = True):
         """Data re-uploading: every layer starts with the encoding Ry(x_q) again."""

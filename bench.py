@@ -120,12 +120,17 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------- helpers
 
-def algorithmic_counts(ctx, w, B, f64=False):
-    """Per-pass algorithmic FMAs and HBM bytes of the forward and backward pass kernels."""
+def algorithmic_counts(ctx, w, B, f64=False, cnot_passes_per_layer=0):
+    """Algorithmic FMAs and HBM bytes per step of the forward and backward pass kernels."""
     sched = ctx.debug_schedule()
     P = sched[0]
     N = 1 << w.n
     amp = B * N
+    rots = w.n * w.L
+    if cnot_passes_per_layer:  # CNOT entanglers: every layer's passes read and write the state once
+        Pc = cnot_passes_per_layer * w.L
+        return {"passes": Pc, "fwd_fma": FMA_FWD_PER_ROT * rots * amp, "bwd_fma": FMA_BWD_PER_ROT * rots * amp,
+                "fwd_bytes": (16 * Pc - 8) * amp, "bwd_bytes": (32 * Pc - 16) * amp}
     # bytes per amplitude moved by each pass, from the schedule flags
     i = 1
     fwd_bytes = bwd_bytes = 0
@@ -141,7 +146,6 @@ def algorithmic_counts(ctx, w, B, f64=False):
         rd = 8 if last else 16
         wr = 0 if gen else 16
         bwd_bytes += rd + wr + (slot_b if ck >= 0 else 0)
-    rots = w.n * w.L
     return {
         "passes": P,
         "fwd_fma": FMA_FWD_PER_ROT * rots * amp,
@@ -252,9 +256,13 @@ def observable_terms(name, n):
 
 
 def entangler_bonds(name, n):
-    """CZ bonds for --entangler."""
+    """Pairs for --entangler (CZ bonds, or (control, target) for the CNOT ladder)."""
     chain = [(q, q + 1) for q in range(n - 1)]
-    return {"chain": chain, "ring": chain + [(n - 1, 0)], "none": []}[name]
+    return {"chain": chain, "ring": chain + [(n - 1, 0)], "none": [], "cnot": chain}[name]
+
+
+def entangler_kind(name):
+    return "cnot" if name == "cnot" else "cz"
 
 
 def run_ours(args):
@@ -293,7 +301,7 @@ def run_ours(args):
     obs = observable_terms(args.observable, w.n)
     ctx.set_observable(obs)
     bonds = entangler_bonds(args.entangler, w.n)
-    ctx.set_entangler(bonds)
+    ctx.set_entangler(bonds, kind=entangler_kind(args.entangler))
     ctx.set_reupload(args.reupload)
     psi = ctx.new_state(B)
     lam = ctx.new_state(B)
@@ -346,16 +354,21 @@ def run_ours(args):
     value = world * B * args.steps / (ms / 1e3)
 
     # ---- roofline of the dominant kernel (the backward pass kernel)
-    cnt = algorithmic_counts(ctx, w, B, f64)
+    cnot_ppl = 0
+    if args.entangler == "cnot":  # passes per layer of the one-layer schedule = the set count
+        cnot_ppl = (w.n + 9) // 10 if w.n > 12 else 1
+    cnt = algorithmic_counts(ctx, w, B, f64, cnot_ppl)
     hbm_peak, peak_src = measured_peaks()
     alu_peak = ALU64_PEAK_TFLOPS if f64 else ALU_PEAK_TFLOPS
     bwd_avg_s = bwd_ms / 1e3 / max(1, bwd_n)
     fwd_avg_s = fwd_ms / 1e3 / max(1, fwd_n)
-    P = cnt["passes"]
-    bwd_tflops = 2 * cnt["bwd_fma"] / P / bwd_avg_s / 1e12
-    fwd_tflops = 2 * cnt["fwd_fma"] / P / fwd_avg_s / 1e12
-    bwd_gbs = cnt["bwd_bytes"] / P / bwd_avg_s / 1e9
-    fwd_gbs = cnt["fwd_bytes"] / P / fwd_avg_s / 1e9
+    # per step: the pass kernels' algorithmic work over their summed event time
+    bwd_step_s = bwd_ms / 1e3 / args.steps
+    fwd_step_s = fwd_ms / 1e3 / args.steps
+    bwd_tflops = 2 * cnt["bwd_fma"] / bwd_step_s / 1e12
+    fwd_tflops = 2 * cnt["fwd_fma"] / fwd_step_s / 1e12
+    bwd_gbs = cnt["bwd_bytes"] / bwd_step_s / 1e9
+    fwd_gbs = cnt["fwd_bytes"] / fwd_step_s / 1e9
     traffic = None
     tfile = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tfile):
@@ -385,7 +398,7 @@ def run_ours(args):
         ctx_h = qml.Context(w.n, w.L, B, ckpt_block=w.ckpt_block, storage=w.storage, device=local, host_step=True,
                             precision=args.precision)
         ctx_h.set_observable(obs)
-        ctx_h.set_entangler(bonds)
+        ctx_h.set_entangler(bonds, kind=entangler_kind(args.entangler))
         ctx_h.set_reupload(args.reupload)
         xh = torch.tensor(x, dtype=fdt).pin_memory()
         th = torch.tensor(theta, dtype=fdt).pin_memory()
@@ -426,7 +439,8 @@ def run_ours(args):
 
     cfg = {**workload_config(w, B, f64), "parallelism": f"dp{world}" if world > 1 else "single",
            "observable": "Z0" if obs is None else f"{args.observable} ({len(obs)} Pauli strings)",
-           "entangler": f"CZ {args.entangler} ({len(bonds)} bonds)",
+           "entangler": (f"CNOT ladder ({len(bonds)} pairs)" if args.entangler == "cnot" else
+                         f"CZ {args.entangler} ({len(bonds)} bonds)"),
            "reupload": bool(args.reupload),
            "peak_hbm_bytes": int(torch.cuda.max_memory_allocated(dev))}
     if w.samples_per_epoch:
@@ -460,8 +474,9 @@ def main():
                     help="n,L,B[,ckpt_block[,storage]]: a custom shape with the workload's seeds (for profiling)")
     ap.add_argument("--observable", default="z0", choices=["z0", "tfim"],
                     help="z0: <Z0> (the workloads' readout); tfim: sum_q Z_q Z_q+1 + 0.9 sum_q X_q")
-    ap.add_argument("--entangler", default="chain", choices=["chain", "ring", "none"],
-                    help="CZ bonds ending every layer: chain (q, q+1) as in the workloads, ring, or none")
+    ap.add_argument("--entangler", default="chain", choices=["chain", "ring", "none", "cnot"],
+                    help="gates ending every layer: CZ chain (q, q+1) as in the workloads, CZ ring, none, "
+                         "or the CNOT ladder (q -> q+1)")
     ap.add_argument("--reupload", action="store_true", help="data re-uploading: the encoding again in every layer")
     ap.add_argument("--precision", default="fp32", choices=["fp32", "fp64"],
                     help="arithmetic of the path: fp32, or fp64 (complex128 state, exact checkpoint slots)")

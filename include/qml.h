@@ -179,8 +179,27 @@ QML_API qml_status qml_expect_z0(qml_ctx* ctx, const float* psi_dev, int B, floa
  * stays in force).  Set it before the forward pass whose backward it serves. */
 QML_API qml_status qml_set_entangler(qml_ctx* ctx, int n_bonds, const int* bonds);
 
-/* Number of bonds of the entangler in force. */
+/* Number of bonds (CZ) or pairs (CNOT) of the entangler in force. */
 QML_API int qml_entangler_bonds(const qml_ctx* ctx);
+
+/* CNOT entanglers for the following forward and backward calls: every layer
+ * ends with CNOT(pairs[2e] -> pairs[2e+1]) (control, target) for e = 0 ..
+ * n_pairs-1 in list order, e.g. the ladder (q, q+1).  The pages name CNOT
+ * gates as the other entangler their kernels fuse by recomputing indices
+ * ([Deep-dive] sec. 3.2).  A layer's CNOT list is a linear map of the index
+ * bits; it moves amplitudes across tiles, so each layer runs its rotations as
+ * the fused passes of a one-layer schedule and then one gather pass into a
+ * second state buffer (the workspace grows by B * 2^n complex64: call
+ * qml_workspace_bytes / qml_set_workspace again after this call if the
+ * workspace was set before; the compute calls return QML_ERR_WORKSPACE until
+ * it is large enough).  Checkpoint slots, observables and re-uploading apply
+ * as with CZ.  QML_ERR_INVALID_ARG on a bad pair or count;
+ * QML_ERR_UNSUPPORTED for fp64 contexts and above 20 qubits.
+ * qml_set_entangler switches back to CZ. */
+QML_API qml_status qml_set_entangler_cnot(qml_ctx* ctx, int n_pairs, const int* pairs);
+
+/* Kind of the entangler in force: 0 CZ, 1 CNOT (-1 for NULL). */
+QML_API int qml_entangler_kind(const qml_ctx* ctx);
 
 /* Data re-uploading for the following forward and backward calls: with
  * on != 0 every layer starts with the angle encoding Ry(x[b][q]) on every
