@@ -433,8 +433,9 @@ qml_status run_forward_cnot(qml_ctx* c, const float* theta, const float* x, int 
       span_end(c, s, &sp);
     }
     // the layer's CNOT list: psi'(j) = psi(M^-1 j), on every plane
-    e = launch_gather_bits(cur, other, n, B, c->cnot_fwd, c->sms, s);
-    if (e == cudaSuccess && (B & 1) && l + 1 < L) e = launch_gather_bits(part, part_other, n, 1, c->cnot_fwd, c->sms, s);
+    e = launch_gather_bits(cur, other, n, B, c->cnot_fwd, c->cnot_bwd, c->sms, s);
+    if (e == cudaSuccess && (B & 1) && l + 1 < L)
+      e = launch_gather_bits(part, part_other, n, 1, c->cnot_fwd, c->cnot_bwd, c->sms, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
     c->launches += (B & 1) && l + 1 < L ? 2 : 1;
     std::swap(cur, other);
@@ -511,10 +512,10 @@ qml_status run_backward_cnot(qml_ctx* c, const float* theta, const float* x, int
       ++c->launches;
     }
     // un-apply the layer's CNOT list: psi(b) = psi'(M b), on both planes
-    e = launch_gather_bits(b0, sc, n, B, c->cnot_bwd, c->sms, s);
+    e = launch_gather_bits(b0, sc, n, B, c->cnot_bwd, c->cnot_fwd, c->sms, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
     std::swap(b0, sc);
-    e = launch_gather_bits(b1, sc, n, B, c->cnot_bwd, c->sms, s);
+    e = launch_gather_bits(b1, sc, n, B, c->cnot_bwd, c->cnot_fwd, c->sms, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
     std::swap(b1, sc);
     c->launches += 2;

@@ -19,19 +19,34 @@ namespace qml {
 
 namespace {
 
-// dst[b][j] = src[b][m(j)] for every sample b, with m(j) = XOR of col[k] over
-// the set bits k of j.  Writes are coalesced; for ladders and rings the
-// sources of a warp stay within a few 32-byte sectors.
-__global__ void gather_bits_kernel(const float2* __restrict__ src, float2* __restrict__ dst, int n,
-                                   long long total, const LinMap m) {
+// Gather dst[b][j] = src[b][m(j)] (SCATTER false), or the same permutation
+// written as a scatter dst[b][m(j)] = src[b][j] (SCATTER true, m being the
+// inverse map), for every sample b; m(j) = XOR of col[k] over the set bits k
+// of j.  The side indexed by e is coalesced; the host picks the form whose
+// other side keeps a warp's 32 consecutive indices close together (for the
+// CNOT ladder M^-1 j = j ^ (j << 1) stays within 64 elements, M j = prefix
+// XOR of j spreads over the whole state).
+template <bool SCATTER>
+__global__ void permute_state_kernel(const float2* __restrict__ src, float2* __restrict__ dst, int n,
+                                     long long total, const LinMap m) {
   const long long stride = (long long)gridDim.x * blockDim.x;
   const uint32_t mask = (uint32_t)((1ull << n) - 1);
   for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += stride) {
     const uint32_t j = (uint32_t)e & mask;
     uint32_t s = 0;
     for (uint32_t r = j; r; r &= r - 1u) s ^= m.col[__ffs(r) - 1];
-    dst[e] = __ldg(&src[(e & ~(long long)mask) | s]);
+    const long long o = (e & ~(long long)mask) | s;
+    if (SCATTER) dst[o] = __ldg(&src[e]);
+    else dst[e] = __ldg(&src[o]);
   }
+}
+
+// Highest index bit that a warp's five lowest index bits reach under m.
+int spread(const LinMap& m, int n) {
+  int hi = 0;
+  for (int k = 0; k < 5 && k < n; ++k)
+    if (m.col[k]) hi = std::max(hi, 31 - __builtin_clz(m.col[k]));
+  return hi;
 }
 
 // The psi lanes of the backward planes from a checkpoint slot (standard
@@ -82,11 +97,14 @@ unsigned grid_for(long long count, int sms) {
 
 }  // namespace
 
-cudaError_t launch_gather_bits(const float2* src, float2* dst, int n, int B, const LinMap& m, int sms,
-                               cudaStream_t s) {
+cudaError_t launch_gather_bits(const float2* src, float2* dst, int n, int B, const LinMap& m, const LinMap& m_inv,
+                               int sms, cudaStream_t s) {
   const long long total = (long long)B << n;
   if (total == 0) return cudaSuccess;
-  gather_bits_kernel<<<grid_for(total, sms), 256, 0, s>>>(src, dst, n, total, m);
+  if (spread(m, n) <= spread(m_inv, n))
+    permute_state_kernel<false><<<grid_for(total, sms), 256, 0, s>>>(src, dst, n, total, m);
+  else
+    permute_state_kernel<true><<<grid_for(total, sms), 256, 0, s>>>(src, dst, n, total, m_inv);
   return cudaGetLastError();
 }
 

@@ -103,9 +103,10 @@ cudaError_t launch_ckpt_copy(bool save, const float2* psi_in, float2* psi_out, v
 struct LinMap {
   uint32_t col[kMaxQubits];
 };
-// dst[b][j] = src[b][m(j)] for b < B, j < 2^n (m linear: XOR of col over j's bits).
-cudaError_t launch_gather_bits(const float2* src, float2* dst, int n, int B, const LinMap& m, int sms,
-                               cudaStream_t s);
+// dst[b][j] = src[b][m(j)] for b < B, j < 2^n (m linear: XOR of col over j's
+// bits; m_inv its inverse, used when the scatter form is the more local one).
+cudaError_t launch_gather_bits(const float2* src, float2* dst, int n, int B, const LinMap& m, const LinMap& m_inv,
+                               int sms, cudaStream_t s);
 // Checkpoint slot (standard layout, storage 0 fp32 / 1 bf16) from the forward
 // pass's working layout in buf (and partner: an odd batch's last unit).
 cudaError_t launch_slot_from_planes(const float2* buf, const float2* partner, void* slot, int storage, int B, int n,
