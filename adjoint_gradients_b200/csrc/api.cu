@@ -734,9 +734,18 @@ qml_status run_forward64(qml_ctx* c, const double* theta, const double* x, int B
   if (timed) span_end(c, s, &sp);
   if (expect) {
     c->launches += 2;
-    if (launch_expect64(psi, B, c->cfg.n_qubits, at<double>(c, c->lay.exp_partial), expect,
-                        at<unsigned>(c, c->lay.status), s) != cudaSuccess)
-      return QML_ERR_CUDA;
+    cudaError_t e;
+    if (c->obs_terms.empty()) {
+      e = launch_expect64(psi, B, c->cfg.n_qubits, at<double>(c, c->lay.exp_partial), expect,
+                          at<unsigned>(c, c->lay.status), s);
+    } else {
+      e = upload_observable(c, s);
+      if (e == cudaSuccess)
+        e = launch_obs_expect64(psi, B, c->cfg.n_qubits, at<ObsGroup>(c, c->lay.obs_groups),
+                                (int)c->obs_groups.size(), at<ObsTerm>(c, c->lay.obs_terms),
+                                at<double>(c, c->lay.exp_partial), expect, at<unsigned>(c, c->lay.status), s);
+    }
+    if (e != cudaSuccess) return QML_ERR_CUDA;
   }
   return QML_OK;
 }
@@ -746,7 +755,16 @@ qml_status run_backward64(qml_ctx* c, const double* theta, const double* x, int 
   const int n = c->cfg.n_qubits, L = c->cfg.n_layers;
   for (int m = 0; m < c->plan.n_ckpt; ++m)
     if (c->ckpt_batch[m] != B) return QML_ERR_CKPT_MISMATCH;
-  if (launch_bwd_init64(psi, lam, g, B, n, s) != cudaSuccess) return QML_ERR_CUDA;
+  cudaError_t e0;
+  if (c->obs_terms.empty()) {
+    e0 = launch_bwd_init64(psi, lam, g, B, n, s);
+  } else {
+    e0 = upload_observable(c, s);
+    if (e0 == cudaSuccess)
+      e0 = launch_obs_bwd_init64(psi, lam, g, B, n, at<ObsGroup>(c, c->lay.obs_groups), (int)c->obs_groups.size(),
+                                 at<ObsTerm>(c, c->lay.obs_terms), s);
+  }
+  if (e0 != cudaSuccess) return QML_ERR_CUDA;
   Pass64Args a = pass64_args(c, theta, x, B, psi, lam);
   c->launches += 2;  // lambda init, gradient reduce
   qml_ctx::Span sp{};
@@ -1219,7 +1237,6 @@ qml_status qml_forward_expect_f64(qml_ctx* c, const double* theta, const double*
   qml_status st = check_ready(c, B, true);
   if (st != QML_OK) return st;
   if (!theta || !x || !psi || !expect || misaligned(psi, 16)) return QML_ERR_INVALID_ARG;
-  if (!c->obs_terms.empty()) return QML_ERR_UNSUPPORTED;  // fp64 mode reads out Z0
   DeviceGuard g(c->device);
   return run_forward64(c, theta, x, B, reinterpret_cast<double2*>(psi), expect, static_cast<cudaStream_t>(stream));
 }
@@ -1232,7 +1249,6 @@ qml_status qml_backward_adjoint_f64(qml_ctx* c, const double* theta, const doubl
     return QML_ERR_INVALID_ARG;
   if (psi == lambda) return QML_ERR_INVALID_ARG;
   if (c->reupload && !x) return QML_ERR_INVALID_ARG;
-  if (!c->obs_terms.empty()) return QML_ERR_UNSUPPORTED;
   DeviceGuard g(c->device);
   return run_backward64(c, theta, x, B, reinterpret_cast<double2*>(psi), reinterpret_cast<double2*>(lambda),
                         dLdE, grad, static_cast<cudaStream_t>(stream));
@@ -1254,7 +1270,6 @@ qml_status qml_step_host_f64(qml_ctx* c, const double* x_h, const double* theta_
   if (st != QML_OK) return st;
   if (!x_h || !theta_h || !y_h || !grad_h) return QML_ERR_INVALID_ARG;
   if (c->ws_bytes < c->lay.host_total) return QML_ERR_WORKSPACE;
-  if (!c->obs_terms.empty()) return QML_ERR_UNSUPPORTED;
   DeviceGuard g(c->device);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int n = c->cfg.n_qubits, L = c->cfg.n_layers;

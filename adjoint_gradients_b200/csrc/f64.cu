@@ -385,6 +385,76 @@ __global__ void expect64_final_kernel(const double* partial, int chunks, int B, 
   if (!isfinite(s) && status) atomicOr(status, kErrNumeric);
 }
 
+// Observable O = sum_k c_k i^ny X^x Z^z with terms grouped by x (the same
+// grouping as the fp32 path): the group's weight at m = j ^ x is
+// sum_k c_k i^ny (-1)^popcount(m & z_k).
+__device__ __forceinline__ double2 obs_weight64(const ObsTerm* t, int count, uint32_t m) {
+  double wr = 0.0, wi = 0.0;
+  for (int k = 0; k < count; ++k) {
+    const double c = (__popc(m & t[k].z) & 1) ? -t[k].c : t[k].c;
+    switch (t[k].ny & 3) {
+      case 0: wr += c; break;
+      case 1: wi += c; break;
+      case 2: wr -= c; break;
+      default: wi -= c; break;
+    }
+  }
+  return make_double2(wr, wi);
+}
+
+// Partial sums of <psi|O|psi> = sum_j sum_groups conj(psi(j)) w(j ^ x) psi(j ^ x)
+// over chunks of 2^16 amplitudes (fp64).
+__global__ void obs64_expect_partial_kernel(const double2* psi, int n, const ObsGroup* groups, int ngroups,
+                                            const ObsTerm* terms, double* partial) {
+  const long long N = 1ll << n;
+  const int chunks = (int)((N + (1ll << kExp64ChunkLog) - 1) >> kExp64ChunkLog);
+  const int b = blockIdx.y, c = blockIdx.x;
+  const long long lo = (long long)c << kExp64ChunkLog;
+  const long long hi = min(N, lo + (1ll << kExp64ChunkLog));
+  const double2* p = psi + (size_t)b * N;
+  double s = 0.0;
+  for (int gi = 0; gi < ngroups; ++gi) {
+    const ObsGroup G = groups[gi];
+    for (long long j = lo + threadIdx.x; j < hi; j += kExp64Threads) {
+      const uint32_t m = (uint32_t)j ^ G.x;
+      const double2 a = p[j], q = p[m];
+      const double wr = a.x * q.x + a.y * q.y;  // conj(a) q
+      const double wi = a.x * q.y - a.y * q.x;
+      const double2 d = obs_weight64(terms + G.first, G.count, m);
+      s += wr * d.x - wi * d.y;
+    }
+  }
+  __shared__ double red[kExp64Threads];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = kExp64Threads / 2; w; w >>= 1) {
+    if ((int)threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) partial[(size_t)b * chunks + c] = red[0];
+}
+
+// lambda = g_b O psi (separate buffer; psi unchanged).
+__global__ void obs64_lambda_kernel(const double2* psi, double2* lam, const double* g, int n, long long tot,
+                                    const ObsGroup* groups, int ngroups, const ObsTerm* terms) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= tot) return;
+  const long long N = 1ll << n;
+  const int b = (int)(idx >> n);
+  const uint32_t j = (uint32_t)(idx & (N - 1));
+  const double2* p = psi + (size_t)b * N;
+  double ar = 0.0, ai = 0.0;
+  for (int gi = 0; gi < ngroups; ++gi) {
+    const ObsGroup G = groups[gi];
+    const uint32_t m = j ^ G.x;
+    const double2 q = p[m];
+    const double2 d = obs_weight64(terms + G.first, G.count, m);
+    ar += d.x * q.x - d.y * q.y;
+    ai += d.x * q.y + d.y * q.x;
+  }
+  lam[idx] = make_double2(g[b] * ar, g[b] * ai);
+}
+
 __global__ void grad_reduce64_kernel(const DevPass* passes, const int* slot_pass, const int* slot_index,
                                      const double* partials, int grid, const double* theta, int L, int n,
                                      double* grad, unsigned* status) {
@@ -477,6 +547,24 @@ cudaError_t launch_expect64(const double2* psi, int B, int n, double* partial, d
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   expect64_final_kernel<<<(B + 127) / 128, 128, 0, s>>>(partial, chunks, B, E, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_obs_expect64(const double2* psi, int B, int n, const ObsGroup* groups, int ngroups,
+                                const ObsTerm* terms, double* partial, double* E, unsigned* status, cudaStream_t s) {
+  const long long N = 1ll << n;
+  const int chunks = (int)((N + (1ll << kExp64ChunkLog) - 1) >> kExp64ChunkLog);
+  obs64_expect_partial_kernel<<<dim3(chunks, B), kExp64Threads, 0, s>>>(psi, n, groups, ngroups, terms, partial);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  expect64_final_kernel<<<(B + 127) / 128, 128, 0, s>>>(partial, chunks, B, E, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_obs_bwd_init64(const double2* psi, double2* lam, const double* g, int B, int n,
+                                  const ObsGroup* groups, int ngroups, const ObsTerm* terms, cudaStream_t s) {
+  const long long tot = (long long)B << n;
+  obs64_lambda_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(psi, lam, g, n, tot, groups, ngroups, terms);
   return cudaGetLastError();
 }
 

@@ -153,5 +153,11 @@ cudaError_t launch_grad_reduce64(const DevPass* passes, const int* slot_pass, co
                                  const double* partials, int grid, const double* theta, int L, int n, double* grad,
                                  unsigned* status, cudaStream_t s);
 cudaError_t launch_loss_seed64(const double* E, const double* y, int B, double* g, double* loss, cudaStream_t s);
+// Pauli-sum observables in fp64: E[b] = <psi_b|O|psi_b> (partial: expect64_partial_count(B, n) doubles), and
+// lambda = g_b O psi (separate buffers).
+cudaError_t launch_obs_expect64(const double2* psi, int B, int n, const ObsGroup* groups, int ngroups,
+                                const ObsTerm* terms, double* partial, double* E, unsigned* status, cudaStream_t s);
+cudaError_t launch_obs_bwd_init64(const double2* psi, double2* lam, const double* g, int B, int n,
+                                  const ObsGroup* groups, int ngroups, const ObsTerm* terms, cudaStream_t s);
 
 }  // namespace qml

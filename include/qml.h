@@ -333,9 +333,9 @@ QML_API int qml_debug_layouts(int* out, int cap);
  * (re, im) double pairs, 16-byte aligned.  Checkpoint slots take the
  * config's storage: QML_STORE_FP64 keeps them exact, QML_STORE_FP32 /
  * QML_STORE_BF16 round them (the backward pass then restarts from the
- * rounded state at each slot).  Entanglers (qml_set_entangler) and data
- * re-uploading (qml_set_reupload, any n) apply; the observable is Z0 (a
- * Pauli-sum observable makes the calls below return QML_ERR_UNSUPPORTED).
+ * rounded state at each slot).  CZ entanglers (qml_set_entangler), data
+ * re-uploading (qml_set_reupload, any n) and Pauli-sum observables
+ * (qml_set_observable, evaluated in fp64) apply.
  * The fp32 calls (qml_forward_expect, qml_backward_adjoint, qml_loss_seed,
  * qml_step_host, qml_init_state_encode, qml_ckpt_save / _restore,
  * qml_expect_z0, qml_expect_observable) return QML_ERR_UNSUPPORTED on an

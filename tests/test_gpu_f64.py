@@ -180,3 +180,23 @@ def test_f64_large_sampled_state():
     assert np.max(np.abs(got[:, 0] + 1j * got[:, 1] - psio[0, idx])) <= 1e-12
     gref, _ = oracle.adjoint(x, theta, g)
     assert np.all(np.abs(grad - gref) <= 1e-10 + 1e-9 * np.abs(gref))
+
+
+@pytest.mark.parametrize("n,L,B,ck", [(6, 3, 3, 1), (14, 2, 3, 1)])
+def test_f64_pauli_sum_observable(n, L, B, ck):
+    """O = a transverse-field Ising sum with a Y term, evaluated and seeded in fp64."""
+    obs = [(1.0, "".join("Z" if k in (q, q + 1) else "I" for k in range(n))) for q in range(n - 1)]
+    obs += [(0.9, "".join("X" if k == q else "I" for k in range(n))) for q in range(n)]
+    obs += [(-0.4, "Y" + "I" * (n - 2) + "X")]
+    x, theta, y = random_case(6700 + n, B, n, L)
+    Eo = oracle.forward(x, theta, observable=obs)
+    g = oracle.loss_seed(Eo, y)
+    ctx = qml().Context(n, L, B, ckpt_block=ck, storage="fp64", precision="fp64")
+    ctx.set_observable(obs)
+    xd, td = dev(x), dev(theta)
+    psi, E = ctx.forward(td, xd)
+    grad = ctx.backward(td, xd, psi, ctx.new_state(B), dev(g)).cpu().numpy()
+    ctx.sync()
+    assert np.max(np.abs(E.cpu().numpy() - Eo)) <= 1e-10
+    gref, _ = oracle.adjoint(x, theta, g, observable=obs)
+    assert np.all(np.abs(grad - gref) <= 1e-9 + 1e-9 * np.abs(gref)), np.max(np.abs(grad - gref))
