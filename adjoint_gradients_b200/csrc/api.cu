@@ -8,6 +8,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <string>
@@ -103,6 +104,8 @@ struct qml_ctx {
   std::vector<DevPass> sub[4];
   bool sub_uploaded = false;
   bool f64 = false;       // fp64 compute mode (qml_create_f64)
+  // host-side fault injection for tests of the error paths (QML_FAULT at create)
+  enum Fault { FAULT_NONE, FAULT_ALLOC, FAULT_CKPT, FAULT_NAN } fault = FAULT_NONE;
   std::vector<uint32_t> f64_mask;  // fp64: tile qubits of each pass
   int f64_tmax = 0;                // fp64: largest tile (qubits)
 };
@@ -559,6 +562,8 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
   const int P = (int)c->dpass.size();
   float4* cf = at<float4>(c, c->lay.coef_fwd);
   cudaError_t e = launch_prep_pass_coef(at<DevPass>(c, c->lay.passes), P, theta, cf, at<float4>(c, c->lay.coef_inv), s);
+  if (e == cudaSuccess && c->fault == qml_ctx::FAULT_NAN)  // injected: the first rotation's coefficients become NaN
+    e = cudaMemsetAsync(cf, 0xff, sizeof(float4), s);
   if (e != cudaSuccess) return QML_ERR_CUDA;
   e = launch_prep_enc(x, B, n, at<float2>(c, c->lay.enc), s);
   if (e != cudaSuccess) return QML_ERR_CUDA;
@@ -596,6 +601,7 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
     ++c->launches;
     if (dp.ckpt >= 0) c->ckpt_batch[dp.ckpt] = B;
   }
+  if (c->fault == qml_ctx::FAULT_CKPT) std::fill(c->ckpt_batch.begin(), c->ckpt_batch.end(), -1);  // injected
   if (timed) span_end(c, s, &sp);
   e = convert_layout(c, psi, B, false, s);  // working-state order -> standard order
   if (e != cudaSuccess) return QML_ERR_CUDA;
@@ -833,6 +839,13 @@ static qml_status create_ctx(const qml_config* cfg, int device, bool f64, qml_ct
   if (!c) return QML_ERR_INVALID_ARG;
   c->cfg = *cfg;
   c->f64 = f64;
+  if (const char* f = std::getenv("QML_FAULT")) {
+    const std::string v(f);
+    c->fault = v == "alloc" ? qml_ctx::FAULT_ALLOC
+               : v == "ckpt_corrupt" ? qml_ctx::FAULT_CKPT
+               : v == "nan_theta" ? qml_ctx::FAULT_NAN
+                                  : qml_ctx::FAULT_NONE;
+  }
   c->device = device;
   c->N = 1ll << cfg->n_qubits;
   std::string err = make_plan(cfg->n_qubits, cfg->n_layers, cfg->ckpt_block, &c->plan);
@@ -883,6 +896,7 @@ size_t qml_host_workspace_bytes(const qml_ctx* cctx, int B) {
 
 qml_status qml_set_workspace(qml_ctx* c, void* ws, size_t bytes, void* stream) {
   if (!c || !ws) return QML_ERR_INVALID_ARG;
+  if (c->fault == qml_ctx::FAULT_ALLOC) return QML_ERR_WORKSPACE;  // injected: as if the buffer were too small
   if (misaligned(ws, kAlign)) return QML_ERR_INVALID_ARG;
   ensure_device(c);
   if (!c->dev_ok) return QML_ERR_CUDA;

@@ -88,7 +88,16 @@ QML_API int qml_abi_version(void);
 QML_API const char* qml_status_str(qml_status s);
 
 /* Create a context for one circuit shape on CUDA device `device`.  Builds the
- * host-side pass schedule; touches no device memory.  *out is NULL on error. */
+ * host-side pass schedule; touches no device memory.  *out is NULL on error.
+ * Fault injection for tests of the error paths, read from the environment at
+ * creation (all on the host; no device fault is ever provoked):
+ *   QML_FAULT=alloc         qml_set_workspace returns QML_ERR_WORKSPACE
+ *   QML_FAULT=ckpt_corrupt  every forward pass leaves its checkpoint slots
+ *                           unrecorded: the backward pass returns
+ *                           QML_ERR_CKPT_MISMATCH
+ *   QML_FAULT=nan_theta     the first rotation's coefficients are NaN in
+ *                           every forward pass: qml_sync returns
+ *                           QML_ERR_NUMERIC */
 QML_API qml_status qml_create(const qml_config* cfg, int device, qml_ctx** out);
 
 /* Destroy a context.  The caller frees the workspace afterwards. */
