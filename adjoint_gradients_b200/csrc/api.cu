@@ -456,6 +456,8 @@ qml_status run_forward_cnot(qml_ctx* c, const float* theta, const float* x, int 
     e = cudaMemcpyAsync(psi, cur, sizeof(float2) * (size_t)B * c->N, cudaMemcpyDeviceToDevice, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
   }
+  e = convert_layout(c, psi, B, false, s);  // working-state order -> standard order (three or more sets)
+  if (e != cudaSuccess) return QML_ERR_CUDA;
   if (expect) {
     c->launches += 2;
     e = launch_expectation(c, psi, B, expect, s);
@@ -483,6 +485,8 @@ qml_status run_backward_cnot(qml_ctx* c, const float* theta, const float* x, int
       e = launch_obs_bwd_init(psi, lam, g, B, n, at<ObsGroup>(c, c->lay.obs_groups), (int)c->obs_groups.size(),
                               at<ObsTerm>(c, c->lay.obs_terms), s);
   }
+  if (e == cudaSuccess) e = convert_layout(c, psi, B, true, s);  // both planes: standard -> working order
+  if (e == cudaSuccess) e = convert_layout(c, lam, B, true, s);
   if (e != cudaSuccess) return QML_ERR_CUDA;
   if (c->reupload) {
     e = launch_prep_enc(x, B, n, at<float2>(c, c->lay.enc), s);
@@ -1077,7 +1081,7 @@ qml_status qml_set_entangler_cnot(qml_ctx* c, int n_pairs, const int* pairs) {
     if (ct < 0 || tg < 0 || ct >= n || tg >= n || ct == tg) return QML_ERR_INVALID_ARG;
     v.push_back({ct, tg});
   }
-  if (c->f64 || c->plan.n_sets > 2) return QML_ERR_UNSUPPORTED;  // fp32, up to two qubit sets (n <= 20)
+  if (c->f64) return QML_ERR_UNSUPPORTED;  // fp32 only
   Plan p1;
   if (!make_plan(n, 1, 0, &p1).empty()) return QML_ERR_UNSUPPORTED;
   std::vector<DevPass> d;
@@ -1089,15 +1093,23 @@ qml_status qml_set_entangler_cnot(qml_ctx* c, int n_pairs, const int* pairs) {
     if (!encodes) c->sub[var][0].gen = 0;  // later layers load the previous layer's state
     if (!standard) c->sub[var].back().last = 0;
   }
-  // the layer's CNOT list as a map of index bits: M (in list order) and M^-1
-  for (int k = 0; k < n; ++k) {
-    uint32_t fwd = 1u << k, inv = 1u << k;
+  // the layer's CNOT list as a map of index bits: M (in list order) and M^-1,
+  // on the working-state addresses (the passes keep the state there; the
+  // map in address bits is M with its input and output bits renamed)
+  auto to_addr = [&](uint32_t qbits) {
+    uint32_t a = 0;
+    for (int q = 0; q < n; ++q)
+      if ((qbits >> q) & 1u) a |= 1u << p1.addr_of[q];
+    return a;
+  };
+  for (int k = 0; k < kMaxQubits; ++k) c->cnot_bwd.col[k] = c->cnot_fwd.col[k] = 0;
+  for (int q = 0; q < n; ++q) {
+    uint32_t fwd = 1u << q, inv = 1u << q;
     for (const auto& e : v) fwd ^= ((fwd >> e.first) & 1u) << e.second;
     for (auto it = v.rbegin(); it != v.rend(); ++it) inv ^= ((inv >> it->first) & 1u) << it->second;
-    c->cnot_bwd.col[k] = fwd;
-    c->cnot_fwd.col[k] = inv;
+    c->cnot_bwd.col[p1.addr_of[q]] = to_addr(fwd);
+    c->cnot_fwd.col[p1.addr_of[q]] = to_addr(inv);
   }
-  for (int k = n; k < kMaxQubits; ++k) c->cnot_bwd.col[k] = c->cnot_fwd.col[k] = 0;
   c->plan1 = p1;
   c->cnot_pairs = v;
   c->cnot = true;

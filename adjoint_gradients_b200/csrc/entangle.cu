@@ -26,28 +26,31 @@ namespace {
 // other side keeps a warp's 32 consecutive indices close together (for the
 // CNOT ladder M^-1 j = j ^ (j << 1) stays within 64 elements, M j = prefix
 // XOR of j spreads over the whole state).
-// m(j) = lo[j & 1023] ^ hi[j >> 10] from two 1024-entry shared tables (n <= 20).
+// m(j) = t0[j & 1023] ^ t1[(j >> 10) & 1023] ^ t2[j >> 20] from three
+// 1024-entry shared tables (n <= 30).
 template <bool SCATTER>
 __global__ void permute_state_kernel(const float2* __restrict__ src, float2* __restrict__ dst, int n,
                                      long long total, const LinMap m) {
-  __shared__ uint32_t lo[1024], hi[1024];
+  __shared__ uint32_t t0[1024], t1[1024], t2[1024];
   for (int i = threadIdx.x; i < 1024; i += blockDim.x) {
-    uint32_t a = 0, b = 0;
+    uint32_t a = 0, b = 0, c = 0;
 #pragma unroll
     for (int k = 0; k < 10; ++k)
       if ((i >> k) & 1) {
         a ^= k < n ? m.col[k] : 0u;
         b ^= k + 10 < n ? m.col[k + 10] : 0u;
+        c ^= k + 20 < n ? m.col[k + 20] : 0u;
       }
-    lo[i] = a;
-    hi[i] = b;
+    t0[i] = a;
+    t1[i] = b;
+    t2[i] = c;
   }
   __syncthreads();
   const long long stride = (long long)gridDim.x * blockDim.x;
   const uint32_t mask = (uint32_t)((1ull << n) - 1);
   for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += stride) {
     const uint32_t j = (uint32_t)e & mask;
-    const uint32_t s = lo[j & 1023u] ^ hi[(j >> 10) & 1023u];
+    const uint32_t s = t0[j & 1023u] ^ t1[(j >> 10) & 1023u] ^ t2[(j >> 20) & 1023u];
     const long long o = (e & ~(long long)mask) | s;
     if (SCATTER) dst[o] = __ldg(&src[e]);
     else dst[e] = __ldg(&src[o]);
@@ -113,7 +116,7 @@ unsigned grid_for(long long count, int sms) {
 cudaError_t launch_gather_bits(const float2* src, float2* dst, int n, int B, const LinMap& m, const LinMap& m_inv,
                                int sms, cudaStream_t s) {
   const long long total = (long long)B << n;
-  if (n > 20) return cudaErrorInvalidValue;  // two 10-bit tables
+  if (n > kMaxQubits) return cudaErrorInvalidValue;  // three 10-bit tables
   if (total == 0) return cudaSuccess;
   if (spread(m, n) <= spread(m_inv, n))
     permute_state_kernel<false><<<grid_for(total, sms), 256, 0, s>>>(src, dst, n, total, m);
