@@ -1081,7 +1081,7 @@ qml_status qml_set_entangler_cnot(qml_ctx* c, int n_pairs, const int* pairs) {
     if (ct < 0 || tg < 0 || ct >= n || tg >= n || ct == tg) return QML_ERR_INVALID_ARG;
     v.push_back({ct, tg});
   }
-  if (c->f64 || c->plan.n_sets > 2) return QML_ERR_UNSUPPORTED;  // fp32, up to two qubit sets (n <= 20)
+  if (c->f64) return QML_ERR_UNSUPPORTED;  // fp32 only
   Plan p1;
   if (!make_plan(n, 1, 0, &p1).empty()) return QML_ERR_UNSUPPORTED;
   std::vector<DevPass> d;

@@ -203,7 +203,7 @@ QML_API int qml_entangler_bonds(const qml_ctx* ctx);
  * workspace was set before; the compute calls return QML_ERR_WORKSPACE until
  * it is large enough).  Checkpoint slots, observables and re-uploading apply
  * as with CZ.  QML_ERR_INVALID_ARG on a bad pair or count;
- * QML_ERR_UNSUPPORTED for fp64 contexts and above 20 qubits.
+ * QML_ERR_UNSUPPORTED for fp64 contexts.
  * qml_set_entangler switches back to CZ. */
 QML_API qml_status qml_set_entangler_cnot(qml_ctx* ctx, int n_pairs, const int* pairs);
 

@@ -44,6 +44,8 @@ CASES = [
     (14, 2, 3, 1, "fp32", "ladder"),
     (17, 3, 2, 0, "fp32", "random"),
     (20, 2, 3, 1, "fp32", "ladder"),
+    (21, 2, 3, 1, "fp32", "ladder"),  # three qubit sets: permuted working-state addresses
+    (23, 2, 1, 0, "fp32", "random"),
 ]
 
 
