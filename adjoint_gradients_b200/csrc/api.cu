@@ -99,7 +99,9 @@ struct qml_ctx {
   // standard layout), and the layer's CNOT list as a gather between buffers
   bool cnot = false;
   std::vector<std::pair<int, int>> cnot_pairs;
-  LinMap cnot_fwd{}, cnot_bwd{};  // M^-1 (apply) and M (un-apply) of a layer's CNOT list
+  LinMap cnot_fwd{}, cnot_bwd{};  // M^-1 (apply) and M (un-apply) of a layer's CNOT list, on addresses
+  LinMap cnot_fwd_q{}, cnot_bwd_q{};  // the same on qubit bits (fp64 mode: standard order)
+  std::vector<uint32_t> sub_mask;     // fp64 tiles of the one-layer passes
   Plan plan1;
   std::vector<DevPass> sub[4];
   bool sub_uploaded = false;
@@ -192,7 +194,7 @@ void compute_layout(qml_ctx* c) {
   const size_t slot_elem = slot_bytes(c);
   l.ckpt = take(slot_elem * (size_t)c->plan.n_ckpt * Bm * (size_t)N + 16);
   if (c->cnot) {  // second state buffer and partner plane for the gathers, the one-layer schedules
-    l.scratch = take(sizeof(float2) * (size_t)Bm * N);
+    l.scratch = take((c->f64 ? sizeof(double2) : sizeof(float2)) * (size_t)Bm * N);
     l.dummy2 = take(sizeof(float2) * (size_t)N);
     l.sub_passes = take(sizeof(DevPass) * 4 * c->sub[0].size());
     l.sub_slot_pass = take(sizeof(int) * (size_t)n);
@@ -686,17 +688,22 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
 // fp64 tiles: the schedule's tile qubits, less the highest qubit the pass
 // does not rotate when the tile has 12 (2^11-position tiles let two blocks
 // share an SM; a passive qubit can leave the tile because CZ is diagonal).
+uint32_t f64_tile_mask(const DevPass& dp, int n) {
+  uint32_t m = 0, rot = 0;
+  for (int b = 0; b < kTileBits; ++b)
+    if (dp.tile_q[b] >= 0 && dp.tile_q[b] < n) m |= 1u << dp.tile_q[b];
+  for (int s = 0; s < dp.nslots; ++s) rot |= 1u << (dp.slot_lq[s] % n);
+  const uint32_t passive = m & ~rot;
+  if (__builtin_popcount(m) == kTileBits && passive) m &= ~(1u << (31 - __builtin_clz(passive)));
+  return m;
+}
+
 void set_f64_tiles(qml_ctx* c) {
   const int n = c->cfg.n_qubits;
   c->f64_mask.clear();
   c->f64_tmax = 1;
   for (const DevPass& dp : c->dpass) {
-    uint32_t m = 0, rot = 0;
-    for (int b = 0; b < kTileBits; ++b)
-      if (dp.tile_q[b] >= 0 && dp.tile_q[b] < n) m |= 1u << dp.tile_q[b];
-    for (int s = 0; s < dp.nslots; ++s) rot |= 1u << (dp.slot_lq[s] % n);
-    const uint32_t passive = m & ~rot;
-    if (__builtin_popcount(m) == kTileBits && passive) m &= ~(1u << (31 - __builtin_clz(passive)));
+    const uint32_t m = f64_tile_mask(dp, n);
     c->f64_mask.push_back(m);
     c->f64_tmax = std::max(c->f64_tmax, __builtin_popcount(m));
   }
@@ -728,8 +735,148 @@ void set_pass_tile(const qml_ctx* c, int p, int B, Pass64Args* a) {
   a->n_tiles = (long long)B << (c->cfg.n_qubits - a->T);
 }
 
+void set_sub_tile(const qml_ctx* c, int p, int B, Pass64Args* a) {
+  a->tile_mask = c->sub_mask[p];
+  a->T = __builtin_popcount(a->tile_mask);
+  a->n_tiles = (long long)B << (c->cfg.n_qubits - a->T);
+}
+
+// fp64 with CNOT entanglers: the one-layer passes, then the layer's CNOT
+// list as a permutation of the standard-order state (qubit-bit maps).
+qml_status run_forward64_cnot(qml_ctx* c, const double* theta, const double* x, int B, double2* psi,
+                              double* expect, cudaStream_t s);
+qml_status run_backward64_cnot(qml_ctx* c, const double* theta, const double* x, int B, double2* psi,
+                               double2* lam, const double* g, double* grad, cudaStream_t s);
+
+// E = <psi|O|psi> in fp64 (O = Z0 or the Pauli sum in force).
+cudaError_t expect64(qml_ctx* c, const double2* psi, int B, double* expect, cudaStream_t s) {
+  c->launches += 2;
+  if (c->obs_terms.empty())
+    return launch_expect64(psi, B, c->cfg.n_qubits, at<double>(c, c->lay.exp_partial), expect,
+                           at<unsigned>(c, c->lay.status), s);
+  cudaError_t e = upload_observable(c, s);
+  if (e != cudaSuccess) return e;
+  return launch_obs_expect64(psi, B, c->cfg.n_qubits, at<ObsGroup>(c, c->lay.obs_groups), (int)c->obs_groups.size(),
+                             at<ObsTerm>(c, c->lay.obs_terms), at<double>(c, c->lay.exp_partial), expect,
+                             at<unsigned>(c, c->lay.status), s);
+}
+
+// lambda = g O psi in fp64.
+cudaError_t seed64(qml_ctx* c, const double2* psi, double2* lam, const double* g, int B, cudaStream_t s) {
+  ++c->launches;
+  if (c->obs_terms.empty()) return launch_bwd_init64(psi, lam, g, B, c->cfg.n_qubits, s);
+  cudaError_t e = upload_observable(c, s);
+  if (e != cudaSuccess) return e;
+  return launch_obs_bwd_init64(psi, lam, g, B, c->cfg.n_qubits, at<ObsGroup>(c, c->lay.obs_groups),
+                               (int)c->obs_groups.size(), at<ObsTerm>(c, c->lay.obs_terms), s);
+}
+
+qml_status run_forward64_cnot(qml_ctx* c, const double* theta, const double* x, int B, double2* psi,
+                              double* expect, cudaStream_t s) {
+  const int n = c->cfg.n_qubits, L = c->cfg.n_layers, cb = c->cfg.ckpt_block;
+  if (c->ws_bytes < c->lay.base_total) return QML_ERR_WORKSPACE;
+  cudaError_t e = upload_sub(c, s);
+  if (e != cudaSuccess) return QML_ERR_CUDA;
+  const int P1 = (int)c->sub[0].size();
+  Pass64Args a = pass64_args(c, theta, x, B, psi, nullptr);
+  for (int q = 0; q < kMaxQubits; ++q) a.nb[q] = a.nbhi[q] = 0;  // no CZ in this mode
+  double2* cur = psi;
+  double2* other = at<double2>(c, c->lay.scratch);
+  for (int l = 0; l < L; ++l) {
+    const int v = sub_variant(l, L);
+    a.theta = theta + (size_t)l * n * 3;  // the one-layer passes read layer 0 of this pointer
+    a.psi = cur;
+    qml_ctx::Span sp{};
+    const bool timed = span_begin(c, s, &sp, false);
+    for (int p = 0; p < P1; ++p) {
+      set_sub_tile(c, p, B, &a);
+      if (launch_pass64(false, a, c->sub[v][p], (int)std::min<long long>(c->grid_fwd, a.n_tiles), s) != cudaSuccess)
+        return QML_ERR_CUDA;
+      ++c->launches;
+    }
+    if (timed) {
+      sp.passes = P1;
+      span_end(c, s, &sp);
+    }
+    e = launch_gather_bits64(cur, other, n, B, c->cnot_fwd_q, c->cnot_bwd_q, c->sms, s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+    ++c->launches;
+    std::swap(cur, other);
+    if (cb > 0 && (l + 1) % cb == 0 && l + 1 < L) {
+      const int m = (l + 1) / cb - 1;
+      void* slot = c->ws + c->lay.ckpt + slot_bytes(c) * (size_t)m * c->cfg.max_batch * (size_t)c->N;
+      e = launch_slot_copy64(true, cur, slot, a.storage, (long long)B * c->N, c->sms, s);
+      if (e != cudaSuccess) return QML_ERR_CUDA;
+      ++c->launches;
+      c->ckpt_batch[m] = B;
+    }
+  }
+  if (cur != psi) {
+    e = cudaMemcpyAsync(psi, cur, sizeof(double2) * (size_t)B * c->N, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+  }
+  if (expect && expect64(c, psi, B, expect, s) != cudaSuccess) return QML_ERR_CUDA;
+  return QML_OK;
+}
+
+qml_status run_backward64_cnot(qml_ctx* c, const double* theta, const double* x, int B, double2* psi,
+                               double2* lam, const double* g, double* grad, cudaStream_t s) {
+  const int n = c->cfg.n_qubits, L = c->cfg.n_layers, cb = c->cfg.ckpt_block;
+  if (c->ws_bytes < c->lay.base_total) return QML_ERR_WORKSPACE;
+  for (int m = 0; m < c->plan.n_ckpt; ++m)
+    if (c->ckpt_batch[m] != B) return QML_ERR_CKPT_MISMATCH;
+  cudaError_t e = upload_sub(c, s);
+  if (e == cudaSuccess) e = seed64(c, psi, lam, g, B, s);
+  if (e != cudaSuccess) return QML_ERR_CUDA;
+  const int P1 = (int)c->sub[0].size();
+  Pass64Args a = pass64_args(c, theta, x, B, psi, lam);
+  for (int q = 0; q < kMaxQubits; ++q) a.nb[q] = a.nbhi[q] = 0;
+  double2* b0 = psi;
+  double2* b1 = lam;
+  double2* sc = at<double2>(c, c->lay.scratch);
+  for (int l = L - 1; l >= 0; --l) {
+    if (cb > 0 && (l + 1) % cb == 0 && l + 1 < L) {  // the stored state after layer l replaces the uncomputed one
+      const int m = (l + 1) / cb - 1;
+      void* slot = c->ws + c->lay.ckpt + slot_bytes(c) * (size_t)m * c->cfg.max_batch * (size_t)c->N;
+      e = launch_slot_copy64(false, b0, slot, a.storage, (long long)B * c->N, c->sms, s);
+      if (e != cudaSuccess) return QML_ERR_CUDA;
+      ++c->launches;
+    }
+    e = launch_gather_bits64(b0, sc, n, B, c->cnot_bwd_q, c->cnot_fwd_q, c->sms, s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+    std::swap(b0, sc);
+    e = launch_gather_bits64(b1, sc, n, B, c->cnot_bwd_q, c->cnot_fwd_q, c->sms, s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+    std::swap(b1, sc);
+    c->launches += 2;
+    const int v = sub_variant(l, L);
+    a.theta = theta + (size_t)l * n * 3;
+    a.psi = b0;
+    a.lam = b1;
+    qml_ctx::Span sp{};
+    const bool timed = span_begin(c, s, &sp, true);
+    for (int p = P1 - 1; p >= 0; --p) {
+      set_sub_tile(c, p, B, &a);
+      if (launch_pass64(true, a, c->sub[v][p], c->grid_bwd, s) != cudaSuccess) return QML_ERR_CUDA;
+      ++c->launches;
+    }
+    if (timed) {
+      sp.passes = P1;
+      span_end(c, s, &sp);
+    }
+    const DevPass* dsub = at<DevPass>(c, c->lay.sub_passes) + (size_t)P1 * v;
+    e = launch_grad_reduce64(dsub, at<int>(c, c->lay.sub_slot_pass), at<int>(c, c->lay.sub_slot_index),
+                             at<double>(c, c->lay.partials), c->grid_bwd, theta + (size_t)l * n * 3, 1, n,
+                             grad + (size_t)l * n * 3, at<unsigned>(c, c->lay.status), s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+    ++c->launches;
+  }
+  return QML_OK;
+}
+
 qml_status run_forward64(qml_ctx* c, const double* theta, const double* x, int B, double2* psi, double* expect,
                          cudaStream_t s) {
+  if (c->cnot) return run_forward64_cnot(c, theta, x, B, psi, expect, s);
   Pass64Args a = pass64_args(c, theta, x, B, psi, nullptr);
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, false);
@@ -742,41 +889,19 @@ qml_status run_forward64(qml_ctx* c, const double* theta, const double* x, int B
     if (dp.ckpt >= 0) c->ckpt_batch[dp.ckpt] = B;
   }
   if (timed) span_end(c, s, &sp);
-  if (expect) {
-    c->launches += 2;
-    cudaError_t e;
-    if (c->obs_terms.empty()) {
-      e = launch_expect64(psi, B, c->cfg.n_qubits, at<double>(c, c->lay.exp_partial), expect,
-                          at<unsigned>(c, c->lay.status), s);
-    } else {
-      e = upload_observable(c, s);
-      if (e == cudaSuccess)
-        e = launch_obs_expect64(psi, B, c->cfg.n_qubits, at<ObsGroup>(c, c->lay.obs_groups),
-                                (int)c->obs_groups.size(), at<ObsTerm>(c, c->lay.obs_terms),
-                                at<double>(c, c->lay.exp_partial), expect, at<unsigned>(c, c->lay.status), s);
-    }
-    if (e != cudaSuccess) return QML_ERR_CUDA;
-  }
+  if (expect && expect64(c, psi, B, expect, s) != cudaSuccess) return QML_ERR_CUDA;
   return QML_OK;
 }
 
 qml_status run_backward64(qml_ctx* c, const double* theta, const double* x, int B, double2* psi, double2* lam,
                           const double* g, double* grad, cudaStream_t s) {
+  if (c->cnot) return run_backward64_cnot(c, theta, x, B, psi, lam, g, grad, s);
   const int n = c->cfg.n_qubits, L = c->cfg.n_layers;
   for (int m = 0; m < c->plan.n_ckpt; ++m)
     if (c->ckpt_batch[m] != B) return QML_ERR_CKPT_MISMATCH;
-  cudaError_t e0;
-  if (c->obs_terms.empty()) {
-    e0 = launch_bwd_init64(psi, lam, g, B, n, s);
-  } else {
-    e0 = upload_observable(c, s);
-    if (e0 == cudaSuccess)
-      e0 = launch_obs_bwd_init64(psi, lam, g, B, n, at<ObsGroup>(c, c->lay.obs_groups), (int)c->obs_groups.size(),
-                                 at<ObsTerm>(c, c->lay.obs_terms), s);
-  }
-  if (e0 != cudaSuccess) return QML_ERR_CUDA;
+  if (seed64(c, psi, lam, g, B, s) != cudaSuccess) return QML_ERR_CUDA;
   Pass64Args a = pass64_args(c, theta, x, B, psi, lam);
-  c->launches += 2;  // lambda init, gradient reduce
+  ++c->launches;  // gradient reduce
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, true);
   // every block writes its partials, so the grid is the one the layout counted
@@ -1081,7 +1206,7 @@ qml_status qml_set_entangler_cnot(qml_ctx* c, int n_pairs, const int* pairs) {
     if (ct < 0 || tg < 0 || ct >= n || tg >= n || ct == tg) return QML_ERR_INVALID_ARG;
     v.push_back({ct, tg});
   }
-  if (c->f64) return QML_ERR_UNSUPPORTED;  // fp32 only
+
   Plan p1;
   if (!make_plan(n, 1, 0, &p1).empty()) return QML_ERR_UNSUPPORTED;
   std::vector<DevPass> d;
@@ -1102,14 +1227,19 @@ qml_status qml_set_entangler_cnot(qml_ctx* c, int n_pairs, const int* pairs) {
       if ((qbits >> q) & 1u) a |= 1u << p1.addr_of[q];
     return a;
   };
-  for (int k = 0; k < kMaxQubits; ++k) c->cnot_bwd.col[k] = c->cnot_fwd.col[k] = 0;
+  for (int k = 0; k < kMaxQubits; ++k)
+    c->cnot_bwd.col[k] = c->cnot_fwd.col[k] = c->cnot_bwd_q.col[k] = c->cnot_fwd_q.col[k] = 0;
   for (int q = 0; q < n; ++q) {
     uint32_t fwd = 1u << q, inv = 1u << q;
     for (const auto& e : v) fwd ^= ((fwd >> e.first) & 1u) << e.second;
     for (auto it = v.rbegin(); it != v.rend(); ++it) inv ^= ((inv >> it->first) & 1u) << it->second;
     c->cnot_bwd.col[p1.addr_of[q]] = to_addr(fwd);
     c->cnot_fwd.col[p1.addr_of[q]] = to_addr(inv);
+    c->cnot_bwd_q.col[q] = fwd;
+    c->cnot_fwd_q.col[q] = inv;
   }
+  c->sub_mask.clear();
+  for (const DevPass& dp : c->sub[0]) c->sub_mask.push_back(f64_tile_mask(dp, n));
   c->plan1 = p1;
   c->cnot_pairs = v;
   c->cnot = true;

@@ -28,9 +28,9 @@ namespace {
 // XOR of j spreads over the whole state).
 // m(j) = t0[j & 1023] ^ t1[(j >> 10) & 1023] ^ t2[j >> 20] from three
 // 1024-entry shared tables (n <= 30).
-template <bool SCATTER>
-__global__ void permute_state_kernel(const float2* __restrict__ src, float2* __restrict__ dst, int n,
-                                     long long total, const LinMap m) {
+template <bool SCATTER, class T>
+__global__ void permute_state_kernel(const T* __restrict__ src, T* __restrict__ dst, int n, long long total,
+                                     const LinMap m) {
   __shared__ uint32_t t0[1024], t1[1024], t2[1024];
   for (int i = threadIdx.x; i < 1024; i += blockDim.x) {
     uint32_t a = 0, b = 0, c = 0;
@@ -106,6 +106,33 @@ __global__ void slot_from_planes_kernel(const float2* buf, const float2* partner
   }
 }
 
+// fp64 mode (standard layout): slot <- psi (save) or psi <- slot, the slot in
+// fp64 (storage 2), fp32 (0) or bf16 (1, round to nearest even).
+__global__ void slot_copy64_kernel(bool save, double2* psi, void* slot, int storage, long long count) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += stride) {
+    if (save) {
+      const double2 v = psi[i];
+      if (storage == 2) reinterpret_cast<double2*>(slot)[i] = v;
+      else if (storage == 1)
+        reinterpret_cast<__nv_bfloat162*>(slot)[i] = __floats2bfloat162_rn((float)v.x, (float)v.y);
+      else reinterpret_cast<float2*>(slot)[i] = make_float2((float)v.x, (float)v.y);
+    } else {
+      double2 v;
+      if (storage == 2) {
+        v = reinterpret_cast<const double2*>(slot)[i];
+      } else if (storage == 1) {
+        const float2 f = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(slot)[i]);
+        v = make_double2(f.x, f.y);
+      } else {
+        const float2 f = reinterpret_cast<const float2*>(slot)[i];
+        v = make_double2(f.x, f.y);
+      }
+      psi[i] = v;
+    }
+  }
+}
+
 unsigned grid_for(long long count, int sms) {
   const long long blocks = (count + 255) / 256;
   return (unsigned)std::min<long long>(blocks, (long long)sms * 16);
@@ -113,15 +140,33 @@ unsigned grid_for(long long count, int sms) {
 
 }  // namespace
 
-cudaError_t launch_gather_bits(const float2* src, float2* dst, int n, int B, const LinMap& m, const LinMap& m_inv,
-                               int sms, cudaStream_t s) {
+template <class T>
+cudaError_t permute_state(const T* src, T* dst, int n, int B, const LinMap& m, const LinMap& m_inv, int sms,
+                          cudaStream_t s) {
   const long long total = (long long)B << n;
   if (n > kMaxQubits) return cudaErrorInvalidValue;  // three 10-bit tables
   if (total == 0) return cudaSuccess;
   if (spread(m, n) <= spread(m_inv, n))
-    permute_state_kernel<false><<<grid_for(total, sms), 256, 0, s>>>(src, dst, n, total, m);
+    permute_state_kernel<false, T><<<grid_for(total, sms), 256, 0, s>>>(src, dst, n, total, m);
   else
-    permute_state_kernel<true><<<grid_for(total, sms), 256, 0, s>>>(src, dst, n, total, m_inv);
+    permute_state_kernel<true, T><<<grid_for(total, sms), 256, 0, s>>>(src, dst, n, total, m_inv);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_bits(const float2* src, float2* dst, int n, int B, const LinMap& m, const LinMap& m_inv,
+                               int sms, cudaStream_t s) {
+  return permute_state(src, dst, n, B, m, m_inv, sms, s);
+}
+
+cudaError_t launch_gather_bits64(const double2* src, double2* dst, int n, int B, const LinMap& m,
+                                 const LinMap& m_inv, int sms, cudaStream_t s) {
+  return permute_state(src, dst, n, B, m, m_inv, sms, s);
+}
+
+cudaError_t launch_slot_copy64(bool save, double2* psi, void* slot, int storage, long long count, int sms,
+                               cudaStream_t s) {
+  if (count == 0) return cudaSuccess;
+  slot_copy64_kernel<<<grid_for(count, sms), 256, 0, s>>>(save, psi, slot, storage, count);
   return cudaGetLastError();
 }
 

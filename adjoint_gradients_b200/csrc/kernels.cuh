@@ -107,6 +107,12 @@ struct LinMap {
 // bits; m_inv its inverse, used when the scatter form is the more local one).
 cudaError_t launch_gather_bits(const float2* src, float2* dst, int n, int B, const LinMap& m, const LinMap& m_inv,
                                int sms, cudaStream_t s);
+// fp64 mode: the same permutation of complex128 states, and slot save / restore
+// (storage 0 fp32, 1 bf16, 2 fp64) of standard-layout states.
+cudaError_t launch_gather_bits64(const double2* src, double2* dst, int n, int B, const LinMap& m,
+                                 const LinMap& m_inv, int sms, cudaStream_t s);
+cudaError_t launch_slot_copy64(bool save, double2* psi, void* slot, int storage, long long count, int sms,
+                               cudaStream_t s);
 // Checkpoint slot (standard layout, storage 0 fp32 / 1 bf16) from the forward
 // pass's working layout in buf (and partner: an odd batch's last unit).
 cudaError_t launch_slot_from_planes(const float2* buf, const float2* partner, void* slot, int storage, int B, int n,

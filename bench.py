@@ -129,8 +129,9 @@ def algorithmic_counts(ctx, w, B, f64=False, cnot_passes_per_layer=0):
     rots = w.n * w.L
     if cnot_passes_per_layer:  # CNOT entanglers: every layer's passes read and write the state once
         Pc = cnot_passes_per_layer * w.L
+        c = 16 if f64 else 8
         return {"passes": Pc, "fwd_fma": FMA_FWD_PER_ROT * rots * amp, "bwd_fma": FMA_BWD_PER_ROT * rots * amp,
-                "fwd_bytes": (16 * Pc - 8) * amp, "bwd_bytes": (32 * Pc - 16) * amp}
+                "fwd_bytes": (2 * c * Pc - c) * amp, "bwd_bytes": (4 * c * Pc - 2 * c) * amp}
     # bytes per amplitude moved by each pass, from the schedule flags
     i = 1
     fwd_bytes = bwd_bytes = 0

@@ -202,8 +202,8 @@ QML_API int qml_entangler_bonds(const qml_ctx* ctx);
  * qml_workspace_bytes / qml_set_workspace again after this call if the
  * workspace was set before; the compute calls return QML_ERR_WORKSPACE until
  * it is large enough).  Checkpoint slots, observables and re-uploading apply
- * as with CZ.  QML_ERR_INVALID_ARG on a bad pair or count;
- * QML_ERR_UNSUPPORTED for fp64 contexts.
+ * as with CZ, in both precisions (fp64 contexts keep the standard order and
+ * need B * 2^n complex128 more).  QML_ERR_INVALID_ARG on a bad pair or count.
  * qml_set_entangler switches back to CZ. */
 QML_API qml_status qml_set_entangler_cnot(qml_ctx* ctx, int n_pairs, const int* pairs);
 
@@ -342,9 +342,9 @@ QML_API int qml_debug_layouts(int* out, int cap);
  * (re, im) double pairs, 16-byte aligned.  Checkpoint slots take the
  * config's storage: QML_STORE_FP64 keeps them exact, QML_STORE_FP32 /
  * QML_STORE_BF16 round them (the backward pass then restarts from the
- * rounded state at each slot).  CZ entanglers (qml_set_entangler), data
- * re-uploading (qml_set_reupload, any n) and Pauli-sum observables
- * (qml_set_observable, evaluated in fp64) apply.
+ * rounded state at each slot).  CZ and CNOT entanglers, data re-uploading
+ * (qml_set_reupload, any n) and Pauli-sum observables (qml_set_observable,
+ * evaluated in fp64) apply.
  * The fp32 calls (qml_forward_expect, qml_backward_adjoint, qml_loss_seed,
  * qml_step_host, qml_init_state_encode, qml_ckpt_save / _restore,
  * qml_expect_z0, qml_expect_observable) return QML_ERR_UNSUPPORTED on an

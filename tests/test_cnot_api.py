@@ -33,9 +33,10 @@ def test_cnot_setter_validates_and_switches_kind():
     lib.qml_destroy(h)
 
 
-def test_cnot_unsupported_for_fp64_only():
+def test_cnot_in_both_precisions_and_three_qubit_sets():
     lib, h = _ctx(8, 2, 2, f64=True)
-    assert lib.qml_set_entangler_cnot(h, 1, _pairs([(0, 1)])) == 2
+    assert lib.qml_set_entangler_cnot(h, 1, _pairs([(0, 1)])) == qml.QML_OK
+    assert lib.qml_entangler_kind(h) == 1
     lib.qml_destroy(h)
     lib, h = _ctx(23, 1, 1)  # three qubit sets: the map is taken to the working-state addresses
     assert lib.qml_set_entangler_cnot(h, 2, _pairs([(0, 22), (12, 3)])) == qml.QML_OK

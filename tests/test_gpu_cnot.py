@@ -103,3 +103,29 @@ def test_switching_back_to_cz_restores_the_chain():
     E = ctx.forward(dev(theta), dev(x))[1].cpu().numpy().astype(np.float64)
     ctx.sync()
     np.testing.assert_allclose(E, oracle.forward(x, theta), atol=1e-4)
+
+
+@pytest.mark.parametrize("n,L,B,ck,st,kind", [(5, 3, 3, 1, "fp64", "ladder"), (13, 3, 2, 1, "fp64", "ring"),
+                                              (14, 2, 3, 1, "bf16", "ladder"), (21, 2, 2, 1, "fp64", "ladder")])
+def test_cnot_fp64(n, L, B, ck, st, kind):
+    """fp64 mode with CNOT lists: tolerances of the fp64 parity tests (1e-10 + 1e-9 |g| with fp64 or no
+    slots; bf16 slots round the restarted state to 2^-8: 2e-2 + 1e-3 |g|)."""
+    rng = np.random.default_rng(7500 + n)
+    pairs = pairs_of(kind, n, rng)
+    x, theta, y = random_case(7600 + n, B, n, L)
+    Eo, psio = oracle.forward(x, theta, want_state=True, bonds=pairs, entangler="cnot")
+    g = oracle.loss_seed(Eo, y)
+    ctx = qml().Context(n, L, B, ckpt_block=ck, storage=st, precision="fp64")
+    ctx.set_entangler(pairs, kind="cnot")
+    d64 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64)).cuda()
+    xd, td = d64(x), d64(theta)
+    psi, E = ctx.forward(td, xd)
+    got = psi.cpu().numpy()
+    got = got[..., 0] + 1j * got[..., 1]
+    grad = ctx.backward(td, xd, psi, ctx.new_state(B), d64(g)).cpu().numpy()
+    ctx.sync()
+    assert np.max(np.abs(E.cpu().numpy() - Eo)) <= 1e-11
+    assert np.max(np.abs(got - psio)) <= 1e-12
+    gref, _ = oracle.adjoint(x, theta, g, bonds=pairs, entangler="cnot")
+    a, r = (2e-2, 1e-3) if st == "bf16" else (1e-10, 1e-9)
+    assert np.all(np.abs(grad - gref) <= a + r * np.abs(gref)), np.max(np.abs(grad - gref))
