@@ -191,7 +191,7 @@ __device__ void rot_chunk(const Pass64Args& a, const DevPass& P, const Ctx64& cx
 }
 
 template <bool BWD>
-__global__ void __launch_bounds__(kT, 2) pass64_kernel(const Pass64Args a, const __grid_constant__ DevPass P) {
+__global__ void __launch_bounds__(kT, BWD ? 2 : 3) pass64_kernel(const Pass64Args a, const __grid_constant__ DevPass P) {
   extern __shared__ __align__(16) unsigned char smem64[];
   double2* tp = reinterpret_cast<double2*>(smem64);
   const int plane = plane_slots(a.tmax);
