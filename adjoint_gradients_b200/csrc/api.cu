@@ -1249,6 +1249,19 @@ qml_status qml_set_entangler_cnot(qml_ctx* c, int n_pairs, const int* pairs) {
 
 int qml_entangler_kind(const qml_ctx* c) { return c ? (c->cnot ? 1 : 0) : -1; }
 
+int qml_debug_entangler_map(const qml_ctx* c, int* out, int cap) {
+  if (!c || !c->cnot) return -1;
+  const int n = c->cfg.n_qubits;
+  std::vector<int> v;
+  v.push_back(n);
+  for (int q = 0; q < n; ++q) v.push_back((int)c->cnot_bwd_q.col[q]);  // M
+  for (int q = 0; q < n; ++q) v.push_back((int)c->cnot_fwd_q.col[q]);  // M^-1
+  for (int a = 0; a < n; ++a) v.push_back((int)c->cnot_bwd.col[a]);    // M on working-state addresses
+  for (int a = 0; a < n; ++a) v.push_back((int)c->cnot_fwd.col[a]);
+  for (int i = 0; i < (int)v.size() && out && i < cap; ++i) out[i] = v[i];
+  return (int)v.size();
+}
+
 qml_status qml_set_reupload(qml_ctx* c, int on) {
   if (!c) return QML_ERR_INVALID_ARG;
   if (on && c->slow && !c->f64) return QML_ERR_UNSUPPORTED;  // fp32, n < 5: batch-unit register bits

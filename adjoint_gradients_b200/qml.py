@@ -34,7 +34,7 @@ EXPORTS = [
     "qml_debug_tile_view", "qml_debug_layouts", "qml_set_observable", "qml_observable_terms",
     "qml_expect_observable", "qml_set_entangler", "qml_entangler_bonds", "qml_set_reupload", "qml_reupload",
     "qml_create_f64", "qml_precision", "qml_forward_expect_f64", "qml_backward_adjoint_f64", "qml_loss_seed_f64",
-    "qml_step_host_f64", "qml_set_entangler_cnot", "qml_entangler_kind",
+    "qml_step_host_f64", "qml_set_entangler_cnot", "qml_entangler_kind", "qml_debug_entangler_map",
 ]
 
 
@@ -119,6 +119,7 @@ def load_library(path: str = LIB_PATH):
         "qml_step_host_f64": ([_vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp], _i),
         "qml_set_entangler_cnot": ([_vp, _i, ctypes.POINTER(_i)], _i),
         "qml_entangler_kind": ([_vp], _i),
+        "qml_debug_entangler_map": ([_vp, ctypes.POINTER(_i), _i], _i),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)

@@ -210,6 +210,13 @@ QML_API qml_status qml_set_entangler_cnot(qml_ctx* ctx, int n_pairs, const int* 
 /* Kind of the entangler in force: 0 CZ, 1 CNOT (-1 for NULL). */
 QML_API int qml_entangler_kind(const qml_ctx* ctx);
 
+/* Debugging aid (host only): the CNOT layer map as images of single index
+ * bits, written like qml_debug_schedule (returns the number of ints, -1 when
+ * the entangler is not CNOT).  Layout: [n, then n images of M (the layer
+ * sends the amplitude at b to M b) on qubit bits, n images of M^-1, then the
+ * same two maps on working-state address bits]. */
+QML_API int qml_debug_entangler_map(const qml_ctx* ctx, int* out, int cap);
+
 /* Data re-uploading for the following forward and backward calls: with
  * on != 0 every layer starts with the angle encoding Ry(x[b][q]) on every
  * qubit again (no parameters; its inverse is un-applied in the backward pass,

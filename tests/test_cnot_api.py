@@ -52,3 +52,58 @@ def test_cnot_workspace_holds_a_second_state():
     after = lib.qml_workspace_bytes(h, B)
     assert after - before >= 8 * B * (1 << n) + 8 * (1 << n)
     lib.qml_destroy(h)
+
+
+def _map(lib, h):
+    need = lib.qml_debug_entangler_map(h, None, 0)
+    buf = (ctypes.c_int * need)()
+    lib.qml_debug_entangler_map(h, buf, need)
+    v = list(buf)
+    n = v[0]
+    return n, v[1:1 + n], v[1 + n:1 + 2 * n], v[1 + 2 * n:1 + 3 * n], v[1 + 3 * n:1 + 4 * n]
+
+
+def _apply(cols, b):
+    out = 0
+    for k, c in enumerate(cols):
+        if (b >> k) & 1:
+            out ^= c
+    return out
+
+
+def _simulate(pairs, b):
+    """A basis index through the CNOT list, one gate at a time."""
+    for c, t in pairs:
+        if (b >> c) & 1:
+            b ^= 1 << t
+    return b
+
+
+def test_ladder_map_is_the_prefix_xor():
+    n = 9
+    lib, h = _ctx(n, 2, 2)
+    ladder = [(q, q + 1) for q in range(n - 1)]
+    assert lib.qml_set_entangler_cnot(h, len(ladder), _pairs(ladder)) == qml.QML_OK
+    _, M, Minv, _, _ = _map(lib, h)
+    for k in range(n):
+        assert M[k] == ((1 << n) - 1) & ~((1 << k) - 1)  # bit k reaches bits k..n-1
+        assert Minv[k] == (1 << k) | ((1 << (k + 1)) if k + 1 < n else 0)
+    lib.qml_destroy(h)
+
+
+def test_map_matches_gate_by_gate_action_and_inverts():
+    import numpy as np
+
+    rng = np.random.default_rng(5)
+    for n, L in [(6, 1), (14, 2), (23, 1)]:
+        lib, h = _ctx(n, L, 1)
+        allp = [(a, b) for a in range(n) for b in range(n) if a != b]
+        pairs = [allp[i] for i in rng.choice(len(allp), size=n + 3, replace=False)]
+        assert lib.qml_set_entangler_cnot(h, len(pairs), _pairs(pairs)) == qml.QML_OK
+        _, M, Minv, Ma, Mainv = _map(lib, h)
+        for b in rng.integers(0, 1 << n, size=64):
+            b = int(b)
+            assert _apply(M, b) == _simulate(pairs, b)
+            assert _apply(Minv, _apply(M, b)) == b
+            assert _apply(Mainv, _apply(Ma, b)) == b
+        lib.qml_destroy(h)
