@@ -107,3 +107,41 @@ def test_map_matches_gate_by_gate_action_and_inverts():
             assert _apply(Minv, _apply(M, b)) == b
             assert _apply(Mainv, _apply(Ma, b)) == b
         lib.qml_destroy(h)
+
+
+def test_address_map_is_the_qubit_map_with_renamed_bits():
+    """Three qubit sets: the working state sits at permuted addresses (qubit q at
+    address bit addr[q], read from the pass view), and the layer map on
+    addresses must send addr(b) to addr(M b)."""
+    import numpy as np
+
+    n = 23
+    lib, h = _ctx(n, 1, 1)
+    need = lib.qml_debug_tile_view(h, 0, None, 0)
+    buf = (ctypes.c_int * need)()
+    lib.qml_debug_tile_view(h, 0, buf, need)
+    v = list(buf)
+    tile_q = [v[21 + 2 * b] for b in range(12)]
+    n_out = v[21 + 24]
+    out_q = v[21 + 25:21 + 25 + n_out]
+    j = 21 + 25 + n_out
+    tile_a, out_a = v[j:j + 12], v[j + 12:j + 12 + n_out]
+    addr = {}
+    for q, a in list(zip(tile_q, tile_a)) + list(zip(out_q, out_a)):
+        if q >= 0:
+            addr[q] = a
+    assert sorted(addr) == list(range(n)) and sorted(addr.values()) == list(range(n))
+    assert any(addr[q] != q for q in range(n))  # the permuted layout is in force
+
+    def to_addr(b):
+        return sum(1 << addr[q] for q in range(n) if (b >> q) & 1)
+
+    ladder = [(q, q + 1) for q in range(n - 1)] + [(n - 1, 0)]
+    assert lib.qml_set_entangler_cnot(h, len(ladder), _pairs(ladder)) == qml.QML_OK
+    _, M, _, Ma, Mainv = _map(lib, h)
+    rng = np.random.default_rng(9)
+    for b in rng.integers(0, 1 << n, size=128):
+        b = int(b)
+        assert _apply(Ma, to_addr(b)) == to_addr(_apply(M, b))
+        assert _apply(Mainv, _apply(Ma, to_addr(b))) == to_addr(b)
+    lib.qml_destroy(h)
