@@ -29,6 +29,8 @@ struct Layout {
   size_t status, passes, slot_pass, slot_index;
   size_t coef_fwd, coef_inv, enc, dummy, exp_partial, partials, obs_groups, obs_terms, ckpt;
   size_t scratch, dummy2, sub_passes, sub_slot_pass, sub_slot_index;  // CNOT entanglers only
+  size_t passes_split, undo, s_rot, s_lay, s_gfix, s_dqf, s_dqb, rscale;  // split form (fp32 only)
+  size_t fault_theta;  // QML_FAULT=nan_theta, fp64: a copy of theta with a NaN angle
   size_t base_total;
   // host-step extras
   size_t h_psi, h_lam, h_x, h_theta, h_y, h_E, h_g, h_loss, h_grad;
@@ -57,6 +59,10 @@ struct qml_ctx {
   int device = 0;
   Plan plan;
   std::vector<DevPass> dpass;
+  // the same passes in split form (OP_RY / OP_DIAG), used by fp32 contexts
+  // without re-uploading or CNOT entanglers
+  std::vector<DevPass> dpass_split;
+  std::vector<int> undo;  // split form: [L][n] backward un-apply order of each layer's qubits
   size_t smem = 0;
   bool probed = false, dev_ok = false;
   bool slow = false;  // the plan puts a batch-unit bit in registers (n < 5)
@@ -181,8 +187,8 @@ void compute_layout(qml_ctx* c) {
   l.passes = take(sizeof(DevPass) * c->dpass.size());
   l.slot_pass = take(sizeof(int) * (size_t)L * n);
   l.slot_index = take(sizeof(int) * (size_t)L * n);
-  l.coef_fwd = take(sizeof(float4) * 4 * (size_t)kMaxSlots * c->dpass.size());
-  l.coef_inv = take(sizeof(float4) * 4 * (size_t)kMaxSlots * c->dpass.size());
+  l.coef_fwd = take(sizeof(CoefRegion) * std::max(c->dpass.size(), c->sub[0].size()));
+  l.coef_inv = take(sizeof(CoefRegion) * std::max(c->dpass.size(), c->sub[0].size()));
   l.enc = take(sizeof(float2) * 2 * U * n);
   l.dummy = take(sizeof(float2) * (size_t)N);
   l.exp_partial = take(sizeof(double) * (c->f64 ? expect64_partial_count(Bm, n) : expect_partial_count(Bm, n)));
@@ -200,6 +206,17 @@ void compute_layout(qml_ctx* c) {
     l.sub_slot_pass = take(sizeof(int) * (size_t)n);
     l.sub_slot_index = take(sizeof(int) * (size_t)n);
   }
+  if (!c->f64) {
+    l.passes_split = take(sizeof(DevPass) * c->dpass_split.size());
+    l.undo = take(sizeof(int) * (size_t)L * n);
+    l.s_rot = take(sizeof(SplitRot) * (size_t)L * n);
+    l.s_lay = take(sizeof(SplitLayer) * (size_t)L);
+    l.s_gfix = take(sizeof(double) * 2 * (size_t)L * n);
+    l.s_dqf = take(sizeof(float2) * 2 * (size_t)(L + 1) * n);
+    l.s_dqb = take(sizeof(float2) * 2 * (size_t)(L + 1) * n);
+    l.rscale = take(sizeof(float) * c->dpass_split.size());
+  }
+  if (c->f64 && c->fault == qml_ctx::FAULT_NAN) l.fault_theta = take(sizeof(double) * 3 * (size_t)L * n);
   l.base_total = o;
   const size_t fe = c->f64 ? sizeof(double) : sizeof(float);  // real element of the host-step buffers
   l.h_psi = take(2 * fe * (size_t)Bm * N);
@@ -214,9 +231,10 @@ void compute_layout(qml_ctx* c) {
   l.host_total = o;
   // gradient partial offsets per pass
   long long off = 0;
-  for (DevPass& p : c->dpass) {
-    p.partial_off = off;
-    off += (long long)c->grid_bwd * p.nslots * 3;
+  for (size_t i = 0; i < c->dpass.size(); ++i) {
+    c->dpass[i].partial_off = off;
+    if (i < c->dpass_split.size()) c->dpass_split[i].partial_off = off;
+    off += (long long)c->grid_bwd * c->dpass[i].nslots * 3;
   }
   // one-layer schedules: one layer's partials at a time, in the same area
   for (auto& v : c->sub) {
@@ -264,6 +282,13 @@ T* at(qml_ctx* c, size_t off) {
   return reinterpret_cast<T*>(c->ws + off);
 }
 
+// fp32 contexts run the split form unless a mode needs the fused SU(2)
+// (re-uploading folds per-sample encodings into the rotations; CNOT layers
+// run as one-layer schedules).
+bool use_split(const qml_ctx* c) { return !c->f64 && !c->reupload && !c->cnot; }
+
+const std::vector<DevPass>& fp32_passes(const qml_ctx* c) { return use_split(c) ? c->dpass_split : c->dpass; }
+
 // Readiness of a context for a call with batch B; f64 is the precision the
 // call is made for (a context computes in one precision only).
 qml_status check_ready(qml_ctx* c, int B, bool f64 = false) {
@@ -298,7 +323,7 @@ const PassMaps* pass_maps_for(qml_ctx* c, const DevPass& dp, bool backward, int 
 }
 
 const PassMaps* pass_maps(qml_ctx* c, int p, bool backward, int B, const void* buf0, const void* buf1) {
-  return pass_maps_for(c, c->dpass[p], backward, B, buf0, buf1);
+  return pass_maps_for(c, fp32_passes(c)[p], backward, B, buf0, buf1);
 }
 
 // Copy the observable's terms into the workspace if they changed since the
@@ -391,8 +416,8 @@ qml_status run_forward_cnot(qml_ctx* c, const float* theta, const float* x, int 
   cudaError_t e = upload_sub(c, s);
   if (e != cudaSuccess) return QML_ERR_CUDA;
   const int P1 = (int)c->sub[0].size();
-  float4* cf = at<float4>(c, c->lay.coef_fwd);
-  float4* ci = at<float4>(c, c->lay.coef_inv);
+  CoefRegion* cf = at<CoefRegion>(c, c->lay.coef_fwd);
+  CoefRegion* ci = at<CoefRegion>(c, c->lay.coef_inv);
   e = launch_prep_enc(x, B, n, at<float2>(c, c->lay.enc), s);
   if (e != cudaSuccess) return QML_ERR_CUDA;
   PassArgs a{};
@@ -416,6 +441,8 @@ qml_status run_forward_cnot(qml_ctx* c, const float* theta, const float* x, int 
     const int v = sub_variant(l, L);
     const DevPass* dsub = at<DevPass>(c, c->lay.sub_passes) + (size_t)P1 * v;
     e = launch_prep_pass_coef(dsub, P1, theta + (size_t)l * n * 3, cf, ci, s);
+    if (e == cudaSuccess && l == 0 && c->fault == qml_ctx::FAULT_NAN)  // injected: as in run_forward
+      e = cudaMemsetAsync(cf, 0xff, sizeof(float4), s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
     ++c->launches;
     qml_ctx::Span sp{};
@@ -425,7 +452,7 @@ qml_status run_forward_cnot(qml_ctx* c, const float* theta, const float* x, int 
       a.n_tiles = (int)(((a.U + (1ll << dp.unit_bits) - 1) >> dp.unit_bits) << dp.n_out);
       a.buf0 = cur;
       a.dummy = part;
-      e = copy_pass_coef(c->region, cf + (size_t)p * kMaxSlots * 4, dp.nslots, s);
+      e = copy_pass_coef(c->region, cf + p, dp.nslots, 0, s);
       if (e != cudaSuccess) return QML_ERR_CUDA;
       const PassMaps* maps = pass_maps_for(c, dp, false, B, cur, part);
       if (!maps) return QML_ERR_CUDA;
@@ -477,8 +504,8 @@ qml_status run_backward_cnot(qml_ctx* c, const float* theta, const float* x, int
   cudaError_t e = upload_sub(c, s);
   if (e != cudaSuccess) return QML_ERR_CUDA;
   const int P1 = (int)c->sub[0].size();
-  float4* cf = at<float4>(c, c->lay.coef_fwd);
-  float4* ci = at<float4>(c, c->lay.coef_inv);
+  CoefRegion* cf = at<CoefRegion>(c, c->lay.coef_fwd);
+  CoefRegion* ci = at<CoefRegion>(c, c->lay.coef_inv);
   if (c->obs_terms.empty()) {
     e = launch_bwd_init(psi, lam, g, B, n, s);
   } else {
@@ -540,7 +567,7 @@ qml_status run_backward_cnot(qml_ctx* c, const float* theta, const float* x, int
       a.n_tiles = (int)(((a.U + (1ll << dp.unit_bits) - 1) >> dp.unit_bits) << dp.n_out);
       a.buf0 = b0;
       a.buf1 = b1;
-      e = copy_pass_coef(c->region, ci + (size_t)p * kMaxSlots * 4, dp.nslots, s);
+      e = copy_pass_coef(c->region, ci + p, dp.nslots, 0, s);
       if (e != cudaSuccess) return QML_ERR_CUDA;
       const PassMaps* maps = pass_maps_for(c, dp, true, B, b0, b1);
       if (!maps) return QML_ERR_CUDA;
@@ -553,7 +580,7 @@ qml_status run_backward_cnot(qml_ctx* c, const float* theta, const float* x, int
       span_end(c, s, &sp);
     }
     e = launch_grad_reduce(dsub, at<int>(c, c->lay.sub_slot_pass), at<int>(c, c->lay.sub_slot_index),
-                           at<float>(c, c->lay.partials), c->grid_bwd, theta + (size_t)l * n * 3, 1, n,
+                           at<float>(c, c->lay.partials), c->grid_bwd, theta + (size_t)l * n * 3, nullptr, 1, n,
                            grad + (size_t)l * n * 3, at<unsigned>(c, c->lay.status), s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
     ++c->launches;
@@ -561,13 +588,28 @@ qml_status run_backward_cnot(qml_ctx* c, const float* theta, const float* x, int
   return QML_OK;
 }
 
+// Coefficient tables of the fp32 passes from theta (both directions).
+cudaError_t prep_coefficients(qml_ctx* c, const float* theta, cudaStream_t s) {
+  CoefRegion* cf = at<CoefRegion>(c, c->lay.coef_fwd);
+  CoefRegion* ci = at<CoefRegion>(c, c->lay.coef_inv);
+  if (!use_split(c))
+    return launch_prep_pass_coef(at<DevPass>(c, c->lay.passes), (int)c->dpass.size(), theta, cf, ci, s);
+  return launch_prep_split(at<DevPass>(c, c->lay.passes_split), (int)c->dpass_split.size(), theta,
+                           c->cfg.n_layers, c->cfg.n_qubits, at<int>(c, c->lay.undo), at<SplitRot>(c, c->lay.s_rot),
+                           at<SplitLayer>(c, c->lay.s_lay), at<double>(c, c->lay.s_gfix),
+                           at<float2>(c, c->lay.s_dqf), at<float2>(c, c->lay.s_dqb), cf, ci,
+                           at<float>(c, c->lay.rscale), s);
+}
+
 qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, float2* psi,
                        float* expect, cudaStream_t s) {
   if (c->cnot) return run_forward_cnot(c, theta, x, B, psi, expect, s);
   const int n = c->cfg.n_qubits;
-  const int P = (int)c->dpass.size();
-  float4* cf = at<float4>(c, c->lay.coef_fwd);
-  cudaError_t e = launch_prep_pass_coef(at<DevPass>(c, c->lay.passes), P, theta, cf, at<float4>(c, c->lay.coef_inv), s);
+  const bool split = use_split(c);
+  const std::vector<DevPass>& passes = fp32_passes(c);
+  const int P = (int)passes.size();
+  CoefRegion* cf = at<CoefRegion>(c, c->lay.coef_fwd);
+  cudaError_t e = prep_coefficients(c, theta, s);
   if (e == cudaSuccess && c->fault == qml_ctx::FAULT_NAN)  // injected: the first rotation's coefficients become NaN
     e = cudaMemsetAsync(cf, 0xff, sizeof(float4), s);
   if (e != cudaSuccess) return QML_ERR_CUDA;
@@ -591,14 +633,16 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
   a.status = at<unsigned>(c, c->lay.status);
   for (int q = 0; q < kMaxQubits; ++q) a.cz_nb[q] = c->nb[q], a.cz_nbhi[q] = c->nbhi[q];
   a.reupload = c->reupload ? 1 : 0;
-  c->launches += 2;
+  a.dq = split ? at<float2>(c, c->lay.s_dqf) : nullptr;
+  a.rscale = nullptr;
+  c->launches += split ? 5 : 2;
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, false);
   for (int p = 0; p < P; ++p) {
-    const DevPass& dp = c->dpass[p];
+    const DevPass& dp = passes[p];
     const long long units_per_tile = 1ll << dp.unit_bits;
     a.n_tiles = (int)(((a.U + units_per_tile - 1) / units_per_tile) << dp.n_out);
-    e = copy_pass_coef(c->region, cf + (size_t)p * kMaxSlots * 4, dp.nslots, s);
+    e = copy_pass_coef(c->region, cf + p, dp.nslots, dp.ndiag, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
     const PassMaps* maps = pass_maps(c, p, false, B, psi, a.dummy);
     if (!maps) return QML_ERR_CUDA;
@@ -623,11 +667,13 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
                         float2* lam, const float* g, float* grad, cudaStream_t s) {
   if (c->cnot) return run_backward_cnot(c, theta, x, B, psi, lam, g, grad, s);
   const int n = c->cfg.n_qubits, L = c->cfg.n_layers;
-  const int P = (int)c->dpass.size();
+  const bool split = use_split(c);
+  const std::vector<DevPass>& passes = fp32_passes(c);
+  const int P = (int)passes.size();
   for (int m = 0; m < c->plan.n_ckpt; ++m)
     if (c->ckpt_batch[m] != B) return QML_ERR_CKPT_MISMATCH;
-  float4* ci = at<float4>(c, c->lay.coef_inv);
-  cudaError_t e = launch_prep_pass_coef(at<DevPass>(c, c->lay.passes), P, theta, at<float4>(c, c->lay.coef_fwd), ci, s);
+  CoefRegion* ci = at<CoefRegion>(c, c->lay.coef_inv);
+  cudaError_t e = prep_coefficients(c, theta, s);
   if (e != cudaSuccess) return QML_ERR_CUDA;
   if (c->obs_terms.empty()) {
     e = launch_bwd_init(psi, lam, g, B, n, s);
@@ -663,14 +709,16 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
   a.status = at<unsigned>(c, c->lay.status);
   for (int q = 0; q < kMaxQubits; ++q) a.cz_nb[q] = c->nb[q], a.cz_nbhi[q] = c->nbhi[q];
   a.reupload = c->reupload ? 1 : 0;
-  c->launches += 3;  // coefficient prep, lambda init, gradient reduce
+  a.dq = split ? at<float2>(c, c->lay.s_dqb) : nullptr;
+  c->launches += split ? 6 : 3;  // coefficient prep, lambda init, gradient reduce
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, true);
   for (int p = P - 1; p >= 0; --p) {
-    const DevPass& dp = c->dpass[p];
+    const DevPass& dp = passes[p];
     const long long units_per_tile = 1ll << dp.unit_bits;
     a.n_tiles = (int)(((a.U + units_per_tile - 1) / units_per_tile) << dp.n_out);
-    e = copy_pass_coef(c->region, ci + (size_t)p * kMaxSlots * 4, dp.nslots, s);
+    a.rscale = (split && dp.ckpt >= 0) ? at<float>(c, c->lay.rscale) + p : nullptr;
+    e = copy_pass_coef(c->region, ci + p, dp.nslots, dp.ndiag, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
     const PassMaps* maps = pass_maps(c, p, true, B, psi, lam);
     if (!maps) return QML_ERR_CUDA;
@@ -681,7 +729,8 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
   if (timed) span_end(c, s, &sp);
   e = launch_grad_reduce(at<DevPass>(c, c->lay.passes), at<int>(c, c->lay.slot_pass),
                          at<int>(c, c->lay.slot_index), at<float>(c, c->lay.partials), c->grid_bwd,
-                         theta, L, n, grad, at<unsigned>(c, c->lay.status), s);
+                         theta, split ? at<double>(c, c->lay.s_gfix) : nullptr, L, n, grad,
+                         at<unsigned>(c, c->lay.status), s);
   return cuda_status(e);
 }
 
@@ -983,8 +1032,11 @@ static qml_status create_ctx(const qml_config* cfg, int device, bool f64, qml_ct
     return QML_ERR_UNSUPPORTED;
   }
   flatten_plan(c->plan, &c->dpass);
+  flatten_plan(c->plan, &c->dpass_split, true);
+  c->undo = undo_order(c->plan, c->dpass_split);
   c->bonds = chain_bonds(cfg->n_qubits);
   set_pass_entangler(c->plan, c->bonds, &c->dpass);
+  set_pass_entangler(c->plan, c->bonds, &c->dpass_split);
   set_bond_masks(c);
   static std::atomic<int> next_region{0};
   c->region = next_region.fetch_add(1) % kCoefRegions;
@@ -1046,6 +1098,11 @@ qml_status qml_set_workspace(qml_ctx* c, void* ws, size_t bytes, void* stream) {
   if (e == cudaSuccess)
     e = cudaMemcpyAsync(c->ws + c->lay.slot_index, si.data(), sizeof(int) * si.size(), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(c->ws + c->lay.dummy, 0, sizeof(float2) * (size_t)c->N, s);
+  if (e == cudaSuccess && !c->f64)
+    e = cudaMemcpyAsync(c->ws + c->lay.passes_split, c->dpass_split.data(), sizeof(DevPass) * c->dpass_split.size(),
+                        cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && !c->f64)
+    e = cudaMemcpyAsync(c->ws + c->lay.undo, c->undo.data(), sizeof(int) * c->undo.size(), cudaMemcpyHostToDevice, s);
   // the host vectors above are pageable: the copies complete before return
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   std::fill(c->ckpt_batch.begin(), c->ckpt_batch.end(), -1);
@@ -1192,6 +1249,7 @@ qml_status qml_set_entangler(qml_ctx* c, int n_bonds, const int* bonds) {
   c->bonds = b;
   set_bond_masks(c);
   set_pass_entangler(c->plan, c->bonds, &c->dpass);
+  set_pass_entangler(c->plan, c->bonds, &c->dpass_split);
   c->cnot = false;
   c->cnot_pairs.clear();
   return QML_OK;
@@ -1270,6 +1328,8 @@ qml_status qml_set_reupload(qml_ctx* c, int on) {
 }
 
 int qml_reupload(const qml_ctx* c) { return c ? (c->reupload ? 1 : 0) : -1; }
+
+int qml_split_form(const qml_ctx* c) { return c ? (use_split(c) ? 1 : 0) : -1; }
 
 int qml_entangler_bonds(const qml_ctx* c) {
   return c ? (int)(c->cnot ? c->cnot_pairs.size() : c->bonds.size()) : -1;
@@ -1407,6 +1467,15 @@ qml_status qml_forward_expect_f64(qml_ctx* c, const double* theta, const double*
   if (st != QML_OK) return st;
   if (!theta || !x || !psi || !expect || misaligned(psi, 16)) return QML_ERR_INVALID_ARG;
   DeviceGuard g(c->device);
+  if (c->fault == qml_ctx::FAULT_NAN) {  // injected: the first angle becomes NaN (in a copy of theta)
+    double* t = at<double>(c, c->lay.fault_theta);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t bytes = sizeof(double) * 3 * (size_t)c->cfg.n_layers * c->cfg.n_qubits;
+    cudaError_t e = cudaMemcpyAsync(t, theta, bytes, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(t, 0xff, sizeof(double), s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+    theta = t;
+  }
   return run_forward64(c, theta, x, B, reinterpret_cast<double2*>(psi), expect, static_cast<cudaStream_t>(stream));
 }
 

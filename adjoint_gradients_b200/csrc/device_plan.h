@@ -34,9 +34,15 @@ constexpr int kMaxOut = 30;           // out-of-tile qubits
 constexpr int kMaxQubits = 30;
 constexpr int kMaxOps = 24;
 constexpr int kMaxSlots = kMaxLayersPerPass * kTileBits;  // rotations per pass
-constexpr int kCoefRegions = 40;      // per-context regions of constant memory
+constexpr int kCoefRegions = 16;      // per-context regions of constant memory
+constexpr int kMaxDiag = kMaxLayersPerPass + 1;  // diagonal ops per pass (split rotations)
 
-enum : int { OP_EXCH = 1, OP_ROT = 2, OP_CZ = 3, OP_GEN = 4 };
+// OP_RY and OP_DIAG are the split form of OP_ROT and OP_CZ: every fused
+// rotation U = Rz(g) Ry(b) Rx(a) is rewritten exactly as Rz(phi1) Ry(vt)
+// Rz(phi2).  The Rz factors of consecutive layers and the layer's CZ bonds
+// are all diagonal and meet between the layers, so each layer boundary is one
+// diagonal op, and each rotation is a real Ry applied in tangent form.
+enum : int { OP_EXCH = 1, OP_ROT = 2, OP_CZ = 3, OP_GEN = 4, OP_RY = 5, OP_DIAG = 6 };
 
 // Tensor-copy (TMA) view of a pass's tile, used when n > 12: the state
 // [B][2^n] (working-state address order) is seen as a rank-5 tensor whose
@@ -53,6 +59,9 @@ enum : int { TD_PAD = 0, TD_IN = 1, TD_OUT = 2, TD_SAMPLE = 3, TD_OUT_SAMPLE = 4
 // OP_ROT : a = phase, b = register-bit mask, c = layer, d = first slot
 // OP_CZ  : a = phase, c = layer
 // OP_GEN : a = phase
+// OP_RY  : as OP_ROT (split form)
+// OP_DIAG: a = phase, c = layer l (the diagonal between layers l and l+1;
+//          -1: the one before layer 0), d = its table in the pass (0..kMaxDiag-1)
 struct DevOp {
   int kind, a, b, c, d;
 };
@@ -80,6 +89,9 @@ struct DevPass {
   uint32_t out_abit[kMaxOut];     // out-of-tile qubit -> its address bit
   uint32_t cz_reg[kPhases];  // bit j: entangler parity of the register part of position j
   uint32_t cz_nb[kPhases][kRegBits];  // CZ neighbours (qubit mask) of each register bit's qubit
+  int ndiag;                 // OP_DIAG ops in the pass (split form)
+  int rs_layer;              // split form, checkpoint pass: layer of the next diagonal op after the pass
+  uint32_t rs_mask;          // ... and the qubits it rotates between the pass's end and that op
   long long partial_off;     // float offset of this pass's gradient partials
   int slot_lq[kMaxSlots];    // slot -> layer * n + qubit
   DevOp ops[kMaxOps];        // forward order

@@ -33,11 +33,11 @@
 
 namespace qml {
 
-// Gate coefficients of the current pass, per context region: for slot s,
-// four float4 = broadcast pairs (ar, ai, -ai, br, bi, -bi, -br, 0).  Read
-// through the constant cache with warp-uniform indices, they feed the packed
-// FMAs from uniform registers instead of the vector register file.
-__constant__ float4 c_coef[kCoefRegions][kMaxSlots][4];
+// Gate coefficients of the current pass, per context region (CoefRegion in
+// kernels.cuh).  Read through the constant cache with warp-uniform indices,
+// they feed the packed FMAs from uniform registers instead of the vector
+// register file.
+__constant__ CoefRegion c_reg[kCoefRegions];
 
 namespace {
 
@@ -55,8 +55,8 @@ struct Coef {
 };
 
 __device__ __forceinline__ Coef const_coef(int region, int slot) {
-  const float4 f0 = c_coef[region][slot][0], f1 = c_coef[region][slot][1];
-  const float4 f2 = c_coef[region][slot][2], f3 = c_coef[region][slot][3];
+  const float4 f0 = c_reg[region].rot[slot][0], f1 = c_reg[region].rot[slot][1];
+  const float4 f2 = c_reg[region].rot[slot][2], f3 = c_reg[region].rot[slot][3];
   Coef c;
   c.ar = make_float2(f0.x, f0.y);
   c.ai = make_float2(f0.z, f0.w);
@@ -120,6 +120,57 @@ __device__ __forceinline__ void rot_fwd_k(int k, float2 (&re)[kPos], float2 (&im
   }
 }
 
+// Split form: the real rotation Ry on register pairs (x, y) = (j, j | 1 << K)
+// with one packed FMA per output, p = (t, t) and np = (-t, -t):
+//   tangent form   x <- x + np y,  y <- y + p x   ([[1, -t], [t, 1]] for p = t)
+//   cotangent form x <- y + np x,  y <- x + p y   ([[-u, 1], [1, u]] for p = u)
+// The backward pass un-applies a tangent-form rotation with p = -t (the
+// inverse up to the scale 1 + t^2) and a cotangent-form one with the same p
+// (that matrix squares to (1 + u^2) I).
+template <bool COT>
+__device__ __forceinline__ void ry_pair(float2& xr, float2& xi, float2& yr, float2& yi, float2 p, float2 np) {
+  const float2 x0r = xr, x0i = xi;
+  if (!COT) {
+    xr = __ffma2_rn(np, yr, x0r);
+    xi = __ffma2_rn(np, yi, x0i);
+    yr = __ffma2_rn(p, x0r, yr);
+    yi = __ffma2_rn(p, x0i, yi);
+  } else {
+    xr = __ffma2_rn(np, x0r, yr);
+    xi = __ffma2_rn(np, x0i, yi);
+    yr = __ffma2_rn(p, yr, x0r);
+    yi = __ffma2_rn(p, yi, x0i);
+  }
+}
+
+template <int K, bool COT>
+__device__ __forceinline__ void ry_fwd(float2 (&re)[kPos], float2 (&im)[kPos], float2 p, float2 np) {
+#pragma unroll
+  for (int j = 0; j < kPos; ++j)
+    if (!(j & (1 << K))) ry_pair<COT>(re[j], im[j], re[j | (1 << K)], im[j | (1 << K)], p, np);
+}
+
+template <bool COT>
+__device__ __forceinline__ void ry_fwd_k(int k, float2 (&re)[kPos], float2 (&im)[kPos], float2 p, float2 np) {
+  switch (k) {
+    case 0: ry_fwd<0, COT>(re, im, p, np); break;
+    case 1: ry_fwd<1, COT>(re, im, p, np); break;
+    case 2: ry_fwd<2, COT>(re, im, p, np); break;
+    case 3: ry_fwd<3, COT>(re, im, p, np); break;
+    default: ry_fwd<4, COT>(re, im, p, np); break;
+  }
+}
+
+// Applier of a register pair's 2x2 gate for rot_bwd_red: the fused SU(2)
+// with per-pair coefficients.
+template <class CF>
+struct Su2Ap {
+  CF cf;
+  __device__ __forceinline__ void operator()(int j, float2& xr, float2& xi, float2& yr, float2& yi) const {
+    su2(xr, xi, yr, yi, cf(j));
+  }
+};
+
 // Gradient terms of one qubit at the state just after its fused rotation, then
 // U^dagger on psi and lambda.  With psi in lane x and lambda in lane y:
 //   s_z = Im<lambda|Z|psi>, s_x = Im<lambda|X|psi>, s_y = Im<lambda|Y|psi>.
@@ -131,10 +182,10 @@ __device__ __forceinline__ void rot_fwd_k(int k, float2 (&re)[kPos], float2 (&im
 // The same call also finishes the warp sum of the previous qubit's terms
 // (pv): the shuffle steps of warp_reduce3 are spread over the pair loop so
 // that their latency hides behind this qubit's FMAs.  *r_prev receives the
-// sum as warp_reduce3 returns it.  cf(j) gives the coefficients of U^dagger
-// for register pair (j, j | 1 << K).
-template <int K, class CF>
-__device__ __forceinline__ float3 rot_bwd_red(float2 (&re)[kPos], float2 (&im)[kPos], const CF& cf, float3 pv,
+// sum as warp_reduce3 returns it.  ap(j, ...) un-applies the gate on register
+// pair (j, j | 1 << K).
+template <int K, class AP>
+__device__ __forceinline__ float3 rot_bwd_red(float2 (&re)[kPos], float2 (&im)[kPos], const AP& ap, float3 pv,
                                               int lane, float* r_prev) {
   const bool h16 = (lane & 16) != 0, h8 = (lane & 8) != 0;
   float k0 = h16 ? pv.z : pv.x, k1 = h16 ? 0.f : pv.y;
@@ -166,22 +217,80 @@ __device__ __forceinline__ float3 rot_bwd_red(float2 (&re)[kPos], float2 (&im)[k
     ax = __ffma2_rn(re[jj], si0, ax);    // y - x: l1r p0i - p1r l0i
     ay = __ffma2_rn(re[j], sr1, ay);     // x - y: p0r l1r - l0r p1r
     ay = __ffma2_rn(im[j], si1, ay);     // x - y: p0i l1i - l0i p1i
-    su2(re[j], im[j], re[jj], im[jj], cf(j));
+    ap(j, re[j], im[j], re[jj], im[jj]);
   }
   *r_prev = v;
   return make_float3(ax.y - ax.x, ay.x - ay.y, (az0.y - az0.x) - (az1.y - az1.x));
 }
 
+// Split form: only the gradient sums of qubit K (with the warp sum of the
+// previous qubit finished inside, as in rot_bwd_red); the caller then
+// un-applies Ry with ry_fwd.
+template <int K>
+__device__ __forceinline__ float3 rot_bwd_sums(const float2 (&re)[kPos], const float2 (&im)[kPos], float3 pv,
+                                               int lane, float* r_prev) {
+  const bool h16 = (lane & 16) != 0, h8 = (lane & 8) != 0;
+  float k0 = h16 ? pv.z : pv.x, k1 = h16 ? 0.f : pv.y;
+  const float s0 = h16 ? pv.x : pv.z, s1 = h16 ? pv.y : 0.f;
+  float v = 0.f;
+  float2 ax = make_float2(0.f, 0.f), ay = ax, az0 = ax, az1 = ax;
+#pragma unroll
+  for (int j = 0; j < kPos; ++j) {
+    if (j & (1 << K)) continue;
+    const int pi = (j & ((1 << K) - 1)) | ((j >> (K + 1)) << K);
+    if (pi == 0) {
+      k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+      k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+    } else if (pi == 3) {
+      v = h8 ? k1 : k0;
+      v += __shfl_xor_sync(0xffffffffu, h8 ? k0 : k1, 8);
+    } else if (pi == 6) {
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+    } else if (pi == 9) {
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+    } else if (pi == 12) {
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+    }
+    const int jj = j | (1 << K);
+    const float2 si0 = swap2(im[j]), si1 = swap2(im[jj]), sr1 = swap2(re[jj]);
+    az0 = __ffma2_rn(re[j], si0, az0);
+    az1 = __ffma2_rn(re[jj], si1, az1);
+    ax = __ffma2_rn(re[j], si1, ax);
+    ax = __ffma2_rn(re[jj], si0, ax);
+    ay = __ffma2_rn(re[j], sr1, ay);
+    ay = __ffma2_rn(im[j], si1, ay);
+  }
+  *r_prev = v;
+  return make_float3(ax.y - ax.x, ay.x - ay.y, (az0.y - az0.x) - (az1.y - az1.x));
+}
+
+__device__ __forceinline__ float3 rot_bwd_sums_k(int k, const float2 (&re)[kPos], const float2 (&im)[kPos],
+                                                 float3 pv, int lane, float* r_prev) {
+  switch (k) {
+    case 0: return rot_bwd_sums<0>(re, im, pv, lane, r_prev);
+    case 1: return rot_bwd_sums<1>(re, im, pv, lane, r_prev);
+    case 2: return rot_bwd_sums<2>(re, im, pv, lane, r_prev);
+    case 3: return rot_bwd_sums<3>(re, im, pv, lane, r_prev);
+    default: return rot_bwd_sums<4>(re, im, pv, lane, r_prev);
+  }
+}
+
+template <class AP>
+__device__ __forceinline__ float3 rot_bwd_red_ap(int k, float2 (&re)[kPos], float2 (&im)[kPos], const AP& ap,
+                                                 float3 pv, int lane, float* r_prev) {
+  switch (k) {
+    case 0: return rot_bwd_red<0>(re, im, ap, pv, lane, r_prev);
+    case 1: return rot_bwd_red<1>(re, im, ap, pv, lane, r_prev);
+    case 2: return rot_bwd_red<2>(re, im, ap, pv, lane, r_prev);
+    case 3: return rot_bwd_red<3>(re, im, ap, pv, lane, r_prev);
+    default: return rot_bwd_red<4>(re, im, ap, pv, lane, r_prev);
+  }
+}
+
 template <class CF>
 __device__ __forceinline__ float3 rot_bwd_red_k(int k, float2 (&re)[kPos], float2 (&im)[kPos], const CF& cf,
                                                 float3 pv, int lane, float* r_prev) {
-  switch (k) {
-    case 0: return rot_bwd_red<0>(re, im, cf, pv, lane, r_prev);
-    case 1: return rot_bwd_red<1>(re, im, cf, pv, lane, r_prev);
-    case 2: return rot_bwd_red<2>(re, im, cf, pv, lane, r_prev);
-    case 3: return rot_bwd_red<3>(re, im, cf, pv, lane, r_prev);
-    default: return rot_bwd_red<4>(re, im, cf, pv, lane, r_prev);
-  }
+  return rot_bwd_red_ap(k, re, im, Su2Ap<CF>{cf}, pv, lane, r_prev);
 }
 
 // Data re-uploading: Ry(x_q) (forward) or Ry(-x_q) (backward) on qubit K's
@@ -424,14 +533,21 @@ __device__ __forceinline__ void exchange(int x, int y, float2 (&re)[kPos], float
 // Per thread and layout the terms in T alone are one 32-bit word over the
 // register index (with the per-pass table S(R)), kept in shared memory; S(O)
 // is computed once per tile.
-__device__ __forceinline__ void apply_cz(float2 (&re)[kPos], float2 (&im)[kPos], uint32_t w_t, uint32_t n_t,
-                                         const uint32_t (&nb)[kRegBits], uint32_t base_q, uint32_t s_o) {
+// Bit j of the returned word: the entangler parity of this thread's position j.
+__device__ __forceinline__ uint32_t cz_word(uint32_t w_t, uint32_t n_t, const uint32_t (&nb)[kRegBits],
+                                           uint32_t base_q, uint32_t s_o) {
   const uint32_t qo = (s_o ^ (uint32_t)__popc(base_q & n_t)) & 1u;
   uint32_t w = w_t ^ (qo ? 0xffffffffu : 0u);
   const uint32_t pat[5] = {0xAAAAAAAAu, 0xCCCCCCCCu, 0xF0F0F0F0u, 0xFF00FF00u, 0xFFFF0000u};
 #pragma unroll
   for (int k = 0; k < kRegBits; ++k)
     if (__popc(base_q & nb[k]) & 1) w ^= pat[k];
+  return w;
+}
+
+__device__ __forceinline__ void apply_cz(float2 (&re)[kPos], float2 (&im)[kPos], uint32_t w_t, uint32_t n_t,
+                                         const uint32_t (&nb)[kRegBits], uint32_t base_q, uint32_t s_o) {
+  const uint32_t w = cz_word(w_t, n_t, nb, base_q, s_o);
 #pragma unroll
   for (int j = 0; j < kPos; ++j) {
     const uint32_t sb = (w << (31 - j)) & 0x80000000u;
@@ -475,7 +591,7 @@ enum MemOp { M_LOAD, M_STORE, M_STORE_STD, M_GEN, M_CKPT_STORE, M_CKPT_RESTORE }
 template <bool BWD, bool SLOW, int P, int V, int OP>
 __device__ __forceinline__ void mem_t(const PassArgs& a, const BlockCtx& bc, uint32_t tid, uint32_t base_q,
                                       uint32_t base_a, uint32_t unit_base, float2 (&re)[kPos], float2 (&im)[kPos],
-                                      int slot) {
+                                      int slot, float rs) {
   uint32_t aq, ut;
   thread_pos<P, V>(bc, tid, &aq, &ut);
   constexpr bool std_index = !(OP == M_LOAD || OP == M_STORE || OP == M_STORE_STD);
@@ -535,8 +651,8 @@ __device__ __forceinline__ void mem_t(const PassArgs& a, const BlockCtx& bc, uin
         float2 v;
         if (a.storage == 0) v = reinterpret_cast<const float2*>(a.ckpt)[e];
         else v = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(a.ckpt)[e]);
-        re[j].x = v.x;
-        im[j].x = v.y;
+        re[j].x = v.x * rs;
+        im[j].x = v.y * rs;
       }
     }
   }
@@ -545,10 +661,10 @@ __device__ __forceinline__ void mem_t(const PassArgs& a, const BlockCtx& bc, uin
 template <bool BWD, bool SLOW, int V, int OP>
 __device__ __forceinline__ void mem_op(int phase, const PassArgs& a, const BlockCtx& bc, uint32_t tid,
                                        uint32_t base_q, uint32_t base_a, uint32_t unit_base, float2 (&re)[kPos],
-                                       float2 (&im)[kPos], int slot = 0) {
+                                       float2 (&im)[kPos], int slot = 0, float rs = 1.f) {
   // memory ops run in phase 0 or 1 (the planner never picks phase 2)
-  if (phase == 0) mem_t<BWD, SLOW, 0, V, OP>(a, bc, tid, base_q, base_a, unit_base, re, im, slot);
-  else mem_t<BWD, SLOW, 1, V, OP>(a, bc, tid, base_q, base_a, unit_base, re, im, slot);
+  if (phase == 0) mem_t<BWD, SLOW, 0, V, OP>(a, bc, tid, base_q, base_a, unit_base, re, im, slot, rs);
+  else mem_t<BWD, SLOW, 1, V, OP>(a, bc, tid, base_q, base_a, unit_base, re, im, slot, rs);
 }
 
 // Prefetch of the block's next tile: each thread copies its own positions of
@@ -694,7 +810,7 @@ __device__ __forceinline__ void load_tma_t(float2 (&re)[kPos], float2 (&im)[kPos
 // is read into registers (so no state registers are live here).
 template <int P, int V>
 __device__ __forceinline__ void restore_tma_t(const PassArgs& a, const BlockCtx& bc, const DevPass& Pp, uint32_t tid,
-                                              uint32_t base_q, uint32_t unit_base, float2* buf, int slot) {
+                                              uint32_t base_q, uint32_t unit_base, float2* buf, int slot, float rs) {
   uint32_t aq, ut;
   thread_pos<P, V>(bc, tid, &aq, &ut);
   aq |= base_q;
@@ -716,8 +832,8 @@ __device__ __forceinline__ void restore_tma_t(const PassArgs& a, const BlockCtx&
     float2 v;
     if (a.storage == 0) v = reinterpret_cast<const float2*>(a.ckpt)[e];
     else v = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(a.ckpt)[e]);
-    buf[off].x = v.x;
-    buf[off + kTilePos].x = v.y;
+    buf[off].x = v.x * rs;
+    buf[off + kTilePos].x = v.y * rs;
   }
 }
 
@@ -758,6 +874,65 @@ __device__ __forceinline__ void cz_op(int phase, float2 (&re)[kPos], float2 (&im
     case 0: cz_t<0, V>(re, im, bc, Pp, tid, base_q, s_o); break;
     case 1: cz_t<1, V>(re, im, bc, Pp, tid, base_q, s_o); break;
     default: cz_t<2, V>(re, im, bc, Pp, tid, base_q, s_o); break;
+  }
+}
+
+// Split form: the diagonal op d (layer l) in layout P.  A position i = T | O |
+// R (thread, out-of-tile and register bits) is multiplied by
+//   (-1)^{S(i)} * f(T) f(O) * R_d[j],
+// with S the entangler parity (l >= 0 only), f the product of the per-qubit
+// factors dq[l + 1][q][bit] over the bits named, and R_d[j] the pass's
+// constant table for the register part j (the global scale folded in).  The
+// factor applies to both lanes of a pair (two samples, or psi and lambda).
+template <int P, int V>
+__device__ __forceinline__ void diag_t(float2 (&re)[kPos], float2 (&im)[kPos], const BlockCtx& bc,
+                                       const DevPass& Pp, const PassArgs& a, int region, int d, int l, uint32_t tid,
+                                       uint32_t base_q, uint32_t s_o) {
+  const float2* dq = a.dq + (size_t)(l + 1) * a.n * 2;
+  float fr = 1.f, fi = 0.f;
+  auto mul = [&](float2 v) {
+    const float r = fr * v.x - fi * v.y;
+    fi = fmaf(fr, v.y, fi * v.x);
+    fr = r;
+  };
+#pragma unroll
+  for (int m = 0; m < kThrBits; ++m) {
+    const int q = Pp.tile_q[thr_tbit<P, V>(m)];
+    if (q >= 0) mul(__ldg(&dq[2 * q + ((tid >> m) & 1u)]));
+  }
+  for (int k = 0; k < Pp.n_out; ++k) {
+    const int q = Pp.out_q[k];
+    mul(__ldg(&dq[2 * q + ((base_q >> q) & 1u)]));
+  }
+  uint32_t w = 0;
+  if (l >= 0) {
+    uint32_t nb[kRegBits];
+#pragma unroll
+    for (int k = 0; k < kRegBits; ++k) nb[k] = Pp.cz_nb[P][k];
+    w = cz_word(bc.cz_w[P][tid], bc.cz_n[P][tid], nb, base_q, s_o);
+  }
+  // per position: the factor (scalar complex, table entries as constant
+  // operands), its sign, then the product with both lanes
+#pragma unroll
+  for (int j = 0; j < kPos; ++j) {
+    const float2 r = c_reg[region].diag[d][j];
+    const uint32_t sb = (w << (31 - j)) & 0x80000000u;
+    const float gr = __uint_as_float(__float_as_uint(fmaf(-fi, r.y, fr * r.x)) ^ sb);
+    const float gi = __uint_as_float(__float_as_uint(fmaf(fr, r.y, fi * r.x)) ^ sb);
+    const float2 xr = re[j], xi = im[j];
+    re[j] = make_float2(fmaf(gr, xr.x, -gi * xi.x), fmaf(gr, xr.y, -gi * xi.y));
+    im[j] = make_float2(fmaf(gi, xr.x, gr * xi.x), fmaf(gi, xr.y, gr * xi.y));
+  }
+}
+
+template <int V>
+__device__ __forceinline__ void diag_op(int phase, float2 (&re)[kPos], float2 (&im)[kPos], const BlockCtx& bc,
+                                        const DevPass& Pp, const PassArgs& a, int region, int d, int l, uint32_t tid,
+                                        uint32_t base_q, uint32_t s_o) {
+  switch (phase) {
+    case 0: diag_t<0, V>(re, im, bc, Pp, a, region, d, l, tid, base_q, s_o); break;
+    case 1: diag_t<1, V>(re, im, bc, Pp, a, region, d, l, tid, base_q, s_o); break;
+    default: diag_t<2, V>(re, im, bc, Pp, a, region, d, l, tid, base_q, s_o); break;
   }
 }
 
@@ -816,7 +991,8 @@ __device__ __forceinline__ void cz_thread_terms(BlockCtx& bc, const DevPass& Pp,
 // into the layer's rotations.  RE 1: the tile holds no batch-unit bit, so each
 // thread's amplitudes belong to one batch unit and each rotation takes one set
 // of coefficients.  RE 2: tiles with batch-unit bits (n < 12), coefficients
-// per register pair.
+// per register pair.  RE 3: the split form (OP_RY and OP_DIAG ops; no
+// re-uploading).
 
 template <bool BWD, int MODE, int V, int RE>
 __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
@@ -824,6 +1000,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
                 const __grid_constant__ CUtensorMap tm1) {
   constexpr bool SLOW = MODE == 0;
   constexpr bool TMA = MODE == 2;
+  constexpr bool REUP = RE == 1 || RE == 2;  // data re-uploading folded into the fused rotations
+  constexpr bool SPLIT = RE == 3;            // split form: OP_RY / OP_DIAG instead of OP_ROT / OP_CZ
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   float4* tile = reinterpret_cast<float4*>(smem_raw);
   BlockCtx* bc = reinterpret_cast<BlockCtx*>(smem_raw + (size_t)kSmemSlots * sizeof(float4));
@@ -834,6 +1012,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   const int region = a.region;
   const int nacc = P.nslots * 3;
   const bool loads = BWD || !P.gen;  // the forward's encoding pass reads nothing
+  const float rs = (BWD && a.rscale) ? __ldg(a.rscale) : 1.f;  // scale of a restored checkpoint (split form)
   const uint32_t tile_s = (uint32_t)__cvta_generic_to_shared(tile);
   const uint32_t mbar = (uint32_t)__cvta_generic_to_shared(&bc->mbar);
 
@@ -906,8 +1085,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
       }
       float2* tb = reinterpret_cast<float2*>(tile);
       if (BWD && P.ckpt >= 0) {
-        if (mem_ph == 0) restore_tma_t<0, V>(a, *bc, P, tid, base_q, unit_base, tb, P.ckpt);
-        else restore_tma_t<1, V>(a, *bc, P, tid, base_q, unit_base, tb, P.ckpt);
+        if (mem_ph == 0) restore_tma_t<0, V>(a, *bc, P, tid, base_q, unit_base, tb, P.ckpt, rs);
+        else restore_tma_t<1, V>(a, *bc, P, tid, base_q, unit_base, tb, P.ckpt, rs);
       }
       load_tma<V>(mem_ph, re, im, tb, P, tid);
     }
@@ -921,9 +1100,25 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
         const DevOp op = P.ops[oi];
         if (op.kind == OP_EXCH) {
           exchange<V>(op.a, op.b, re, im, tile, tid);
+        } else if constexpr (SPLIT) {
+          if (op.kind == OP_RY) {
+            int slot = op.d;
+#pragma unroll
+            for (int k = 0; k < kRegBits; ++k)
+              if ((op.b >> k) & 1) {
+                const float4 f0 = c_reg[region].rot[slot][0];
+                const bool cot = c_reg[region].rot[slot][1].x != 0.f;
+                ++slot;
+                const float2 p = make_float2(f0.x, f0.y), np = make_float2(f0.z, f0.w);
+                if (cot) ry_fwd_k<true>(k, re, im, p, np);
+                else ry_fwd_k<false>(k, re, im, p, np);
+              }
+          } else if (op.kind == OP_DIAG) {
+            diag_op<V>(op.a, re, im, *bc, P, a, region, op.d, op.c, tid, base_q, s_o);
+          }
         } else if (op.kind == OP_ROT) {
           int slot = op.d;
-          if (RE != 0) {  // the encoding again, folded into the layer's rotations
+          if (REUP) {  // the encoding again, folded into the layer's rotations
             uint32_t unit, mu[kRegBits];
             int rq[kRegBits];
             unit_maps<V>(op.a, *bc, tid, unit_base, &unit, mu, rq);
@@ -956,12 +1151,41 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
       if (TMA) {
       } else if (have_pf) load_prefetched<V>(P.store_phase, re, im, tile, tid);
       else mem_op<true, SLOW, V, M_LOAD>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
-      if (!TMA && P.ckpt >= 0) mem_op<true, SLOW, V, M_CKPT_RESTORE>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im, P.ckpt);
+      if (!TMA && P.ckpt >= 0)
+        mem_op<true, SLOW, V, M_CKPT_RESTORE>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im, P.ckpt, rs);
       if (pf_next && pf_at < 0) prefetch_next();
       for (int oi = P.nops - 1; oi >= 0; --oi) {
         const DevOp op = P.ops[oi];
         if (op.kind == OP_EXCH) {
           exchange<V>(op.b, op.a, re, im, tile, tid);
+        } else if constexpr (SPLIT) {
+          if (op.kind == OP_RY) {
+            // the same sums, then Ry un-applied (tangent or cotangent form)
+            int slot = op.d, pslot = -1;
+            float3 pend = make_float3(0.f, 0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < kRegBits; ++k)
+              if ((op.b >> k) & 1) {
+                float r;
+                float3 v;
+                const float4 f0 = c_reg[region].rot[slot][0];
+                const bool cot = c_reg[region].rot[slot][1].x != 0.f;
+                const float2 p = make_float2(f0.x, f0.y), np = make_float2(f0.z, f0.w);
+                v = rot_bwd_sums_k(k, re, im, pend, lane, &r);
+                if (cot) ry_fwd_k<true>(k, re, im, p, np);
+                else ry_fwd_k<false>(k, re, im, p, np);
+                if (pslot >= 0 && (lane & 7) == 0 && lane < 24) acc[warp * nacc + pslot * 3 + (lane >> 3)] += r;
+                pend = v;
+                pslot = slot++;
+              }
+            if (pslot >= 0) {
+              const float r = warp_reduce3(pend.x, pend.y, pend.z, lane);
+              if ((lane & 7) == 0 && lane < 24) acc[warp * nacc + pslot * 3 + (lane >> 3)] += r;
+            }
+          } else if (op.kind == OP_DIAG) {
+            // the diagonal before layer 0 needs no un-applying: nothing reads the state after it
+            if (op.c >= 0) diag_op<V>(op.a, re, im, *bc, P, a, region, op.d, op.c, tid, base_q, s_o);
+          }
         } else if (op.kind == OP_ROT) {
           // each rotation finishes the warp sum of the previous one
           int slot = op.d, pslot = -1;
@@ -969,7 +1193,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
           // re-uploading: Ry(-x) of the layer's encoding joins U^dagger
           uint32_t unit = 0, mu[kRegBits] = {0u, 0u, 0u, 0u, 0u};
           int rq[kRegBits] = {0, 0, 0, 0, 0};
-          if (RE != 0) unit_maps<V>(op.a, *bc, tid, unit_base, &unit, mu, rq);
+          if (REUP) unit_maps<V>(op.a, *bc, tid, unit_base, &unit, mu, rq);
 #pragma unroll
           for (int k = 0; k < kRegBits; ++k)
             if ((op.b >> k) & 1) {
@@ -1017,18 +1241,9 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
 
 // ----------------------------------------------------------------- helpers
 
-// Gate coefficients of every pass slot: U = Rz(g) Ry(b) Rx(a) =
-// [[A, B], [-conj B, conj A]] computed in fp64 and rounded to fp32 broadcast
-// pairs, and U^dagger = [[conj A, -B], ...] for the backward passes.
-// Output: [pass][kMaxSlots][4] float4 per direction.
-__global__ void prep_pass_coef_kernel(const DevPass* passes, int n_passes, const float* theta, float4* cf,
-                                      float4* ci) {
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= n_passes * kMaxSlots) return;
-  const int p = idx / kMaxSlots, s = idx % kMaxSlots;
-  if (s >= passes[p].nslots) return;
-  const int lq = passes[p].slot_lq[s];
-  const double al = theta[lq * 3 + 0], be = theta[lq * 3 + 1], ga = theta[lq * 3 + 2];
+// U = Rz(g) Ry(b) Rx(a) = [[A, B], [-conj B, conj A]] in fp64 (half angles).
+__device__ __forceinline__ void su2_of(const float* th, double* ar, double* ai, double* br, double* bi) {
+  const double al = th[0], be = th[1], ga = th[2];
   double sa, ca, sb, cb, sg, cg;
   sincos(0.5 * al, &sa, &ca);
   sincos(0.5 * be, &sb, &cb);
@@ -1036,20 +1251,183 @@ __global__ void prep_pass_coef_kernel(const DevPass* passes, int n_passes, const
   // (Ry Rx)[0][0] = cb ca + i sb sa, (Ry Rx)[0][1] = -sb ca - i cb sa; row 0 of Rz is e^{-i g/2}
   const double p_re = cb * ca, p_im = sb * sa;
   const double q_re = -sb * ca, q_im = -cb * sa;
-  const double ar = cg * p_re + sg * p_im, ai = cg * p_im - sg * p_re;
-  const double br = cg * q_re + sg * q_im, bi = cg * q_im - sg * q_re;
+  *ar = cg * p_re + sg * p_im;
+  *ai = cg * p_im - sg * p_re;
+  *br = cg * q_re + sg * q_im;
+  *bi = cg * q_im - sg * q_re;
+}
+
+// Gate coefficients of every pass slot: U computed in fp64 and rounded to
+// fp32 broadcast pairs, and U^dagger = [[conj A, -B], ...] for the backward
+// passes.  Output: one CoefRegion per pass and direction.
+__global__ void prep_pass_coef_kernel(const DevPass* passes, int n_passes, const float* theta, CoefRegion* cf,
+                                      CoefRegion* ci) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n_passes * kMaxSlots) return;
+  const int p = idx / kMaxSlots, s = idx % kMaxSlots;
+  if (s >= passes[p].nslots) return;
+  const int lq = passes[p].slot_lq[s];
+  double ar, ai, br, bi;
+  su2_of(theta + lq * 3, &ar, &ai, &br, &bi);
   const float far = (float)ar, fai = (float)ai, fbr = (float)br, fbi = (float)bi;
-  float4* f = cf + (size_t)idx * 4;
+  float4* f = cf[p].rot[s];
   f[0] = make_float4(far, far, fai, fai);
   f[1] = make_float4(-fai, -fai, fbr, fbr);
   f[2] = make_float4(fbi, fbi, -fbi, -fbi);
   f[3] = make_float4(-fbr, -fbr, 0.f, 0.f);
   // U^dagger: A' = conj A, B' = -B
-  float4* g = ci + (size_t)idx * 4;
+  float4* g = ci[p].rot[s];
   g[0] = make_float4(far, far, -fai, -fai);
   g[1] = make_float4(fai, fai, -fbr, -fbr);
   g[2] = make_float4(-fbi, -fbi, fbi, fbi);
   g[3] = make_float4(fbr, fbr, 0.f, 0.f);
+}
+
+// ----------------------------------------------------- split-form tables
+//
+// U = Rz(g) Ry(b) Rx(a) = Rz(phi1) Ry(vt) Rz(phi2) with A = e^{-i sig} c,
+// B = -e^{-i del} s, c = |A|, s = |B|, sig = (phi1 + phi2) / 2,
+// del = (phi1 - phi2) / 2.  Every state the split passes hold is the split
+// circuit's state times a "frame": a real scale and a sign (-1 on the 0 half)
+// for each qubit rotated in cotangent form since the last diagonal op.  Each
+// diagonal op removes the frame of its layer's rotations (forward) or restores
+// it (backward), so that the last pass leaves the exact final state.
+
+__global__ void split_rot_kernel(const float* theta, int total, SplitRot* out) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= total) return;
+  double ar, ai, br, bi;
+  su2_of(theta + (size_t)idx * 3, &ar, &ai, &br, &bi);
+  const double c = sqrt(ar * ar + ai * ai), s = sqrt(br * br + bi * bi);
+  const double sig = -atan2(ai, ar), del = -atan2(-bi, -br);
+  SplitRot r;
+  r.phi1 = sig + del;
+  r.phi2 = sig - del;
+  r.cot = s > c ? 1 : 0;
+  r.tau = r.cot ? c / s : s / c;
+  r.g = r.cot ? -1.0 / s : 1.0 / c;
+  r.k2 = r.g * r.g;
+  r.pad = 0;
+  out[idx] = r;
+}
+
+// Per layer: the frame of all its rotations, and per rotation the scale of
+// the backward sums.  At the sum of rotation j the backward state is
+// rho * gam * Z^m times the split circuit's (psi, lambda), where rho is the
+// product of k2 over the layer's rotations already un-applied and gam the
+// product of g over those still applied; the sums scale by (rho gam)^2, and
+// their X and Y parts flip sign when j itself is in cotangent form.
+__global__ void split_layer_kernel(const SplitRot* rot, const int* undo, int L, int n, SplitLayer* lay,
+                                   double* gfix) {
+  const int l = blockIdx.x * blockDim.x + threadIdx.x;
+  if (l >= L) return;
+  const SplitRot* r = rot + (size_t)l * n;
+  double gam = 1.0, rho = 1.0;
+  uint32_t m = 0;
+  for (int q = 0; q < n; ++q) {
+    gam *= r[q].g;
+    rho *= r[q].k2;
+    if (r[q].cot) m |= 1u << q;
+  }
+  lay[l].gam = gam;
+  lay[l].rho = rho;
+  lay[l].cot_mask = m;
+  lay[l].pad = 0;
+  double undone_k2 = 1.0, applied_g = gam;
+  for (int i = 0; i < n; ++i) {
+    const int q = undo[(size_t)l * n + i];
+    const double f = undone_k2 * applied_g;
+    const double sc = (r[q].cot ? -1.0 : 1.0) / (f * f);
+    gfix[((size_t)l * n + q) * 2 + 0] = sc;
+    gfix[((size_t)l * n + q) * 2 + 1] = r[q].phi1;
+    undone_k2 *= r[q].k2;
+    applied_g /= r[q].g;
+  }
+}
+
+// Factor of qubit q's bit b in the diagonal op after layer l (l = -1: before
+// layer 0): Rz(phi1 of layer l + phi2 of layer l + 1), times -1 on b = 1 when
+// q was rotated in cotangent form in layer l; conjugated for the backward.
+__device__ __forceinline__ double2 diag_factor(const SplitRot* rot, const SplitLayer* lay, int L, int n, int l, int q,
+                                               int b, bool bwd) {
+  const double w = (l >= 0 ? rot[(size_t)l * n + q].phi1 : 0.0) + (l + 1 < L ? rot[(size_t)(l + 1) * n + q].phi2 : 0.0);
+  double sn, cs;
+  sincos(0.5 * w, &sn, &cs);
+  double re = cs, im = b ? sn : -sn;
+  if (bwd) im = -im;
+  if (l >= 0 && b && ((lay[l].cot_mask >> q) & 1u)) re = -re, im = -im;
+  return make_double2(re, im);
+}
+
+__global__ void split_diag_kernel(const SplitRot* rot, const SplitLayer* lay, int L, int n, float2* dq_f,
+                                  float2* dq_b) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;  // ((l + 1) * n + q) * 2 + b
+  if (idx >= (L + 1) * n * 2) return;
+  const int b = idx & 1, q = (idx >> 1) % n, l = (idx >> 1) / n - 1;
+  const double2 f = diag_factor(rot, lay, L, n, l, q, b, false);
+  const double2 g = diag_factor(rot, lay, L, n, l, q, b, true);
+  dq_f[idx] = make_float2((float)f.x, (float)f.y);
+  dq_b[idx] = make_float2((float)g.x, (float)g.y);
+}
+
+// Per pass: rotation slots, the register tables of its diagonal ops, and the
+// restore scale.  Items per pass: kMaxSlots slots, kMaxDiag * kPos table
+// entries, one scale.
+constexpr int kSplitItems = kMaxSlots + kMaxDiag * kPos + 1;
+
+__global__ void split_pass_kernel(const DevPass* passes, int n_passes, const SplitRot* rot, const SplitLayer* lay,
+                                  int L, int n, CoefRegion* cf, CoefRegion* ci, float* rscale) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n_passes * kSplitItems) return;
+  const int p = idx / kSplitItems, it = idx % kSplitItems;
+  const DevPass& P = passes[p];
+  if (it < kMaxSlots) {
+    if (it >= P.nslots) return;
+    const SplitRot r = rot[P.slot_lq[it]];
+    const float t = (float)r.tau;
+    // forward: p = tau in both forms; backward: -tau in tangent form
+    cf[p].rot[it][0] = make_float4(t, t, -t, -t);
+    cf[p].rot[it][1] = make_float4((float)r.cot, 0.f, 0.f, 0.f);
+    const float tb = r.cot ? t : -t;
+    ci[p].rot[it][0] = make_float4(tb, tb, -tb, -tb);
+    ci[p].rot[it][1] = make_float4((float)r.cot, 0.f, 0.f, 0.f);
+    return;
+  }
+  if (it == kSplitItems - 1) {
+    // backward checkpoint pass: the restored state takes the scale rho that
+    // the un-applied rotations between the pass's end and the next diagonal
+    // op have given the backward state
+    double rho = 1.0;
+    if (P.ckpt >= 0 && P.rs_layer >= 0)
+      for (int q = 0; q < n; ++q)
+        if ((P.rs_mask >> q) & 1u) rho *= rot[(size_t)P.rs_layer * n + q].k2;
+    rscale[p] = (float)rho;
+    return;
+  }
+  const int e = it - kMaxSlots, d = e / kPos, j = e % kPos;
+  int ph = -1, l = 0;
+  for (int o = 0; o < P.nops; ++o)
+    if (P.ops[o].kind == OP_DIAG && P.ops[o].d == d) ph = P.ops[o].a, l = P.ops[o].c;
+  if (ph < 0) return;
+  // the global scale: forward 1 / gam(l); backward gam(l) / rho(l + 1)
+  double fr = l >= 0 ? 1.0 / lay[l].gam : 1.0, fi = 0.0;
+  double br = l >= 0 ? lay[l].gam / (l + 1 < L ? lay[l + 1].rho : 1.0) : 0.0, bi = 0.0;
+  for (int k = 0; k < kRegBits; ++k) {
+    const int tb = ph == 0 ? k : ph == 1 ? 5 + k : (k < 2 ? 10 + k : k - 2);  // reg_tbit
+    const int q = P.tile_q[tb];
+    if (q < 0) continue;  // a batch-unit bit
+    const int b = (j >> k) & 1;
+    const double2 f = diag_factor(rot, lay, L, n, l, q, b, false);
+    const double2 g = diag_factor(rot, lay, L, n, l, q, b, true);
+    double t = fr * f.x - fi * f.y;
+    fi = fr * f.y + fi * f.x;
+    fr = t;
+    t = br * g.x - bi * g.y;
+    bi = br * g.y + bi * g.x;
+    br = t;
+  }
+  cf[p].diag[d][j] = make_float2((float)fr, (float)fi);
+  ci[p].diag[d][j] = make_float2((float)br, (float)bi);
 }
 
 // (cos, sin)(x/2) for the two samples of each forward unit.
@@ -1105,9 +1483,13 @@ __global__ void expect_final_kernel(const double* partial, int chunks, int B, fl
 // (s_x, s_y, s_z) = Im<lambda|(X, Y, Z)|psi> into the three angle gradients:
 //   d/dg = s_z,  d/db = cos g s_y - sin g s_x,
 //   d/da = cos b (cos g s_x + sin g s_y) - sin b s_z.
+// Split form (gfix non-null): the sums were taken after Ry of the rotation,
+// in the backward state's frame; gfix[.][0] takes them to the split circuit's
+// states and Rz(phi1) (gfix[.][1]) to the state after the whole rotation:
+// Rz(f)^dagger X Rz(f) = cos f X - sin f Y, Rz(f)^dagger Y Rz(f) = sin f X + cos f Y.
 __global__ void grad_reduce_kernel(const DevPass* passes, const int* slot_pass,
                                    const int* slot_index, const float* partials, int grid,
-                                   const float* theta, int L, int n, float* grad,
+                                   const float* theta, const double* gfix, int L, int n, float* grad,
                                    unsigned* status) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= L * n) return;
@@ -1120,6 +1502,17 @@ __global__ void grad_reduce_kernel(const DevPass* passes, const int* slot_pass,
     sx += base[(size_t)c * stride + 0];
     sy += base[(size_t)c * stride + 1];
     sz += base[(size_t)c * stride + 2];
+  }
+  if (gfix) {
+    const double sc = gfix[(size_t)idx * 2 + 0], f = gfix[(size_t)idx * 2 + 1];
+    double sf, cf;
+    sincos(f, &sf, &cf);
+    sx *= sc;
+    sy *= sc;
+    sz *= fabs(sc);
+    const double tx = cf * sx - sf * sy;
+    sy = sf * sx + cf * sy;
+    sx = tx;
   }
   const double be = theta[idx * 3 + 1], ga = theta[idx * 3 + 2];
   double sb, cb, sg, cg;
@@ -1293,7 +1686,9 @@ size_t pass_smem_bytes(int max_slots) {
   X(false, 0, 0, 0) X(true, 0, 0, 0) X(false, 1, 0, 0) X(true, 1, 0, 0) X(false, 1, 1, 0) X(true, 1, 1, 0)         \
   X(false, 2, 0, 0) X(true, 2, 0, 0) X(false, 2, 1, 0) X(true, 2, 1, 0) X(false, 1, 0, 1) X(true, 1, 0, 1)         \
   X(false, 1, 1, 1) X(true, 1, 1, 1) X(false, 2, 0, 1) X(true, 2, 0, 1) X(false, 2, 1, 1) X(true, 2, 1, 1)         \
-  X(false, 1, 0, 2) X(true, 1, 0, 2) X(false, 1, 1, 2) X(true, 1, 1, 2)
+  X(false, 1, 0, 2) X(true, 1, 0, 2) X(false, 1, 1, 2) X(true, 1, 1, 2) X(false, 0, 0, 3) X(true, 0, 0, 3)         \
+  X(false, 1, 0, 3) X(true, 1, 0, 3) X(false, 1, 1, 3) X(true, 1, 1, 3) X(false, 2, 0, 3) X(true, 2, 0, 3)         \
+  X(false, 2, 1, 3) X(true, 2, 1, 3)
 
 cudaError_t set_pass_smem_attr(size_t smem) {
   cudaError_t e = cudaSuccess;
@@ -1335,8 +1730,11 @@ cudaError_t launch_pass(bool backward, const PassArgs& a, const DevPass& p, cons
   const int mode = p.slow ? 0 : p.tma ? 2 : 1;
   const CUtensorMap& m0 = *reinterpret_cast<const CUtensorMap*>(maps.m0);
   const CUtensorMap& m1 = *reinterpret_cast<const CUtensorMap*>(maps.m1);
-  // re-uploading: RE 2 where the tile holds a batch-unit bit, else RE 1
+  // re-uploading: RE 2 where the tile holds a batch-unit bit, else RE 1;
+  // split-form passes: RE 3
   int re = 0;
+  for (int o = 0; o < p.nops; ++o)
+    if (p.ops[o].kind == OP_RY || p.ops[o].kind == OP_DIAG) re = 3;
   if (a.reupload) {
     re = 1;
     for (int b = 0; b < kTileBits; ++b)
@@ -1411,16 +1809,35 @@ cudaError_t encode_pass_maps(const DevPass& p, int n, int B, bool backward, cons
   return cudaSuccess;
 }
 
-cudaError_t copy_pass_coef(int region, const float4* src, int nslots, cudaStream_t s) {
-  if (nslots <= 0) return cudaSuccess;
-  const size_t off = (size_t)region * kMaxSlots * 4 * sizeof(float4);
-  return cudaMemcpyToSymbolAsync(c_coef, src, (size_t)nslots * 4 * sizeof(float4), off, cudaMemcpyDeviceToDevice, s);
+cudaError_t copy_pass_coef(int region, const CoefRegion* src, int nslots, int ndiag, cudaStream_t s) {
+  const size_t off = (size_t)region * sizeof(CoefRegion);
+  // the rotation slots, and with diagonal ops the whole region (its tables follow the slots)
+  const size_t bytes = ndiag > 0 ? sizeof(CoefRegion) : (size_t)nslots * sizeof(src->rot[0]);
+  if (bytes == 0) return cudaSuccess;
+  return cudaMemcpyToSymbolAsync(c_reg, src, bytes, off, cudaMemcpyDeviceToDevice, s);
 }
 
-cudaError_t launch_prep_pass_coef(const DevPass* passes, int n_passes, const float* theta, float4* cf, float4* ci,
-                                  cudaStream_t s) {
+cudaError_t launch_prep_pass_coef(const DevPass* passes, int n_passes, const float* theta, CoefRegion* cf,
+                                  CoefRegion* ci, cudaStream_t s) {
   const int tot = n_passes * kMaxSlots;
   prep_pass_coef_kernel<<<(tot + 127) / 128, 128, 0, s>>>(passes, n_passes, theta, cf, ci);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prep_split(const DevPass* passes, int n_passes, const float* theta, int L, int n,
+                              const int* undo, SplitRot* rot, SplitLayer* lay, double* gfix, float2* dq_f,
+                              float2* dq_b, CoefRegion* cf, CoefRegion* ci, float* rscale, cudaStream_t s) {
+  const int nr = L * n;
+  split_rot_kernel<<<(nr + 127) / 128, 128, 0, s>>>(theta, nr, rot);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  split_layer_kernel<<<(L + 127) / 128, 128, 0, s>>>(rot, undo, L, n, lay, gfix);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int nd = (L + 1) * n * 2;
+  split_diag_kernel<<<(nd + 127) / 128, 128, 0, s>>>(rot, lay, L, n, dq_f, dq_b);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int np = n_passes * kSplitItems;
+  split_pass_kernel<<<(np + 127) / 128, 128, 0, s>>>(passes, n_passes, rot, lay, L, n, cf, ci, rscale);
   return cudaGetLastError();
 }
 
@@ -1449,11 +1866,11 @@ cudaError_t launch_expect(const float2* psi, int B, int n, double* partial, floa
 }
 
 cudaError_t launch_grad_reduce(const DevPass* passes, const int* slot_pass, const int* slot_index,
-                               const float* partials, int grid, const float* theta, int L, int n,
-                               float* grad, unsigned* status, cudaStream_t s) {
+                               const float* partials, int grid, const float* theta, const double* gfix, int L,
+                               int n, float* grad, unsigned* status, cudaStream_t s) {
   const int tot = L * n;
   grad_reduce_kernel<<<(tot + 127) / 128, 128, 0, s>>>(passes, slot_pass, slot_index, partials,
-                                                       grid, theta, L, n, grad, status);
+                                                       grid, theta, gfix, L, n, grad, status);
   return cudaGetLastError();
 }
 

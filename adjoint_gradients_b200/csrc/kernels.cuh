@@ -8,6 +8,35 @@
 
 namespace qml {
 
+// Gate coefficients of one pass, as copied into a context's constant-memory
+// region before the pass is launched.
+//   rot[s]: rotation slot s.  Full SU(2) (OP_ROT): four float4 of broadcast
+//     pairs (ar, ai, -ai, br, bi, -bi, -br, 0).  Split form (OP_RY): rot[s][0]
+//     = (p, p, -p, -p) with p the tangent-form coefficient, rot[s][1].x = 1
+//     for the cotangent form (see ry_apply in kernels.cu).
+//   diag[d][j]: split form, diagonal op d: the complex factor (re, im) of
+//     the register part j of a position.
+struct CoefRegion {
+  float4 rot[kMaxSlots][4];
+  float2 diag[kMaxDiag][1 << kRegBits];
+};
+
+// Split form, per (layer, qubit): U = Rz(g) Ry(b) Rx(a) = Rz(phi1) Ry(vt) Rz(phi2)
+// with (c, s) = (cos, sin)(vt / 2) >= 0.  The kernels apply Ry(vt) as
+// tangent form [[1, -t], [t, 1]] (t = s / c, when c >= s; the state is then
+// scaled by 1 / c) or cotangent form [[-u, 1], [1, u]] (u = c / s; scale
+// -1 / s and a sign on the qubit's 0 half); g is that scale, k2 = g^2.
+struct SplitRot {
+  double tau, g, k2, phi1, phi2;
+  int cot, pad;
+};
+// Split form, per layer l: the product of the layer's scales, of its k2, and
+// the qubits rotated in cotangent form.
+struct SplitLayer {
+  double gam, rho;
+  uint32_t cot_mask, pad;
+};
+
 // Arguments of one pass launch (forward or backward).
 struct PassArgs {
   int region;            // constant-memory coefficient region of the context
@@ -25,6 +54,8 @@ struct PassArgs {
   float* partials;       // backward gradient partials
   unsigned* status;
   int reupload;          // every layer starts with the encoding Ry(x_q) again
+  const float2* dq;      // split form: [L + 1][n][2] per-qubit factors of the diagonal ops (this direction)
+  const float* rscale;   // split form, backward checkpoint pass: scale of the restored state (null: 1)
   uint32_t cz_nb[kMaxQubits];    // CZ neighbours of each qubit (qubit mask)
   uint32_t cz_nbhi[kMaxQubits];  // CZ neighbours of each qubit above it (qubit mask)
 };
@@ -52,11 +83,21 @@ cudaError_t encode_pass_maps(const DevPass& p, int n, int B, bool backward, cons
 // how its tiles are loaded (n < 5: generic; tensor copies when p.tma).
 cudaError_t launch_pass(bool backward, const PassArgs& a, const DevPass& p, const PassMaps& maps, int grid,
                         size_t smem, cudaStream_t s);
-// Copy one pass's gate coefficients ([nslots][4] float4, device memory) into
-// the context's constant-memory region, in stream order.
-cudaError_t copy_pass_coef(int region, const float4* src, int nslots, cudaStream_t s);
-cudaError_t launch_prep_pass_coef(const DevPass* passes, int n_passes, const float* theta, float4* cf, float4* ci,
-                                  cudaStream_t s);
+// Copy one pass's gate coefficients (device memory) into the context's
+// constant-memory region, in stream order: the first nslots rotation slots,
+// and the diagonal tables when the pass has any.
+cudaError_t copy_pass_coef(int region, const CoefRegion* src, int nslots, int ndiag, cudaStream_t s);
+// Full SU(2) coefficients of every pass slot: cf forward, ci backward ([P] regions).
+cudaError_t launch_prep_pass_coef(const DevPass* passes, int n_passes, const float* theta, CoefRegion* cf,
+                                  CoefRegion* ci, cudaStream_t s);
+// Split form: every table the split passes need, from theta (fp64):
+//   rot [L][n], lay [L], gfix [L][n][2] (gradient scale and phi1 per rotation),
+//   dq_f / dq_b [L + 1][n][2] per-qubit diagonal factors, cf / ci [P] regions,
+//   rscale [P] (restore scale of the backward checkpoint passes).
+// undo: [L][n] qubits of each layer in the backward pass's un-apply order.
+cudaError_t launch_prep_split(const DevPass* passes, int n_passes, const float* theta, int L, int n,
+                              const int* undo, SplitRot* rot, SplitLayer* lay, double* gfix, float2* dq_f,
+                              float2* dq_b, CoefRegion* cf, CoefRegion* ci, float* rscale, cudaStream_t s);
 cudaError_t set_pass_smem_attr(size_t smem);
 cudaError_t pass_occupancy(bool backward, bool slow, size_t smem, int* blocks_per_sm);
 
@@ -64,9 +105,10 @@ cudaError_t launch_prep_enc(const float* x, int B, int n, float2* enc, cudaStrea
 cudaError_t launch_expect(const float2* psi, int B, int n, double* partial, float* E,
                           unsigned* status, cudaStream_t s);
 size_t expect_partial_count(int B, int n);
+// gfix: split form, [L][n][2] (scale of the sums, phi1) per rotation; null otherwise.
 cudaError_t launch_grad_reduce(const DevPass* passes, const int* slot_pass, const int* slot_index,
-                               const float* partials, int grid, const float* theta, int L, int n,
-                               float* grad, unsigned* status, cudaStream_t s);
+                               const float* partials, int grid, const float* theta, const double* gfix, int L,
+                               int n, float* grad, unsigned* status, cudaStream_t s);
 cudaError_t launch_loss_seed(const float* E, const float* y, int B, float* g, float* loss,
                              cudaStream_t s);
 cudaError_t launch_bwd_init(float2* psi, float2* lam, const float* g, int B, int n, cudaStream_t s);

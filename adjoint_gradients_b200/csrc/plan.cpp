@@ -289,7 +289,8 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
     }
     if (cur != mem) ps.ops.push_back({OP_EXCH, cur, mem, 0, 0});
     ps.store_phase = mem;
-    if ((int)ps.ops.size() > kMaxOps) return "internal: too many ops in a pass";
+    // (the split form adds one op after the encoding)
+    if ((int)ps.ops.size() + (ps.gen ? 1 : 0) > kMaxOps) return "internal: too many ops in a pass";
     if ((int)ps.slot_lq.size() > kMaxSlots) return "internal: too many gradient slots in a pass";
     p.max_slots = std::max(p.max_slots, (int)ps.slot_lq.size());
     p.passes.push_back(ps);
@@ -300,11 +301,31 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
   return "";
 }
 
-void flatten_plan(const Plan& p, std::vector<DevPass>* passes) {
+void flatten_plan(const Plan& p, std::vector<DevPass>* passes, bool split) {
   passes->clear();
-  for (const HostPass& ps : p.passes) {
+  // qubit mask of a rotation op of pass ps
+  auto op_qubits = [](const HostPass& ps, const HostOp& o) {
+    uint32_t m = 0;
+    for (int k = 0; k < kRegBits; ++k)
+      if (o.b & (1 << k)) m |= 1u << ps.tile_q[reg_tbit(o.a, k)];
+    return m;
+  };
+  for (size_t pi = 0; pi < p.passes.size(); ++pi) {
+    const HostPass& ps = p.passes[pi];
     DevPass d{};
-    d.nops = (int)ps.ops.size();
+    // op list (the split form renames rotations and entanglers, and adds the
+    // diagonal that precedes layer 0 right after the encoding)
+    std::vector<HostOp> ops;
+    int ndiag = 0;
+    for (const HostOp& h : ps.ops) {
+      HostOp o = h;
+      if (split && o.kind == OP_ROT) o.kind = OP_RY;
+      if (split && o.kind == OP_CZ) o = {OP_DIAG, h.a, 0, h.c, ndiag++};
+      ops.push_back(o);
+      if (split && h.kind == OP_GEN) ops.push_back({OP_DIAG, h.a, 0, -1, ndiag++});
+    }
+    d.nops = (int)ops.size();
+    d.ndiag = ndiag;
     d.load_phase = ps.load_phase;
     d.store_phase = ps.store_phase;
     d.gen = ps.gen ? 1 : 0;
@@ -317,11 +338,27 @@ void flatten_plan(const Plan& p, std::vector<DevPass>* passes) {
     d.variant = ps.variant;
     // forward: after the last exchange; backward (ops run in reverse): after the first
     d.pf_fwd = d.pf_bwd = -1;
-    for (int o = 0; o < (int)ps.ops.size(); ++o)
-      if (ps.ops[o].kind == OP_EXCH) {
+    for (int o = 0; o < (int)ops.size(); ++o)
+      if (ops[o].kind == OP_EXCH) {
         d.pf_fwd = o;
         if (d.pf_bwd < 0) d.pf_bwd = o;
       }
+    // split form, checkpoint pass: the rotations between the pass's end and
+    // the next diagonal op (all of that op's layer)
+    d.rs_layer = -1;
+    d.rs_mask = 0;
+    if (split && ps.ckpt >= 0) {
+      bool found = false;
+      for (size_t pj = pi + 1; pj < p.passes.size() && !found; ++pj)
+        for (const HostOp& h : p.passes[pj].ops) {
+          if (h.kind == OP_CZ) {
+            d.rs_layer = h.c;
+            found = true;
+            break;
+          }
+          if (h.kind == OP_ROT) d.rs_mask |= op_qubits(p.passes[pj], h);
+        }
+    }
     for (int t = 0; t < kTileBits; ++t) d.tile_q[t] = ps.tile_q[t];
     set_tma_view(p.n, ps, p.addr_of, &d);
     for (int b = 0; b < kTileBits; ++b) d.tile_abit[b] = ps.tile_q[b] >= 0 ? 1u << p.addr_of[ps.tile_q[b]] : 0u;
@@ -331,7 +368,7 @@ void flatten_plan(const Plan& p, std::vector<DevPass>* passes) {
     for (int s = 0; s < kMaxSlots; ++s) d.slot_lq[s] = s < d.nslots ? ps.slot_lq[s] : 0;
     for (int o = 0; o < kMaxOps; ++o) {
       if (o < d.nops) {
-        const HostOp& h = ps.ops[o];
+        const HostOp& h = ops[o];
         d.ops[o] = {h.kind, h.a, h.b, h.c, h.d};
       } else {
         d.ops[o] = {0, 0, 0, 0, 0};
@@ -339,6 +376,22 @@ void flatten_plan(const Plan& p, std::vector<DevPass>* passes) {
     }
     passes->push_back(d);
   }
+}
+
+std::vector<int> undo_order(const Plan& p, const std::vector<DevPass>& sp) {
+  const int n = p.n;
+  std::vector<int> order((size_t)p.L * n, -1);
+  std::vector<int> fill(p.L, 0);
+  for (int pi = (int)sp.size() - 1; pi >= 0; --pi) {
+    const DevPass& d = sp[pi];
+    for (int o = d.nops - 1; o >= 0; --o) {
+      const DevOp& op = d.ops[o];
+      if (op.kind != OP_RY && op.kind != OP_ROT) continue;
+      for (int k = 0; k < kRegBits; ++k)  // the kernel un-applies one op's rotations in increasing k
+        if (op.b & (1 << k)) order[(size_t)op.c * n + fill[op.c]++] = d.tile_q[reg_tbit(op.a, k)];
+    }
+  }
+  return order;
 }
 
 Bonds chain_bonds(int n) {

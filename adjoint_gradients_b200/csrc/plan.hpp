@@ -68,8 +68,14 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out);
 using Bonds = std::vector<std::pair<int, int>>;
 Bonds chain_bonds(int n);
 
-// Flatten to the device representation.
-void flatten_plan(const Plan& p, std::vector<DevPass>* passes);
+// Flatten to the device representation.  split: rotations as OP_RY and
+// entanglers as OP_DIAG (the split form, see device_plan.h), with one more
+// OP_DIAG right after the encoding.
+void flatten_plan(const Plan& p, std::vector<DevPass>* passes, bool split = false);
+
+// Split form: the qubits of every layer in the order the backward pass
+// un-applies their rotations ([L][n], layer-major).
+std::vector<int> undo_order(const Plan& p, const std::vector<DevPass>& split_passes);
 
 // Entangler tables of each pass (cz_reg, cz_nb) for the bond list.
 void set_pass_entangler(const Plan& p, const Bonds& bonds, std::vector<DevPass>* passes);

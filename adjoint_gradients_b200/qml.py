@@ -35,7 +35,19 @@ EXPORTS = [
     "qml_expect_observable", "qml_set_entangler", "qml_entangler_bonds", "qml_set_reupload", "qml_reupload",
     "qml_create_f64", "qml_precision", "qml_forward_expect_f64", "qml_backward_adjoint_f64", "qml_loss_seed_f64",
     "qml_step_host_f64", "qml_set_entangler_cnot", "qml_entangler_kind", "qml_debug_entangler_map",
+    "qml_split_form", "qml_measure_fma_peak",
 ]
+
+
+def measure_fma_peak(fp64: bool, iters: int = 200000, stream=None) -> tuple[float, float]:
+    """(TFLOP/s, launch ms) of independent FMA chains on the current device
+    (qml_measure_fma_peak): DFMA when fp64, else the packed f32x2 FMA."""
+    lib = load_library()
+    tf = ctypes.c_double()
+    ms = ctypes.c_float()
+    _check(lib.qml_measure_fma_peak(1 if fp64 else 0, iters, _stream_handle(stream), ctypes.byref(tf),
+                                    ctypes.byref(ms)), "qml_measure_fma_peak")
+    return tf.value, ms.value
 
 
 def debug_layouts() -> dict:
@@ -111,6 +123,8 @@ def load_library(path: str = LIB_PATH):
         "qml_entangler_bonds": ([_vp], _i),
         "qml_set_reupload": ([_vp, _i], _i),
         "qml_reupload": ([_vp], _i),
+        "qml_split_form": ([_vp], _i),
+        "qml_measure_fma_peak": ([_i, _i, _vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_float)], _i),
         "qml_create_f64": ([ctypes.POINTER(_Config), _i, ctypes.POINTER(_vp)], _i),
         "qml_precision": ([_vp], _i),
         "qml_forward_expect_f64": ([_vp, _vp, _vp, _i, _vp, _vp, _vp], _i),
@@ -258,6 +272,11 @@ class Context:
     @property
     def reupload(self) -> bool:
         return bool(self.lib.qml_reupload(self._h))
+
+    @property
+    def split_form(self) -> bool:
+        """True when the passes run in split form (see qml_split_form)."""
+        return bool(self.lib.qml_split_form(self._h))
 
     @property
     def entangler_bonds(self) -> int:

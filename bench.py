@@ -43,6 +43,13 @@ FP64_LANES = 64       # FP64 FMA lanes per SM (B200 data sheet: 40 TFLOP/s FP64 
 ALU64_PEAK_TFLOPS = SMS * FP64_LANES * 2 * SM_MAX_MHZ * 1e6 / 1e12
 FMA_FWD_PER_ROT = 8   # per amplitude: one fused SU(2) on a pair = 16 FMA / 2 amplitudes
 FMA_BWD_PER_ROT = 22  # per amplitude: U^dagger on psi (8) and lambda (8) + three Im<l|P|p> terms (6)
+# split form (qml_split_form): per amplitude and rotation, Ry in tangent form
+# on a pair = 4 FMA / 2 amplitudes; backward the same on psi and lambda (4)
+# plus the three Im<l|P|p> terms (6).  Per amplitude and diagonal op: the
+# complex factor (4 FMA, shared by the two lanes of a pair) and its product
+# with each lane (4 FMA per complex value): forward 2 + 4, backward 4 + 8.
+FMA_FWD_PER_RY, FMA_BWD_PER_RY = 2, 10
+FMA_FWD_PER_DIAG, FMA_BWD_PER_DIAG = 6, 12
 CPU_SAMPLE_LAYERS = 16  # oracle sample depth (cost is linear in depth)
 
 
@@ -127,10 +134,15 @@ def algorithmic_counts(ctx, w, B, f64=False, cnot_passes_per_layer=0):
     N = 1 << w.n
     amp = B * N
     rots = w.n * w.L
+    if ctx.split_form:  # one diagonal op per layer boundary (forward: also the one before layer 0)
+        fma_f = FMA_FWD_PER_RY * rots + FMA_FWD_PER_DIAG * (w.L + 1)
+        fma_b = FMA_BWD_PER_RY * rots + FMA_BWD_PER_DIAG * w.L
+    else:
+        fma_f, fma_b = FMA_FWD_PER_ROT * rots, FMA_BWD_PER_ROT * rots
     if cnot_passes_per_layer:  # CNOT entanglers: every layer's passes read and write the state once
         Pc = cnot_passes_per_layer * w.L
         c = 16 if f64 else 8
-        return {"passes": Pc, "fwd_fma": FMA_FWD_PER_ROT * rots * amp, "bwd_fma": FMA_BWD_PER_ROT * rots * amp,
+        return {"passes": Pc, "fwd_fma": fma_f * amp, "bwd_fma": fma_b * amp,
                 "fwd_bytes": (2 * c * Pc - c) * amp, "bwd_bytes": (4 * c * Pc - 2 * c) * amp}
     # bytes per amplitude moved by each pass, from the schedule flags
     i = 1
@@ -149,8 +161,9 @@ def algorithmic_counts(ctx, w, B, f64=False, cnot_passes_per_layer=0):
         bwd_bytes += rd + wr + (slot_b if ck >= 0 else 0)
     return {
         "passes": P,
-        "fwd_fma": FMA_FWD_PER_ROT * rots * amp,
-        "bwd_fma": FMA_BWD_PER_ROT * rots * amp,
+        "fwd_fma": fma_f * amp,
+        "bwd_fma": fma_b * amp,
+        "split": bool(ctx.split_form),
         "fwd_bytes": fwd_bytes * amp,
         "bwd_bytes": bwd_bytes * amp,
     }
@@ -280,12 +293,14 @@ def run_ours(args):
         import torch.distributed as dist
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    import dataclasses
+
     w = WORKLOADS[args.workload]
     f64 = args.precision == "fp64"
     if f64:  # fp64 mode keeps its checkpoint slots exact
-        import dataclasses
-
         w = dataclasses.replace(w, storage="fp64")
+    if args.ckpt_block is not None:  # checkpoint-block sweeps
+        w = dataclasses.replace(w, ckpt_block=args.ckpt_block)
     fdt = torch.float64 if f64 else torch.float32
     B = w.B
     dev = f"cuda:{local}"
@@ -379,10 +394,16 @@ def run_ours(args):
         default_path = not f64 and args.entangler == "chain" and not args.reupload and obs is None
         if tr.get("kernel_sources_sha256") == kernel_sources_digest() and default_path:
             traffic = tr.get("bwd_pass_bytes_per_launch")
+    # the bound is the resource the dominant kernel uses the larger fraction of
+    hbm_bound = bwd_gbs / hbm_peak > bwd_tflops / alu_peak
     roofline = {
-        "kernel": "pass64_kernel<backward>" if f64 else "pass_kernel<backward>", "bound": "alu",
-        "achieved": bwd_tflops, "peak": alu_peak,
-        "unit": "TFLOP/s", "frac": bwd_tflops / alu_peak, "traffic": traffic,
+        "kernel": "pass64_kernel<backward>" if f64 else "pass_kernel<backward>",
+        "bound": "hbm" if hbm_bound else "alu",
+        "achieved": bwd_gbs if hbm_bound else bwd_tflops, "peak": hbm_peak if hbm_bound else alu_peak,
+        "unit": "GB/s" if hbm_bound else "TFLOP/s",
+        "frac": bwd_gbs / hbm_peak if hbm_bound else bwd_tflops / alu_peak, "traffic": traffic,
+        "alu_achieved_tflops": bwd_tflops, "alu_peak_tflops": alu_peak, "alu_frac": bwd_tflops / alu_peak,
+        "fma_per_step": cnt["bwd_fma"], "bytes_per_step": cnt["bwd_bytes"], "split_form": cnt.get("split", False),
         "peak_src": ("148 SMs x 64 FP64 lanes x 2 x 1965 MHz (DFMA; derived from unit counts)" if f64 else
                      "148 SMs x 128 FP32 lanes x 2 x 1965 MHz (FFMA; packed f32x2 FMA measured at the same rate)"),
         "avg_launch_ms": bwd_avg_s * 1e3, "launches": bwd_n,
@@ -435,6 +456,40 @@ def run_ours(args):
         ctx_h.sync()
         del ctx_h
 
+    # ---- one real epoch: samples_per_epoch samples in mini-batches of B, the
+    # short last batch run as it is (its own x and y), timed on the device
+    epoch = None
+    if args.epoch and w.samples_per_epoch:
+        S = w.samples_per_epoch
+        xe = np.random.default_rng(1000 + w.index + 7919 * rank).uniform(0, np.pi, (S, w.n))
+        ye = np.random.default_rng(3000 + w.index + 7919 * rank).integers(0, 2, S) * 2.0 - 1.0
+        batches = [(i, min(B, S - i)) for i in range(0, S, B)]
+        xb = [torch.tensor(xe[i:i + b], dtype=fdt, device=dev) for i, b in batches]
+        yb = [torch.tensor(ye[i:i + b], dtype=fdt, device=dev) for i, b in batches]
+        torch.cuda.reset_peak_memory_stats(dev)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        q0.record(stream)
+        for (i, b), xi, yi in zip(batches, xb, yb):
+            Ei = E[:b]
+            ctx.forward(td, xi, psi[:b], Ei)
+            gi, _ = ctx.loss_seed(Ei, yi)
+            ctx.backward(td, xi, psi[:b], lam[:b], gi, grad)
+            if dist is not None:
+                dp.average_gradients(grad)
+        q1.record(stream)
+        torch.cuda.synchronize()
+        ctx.sync()
+        es = q0.elapsed_time(q1) / 1e3
+        if dist is not None:
+            t = torch.tensor([es], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            es = float(t.item())
+        epoch = {"s_per_epoch_measured": es, "samples": S, "batches": [b for _, b in batches][-2:],
+                 "n_batches": len(batches), "peak_hbm_bytes_epoch": int(torch.cuda.max_memory_allocated(dev))}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w)
@@ -448,6 +503,8 @@ def run_ours(args):
     if w.samples_per_epoch:
         cfg["s_per_epoch"] = w.samples_per_epoch / (value / world)
         cfg["epoch"] = f"{w.samples_per_epoch} samples per GPU at the measured samples/s (mini-batch {B})"
+    if epoch is not None:
+        cfg["epoch_run"] = epoch
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -482,6 +539,10 @@ def main():
     ap.add_argument("--reupload", action="store_true", help="data re-uploading: the encoding again in every layer")
     ap.add_argument("--precision", default="fp32", choices=["fp32", "fp64"],
                     help="arithmetic of the path: fp32, or fp64 (complex128 state, exact checkpoint slots)")
+    ap.add_argument("--ckpt-block", type=int, default=None,
+                    help="override the workload's checkpoint block (layers per block; 0: none)")
+    ap.add_argument("--epoch", action="store_true",
+                    help="also time one real epoch of the workload (its samples in mini-batches, short last batch as is)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

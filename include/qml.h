@@ -96,7 +96,9 @@ QML_API const char* qml_status_str(qml_status s);
  *                           unrecorded: the backward pass returns
  *                           QML_ERR_CKPT_MISMATCH
  *   QML_FAULT=nan_theta     the first rotation's coefficients are NaN in
- *                           every forward pass: qml_sync returns
+ *                           every forward pass (fp64 contexts: the first
+ *                           angle, in a copy of theta inside the workspace),
+ *                           with any entangler: qml_sync returns
  *                           QML_ERR_NUMERIC */
 QML_API qml_status qml_create(const qml_config* cfg, int device, qml_ctx** out);
 
@@ -225,6 +227,26 @@ QML_API int qml_debug_entangler_map(const qml_ctx* ctx, int* out, int cap);
 QML_API qml_status qml_set_reupload(qml_ctx* ctx, int on);
 QML_API int qml_reupload(const qml_ctx* ctx);
 
+/* 1 when the context's passes run in split form, 0 when they apply fused
+ * SU(2) rotations, -1 for a null context.  The split form (fp32 contexts
+ * without re-uploading or CNOT entanglers) rewrites every fused rotation
+ * U = Rz(g) Ry(b) Rx(a) exactly as Rz(phi1) Ry(vt) Rz(phi2), applies the real
+ * Ry in tangent form and merges each layer's Rz factors with its CZ bonds
+ * into one diagonal (Deep-dive blog sec. 1.4, forward and backward gate
+ * fusion: the gates are fused differently, the results are the same up to
+ * rounding).  Informational: every entry point gives the same results either
+ * way. */
+QML_API int qml_split_form(const qml_ctx* ctx);
+
+/* Measurement aid (not part of the simulation): the FMA throughput of the
+ * current device, for the ALU rooflines of the pass kernels.  One launch of
+ * independent FMA chains over every SM, `iters` steps of 8 chains per thread,
+ * timed with CUDA events on `stream` (the call synchronises).  fp64 != 0:
+ * DFMA; otherwise the packed f32x2 FMA of the fp32 kernels.  *tflops =
+ * 2 x FMAs / time (TFLOP/s); *ms (optional) = the launch's duration.
+ * Allocates nothing. */
+QML_API qml_status qml_measure_fma_peak(int fp64, int iters, void* stream, double* tflops, float* ms);
+
 /* Largest number of Pauli-string terms an observable may have. */
 #define QML_MAX_OBS_TERMS 4096
 
@@ -270,11 +292,15 @@ QML_API qml_status qml_expect_observable(qml_ctx* ctx, const float* psi_dev, int
  *     nothing.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current and caches it; make
- *     that first call before any stream capture.
+ *     that first call before any stream capture.  The cache is tied to the
+ *     device's CUDA context: the first call after a cudaDeviceReset looks the
+ *     address up again (so it, too, belongs before any capture).
  *   - All calls on a device share the one array.  Each call overwrites every
  *     partial it later reads, so stale contents are never used, but calls
  *     whose kernels overlap on the GPU (different streams, no ordering) race
  *     on it.
+ *   - No status word: a non-finite expectation is written to expect_dev as
+ *     it is, and nothing is latched for a later qml_sync.
  *   - No cudaMalloc, cudaFree or allocating library routine is called. */
 QML_API qml_status qml_expect_z0_static(const float* psi_dev, int n_qubits, int B, float* expect_dev,
                                         void* stream);

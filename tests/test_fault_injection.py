@@ -70,6 +70,32 @@ def test_injected_nan_coefficients(monkeypatch):
 
 
 @pytest.mark.gpu
+def test_injected_nan_coefficients_cnot(monkeypatch):
+    monkeypatch.setenv("QML_FAULT", "nan_theta")
+    n, L, B = 9, 2, 3
+    x, theta, _ = random_case(8210, B, n, L)
+    ctx = qml.Context(n, L, B)
+    ctx.set_entangler([(q, q + 1) for q in range(n - 1)], kind="cnot")
+    ctx.forward(dev(theta), dev(x))
+    with pytest.raises(qml.QmlError) as ei:
+        ctx.sync()
+    assert ei.value.code == 6
+
+
+@pytest.mark.gpu
+def test_injected_nan_angle_fp64(monkeypatch):
+    monkeypatch.setenv("QML_FAULT", "nan_theta")
+    n, L, B = 9, 2, 2
+    x, theta, _ = random_case(8220, B, n, L)
+    ctx = qml.Context(n, L, B, precision="fp64")
+    d64 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64)).cuda()
+    ctx.forward(d64(theta), d64(x))
+    with pytest.raises(qml.QmlError) as ei:
+        ctx.sync()
+    assert ei.value.code == 6
+
+
+@pytest.mark.gpu
 def test_injected_lost_checkpoints(monkeypatch):
     monkeypatch.setenv("QML_FAULT", "ckpt_corrupt")
     n, L, B = 14, 4, 2
