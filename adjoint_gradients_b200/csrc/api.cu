@@ -142,7 +142,12 @@ void ensure_device(qml_ctx* c) {
     c->dev_ok = true;
     return;
   }
-  c->smem = pass_smem_bytes(c->plan.max_slots);
+  // every pass of a context loads the same way: tensor copies for n > 12
+  const bool tma = !c->dpass.empty() && c->dpass[0].tma;
+  const int mode = tma ? 2 : c->slow ? 0 : 1;
+  // the function attribute is shared by all contexts: set it for the largest pass
+  const size_t smem_thr = pass_smem_bytes(kMaxSlots, false), smem_tma = pass_smem_bytes(kMaxSlots, true);
+  c->smem = tma ? smem_tma : smem_thr;
   cudaDeviceProp prop;
   if (cudaGetDeviceProperties(&prop, c->device) != cudaSuccess) {
     cudaGetLastError();
@@ -154,8 +159,8 @@ void ensure_device(qml_ctx* c) {
   DeviceGuard g(c->device);
   c->sms = prop.multiProcessorCount;
   int of = 0, ob = 0;
-  if (set_pass_smem_attr(c->smem) != cudaSuccess || pass_occupancy(false, c->slow, c->smem, &of) != cudaSuccess ||
-      pass_occupancy(true, c->slow, c->smem, &ob) != cudaSuccess || of < 1 || ob < 1) {
+  if (set_pass_smem_attr(smem_thr, smem_tma) != cudaSuccess || pass_occupancy(false, mode, c->smem, &of) != cudaSuccess ||
+      pass_occupancy(true, mode, c->smem, &ob) != cudaSuccess || of < 1 || ob < 1) {
     cudaGetLastError();
     c->dev_ok = false;
     c->grid_fwd = c->sms * 3;

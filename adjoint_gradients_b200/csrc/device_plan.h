@@ -26,6 +26,9 @@ constexpr int kThreads = 1 << kThrBits;
 // Resident pass blocks per SM: 3 x 128 threads x 168 registers fill the
 // register file, 3 x ~69 KB of tile buffer fit the shared memory.
 constexpr int kBlocksPerSm = 3;
+// Passes that load tiles by tensor copies keep a 64 KB landing buffer next to
+// their exchange buffer: two blocks per SM (up to 255 registers a thread).
+constexpr int kBlocksPerSmTma = 2;
 constexpr int kTilePos = 1 << kTileBits;
 constexpr int kSmemSlots = kTilePos + (kTilePos >> 5) + 8;  // exchange slots (see wbit in the kernels)
 constexpr int kMaxSet = 10;           // qubits rotated per pass when n > 12

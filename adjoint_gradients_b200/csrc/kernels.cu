@@ -524,6 +524,65 @@ __device__ __forceinline__ void exchange(int x, int y, float2 (&re)[kPos], float
   }
 }
 
+// Tensor-copy passes keep the copied tile in a landing buffer of its own, so
+// their layout exchanges go through a second, smaller buffer: the re pairs
+// first, then the im pairs, 8 bytes per position.  Slot of position t:
+// sum over the set bits b of t of wbit8(b) (additive and injective; every
+// half warp of every layout's 8-byte accesses hits 16 different bank pairs).
+__host__ __device__ constexpr uint32_t wbit8(int b) {
+  return b < 5 ? (1u << b) : b == 5 ? 33u : b == 6 ? 66u : b == 7 ? 132u : b == 8 ? 264u : b == 9 ? 528u : b == 10 ? 1060u
+                                                                                                                 : 2120u;
+}
+constexpr int kExch8Slots = 4235;  // largest slot (sum of all wbit8) + 1
+
+template <int P>
+__host__ __device__ constexpr uint32_t reg_slot8(int j) {
+  uint32_t s = 0;
+  for (int k = 0; k < kRegBits; ++k)
+    if ((j >> k) & 1) s += wbit8(reg_tbit<P>(k));
+  return s;
+}
+
+template <int P, int V>
+__device__ __forceinline__ uint32_t thr_slot8(uint32_t tid) {
+  uint32_t s = 0;
+#pragma unroll
+  for (int m = 0; m < kThrBits; ++m)
+    if ((tid >> m) & 1u) s += wbit8(thr_tbit<P, V>(m));
+  return s;
+}
+
+template <int X, int Y, int V>
+__device__ __forceinline__ void exchange8_t(float2 (&re)[kPos], float2 (&im)[kPos], float2* ex, uint32_t tid) {
+  const uint32_t sx = thr_slot8<X, V>(tid);
+  const uint32_t sy = thr_slot8<Y, V>(tid);
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kPos; ++j) ex[sx + reg_slot8<X>(j)] = re[j];
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kPos; ++j) re[j] = ex[sy + reg_slot8<Y>(j)];
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kPos; ++j) ex[sx + reg_slot8<X>(j)] = im[j];
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kPos; ++j) im[j] = ex[sy + reg_slot8<Y>(j)];
+}
+
+template <int V>
+__device__ __forceinline__ void exchange8(int x, int y, float2 (&re)[kPos], float2 (&im)[kPos], float2* ex,
+                                          uint32_t tid) {
+  switch (x * 3 + y) {
+    case 1: exchange8_t<0, 1, V>(re, im, ex, tid); break;
+    case 2: exchange8_t<0, 2, V>(re, im, ex, tid); break;
+    case 3: exchange8_t<1, 0, V>(re, im, ex, tid); break;
+    case 5: exchange8_t<1, 2, V>(re, im, ex, tid); break;
+    case 6: exchange8_t<2, 0, V>(re, im, ex, tid); break;
+    default: exchange8_t<2, 1, V>(re, im, ex, tid); break;
+  }
+}
+
 // CZ on every bond (a, b) of the entangler: sign (-1)^{S(i)}, S(i) = sum over
 // bonds of i_a i_b, of the global index i.  Split i = T | O | R (thread bits,
 // out-of-tile bits, register bits; disjoint).  S is a quadratic form, so
@@ -994,8 +1053,20 @@ __device__ __forceinline__ void cz_thread_terms(BlockCtx& bc, const DevPass& Pp,
 // per register pair.  RE 3: the split form (OP_RY and OP_DIAG ops; no
 // re-uploading).
 
+// Shared memory of a pass block.  Tensor-copy passes (MODE 2): the landing
+// buffer of the copied tile (both planes, 64 KB), then the 8-byte exchange
+// buffer; the next tile's copy is issued as soon as the current tile is in
+// registers, so it is in flight during the whole tile (two blocks per SM).
+// Other passes: one buffer for the exchanges and the cp.async prefetch (three
+// blocks per SM).  Then the block's context and gradient accumulators.
+constexpr size_t kLandBytes = (size_t)kTilePos * 16;
+constexpr size_t kExch8Bytes = ((size_t)kExch8Slots * 8 + 127) & ~(size_t)127;
+__host__ __device__ constexpr size_t pass_buf_bytes(bool tma) {
+  return tma ? kLandBytes + kExch8Bytes : (size_t)kSmemSlots * sizeof(float4);
+}
+
 template <bool BWD, int MODE, int V, int RE>
-__global__ void __launch_bounds__(kThreads, kBlocksPerSm)
+__global__ void __launch_bounds__(kThreads, MODE == 2 ? kBlocksPerSmTma : kBlocksPerSm)
     pass_kernel(const PassArgs a, const __grid_constant__ DevPass P, const __grid_constant__ CUtensorMap tm0,
                 const __grid_constant__ CUtensorMap tm1) {
   constexpr bool SLOW = MODE == 0;
@@ -1003,8 +1074,9 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   constexpr bool REUP = RE == 1 || RE == 2;  // data re-uploading folded into the fused rotations
   constexpr bool SPLIT = RE == 3;            // split form: OP_RY / OP_DIAG instead of OP_ROT / OP_CZ
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  float4* tile = reinterpret_cast<float4*>(smem_raw);
-  BlockCtx* bc = reinterpret_cast<BlockCtx*>(smem_raw + (size_t)kSmemSlots * sizeof(float4));
+  float4* tile = reinterpret_cast<float4*>(smem_raw);  // MODE 2: the landing buffer
+  float2* ex8 = reinterpret_cast<float2*>(smem_raw + kLandBytes);  // MODE 2: the exchange buffer
+  BlockCtx* bc = reinterpret_cast<BlockCtx*>(smem_raw + pass_buf_bytes(TMA));
   float* acc = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(bc) + sizeof(BlockCtx));  // [warps][nslots*3]
   const uint32_t tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
@@ -1045,9 +1117,11 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   }
   uint32_t parity = 0;
 
-  // The next tile is fetched into the shared tile buffer once the buffer is
-  // free (after the pass's last exchange), so its latency hides behind the last
-  // register phase.  n < 5 loads directly.
+  // Without tensor copies the next tile is fetched into the shared tile
+  // buffer once the buffer is free (after the pass's last exchange), so its
+  // latency hides behind the last register phase; n < 5 loads directly.  The
+  // tensor copy of the next tile is issued right after the current tile is in
+  // registers.
   const bool can_pf = !SLOW && loads;
   const int mem_ph = BWD ? P.store_phase : P.load_phase;
   const int pf_at = BWD ? P.pf_bwd : P.pf_fwd;  // op index after which to prefetch (-1: after the load)
@@ -1059,10 +1133,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     const int tn = t + (int)gridDim.x;
     const bool pf_next = can_pf && tn < a.n_tiles;
     auto prefetch_next = [&]() {
-      __syncthreads();  // every thread is done with the tile buffer
-      if (TMA) {
-        if (tid == 0) tma_load_tile(&tm0, &tm1, bc->tma_sel, bc->tma_c, tile_s, mbar);
-      } else {
+      if constexpr (!TMA) {
+        __syncthreads();  // every thread is done with the tile buffer
         uint32_t bq, ba, ub;
         tile_base(P, tn, &bq, &ba, &ub);
         prefetch_op<BWD, V>(mem_ph, a, *bc, tid, bq, ba, ub, tile);
@@ -1089,6 +1161,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
         else restore_tma_t<1, V>(a, *bc, P, tid, base_q, unit_base, tb, P.ckpt, rs);
       }
       load_tma<V>(mem_ph, re, im, tb, P, tid);
+      __syncthreads();  // every thread has its positions: the landing buffer is free
+      if (pf_next && tid == 0) tma_load_tile(&tm0, &tm1, bc->tma_sel, bc->tma_c, tile_s, mbar);
     }
     if (!BWD) {
       if (P.gen) mem_op<false, SLOW, V, M_GEN>(P.load_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
@@ -1099,7 +1173,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
       for (int oi = 0; oi < P.nops; ++oi) {
         const DevOp op = P.ops[oi];
         if (op.kind == OP_EXCH) {
-          exchange<V>(op.a, op.b, re, im, tile, tid);
+          if constexpr (TMA) exchange8<V>(op.a, op.b, re, im, ex8, tid);
+          else exchange<V>(op.a, op.b, re, im, tile, tid);
         } else if constexpr (SPLIT) {
           if (op.kind == OP_RY) {
             int slot = op.d;
@@ -1157,7 +1232,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
       for (int oi = P.nops - 1; oi >= 0; --oi) {
         const DevOp op = P.ops[oi];
         if (op.kind == OP_EXCH) {
-          exchange<V>(op.b, op.a, re, im, tile, tid);
+          if constexpr (TMA) exchange8<V>(op.b, op.a, re, im, ex8, tid);
+          else exchange<V>(op.b, op.a, re, im, tile, tid);
         } else if constexpr (SPLIT) {
           if (op.kind == OP_RY) {
             // the same sums, then Ry un-applied (tangent or cotangent form)
@@ -1678,8 +1754,8 @@ __global__ void ckpt_copy_kernel(bool save, const float2* in, float2* out, void*
 
 }  // namespace
 
-size_t pass_smem_bytes(int max_slots) {
-  return (size_t)kSmemSlots * sizeof(float4) + sizeof(BlockCtx) + (size_t)(kThreads / 32) * max_slots * 3 * sizeof(float);
+size_t pass_smem_bytes(int max_slots, bool tma) {
+  return pass_buf_bytes(tma) + sizeof(BlockCtx) + (size_t)(kThreads / 32) * max_slots * 3 * sizeof(float);
 }
 
 #define QML_FOR_EACH_PASS_KERNEL(X)                                                                          \
@@ -1690,11 +1766,12 @@ size_t pass_smem_bytes(int max_slots) {
   X(false, 1, 0, 3) X(true, 1, 0, 3) X(false, 1, 1, 3) X(true, 1, 1, 3) X(false, 2, 0, 3) X(true, 2, 0, 3)         \
   X(false, 2, 1, 3) X(true, 2, 1, 3)
 
-cudaError_t set_pass_smem_attr(size_t smem) {
+cudaError_t set_pass_smem_attr(size_t smem_thr, size_t smem_tma) {
   cudaError_t e = cudaSuccess;
 #define QML_SET_ATTR(B, S, V, R)                                                                                 \
   if (e == cudaSuccess)                                                                                          \
-    e = cudaFuncSetAttribute(pass_kernel<B, S, V, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+    e = cudaFuncSetAttribute(pass_kernel<B, S, V, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,             \
+                             (int)(S == 2 ? smem_tma : smem_thr));                                             \
   if (e == cudaSuccess)                                                                                          \
     e = cudaFuncSetAttribute(pass_kernel<B, S, V, R>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   QML_FOR_EACH_PASS_KERNEL(QML_SET_ATTR)
@@ -1703,7 +1780,7 @@ cudaError_t set_pass_smem_attr(size_t smem) {
 }
 
 int debug_layouts(int* out, int cap) {
-  int v[2 * 3 * 12 + kTileBits + 1];
+  int v[2 * 3 * 12 + 2 * (kTileBits + 1)];
   int k = 0;
   for (int P = 0; P < kPhases; ++P)
     for (int V = 0; V < 2; ++V) {
@@ -1713,16 +1790,20 @@ int debug_layouts(int* out, int cap) {
     }
   for (int b = 0; b < kTileBits; ++b) v[k++] = (int)wbit(b);
   v[k++] = kSmemSlots;
+  for (int b = 0; b < kTileBits; ++b) v[k++] = (int)wbit8(b);
+  v[k++] = kExch8Slots;
   for (int i = 0; i < k && i < cap; ++i) out[i] = v[i];
   return k;
 }
 
-cudaError_t pass_occupancy(bool backward, bool slow, size_t smem, int* blocks_per_sm) {
+cudaError_t pass_occupancy(bool backward, int mode, size_t smem, int* blocks_per_sm) {
   if (backward)
-    return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, 0, 0, 0>, kThreads, smem)
-                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, 2, 1, 0>, kThreads, smem);
-  return slow ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, 0, 0, 0>, kThreads, smem)
-              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, 2, 1, 0>, kThreads, smem);
+    return mode == 0   ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, 0, 0, 0>, kThreads, smem)
+           : mode == 1 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, 1, 1, 0>, kThreads, smem)
+                       : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<true, 2, 1, 0>, kThreads, smem);
+  return mode == 0   ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, 0, 0, 0>, kThreads, smem)
+         : mode == 1 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, 1, 1, 0>, kThreads, smem)
+                     : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pass_kernel<false, 2, 1, 0>, kThreads, smem);
 }
 
 cudaError_t launch_pass(bool backward, const PassArgs& a, const DevPass& p, const PassMaps& maps, int grid,

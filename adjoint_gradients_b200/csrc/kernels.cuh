@@ -60,11 +60,13 @@ struct PassArgs {
   uint32_t cz_nbhi[kMaxQubits];  // CZ neighbours of each qubit above it (qubit mask)
 };
 
-size_t pass_smem_bytes(int max_slots);
+// Dynamic shared memory of a pass block (tma: tensor-copy passes).
+size_t pass_smem_bytes(int max_slots, bool tma);
 
 // Register layouts for tests: per (phase, variant) the tile bit of each of the
 // 7 thread-index bits and 5 register-index bits, then the 12 slot weights and
-// the slot count.  Returns the number of ints.
+// the slot count of the 16-byte exchanges, then the same for the 8-byte
+// exchanges of tensor-copy passes.  Returns the number of ints.
 int debug_layouts(int* out, int cap);
 
 // Tensor maps (CUtensorMap, 128 bytes each) of a pass whose tiles are loaded
@@ -98,8 +100,9 @@ cudaError_t launch_prep_pass_coef(const DevPass* passes, int n_passes, const flo
 cudaError_t launch_prep_split(const DevPass* passes, int n_passes, const float* theta, int L, int n,
                               const int* undo, SplitRot* rot, SplitLayer* lay, double* gfix, float2* dq_f,
                               float2* dq_b, CoefRegion* cf, CoefRegion* ci, float* rscale, cudaStream_t s);
-cudaError_t set_pass_smem_attr(size_t smem);
-cudaError_t pass_occupancy(bool backward, bool slow, size_t smem, int* blocks_per_sm);
+cudaError_t set_pass_smem_attr(size_t smem_thr, size_t smem_tma);
+// mode: 0 generic addressing (n < 5), 1 thread loads, 2 tensor copies.
+cudaError_t pass_occupancy(bool backward, int mode, size_t smem, int* blocks_per_sm);
 
 cudaError_t launch_prep_enc(const float* x, int B, int n, float2* enc, cudaStream_t s);
 cudaError_t launch_expect(const float2* psi, int B, int n, double* partial, float* E,

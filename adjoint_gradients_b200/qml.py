@@ -63,7 +63,7 @@ def debug_layouts() -> dict:
         for V in range(2):
             lay[(P, V)] = (v[k:k + 7], v[k + 7:k + 12])
             k += 12
-    return dict(layouts=lay, weights=v[k:k + 12], slots=v[k + 12])
+    return dict(layouts=lay, weights=v[k:k + 12], slots=v[k + 12], weights8=v[k + 13:k + 25], slots8=v[k + 25])
 
 
 class QmlError(RuntimeError):

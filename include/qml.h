@@ -362,8 +362,9 @@ QML_API int qml_debug_tile_view(const qml_ctx* ctx, int pass, int* out, int cap)
  * qml_debug_schedule.  Layout: for phase 0..2 and layout variant 0..1, the
  * tile bit of each of the 7 thread-index bits then of each of the 5
  * register-index bits; then the 12 shared-memory slot weights of the tile
- * bits (slot of a position = sum of the weights of its set bits); then the
- * number of slots. */
+ * bits (slot of a position = sum of the weights of its set bits) and the
+ * number of slots of the 16-byte exchanges; then the same two for the 8-byte
+ * exchanges of the passes that load tiles by tensor copies. */
 QML_API int qml_debug_layouts(int* out, int cap);
 
 /* ------------------------------------------------------------------------

@@ -8,6 +8,10 @@ The tables come from the library itself (qml_debug_layouts, qml_debug_tile_view)
   * layout exchanges are free of bank conflicts: the eight lanes of each
     quarter warp (one 128-byte wavefront of 16-byte accesses) hit eight
     different 16-byte bank groups;
+  * the 8-byte exchanges of tensor-copy passes (re pairs, then im pairs,
+    through a buffer of their own) are injective, fit their buffer and are
+    free of bank conflicts: the 16 lanes of each half warp hit 16 different
+    8-byte bank pairs, for every layout and register;
   * reading a tile that arrived by tensor copy is free of bank conflicts: in
     the memory layout, the 16 lanes of each half warp (8-byte accesses) hit 16
     different 8-byte bank pairs.
@@ -37,6 +41,22 @@ def test_exchanges_have_no_bank_conflicts():
                 s = sum(w[thr[m]] for m in range(5) if (lane >> m) & 1)
                 groups.add(s % 8)
             assert len(groups) == 8, (P, V, q)
+
+
+def test_8_byte_exchanges_fit_and_have_no_bank_conflicts():
+    d = qml.debug_layouts()
+    w = d["weights8"]
+    slots = {sum(w[b] for b in range(12) if (t >> b) & 1) for t in range(4096)}
+    assert len(slots) == 4096
+    assert max(slots) < d["slots8"]
+    for (P, V), (thr, reg) in d["layouts"].items():
+        for j in range(32):
+            r = sum(w[reg[k]] for k in range(5) if (j >> k) & 1)
+            for h in range(2):
+                pairs = set()
+                for lane in range(16 * h, 16 * h + 16):
+                    pairs.add((r + sum(w[thr[m]] for m in range(5) if (lane >> m) & 1)) % 16)
+                assert len(pairs) == 16, (P, V, j, h)
 
 
 @pytest.mark.parametrize("n", [13, 16, 17, 20, 21, 25, 26, 29, 30])
