@@ -643,7 +643,20 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
   c->launches += split ? 5 : 2;
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, false);
-  for (int p = 0; p < P; ++p) {
+  if (split && !passes[0].tma) {  // one tile holds the state: every pass in one launch
+    const DevPass& dp = passes[0];
+    a.npass = P;
+    a.passes = at<DevPass>(c, c->lay.passes_split);
+    a.coef = cf;
+    a.n_tiles = (int)(((a.U + (1ll << dp.unit_bits) - 1) >> dp.unit_bits) << dp.n_out);
+    static const PassMaps none{};
+    e = launch_pass(false, a, dp, none, c->grid_fwd, c->smem, s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+    ++c->launches;
+    for (const DevPass& q : passes)
+      if (q.ckpt >= 0) c->ckpt_batch[q.ckpt] = B;
+  }
+  for (int p = 0; p < P && !(split && !passes[0].tma); ++p) {
     const DevPass& dp = passes[p];
     const long long units_per_tile = 1ll << dp.unit_bits;
     a.n_tiles = (int)(((a.U + units_per_tile - 1) / units_per_tile) << dp.n_out);
@@ -718,7 +731,20 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
   c->launches += split ? 6 : 3;  // coefficient prep, lambda init, gradient reduce
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, true);
-  for (int p = P - 1; p >= 0; --p) {
+  const bool one_launch = split && !passes[0].tma;  // one tile holds the state: every pass in one launch
+  if (one_launch) {
+    const DevPass& dp = passes[0];
+    a.npass = P;
+    a.passes = at<DevPass>(c, c->lay.passes_split);
+    a.coef = ci;
+    a.rscale = at<float>(c, c->lay.rscale);
+    a.n_tiles = (int)(((a.U + (1ll << dp.unit_bits) - 1) >> dp.unit_bits) << dp.n_out);
+    static const PassMaps none{};
+    e = launch_pass(true, a, dp, none, c->grid_bwd, c->smem, s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+    ++c->launches;
+  }
+  for (int p = P - 1; p >= 0 && !one_launch; --p) {
     const DevPass& dp = passes[p];
     const long long units_per_tile = 1ll << dp.unit_bits;
     a.n_tiles = (int)(((a.U + units_per_tile - 1) / units_per_tile) << dp.n_out);

@@ -294,6 +294,22 @@ __global__ void __launch_bounds__(kT, BWD ? 2 : 3) pass64_kernel(const Pass64Arg
       tp[padp(v)] = pv;
       if (BWD) tl[padp(v)] = a.lam[g];
     }
+    // the block's next tile into L2 while this one is computed (its loads then
+    // hit L2): each thread its own positions of both planes
+    const long long tn = t + gridDim.x;
+    if (tn < a.n_tiles && (BWD || !P.gen)) {
+      const int bn = (int)(tn >> no);
+      const uint32_t on = (uint32_t)(tn & ((1ll << no) - 1));
+      uint32_t bsn = 0;
+      for (int k = 0; k < no; ++k)
+        if ((on >> k) & 1u) bsn |= 1u << cx.oq[k];
+      const size_t gn = ((size_t)bn << n) + bsn;
+      for (int v = tid; v < P2; v += kT) {
+        const size_t g = gn + (cx.off_lo[v & 63] | cx.off_hi[(v >> 6) & 63]);
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(a.psi + g));
+        if (BWD) asm volatile("prefetch.global.L2 [%0];" ::"l"(a.lam + g));
+      }
+    }
     __syncthreads();
 
     for (int k = 0; k < P.nops; ++k) {
@@ -458,18 +474,27 @@ __global__ void obs64_lambda_kernel(const double2* psi, double2* lam, const doub
 __global__ void grad_reduce64_kernel(const DevPass* passes, const int* slot_pass, const int* slot_index,
                                      const double* partials, int grid, const double* theta, int L, int n,
                                      double* grad, unsigned* status) {
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= L * n) return;
+  // one warp per (layer, qubit): strided lane sums, then a fixed butterfly
+  const int idx = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (idx >= L * n) return;  // whole warps leave together
   const int p = slot_pass[idx], s = slot_index[idx];
   const DevPass& ps = passes[p];
   const int stride = ps.nslots * 3;
   const double* base = partials + ps.partial_off + s * 3;
   double sx = 0.0, sy = 0.0, sz = 0.0;
-  for (int c = 0; c < grid; ++c) {
+  for (int c = lane; c < grid; c += 32) {
     sx += base[(size_t)c * stride + 0];
     sy += base[(size_t)c * stride + 1];
     sz += base[(size_t)c * stride + 2];
   }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    sx += __shfl_xor_sync(0xffffffffu, sx, o);
+    sy += __shfl_xor_sync(0xffffffffu, sy, o);
+    sz += __shfl_xor_sync(0xffffffffu, sz, o);
+  }
+  if (lane != 0) return;
   // (s_x, s_y, s_z) are Im<lambda|P|psi> at the rotation's output; the angle
   // gradients take X and Y back through the Rz and Ry that follow them
   double sb, cb, sg, cg;
@@ -571,9 +596,9 @@ cudaError_t launch_obs_bwd_init64(const double2* psi, double2* lam, const double
 cudaError_t launch_grad_reduce64(const DevPass* passes, const int* slot_pass, const int* slot_index,
                                  const double* partials, int grid, const double* theta, int L, int n, double* grad,
                                  unsigned* status, cudaStream_t s) {
-  const int tot = L * n;
-  grad_reduce64_kernel<<<(tot + 127) / 128, 128, 0, s>>>(passes, slot_pass, slot_index, partials, grid, theta, L,
-                                                          n, grad, status);
+  const long long threads = (long long)L * n * 32;  // one warp per (layer, qubit)
+  grad_reduce64_kernel<<<(unsigned)((threads + 127) / 128), 128, 0, s>>>(passes, slot_pass, slot_index, partials,
+                                                                         grid, theta, L, n, grad, status);
   return cudaGetLastError();
 }
 

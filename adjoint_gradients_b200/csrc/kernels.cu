@@ -936,18 +936,19 @@ __device__ __forceinline__ void cz_op(int phase, float2 (&re)[kPos], float2 (&im
   }
 }
 
-// Split form: the diagonal op d (layer l) in layout P.  A position i = T | O |
-// R (thread, out-of-tile and register bits) is multiplied by
+// Split form: the diagonal op d (layer l).  A position i = T | O | R (thread,
+// out-of-tile and register bits) is multiplied by
 //   (-1)^{S(i)} * f(T) f(O) * R_d[j],
 // with S the entangler parity (l >= 0 only), f the product of the per-qubit
 // factors dq[l + 1][q][bit] over the bits named, and R_d[j] the pass's
 // constant table for the register part j (the global scale folded in).  The
 // factor applies to both lanes of a pair (two samples, or psi and lambda).
+// Only the thread part depends on the layout P; the loop over positions is
+// shared by all layouts (one copy of its code).
 template <int P, int V>
-__device__ __forceinline__ void diag_t(float2 (&re)[kPos], float2 (&im)[kPos], const BlockCtx& bc,
-                                       const DevPass& Pp, const PassArgs& a, int region, int d, int l, uint32_t tid,
-                                       uint32_t base_q, uint32_t s_o) {
-  const float2* dq = a.dq + (size_t)(l + 1) * a.n * 2;
+__device__ __forceinline__ void diag_thread_t(const BlockCtx& bc, const DevPass& Pp, const float2* dq, int l,
+                                              uint32_t tid, uint32_t base_q, uint32_t s_o, float* fr_out,
+                                              float* fi_out, uint32_t* w_out) {
   float fr = 1.f, fi = 0.f;
   auto mul = [&](float2 v) {
     const float r = fr * v.x - fi * v.y;
@@ -970,28 +971,34 @@ __device__ __forceinline__ void diag_t(float2 (&re)[kPos], float2 (&im)[kPos], c
     for (int k = 0; k < kRegBits; ++k) nb[k] = Pp.cz_nb[P][k];
     w = cz_word(bc.cz_w[P][tid], bc.cz_n[P][tid], nb, base_q, s_o);
   }
-  // per position: the factor (scalar complex, table entries as constant
-  // operands), its sign, then the product with both lanes
+  *fr_out = fr;
+  *fi_out = fi;
+  *w_out = w;
+}
+
+template <int V>
+__device__ __forceinline__ void diag_op(int phase, float2 (&re)[kPos], float2 (&im)[kPos], const BlockCtx& bc,
+                                        const DevPass& Pp, const PassArgs& a, const CoefRegion* C, int d, int l,
+                                        uint32_t tid, uint32_t base_q, uint32_t s_o) {
+  const float2* dq = a.dq + (size_t)(l + 1) * a.n * 2;
+  float fr, fi;
+  uint32_t w;
+  switch (phase) {
+    case 0: diag_thread_t<0, V>(bc, Pp, dq, l, tid, base_q, s_o, &fr, &fi, &w); break;
+    case 1: diag_thread_t<1, V>(bc, Pp, dq, l, tid, base_q, s_o, &fr, &fi, &w); break;
+    default: diag_thread_t<2, V>(bc, Pp, dq, l, tid, base_q, s_o, &fr, &fi, &w); break;
+  }
+  // per position: the factor (scalar complex, table entries from the constant
+  // bank), its sign, then the product with both lanes
 #pragma unroll
   for (int j = 0; j < kPos; ++j) {
-    const float2 r = c_reg[region].diag[d][j];
+    const float2 r = C->diag[d][j];
     const uint32_t sb = (w << (31 - j)) & 0x80000000u;
     const float gr = __uint_as_float(__float_as_uint(fmaf(-fi, r.y, fr * r.x)) ^ sb);
     const float gi = __uint_as_float(__float_as_uint(fmaf(fr, r.y, fi * r.x)) ^ sb);
     const float2 xr = re[j], xi = im[j];
     re[j] = make_float2(fmaf(gr, xr.x, -gi * xi.x), fmaf(gr, xr.y, -gi * xi.y));
     im[j] = make_float2(fmaf(gi, xr.x, gr * xi.x), fmaf(gi, xr.y, gr * xi.y));
-  }
-}
-
-template <int V>
-__device__ __forceinline__ void diag_op(int phase, float2 (&re)[kPos], float2 (&im)[kPos], const BlockCtx& bc,
-                                        const DevPass& Pp, const PassArgs& a, int region, int d, int l, uint32_t tid,
-                                        uint32_t base_q, uint32_t s_o) {
-  switch (phase) {
-    case 0: diag_t<0, V>(re, im, bc, Pp, a, region, d, l, tid, base_q, s_o); break;
-    case 1: diag_t<1, V>(re, im, bc, Pp, a, region, d, l, tid, base_q, s_o); break;
-    default: diag_t<2, V>(re, im, bc, Pp, a, region, d, l, tid, base_q, s_o); break;
   }
 }
 
@@ -1065,14 +1072,20 @@ __host__ __device__ constexpr size_t pass_buf_bytes(bool tma) {
   return tma ? kLandBytes + kExch8Bytes : (size_t)kSmemSlots * sizeof(float4);
 }
 
+// Register budget: tensor-copy passes and the one-launch passes of
+// single-tile circuits (split form, n <= 12, at most a few hundred tiles a
+// launch) run two blocks per SM (up to 255 registers); the others three.
 template <bool BWD, int MODE, int V, int RE>
-__global__ void __launch_bounds__(kThreads, MODE == 2 ? kBlocksPerSmTma : kBlocksPerSm)
+__global__ void __launch_bounds__(kThreads, (MODE == 2 || RE == 3) ? kBlocksPerSmTma : kBlocksPerSm)
     pass_kernel(const PassArgs a, const __grid_constant__ DevPass P, const __grid_constant__ CUtensorMap tm0,
                 const __grid_constant__ CUtensorMap tm1) {
   constexpr bool SLOW = MODE == 0;
   constexpr bool TMA = MODE == 2;
   constexpr bool REUP = RE == 1 || RE == 2;  // data re-uploading folded into the fused rotations
   constexpr bool SPLIT = RE == 3;            // split form: OP_RY / OP_DIAG instead of OP_ROT / OP_CZ
+  // split passes of circuits that fit one tile (n <= 12): every pass in one
+  // launch, coefficients from the workspace (see MULTI below)
+  constexpr bool MULTI = SPLIT && !TMA;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   float4* tile = reinterpret_cast<float4*>(smem_raw);  // MODE 2: the landing buffer
   float2* ex8 = reinterpret_cast<float2*>(smem_raw + kLandBytes);  // MODE 2: the exchange buffer
@@ -1122,10 +1135,203 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? kBlocksPerSmTma : kBlock
   // latency hides behind the last register phase; n < 5 loads directly.  The
   // tensor copy of the next tile is issued right after the current tile is in
   // registers.
-  const bool can_pf = !SLOW && loads;
+  const bool can_pf = !SLOW && loads && !MULTI;
   const int mem_ph = BWD ? P.store_phase : P.load_phase;
   const int pf_at = BWD ? P.pf_bwd : P.pf_fwd;  // op index after which to prefetch (-1: after the load)
   bool have_pf = false;
+
+  // The ops of one pass on the registers, forward order (PP: the pass, C: its
+  // coefficients; the layout is P's, the same for every pass of a launch).
+  auto run_fwd_ops = [&](const DevPass& PP, const CoefRegion* C, uint32_t base_q, uint32_t s_o, uint32_t unit_base,
+                         float2 (&re)[kPos], float2 (&im)[kPos], bool pf_next, auto&& prefetch_next) {
+    const int nops = PP.nops;
+    for (int oi = 0; oi < nops; ++oi) {
+      const DevOp op = PP.ops[oi];
+      if (op.kind == OP_EXCH) {
+        if constexpr (TMA) exchange8<V>(op.a, op.b, re, im, ex8, tid);
+        else exchange<V>(op.a, op.b, re, im, tile, tid);
+      } else if constexpr (SPLIT) {
+        if (op.kind == OP_RY) {
+          int slot = op.d;
+#pragma unroll
+          for (int k = 0; k < kRegBits; ++k)
+            if ((op.b >> k) & 1) {
+              const float4 f0 = C->rot[slot][0];
+              const bool cot = C->rot[slot][1].x != 0.f;
+              ++slot;
+              const float2 p = make_float2(f0.x, f0.y), np = make_float2(f0.z, f0.w);
+              if (cot) ry_fwd_k<true>(k, re, im, p, np);
+              else ry_fwd_k<false>(k, re, im, p, np);
+            }
+        } else if (op.kind == OP_DIAG) {
+          diag_op<V>(op.a, re, im, *bc, P, a, C, op.d, op.c, tid, base_q, s_o);
+        }
+      } else if (op.kind == OP_ROT) {
+        int slot = op.d;
+        if (REUP) {  // the encoding again, folded into the layer's rotations
+          uint32_t unit, mu[kRegBits];
+          int rq[kRegBits];
+          unit_maps<V>(op.a, *bc, tid, unit_base, &unit, mu, rq);
+#pragma unroll
+          for (int k = 0; k < kRegBits; ++k)
+            if ((op.b >> k) & 1) {
+              const Coef c = const_coef(region, slot++);
+              if (RE == 1) {
+                float2 cs, sn;
+                enc_coef<false>(a, unit, rq[k], &cs, &sn);
+                rot_fwd_k(k, re, im, SameCoef{reup_coef<false>(c, cs, sn)});
+              } else {
+                rot_fwd_k(k, re, im, ReupPairCoef<false>{c, a, rq[k], unit, mu});
+              }
+            }
+        } else {
+#pragma unroll
+          for (int k = 0; k < kRegBits; ++k)
+            if ((op.b >> k) & 1) rot_fwd_k(k, re, im, SameCoef{const_coef(region, slot++)});
+        }
+      } else if (op.kind == OP_CZ) {
+        cz_op<V>(op.a, re, im, *bc, P, tid, base_q, s_o);
+      }
+      if (pf_next && oi == pf_at) prefetch_next();
+    }
+  };
+
+  // The ops of one pass in reverse (un-applied), with the gradient sums into acc.
+  auto run_bwd_ops = [&](const DevPass& PP, const CoefRegion* C, uint32_t base_q, uint32_t s_o, uint32_t unit_base,
+                         float2 (&re)[kPos], float2 (&im)[kPos], bool pf_next, auto&& prefetch_next) {
+    const int pacc = PP.nslots * 3;  // row stride of the pass's sums
+    for (int oi = PP.nops - 1; oi >= 0; --oi) {
+      const DevOp op = PP.ops[oi];
+      if (op.kind == OP_EXCH) {
+        if constexpr (TMA) exchange8<V>(op.b, op.a, re, im, ex8, tid);
+        else exchange<V>(op.b, op.a, re, im, tile, tid);
+      } else if constexpr (SPLIT) {
+        if (op.kind == OP_RY) {
+          // the same sums, then Ry un-applied (tangent or cotangent form)
+          int slot = op.d, pslot = -1;
+          float3 pend = make_float3(0.f, 0.f, 0.f);
+#pragma unroll
+          for (int k = 0; k < kRegBits; ++k)
+            if ((op.b >> k) & 1) {
+              float r;
+              float3 v;
+              const float4 f0 = C->rot[slot][0];
+              const bool cot = C->rot[slot][1].x != 0.f;
+              const float2 p = make_float2(f0.x, f0.y), np = make_float2(f0.z, f0.w);
+              v = rot_bwd_sums_k(k, re, im, pend, lane, &r);
+              if (cot) ry_fwd_k<true>(k, re, im, p, np);
+              else ry_fwd_k<false>(k, re, im, p, np);
+              if (pslot >= 0 && (lane & 7) == 0 && lane < 24) acc[warp * pacc + pslot * 3 + (lane >> 3)] += r;
+              pend = v;
+              pslot = slot++;
+            }
+          if (pslot >= 0) {
+            const float r = warp_reduce3(pend.x, pend.y, pend.z, lane);
+            if ((lane & 7) == 0 && lane < 24) acc[warp * pacc + pslot * 3 + (lane >> 3)] += r;
+          }
+        } else if (op.kind == OP_DIAG) {
+          // the diagonal before layer 0 needs no un-applying: nothing reads the state after it
+          if (op.c >= 0) diag_op<V>(op.a, re, im, *bc, P, a, C, op.d, op.c, tid, base_q, s_o);
+        }
+      } else if (op.kind == OP_ROT) {
+        // each rotation finishes the warp sum of the previous one
+        int slot = op.d, pslot = -1;
+        float3 pend = make_float3(0.f, 0.f, 0.f);
+        // re-uploading: Ry(-x) of the layer's encoding joins U^dagger
+        uint32_t unit = 0, mu[kRegBits] = {0u, 0u, 0u, 0u, 0u};
+        int rq[kRegBits] = {0, 0, 0, 0, 0};
+        if (REUP) unit_maps<V>(op.a, *bc, tid, unit_base, &unit, mu, rq);
+#pragma unroll
+        for (int k = 0; k < kRegBits; ++k)
+          if ((op.b >> k) & 1) {
+            float r;
+            float3 v;
+            const Coef c = const_coef(region, slot);
+            if (RE == 0) {
+              v = rot_bwd_red_k(k, re, im, SameCoef{c}, pend, lane, &r);
+            } else if (RE == 1) {
+              float2 cs, sn;
+              enc_coef<true>(a, unit, rq[k], &cs, &sn);
+              v = rot_bwd_red_k(k, re, im, SameCoef{reup_coef<true>(c, cs, sn)}, pend, lane, &r);
+            } else {
+              v = rot_bwd_red_k(k, re, im, ReupPairCoef<true>{c, a, rq[k], unit, mu}, pend, lane, &r);
+            }
+            if (pslot >= 0 && (lane & 7) == 0 && lane < 24) acc[warp * pacc + pslot * 3 + (lane >> 3)] += r;
+            pend = v;
+            pslot = slot++;
+          }
+        if (pslot >= 0) {
+          const float r = warp_reduce3(pend.x, pend.y, pend.z, lane);
+          if ((lane & 7) == 0 && lane < 24) acc[warp * pacc + pslot * 3 + (lane >> 3)] += r;
+        }
+      } else if (op.kind == OP_CZ) {
+        cz_op<V>(op.a, re, im, *bc, P, tid, base_q, s_o);
+      }
+      if (pf_next && oi == pf_at) prefetch_next();
+    }
+  };
+
+  if constexpr (MULTI) {
+    // Every pass of the launch (a.npass of them, all with P's tile layout) on
+    // each tile, the state kept in registers in between.  The backward's sums
+    // go to the block's row of each pass after that pass, so start the rows
+    // at zero.
+    if (BWD) {
+      for (int pi = 0; pi < a.npass; ++pi) {
+        const int pn = a.passes[pi].nslots * 3;
+        float* row = a.partials + a.passes[pi].partial_off + (size_t)blockIdx.x * pn;
+        for (int i = tid; i < pn; i += kThreads) row[i] = 0.f;
+      }
+    }
+    auto none = []() {};
+    for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x) {
+      uint32_t base_q, base_a, unit_base;
+      tile_base(P, t, &base_q, &base_a, &unit_base);
+      const uint32_t s_o = bond_parity(base_q, a);
+      float2 re[kPos], im[kPos];
+      if (!BWD) {
+        const DevPass& P0 = a.passes[0];
+        if (P0.gen) mem_op<false, SLOW, V, M_GEN>(P0.load_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
+        else mem_op<false, SLOW, V, M_LOAD>(P0.load_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
+        for (int pi = 0; pi < a.npass; ++pi) {
+          const DevPass& PP = a.passes[pi];
+          run_fwd_ops(PP, a.coef + pi, base_q, s_o, unit_base, re, im, false, none);
+          if (PP.ckpt >= 0)
+            mem_op<false, SLOW, V, M_CKPT_STORE>(PP.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im, PP.ckpt);
+        }
+        const DevPass& PL = a.passes[a.npass - 1];
+        if (PL.last) mem_op<false, SLOW, V, M_STORE_STD>(PL.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
+        else mem_op<false, SLOW, V, M_STORE>(PL.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
+      } else {
+        const DevPass& PL = a.passes[a.npass - 1];
+        mem_op<true, SLOW, V, M_LOAD>(PL.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
+        for (int pi = a.npass - 1; pi >= 0; --pi) {
+          const DevPass& PP = a.passes[pi];
+          if (PP.ckpt >= 0)
+            mem_op<true, SLOW, V, M_CKPT_RESTORE>(PP.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im,
+                                                  PP.ckpt, a.rscale ? __ldg(a.rscale + pi) : 1.f);
+          for (int i = tid; i < kWarps * kMaxSlots * 3; i += kThreads) acc[i] = 0.f;
+          __syncthreads();
+          run_bwd_ops(PP, a.coef + pi, base_q, s_o, unit_base, re, im, false, none);
+          __syncthreads();
+          const int pn = PP.nslots * 3;
+          float* row = a.partials + PP.partial_off + (size_t)blockIdx.x * pn;
+          for (int i = tid; i < pn; i += kThreads) {
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) v += acc[w * pn + i];
+            row[i] += v;
+          }
+          __syncthreads();
+        }
+        // the first pass is the encoding pass: nothing reads the state after it
+        if (!a.passes[0].gen) mem_op<true, SLOW, V, M_STORE>(a.passes[0].load_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
+      }
+    }
+    return;
+  }
+
+  const CoefRegion* creg = &c_reg[region];
   for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x) {
     uint32_t base_q, base_a, unit_base;
     tile_base(P, t, &base_q, &base_a, &unit_base);
@@ -1170,55 +1376,7 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? kBlocksPerSmTma : kBlock
       } else if (have_pf) load_prefetched<V>(P.load_phase, re, im, tile, tid);
       else mem_op<false, SLOW, V, M_LOAD>(P.load_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
       if (pf_next && pf_at < 0) prefetch_next();
-      for (int oi = 0; oi < P.nops; ++oi) {
-        const DevOp op = P.ops[oi];
-        if (op.kind == OP_EXCH) {
-          if constexpr (TMA) exchange8<V>(op.a, op.b, re, im, ex8, tid);
-          else exchange<V>(op.a, op.b, re, im, tile, tid);
-        } else if constexpr (SPLIT) {
-          if (op.kind == OP_RY) {
-            int slot = op.d;
-#pragma unroll
-            for (int k = 0; k < kRegBits; ++k)
-              if ((op.b >> k) & 1) {
-                const float4 f0 = c_reg[region].rot[slot][0];
-                const bool cot = c_reg[region].rot[slot][1].x != 0.f;
-                ++slot;
-                const float2 p = make_float2(f0.x, f0.y), np = make_float2(f0.z, f0.w);
-                if (cot) ry_fwd_k<true>(k, re, im, p, np);
-                else ry_fwd_k<false>(k, re, im, p, np);
-              }
-          } else if (op.kind == OP_DIAG) {
-            diag_op<V>(op.a, re, im, *bc, P, a, region, op.d, op.c, tid, base_q, s_o);
-          }
-        } else if (op.kind == OP_ROT) {
-          int slot = op.d;
-          if (REUP) {  // the encoding again, folded into the layer's rotations
-            uint32_t unit, mu[kRegBits];
-            int rq[kRegBits];
-            unit_maps<V>(op.a, *bc, tid, unit_base, &unit, mu, rq);
-#pragma unroll
-            for (int k = 0; k < kRegBits; ++k)
-              if ((op.b >> k) & 1) {
-                const Coef c = const_coef(region, slot++);
-                if (RE == 1) {
-                  float2 cs, sn;
-                  enc_coef<false>(a, unit, rq[k], &cs, &sn);
-                  rot_fwd_k(k, re, im, SameCoef{reup_coef<false>(c, cs, sn)});
-                } else {
-                  rot_fwd_k(k, re, im, ReupPairCoef<false>{c, a, rq[k], unit, mu});
-                }
-              }
-          } else {
-#pragma unroll
-            for (int k = 0; k < kRegBits; ++k)
-              if ((op.b >> k) & 1) rot_fwd_k(k, re, im, SameCoef{const_coef(region, slot++)});
-          }
-        } else if (op.kind == OP_CZ) {
-          cz_op<V>(op.a, re, im, *bc, P, tid, base_q, s_o);
-        }
-        if (pf_next && oi == pf_at) prefetch_next();
-      }
+      run_fwd_ops(P, creg, base_q, s_o, unit_base, re, im, pf_next, prefetch_next);
       if (P.ckpt >= 0) mem_op<false, SLOW, V, M_CKPT_STORE>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im, P.ckpt);
       if (P.last) mem_op<false, SLOW, V, M_STORE_STD>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
       else mem_op<false, SLOW, V, M_STORE>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
@@ -1229,75 +1387,7 @@ __global__ void __launch_bounds__(kThreads, MODE == 2 ? kBlocksPerSmTma : kBlock
       if (!TMA && P.ckpt >= 0)
         mem_op<true, SLOW, V, M_CKPT_RESTORE>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im, P.ckpt, rs);
       if (pf_next && pf_at < 0) prefetch_next();
-      for (int oi = P.nops - 1; oi >= 0; --oi) {
-        const DevOp op = P.ops[oi];
-        if (op.kind == OP_EXCH) {
-          if constexpr (TMA) exchange8<V>(op.b, op.a, re, im, ex8, tid);
-          else exchange<V>(op.b, op.a, re, im, tile, tid);
-        } else if constexpr (SPLIT) {
-          if (op.kind == OP_RY) {
-            // the same sums, then Ry un-applied (tangent or cotangent form)
-            int slot = op.d, pslot = -1;
-            float3 pend = make_float3(0.f, 0.f, 0.f);
-#pragma unroll
-            for (int k = 0; k < kRegBits; ++k)
-              if ((op.b >> k) & 1) {
-                float r;
-                float3 v;
-                const float4 f0 = c_reg[region].rot[slot][0];
-                const bool cot = c_reg[region].rot[slot][1].x != 0.f;
-                const float2 p = make_float2(f0.x, f0.y), np = make_float2(f0.z, f0.w);
-                v = rot_bwd_sums_k(k, re, im, pend, lane, &r);
-                if (cot) ry_fwd_k<true>(k, re, im, p, np);
-                else ry_fwd_k<false>(k, re, im, p, np);
-                if (pslot >= 0 && (lane & 7) == 0 && lane < 24) acc[warp * nacc + pslot * 3 + (lane >> 3)] += r;
-                pend = v;
-                pslot = slot++;
-              }
-            if (pslot >= 0) {
-              const float r = warp_reduce3(pend.x, pend.y, pend.z, lane);
-              if ((lane & 7) == 0 && lane < 24) acc[warp * nacc + pslot * 3 + (lane >> 3)] += r;
-            }
-          } else if (op.kind == OP_DIAG) {
-            // the diagonal before layer 0 needs no un-applying: nothing reads the state after it
-            if (op.c >= 0) diag_op<V>(op.a, re, im, *bc, P, a, region, op.d, op.c, tid, base_q, s_o);
-          }
-        } else if (op.kind == OP_ROT) {
-          // each rotation finishes the warp sum of the previous one
-          int slot = op.d, pslot = -1;
-          float3 pend = make_float3(0.f, 0.f, 0.f);
-          // re-uploading: Ry(-x) of the layer's encoding joins U^dagger
-          uint32_t unit = 0, mu[kRegBits] = {0u, 0u, 0u, 0u, 0u};
-          int rq[kRegBits] = {0, 0, 0, 0, 0};
-          if (REUP) unit_maps<V>(op.a, *bc, tid, unit_base, &unit, mu, rq);
-#pragma unroll
-          for (int k = 0; k < kRegBits; ++k)
-            if ((op.b >> k) & 1) {
-              float r;
-              float3 v;
-              const Coef c = const_coef(region, slot);
-              if (RE == 0) {
-                v = rot_bwd_red_k(k, re, im, SameCoef{c}, pend, lane, &r);
-              } else if (RE == 1) {
-                float2 cs, sn;
-                enc_coef<true>(a, unit, rq[k], &cs, &sn);
-                v = rot_bwd_red_k(k, re, im, SameCoef{reup_coef<true>(c, cs, sn)}, pend, lane, &r);
-              } else {
-                v = rot_bwd_red_k(k, re, im, ReupPairCoef<true>{c, a, rq[k], unit, mu}, pend, lane, &r);
-              }
-              if (pslot >= 0 && (lane & 7) == 0 && lane < 24) acc[warp * nacc + pslot * 3 + (lane >> 3)] += r;
-              pend = v;
-              pslot = slot++;
-            }
-          if (pslot >= 0) {
-            const float r = warp_reduce3(pend.x, pend.y, pend.z, lane);
-            if ((lane & 7) == 0 && lane < 24) acc[warp * nacc + pslot * 3 + (lane >> 3)] += r;
-          }
-        } else if (op.kind == OP_CZ) {
-          cz_op<V>(op.a, re, im, *bc, P, tid, base_q, s_o);
-        }
-        if (pf_next && oi == pf_at) prefetch_next();
-      }
+      run_bwd_ops(P, creg, base_q, s_o, unit_base, re, im, pf_next, prefetch_next);
       if (!P.gen) mem_op<true, SLOW, V, M_STORE>(P.load_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
     }
     have_pf = pf_next;
@@ -1563,22 +1653,33 @@ __global__ void expect_final_kernel(const double* partial, int chunks, int B, fl
 // in the backward state's frame; gfix[.][0] takes them to the split circuit's
 // states and Rz(phi1) (gfix[.][1]) to the state after the whole rotation:
 // Rz(f)^dagger X Rz(f) = cos f X - sin f Y, Rz(f)^dagger Y Rz(f) = sin f X + cos f Y.
+// One warp per (layer, qubit): lane i sums rows i, i + 32, ... in fp64, then
+// a fixed butterfly combines the lanes, so the order (and the result) does
+// not depend on timing.
 __global__ void grad_reduce_kernel(const DevPass* passes, const int* slot_pass,
                                    const int* slot_index, const float* partials, int grid,
                                    const float* theta, const double* gfix, int L, int n, float* grad,
                                    unsigned* status) {
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= L * n) return;
+  const int idx = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (idx >= L * n) return;  // whole warps leave together
   const int p = slot_pass[idx], s = slot_index[idx];
   const DevPass& ps = passes[p];
   const int stride = ps.nslots * 3;
   const float* base = partials + ps.partial_off + s * 3;
   double sx = 0.0, sy = 0.0, sz = 0.0;
-  for (int c = 0; c < grid; ++c) {
+  for (int c = lane; c < grid; c += 32) {
     sx += base[(size_t)c * stride + 0];
     sy += base[(size_t)c * stride + 1];
     sz += base[(size_t)c * stride + 2];
   }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    sx += __shfl_xor_sync(0xffffffffu, sx, o);
+    sy += __shfl_xor_sync(0xffffffffu, sy, o);
+    sz += __shfl_xor_sync(0xffffffffu, sz, o);
+  }
+  if (lane != 0) return;
   if (gfix) {
     const double sc = gfix[(size_t)idx * 2 + 0], f = gfix[(size_t)idx * 2 + 1];
     double sf, cf;
@@ -1949,9 +2050,9 @@ cudaError_t launch_expect(const float2* psi, int B, int n, double* partial, floa
 cudaError_t launch_grad_reduce(const DevPass* passes, const int* slot_pass, const int* slot_index,
                                const float* partials, int grid, const float* theta, const double* gfix, int L,
                                int n, float* grad, unsigned* status, cudaStream_t s) {
-  const int tot = L * n;
-  grad_reduce_kernel<<<(tot + 127) / 128, 128, 0, s>>>(passes, slot_pass, slot_index, partials,
-                                                       grid, theta, gfix, L, n, grad, status);
+  const long long threads = (long long)L * n * 32;  // one warp per (layer, qubit)
+  grad_reduce_kernel<<<(unsigned)((threads + 127) / 128), 128, 0, s>>>(passes, slot_pass, slot_index, partials,
+                                                                       grid, theta, gfix, L, n, grad, status);
   return cudaGetLastError();
 }
 

@@ -55,7 +55,12 @@ struct PassArgs {
   unsigned* status;
   int reupload;          // every layer starts with the encoding Ry(x_q) again
   const float2* dq;      // split form: [L + 1][n][2] per-qubit factors of the diagonal ops (this direction)
-  const float* rscale;   // split form, backward checkpoint pass: scale of the restored state (null: 1)
+  const float* rscale;   // split form, backward checkpoint pass: scale of the restored state (null: 1);
+                         // with npass > 0: the scales of all passes, by pass index
+  // split form, circuits that fit one tile: every pass in one launch
+  int npass;                 // passes of the launch (0: one pass, the kernel's parameter)
+  const DevPass* passes;     // [npass] device copy, forward order
+  const CoefRegion* coef;    // [npass] coefficients of this direction
   uint32_t cz_nb[kMaxQubits];    // CZ neighbours of each qubit (qubit mask)
   uint32_t cz_nbhi[kMaxQubits];  // CZ neighbours of each qubit above it (qubit mask)
 };

@@ -13,7 +13,9 @@ from dataclasses import dataclass
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libqml.so")
+# QML_LIBRARY: the path of another build of the library (e.g. one made with other
+# compile flags); the in-tree build by default
+LIB_PATH = os.environ.get("QML_LIBRARY") or os.path.join(_HERE, "libqml.so")
 
 QML_OK = 0
 STATUS_NAMES = {
