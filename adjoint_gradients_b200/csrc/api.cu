@@ -31,6 +31,7 @@ struct Layout {
   size_t scratch, dummy2, sub_passes, sub_slot_pass, sub_slot_index;  // CNOT entanglers only
   size_t passes_split, undo, s_rot, s_lay, s_gfix, s_dqf, s_dqb, rscale;  // split form (fp32 only)
   size_t fault_theta;  // QML_FAULT=nan_theta, fp64: a copy of theta with a NaN angle
+  size_t s_dq64f, s_dq64b, rscale64;  // split form, fp64 contexts
   size_t base_total;
   // host-step extras
   size_t h_psi, h_lam, h_x, h_theta, h_y, h_E, h_g, h_loss, h_grad;
@@ -211,15 +212,19 @@ void compute_layout(qml_ctx* c) {
     l.sub_slot_pass = take(sizeof(int) * (size_t)n);
     l.sub_slot_index = take(sizeof(int) * (size_t)n);
   }
+  l.passes_split = take(sizeof(DevPass) * c->dpass_split.size());
+  l.undo = take(sizeof(int) * (size_t)L * n);
+  l.s_rot = take(sizeof(SplitRot) * (size_t)L * n);
+  l.s_lay = take(sizeof(SplitLayer) * (size_t)L);
+  l.s_gfix = take(sizeof(double) * 2 * (size_t)L * n);
   if (!c->f64) {
-    l.passes_split = take(sizeof(DevPass) * c->dpass_split.size());
-    l.undo = take(sizeof(int) * (size_t)L * n);
-    l.s_rot = take(sizeof(SplitRot) * (size_t)L * n);
-    l.s_lay = take(sizeof(SplitLayer) * (size_t)L);
-    l.s_gfix = take(sizeof(double) * 2 * (size_t)L * n);
     l.s_dqf = take(sizeof(float2) * 2 * (size_t)(L + 1) * n);
     l.s_dqb = take(sizeof(float2) * 2 * (size_t)(L + 1) * n);
     l.rscale = take(sizeof(float) * c->dpass_split.size());
+  } else {
+    l.s_dq64f = take(sizeof(double2) * 2 * (size_t)(L + 1) * n);
+    l.s_dq64b = take(sizeof(double2) * 2 * (size_t)(L + 1) * n);
+    l.rscale64 = take(sizeof(double) * c->dpass_split.size());
   }
   if (c->f64 && c->fault == qml_ctx::FAULT_NAN) l.fault_theta = take(sizeof(double) * 3 * (size_t)L * n);
   l.base_total = o;
@@ -291,6 +296,8 @@ T* at(qml_ctx* c, size_t off) {
 // (re-uploading folds per-sample encodings into the rotations; CNOT layers
 // run as one-layer schedules).
 bool use_split(const qml_ctx* c) { return !c->f64 && !c->reupload && !c->cnot; }
+// fp64 contexts: the same rule
+bool use_split64(const qml_ctx* c) { return c->f64 && !c->reupload && !c->cnot; }
 
 const std::vector<DevPass>& fp32_passes(const qml_ctx* c) { return use_split(c) ? c->dpass_split : c->dpass; }
 
@@ -806,7 +813,22 @@ Pass64Args pass64_args(qml_ctx* c, const double* theta, const double* x, int B, 
   a.status = at<unsigned>(c, c->lay.status);
   a.reupload = c->reupload ? 1 : 0;
   for (int q = 0; q < kMaxQubits; ++q) a.nb[q] = c->nb[q], a.nbhi[q] = c->nbhi[q];
+  a.L = c->cfg.n_layers;
+  if (use_split64(c)) {
+    a.srot = at<SplitRot>(c, c->lay.s_rot);
+    a.slay = at<SplitLayer>(c, c->lay.s_lay);
+  }
   return a;
+}
+
+// Split-form tables of an fp64 context from theta (both directions).
+cudaError_t prep_split64(qml_ctx* c, const double* theta, cudaStream_t s) {
+  c->launches += 4;
+  return launch_prep_split64(at<DevPass>(c, c->lay.passes_split), (int)c->dpass_split.size(), theta,
+                             c->cfg.n_layers, c->cfg.n_qubits, at<int>(c, c->lay.undo),
+                             at<SplitRot>(c, c->lay.s_rot), at<SplitLayer>(c, c->lay.s_lay),
+                             at<double>(c, c->lay.s_gfix), at<double2>(c, c->lay.s_dq64f),
+                             at<double2>(c, c->lay.s_dq64b), at<double>(c, c->lay.rscale64), s);
 }
 
 void set_pass_tile(const qml_ctx* c, int p, int B, Pass64Args* a) {
@@ -946,8 +968,8 @@ qml_status run_backward64_cnot(qml_ctx* c, const double* theta, const double* x,
     }
     const DevPass* dsub = at<DevPass>(c, c->lay.sub_passes) + (size_t)P1 * v;
     e = launch_grad_reduce64(dsub, at<int>(c, c->lay.sub_slot_pass), at<int>(c, c->lay.sub_slot_index),
-                             at<double>(c, c->lay.partials), c->grid_bwd, theta + (size_t)l * n * 3, 1, n,
-                             grad + (size_t)l * n * 3, at<unsigned>(c, c->lay.status), s);
+                             at<double>(c, c->lay.partials), c->grid_bwd, theta + (size_t)l * n * 3, nullptr, 1,
+                             n, grad + (size_t)l * n * 3, at<unsigned>(c, c->lay.status), s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
     ++c->launches;
   }
@@ -958,10 +980,16 @@ qml_status run_forward64(qml_ctx* c, const double* theta, const double* x, int B
                          cudaStream_t s) {
   if (c->cnot) return run_forward64_cnot(c, theta, x, B, psi, expect, s);
   Pass64Args a = pass64_args(c, theta, x, B, psi, nullptr);
+  const bool split = use_split64(c);
+  if (split) {
+    if (prep_split64(c, theta, s) != cudaSuccess) return QML_ERR_CUDA;
+    a.dq = at<double2>(c, c->lay.s_dq64f);
+  }
+  const std::vector<DevPass>& passes = split ? c->dpass_split : c->dpass;
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, false);
-  for (int p = 0; p < (int)c->dpass.size(); ++p) {
-    const DevPass& dp = c->dpass[p];
+  for (int p = 0; p < (int)passes.size(); ++p) {
+    const DevPass& dp = passes[p];
     set_pass_tile(c, p, B, &a);
     if (launch_pass64(false, a, dp, (int)std::min<long long>(c->grid_fwd, a.n_tiles), s) != cudaSuccess)
       return QML_ERR_CUDA;
@@ -981,19 +1009,27 @@ qml_status run_backward64(qml_ctx* c, const double* theta, const double* x, int 
     if (c->ckpt_batch[m] != B) return QML_ERR_CKPT_MISMATCH;
   if (seed64(c, psi, lam, g, B, s) != cudaSuccess) return QML_ERR_CUDA;
   Pass64Args a = pass64_args(c, theta, x, B, psi, lam);
+  const bool split = use_split64(c);
+  if (split) {
+    if (prep_split64(c, theta, s) != cudaSuccess) return QML_ERR_CUDA;
+    a.dq = at<double2>(c, c->lay.s_dq64b);
+  }
+  const std::vector<DevPass>& passes = split ? c->dpass_split : c->dpass;
   ++c->launches;  // gradient reduce
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, true);
   // every block writes its partials, so the grid is the one the layout counted
-  for (int p = (int)c->dpass.size() - 1; p >= 0; --p) {
+  for (int p = (int)passes.size() - 1; p >= 0; --p) {
     set_pass_tile(c, p, B, &a);
-    if (launch_pass64(true, a, c->dpass[p], c->grid_bwd, s) != cudaSuccess) return QML_ERR_CUDA;
+    a.rscale = (split && passes[p].ckpt >= 0) ? at<double>(c, c->lay.rscale64) + p : nullptr;
+    if (launch_pass64(true, a, passes[p], c->grid_bwd, s) != cudaSuccess) return QML_ERR_CUDA;
     ++c->launches;
   }
   if (timed) span_end(c, s, &sp);
   return cuda_status(launch_grad_reduce64(at<DevPass>(c, c->lay.passes), at<int>(c, c->lay.slot_pass),
                                           at<int>(c, c->lay.slot_index), at<double>(c, c->lay.partials),
-                                          c->grid_bwd, theta, L, n, grad, at<unsigned>(c, c->lay.status), s));
+                                          c->grid_bwd, theta, split ? at<double>(c, c->lay.s_gfix) : nullptr, L, n,
+                                          grad, at<unsigned>(c, c->lay.status), s));
 }
 
 }  // namespace
@@ -1129,10 +1165,10 @@ qml_status qml_set_workspace(qml_ctx* c, void* ws, size_t bytes, void* stream) {
   if (e == cudaSuccess)
     e = cudaMemcpyAsync(c->ws + c->lay.slot_index, si.data(), sizeof(int) * si.size(), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(c->ws + c->lay.dummy, 0, sizeof(float2) * (size_t)c->N, s);
-  if (e == cudaSuccess && !c->f64)
+  if (e == cudaSuccess)
     e = cudaMemcpyAsync(c->ws + c->lay.passes_split, c->dpass_split.data(), sizeof(DevPass) * c->dpass_split.size(),
                         cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess && !c->f64)
+  if (e == cudaSuccess)
     e = cudaMemcpyAsync(c->ws + c->lay.undo, c->undo.data(), sizeof(int) * c->undo.size(), cudaMemcpyHostToDevice, s);
   // the host vectors above are pageable: the copies complete before return
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
@@ -1360,7 +1396,7 @@ qml_status qml_set_reupload(qml_ctx* c, int on) {
 
 int qml_reupload(const qml_ctx* c) { return c ? (c->reupload ? 1 : 0) : -1; }
 
-int qml_split_form(const qml_ctx* c) { return c ? (use_split(c) ? 1 : 0) : -1; }
+int qml_split_form(const qml_ctx* c) { return c ? ((use_split(c) || use_split64(c)) ? 1 : 0) : -1; }
 
 int qml_entangler_bonds(const qml_ctx* c) {
   return c ? (int)(c->cnot ? c->cnot_pairs.size() : c->bonds.size()) : -1;

@@ -47,8 +47,9 @@ struct Ctx64 {
   int pos_of_q[kMaxQubits];
   uint32_t off_lo[64], off_hi[64];  // index offset of position bits 0-5 / 6-11
   uint32_t s_off[kTilePos / 32];    // entangler parity of the in-tile part of each position
-  double4 coef[kMaxSlots];          // (ar, ai, br, bi): U forward, U^dagger backward
+  double4 coef[kMaxSlots];          // (ar, ai, br, bi): U forward, U^dagger backward; split form: (p, cot, 0, 0)
   double cs[kMaxQubits], sn[kMaxQubits];  // (cos, sin)(x/2) of the tile's sample
+  double2 dlo[64], dhi[64];         // split form, diagonal op: factors of position bits 0-5 / 6-11
 };
 
 size_t f64_smem_bytes(bool bwd, int tmax) {
@@ -74,6 +75,22 @@ template <bool BWD>
 __device__ __forceinline__ double4 reup64(double4 u, double c, double s) {
   if (!BWD) return make_double4(u.x * c + u.z * s, u.y * c + u.w * s, u.z * c - u.x * s, u.w * c - u.y * s);
   return make_double4(u.x * c - u.z * s, u.y * c + u.w * s, u.z * c + u.x * s, u.w * c - u.y * s);
+}
+
+// Split form: Ry on the pair (x, y), p = u.x, cotangent form when u.y != 0
+// (the same forms and the same parameter convention as the fp32 passes:
+// tangent x <- x - p y, y <- y + p x; cotangent x <- y - p x, y <- x + p y;
+// the backward pass un-applies with -p (tangent) or p (cotangent)).
+__device__ __forceinline__ void ry64(double2& x, double2& y, const double4& u) {
+  const double p = u.x;
+  const double2 x0 = x;
+  if (u.y == 0.0) {
+    x = make_double2(fma(-p, y.x, x0.x), fma(-p, y.y, x0.y));
+    y = make_double2(fma(p, x0.x, y.x), fma(p, x0.y, y.y));
+  } else {
+    x = make_double2(fma(-p, x0.x, y.x), fma(-p, x0.y, y.y));
+    y = make_double2(fma(p, y.x, x0.x), fma(p, y.y, x0.y));
+  }
 }
 
 template <typename T>
@@ -109,7 +126,7 @@ __device__ __forceinline__ void slot_store(const Pass64Args& a, int slot, size_t
 }
 
 // One rotation chunk of K qubits (slots s0 .. s0+K-1) over the tile.
-template <bool BWD, int K>
+template <bool BWD, int K, bool SPLIT>
 __device__ void rot_chunk(const Pass64Args& a, const DevPass& P, const Ctx64& cx, double2* tp, double2* tl,
                           double* acc, int s0, int warp, int lane) {
   int pb[K], srt[K];
@@ -165,9 +182,11 @@ __device__ void rot_chunk(const Pass64Args& a, const DevPass& P, const Ctx64& cx
           sx[i] += l0.x * p1v.y - l0.y * p1v.x + l1.x * p0v.y - l1.y * p0v.x;  // Im(conj l0 p1 + conj l1 p0)
           sy[i] += l1.x * p0v.x + l1.y * p0v.y - l0.x * p1v.x - l0.y * p1v.y;  // Re(conj l1 p0 - conj l0 p1)
           sz[i] += l0.x * p0v.y - l0.y * p0v.x - l1.x * p1v.y + l1.y * p1v.x;  // Im(conj l0 p0 - conj l1 p1)
-          su2_64(w[j], w[jj], u[i]);
+          if (SPLIT) ry64(w[j], w[jj], u[i]);
+          else su2_64(w[j], w[jj], u[i]);
         }
-        su2_64(v[j], v[jj], u[i]);
+        if (SPLIT) ry64(v[j], v[jj], u[i]);
+        else su2_64(v[j], v[jj], u[i]);
       }
     }
 #pragma unroll
@@ -190,7 +209,9 @@ __device__ void rot_chunk(const Pass64Args& a, const DevPass& P, const Ctx64& cx
   }
 }
 
-template <bool BWD>
+// SPLIT: the split form (OP_RY / OP_DIAG passes, a.srot set); otherwise the
+// fused SU(2) (OP_ROT / OP_CZ).
+template <bool BWD, bool SPLIT>
 __global__ void __launch_bounds__(kT, BWD ? 2 : 3) pass64_kernel(const Pass64Args a, const __grid_constant__ DevPass P) {
   extern __shared__ __align__(16) unsigned char smem64[];
   double2* tp = reinterpret_cast<double2*>(smem64);
@@ -216,8 +237,15 @@ __global__ void __launch_bounds__(kT, BWD ? 2 : 3) pass64_kernel(const Pass64Arg
     cx.T = T;
     cx.n_out = no;
   }
-  // gate coefficients of the pass's slots: U = Rz Ry Rx, in fp64
-  for (int s = tid; s < P.nslots; s += kT) {
+  // gate coefficients of the pass's slots: U = Rz Ry Rx, in fp64; split
+  // form: the tangent-form parameter of Ry (backward: its inverse's)
+  constexpr bool split = SPLIT;
+  for (int s = tid; s < P.nslots && split; s += kT) {
+    const SplitRot r = a.srot[P.slot_lq[s]];
+    const double pr = (BWD && !r.cot) ? -r.tau : r.tau;
+    cx.coef[s] = make_double4(pr, (double)r.cot, 0.0, 0.0);
+  }
+  for (int s = tid; s < P.nslots && !split; s += kT) {
     const int lq = P.slot_lq[s];
     double sa, ca, sb, cb, sg, cg;
     sincos(0.5 * a.theta[lq * 3 + 0], &sa, &ca);
@@ -288,6 +316,10 @@ __global__ void __launch_bounds__(kT, BWD ? 2 : 3) pass64_kernel(const Pass64Arg
         pv = make_double2(r, 0.0);
       } else if (BWD && P.ckpt >= 0) {
         pv = slot_load(a, P.ckpt, g);  // the checkpoint replaces the uncomputed state
+        if (a.rscale) {  // split form: in the backward state's scale
+          const double r = *a.rscale;
+          pv = make_double2(pv.x * r, pv.y * r);
+        }
       } else {
         pv = a.psi[g];
       }
@@ -314,16 +346,66 @@ __global__ void __launch_bounds__(kT, BWD ? 2 : 3) pass64_kernel(const Pass64Arg
 
     for (int k = 0; k < P.nops; ++k) {
       const DevOp op = P.ops[BWD ? P.nops - 1 - k : k];
-      if (op.kind == OP_ROT) {
+      if (op.kind == OP_ROT || op.kind == OP_RY) {
         const int m = __popc((unsigned)op.b);
         for (int c0 = 0; c0 < m; c0 += 3) {
           const int kk = min(3, m - c0);
-          if (kk == 3) rot_chunk<BWD, 3>(a, P, cx, tp, tl, acc, op.d + c0, warp, lane);
-          else if (kk == 2) rot_chunk<BWD, 2>(a, P, cx, tp, tl, acc, op.d + c0, warp, lane);
-          else rot_chunk<BWD, 1>(a, P, cx, tp, tl, acc, op.d + c0, warp, lane);
+          if (split) {
+            if (kk == 3) rot_chunk<BWD, 3, true>(a, P, cx, tp, tl, acc, op.d + c0, warp, lane);
+            else if (kk == 2) rot_chunk<BWD, 2, true>(a, P, cx, tp, tl, acc, op.d + c0, warp, lane);
+            else rot_chunk<BWD, 1, true>(a, P, cx, tp, tl, acc, op.d + c0, warp, lane);
+          } else {
+            if (kk == 3) rot_chunk<BWD, 3, false>(a, P, cx, tp, tl, acc, op.d + c0, warp, lane);
+            else if (kk == 2) rot_chunk<BWD, 2, false>(a, P, cx, tp, tl, acc, op.d + c0, warp, lane);
+            else rot_chunk<BWD, 1, false>(a, P, cx, tp, tl, acc, op.d + c0, warp, lane);
+          }
           __syncthreads();
         }
-      } else if (op.kind == OP_CZ) {
+      } else if (SPLIT && op.kind == OP_DIAG) {
+        // split form: position v (global index base | idx(v)) times
+        // dlo[v & 63] dhi[v >> 6] f_out scale, and the entangler sign (l >= 0)
+        const int l = op.c;
+        if (BWD && l < 0) continue;  // nothing reads the state before layer 0's rotations
+        const double2* dq = a.dq + (size_t)(l + 1) * n * 2;
+        if (tid < 128) {
+          const int i = tid & 63, hi = tid >> 6;
+          double2 f = make_double2(1.0, 0.0);
+          for (int k = 0; k < 6; ++k) {
+            const int pb = k + 6 * hi;
+            if (pb >= T) break;
+            const double2 d = dq[2 * cx.tq[pb] + ((i >> k) & 1)];
+            f = make_double2(f.x * d.x - f.y * d.y, f.x * d.y + f.y * d.x);
+          }
+          if (hi) cx.dhi[i] = f;
+          else cx.dlo[i] = f;
+        }
+        double sc = 1.0;
+        if (l >= 0) sc = BWD ? a.slay[l].gam / (l + 1 < a.L ? a.slay[l + 1].rho : 1.0) : 1.0 / a.slay[l].gam;
+        double2 fo = make_double2(sc, 0.0);
+        for (int k = 0; k < no; ++k) {
+          const int q = cx.oq[k];
+          const double2 d = dq[2 * q + ((base >> q) & 1u)];
+          fo = make_double2(fo.x * d.x - fo.y * d.y, fo.x * d.y + fo.y * d.x);
+        }
+        __syncthreads();
+        for (int v = tid; v < P2; v += kT) {
+          const double2 fl = cx.dlo[v & 63], fh = cx.dhi[(v >> 6) & 63];
+          const double2 f1 = make_double2(fl.x * fh.x - fl.y * fh.y, fl.x * fh.y + fl.y * fh.x);
+          double2 f = make_double2(f1.x * fo.x - f1.y * fo.y, f1.x * fo.y + f1.y * fo.x);
+          if (l >= 0) {
+            const uint32_t par = s_base ^ ((cx.s_off[v >> 5] >> (v & 31)) & 1u) ^ ((uint32_t)__popc(v & cm) & 1u);
+            if (par) f = make_double2(-f.x, -f.y);
+          }
+          const int pp = padp(v);
+          const double2 x = tp[pp];
+          tp[pp] = make_double2(f.x * x.x - f.y * x.y, f.x * x.y + f.y * x.x);
+          if (BWD) {
+            const double2 y = tl[pp];
+            tl[pp] = make_double2(f.x * y.x - f.y * y.y, f.x * y.y + f.y * y.x);
+          }
+        }
+        __syncthreads();
+      } else if (!SPLIT && op.kind == OP_CZ) {
         for (int v = tid; v < P2; v += kT) {
           const uint32_t par = s_base ^ ((cx.s_off[v >> 5] >> (v & 31)) & 1u) ^ ((uint32_t)__popc(v & cm) & 1u);
           if (par) {
@@ -471,9 +553,11 @@ __global__ void obs64_lambda_kernel(const double2* psi, double2* lam, const doub
   lam[idx] = make_double2(g[b] * ar, g[b] * ai);
 }
 
+// gfix (split form, else null): as in the fp32 reduction, the sums scaled to
+// the split circuit's states and rotated by phi1 first.
 __global__ void grad_reduce64_kernel(const DevPass* passes, const int* slot_pass, const int* slot_index,
-                                     const double* partials, int grid, const double* theta, int L, int n,
-                                     double* grad, unsigned* status) {
+                                     const double* partials, int grid, const double* theta, const double* gfix,
+                                     int L, int n, double* grad, unsigned* status) {
   // one warp per (layer, qubit): strided lane sums, then a fixed butterfly
   const int idx = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
@@ -495,6 +579,17 @@ __global__ void grad_reduce64_kernel(const DevPass* passes, const int* slot_pass
     sz += __shfl_xor_sync(0xffffffffu, sz, o);
   }
   if (lane != 0) return;
+  if (gfix) {
+    const double sc = gfix[(size_t)idx * 2 + 0], f = gfix[(size_t)idx * 2 + 1];
+    double sf, cf;
+    sincos(f, &sf, &cf);
+    sx *= sc;
+    sy *= sc;
+    sz *= fabs(sc);
+    const double tx = cf * sx - sf * sy;
+    sy = sf * sx + cf * sy;
+    sx = tx;
+  }
   // (s_x, s_y, s_z) are Im<lambda|P|psi> at the rotation's output; the angle
   // gradients take X and Y back through the Rz and Ry that follow them
   double sb, cb, sg, cg;
@@ -532,24 +627,40 @@ __global__ void loss_seed64_kernel(const double* E, const double* y, int B, doub
 size_t pass64_smem_bytes(bool backward, int tmax) { return f64_smem_bytes(backward, tmax); }
 
 cudaError_t pass64_setup(int tmax, int* blocks_fwd, int* blocks_bwd) {
-  cudaError_t e = cudaFuncSetAttribute(pass64_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)f64_smem_bytes(false, kTileBits));
+  cudaError_t e = cudaSuccess;
+  for (int sp = 0; sp < 2 && e == cudaSuccess; ++sp) {
+    e = cudaFuncSetAttribute(sp ? pass64_kernel<false, true> : pass64_kernel<false, false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)f64_smem_bytes(false, kTileBits));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(sp ? pass64_kernel<true, true> : pass64_kernel<true, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)f64_smem_bytes(true, kTileBits));
+  }
+  // the grid is the same for both forms: take the smaller occupancy
+  int f0 = 0, f1 = 0, b0 = 0, b1 = 0;
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(pass64_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)f64_smem_bytes(true, kTileBits));
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&f0, pass64_kernel<false, false>, kT, f64_smem_bytes(false, tmax));
   if (e == cudaSuccess)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_fwd, pass64_kernel<false>, kT,
-                                                      f64_smem_bytes(false, tmax));
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&f1, pass64_kernel<false, true>, kT, f64_smem_bytes(false, tmax));
   if (e == cudaSuccess)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_bwd, pass64_kernel<true>, kT,
-                                                      f64_smem_bytes(true, tmax));
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b0, pass64_kernel<true, false>, kT, f64_smem_bytes(true, tmax));
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b1, pass64_kernel<true, true>, kT, f64_smem_bytes(true, tmax));
+  *blocks_fwd = std::min(f0, f1);
+  *blocks_bwd = std::min(b0, b1);
   return e;
 }
 
 cudaError_t launch_pass64(bool backward, const Pass64Args& a, const DevPass& p, int grid, cudaStream_t s) {
   if (a.tmax < a.T || a.tmax > kTileBits) return cudaErrorInvalidValue;
-  if (backward) pass64_kernel<true><<<grid, kT, f64_smem_bytes(true, a.tmax), s>>>(a, p);
-  else pass64_kernel<false><<<grid, kT, f64_smem_bytes(false, a.tmax), s>>>(a, p);
+  const bool split = a.srot != nullptr;
+  const size_t smem = f64_smem_bytes(backward, a.tmax);
+  if (backward) {
+    if (split) pass64_kernel<true, true><<<grid, kT, smem, s>>>(a, p);
+    else pass64_kernel<true, false><<<grid, kT, smem, s>>>(a, p);
+  } else {
+    if (split) pass64_kernel<false, true><<<grid, kT, smem, s>>>(a, p);
+    else pass64_kernel<false, false><<<grid, kT, smem, s>>>(a, p);
+  }
   return cudaGetLastError();
 }
 
@@ -594,11 +705,11 @@ cudaError_t launch_obs_bwd_init64(const double2* psi, double2* lam, const double
 }
 
 cudaError_t launch_grad_reduce64(const DevPass* passes, const int* slot_pass, const int* slot_index,
-                                 const double* partials, int grid, const double* theta, int L, int n, double* grad,
-                                 unsigned* status, cudaStream_t s) {
+                                 const double* partials, int grid, const double* theta, const double* gfix, int L,
+                                 int n, double* grad, unsigned* status, cudaStream_t s) {
   const long long threads = (long long)L * n * 32;  // one warp per (layer, qubit)
   grad_reduce64_kernel<<<(unsigned)((threads + 127) / 128), 128, 0, s>>>(passes, slot_pass, slot_index, partials,
-                                                                         grid, theta, L, n, grad, status);
+                                                                         grid, theta, gfix, L, n, grad, status);
   return cudaGetLastError();
 }
 

@@ -1407,195 +1407,6 @@ __global__ void __launch_bounds__(kThreads, (MODE == 2 || RE == 3) ? kBlocksPerS
 
 // ----------------------------------------------------------------- helpers
 
-// U = Rz(g) Ry(b) Rx(a) = [[A, B], [-conj B, conj A]] in fp64 (half angles).
-__device__ __forceinline__ void su2_of(const float* th, double* ar, double* ai, double* br, double* bi) {
-  const double al = th[0], be = th[1], ga = th[2];
-  double sa, ca, sb, cb, sg, cg;
-  sincos(0.5 * al, &sa, &ca);
-  sincos(0.5 * be, &sb, &cb);
-  sincos(0.5 * ga, &sg, &cg);
-  // (Ry Rx)[0][0] = cb ca + i sb sa, (Ry Rx)[0][1] = -sb ca - i cb sa; row 0 of Rz is e^{-i g/2}
-  const double p_re = cb * ca, p_im = sb * sa;
-  const double q_re = -sb * ca, q_im = -cb * sa;
-  *ar = cg * p_re + sg * p_im;
-  *ai = cg * p_im - sg * p_re;
-  *br = cg * q_re + sg * q_im;
-  *bi = cg * q_im - sg * q_re;
-}
-
-// Gate coefficients of every pass slot: U computed in fp64 and rounded to
-// fp32 broadcast pairs, and U^dagger = [[conj A, -B], ...] for the backward
-// passes.  Output: one CoefRegion per pass and direction.
-__global__ void prep_pass_coef_kernel(const DevPass* passes, int n_passes, const float* theta, CoefRegion* cf,
-                                      CoefRegion* ci) {
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= n_passes * kMaxSlots) return;
-  const int p = idx / kMaxSlots, s = idx % kMaxSlots;
-  if (s >= passes[p].nslots) return;
-  const int lq = passes[p].slot_lq[s];
-  double ar, ai, br, bi;
-  su2_of(theta + lq * 3, &ar, &ai, &br, &bi);
-  const float far = (float)ar, fai = (float)ai, fbr = (float)br, fbi = (float)bi;
-  float4* f = cf[p].rot[s];
-  f[0] = make_float4(far, far, fai, fai);
-  f[1] = make_float4(-fai, -fai, fbr, fbr);
-  f[2] = make_float4(fbi, fbi, -fbi, -fbi);
-  f[3] = make_float4(-fbr, -fbr, 0.f, 0.f);
-  // U^dagger: A' = conj A, B' = -B
-  float4* g = ci[p].rot[s];
-  g[0] = make_float4(far, far, -fai, -fai);
-  g[1] = make_float4(fai, fai, -fbr, -fbr);
-  g[2] = make_float4(-fbi, -fbi, fbi, fbi);
-  g[3] = make_float4(fbr, fbr, 0.f, 0.f);
-}
-
-// ----------------------------------------------------- split-form tables
-//
-// U = Rz(g) Ry(b) Rx(a) = Rz(phi1) Ry(vt) Rz(phi2) with A = e^{-i sig} c,
-// B = -e^{-i del} s, c = |A|, s = |B|, sig = (phi1 + phi2) / 2,
-// del = (phi1 - phi2) / 2.  Every state the split passes hold is the split
-// circuit's state times a "frame": a real scale and a sign (-1 on the 0 half)
-// for each qubit rotated in cotangent form since the last diagonal op.  Each
-// diagonal op removes the frame of its layer's rotations (forward) or restores
-// it (backward), so that the last pass leaves the exact final state.
-
-__global__ void split_rot_kernel(const float* theta, int total, SplitRot* out) {
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= total) return;
-  double ar, ai, br, bi;
-  su2_of(theta + (size_t)idx * 3, &ar, &ai, &br, &bi);
-  const double c = sqrt(ar * ar + ai * ai), s = sqrt(br * br + bi * bi);
-  const double sig = -atan2(ai, ar), del = -atan2(-bi, -br);
-  SplitRot r;
-  r.phi1 = sig + del;
-  r.phi2 = sig - del;
-  r.cot = s > c ? 1 : 0;
-  r.tau = r.cot ? c / s : s / c;
-  r.g = r.cot ? -1.0 / s : 1.0 / c;
-  r.k2 = r.g * r.g;
-  r.pad = 0;
-  out[idx] = r;
-}
-
-// Per layer: the frame of all its rotations, and per rotation the scale of
-// the backward sums.  At the sum of rotation j the backward state is
-// rho * gam * Z^m times the split circuit's (psi, lambda), where rho is the
-// product of k2 over the layer's rotations already un-applied and gam the
-// product of g over those still applied; the sums scale by (rho gam)^2, and
-// their X and Y parts flip sign when j itself is in cotangent form.
-__global__ void split_layer_kernel(const SplitRot* rot, const int* undo, int L, int n, SplitLayer* lay,
-                                   double* gfix) {
-  const int l = blockIdx.x * blockDim.x + threadIdx.x;
-  if (l >= L) return;
-  const SplitRot* r = rot + (size_t)l * n;
-  double gam = 1.0, rho = 1.0;
-  uint32_t m = 0;
-  for (int q = 0; q < n; ++q) {
-    gam *= r[q].g;
-    rho *= r[q].k2;
-    if (r[q].cot) m |= 1u << q;
-  }
-  lay[l].gam = gam;
-  lay[l].rho = rho;
-  lay[l].cot_mask = m;
-  lay[l].pad = 0;
-  double undone_k2 = 1.0, applied_g = gam;
-  for (int i = 0; i < n; ++i) {
-    const int q = undo[(size_t)l * n + i];
-    const double f = undone_k2 * applied_g;
-    const double sc = (r[q].cot ? -1.0 : 1.0) / (f * f);
-    gfix[((size_t)l * n + q) * 2 + 0] = sc;
-    gfix[((size_t)l * n + q) * 2 + 1] = r[q].phi1;
-    undone_k2 *= r[q].k2;
-    applied_g /= r[q].g;
-  }
-}
-
-// Factor of qubit q's bit b in the diagonal op after layer l (l = -1: before
-// layer 0): Rz(phi1 of layer l + phi2 of layer l + 1), times -1 on b = 1 when
-// q was rotated in cotangent form in layer l; conjugated for the backward.
-__device__ __forceinline__ double2 diag_factor(const SplitRot* rot, const SplitLayer* lay, int L, int n, int l, int q,
-                                               int b, bool bwd) {
-  const double w = (l >= 0 ? rot[(size_t)l * n + q].phi1 : 0.0) + (l + 1 < L ? rot[(size_t)(l + 1) * n + q].phi2 : 0.0);
-  double sn, cs;
-  sincos(0.5 * w, &sn, &cs);
-  double re = cs, im = b ? sn : -sn;
-  if (bwd) im = -im;
-  if (l >= 0 && b && ((lay[l].cot_mask >> q) & 1u)) re = -re, im = -im;
-  return make_double2(re, im);
-}
-
-__global__ void split_diag_kernel(const SplitRot* rot, const SplitLayer* lay, int L, int n, float2* dq_f,
-                                  float2* dq_b) {
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;  // ((l + 1) * n + q) * 2 + b
-  if (idx >= (L + 1) * n * 2) return;
-  const int b = idx & 1, q = (idx >> 1) % n, l = (idx >> 1) / n - 1;
-  const double2 f = diag_factor(rot, lay, L, n, l, q, b, false);
-  const double2 g = diag_factor(rot, lay, L, n, l, q, b, true);
-  dq_f[idx] = make_float2((float)f.x, (float)f.y);
-  dq_b[idx] = make_float2((float)g.x, (float)g.y);
-}
-
-// Per pass: rotation slots, the register tables of its diagonal ops, and the
-// restore scale.  Items per pass: kMaxSlots slots, kMaxDiag * kPos table
-// entries, one scale.
-constexpr int kSplitItems = kMaxSlots + kMaxDiag * kPos + 1;
-
-__global__ void split_pass_kernel(const DevPass* passes, int n_passes, const SplitRot* rot, const SplitLayer* lay,
-                                  int L, int n, CoefRegion* cf, CoefRegion* ci, float* rscale) {
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= n_passes * kSplitItems) return;
-  const int p = idx / kSplitItems, it = idx % kSplitItems;
-  const DevPass& P = passes[p];
-  if (it < kMaxSlots) {
-    if (it >= P.nslots) return;
-    const SplitRot r = rot[P.slot_lq[it]];
-    const float t = (float)r.tau;
-    // forward: p = tau in both forms; backward: -tau in tangent form
-    cf[p].rot[it][0] = make_float4(t, t, -t, -t);
-    cf[p].rot[it][1] = make_float4((float)r.cot, 0.f, 0.f, 0.f);
-    const float tb = r.cot ? t : -t;
-    ci[p].rot[it][0] = make_float4(tb, tb, -tb, -tb);
-    ci[p].rot[it][1] = make_float4((float)r.cot, 0.f, 0.f, 0.f);
-    return;
-  }
-  if (it == kSplitItems - 1) {
-    // backward checkpoint pass: the restored state takes the scale rho that
-    // the un-applied rotations between the pass's end and the next diagonal
-    // op have given the backward state
-    double rho = 1.0;
-    if (P.ckpt >= 0 && P.rs_layer >= 0)
-      for (int q = 0; q < n; ++q)
-        if ((P.rs_mask >> q) & 1u) rho *= rot[(size_t)P.rs_layer * n + q].k2;
-    rscale[p] = (float)rho;
-    return;
-  }
-  const int e = it - kMaxSlots, d = e / kPos, j = e % kPos;
-  int ph = -1, l = 0;
-  for (int o = 0; o < P.nops; ++o)
-    if (P.ops[o].kind == OP_DIAG && P.ops[o].d == d) ph = P.ops[o].a, l = P.ops[o].c;
-  if (ph < 0) return;
-  // the global scale: forward 1 / gam(l); backward gam(l) / rho(l + 1)
-  double fr = l >= 0 ? 1.0 / lay[l].gam : 1.0, fi = 0.0;
-  double br = l >= 0 ? lay[l].gam / (l + 1 < L ? lay[l + 1].rho : 1.0) : 0.0, bi = 0.0;
-  for (int k = 0; k < kRegBits; ++k) {
-    const int tb = ph == 0 ? k : ph == 1 ? 5 + k : (k < 2 ? 10 + k : k - 2);  // reg_tbit
-    const int q = P.tile_q[tb];
-    if (q < 0) continue;  // a batch-unit bit
-    const int b = (j >> k) & 1;
-    const double2 f = diag_factor(rot, lay, L, n, l, q, b, false);
-    const double2 g = diag_factor(rot, lay, L, n, l, q, b, true);
-    double t = fr * f.x - fi * f.y;
-    fi = fr * f.y + fi * f.x;
-    fr = t;
-    t = br * g.x - bi * g.y;
-    bi = br * g.y + bi * g.x;
-    br = t;
-  }
-  cf[p].diag[d][j] = make_float2((float)fr, (float)fi);
-  ci[p].diag[d][j] = make_float2((float)br, (float)bi);
-}
-
 // (cos, sin)(x/2) for the two samples of each forward unit.
 __global__ void prep_enc_kernel(const float* x, int B, int n, float2* enc) {
   const int U = (B + 1) / 2;
@@ -1997,30 +1808,6 @@ cudaError_t copy_pass_coef(int region, const CoefRegion* src, int nslots, int nd
   const size_t bytes = ndiag > 0 ? sizeof(CoefRegion) : (size_t)nslots * sizeof(src->rot[0]);
   if (bytes == 0) return cudaSuccess;
   return cudaMemcpyToSymbolAsync(c_reg, src, bytes, off, cudaMemcpyDeviceToDevice, s);
-}
-
-cudaError_t launch_prep_pass_coef(const DevPass* passes, int n_passes, const float* theta, CoefRegion* cf,
-                                  CoefRegion* ci, cudaStream_t s) {
-  const int tot = n_passes * kMaxSlots;
-  prep_pass_coef_kernel<<<(tot + 127) / 128, 128, 0, s>>>(passes, n_passes, theta, cf, ci);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_prep_split(const DevPass* passes, int n_passes, const float* theta, int L, int n,
-                              const int* undo, SplitRot* rot, SplitLayer* lay, double* gfix, float2* dq_f,
-                              float2* dq_b, CoefRegion* cf, CoefRegion* ci, float* rscale, cudaStream_t s) {
-  const int nr = L * n;
-  split_rot_kernel<<<(nr + 127) / 128, 128, 0, s>>>(theta, nr, rot);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  split_layer_kernel<<<(L + 127) / 128, 128, 0, s>>>(rot, undo, L, n, lay, gfix);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const int nd = (L + 1) * n * 2;
-  split_diag_kernel<<<(nd + 127) / 128, 128, 0, s>>>(rot, lay, L, n, dq_f, dq_b);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const int np = n_passes * kSplitItems;
-  split_pass_kernel<<<(np + 127) / 128, 128, 0, s>>>(passes, n_passes, rot, lay, L, n, cf, ci, rscale);
-  return cudaGetLastError();
 }
 
 cudaError_t launch_prep_enc(const float* x, int B, int n, float2* enc, cudaStream_t s) {

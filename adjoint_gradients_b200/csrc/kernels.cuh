@@ -105,6 +105,11 @@ cudaError_t launch_prep_pass_coef(const DevPass* passes, int n_passes, const flo
 cudaError_t launch_prep_split(const DevPass* passes, int n_passes, const float* theta, int L, int n,
                               const int* undo, SplitRot* rot, SplitLayer* lay, double* gfix, float2* dq_f,
                               float2* dq_b, CoefRegion* cf, CoefRegion* ci, float* rscale, cudaStream_t s);
+// fp64 mode (coef.cu): the same tables from an fp64 theta, with the per-qubit
+// diagonal factors dq_f / dq_b in fp64 and the restore scale of every pass.
+cudaError_t launch_prep_split64(const DevPass* passes, int n_passes, const double* theta, int L, int n,
+                                const int* undo, SplitRot* rot, SplitLayer* lay, double* gfix, double2* dq_f,
+                                double2* dq_b, double* rscale, cudaStream_t s);
 cudaError_t set_pass_smem_attr(size_t smem_thr, size_t smem_tma);
 // mode: 0 generic addressing (n < 5), 1 thread loads, 2 tensor copies.
 cudaError_t pass_occupancy(bool backward, int mode, size_t smem, int* blocks_per_sm);
@@ -194,6 +199,12 @@ struct Pass64Args {
   int reupload;           // every layer starts with the encoding Ry(x_q) again
   uint32_t nb[kMaxQubits];    // CZ neighbours of each qubit (qubit mask)
   uint32_t nbhi[kMaxQubits];  // CZ neighbours of each qubit above it
+  // split form (OP_RY / OP_DIAG passes; null otherwise)
+  int L;                      // layers
+  const SplitRot* srot;       // [L][n]
+  const SplitLayer* slay;     // [L]
+  const double2* dq;          // [L + 1][n][2] per-qubit diagonal factors of this direction
+  const double* rscale;       // backward checkpoint pass: scale of the restored state (null: 1)
 };
 
 size_t pass64_smem_bytes(bool backward, int tmax);
@@ -205,9 +216,10 @@ cudaError_t launch_bwd_init64(const double2* psi, double2* lam, const double* g,
 size_t expect64_partial_count(int B, int n);
 cudaError_t launch_expect64(const double2* psi, int B, int n, double* partial, double* E, unsigned* status,
                             cudaStream_t s);
+// gfix: split form, [L][n][2] (scale of the sums, phi1) per rotation; null otherwise.
 cudaError_t launch_grad_reduce64(const DevPass* passes, const int* slot_pass, const int* slot_index,
-                                 const double* partials, int grid, const double* theta, int L, int n, double* grad,
-                                 unsigned* status, cudaStream_t s);
+                                 const double* partials, int grid, const double* theta, const double* gfix, int L,
+                                 int n, double* grad, unsigned* status, cudaStream_t s);
 cudaError_t launch_loss_seed64(const double* E, const double* y, int B, double* g, double* loss, cudaStream_t s);
 // Pauli-sum observables in fp64: E[b] = <psi_b|O|psi_b> (partial: expect64_partial_count(B, n) doubles), and
 // lambda = g_b O psi (separate buffers).

@@ -135,7 +135,8 @@ def algorithmic_counts(ctx, w, B, f64=False, cnot_passes_per_layer=0):
     amp = B * N
     rots = w.n * w.L
     if ctx.split_form:  # one diagonal op per layer boundary (forward: also the one before layer 0)
-        fma_f = FMA_FWD_PER_RY * rots + FMA_FWD_PER_DIAG * (w.L + 1)
+        # fp64 mode keeps one sample per tile: its forward factor is not shared by two lanes (4 + 4)
+        fma_f = FMA_FWD_PER_RY * rots + (8 if f64 else FMA_FWD_PER_DIAG) * (w.L + 1)
         fma_b = FMA_BWD_PER_RY * rots + FMA_BWD_PER_DIAG * w.L
     else:
         fma_f, fma_b = FMA_FWD_PER_ROT * rots, FMA_BWD_PER_ROT * rots
