@@ -357,8 +357,11 @@ struct ReupPairCoef {
 #pragma unroll
     for (int k = 0; k < kRegBits; ++k)
       if ((j >> k) & 1) du += mu[k];
+    // padding units past the batch hold zero amplitudes; their angles are
+    // not written, so take unit 0's (any finite coefficients keep them zero)
+    const uint32_t u = unit + du < (uint32_t)a.U ? unit + du : 0u;
     float2 cs, sn;
-    enc_coef<BWD>(a, unit + du, q, &cs, &sn);
+    enc_coef<BWD>(a, u, q, &cs, &sn);
     return reup_coef<BWD>(c, cs, sn);
   }
 };
@@ -1072,11 +1075,13 @@ __host__ __device__ constexpr size_t pass_buf_bytes(bool tma) {
   return tma ? kLandBytes + kExch8Bytes : (size_t)kSmemSlots * sizeof(float4);
 }
 
-// Register budget: tensor-copy passes and the one-launch passes of
-// single-tile circuits (split form, n <= 12, at most a few hundred tiles a
-// launch) run two blocks per SM (up to 255 registers); the others three.
+// Register budget: the split-form passes (tensor copies, and the one-launch
+// passes of single-tile circuits) may use up to 255 registers (two blocks per
+// SM); the fused-SU(2) and re-uploading forms are held to 168 (three blocks'
+// worth), where their code does not spill, although the shared memory of a
+// tensor-copy block still allows only two per SM.
 template <bool BWD, int MODE, int V, int RE>
-__global__ void __launch_bounds__(kThreads, (MODE == 2 || RE == 3) ? kBlocksPerSmTma : kBlocksPerSm)
+__global__ void __launch_bounds__(kThreads, RE == 3 ? kBlocksPerSmTma : kBlocksPerSm)
     pass_kernel(const PassArgs a, const __grid_constant__ DevPass P, const __grid_constant__ CUtensorMap tm0,
                 const __grid_constant__ CUtensorMap tm1) {
   constexpr bool SLOW = MODE == 0;
