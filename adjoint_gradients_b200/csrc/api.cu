@@ -112,6 +112,12 @@ struct qml_ctx {
   Plan plan1;
   std::vector<DevPass> sub[4];
   bool sub_uploaded = false;
+  // Fused CNOT layers (fp32, two qubit sets, a list whose map factors as
+  // M2 M1, see plan.hpp): plan and dpass are then the fused schedule, whose
+  // passes apply M1 and M2 inside their tiles; re-uploading still takes the
+  // one-layer schedules above.
+  bool cnot_fused = false;
+  CnotLayers cnot_map{};  // M1, M2 of the fused schedule
   bool f64 = false;       // fp64 compute mode (qml_create_f64)
   // host-side fault injection for tests of the error paths (QML_FAULT at create)
   enum Fault { FAULT_NONE, FAULT_ALLOC, FAULT_CKPT, FAULT_NAN } fault = FAULT_NONE;
@@ -296,6 +302,9 @@ T* at(qml_ctx* c, size_t off) {
 // (re-uploading folds per-sample encodings into the rotations; CNOT layers
 // run as one-layer schedules).
 bool use_split(const qml_ctx* c) { return !c->f64 && !c->reupload && !c->cnot; }
+// CNOT entanglers through the fused schedule (the generic pass loop), or the
+// one-layer schedules with a gather per layer
+bool cnot_fused_now(const qml_ctx* c) { return c->cnot && c->cnot_fused && !c->reupload && !c->f64; }
 // fp64 contexts: the same rule
 bool use_split64(const qml_ctx* c) { return c->f64 && !c->reupload && !c->cnot; }
 
@@ -615,7 +624,7 @@ cudaError_t prep_coefficients(qml_ctx* c, const float* theta, cudaStream_t s) {
 
 qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, float2* psi,
                        float* expect, cudaStream_t s) {
-  if (c->cnot) return run_forward_cnot(c, theta, x, B, psi, expect, s);
+  if (c->cnot && !cnot_fused_now(c)) return run_forward_cnot(c, theta, x, B, psi, expect, s);
   const int n = c->cfg.n_qubits;
   const bool split = use_split(c);
   const std::vector<DevPass>& passes = fp32_passes(c);
@@ -690,7 +699,7 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
 
 qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, float2* psi,
                         float2* lam, const float* g, float* grad, cudaStream_t s) {
-  if (c->cnot) return run_backward_cnot(c, theta, x, B, psi, lam, g, grad, s);
+  if (c->cnot && !cnot_fused_now(c)) return run_backward_cnot(c, theta, x, B, psi, lam, g, grad, s);
   const int n = c->cfg.n_qubits, L = c->cfg.n_layers;
   const bool split = use_split(c);
   const std::vector<DevPass>& passes = fp32_passes(c);
@@ -1304,6 +1313,26 @@ qml_status qml_set_observable(qml_ctx* c, int n_terms, const char* paulis, const
   return QML_OK;
 }
 
+// The schedule, its device copies and the workspace layout belong together:
+// after a change of schedule the caller sets the workspace again.
+static void drop_workspace(qml_ctx* c) {
+  c->ws = nullptr;
+  c->ws_bytes = 0;
+  c->maps.clear();
+}
+
+// Back to the schedule of qml_create (CZ entanglers, or CNOT lists through
+// the one-layer schedules).
+static void restore_default_plan(qml_ctx* c) {
+  Plan p;
+  make_plan(c->cfg.n_qubits, c->cfg.n_layers, c->cfg.ckpt_block, &p);  // succeeded in qml_create
+  c->plan = p;
+  flatten_plan(p, &c->dpass);
+  set_pass_entangler(p, c->bonds, &c->dpass);
+  c->cnot_fused = false;
+  if (c->ws) drop_workspace(c);
+}
+
 qml_status qml_set_entangler(qml_ctx* c, int n_bonds, const int* bonds) {
   if (!c || n_bonds < 0 || n_bonds > QML_MAX_BONDS || (n_bonds > 0 && !bonds)) return QML_ERR_INVALID_ARG;
   const int n = c->cfg.n_qubits;
@@ -1315,6 +1344,7 @@ qml_status qml_set_entangler(qml_ctx* c, int n_bonds, const int* bonds) {
   }
   c->bonds = b;
   set_bond_masks(c);
+  if (c->cnot_fused) restore_default_plan(c);
   set_pass_entangler(c->plan, c->bonds, &c->dpass);
   set_pass_entangler(c->plan, c->bonds, &c->dpass_split);
   c->cnot = false;
@@ -1368,6 +1398,23 @@ qml_status qml_set_entangler_cnot(qml_ctx* c, int n_pairs, const int* pairs) {
   c->plan1 = p1;
   c->cnot_pairs = v;
   c->cnot = true;
+  // fused schedule (fp32): M1 and M2 of every layer inside the rotation passes
+  bool fused = false;
+  if (!c->f64) {
+    CnotLayers cl;
+    Plan fp;
+    if (factor_cnot_layer(n, v, &cl) && make_plan(n, c->cfg.n_layers, c->cfg.ckpt_block, &fp, &cl).empty()) {
+      std::vector<DevPass> dp;
+      flatten_plan(fp, &dp);
+      set_pass_entangler(fp, Bonds{}, &dp);
+      c->plan = fp;
+      c->dpass = dp;
+      c->cnot_fused = fused = true;
+      c->cnot_map = cl;
+    }
+  }
+  if (!fused && c->cnot_fused) restore_default_plan(c);
+  if (c->ws) drop_workspace(c);  // the schedule's device copies and the layout change with it
   compute_layout(c);  // the gathers need a second state buffer in the workspace
   return QML_OK;
 }
@@ -1383,6 +1430,9 @@ int qml_debug_entangler_map(const qml_ctx* c, int* out, int cap) {
   for (int q = 0; q < n; ++q) v.push_back((int)c->cnot_fwd_q.col[q]);  // M^-1
   for (int a = 0; a < n; ++a) v.push_back((int)c->cnot_bwd.col[a]);    // M on working-state addresses
   for (int a = 0; a < n; ++a) v.push_back((int)c->cnot_fwd.col[a]);
+  v.push_back(c->cnot_fused ? 1 : 0);  // then M1 and M2 of the fused schedule (qubit bits)
+  for (int g = 0; g < 2; ++g)
+    for (int q = 0; q < n; ++q) v.push_back(c->cnot_fused ? (int)c->cnot_map.fwd[g][q] : 0);
   for (int i = 0; i < (int)v.size() && out && i < cap; ++i) out[i] = v[i];
   return (int)v.size();
 }

@@ -40,12 +40,23 @@ constexpr int kMaxSlots = kMaxLayersPerPass * kTileBits;  // rotations per pass
 constexpr int kCoefRegions = 16;      // per-context regions of constant memory
 constexpr int kMaxDiag = kMaxLayersPerPass + 1;  // diagonal ops per pass (split rotations)
 
+// Exchange slot of tile position x in a permuted exchange: linear over GF(2)
+// (so a gather map and the slot map compose into one set of columns) and
+// conflict-free for the 8-byte accesses of every layout's unpermuted side:
+// the lanes of a half warp vary tile bits {5,6,7,8}, {0,1,2,3}, {10,11,0,1}
+// or {5,6,7,3}, which this map sends to four independent low slot bits.
+constexpr uint32_t perm_slot(uint32_t x) { return x ^ ((x >> 5) & 15u) ^ ((x >> 8) & 12u); }
+
 // OP_RY and OP_DIAG are the split form of OP_ROT and OP_CZ: every fused
 // rotation U = Rz(g) Ry(b) Rx(a) is rewritten exactly as Rz(phi1) Ry(vt)
 // Rz(phi2).  The Rz factors of consecutive layers and the layer's CZ bonds
 // are all diagonal and meet between the layers, so each layer boundary is one
 // diagonal op, and each rotation is a real Ry applied in tangent form.
-enum : int { OP_EXCH = 1, OP_ROT = 2, OP_CZ = 3, OP_GEN = 4, OP_RY = 5, OP_DIAG = 6 };
+// OP_PERM: the part of a layer's CNOT list that changes only the bits of
+// the pass's tile (fused CNOT layers, see plan.hpp), applied as a gather of
+// the tile's positions: while reading the copied tile, or in a layout
+// exchange whose reads are permuted.
+enum : int { OP_EXCH = 1, OP_ROT = 2, OP_CZ = 3, OP_GEN = 4, OP_RY = 5, OP_DIAG = 6, OP_PERM = 7 };
 
 // Tensor-copy (TMA) view of a pass's tile, used when n > 12: the state
 // [B][2^n] (working-state address order) is seen as a rank-5 tensor whose
@@ -65,6 +76,7 @@ enum : int { TD_PAD = 0, TD_IN = 1, TD_OUT = 2, TD_SAMPLE = 3, TD_OUT_SAMPLE = 4
 // OP_RY  : as OP_ROT (split form)
 // OP_DIAG: a = phase, c = layer l (the diagonal between layers l and l+1;
 //          -1: the one before layer 0), d = its table in the pass (0..kMaxDiag-1)
+// OP_PERM: a = from phase, b = to phase, c = factor (0: M1, 1: M2), d = layer
 struct DevOp {
   int kind, a, b, c, d;
 };
@@ -92,6 +104,16 @@ struct DevPass {
   uint32_t out_abit[kMaxOut];     // out-of-tile qubit -> its address bit
   uint32_t cz_reg[kPhases];  // bit j: entangler parity of the register part of position j
   uint32_t cz_nb[kPhases][kRegBits];  // CZ neighbours (qubit mask) of each register bit's qubit
+  // OP_PERM (at most one per pass).  In direction dir (0 forward, 1
+  // backward) position y of the tile after the op holds the position
+  // G y + G_o o of the tile before it (o: the tile's out-of-tile bits; GF(2)
+  // products, i.e. the xor of the columns of the set bits).  perm_at[dir]:
+  // 0 none, 1 applied while reading the copied tile (columns as element
+  // offsets in the landing buffer), 2 in the op's layout exchange (columns
+  // as exchange slots, perm_slot).
+  int perm_at[2];
+  uint16_t pcol[2][kTileBits];
+  uint16_t pcol_o[2][kMaxOut];
   int ndiag;                 // OP_DIAG ops in the pass (split form)
   int rs_layer;              // split form, checkpoint pass: layer of the next diagonal op after the pass
   uint32_t rs_mask;          // ... and the qubits it rotates between the pass's end and that op

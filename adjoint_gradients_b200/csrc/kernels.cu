@@ -586,6 +586,70 @@ __device__ __forceinline__ void exchange8(int x, int y, float2 (&re)[kPos], floa
   }
 }
 
+// Fused CNOT layers: a layout exchange whose reads are permuted.  Each
+// thread writes its positions (layout X) at perm_slot of their tile position,
+// then reads for its position y (layout Y) the slot G y + G_o o of the
+// direction's gather map, given as columns already in slot space: cy is the
+// part of the thread bits and the out-of-tile bits, dc[k] the column of
+// register bit k (perm_slot is linear, so the slot of a gathered position is
+// the xor of these).
+template <int P>
+__host__ __device__ constexpr uint32_t reg_pattern(int j) {
+  uint32_t t = 0;
+  for (int k = 0; k < kRegBits; ++k)
+    if ((j >> k) & 1) t |= 1u << reg_tbit<P>(k);
+  return t;
+}
+
+template <int P, int V>
+__device__ __forceinline__ uint32_t thr_pattern(uint32_t tid) {
+  uint32_t t = 0;
+#pragma unroll
+  for (int m = 0; m < kThrBits; ++m) t |= ((tid >> m) & 1u) << thr_tbit<P, V>(m);
+  return t;
+}
+
+template <int X, int Y, int V>
+__device__ __forceinline__ void exchange8p_t(float2 (&re)[kPos], float2 (&im)[kPos], float2* ex, uint32_t tid,
+                                             const DevPass& Pp, int dir, uint32_t co) {
+  const uint32_t sx = perm_slot(thr_pattern<X, V>(tid));
+  uint32_t cy = co;
+#pragma unroll
+  for (int m = 0; m < kThrBits; ++m)
+    if ((tid >> m) & 1u) cy ^= Pp.pcol[dir][thr_tbit<Y, V>(m)];
+  uint32_t dc[kRegBits];
+#pragma unroll
+  for (int k = 0; k < kRegBits; ++k) dc[k] = Pp.pcol[dir][reg_tbit<Y>(k)];
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kPos; ++j) ex[sx ^ perm_slot(reg_pattern<X>(j))] = re[j];
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kPos; ++j) re[j] = ex[cy ^ REG_COMBINE(dc, j, ^=)];
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kPos; ++j) ex[sx ^ perm_slot(reg_pattern<X>(j))] = im[j];
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kPos; ++j) im[j] = ex[cy ^ REG_COMBINE(dc, j, ^=)];
+}
+
+template <int V>
+__device__ __forceinline__ void exchange8p(int x, int y, float2 (&re)[kPos], float2 (&im)[kPos], float2* ex,
+                                           uint32_t tid, const DevPass& Pp, int dir, uint32_t co) {
+  switch (x * 3 + y) {
+    case 0: exchange8p_t<0, 0, V>(re, im, ex, tid, Pp, dir, co); break;
+    case 1: exchange8p_t<0, 1, V>(re, im, ex, tid, Pp, dir, co); break;
+    case 2: exchange8p_t<0, 2, V>(re, im, ex, tid, Pp, dir, co); break;
+    case 3: exchange8p_t<1, 0, V>(re, im, ex, tid, Pp, dir, co); break;
+    case 4: exchange8p_t<1, 1, V>(re, im, ex, tid, Pp, dir, co); break;
+    case 5: exchange8p_t<1, 2, V>(re, im, ex, tid, Pp, dir, co); break;
+    case 6: exchange8p_t<2, 0, V>(re, im, ex, tid, Pp, dir, co); break;
+    case 7: exchange8p_t<2, 1, V>(re, im, ex, tid, Pp, dir, co); break;
+    default: exchange8p_t<2, 2, V>(re, im, ex, tid, Pp, dir, co); break;
+  }
+}
+
 // CZ on every bond (a, b) of the entangler: sign (-1)^{S(i)}, S(i) = sum over
 // bonds of i_a i_b, of the global index i.  Split i = T | O | R (thread bits,
 // out-of-tile bits, register bits; disjoint).  S is a quadratic form, so
@@ -906,6 +970,36 @@ __device__ __forceinline__ void load_tma(int phase, float2 (&re)[kPos], float2 (
   else load_tma_t<1, V>(re, im, buf, Pp, tid);
 }
 
+// Fused CNOT layers: registers of layout P gathered from the copied tile
+// through the direction's map (columns as landing-buffer offsets: the offset
+// of a tile position is a bit permutation of it, so the offset of a gathered
+// position is the xor of the columns of its set bits, co for the out-of-tile
+// bits).
+template <int P, int V>
+__device__ __forceinline__ void load_tma_perm_t(float2 (&re)[kPos], float2 (&im)[kPos], const float2* buf,
+                                                const DevPass& Pp, int dir, uint32_t co, uint32_t tid) {
+  uint32_t s0 = co;
+#pragma unroll
+  for (int m = 0; m < kThrBits; ++m)
+    if ((tid >> m) & 1u) s0 ^= Pp.pcol[dir][thr_tbit<P, V>(m)];
+  uint32_t r[kRegBits];
+#pragma unroll
+  for (int k = 0; k < kRegBits; ++k) r[k] = Pp.pcol[dir][reg_tbit<P>(k)];
+#pragma unroll
+  for (int j = 0; j < kPos; ++j) {
+    const uint32_t off = s0 ^ REG_COMBINE(r, j, ^=);
+    re[j] = buf[off];
+    im[j] = buf[off + kTilePos];
+  }
+}
+
+template <int V>
+__device__ __forceinline__ void load_tma_perm(int phase, float2 (&re)[kPos], float2 (&im)[kPos], const float2* buf,
+                                              const DevPass& Pp, int dir, uint32_t co, uint32_t tid) {
+  if (phase == 0) load_tma_perm_t<0, V>(re, im, buf, Pp, dir, co, tid);
+  else load_tma_perm_t<1, V>(re, im, buf, Pp, dir, co, tid);
+}
+
 // Out-of-tile qubit bits and first batch unit of tile t.
 // (out-of-tile bits as qubit bits and as working-state address bits)
 __device__ __forceinline__ void tile_base(const DevPass& P, int t, uint32_t* base_q, uint32_t* base_a,
@@ -1076,12 +1170,13 @@ __host__ __device__ constexpr size_t pass_buf_bytes(bool tma) {
 }
 
 // Register budget: the split-form passes (tensor copies, and the one-launch
-// passes of single-tile circuits) may use up to 255 registers (two blocks per
-// SM); the fused-SU(2) and re-uploading forms are held to 168 (three blocks'
-// worth), where their code does not spill, although the shared memory of a
-// tensor-copy block still allows only two per SM.
+// passes of single-tile circuits) and the fused-SU(2) tensor-copy passes
+// (CNOT entanglers, with their permuted exchanges) may use up to 255
+// registers (two blocks per SM); the re-uploading forms are held to 168
+// (three blocks' worth), where their code does not spill, although the
+// shared memory of a tensor-copy block still allows only two per SM.
 template <bool BWD, int MODE, int V, int RE>
-__global__ void __launch_bounds__(kThreads, RE == 3 ? kBlocksPerSmTma : kBlocksPerSm)
+__global__ void __launch_bounds__(kThreads, (RE == 3 || (RE == 0 && MODE == 2)) ? kBlocksPerSmTma : kBlocksPerSm)
     pass_kernel(const PassArgs a, const __grid_constant__ DevPass P, const __grid_constant__ CUtensorMap tm0,
                 const __grid_constant__ CUtensorMap tm1) {
   constexpr bool SLOW = MODE == 0;
@@ -1091,6 +1186,8 @@ __global__ void __launch_bounds__(kThreads, RE == 3 ? kBlocksPerSmTma : kBlocksP
   // split passes of circuits that fit one tile (n <= 12): every pass in one
   // launch, coefficients from the workspace (see MULTI below)
   constexpr bool MULTI = SPLIT && !TMA;
+  // fused CNOT layers (OP_PERM): fused-SU(2) passes loaded by tensor copies
+  constexpr bool CNOTF = TMA && RE == 0;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   float4* tile = reinterpret_cast<float4*>(smem_raw);  // MODE 2: the landing buffer
   float2* ex8 = reinterpret_cast<float2*>(smem_raw + kLandBytes);  // MODE 2: the exchange buffer
@@ -1144,6 +1241,7 @@ __global__ void __launch_bounds__(kThreads, RE == 3 ? kBlocksPerSmTma : kBlocksP
   const int mem_ph = BWD ? P.store_phase : P.load_phase;
   const int pf_at = BWD ? P.pf_bwd : P.pf_fwd;  // op index after which to prefetch (-1: after the load)
   bool have_pf = false;
+  uint32_t pco = 0;  // fused CNOT layers: the out-of-tile part of the tile's gather
 
   // The ops of one pass on the registers, forward order (PP: the pass, C: its
   // coefficients; the layout is P's, the same for every pass of a launch).
@@ -1196,6 +1294,9 @@ __global__ void __launch_bounds__(kThreads, RE == 3 ? kBlocksPerSmTma : kBlocksP
         }
       } else if (op.kind == OP_CZ) {
         cz_op<V>(op.a, re, im, *bc, P, tid, base_q, s_o);
+      } else if (op.kind == OP_PERM) {
+        if constexpr (CNOTF)
+          if (PP.perm_at[0] == 2) exchange8p<V>(op.a, op.b, re, im, ex8, tid, PP, 0, pco);
       }
       if (pf_next && oi == pf_at) prefetch_next();
     }
@@ -1271,6 +1372,9 @@ __global__ void __launch_bounds__(kThreads, RE == 3 ? kBlocksPerSmTma : kBlocksP
         }
       } else if (op.kind == OP_CZ) {
         cz_op<V>(op.a, re, im, *bc, P, tid, base_q, s_o);
+      } else if (op.kind == OP_PERM) {
+        if constexpr (CNOTF)
+          if (PP.perm_at[1] == 2) exchange8p<V>(op.b, op.a, re, im, ex8, tid, PP, 1, pco);
       }
       if (pf_next && oi == pf_at) prefetch_next();
     }
@@ -1341,6 +1445,14 @@ __global__ void __launch_bounds__(kThreads, RE == 3 ? kBlocksPerSmTma : kBlocksP
     uint32_t base_q, base_a, unit_base;
     tile_base(P, t, &base_q, &base_a, &unit_base);
     const uint32_t s_o = bond_parity(base_q, a);  // entangler terms of the out-of-tile bits
+    if constexpr (CNOTF) {
+      if (P.perm_at[BWD]) {
+        const uint32_t o = (uint32_t)t & ((1u << P.n_out) - 1u);
+        pco = 0;
+        for (int k = 0; k < P.n_out; ++k)
+          if ((o >> k) & 1u) pco ^= P.pcol_o[BWD][k];
+      }
+    }
     const int tn = t + (int)gridDim.x;
     const bool pf_next = can_pf && tn < a.n_tiles;
     auto prefetch_next = [&]() {
@@ -1371,7 +1483,8 @@ __global__ void __launch_bounds__(kThreads, RE == 3 ? kBlocksPerSmTma : kBlocksP
         if (mem_ph == 0) restore_tma_t<0, V>(a, *bc, P, tid, base_q, unit_base, tb, P.ckpt, rs);
         else restore_tma_t<1, V>(a, *bc, P, tid, base_q, unit_base, tb, P.ckpt, rs);
       }
-      load_tma<V>(mem_ph, re, im, tb, P, tid);
+      if (CNOTF && P.perm_at[BWD] == 1) load_tma_perm<V>(mem_ph, re, im, tb, P, BWD ? 1 : 0, pco, tid);
+      else load_tma<V>(mem_ph, re, im, tb, P, tid);
       __syncthreads();  // every thread has its positions: the landing buffer is free
       if (pf_next && tid == 0) tma_load_tile(&tm0, &tm1, bc->tma_sel, bc->tma_c, tile_s, mbar);
     }

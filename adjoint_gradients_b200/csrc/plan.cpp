@@ -6,11 +6,12 @@
 namespace qml {
 namespace {
 
-enum TaskKind { T_GEN, T_ROT, T_CZ };
+enum TaskKind { T_GEN, T_ROT, T_CZ, T_PERM };
 struct Task {
   TaskKind kind;
   int layer;
   int set;
+  int group;  // T_PERM: factor of the layer's CNOT map (0: M1, 1: M2)
 };
 
 // Tile bit addressed by register-index bit k in phase p (mirrors the kernels).
@@ -75,9 +76,146 @@ void set_tma_view(int n, const HostPass& ps, const std::vector<int>& addr_of, De
   d->tma = 1;
 }
 
+// Qubit sets rotated together: the whole register for n <= 12, else
+// ceil(n / 10) runs of consecutive qubits of near-equal size.
+std::vector<std::vector<int>> qubit_sets(int n) {
+  std::vector<std::vector<int>> sets;
+  if (n <= kTileBits) {
+    sets.push_back({});
+    for (int q = 0; q < n; ++q) sets[0].push_back(q);
+    return sets;
+  }
+  const int s = (n + kMaxSet - 1) / kMaxSet;
+  const int base = n / s, extra = n % s;
+  int q = 0;
+  for (int i = 0; i < s; ++i) {
+    const int sz = base + (i < extra ? 1 : 0);
+    std::vector<int> set;
+    for (int k = 0; k < sz; ++k) set.push_back(q++);
+    sets.push_back(set);
+  }
+  return sets;
+}
+
+// GF(2) linear maps on qubit bits, stored as columns (the image of each
+// single qubit as a qubit mask).
+uint32_t gf2_apply(const uint32_t* cols, int n, uint32_t x) {
+  uint32_t y = 0;
+  for (int q = 0; q < n; ++q)
+    if ((x >> q) & 1u) y ^= cols[q];
+  return y;
+}
+
+// Inverse by Gauss-Jordan elimination on the rows; false if singular.
+bool gf2_inverse(const uint32_t* cols, int n, uint32_t* inv) {
+  // row r of the matrix: bit c = bit r of column c; augmented with identity
+  std::vector<uint32_t> row(n), aug(n);
+  for (int r = 0; r < n; ++r) {
+    row[r] = 0;
+    for (int c = 0; c < n; ++c)
+      if ((cols[c] >> r) & 1u) row[r] |= 1u << c;
+    aug[r] = 1u << r;
+  }
+  for (int c = 0; c < n; ++c) {
+    int piv = -1;
+    for (int r = c; r < n; ++r)
+      if ((row[r] >> c) & 1u) {
+        piv = r;
+        break;
+      }
+    if (piv < 0) return false;
+    std::swap(row[c], row[piv]);
+    std::swap(aug[c], aug[piv]);
+    for (int r = 0; r < n; ++r)
+      if (r != c && ((row[r] >> c) & 1u)) row[r] ^= row[c], aug[r] ^= aug[c];
+  }
+  // rows of the inverse are aug; back to columns
+  for (int c = 0; c < n; ++c) {
+    inv[c] = 0;
+    for (int r = 0; r < n; ++r)
+      if ((aug[r] >> c) & 1u) inv[c] |= 1u << r;
+  }
+  return true;
+}
+
+// Fused CNOT layers: the gather columns of the pass's OP_PERM in both
+// directions (see DevPass::perm_at).  The forward gathers through M_g^-1,
+// the backward through M_g.  M1 (M2) changes only the bits of the first
+// (second) set, all inside this pass's tile, and reads the others: in-tile
+// columns stay in the tile, an out-of-tile qubit's column is itself plus
+// in-tile bits.
+void set_pass_perm(const Plan& p, const HostPass& ps, const std::vector<HostOp>& ops, DevPass* d) {
+  d->perm_at[0] = d->perm_at[1] = 0;
+  for (int dir = 0; dir < 2; ++dir) {
+    for (int b = 0; b < kTileBits; ++b) d->pcol[dir][b] = 0;
+    for (int k = 0; k < kMaxOut; ++k) d->pcol_o[dir][k] = 0;
+  }
+  int oi = -1;
+  for (int o = 0; o < (int)ops.size(); ++o)
+    if (ops[o].kind == OP_PERM) oi = o;
+  if (oi < 0 || !p.cnot || !d->tma) return;
+  const HostOp& op = ops[oi];
+  const int g = op.c;
+  auto tile_pattern = [&](uint32_t qmask) {
+    uint32_t t = 0;
+    for (int b = 0; b < kTileBits; ++b)
+      if (ps.tile_q[b] >= 0 && ((qmask >> ps.tile_q[b]) & 1u)) t |= 1u << b;
+    return t;
+  };
+  auto offset = [&](uint32_t t) {  // element offset in the copied tile (a bit permutation of t)
+    uint32_t e = 0;
+    for (int b = 0; b < kTileBits; ++b)
+      if ((t >> b) & 1u) e += (uint32_t)d->sstride[b];
+    return e;
+  };
+  d->perm_at[0] = (oi == 0 && op.a == op.b && op.a == ps.load_phase && !ps.gen) ? 1 : 2;
+  d->perm_at[1] = (oi + 1 == (int)ops.size() && op.a == op.b && op.a == ps.store_phase) ? 1 : 2;
+  for (int dir = 0; dir < 2; ++dir) {
+    const uint32_t* G = dir == 0 ? p.cl.inv[g] : p.cl.fwd[g];
+    auto space = [&](uint32_t t) { return (uint16_t)(d->perm_at[dir] == 1 ? offset(t) : perm_slot(t)); };
+    for (int b = 0; b < kTileBits; ++b)
+      if (ps.tile_q[b] >= 0) d->pcol[dir][b] = space(tile_pattern(G[ps.tile_q[b]]));
+    for (int k = 0; k < (int)ps.out_q.size(); ++k) d->pcol_o[dir][k] = space(tile_pattern(G[ps.out_q[k]]));
+  }
+}
+
 }  // namespace
 
-std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
+void cnot_list_map(int n, const std::vector<std::pair<int, int>>& pairs, uint32_t* fwd, uint32_t* inv) {
+  for (int q = 0; q < n; ++q) {
+    uint32_t f = 1u << q, b = 1u << q;
+    for (const auto& e : pairs) f ^= ((f >> e.first) & 1u) << e.second;
+    for (auto it = pairs.rbegin(); it != pairs.rend(); ++it) b ^= ((b >> it->first) & 1u) << it->second;
+    fwd[q] = f;
+    inv[q] = b;
+  }
+}
+
+bool factor_cnot_layer(int n, const std::vector<std::pair<int, int>>& pairs, CnotLayers* out) {
+  const auto sets = qubit_sets(n);
+  if (sets.size() != 2) return false;
+  uint32_t mA = 0;
+  for (int q : sets[0]) mA |= 1u << q;
+  const uint32_t mB = ((n >= 32) ? ~0u : ((1u << n) - 1u)) & ~mA;
+  uint32_t M[kMaxQubits], Mi[kMaxQubits], M1[kMaxQubits], M1i[kMaxQubits], M2[kMaxQubits], M2i[kMaxQubits];
+  cnot_list_map(n, pairs, M, Mi);
+  // M1: A's bits as M leaves them, B's bits unchanged
+  for (int q = 0; q < n; ++q) M1[q] = (M[q] & mA) | ((1u << q) & mB);
+  if (!gf2_inverse(M1, n, M1i)) return false;
+  for (int q = 0; q < n; ++q) {
+    M2[q] = gf2_apply(M, n, M1i[q]);     // M M1^-1
+    M2i[q] = gf2_apply(M1, n, Mi[q]);    // M1 M^-1
+    if ((M2[q] & mA) != ((1u << q) & mA)) return false;  // M2 must leave A's bits alone
+  }
+  *out = CnotLayers{};
+  for (int q = 0; q < n; ++q) {
+    out->fwd[0][q] = M1[q], out->inv[0][q] = M1i[q];
+    out->fwd[1][q] = M2[q], out->inv[1][q] = M2i[q];
+  }
+  return true;
+}
+
+std::string make_plan(int n, int L, int ckpt_block, Plan* out, const CnotLayers* cl) {
   if (n < 1 || n > 30) return "n_qubits must be in [1, 30]";
   if (L < 1 || L > 100000) return "n_layers must be in [1, 100000]";
   if (ckpt_block < 0) return "ckpt_block must be >= 0";
@@ -86,23 +224,12 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
   p.L = L;
   p.ckpt_block = ckpt_block;
 
-  // ---- qubit sets rotated together
-  if (n <= kTileBits) {
-    p.sets.push_back({});
-    for (int q = 0; q < n; ++q) p.sets[0].push_back(q);
-  } else {
-    const int s = (n + kMaxSet - 1) / kMaxSet;
-    const int base = n / s, extra = n % s;
-    int q = 0;
-    for (int i = 0; i < s; ++i) {
-      const int sz = base + (i < extra ? 1 : 0);
-      std::vector<int> set;
-      for (int k = 0; k < sz; ++k) set.push_back(q++);
-      p.sets.push_back(set);
-    }
-  }
+  p.sets = qubit_sets(n);
   p.n_sets = (int)p.sets.size();
   const int S = p.n_sets;
+  if (cl && S != 2) return "fused CNOT layers need two qubit sets";
+  p.cnot = cl != nullptr;
+  if (cl) p.cl = *cl;
   // ---- working-state address bits: identity, except that plans with three
   // or more sets move the second set's first two qubits to address bits 2
   // and 3 (every set's tile then covers address bits 0-3 or 0-2: HBM runs of
@@ -122,13 +249,23 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
   }
   p.n_ckpt = (ckpt_block > 0) ? (L + ckpt_block - 1) / ckpt_block - 1 : 0;
 
-  // ---- task list: encode, then per layer the sets in boustrophedon order, then CZ
+  // ---- task list: encode, then per layer the sets in boustrophedon order, then CZ;
+  // fused CNOT layers: per layer [M2 of the layer before] the second set, the
+  // first set, M1; at the end the last layer's M2
   std::vector<Task> tasks;
-  tasks.push_back({T_GEN, -1, -1});
+  tasks.push_back({T_GEN, -1, -1, 0});
   for (int l = 0; l < L; ++l) {
-    for (int i = 0; i < S; ++i) tasks.push_back({T_ROT, l, (l % 2 == 0) ? i : S - 1 - i});
-    tasks.push_back({T_CZ, l, -1});
+    if (cl) {
+      if (l > 0) tasks.push_back({T_PERM, l - 1, 1, 1});
+      tasks.push_back({T_ROT, l, 1, 0});
+      tasks.push_back({T_ROT, l, 0, 0});
+      tasks.push_back({T_PERM, l, 0, 0});
+      continue;
+    }
+    for (int i = 0; i < S; ++i) tasks.push_back({T_ROT, l, (l % 2 == 0) ? i : S - 1 - i, 0});
+    tasks.push_back({T_CZ, l, -1, 0});
   }
+  if (cl) tasks.push_back({T_PERM, L - 1, 1, 1});
 
   // ---- group tasks into passes: a new pass starts when the rotated set
   // changes, when a single-tile pass is full, or after a checkpoint boundary
@@ -142,17 +279,17 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
   std::vector<Proto> protos(1);
   for (const Task& tk : tasks) {
     Proto* cur = &protos.back();
-    if (tk.kind == T_ROT) {
+    if (tk.kind == T_ROT || tk.kind == T_PERM) {
       bool need_new = (cur->set >= 0 && cur->set != tk.set) || (S == 1 && cur->rots >= kMaxLayersPerPass);
       if (need_new) {
         protos.emplace_back();
         cur = &protos.back();
       }
       cur->set = tk.set;
-      cur->rots++;
+      if (tk.kind == T_ROT) cur->rots++;
     }
     cur->t.push_back(tk);
-    if (tk.kind == T_CZ && ckpt_block > 0) {
+    if (((tk.kind == T_CZ && !cl) || (tk.kind == T_PERM && tk.group == 0)) && ckpt_block > 0) {
       const int l = tk.layer;
       if ((l + 1) % ckpt_block == 0 && l + 1 < L) {
         cur->ckpt = (l + 1) / ckpt_block - 1;  // slot m-1 holds the state after layer m*b-1
@@ -285,6 +422,12 @@ std::string make_plan(int n, int L, int ckpt_block, Plan* out) {
         }
       } else if (tk.kind == T_CZ) {
         ps.ops.push_back({OP_CZ, cur, 0, tk.layer, 0});
+      } else if (tk.kind == T_PERM) {
+        // M1 ends the pass: its permuted exchange goes to the memory phase;
+        // M2 starts one, in the phase it is in (the memory phase)
+        const int to = tk.group == 0 ? mem : cur;
+        ps.ops.push_back({OP_PERM, cur, to, tk.group, tk.layer});
+        cur = to;
       }
     }
     if (cur != mem) ps.ops.push_back({OP_EXCH, cur, mem, 0, 0});
@@ -366,6 +509,7 @@ void flatten_plan(const Plan& p, std::vector<DevPass>* passes, bool split) {
     for (int i = 0; i < kMaxOut; ++i) d.out_q[i] = i < d.n_out ? ps.out_q[i] : -1;
     d.partial_off = 0;
     for (int s = 0; s < kMaxSlots; ++s) d.slot_lq[s] = s < d.nslots ? ps.slot_lq[s] : 0;
+    set_pass_perm(p, ps, ops, &d);
     for (int o = 0; o < kMaxOps; ++o) {
       if (o < d.nops) {
         const HostOp& h = ops[o];

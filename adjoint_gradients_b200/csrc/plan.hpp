@@ -44,8 +44,26 @@ struct HostPass {
   int variant;                // see DevPass::variant
 };
 
+// Fused CNOT layers (two qubit sets A = sets[0], B = sets[1]).  A layer's
+// CNOT list is a linear map M of the index bits over GF(2) (the amplitude at
+// x moves to M x).  When the block of M from A's bits to A's bits is
+// invertible, M = M2 M1 exactly, where M1 changes only A's bits ((M1 x)_A =
+// (M x)_A) and M2 = M M1^-1 changes only B's bits.  M1 acts inside the tile
+// of A's passes (B's bits, in or out of that tile, are only read), M2 inside
+// B's.  So each layer runs as two passes and the state is never gathered
+// through HBM: [M2 of the layer before, rotations of B], [rotations of A,
+// M1]; one more pass applies the last layer's M2.  fwd[g] / inv[g] hold the
+// columns of M_g / M_g^-1 (g = 0: M1, 1: M2) as qubit masks: the image of
+// the single qubit q.
+struct CnotLayers {
+  uint32_t fwd[2][kMaxQubits];
+  uint32_t inv[2][kMaxQubits];
+};
+
 struct Plan {
   int n = 0, L = 0, ckpt_block = 0;
+  bool cnot = false;  // fused CNOT layers (CnotLayers)
+  CnotLayers cl{};
   int n_sets = 0;
   // Address bit of each qubit in the working state between passes (HBM
   // layout; the standard layout is addr_of[q] = q).  Multi-set plans put the
@@ -61,7 +79,17 @@ struct Plan {
 };
 
 // Build the schedule.  Returns an empty string on success, else an error.
-std::string make_plan(int n, int L, int ckpt_block, Plan* out);
+// With cl, the fused CNOT schedule (two qubit sets only).
+std::string make_plan(int n, int L, int ckpt_block, Plan* out, const CnotLayers* cl = nullptr);
+
+// Factor the map of a CNOT list (control, target; applied in list order)
+// into M2 M1 for the fused schedule of an n-qubit circuit; false when n does
+// not give two qubit sets or the A-to-A block of the map is singular.
+bool factor_cnot_layer(int n, const std::vector<std::pair<int, int>>& pairs, CnotLayers* out);
+
+// Columns of the map of a CNOT list on qubit bits: fwd[q] = M e_q and
+// inv[q] = M^-1 e_q.
+void cnot_list_map(int n, const std::vector<std::pair<int, int>>& pairs, uint32_t* fwd, uint32_t* inv);
 
 // Entangler of every layer: CZ on each bond (a, b).  The default is the
 // chain (q, q+1), q = 0 .. n-2.

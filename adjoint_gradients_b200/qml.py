@@ -258,10 +258,22 @@ class Context:
             _check(self.lib.qml_set_entangler(self._h, len(bonds), arr), "qml_set_entangler")
         elif kind == "cnot":
             _check(self.lib.qml_set_entangler_cnot(self._h, len(bonds), arr), "qml_set_entangler_cnot")
-            if self.ws is not None and self.ws.numel() - 256 < self.workspace_bytes(self._host_step):
-                self.allocate_workspace(host_step=self._host_step)
         else:
             raise ValueError("kind must be 'cz' or 'cnot'")
+        self._reset_workspace()
+
+    def _reset_workspace(self):
+        """Set the workspace again after a change of entangler (the schedule's
+        device copies and the layout may change with it); a larger one is
+        allocated when the current buffer is too small."""
+        if self.ws is None:
+            return
+        nbytes = self.workspace_bytes(self._host_step)
+        if self.ws.numel() - 256 < nbytes:
+            self.allocate_workspace(host_step=self._host_step)
+            return
+        aligned = (self.ws.data_ptr() + 255) // 256 * 256
+        _check(self.lib.qml_set_workspace(self._h, aligned, nbytes, _stream_handle(None)), "qml_set_workspace")
 
     @property
     def entangler_kind(self) -> str:

@@ -197,16 +197,23 @@ QML_API int qml_entangler_bonds(const qml_ctx* ctx);
  * ends with CNOT(pairs[2e] -> pairs[2e+1]) (control, target) for e = 0 ..
  * n_pairs-1 in list order, e.g. the ladder (q, q+1).  The pages name CNOT
  * gates as the other entangler their kernels fuse by recomputing indices
- * ([Deep-dive] sec. 3.2).  A layer's CNOT list is a linear map of the index
- * bits; it moves amplitudes across tiles, so each layer runs its rotations as
- * the fused passes of a one-layer schedule and then one gather pass into a
- * second state buffer (the workspace grows by B * 2^n complex64: call
- * qml_workspace_bytes / qml_set_workspace again after this call if the
- * workspace was set before; the compute calls return QML_ERR_WORKSPACE until
- * it is large enough).  Checkpoint slots, observables and re-uploading apply
- * as with CZ, in both precisions (fp64 contexts keep the standard order and
- * need B * 2^n complex128 more).  QML_ERR_INVALID_ARG on a bad pair or count.
- * qml_set_entangler switches back to CZ. */
+ * ([Deep-dive] sec. 3.2).  A layer's CNOT list is a linear map M of the
+ * index bits over GF(2).  fp32 contexts of 13..20 qubits (two qubit sets A,
+ * B) whose map factors as M = M2 M1, M1 changing only A's bits and M2 only
+ * B's (true whenever the A-to-A block of M is invertible, e.g. the ladder or
+ * the ring), run fused: M1 and M2 are applied inside the rotation passes, as
+ * a permutation of each tile's positions while it is read or in a layout
+ * exchange, and each layer costs two passes with no gather through HBM.
+ * Other contexts (other sizes, fp64, re-uploading, maps that do not factor)
+ * run each layer's rotations as the fused passes of a one-layer schedule and
+ * then one gather pass into a second state buffer (the workspace grows by B
+ * * 2^n complex64, or complex128 in fp64).  Either way the schedule changes:
+ * if a workspace was set before, it is released by this call and must be set
+ * again (qml_workspace_bytes / qml_set_workspace); the compute calls return
+ * QML_ERR_WORKSPACE until then.  Checkpoint slots, observables and
+ * re-uploading apply as with CZ, in both precisions.  QML_ERR_INVALID_ARG on
+ * a bad pair or count.  qml_set_entangler switches back to CZ (and releases
+ * the workspace the same way when the fused schedule was in force). */
 QML_API qml_status qml_set_entangler_cnot(qml_ctx* ctx, int n_pairs, const int* pairs);
 
 /* Kind of the entangler in force: 0 CZ, 1 CNOT (-1 for NULL). */
@@ -216,7 +223,9 @@ QML_API int qml_entangler_kind(const qml_ctx* ctx);
  * bits, written like qml_debug_schedule (returns the number of ints, -1 when
  * the entangler is not CNOT).  Layout: [n, then n images of M (the layer
  * sends the amplitude at b to M b) on qubit bits, n images of M^-1, then the
- * same two maps on working-state address bits]. */
+ * same two maps on working-state address bits, then 1 if the fused schedule
+ * is in force (else 0), then n images of M1 and n images of M2 on qubit bits
+ * (M = M2 M1; zeros when not fused)]. */
 QML_API int qml_debug_entangler_map(const qml_ctx* ctx, int* out, int cap);
 
 /* Data re-uploading for the following forward and backward calls: with

@@ -145,3 +145,85 @@ def test_address_map_is_the_qubit_map_with_renamed_bits():
         assert _apply(Ma, to_addr(b)) == to_addr(_apply(M, b))
         assert _apply(Mainv, _apply(Ma, to_addr(b))) == to_addr(b)
     lib.qml_destroy(h)
+
+
+def _fused(lib, h):
+    need = lib.qml_debug_entangler_map(h, None, 0)
+    buf = (ctypes.c_int * need)()
+    lib.qml_debug_entangler_map(h, buf, need)
+    v = list(buf)
+    n = v[0]
+    j = 1 + 4 * n
+    return v[j], v[j + 1:j + 1 + n], v[j + 1 + n:j + 1 + 2 * n]
+
+
+def _sets(n):
+    """The two qubit sets of a 13..20-qubit circuit: consecutive runs, the first one longer when n is odd."""
+    a = (n + 1) // 2
+    return list(range(a)), list(range(a, n))
+
+
+def test_fused_factors_recompose_the_layer_and_touch_one_set_each():
+    """M = M2 M1 with M1 changing only the first set's bits and M2 only the second's, checked on
+    basis states pushed through the list gate by gate (an independent simulation of the list)."""
+    import numpy as np
+
+    rng = np.random.default_rng(11)
+    for n in (13, 16, 20):
+        A, Bq = _sets(n)
+        mA = sum(1 << q for q in A)
+        allp = [(a, b) for a in range(n) for b in range(n) if a != b]
+        lists = [[(q, q + 1) for q in range(n - 1)], [(q, (q + 1) % n) for q in range(n)]]
+        lists += [[allp[i] for i in rng.choice(len(allp), size=n + 2, replace=False)] for _ in range(4)]
+        n_fused = 0
+        for pairs in lists:
+            lib, h = _ctx(n, 3, 2, 1)
+            assert lib.qml_set_entangler_cnot(h, len(pairs), _pairs(pairs)) == qml.QML_OK
+            fused, M1, M2 = _fused(lib, h)
+            if fused:
+                n_fused += 1
+                for b in [int(v) for v in rng.integers(0, 1 << n, size=48)] + [1 << q for q in range(n)]:
+                    y1 = _apply(M1, b)
+                    assert (y1 ^ b) & ~mA == 0  # M1 leaves the second set alone
+                    y2 = _apply(M2, y1)
+                    assert (y2 ^ y1) & mA == 0  # M2 leaves the first set alone
+                    assert y2 == _simulate(pairs, b)
+            lib.qml_destroy(h)
+        assert n_fused >= 2  # the ladder and the ring always factor
+
+
+def test_fused_schedule_has_two_passes_per_layer():
+    n, L = 16, 5
+    lib, h = _ctx(n, L, 2, 2)
+    ladder = [(q, q + 1) for q in range(n - 1)]
+    assert lib.qml_set_entangler_cnot(h, len(ladder), _pairs(ladder)) == qml.QML_OK
+    need = lib.qml_debug_schedule(h, None, 0)
+    buf = (ctypes.c_int * need)()
+    lib.qml_debug_schedule(h, buf, need)
+    v = list(buf)
+    assert v[0] == 2 * L + 1  # [M2 of the layer before, second set], [first set, M1]; then the last M2
+    # every pass holds at most one permutation op (kind 7)
+    i, perms = 1, []
+    for _ in range(v[0]):
+        nops = v[i + 4]
+        kinds = [v[i + 5 + 4 * k] for k in range(nops)]
+        perms.append(kinds.count(7))
+        i += 5 + 4 * nops
+    assert perms[0] == 0 and all(p == 1 for p in perms[1:])
+    lib.qml_destroy(h)
+
+
+def test_unfactorable_maps_and_other_sizes_stay_on_the_gather_path():
+    # SWAP(0, 9) from three CNOTs at n = 16 (sets 0-7 and 8-15): the first set's block of the map is
+    # singular (qubit 0's new value comes from the second set only)
+    lib, h = _ctx(16, 2, 2)
+    swap = [(0, 9), (9, 0), (0, 9)]
+    assert lib.qml_set_entangler_cnot(h, 3, _pairs(swap)) == qml.QML_OK
+    assert _fused(lib, h)[0] == 0
+    lib.qml_destroy(h)
+    for n, f64 in [(12, False), (21, False), (16, True)]:
+        lib, h = _ctx(n, 2, 2, f64=f64)
+        ladder = [(q, q + 1) for q in range(n - 1)]
+        assert lib.qml_set_entangler_cnot(h, len(ladder), _pairs(ladder)) == qml.QML_OK
+        assert _fused(lib, h)[0] == 0
+        lib.qml_destroy(h)

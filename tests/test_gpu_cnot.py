@@ -44,7 +44,15 @@ CASES = [
     (14, 2, 3, 1, "fp32", "ladder"),
     (17, 3, 2, 0, "fp32", "random"),
     (20, 2, 3, 1, "fp32", "ladder"),
+    # two qubit sets, fp32: the layer maps are applied inside the rotation passes (fused schedule)
+    (13, 3, 5, 1, "bf16", "ladder"),
+    (15, 4, 3, 2, "fp32", "ring"),
+    (16, 3, 2, 1, "fp32", "random"),
+    (19, 3, 1, 1, "fp32", "random"),
+    (20, 3, 2, 1, "bf16", "ring"),
+    (20, 4, 3, 0, "fp32", "ladder"),
     (21, 2, 3, 1, "fp32", "ladder"),  # three qubit sets: permuted working-state addresses
+    (22, 3, 3, 1, "bf16", "ladder"),  # three sets with bf16 checkpoints on the working-state layout
     (23, 2, 1, 0, "fp32", "random"),
 ]
 
