@@ -118,6 +118,20 @@ struct qml_ctx {
   // one-layer schedules above.
   bool cnot_fused = false;
   CnotLayers cnot_map{};  // M1, M2 of the fused schedule
+  // qml_step_host replays a CUDA graph of its copies and launches once the
+  // same call (buffers, batch, settings) has run eagerly; gen counts changes
+  // of the settings a captured step depends on
+  struct HostGraph {
+    cudaGraphExec_t exec = nullptr;
+    const void* key[7] = {};
+    int B = 0;
+    unsigned gen = 0;
+    long long launches = 0;  // kernel launches inside the graph
+    bool seen = false;       // the keyed call ran eagerly once
+    bool failed = false;     // its capture failed: stay eager
+  } hg;
+  unsigned gen = 1;
+  cudaStream_t cap = nullptr;  // capture stream of the host-step graph
   bool f64 = false;       // fp64 compute mode (qml_create_f64)
   // host-side fault injection for tests of the error paths (QML_FAULT at create)
   enum Fault { FAULT_NONE, FAULT_ALLOC, FAULT_CKPT, FAULT_NAN } fault = FAULT_NONE;
@@ -274,6 +288,18 @@ cudaEvent_t take_event(qml_ctx* c) {
   return e;
 }
 
+// A timing event on s; inside a stream capture it becomes an event-record
+// node of the graph (so every replay records it).  A failed record is
+// cleared, so that it is not reported by the next launch check.
+bool record_span_event(cudaEvent_t ev, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) cs = cudaStreamCaptureStatusNone;
+  const cudaError_t e = cs == cudaStreamCaptureStatusActive ? cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal)
+                                                            : cudaEventRecord(ev, s);
+  if (e != cudaSuccess) cudaGetLastError();
+  return e == cudaSuccess;
+}
+
 // Record the start of a run of pass launches; returns false if timing is off.
 bool span_begin(qml_ctx* c, cudaStream_t s, qml_ctx::Span* sp, bool bwd) {
   if (!c->timing) return false;
@@ -282,11 +308,11 @@ bool span_begin(qml_ctx* c, cudaStream_t s, qml_ctx::Span* sp, bool bwd) {
   sp->bwd = bwd;
   sp->passes = (int)c->dpass.size();
   if (!sp->a || !sp->b) return false;
-  return cudaEventRecord(sp->a, s) == cudaSuccess;
+  return record_span_event(sp->a, s);
 }
 
 void span_end(qml_ctx* c, cudaStream_t s, qml_ctx::Span* sp) {
-  if (cudaEventRecord(sp->b, s) == cudaSuccess) c->spans.push_back(*sp);
+  if (record_span_event(sp->b, s)) c->spans.push_back(*sp);
 }
 
 bool misaligned(const void* p, size_t a) { return ((uintptr_t)p) % a != 0; }
@@ -1126,6 +1152,11 @@ static qml_status create_ctx(const qml_config* cfg, int device, bool f64, qml_ct
 
 qml_status qml_destroy(qml_ctx* ctx) {
   if (!ctx) return QML_ERR_INVALID_ARG;
+  {
+    DeviceGuard g(ctx->device);
+    if (ctx->hg.exec) cudaGraphExecDestroy(ctx->hg.exec);
+    if (ctx->cap) cudaStreamDestroy(ctx->cap);
+  }
   for (auto& sp : ctx->spans) {
     cudaEventDestroy(sp.a);
     cudaEventDestroy(sp.b);
@@ -1153,6 +1184,7 @@ size_t qml_host_workspace_bytes(const qml_ctx* cctx, int B) {
 
 qml_status qml_set_workspace(qml_ctx* c, void* ws, size_t bytes, void* stream) {
   if (!c || !ws) return QML_ERR_INVALID_ARG;
+  ++c->gen;  // a captured host step no longer matches
   if (c->fault == qml_ctx::FAULT_ALLOC) return QML_ERR_WORKSPACE;  // injected: as if the buffer were too small
   if (misaligned(ws, kAlign)) return QML_ERR_INVALID_ARG;
   ensure_device(c);
@@ -1278,6 +1310,7 @@ qml_status qml_expect_z0(qml_ctx* c, const float* psi, int B, float* expect, voi
 
 qml_status qml_set_observable(qml_ctx* c, int n_terms, const char* paulis, const double* coeffs) {
   if (!c || n_terms < 0 || n_terms > QML_MAX_OBS_TERMS) return QML_ERR_INVALID_ARG;
+  ++c->gen;  // a captured host step no longer matches
   if (n_terms > 0 && (!paulis || !coeffs)) return QML_ERR_INVALID_ARG;
   const int n = c->cfg.n_qubits;
   struct Term {
@@ -1335,6 +1368,7 @@ static void restore_default_plan(qml_ctx* c) {
 
 qml_status qml_set_entangler(qml_ctx* c, int n_bonds, const int* bonds) {
   if (!c || n_bonds < 0 || n_bonds > QML_MAX_BONDS || (n_bonds > 0 && !bonds)) return QML_ERR_INVALID_ARG;
+  ++c->gen;  // a captured host step no longer matches
   const int n = c->cfg.n_qubits;
   Bonds b;
   for (int e = 0; e < n_bonds; ++e) {
@@ -1354,6 +1388,7 @@ qml_status qml_set_entangler(qml_ctx* c, int n_bonds, const int* bonds) {
 
 qml_status qml_set_entangler_cnot(qml_ctx* c, int n_pairs, const int* pairs) {
   if (!c || n_pairs < 1 || n_pairs > QML_MAX_BONDS || !pairs) return QML_ERR_INVALID_ARG;
+  ++c->gen;  // a captured host step no longer matches
   const int n = c->cfg.n_qubits;
   std::vector<std::pair<int, int>> v;
   for (int e = 0; e < n_pairs; ++e) {
@@ -1439,6 +1474,7 @@ int qml_debug_entangler_map(const qml_ctx* c, int* out, int cap) {
 
 qml_status qml_set_reupload(qml_ctx* c, int on) {
   if (!c) return QML_ERR_INVALID_ARG;
+  ++c->gen;  // a captured host step no longer matches
   if (on && c->slow && !c->f64) return QML_ERR_UNSUPPORTED;  // fp32, n < 5: batch-unit register bits
   c->reupload = on != 0;
   return QML_OK;
@@ -1463,14 +1499,9 @@ qml_status qml_expect_observable(qml_ctx* c, const float* psi, int B, float* exp
                                         static_cast<cudaStream_t>(stream)));
 }
 
-qml_status qml_step_host(qml_ctx* c, const float* x_h, const float* theta_h, const float* y_h, int B,
-                         float* expect_h, float* loss_h, float* grad_h, void* stream) {
-  qml_status st = check_ready(c, B);
-  if (st != QML_OK) return st;
-  if (!x_h || !theta_h || !y_h || !grad_h) return QML_ERR_INVALID_ARG;
-  if (c->ws_bytes < c->lay.host_total) return QML_ERR_WORKSPACE;
-  DeviceGuard g(c->device);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+// The copies and launches of one host step, enqueued on s (no synchronisation).
+static qml_status enqueue_step_host(qml_ctx* c, const float* x_h, const float* theta_h, const float* y_h, int B,
+                                    float* expect_h, float* loss_h, float* grad_h, cudaStream_t s) {
   const int n = c->cfg.n_qubits, L = c->cfg.n_layers;
   const Layout& l = c->lay;
   cudaError_t e = cudaMemcpyAsync(c->ws + l.h_x, x_h, sizeof(float) * (size_t)B * n, cudaMemcpyHostToDevice, s);
@@ -1480,7 +1511,7 @@ qml_status qml_step_host(qml_ctx* c, const float* x_h, const float* theta_h, con
   if (e != cudaSuccess) return QML_ERR_CUDA;
   float2* psi = at<float2>(c, l.h_psi);
   float2* lam = at<float2>(c, l.h_lam);
-  st = run_forward(c, at<float>(c, l.h_theta), at<float>(c, l.h_x), B, psi, at<float>(c, l.h_E), s);
+  qml_status st = run_forward(c, at<float>(c, l.h_theta), at<float>(c, l.h_x), B, psi, at<float>(c, l.h_E), s);
   if (st != QML_OK) return st;
   e = launch_loss_seed(at<float>(c, l.h_E), at<float>(c, l.h_y), B, at<float>(c, l.h_g), at<float>(c, l.h_loss), s);
   ++c->launches;
@@ -1492,6 +1523,78 @@ qml_status qml_step_host(qml_ctx* c, const float* x_h, const float* theta_h, con
   if (e == cudaSuccess && expect_h)
     e = cudaMemcpyAsync(expect_h, c->ws + l.h_E, sizeof(float) * (size_t)B, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess && loss_h) e = cudaMemcpyAsync(loss_h, c->ws + l.h_loss, sizeof(float), cudaMemcpyDeviceToHost, s);
+  return cuda_status(e);
+}
+
+static void drop_host_graph(qml_ctx* c) {
+  if (c->hg.exec) cudaGraphExecDestroy(c->hg.exec);
+  c->hg = qml_ctx::HostGraph{};
+}
+
+// Capture one host step on the context's own stream into an executable graph
+// (false, and nothing kept, if any part of it cannot be captured).
+static bool capture_step_host(qml_ctx* c, const float* x_h, const float* theta_h, const float* y_h, int B,
+                              float* expect_h, float* loss_h, float* grad_h) {
+  if (!c->cap && cudaStreamCreateWithFlags(&c->cap, cudaStreamNonBlocking) != cudaSuccess) {
+    cudaGetLastError();
+    c->cap = nullptr;
+    return false;
+  }
+  const long long l0 = c->launches;
+  if (cudaStreamBeginCapture(c->cap, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  const qml_status st = enqueue_step_host(c, x_h, theta_h, y_h, B, expect_h, loss_h, grad_h, c->cap);
+  cudaGraph_t g = nullptr;
+  const cudaError_t e = cudaStreamEndCapture(c->cap, &g);
+  const long long nl = c->launches - l0;
+  c->launches = l0;
+  bool ok = st == QML_OK && e == cudaSuccess && g != nullptr;
+  cudaGraphExec_t exec = nullptr;
+  if (ok) ok = cudaGraphInstantiate(&exec, g, 0) == cudaSuccess;
+  if (g) cudaGraphDestroy(g);
+  if (!ok) {
+    cudaGetLastError();
+    if (exec) cudaGraphExecDestroy(exec);
+    return false;
+  }
+  c->hg.exec = exec;
+  c->hg.launches = nl;
+  return true;
+}
+
+qml_status qml_step_host(qml_ctx* c, const float* x_h, const float* theta_h, const float* y_h, int B,
+                         float* expect_h, float* loss_h, float* grad_h, void* stream) {
+  qml_status st = check_ready(c, B);
+  if (st != QML_OK) return st;
+  if (!x_h || !theta_h || !y_h || !grad_h) return QML_ERR_INVALID_ARG;
+  if (c->ws_bytes < c->lay.host_total) return QML_ERR_WORKSPACE;
+  DeviceGuard g(c->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const void* key[7] = {x_h, theta_h, y_h, expect_h, loss_h, grad_h, c->ws};
+  qml_ctx::HostGraph& hg = c->hg;
+  const bool same = hg.B == B && hg.gen == c->gen && std::memcmp(hg.key, key, sizeof(key)) == 0;
+  if (!same) {
+    drop_host_graph(c);
+    std::memcpy(hg.key, key, sizeof(key));
+    hg.B = B;
+    hg.gen = c->gen;
+  }
+  // the same call again (timing off, every upload done by the eager run):
+  // capture it once, then replay
+  if (same && hg.seen && !hg.exec && !hg.failed && !c->timing)
+    hg.failed = !capture_step_host(c, x_h, theta_h, y_h, B, expect_h, loss_h, grad_h);
+  cudaError_t e;
+  if (same && hg.exec && !c->timing) {
+    e = cudaGraphLaunch(hg.exec, s);
+    c->launches += hg.launches;
+  } else {
+    st = enqueue_step_host(c, x_h, theta_h, y_h, B, expect_h, loss_h, grad_h, s);
+    if (st != QML_OK) return st;
+    hg.seen = true;
+    e = cudaSuccess;
+  }
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   return cuda_status(e);
 }

@@ -293,6 +293,17 @@ class Context:
         return bool(self.lib.qml_split_form(self._h))
 
     @property
+    def cnot_fused(self) -> bool:
+        """True when CNOT layers run through the fused schedule (their maps applied
+        inside the rotation passes; see qml_set_entangler_cnot)."""
+        if self.lib.qml_entangler_kind(self._h) != 1:
+            return False
+        need = self.lib.qml_debug_entangler_map(self._h, None, 0)
+        buf = (ctypes.c_int * need)()
+        self.lib.qml_debug_entangler_map(self._h, buf, need)
+        return bool(buf[1 + 4 * self.n]) and not self.reupload and self.precision == "fp32"
+
+    @property
     def entangler_bonds(self) -> int:
         return int(self.lib.qml_entangler_bonds(self._h))
 

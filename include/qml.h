@@ -321,7 +321,16 @@ QML_API qml_status qml_expect_z0_static(const float* psi_dev, int n_qubits, int 
  * and the staged inputs).  Synchronises `stream` before returning.
  *   x_host [B][n], theta_host [L][n][3], y_host [B]      (in)
  *   expect_host [B], loss_host [1], grad_host [L][n][3]  (out; may be NULL
- *   except grad_host) */
+ *   except grad_host)
+ * Repeated calls: once a call with the same host buffers, batch and
+ * workspace has run, the next such call captures the step's copies and
+ * launches into a CUDA graph (on a stream of the context's own) and later
+ * ones replay it on `stream`, which removes the per-launch host cost of small
+ * circuits.  The buffers' contents are read at each replay, so new inputs in
+ * the same buffers are fine.  Any setter (entangler, observable,
+ * re-uploading, workspace) and timing (qml_enable_timing) return it to the
+ * eager path; a step that cannot be captured (e.g. pageable host buffers on
+ * some systems) stays eager.  Host buffers should be pinned. */
 QML_API size_t qml_host_workspace_bytes(const qml_ctx* ctx, int B);
 QML_API qml_status qml_step_host(qml_ctx* ctx, const float* x_host, const float* theta_host,
                          const float* y_host, int B, float* expect_host, float* loss_host,
