@@ -499,11 +499,9 @@ qml_status run_forward_cnot(qml_ctx* c, const float* theta, const float* x, int 
       a.n_tiles = (int)(((a.U + (1ll << dp.unit_bits) - 1) >> dp.unit_bits) << dp.n_out);
       a.buf0 = cur;
       a.dummy = part;
-      e = copy_pass_coef(c->region, cf + p, dp.nslots, 0, s);
-      if (e != cudaSuccess) return QML_ERR_CUDA;
       const PassMaps* maps = pass_maps_for(c, dp, false, B, cur, part);
       if (!maps) return QML_ERR_CUDA;
-      e = launch_pass(false, a, dp, *maps, c->grid_fwd, c->smem, s);
+      e = launch_pass(false, a, dp, *maps, c->grid_fwd, c->smem, s, cf + p);
       if (e != cudaSuccess) return QML_ERR_CUDA;
       ++c->launches;
     }
@@ -614,11 +612,9 @@ qml_status run_backward_cnot(qml_ctx* c, const float* theta, const float* x, int
       a.n_tiles = (int)(((a.U + (1ll << dp.unit_bits) - 1) >> dp.unit_bits) << dp.n_out);
       a.buf0 = b0;
       a.buf1 = b1;
-      e = copy_pass_coef(c->region, ci + p, dp.nslots, 0, s);
-      if (e != cudaSuccess) return QML_ERR_CUDA;
       const PassMaps* maps = pass_maps_for(c, dp, true, B, b0, b1);
       if (!maps) return QML_ERR_CUDA;
-      e = launch_pass(true, a, dp, *maps, c->grid_bwd, c->smem, s);
+      e = launch_pass(true, a, dp, *maps, c->grid_bwd, c->smem, s, ci + p);
       if (e != cudaSuccess) return QML_ERR_CUDA;
       ++c->launches;
     }
@@ -695,6 +691,7 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
     e = launch_pass(false, a, dp, none, c->grid_fwd, c->smem, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
     ++c->launches;
+    sp.passes = 1;  // the span times one launch
     for (const DevPass& q : passes)
       if (q.ckpt >= 0) c->ckpt_batch[q.ckpt] = B;
   }
@@ -702,11 +699,9 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
     const DevPass& dp = passes[p];
     const long long units_per_tile = 1ll << dp.unit_bits;
     a.n_tiles = (int)(((a.U + units_per_tile - 1) / units_per_tile) << dp.n_out);
-    e = copy_pass_coef(c->region, cf + p, dp.nslots, dp.ndiag, s);
-    if (e != cudaSuccess) return QML_ERR_CUDA;
     const PassMaps* maps = pass_maps(c, p, false, B, psi, a.dummy);
     if (!maps) return QML_ERR_CUDA;
-    e = launch_pass(false, a, dp, *maps, c->grid_fwd, c->smem, s);
+    e = launch_pass(false, a, dp, *maps, c->grid_fwd, c->smem, s, cf + p);
     if (e != cudaSuccess) return QML_ERR_CUDA;
     ++c->launches;
     if (dp.ckpt >= 0) c->ckpt_batch[dp.ckpt] = B;
@@ -785,17 +780,16 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
     e = launch_pass(true, a, dp, none, c->grid_bwd, c->smem, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
     ++c->launches;
+    sp.passes = 1;  // the span times one launch
   }
   for (int p = P - 1; p >= 0 && !one_launch; --p) {
     const DevPass& dp = passes[p];
     const long long units_per_tile = 1ll << dp.unit_bits;
     a.n_tiles = (int)(((a.U + units_per_tile - 1) / units_per_tile) << dp.n_out);
     a.rscale = (split && dp.ckpt >= 0) ? at<float>(c, c->lay.rscale) + p : nullptr;
-    e = copy_pass_coef(c->region, ci + p, dp.nslots, dp.ndiag, s);
-    if (e != cudaSuccess) return QML_ERR_CUDA;
     const PassMaps* maps = pass_maps(c, p, true, B, psi, lam);
     if (!maps) return QML_ERR_CUDA;
-    e = launch_pass(true, a, dp, *maps, c->grid_bwd, c->smem, s);
+    e = launch_pass(true, a, dp, *maps, c->grid_bwd, c->smem, s, ci + p);
     if (e != cudaSuccess) return QML_ERR_CUDA;
     ++c->launches;
   }

@@ -86,14 +86,26 @@ struct PassMaps {
 cudaError_t encode_pass_maps(const DevPass& p, int n, int B, bool backward, const void* buf0, const void* buf1,
                              PassMaps* maps);
 
-// Launch one pass; the kernel instance follows the pass's layout variant and
-// how its tiles are loaded (n < 5: generic; tensor copies when p.tma).
+// Launch one pass; the kernel instance follows the pass's layout variant,
+// how its tiles are loaded (n < 5: generic; tensor copies when p.tma) and
+// the rotation form.  coef (device memory, may be null): the pass's gate
+// coefficients, first copied in stream order into the context's
+// constant-memory region of the unit that holds the instance (the first
+// p.nslots rotation slots, and the diagonal tables when the pass has any).
 cudaError_t launch_pass(bool backward, const PassArgs& a, const DevPass& p, const PassMaps& maps, int grid,
-                        size_t smem, cudaStream_t s);
-// Copy one pass's gate coefficients (device memory) into the context's
-// constant-memory region, in stream order: the first nslots rotation slots,
-// and the diagonal tables when the pass has any.
-cudaError_t copy_pass_coef(int region, const CoefRegion* src, int nslots, int ndiag, cudaStream_t s);
+                        size_t smem, cudaStream_t s, const CoefRegion* coef = nullptr);
+// The units that instantiate the pass kernel (pass_split.cu: split form;
+// pass_fused.cu: fused SU(2) form, CZ or CNOT; pass_reup.cu: re-uploading).
+// form: 0 fused SU(2), 1 and 2 re-uploading (2: per register pair), 3 split.
+#define QML_PASS_UNIT_DECL(NAME)                                                                        \
+  cudaError_t NAME##_launch(bool backward, int mode, int variant, int form, const PassArgs& a,           \
+                            const DevPass& p, const PassMaps& maps, int grid, size_t smem,               \
+                            const CoefRegion* coef, cudaStream_t s);                                    \
+  cudaError_t NAME##_attr(size_t smem_thr, size_t smem_tma);
+QML_PASS_UNIT_DECL(pass_split)
+QML_PASS_UNIT_DECL(pass_fused)
+QML_PASS_UNIT_DECL(pass_reup)
+#undef QML_PASS_UNIT_DECL
 // Full SU(2) coefficients of every pass slot: cf forward, ci backward ([P] regions).
 cudaError_t launch_prep_pass_coef(const DevPass* passes, int n_passes, const float* theta, CoefRegion* cf,
                                   CoefRegion* ci, cudaStream_t s);
