@@ -235,11 +235,12 @@ void compute_layout(qml_ctx* c) {
   l.passes_split = take(sizeof(DevPass) * c->dpass_split.size());
   l.undo = take(sizeof(int) * (size_t)L * n);
   l.s_rot = take(sizeof(SplitRot) * (size_t)L * n);
-  l.s_lay = take(sizeof(SplitLayer) * (size_t)L);
+  l.s_lay = take(sizeof(SplitLayer) * 2 * (size_t)L);  // per layer, or per layer and set (fused CNOT)
   l.s_gfix = take(sizeof(double) * 2 * (size_t)L * n);
   if (!c->f64) {
-    l.s_dqf = take(sizeof(float2) * 2 * (size_t)(L + 1) * n);
-    l.s_dqb = take(sizeof(float2) * 2 * (size_t)(L + 1) * n);
+    // per diagonal op: L + 1 of them, or 4 L in the fused CNOT schedule
+    l.s_dqf = take(sizeof(float2) * 2 * (size_t)(4 * L + 1) * n);
+    l.s_dqb = take(sizeof(float2) * 2 * (size_t)(4 * L + 1) * n);
     l.rscale = take(sizeof(float) * c->dpass_split.size());
   } else {
     l.s_dq64f = take(sizeof(double2) * 2 * (size_t)(L + 1) * n);
@@ -327,7 +328,7 @@ T* at(qml_ctx* c, size_t off) {
 // fp32 contexts run the split form unless a mode needs the fused SU(2)
 // (re-uploading folds per-sample encodings into the rotations; CNOT layers
 // run as one-layer schedules).
-bool use_split(const qml_ctx* c) { return !c->f64 && !c->reupload && !c->cnot; }
+bool use_split(const qml_ctx* c) { return !c->f64 && !c->reupload && (!c->cnot || c->cnot_fused); }
 // CNOT entanglers through the fused schedule (the generic pass loop), or the
 // one-layer schedules with a gather per layer
 bool cnot_fused_now(const qml_ctx* c) { return c->cnot && c->cnot_fused && !c->reupload && !c->f64; }
@@ -637,6 +638,15 @@ cudaError_t prep_coefficients(qml_ctx* c, const float* theta, cudaStream_t s) {
   CoefRegion* ci = at<CoefRegion>(c, c->lay.coef_inv);
   if (!use_split(c))
     return launch_prep_pass_coef(at<DevPass>(c, c->lay.passes), (int)c->dpass.size(), theta, cf, ci, s);
+  if (c->cnot) {  // the fused CNOT schedule: one segment per layer and qubit set
+    uint32_t set0 = 0;
+    for (int q : c->plan.sets[0]) set0 |= 1u << q;
+    return launch_prep_split_cnot(at<DevPass>(c, c->lay.passes_split), (int)c->dpass_split.size(), theta,
+                                  c->cfg.n_layers, c->cfg.n_qubits, set0, at<int>(c, c->lay.undo),
+                                  at<SplitRot>(c, c->lay.s_rot), at<SplitLayer>(c, c->lay.s_lay),
+                                  at<double>(c, c->lay.s_gfix), at<float2>(c, c->lay.s_dqf),
+                                  at<float2>(c, c->lay.s_dqb), cf, ci, at<float>(c, c->lay.rscale), s);
+  }
   return launch_prep_split(at<DevPass>(c, c->lay.passes_split), (int)c->dpass_split.size(), theta,
                            c->cfg.n_layers, c->cfg.n_qubits, at<int>(c, c->lay.undo), at<SplitRot>(c, c->lay.s_rot),
                            at<SplitLayer>(c, c->lay.s_lay), at<double>(c, c->lay.s_gfix),
@@ -674,7 +684,7 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
   a.bmax = c->cfg.max_batch;
   a.partials = nullptr;
   a.status = at<unsigned>(c, c->lay.status);
-  for (int q = 0; q < kMaxQubits; ++q) a.cz_nb[q] = c->nb[q], a.cz_nbhi[q] = c->nbhi[q];
+  for (int q = 0; q < kMaxQubits; ++q) a.cz_nb[q] = c->cnot ? 0u : c->nb[q], a.cz_nbhi[q] = c->cnot ? 0u : c->nbhi[q];
   a.reupload = c->reupload ? 1 : 0;
   a.dq = split ? at<float2>(c, c->lay.s_dqf) : nullptr;
   a.rscale = nullptr;
@@ -762,7 +772,7 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
   a.bmax = c->cfg.max_batch;
   a.partials = at<float>(c, c->lay.partials);
   a.status = at<unsigned>(c, c->lay.status);
-  for (int q = 0; q < kMaxQubits; ++q) a.cz_nb[q] = c->nb[q], a.cz_nbhi[q] = c->nbhi[q];
+  for (int q = 0; q < kMaxQubits; ++q) a.cz_nb[q] = c->cnot ? 0u : c->nb[q], a.cz_nbhi[q] = c->cnot ? 0u : c->nbhi[q];
   a.reupload = c->reupload ? 1 : 0;
   a.dq = split ? at<float2>(c, c->lay.s_dqb) : nullptr;
   c->launches += split ? 6 : 3;  // coefficient prep, lambda init, gradient reduce
@@ -1355,7 +1365,10 @@ static void restore_default_plan(qml_ctx* c) {
   make_plan(c->cfg.n_qubits, c->cfg.n_layers, c->cfg.ckpt_block, &p);  // succeeded in qml_create
   c->plan = p;
   flatten_plan(p, &c->dpass);
+  flatten_plan(p, &c->dpass_split, true);
+  c->undo = undo_order(p, c->dpass_split);
   set_pass_entangler(p, c->bonds, &c->dpass);
+  set_pass_entangler(p, c->bonds, &c->dpass_split);
   c->cnot_fused = false;
   if (c->ws) drop_workspace(c);
 }
@@ -1433,11 +1446,15 @@ qml_status qml_set_entangler_cnot(qml_ctx* c, int n_pairs, const int* pairs) {
     CnotLayers cl;
     Plan fp;
     if (factor_cnot_layer(n, v, &cl) && make_plan(n, c->cfg.n_layers, c->cfg.ckpt_block, &fp, &cl).empty()) {
-      std::vector<DevPass> dp;
+      std::vector<DevPass> dp, dps;
       flatten_plan(fp, &dp);
+      flatten_plan(fp, &dps, true);
       set_pass_entangler(fp, Bonds{}, &dp);
+      set_pass_entangler(fp, Bonds{}, &dps);
       c->plan = fp;
       c->dpass = dp;
+      c->dpass_split = dps;
+      c->undo = undo_order(fp, dps);
       c->cnot_fused = fused = true;
       c->cnot_map = cl;
     }

@@ -228,6 +228,130 @@ __global__ void split_pass_kernel(const DevPass* passes, int n_passes, const Spl
   ci[p].diag[d][j] = make_float2((float)br, (float)bi);
 }
 
+// ---- split form of the fused CNOT schedule.  A segment (l, s) is the
+// rotations of layer l on qubit set s (one pass); it sits between the
+// diagonal D2 (its Rz(phi2) factors) and D1 (its Rz(phi1) factors and the
+// segment's frame), global diagonal indices 4 l + 2 s + 0 / 1.  The state is
+// exact at every pass boundary in both directions: forward D1 = D1_true Z^m
+// / gam(l, s); backward D1 = gam Z^m D1_true^dagger (the forward frame after
+// the segment's rotations), backward D2 = D2_true^dagger / rho(l, s) (the
+// un-applied tangent forms left rho on the state).
+
+// Per segment: its frame, and per rotation the scale of the backward sums
+// (as split_layer_kernel, over the segment's qubits in the un-apply order).
+__global__ void csplit_seg_kernel(const SplitRot* rot, const int* undo, int L, int n, uint32_t set0,
+                                  SplitLayer* seg, double* gfix) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;  // 2 l + s
+  if (idx >= 2 * L) return;
+  const int l = idx >> 1, sid = idx & 1;
+  const uint32_t mask = sid == 0 ? set0 : (((n >= 32) ? ~0u : ((1u << n) - 1u)) & ~set0);
+  const SplitRot* r = rot + (size_t)l * n;
+  double gam = 1.0, rho = 1.0;
+  uint32_t m = 0;
+  for (int q = 0; q < n; ++q)
+    if ((mask >> q) & 1u) {
+      gam *= r[q].g;
+      rho *= r[q].k2;
+      if (r[q].cot) m |= 1u << q;
+    }
+  seg[idx].gam = gam;
+  seg[idx].rho = rho;
+  seg[idx].cot_mask = m;
+  seg[idx].pad = 0;
+  double undone_k2 = 1.0, applied_g = gam;
+  for (int i = 0; i < n; ++i) {
+    const int q = undo[(size_t)l * n + i];
+    if (!((mask >> q) & 1u)) continue;
+    const double f = undone_k2 * applied_g;
+    gfix[((size_t)l * n + q) * 2 + 0] = (r[q].cot ? -1.0 : 1.0) / (f * f);
+    gfix[((size_t)l * n + q) * 2 + 1] = r[q].phi1;
+    undone_k2 *= r[q].k2;
+    applied_g /= r[q].g;
+  }
+}
+
+// Factor of qubit q's bit b in diagonal d (forward; the backward's is its
+// conjugate): Rz(phi2) of (l, q) for side 0, Rz(phi1) of (l, q) times -1 on
+// b = 1 for a cotangent-form rotation for side 1; 1 for qubits outside the
+// segment's set.
+__device__ __forceinline__ double2 csplit_factor(const SplitRot* rot, const SplitLayer* seg, int n, uint32_t set0,
+                                                 int d, int q, int b, bool bwd) {
+  const int l = d >> 2, sid = (d >> 1) & 1, side = d & 1;
+  const bool in0 = (set0 >> q) & 1u;
+  if (in0 != (sid == 0)) return make_double2(1.0, 0.0);
+  const SplitRot& r = rot[(size_t)l * n + q];
+  double sn, cs;
+  sincos(0.5 * (side ? r.phi1 : r.phi2), &sn, &cs);
+  double re = cs, im = b ? sn : -sn;
+  if (bwd) im = -im;
+  if (side && b && ((seg[2 * l + sid].cot_mask >> q) & 1u)) re = -re, im = -im;
+  return make_double2(re, im);
+}
+
+__global__ void csplit_diag_kernel(const SplitRot* rot, const SplitLayer* seg, int L, int n, uint32_t set0,
+                                   float2* dq_f, float2* dq_b) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;  // ((d + 1) * n + q) * 2 + b
+  if (idx >= (4 * L + 1) * n * 2) return;
+  const int b = idx & 1, q = (idx >> 1) % n, d = (idx >> 1) / n - 1;
+  if (d < 0) {  // (no diagonal -1 in this schedule)
+    dq_f[idx] = dq_b[idx] = make_float2(1.f, 0.f);
+    return;
+  }
+  const double2 f = csplit_factor(rot, seg, n, set0, d, q, b, false);
+  const double2 g = csplit_factor(rot, seg, n, set0, d, q, b, true);
+  dq_f[idx] = make_float2((float)f.x, (float)f.y);
+  dq_b[idx] = make_float2((float)g.x, (float)g.y);
+}
+
+// Per pass: rotation slots, the register tables of its two diagonal ops (the
+// global scales folded in) and the restore scale (1: exact boundaries).
+__global__ void csplit_pass_kernel(const DevPass* passes, int n_passes, const SplitRot* rot, const SplitLayer* seg,
+                                   int n, uint32_t set0, CoefRegion* cf, CoefRegion* ci, float* rscale) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n_passes * kSplitItems) return;
+  const int p = idx / kSplitItems, it = idx % kSplitItems;
+  const DevPass& P = passes[p];
+  if (it < kMaxSlots) {
+    if (it >= P.nslots) return;
+    const SplitRot r = rot[P.slot_lq[it]];
+    const float t = (float)r.tau;
+    cf[p].rot[it][0] = make_float4(t, t, -t, -t);
+    cf[p].rot[it][1] = make_float4((float)r.cot, 0.f, 0.f, 0.f);
+    const float tb = r.cot ? t : -t;
+    ci[p].rot[it][0] = make_float4(tb, tb, -tb, -tb);
+    ci[p].rot[it][1] = make_float4((float)r.cot, 0.f, 0.f, 0.f);
+    return;
+  }
+  if (it == kSplitItems - 1) {
+    rscale[p] = 1.f;
+    return;
+  }
+  const int e = it - kMaxSlots, td = e / kPos, j = e % kPos;
+  int ph = -1, d = 0;
+  for (int o = 0; o < P.nops; ++o)
+    if (P.ops[o].kind == OP_DIAG && P.ops[o].d == td) ph = P.ops[o].a, d = P.ops[o].c;
+  if (ph < 0) return;
+  const SplitLayer& S = seg[2 * (d >> 2) + ((d >> 1) & 1)];
+  double fr = (d & 1) ? 1.0 / S.gam : 1.0, fi = 0.0;
+  double br = (d & 1) ? S.gam : 1.0 / S.rho, bi = 0.0;
+  for (int k = 0; k < kRegBits; ++k) {
+    const int tb = ph == 0 ? k : ph == 1 ? 5 + k : (k < 2 ? 10 + k : k - 2);  // reg_tbit
+    const int q = P.tile_q[tb];
+    if (q < 0) continue;
+    const int b = (j >> k) & 1;
+    const double2 f = csplit_factor(rot, seg, n, set0, d, q, b, false);
+    const double2 g = csplit_factor(rot, seg, n, set0, d, q, b, true);
+    double t = fr * f.x - fi * f.y;
+    fi = fr * f.y + fi * f.x;
+    fr = t;
+    t = br * g.x - bi * g.y;
+    bi = br * g.y + bi * g.x;
+    br = t;
+  }
+  cf[p].diag[td][j] = make_float2((float)fr, (float)fi);
+  ci[p].diag[td][j] = make_float2((float)br, (float)bi);
+}
+
 }  // namespace
 
 cudaError_t launch_prep_pass_coef(const DevPass* passes, int n_passes, const float* theta, CoefRegion* cf,
@@ -267,6 +391,24 @@ cudaError_t launch_prep_split64(const DevPass* passes, int n_passes, const doubl
   split_diag64_kernel<<<(nd + 127) / 128, 128, 0, s>>>(rot, lay, L, n, dq_f, dq_b);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   split_rscale64_kernel<<<(n_passes + 127) / 128, 128, 0, s>>>(passes, n_passes, rot, n, rscale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prep_split_cnot(const DevPass* passes, int n_passes, const float* theta, int L, int n,
+                                   uint32_t set0, const int* undo, SplitRot* rot, SplitLayer* seg, double* gfix,
+                                   float2* dq_f, float2* dq_b, CoefRegion* cf, CoefRegion* ci, float* rscale,
+                                   cudaStream_t s) {
+  const int nr = L * n;
+  split_rot_kernel<float><<<(nr + 127) / 128, 128, 0, s>>>(theta, nr, rot);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  csplit_seg_kernel<<<(2 * L + 127) / 128, 128, 0, s>>>(rot, undo, L, n, set0, seg, gfix);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int nd = (4 * L + 1) * n * 2;
+  csplit_diag_kernel<<<(nd + 127) / 128, 128, 0, s>>>(rot, seg, L, n, set0, dq_f, dq_b);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int np = n_passes * kSplitItems;
+  csplit_pass_kernel<<<(np + 127) / 128, 128, 0, s>>>(passes, n_passes, rot, seg, n, set0, cf, ci, rscale);
   return cudaGetLastError();
 }
 

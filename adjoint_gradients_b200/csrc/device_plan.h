@@ -75,7 +75,10 @@ enum : int { TD_PAD = 0, TD_IN = 1, TD_OUT = 2, TD_SAMPLE = 3, TD_OUT_SAMPLE = 4
 // OP_GEN : a = phase
 // OP_RY  : as OP_ROT (split form)
 // OP_DIAG: a = phase, c = layer l (the diagonal between layers l and l+1;
-//          -1: the one before layer 0), d = its table in the pass (0..kMaxDiag-1)
+//          -1: the one before layer 0), d = its table in the pass (0..kMaxDiag-1);
+//          in passes of the fused CNOT schedule c is the diagonal's index
+//          4 l + 2 set + side (side 0 before the set's rotations of layer l,
+//          1 after them)
 // OP_PERM: a = from phase, b = to phase, c = factor (0: M1, 1: M2), d = layer
 struct DevOp {
   int kind, a, b, c, d;
@@ -115,6 +118,7 @@ struct DevPass {
   uint16_t pcol[2][kTileBits];
   uint16_t pcol_o[2][kMaxOut];
   int ndiag;                 // OP_DIAG ops in the pass (split form)
+  int cnot;                  // 1: a pass of the fused CNOT schedule (see plan.hpp)
   int rs_layer;              // split form, checkpoint pass: layer of the next diagonal op after the pass
   uint32_t rs_mask;          // ... and the qubits it rotates between the pass's end and that op
   long long partial_off;     // float offset of this pass's gradient partials

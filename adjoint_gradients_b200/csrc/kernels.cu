@@ -278,6 +278,7 @@ cudaError_t set_pass_smem_attr(size_t smem_thr, size_t smem_tma) {
   cudaError_t e = pass_split_attr(smem_thr, smem_tma);
   if (e == cudaSuccess) e = pass_fused_attr(smem_thr, smem_tma);
   if (e == cudaSuccess) e = pass_reup_attr(smem_thr, smem_tma);
+  if (e == cudaSuccess) e = pass_csplit_attr(smem_thr, smem_tma);
   return e;
 }
 
@@ -311,6 +312,8 @@ cudaError_t launch_pass(bool backward, const PassArgs& a, const DevPass& p, cons
     for (int b = 0; b < kTileBits; ++b)
       if (p.tile_q[b] < 0) form = 2;
   }
+  if (form == 3 && p.cnot) form = 4;
+  if (form == 4) return pass_csplit_launch(backward, mode, p.variant, form, a, p, maps, grid, smem, coef, s);
   if (form == 3) return pass_split_launch(backward, mode, p.variant, form, a, p, maps, grid, smem, coef, s);
   if (form == 0) return pass_fused_launch(backward, mode, p.variant, form, a, p, maps, grid, smem, coef, s);
   return pass_reup_launch(backward, mode, p.variant, form, a, p, maps, grid, smem, coef, s);

@@ -95,8 +95,10 @@ cudaError_t encode_pass_maps(const DevPass& p, int n, int B, bool backward, cons
 cudaError_t launch_pass(bool backward, const PassArgs& a, const DevPass& p, const PassMaps& maps, int grid,
                         size_t smem, cudaStream_t s, const CoefRegion* coef = nullptr);
 // The units that instantiate the pass kernel (pass_split.cu: split form;
-// pass_fused.cu: fused SU(2) form, CZ or CNOT; pass_reup.cu: re-uploading).
-// form: 0 fused SU(2), 1 and 2 re-uploading (2: per register pair), 3 split.
+// pass_fused.cu: fused SU(2) form, CZ or CNOT; pass_reup.cu: re-uploading;
+// pass_csplit.cu: split form of the fused CNOT schedule).
+// form: 0 fused SU(2), 1 and 2 re-uploading (2: per register pair), 3 split,
+// 4 split with CNOT permutations.
 #define QML_PASS_UNIT_DECL(NAME)                                                                        \
   cudaError_t NAME##_launch(bool backward, int mode, int variant, int form, const PassArgs& a,           \
                             const DevPass& p, const PassMaps& maps, int grid, size_t smem,               \
@@ -105,6 +107,7 @@ cudaError_t launch_pass(bool backward, const PassArgs& a, const DevPass& p, cons
 QML_PASS_UNIT_DECL(pass_split)
 QML_PASS_UNIT_DECL(pass_fused)
 QML_PASS_UNIT_DECL(pass_reup)
+QML_PASS_UNIT_DECL(pass_csplit)
 #undef QML_PASS_UNIT_DECL
 // Full SU(2) coefficients of every pass slot: cf forward, ci backward ([P] regions).
 cudaError_t launch_prep_pass_coef(const DevPass* passes, int n_passes, const float* theta, CoefRegion* cf,
@@ -117,6 +120,14 @@ cudaError_t launch_prep_pass_coef(const DevPass* passes, int n_passes, const flo
 cudaError_t launch_prep_split(const DevPass* passes, int n_passes, const float* theta, int L, int n,
                               const int* undo, SplitRot* rot, SplitLayer* lay, double* gfix, float2* dq_f,
                               float2* dq_b, CoefRegion* cf, CoefRegion* ci, float* rscale, cudaStream_t s);
+// Split form of the fused CNOT schedule (two qubit sets; set0: the first
+// set's qubit mask): one segment per layer and set between two diagonal ops
+// (global index 4 l + 2 set + side), seg [2 L] frames, dq_f / dq_b
+// [4 L + 1][n][2], the other tables as above (rscale: 1).
+cudaError_t launch_prep_split_cnot(const DevPass* passes, int n_passes, const float* theta, int L, int n,
+                                   uint32_t set0, const int* undo, SplitRot* rot, SplitLayer* seg, double* gfix,
+                                   float2* dq_f, float2* dq_b, CoefRegion* cf, CoefRegion* ci, float* rscale,
+                                   cudaStream_t s);
 // fp64 mode (coef.cu): the same tables from an fp64 theta, with the per-qubit
 // diagonal factors dq_f / dq_b in fp64 and the restore scale of every pass.
 cudaError_t launch_prep_split64(const DevPass* passes, int n_passes, const double* theta, int L, int n,

@@ -1178,7 +1178,9 @@ __device__ __forceinline__ void cz_thread_terms(BlockCtx& bc, const DevPass& Pp,
 // thread's amplitudes belong to one batch unit and each rotation takes one set
 // of coefficients.  RE 2: tiles with batch-unit bits (n < 12), coefficients
 // per register pair.  RE 3: the split form (OP_RY and OP_DIAG ops; no
-// re-uploading).
+// re-uploading).  RE 4: the split form of the fused CNOT schedule (also
+// OP_PERM; tensor copies only).  RE 0: the fused SU(2) form (OP_ROT and
+// OP_CZ, and OP_PERM with tensor copies).
 
 // Shared memory of a pass block.  Tensor-copy passes (MODE 2): the landing
 // buffer of the copied tile (both planes, 64 KB), then the 8-byte exchange
@@ -1199,18 +1201,19 @@ __host__ __device__ constexpr size_t pass_buf_bytes(bool tma) {
 // (three blocks' worth), where their code does not spill, although the
 // shared memory of a tensor-copy block still allows only two per SM.
 template <bool BWD, int MODE, int V, int RE>
-__global__ void __launch_bounds__(kThreads, (RE == 3 || (RE == 0 && MODE == 2)) ? kBlocksPerSmTma : kBlocksPerSm)
+__global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) ? kBlocksPerSmTma : kBlocksPerSm)
     pass_kernel(const PassArgs a, const __grid_constant__ DevPass P, const __grid_constant__ CUtensorMap tm0,
                 const __grid_constant__ CUtensorMap tm1) {
   constexpr bool SLOW = MODE == 0;
   constexpr bool TMA = MODE == 2;
   constexpr bool REUP = RE == 1 || RE == 2;  // data re-uploading folded into the fused rotations
-  constexpr bool SPLIT = RE == 3;            // split form: OP_RY / OP_DIAG instead of OP_ROT / OP_CZ
+  constexpr bool SPLIT = RE == 3 || RE == 4;  // split form: OP_RY / OP_DIAG instead of OP_ROT / OP_CZ
   // split passes of circuits that fit one tile (n <= 12): every pass in one
   // launch, coefficients from the workspace (see MULTI below)
   constexpr bool MULTI = SPLIT && !TMA;
-  // fused CNOT layers (OP_PERM): fused-SU(2) passes loaded by tensor copies
-  constexpr bool CNOTF = TMA && RE == 0;
+  // fused CNOT layers (OP_PERM): passes loaded by tensor copies, in the
+  // fused SU(2) form (RE 0) or the split form (RE 4)
+  constexpr bool CNOTF = TMA && (RE == 0 || RE == 4);
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   float4* tile = reinterpret_cast<float4*>(smem_raw);  // MODE 2: the landing buffer
   float2* ex8 = reinterpret_cast<float2*>(smem_raw + kLandBytes);  // MODE 2: the exchange buffer
@@ -1291,6 +1294,9 @@ __global__ void __launch_bounds__(kThreads, (RE == 3 || (RE == 0 && MODE == 2)) 
             }
         } else if (op.kind == OP_DIAG) {
           diag_op<V>(op.a, re, im, *bc, P, a, C, op.d, op.c, tid, base_q, s_o);
+        } else if (op.kind == OP_PERM) {
+          if constexpr (CNOTF)
+            if (PP.perm_at[0] == 2) exchange8p<V>(op.a, op.b, re, im, ex8, tid, PP, 0, pco);
         }
       } else if (op.kind == OP_ROT) {
         int slot = op.d;
@@ -1361,6 +1367,9 @@ __global__ void __launch_bounds__(kThreads, (RE == 3 || (RE == 0 && MODE == 2)) 
         } else if (op.kind == OP_DIAG) {
           // the diagonal before layer 0 needs no un-applying: nothing reads the state after it
           if (op.c >= 0) diag_op<V>(op.a, re, im, *bc, P, a, C, op.d, op.c, tid, base_q, s_o);
+        } else if (op.kind == OP_PERM) {
+          if constexpr (CNOTF)
+            if (PP.perm_at[1] == 2) exchange8p<V>(op.b, op.a, re, im, ex8, tid, PP, 1, pco);
         }
       } else if (op.kind == OP_ROT) {
         // each rotation finishes the warp sum of the previous one

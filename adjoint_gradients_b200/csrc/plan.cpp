@@ -460,15 +460,38 @@ void flatten_plan(const Plan& p, std::vector<DevPass>* passes, bool split) {
     // diagonal that precedes layer 0 right after the encoding)
     std::vector<HostOp> ops;
     int ndiag = 0;
-    for (const HostOp& h : ps.ops) {
-      HostOp o = h;
-      if (split && o.kind == OP_ROT) o.kind = OP_RY;
-      if (split && o.kind == OP_CZ) o = {OP_DIAG, h.a, 0, h.c, ndiag++};
-      ops.push_back(o);
-      if (split && h.kind == OP_GEN) ops.push_back({OP_DIAG, h.a, 0, -1, ndiag++});
+    if (split && p.cnot) {
+      // fused CNOT layers: the pass's rotations (one layer of one set) are a
+      // segment of their own between two diagonal ops, D2 (the Rz(phi2)
+      // factors) before and D1 (the Rz(phi1) factors and the segment's
+      // frame) after; global diagonal index 4 l + 2 set + (0: D2, 1: D1)
+      int first_rot = -1, last_rot = -1;
+      for (int o = 0; o < (int)ps.ops.size(); ++o)
+        if (ps.ops[o].kind == OP_ROT) {
+          if (first_rot < 0) first_rot = o;
+          last_rot = o;
+        }
+      for (int o = 0; o < (int)ps.ops.size(); ++o) {
+        const HostOp& h = ps.ops[o];
+        const int dbase = 4 * h.c + 2 * ps.set_id;
+        if (o == first_rot) ops.push_back({OP_DIAG, h.a, 0, dbase, ndiag++});
+        HostOp x = h;
+        if (x.kind == OP_ROT) x.kind = OP_RY;
+        ops.push_back(x);
+        if (o == last_rot) ops.push_back({OP_DIAG, h.a, 0, dbase + 1, ndiag++});
+      }
+    } else {
+      for (const HostOp& h : ps.ops) {
+        HostOp o = h;
+        if (split && o.kind == OP_ROT) o.kind = OP_RY;
+        if (split && o.kind == OP_CZ) o = {OP_DIAG, h.a, 0, h.c, ndiag++};
+        ops.push_back(o);
+        if (split && h.kind == OP_GEN) ops.push_back({OP_DIAG, h.a, 0, -1, ndiag++});
+      }
     }
     d.nops = (int)ops.size();
     d.ndiag = ndiag;
+    d.cnot = p.cnot ? 1 : 0;
     d.load_phase = ps.load_phase;
     d.store_phase = ps.store_phase;
     d.gen = ps.gen ? 1 : 0;
@@ -490,7 +513,7 @@ void flatten_plan(const Plan& p, std::vector<DevPass>* passes, bool split) {
     // the next diagonal op (all of that op's layer)
     d.rs_layer = -1;
     d.rs_mask = 0;
-    if (split && ps.ckpt >= 0) {
+    if (split && ps.ckpt >= 0 && !p.cnot) {  // (fused CNOT layers: exact state at every pass boundary)
       bool found = false;
       for (size_t pj = pi + 1; pj < p.passes.size() && !found; ++pj)
         for (const HostOp& h : p.passes[pj].ops) {

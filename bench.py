@@ -58,7 +58,7 @@ def kernel_sources_digest():
     import hashlib
 
     h = hashlib.sha256()
-    for rel in ("kernels.cu", "device_plan.h", "plan.cpp"):
+    for rel in ("pass_kernel.cuh", "pass_split.cu", "kernels.cu", "device_plan.h", "plan.cpp"):
         with open(os.path.join(ROOT, "adjoint_gradients_b200", "csrc", rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -134,7 +134,10 @@ def algorithmic_counts(ctx, w, B, f64=False, cnot_passes_per_layer=0):
     N = 1 << w.n
     amp = B * N
     rots = w.n * w.L
-    if ctx.split_form:  # one diagonal op per layer boundary (forward: also the one before layer 0)
+    if ctx.split_form and ctx.cnot_fused:  # fused CNOT schedule: two diagonal ops per layer and qubit set
+        fma_f = FMA_FWD_PER_RY * rots + FMA_FWD_PER_DIAG * 4 * w.L
+        fma_b = FMA_BWD_PER_RY * rots + FMA_BWD_PER_DIAG * 4 * w.L
+    elif ctx.split_form:  # one diagonal op per layer boundary (forward: also the one before layer 0)
         # fp64 mode keeps one sample per tile: its forward factor is not shared by two lanes (4 + 4)
         fma_f = FMA_FWD_PER_RY * rots + (8 if f64 else FMA_FWD_PER_DIAG) * (w.L + 1)
         fma_b = FMA_BWD_PER_RY * rots + FMA_BWD_PER_DIAG * w.L
