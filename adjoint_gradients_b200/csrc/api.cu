@@ -65,6 +65,7 @@ struct qml_ctx {
   std::vector<DevPass> dpass_split;
   std::vector<int> undo;  // split form: [L][n] backward un-apply order of each layer's qubits
   size_t smem = 0;
+  size_t smem_multi = 0;  // one-launch split passes of single-tile circuits
   bool probed = false, dev_ok = false;
   bool slow = false;  // the plan puts a batch-unit bit in registers (n < 5)
   int region = 0;     // constant-memory coefficient region
@@ -168,6 +169,7 @@ void ensure_device(qml_ctx* c) {
   const int mode = tma ? 2 : c->slow ? 0 : 1;
   // the function attribute is shared by all contexts: set it for the largest pass
   const size_t smem_thr = pass_smem_bytes(kMaxSlots, false), smem_tma = pass_smem_bytes(kMaxSlots, true);
+  c->smem_multi = pass_multi_smem_bytes();
   c->smem = tma ? smem_tma : smem_thr;
   cudaDeviceProp prop;
   if (cudaGetDeviceProperties(&prop, c->device) != cudaSuccess) {
@@ -180,7 +182,7 @@ void ensure_device(qml_ctx* c) {
   DeviceGuard g(c->device);
   c->sms = prop.multiProcessorCount;
   int of = 0, ob = 0;
-  if (set_pass_smem_attr(smem_thr, smem_tma) != cudaSuccess || pass_occupancy(false, mode, c->smem, &of) != cudaSuccess ||
+  if (set_pass_smem_attr(std::max(smem_thr, c->smem_multi), smem_tma) != cudaSuccess || pass_occupancy(false, mode, c->smem, &of) != cudaSuccess ||
       pass_occupancy(true, mode, c->smem, &ob) != cudaSuccess || of < 1 || ob < 1) {
     cudaGetLastError();
     c->dev_ok = false;
@@ -698,7 +700,7 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
     a.coef = cf;
     a.n_tiles = (int)(((a.U + (1ll << dp.unit_bits) - 1) >> dp.unit_bits) << dp.n_out);
     static const PassMaps none{};
-    e = launch_pass(false, a, dp, none, c->grid_fwd, c->smem, s);
+    e = launch_pass(false, a, dp, none, c->grid_fwd, c->smem_multi, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
     ++c->launches;
     sp.passes = 1;  // the span times one launch
@@ -787,7 +789,7 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
     a.rscale = at<float>(c, c->lay.rscale);
     a.n_tiles = (int)(((a.U + (1ll << dp.unit_bits) - 1) >> dp.unit_bits) << dp.n_out);
     static const PassMaps none{};
-    e = launch_pass(true, a, dp, none, c->grid_bwd, c->smem, s);
+    e = launch_pass(true, a, dp, none, c->grid_bwd, c->smem_multi, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;
     ++c->launches;
     sp.passes = 1;  // the span times one launch

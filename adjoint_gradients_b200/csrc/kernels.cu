@@ -274,6 +274,8 @@ size_t pass_smem_bytes(int max_slots, bool tma) {
   return pass_buf_bytes(tma) + sizeof(BlockCtx) + (size_t)(kThreads / 32) * max_slots * 3 * sizeof(float);
 }
 
+size_t pass_multi_smem_bytes() { return multi_stage_offset() + sizeof(MultiStage); }
+
 cudaError_t set_pass_smem_attr(size_t smem_thr, size_t smem_tma) {
   cudaError_t e = pass_split_attr(smem_thr, smem_tma);
   if (e == cudaSuccess) e = pass_fused_attr(smem_thr, smem_tma);

@@ -67,6 +67,9 @@ struct PassArgs {
 
 // Dynamic shared memory of a pass block (tma: tensor-copy passes).
 size_t pass_smem_bytes(int max_slots, bool tma);
+// The same for the one-launch split passes of single-tile circuits (they
+// also stage each pass's ops and coefficients).
+size_t pass_multi_smem_bytes();
 
 // Register layouts for tests: per (phase, variant) the tile bit of each of the
 // 7 thread-index bits and 5 register-index bits, then the 12 slot weights and

@@ -1194,6 +1194,22 @@ __host__ __device__ constexpr size_t pass_buf_bytes(bool tma) {
   return tma ? kLandBytes + kExch8Bytes : (size_t)kSmemSlots * sizeof(float4);
 }
 
+// Split passes of single-tile circuits (all passes in one launch): the ops
+// and coefficients of the running pass, staged after the block's context and
+// accumulators (the launch asks for pass_stage_bytes() more shared memory).
+struct MultiStage {
+  CoefRegion coef;
+  DevOp ops[kMaxOps];
+  int nops;
+};
+__host__ __device__ constexpr size_t multi_stage_offset() {
+  return (pass_buf_bytes(false) + sizeof(BlockCtx) + (size_t)(kThreads / 32) * kMaxSlots * 3 * sizeof(float) + 15) &
+         ~(size_t)15;
+}
+__device__ __forceinline__ MultiStage* multi_stage(unsigned char* smem) {
+  return reinterpret_cast<MultiStage*>(smem + multi_stage_offset());
+}
+
 // Register budget: the split-form passes (tensor copies, and the one-launch
 // passes of single-tile circuits) and the fused-SU(2) tensor-copy passes
 // (CNOT entanglers, with their permuted exchanges) may use up to 255
@@ -1271,11 +1287,11 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
 
   // The ops of one pass on the registers, forward order (PP: the pass, C: its
   // coefficients; the layout is P's, the same for every pass of a launch).
-  auto run_fwd_ops = [&](const DevPass& PP, const CoefRegion* C, uint32_t base_q, uint32_t s_o, uint32_t unit_base,
+  auto run_fwd_ops = [&](const DevPass& PP, const auto& OPS, int nops, const CoefRegion* C, uint32_t base_q,
+                         uint32_t s_o, uint32_t unit_base,
                          float2 (&re)[kPos], float2 (&im)[kPos], bool pf_next, auto&& prefetch_next) {
-    const int nops = PP.nops;
     for (int oi = 0; oi < nops; ++oi) {
-      const DevOp op = PP.ops[oi];
+      const DevOp op = OPS[oi];
       if (op.kind == OP_EXCH) {
         if constexpr (TMA) exchange8<V>(op.a, op.b, re, im, ex8, tid);
         else exchange<V>(op.a, op.b, re, im, tile, tid);
@@ -1332,11 +1348,12 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
   };
 
   // The ops of one pass in reverse (un-applied), with the gradient sums into acc.
-  auto run_bwd_ops = [&](const DevPass& PP, const CoefRegion* C, uint32_t base_q, uint32_t s_o, uint32_t unit_base,
+  auto run_bwd_ops = [&](const DevPass& PP, const auto& OPS, int nops, const CoefRegion* C, uint32_t base_q,
+                         uint32_t s_o, uint32_t unit_base,
                          float2 (&re)[kPos], float2 (&im)[kPos], bool pf_next, auto&& prefetch_next) {
     const int pacc = PP.nslots * 3;  // row stride of the pass's sums
-    for (int oi = PP.nops - 1; oi >= 0; --oi) {
-      const DevOp op = PP.ops[oi];
+    for (int oi = nops - 1; oi >= 0; --oi) {
+      const DevOp op = OPS[oi];
       if (op.kind == OP_EXCH) {
         if constexpr (TMA) exchange8<V>(op.b, op.a, re, im, ex8, tid);
         else exchange<V>(op.b, op.a, re, im, tile, tid);
@@ -1425,6 +1442,21 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
       }
     }
     auto none = []() {};
+    // each pass's ops and coefficients are staged in shared memory before
+    // the pass runs (read from global memory they would stall every op)
+    MultiStage* stg = multi_stage(smem_raw);
+    auto stage = [&](int pi) {
+      __syncthreads();  // the previous pass is done with the stage
+      const DevPass& PP = a.passes[pi];
+      const int* so = reinterpret_cast<const int*>(PP.ops);
+      int* dop = reinterpret_cast<int*>(stg->ops);
+      for (int i = tid; i < kMaxOps * 5; i += kThreads) dop[i] = so[i];
+      const float4* sc = reinterpret_cast<const float4*>(a.coef + pi);
+      float4* dc = reinterpret_cast<float4*>(&stg->coef);
+      for (int i = tid; i < (int)(sizeof(CoefRegion) / 16); i += kThreads) dc[i] = sc[i];
+      if (tid == 0) stg->nops = PP.nops;
+      __syncthreads();
+    };
     for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x) {
       uint32_t base_q, base_a, unit_base;
       tile_base(P, t, &base_q, &base_a, &unit_base);
@@ -1436,7 +1468,8 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
         else mem_op<false, SLOW, V, M_LOAD>(P0.load_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
         for (int pi = 0; pi < a.npass; ++pi) {
           const DevPass& PP = a.passes[pi];
-          run_fwd_ops(PP, a.coef + pi, base_q, s_o, unit_base, re, im, false, none);
+          stage(pi);
+          run_fwd_ops(PP, stg->ops, stg->nops, &stg->coef, base_q, s_o, unit_base, re, im, false, none);
           if (PP.ckpt >= 0)
             mem_op<false, SLOW, V, M_CKPT_STORE>(PP.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im, PP.ckpt);
         }
@@ -1452,8 +1485,8 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
             mem_op<true, SLOW, V, M_CKPT_RESTORE>(PP.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im,
                                                   PP.ckpt, a.rscale ? __ldg(a.rscale + pi) : 1.f);
           for (int i = tid; i < kWarps * kMaxSlots * 3; i += kThreads) acc[i] = 0.f;
-          __syncthreads();
-          run_bwd_ops(PP, a.coef + pi, base_q, s_o, unit_base, re, im, false, none);
+          stage(pi);
+          run_bwd_ops(PP, stg->ops, stg->nops, &stg->coef, base_q, s_o, unit_base, re, im, false, none);
           __syncthreads();
           const int pn = PP.nslots * 3;
           float* row = a.partials + PP.partial_off + (size_t)blockIdx.x * pn;
@@ -1526,7 +1559,7 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
       } else if (have_pf) load_prefetched<V>(P.load_phase, re, im, tile, tid);
       else mem_op<false, SLOW, V, M_LOAD>(P.load_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
       if (pf_next && pf_at < 0) prefetch_next();
-      run_fwd_ops(P, creg, base_q, s_o, unit_base, re, im, pf_next, prefetch_next);
+      run_fwd_ops(P, P.ops, P.nops, creg, base_q, s_o, unit_base, re, im, pf_next, prefetch_next);
       if (P.ckpt >= 0) mem_op<false, SLOW, V, M_CKPT_STORE>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im, P.ckpt);
       if (P.last) mem_op<false, SLOW, V, M_STORE_STD>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
       else mem_op<false, SLOW, V, M_STORE>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
@@ -1537,7 +1570,7 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
       if (!TMA && P.ckpt >= 0)
         mem_op<true, SLOW, V, M_CKPT_RESTORE>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im, P.ckpt, rs);
       if (pf_next && pf_at < 0) prefetch_next();
-      run_bwd_ops(P, creg, base_q, s_o, unit_base, re, im, pf_next, prefetch_next);
+      run_bwd_ops(P, P.ops, P.nops, creg, base_q, s_o, unit_base, re, im, pf_next, prefetch_next);
       if (!P.gen) mem_op<true, SLOW, V, M_STORE>(P.load_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
     }
     have_pf = pf_next;
