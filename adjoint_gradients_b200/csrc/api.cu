@@ -133,6 +133,11 @@ struct qml_ctx {
   } hg;
   unsigned gen = 1;
   cudaStream_t cap = nullptr;  // capture stream of the host-step graph
+  // the theta buffer (and settings generation) the fp32 coefficient tables
+  // were last prepared from by a forward call; the backward of the same
+  // buffer reuses them
+  const void* prep_theta = nullptr;
+  unsigned prep_gen = 0;
   bool f64 = false;       // fp64 compute mode (qml_create_f64)
   // host-side fault injection for tests of the error paths (QML_FAULT at create)
   enum Fault { FAULT_NONE, FAULT_ALLOC, FAULT_CKPT, FAULT_NAN } fault = FAULT_NONE;
@@ -461,6 +466,7 @@ int sub_variant(int l, int L) { return (l == 0 ? 2 : 0) + (l == L - 1 ? 1 : 0); 
 
 qml_status run_forward_cnot(qml_ctx* c, const float* theta, const float* x, int B, float2* psi, float* expect,
                             cudaStream_t s) {
+  c->prep_theta = nullptr;  // the per-layer tables below overwrite the prepared ones
   const int n = c->cfg.n_qubits, L = c->cfg.n_layers, cb = c->cfg.ckpt_block;
   if (c->ws_bytes < c->lay.base_total) return QML_ERR_WORKSPACE;
   cudaError_t e = upload_sub(c, s);
@@ -545,6 +551,7 @@ qml_status run_forward_cnot(qml_ctx* c, const float* theta, const float* x, int 
 
 qml_status run_backward_cnot(qml_ctx* c, const float* theta, const float* x, int B, float2* psi, float2* lam,
                              const float* g, float* grad, cudaStream_t s) {
+  c->prep_theta = nullptr;
   const int n = c->cfg.n_qubits, L = c->cfg.n_layers, cb = c->cfg.ckpt_block;
   if (c->ws_bytes < c->lay.base_total) return QML_ERR_WORKSPACE;
   for (int m = 0; m < c->plan.n_ckpt; ++m)
@@ -665,6 +672,8 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
   const int P = (int)passes.size();
   CoefRegion* cf = at<CoefRegion>(c, c->lay.coef_fwd);
   cudaError_t e = prep_coefficients(c, theta, s);
+  c->prep_theta = e == cudaSuccess ? theta : nullptr;
+  c->prep_gen = c->gen;
   if (e == cudaSuccess && c->fault == qml_ctx::FAULT_NAN)  // injected: the first rotation's coefficients become NaN
     e = cudaMemsetAsync(cf, 0xff, sizeof(float4), s);
   if (e != cudaSuccess) return QML_ERR_CUDA;
@@ -740,8 +749,12 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
   for (int m = 0; m < c->plan.n_ckpt; ++m)
     if (c->ckpt_batch[m] != B) return QML_ERR_CKPT_MISMATCH;
   CoefRegion* ci = at<CoefRegion>(c, c->lay.coef_inv);
-  cudaError_t e = prep_coefficients(c, theta, s);
+  // the forward call that produced psi prepared the tables of both
+  // directions from the same theta: reuse them
+  const bool reuse = c->prep_theta == theta && c->prep_gen == c->gen;
+  cudaError_t e = reuse ? cudaSuccess : prep_coefficients(c, theta, s);
   if (e != cudaSuccess) return QML_ERR_CUDA;
+  if (reuse) c->launches -= split ? 4 : 1;
   if (c->obs_terms.empty()) {
     e = launch_bwd_init(psi, lam, g, B, n, s);
   } else {

@@ -149,7 +149,11 @@ QML_API qml_status qml_forward_expect(qml_ctx* ctx, const float* theta_dev, cons
  *   lambda_dev  [B][2^n] complex64 working memory, clobbered
  *   (psi_dev and lambda_dev 16-byte aligned, as for the forward pass)
  *   dLdE_dev    [B] float32, dL/dE per sample
- *   grad_dev    [L][n][3] float32, out (overwritten): sum_b dL/dE[b] dE[b]/dtheta */
+ *   grad_dev    [L][n][3] float32, out (overwritten): sum_b dL/dE[b] dE[b]/dtheta
+ * theta_dev must hold the angles of the forward call that produced psi_dev
+ * (the gradient is that circuit's); when it is the same buffer as in the
+ * context's last forward call, with no setter in between, the gate tables
+ * that call prepared for both directions are reused. */
 QML_API qml_status qml_backward_adjoint(qml_ctx* ctx, const float* theta_dev, const float* x_dev, int B,
                                 float* psi_dev, float* lambda_dev, const float* dLdE_dev,
                                 float* grad_dev, void* stream);
