@@ -196,16 +196,36 @@ __device__ void rot_chunk(const Pass64Args& a, const DevPass& P, const Ctx64& cx
     }
   }
   if (BWD) {
+    // warp sums of the chunk's 3K terms as one reduce-scatter: the terms sit
+    // in 16 slots (the unused ones zero); each xor step sends half of a
+    // lane's remaining slots to its partner and adds the other half, so after
+    // four steps lane l holds slot ((l >> 1) & 15) summed over 16 lanes, and
+    // a last step completes it (16 shuffles for up to 9 terms, instead of 5
+    // per term)
+    double r[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) r[i] = 0.0;
 #pragma unroll
     for (int i = 0; i < K; ++i) {
-      const double rx = warp_sum(sx[i]), ry = warp_sum(sy[i]), rz = warp_sum(sz[i]);
-      if (lane == 0) {
-        double* d = acc + ((size_t)warp * kMaxSlots + s0 + i) * 3;
-        d[0] += rx;
-        d[1] += ry;
-        d[2] += rz;
+      r[3 * i + 0] = sx[i];
+      r[3 * i + 1] = sy[i];
+      r[3 * i + 2] = sz[i];
+    }
+#pragma unroll
+    for (int st = 0; st < 4; ++st) {
+      const int half = 8 >> st, off = 16 >> st;
+      const bool up = (lane & off) != 0;  // keep the upper half of the remaining slots
+#pragma unroll
+      for (int i = 0; i < half; ++i) {
+        const double send = up ? r[i] : r[i + half];
+        const double got = __shfl_xor_sync(0xffffffffu, send, off);
+        r[i] = (up ? r[i + half] : r[i]) + got;
       }
     }
+    const double v = r[0] + __shfl_xor_sync(0xffffffffu, r[0], 1);
+    // lane l now holds the full sum of slot (l>>4)*8 + ((l>>3)&1)*4 + ((l>>2)&1)*2 + ((l>>1)&1)
+    const int slot = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+    if ((lane & 1) == 0 && slot < 3 * K) acc[((size_t)warp * kMaxSlots + s0 + slot / 3) * 3 + slot % 3] += v;
   }
 }
 
