@@ -557,20 +557,20 @@ def run_ours(args):
                          f"{'fused into the rotation passes' if ctx.cnot_fused else 'one gather pass per layer'})"
                          if args.entangler == "cnot" else
                          f"CZ {args.entangler} ({len(bonds)} bonds)"),
-           "reupload": bool(args.reupload),
-           "cuda_graph": graph is not None,
-           "peak_hbm_bytes": int(torch.cuda.max_memory_allocated(dev))}
+           "reupload": bool(args.reupload)}
+    # how this arm ran (kept out of config, which both arms report alike)
+    run = {"cuda_graph": graph is not None, "peak_hbm_bytes": int(torch.cuda.max_memory_allocated(dev))}
     if w.samples_per_epoch:
-        cfg["s_per_epoch"] = w.samples_per_epoch / (value / world)
-        cfg["epoch"] = f"{w.samples_per_epoch} samples per GPU at the measured samples/s (mini-batch {B})"
+        run["s_per_epoch"] = w.samples_per_epoch / (value / world)
+        run["epoch"] = f"{w.samples_per_epoch} samples per GPU at the measured samples/s (mini-batch {B})"
     if epoch is not None:
-        cfg["epoch_run"] = epoch
+        run["epoch_run"] = epoch
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64" if f64 else "f32", "data": "synthetic",
-            "config": cfg,
+            "config": cfg, "run": run,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
             "clocks": clk,
         }
