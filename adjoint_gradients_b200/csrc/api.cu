@@ -338,7 +338,7 @@ T* at(qml_ctx* c, size_t off) {
 bool use_split(const qml_ctx* c) { return !c->f64 && !c->reupload && (!c->cnot || c->cnot_fused); }
 // CNOT entanglers through the fused schedule (the generic pass loop), or the
 // one-layer schedules with a gather per layer
-bool cnot_fused_now(const qml_ctx* c) { return c->cnot && c->cnot_fused && !c->reupload && !c->f64; }
+bool cnot_fused_now(const qml_ctx* c) { return c->cnot && c->cnot_fused && !c->reupload; }
 // fp64 contexts: the same rule
 bool use_split64(const qml_ctx* c) { return c->f64 && !c->reupload && !c->cnot; }
 
@@ -829,8 +829,8 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
 // fp64 tiles: the schedule's tile qubits, less the highest qubit the pass
 // does not rotate when the tile has 12 (2^11-position tiles let two blocks
 // share an SM; a passive qubit can leave the tile because CZ is diagonal).
-uint32_t f64_tile_mask(const DevPass& dp, int n) {
-  uint32_t m = 0, rot = 0;
+uint32_t f64_tile_mask(const DevPass& dp, int n, uint32_t kept = 0) {
+  uint32_t m = 0, rot = kept;
   for (int b = 0; b < kTileBits; ++b)
     if (dp.tile_q[b] >= 0 && dp.tile_q[b] < n) m |= 1u << dp.tile_q[b];
   for (int s = 0; s < dp.nslots; ++s) rot |= 1u << (dp.slot_lq[s] % n);
@@ -844,7 +844,12 @@ void set_f64_tiles(qml_ctx* c) {
   c->f64_mask.clear();
   c->f64_tmax = 1;
   for (const DevPass& dp : c->dpass) {
-    const uint32_t m = f64_tile_mask(dp, n);
+    // fused CNOT layers: the set a pass's permutation changes stays in its tile
+    uint32_t kept = 0;
+    for (int o = 0; o < dp.nops; ++o)
+      if (dp.ops[o].kind == OP_PERM)
+        for (int q : c->plan.sets[dp.ops[o].c]) kept |= 1u << q;
+    const uint32_t m = f64_tile_mask(dp, n, kept);
     c->f64_mask.push_back(m);
     c->f64_tmax = std::max(c->f64_tmax, __builtin_popcount(m));
   }
@@ -866,8 +871,11 @@ Pass64Args pass64_args(qml_ctx* c, const double* theta, const double* x, int B, 
   a.partials = at<double>(c, c->lay.partials);
   a.status = at<unsigned>(c, c->lay.status);
   a.reupload = c->reupload ? 1 : 0;
-  for (int q = 0; q < kMaxQubits; ++q) a.nb[q] = c->nb[q], a.nbhi[q] = c->nbhi[q];
+  for (int q = 0; q < kMaxQubits; ++q) a.nb[q] = c->cnot ? 0u : c->nb[q], a.nbhi[q] = c->cnot ? 0u : c->nbhi[q];
   a.L = c->cfg.n_layers;
+  if (c->cnot_fused)
+    for (int g = 0; g < 2; ++g)
+      for (int q = 0; q < kMaxQubits; ++q) a.perm_fwd[g][q] = c->cnot_map.inv[g][q], a.perm_bwd[g][q] = c->cnot_map.fwd[g][q];
   if (use_split64(c)) {
     a.srot = at<SplitRot>(c, c->lay.s_rot);
     a.slay = at<SplitLayer>(c, c->lay.s_lay);
@@ -1032,7 +1040,7 @@ qml_status run_backward64_cnot(qml_ctx* c, const double* theta, const double* x,
 
 qml_status run_forward64(qml_ctx* c, const double* theta, const double* x, int B, double2* psi, double* expect,
                          cudaStream_t s) {
-  if (c->cnot) return run_forward64_cnot(c, theta, x, B, psi, expect, s);
+  if (c->cnot && !cnot_fused_now(c)) return run_forward64_cnot(c, theta, x, B, psi, expect, s);
   Pass64Args a = pass64_args(c, theta, x, B, psi, nullptr);
   const bool split = use_split64(c);
   if (split) {
@@ -1057,7 +1065,7 @@ qml_status run_forward64(qml_ctx* c, const double* theta, const double* x, int B
 
 qml_status run_backward64(qml_ctx* c, const double* theta, const double* x, int B, double2* psi, double2* lam,
                           const double* g, double* grad, cudaStream_t s) {
-  if (c->cnot) return run_backward64_cnot(c, theta, x, B, psi, lam, g, grad, s);
+  if (c->cnot && !cnot_fused_now(c)) return run_backward64_cnot(c, theta, x, B, psi, lam, g, grad, s);
   const int n = c->cfg.n_qubits, L = c->cfg.n_layers;
   for (int m = 0; m < c->plan.n_ckpt; ++m)
     if (c->ckpt_batch[m] != B) return QML_ERR_CKPT_MISMATCH;
@@ -1385,6 +1393,7 @@ static void restore_default_plan(qml_ctx* c) {
   set_pass_entangler(p, c->bonds, &c->dpass);
   set_pass_entangler(p, c->bonds, &c->dpass_split);
   c->cnot_fused = false;
+  if (c->f64) set_f64_tiles(c);
   if (c->ws) drop_workspace(c);
 }
 
@@ -1455,9 +1464,9 @@ qml_status qml_set_entangler_cnot(qml_ctx* c, int n_pairs, const int* pairs) {
   c->plan1 = p1;
   c->cnot_pairs = v;
   c->cnot = true;
-  // fused schedule (fp32): M1 and M2 of every layer inside the rotation passes
+  // fused schedule: M1 and M2 of every layer inside the rotation passes
   bool fused = false;
-  if (!c->f64) {
+  {
     CnotLayers cl;
     Plan fp;
     if (factor_cnot_layer(n, v, &cl) && make_plan(n, c->cfg.n_layers, c->cfg.ckpt_block, &fp, &cl).empty()) {
@@ -1475,6 +1484,7 @@ qml_status qml_set_entangler_cnot(qml_ctx* c, int n_pairs, const int* pairs) {
     }
   }
   if (!fused && c->cnot_fused) restore_default_plan(c);
+  if (c->f64) set_f64_tiles(c);
   if (c->ws) drop_workspace(c);  // the schedule's device copies and the layout change with it
   compute_layout(c);  // the gathers need a second state buffer in the workspace
   return QML_OK;

@@ -50,6 +50,7 @@ struct Ctx64 {
   double4 coef[kMaxSlots];          // (ar, ai, br, bi): U forward, U^dagger backward; split form: (p, cot, 0, 0)
   double cs[kMaxQubits], sn[kMaxQubits];  // (cos, sin)(x/2) of the tile's sample
   double2 dlo[64], dhi[64];         // split form, diagonal op: factors of position bits 0-5 / 6-11
+  uint32_t pcol[kMaxQubits];        // fused CNOT layers: tile position of the gather map's image of each qubit
 };
 
 size_t f64_smem_bytes(bool bwd, int tmax) {
@@ -425,6 +426,58 @@ __global__ void __launch_bounds__(kT, BWD ? 2 : 3) pass64_kernel(const Pass64Arg
           }
         }
         __syncthreads();
+      } else if (!SPLIT && op.kind == OP_PERM) {
+        // fused CNOT layers (fused-SU(2) passes only): the tile's positions
+        // gathered through the factor's map G (forward M_g^-1, backward
+        // M_g): position v takes the position of G (idx(v) | base).  G
+        // changes only bits of this pass's qubit set, all in the tile, and
+        // the tile position of a qubit pattern is linear in it, so the
+        // source position is the xor of per-qubit columns (pcol: the tile
+        // position of G's image of each qubit's bit), those of v's bits and
+        // of the tile's out-of-tile bits.  psi, then lambda.
+        constexpr int kPer = (1 << 11) / kT;  // positions per thread (tiles of up to 2^11)
+        if (P2 > kPer * kT) {  // (fused CNOT plans have two qubit sets: 11-qubit tiles at most)
+          if (tid == 0) atomicOr(a.status, kErrBounds);
+          continue;
+        }
+        if (tid < n) {
+          // (constant indices into the parameter block: no pointer into it)
+          uint32_t img = 0;
+#pragma unroll
+          for (int q = 0; q < kMaxQubits; ++q)
+            if (q == tid)
+              img = op.c == 0 ? (BWD ? a.perm_bwd[0][q] : a.perm_fwd[0][q]) : (BWD ? a.perm_bwd[1][q] : a.perm_fwd[1][q]);
+          uint32_t u = 0;
+          for (int k = 0; k < T; ++k) u |= ((img >> cx.tq[k]) & 1u) << k;
+          cx.pcol[tid] = u;
+        }
+        __syncthreads();
+        uint32_t ub = 0;  // the out-of-tile bits' part, then this thread's fixed position bits
+        for (uint32_t r = base; r; r &= r - 1u) ub ^= cx.pcol[__ffs(r) - 1];
+        for (int k = 0; k < T && (1 << k) < kT; ++k)
+          if ((tid >> k) & 1) ub ^= cx.pcol[cx.tq[k]];
+        for (int plane = 0; plane < (BWD ? 2 : 1); ++plane) {
+          double2* tb = plane ? tl : tp;
+          double2 tv[kPer];
+#pragma unroll
+          for (int i = 0; i < kPer; ++i) {
+            const int v = tid + i * kT;
+            if (v >= P2) break;
+            uint32_t u = ub;
+#pragma unroll
+            for (int k = 0; k < 3; ++k)  // position bits 8-10 come from i (kT = 256)
+              if ((i >> k) & 1) u ^= cx.pcol[cx.tq[8 + k]];
+            tv[i] = tb[padp((int)u)];
+          }
+          __syncthreads();
+#pragma unroll
+          for (int i = 0; i < kPer; ++i) {
+            const int v = tid + i * kT;
+            if (v >= P2) break;
+            tb[padp(v)] = tv[i];
+          }
+          __syncthreads();
+        }
       } else if (!SPLIT && op.kind == OP_CZ) {
         for (int v = tid; v < P2; v += kT) {
           const uint32_t par = s_base ^ ((cx.s_off[v >> 5] >> (v & 31)) & 1u) ^ ((uint32_t)__popc(v & cm) & 1u);

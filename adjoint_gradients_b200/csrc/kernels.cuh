@@ -231,6 +231,11 @@ struct Pass64Args {
   const SplitLayer* slay;     // [L]
   const double2* dq;          // [L + 1][n][2] per-qubit diagonal factors of this direction
   const double* rscale;       // backward checkpoint pass: scale of the restored state (null: 1)
+  // fused CNOT layers (OP_PERM, factor g = op.c): the gather maps of the
+  // layer's factors on qubit bits, as columns (images of single qubits):
+  // forward M_g^-1, backward M_g
+  uint32_t perm_fwd[2][kMaxQubits];
+  uint32_t perm_bwd[2][kMaxQubits];
 };
 
 size_t pass64_smem_bytes(bool backward, int tmax);

@@ -301,7 +301,7 @@ class Context:
         need = self.lib.qml_debug_entangler_map(self._h, None, 0)
         buf = (ctypes.c_int * need)()
         self.lib.qml_debug_entangler_map(self._h, buf, need)
-        return bool(buf[1 + 4 * self.n]) and not self.reupload and self.precision == "fp32"
+        return bool(buf[1 + 4 * self.n]) and not self.reupload
 
     @property
     def entangler_bonds(self) -> int:

@@ -202,13 +202,14 @@ QML_API int qml_entangler_bonds(const qml_ctx* ctx);
  * n_pairs-1 in list order, e.g. the ladder (q, q+1).  The pages name CNOT
  * gates as the other entangler their kernels fuse by recomputing indices
  * ([Deep-dive] sec. 3.2).  A layer's CNOT list is a linear map M of the
- * index bits over GF(2).  fp32 contexts of 13..20 qubits (two qubit sets A,
- * B) whose map factors as M = M2 M1, M1 changing only A's bits and M2 only
- * B's (true whenever the A-to-A block of M is invertible, e.g. the ladder or
- * the ring), run fused: M1 and M2 are applied inside the rotation passes, as
- * a permutation of each tile's positions while it is read or in a layout
- * exchange, and each layer costs two passes with no gather through HBM.
- * Other contexts (other sizes, fp64, re-uploading, maps that do not factor)
+ * index bits over GF(2).  Contexts of 13..20 qubits (two qubit sets A, B)
+ * whose map factors as M = M2 M1, M1 changing only A's bits and M2 only B's
+ * (true whenever the A-to-A block of M is invertible, e.g. the ladder or the
+ * ring), run fused: M1 and M2 are applied inside the rotation passes, as a
+ * permutation of each tile's positions (fp32: while the tile is read or in a
+ * layout exchange; fp64: in the shared-memory tile), and each layer costs two
+ * passes with no gather through HBM.  Other contexts (other sizes,
+ * re-uploading, maps that do not factor)
  * run each layer's rotations as the fused passes of a one-layer schedule and
  * then one gather pass into a second state buffer (the workspace grows by B
  * * 2^n complex64, or complex128 in fp64).  Either way the schedule changes:

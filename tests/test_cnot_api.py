@@ -214,6 +214,7 @@ def test_fused_schedule_has_two_passes_per_layer():
 
 
 def test_unfactorable_maps_and_other_sizes_stay_on_the_gather_path():
+    """Maps whose first-set block is singular, and circuits of one or three qubit sets."""
     # SWAP(0, 9) from three CNOTs at n = 16 (sets 0-7 and 8-15): the first set's block of the map is
     # singular (qubit 0's new value comes from the second set only)
     lib, h = _ctx(16, 2, 2)
@@ -221,9 +222,9 @@ def test_unfactorable_maps_and_other_sizes_stay_on_the_gather_path():
     assert lib.qml_set_entangler_cnot(h, 3, _pairs(swap)) == qml.QML_OK
     assert _fused(lib, h)[0] == 0
     lib.qml_destroy(h)
-    for n, f64 in [(12, False), (21, False), (16, True)]:
+    for n, f64, fused in [(12, False, 0), (21, False, 0), (21, True, 0), (16, True, 1)]:
         lib, h = _ctx(n, 2, 2, f64=f64)
         ladder = [(q, q + 1) for q in range(n - 1)]
         assert lib.qml_set_entangler_cnot(h, len(ladder), _pairs(ladder)) == qml.QML_OK
-        assert _fused(lib, h)[0] == 0
+        assert _fused(lib, h)[0] == fused  # two qubit sets fuse in both precisions
         lib.qml_destroy(h)

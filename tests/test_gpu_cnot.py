@@ -114,7 +114,10 @@ def test_switching_back_to_cz_restores_the_chain():
 
 
 @pytest.mark.parametrize("n,L,B,ck,st,kind", [(5, 3, 3, 1, "fp64", "ladder"), (13, 3, 2, 1, "fp64", "ring"),
-                                              (14, 2, 3, 1, "bf16", "ladder"), (21, 2, 2, 1, "fp64", "ladder")])
+                                              (14, 2, 3, 1, "bf16", "ladder"), (21, 2, 2, 1, "fp64", "ladder"),
+                                              # two qubit sets: the layer maps inside the fp64 passes
+                                              (16, 4, 3, 2, "fp64", "ladder"), (19, 3, 2, 0, "fp32", "random"),
+                                              (20, 3, 1, 1, "bf16", "ring")])
 def test_cnot_fp64(n, L, B, ck, st, kind):
     """fp64 mode with CNOT lists: tolerances of the fp64 parity tests (1e-10 + 1e-9 |g| with fp64 or no
     slots; bf16 slots round the restarted state to 2^-8: 2e-2 + 1e-3 |g|)."""
