@@ -33,7 +33,11 @@ def sources():
 
 
 def headers():
-    return glob.glob(os.path.join(CSRC, "*.h*")) + [os.path.join(INCLUDE, "qml.h"), __file__]
+    # every header any source includes (.h, .hpp, .cuh): a change rebuilds every object
+    hs = []
+    for pat in ("*.h", "*.hpp", "*.cuh"):
+        hs += glob.glob(os.path.join(CSRC, pat))
+    return hs + [os.path.join(INCLUDE, "qml.h"), __file__]
 
 
 def _stale(target, deps):
