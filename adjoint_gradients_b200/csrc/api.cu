@@ -224,7 +224,10 @@ void compute_layout(qml_ctx* c) {
   l.coef_inv = take(sizeof(CoefRegion) * std::max(c->dpass.size(), c->sub[0].size()));
   l.enc = take(sizeof(float2) * 2 * U * n);
   l.dummy = take(sizeof(float2) * (size_t)N);
-  l.exp_partial = take(sizeof(double) * (c->f64 ? expect64_partial_count(Bm, n) : expect_partial_count(Bm, n)));
+  // (fp32: also room for one partial per 4096-position tile and sample, the Z0 epilogue's)
+  l.exp_partial = take(sizeof(double) * (c->f64 ? expect64_partial_count(Bm, n)
+                                                : std::max(expect_partial_count(Bm, n),
+                                                           (size_t)Bm << (n > kTileBits ? n - kTileBits : 0))));
   size_t nparts = 0;
   for (const DevPass& p : c->dpass) nparts += (size_t)c->grid_bwd * p.nslots * 3;
   l.partials = take((c->f64 ? sizeof(double) : sizeof(float)) * std::max<size_t>(1, nparts));
@@ -343,6 +346,10 @@ bool cnot_fused_now(const qml_ctx* c) { return c->cnot && c->cnot_fused && !c->r
 bool use_split64(const qml_ctx* c) { return c->f64 && !c->reupload && !c->cnot; }
 
 const std::vector<DevPass>& fp32_passes(const qml_ctx* c) { return use_split(c) ? c->dpass_split : c->dpass; }
+// The Z0 expectation fused into the last forward pass: split-form fp32
+// passes with the Z0 observable over the standard order (at most two qubit
+// sets: no working-state permutation), CZ entanglers.
+bool fused_z0(const qml_ctx* c) { return use_split(c) && !c->cnot && c->obs_terms.empty() && c->plan.n_sets <= 2; }
 
 // Readiness of a context for a call with batch B; f64 is the precision the
 // call is made for (a context computes in one precision only).
@@ -699,6 +706,10 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
   a.reupload = c->reupload ? 1 : 0;
   a.dq = split ? at<float2>(c, c->lay.s_dqf) : nullptr;
   a.rscale = nullptr;
+  // Z0 from the last pass's registers (tiles of one batch unit): per tile
+  // partials, then one fixed-order sum per sample
+  const bool epi = expect && fused_z0(c) && passes[P - 1].unit_bits == 0;
+  a.epart = epi ? at<double>(c, c->lay.exp_partial) : nullptr;
   c->launches += split ? 5 : 2;
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, false);
@@ -731,7 +742,12 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
   if (timed) span_end(c, s, &sp);
   e = convert_layout(c, psi, B, false, s);  // working-state order -> standard order
   if (e != cudaSuccess) return QML_ERR_CUDA;
-  if (expect) {
+  if (epi) {
+    c->launches += 1;
+    const int tps = 1 << (n > kTileBits ? n - kTileBits : 0);  // tiles per sample
+    e = launch_expect_final(at<double>(c, c->lay.exp_partial), tps, B, expect, at<unsigned>(c, c->lay.status), s);
+    if (e != cudaSuccess) return QML_ERR_CUDA;
+  } else if (expect) {
     c->launches += 2;
     e = launch_expectation(c, psi, B, expect, s);
     if (e != cudaSuccess) return QML_ERR_CUDA;

@@ -404,6 +404,12 @@ cudaError_t launch_expect(const float2* psi, int B, int n, double* partial, floa
   return cudaGetLastError();
 }
 
+cudaError_t launch_expect_final(const double* partial, int chunks, int B, float* E, unsigned* status,
+                               cudaStream_t s) {
+  expect_final_kernel<<<(B + 127) / 128, 128, 0, s>>>(partial, chunks, B, E, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_grad_reduce(const DevPass* passes, const int* slot_pass, const int* slot_index,
                                const float* partials, int grid, const float* theta, const double* gfix, int L,
                                int n, float* grad, unsigned* status, cudaStream_t s) {

@@ -63,6 +63,10 @@ struct PassArgs {
   const CoefRegion* coef;    // [npass] coefficients of this direction
   uint32_t cz_nb[kMaxQubits];    // CZ neighbours of each qubit (qubit mask)
   uint32_t cz_nbhi[kMaxQubits];  // CZ neighbours of each qubit above it (qubit mask)
+  // Z0 observable, working state in the standard order (at most two qubit
+  // sets), tiles without batch-unit bits:
+  double* epart;         // forward, last pass (non-null): per tile and sample, the partial sum of
+                         // |psi|^2 (1 - 2 b0) over the tile, at [sample][tile's out-of-tile index]
 };
 
 // Dynamic shared memory of a pass block (tma: tensor-copy passes).
@@ -144,6 +148,9 @@ cudaError_t launch_prep_enc(const float* x, int B, int n, float2* enc, cudaStrea
 cudaError_t launch_expect(const float2* psi, int B, int n, double* partial, float* E,
                           unsigned* status, cudaStream_t s);
 size_t expect_partial_count(int B, int n);
+// E[b] = the fixed-order sum of partial[b][0 .. chunks - 1] (fp64).
+cudaError_t launch_expect_final(const double* partial, int chunks, int B, float* E, unsigned* status,
+                               cudaStream_t s);
 // gfix: split form, [L][n][2] (scale of the sums, phi1) per rotation; null otherwise.
 cudaError_t launch_grad_reduce(const DevPass* passes, const int* slot_pass, const int* slot_index,
                                const float* partials, int grid, const float* theta, const double* gfix, int L,

@@ -453,6 +453,7 @@ struct BlockCtx {
   int tma_sel;               // plane 1 of the next tile comes through tm1
   uint32_t cz_w[kPhases][kThreads];  // per layout and thread: entangler terms of the thread bits
   uint32_t cz_n[kPhases][kThreads];  // per layout and thread: xor of the thread bits' neighbours
+  double ez[kThreads / 32][2];       // Z0 epilogue: per warp, the two samples' partial sums
 };
 
 // Qubit-space index and batch unit of (thread, register 0) in phase P.
@@ -744,6 +745,7 @@ __device__ __forceinline__ void mem_t(const PassArgs& a, const BlockCtx& bc, uin
   uint32_t aq, ut;
   thread_pos<P, V>(bc, tid, &aq, &ut);
   constexpr bool std_index = !(OP == M_LOAD || OP == M_STORE || OP == M_STORE_STD);
+  float ez0 = 0.f, ez1 = 0.f;  // M_STORE_STD with a.epart: sum of |psi|^2 (1 - 2 b0) of the two lanes
   if (std_index) aq |= base_q;
   else aq = thread_addr<P, V>(bc, tid) | base_a;
   ut += unit_base;
@@ -771,6 +773,9 @@ __device__ __forceinline__ void mem_t(const PassArgs& a, const BlockCtx& bc, uin
         a.buf0[(size_t)(2 * u) * a.N + i] = make_float2(re[j].x, im[j].x);
         if (2 * u + 1 < (uint32_t)a.B) a.buf0[(size_t)(2 * u + 1) * a.N + i] = make_float2(re[j].y, im[j].y);
       }
+      const float2 pr = __ffma2_rn(re[j], re[j], __fmul2_rn(im[j], im[j]));  // |psi|^2 of both lanes
+      if (i & 1u) ez0 -= pr.x, ez1 -= pr.y;
+      else ez0 += pr.x, ez1 += pr.y;
     } else if constexpr (OP == M_GEN) {  // forward only: angle-encoded product state
       float2 v = make_float2(0.f, 0.f);
       if (ok) {
@@ -803,6 +808,29 @@ __device__ __forceinline__ void mem_t(const PassArgs& a, const BlockCtx& bc, uin
         re[j].x = v.x * rs;
         im[j].x = v.y * rs;
       }
+    }
+  }
+  if constexpr (OP == M_STORE_STD) {
+    // Z0 epilogue: the tile's two partial sums (lanes x, y = samples 2u,
+    // 2u + 1) in a fixed order: warp butterfly, then the warps in order.
+    // slot: the tile's out-of-tile index (tiles of one unit, no unit bits).
+    if (a.epart) {
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        ez0 += __shfl_xor_sync(0xffffffffu, ez0, o);
+        ez1 += __shfl_xor_sync(0xffffffffu, ez1, o);
+      }
+      BlockCtx& w = const_cast<BlockCtx&>(bc);
+      if ((tid & 31) == 0) w.ez[tid >> 5][0] = ez0, w.ez[tid >> 5][1] = ez1;
+      __syncthreads();
+      if (tid == 0 && ut < (uint32_t)a.U) {
+        double s0 = 0.0, s1 = 0.0;
+        for (int k = 0; k < kThreads / 32; ++k) s0 += w.ez[k][0], s1 += w.ez[k][1];
+        const size_t tps = (size_t)1 << (n > kTileBits ? n - kTileBits : 0);  // tiles per sample
+        a.epart[(size_t)(2 * ut) * tps + (size_t)slot] = s0;
+        if (2 * ut + 1 < (uint32_t)a.B) a.epart[(size_t)(2 * ut + 1) * tps + (size_t)slot] = s1;
+      }
+      __syncthreads();
     }
   }
 }
@@ -1223,7 +1251,7 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
   constexpr bool SLOW = MODE == 0;
   constexpr bool TMA = MODE == 2;
   constexpr bool REUP = RE == 1 || RE == 2;  // data re-uploading folded into the fused rotations
-  constexpr bool SPLIT = RE == 3 || RE == 4;  // split form: OP_RY / OP_DIAG instead of OP_ROT / OP_CZ
+  constexpr bool SPLIT = RE >= 3;            // split form: OP_RY / OP_DIAG instead of OP_ROT / OP_CZ
   // split passes of circuits that fit one tile (n <= 12): every pass in one
   // launch, coefficients from the workspace (see MULTI below)
   constexpr bool MULTI = SPLIT && !TMA;
@@ -1474,7 +1502,9 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
             mem_op<false, SLOW, V, M_CKPT_STORE>(PP.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im, PP.ckpt);
         }
         const DevPass& PL = a.passes[a.npass - 1];
-        if (PL.last) mem_op<false, SLOW, V, M_STORE_STD>(PL.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
+        if (PL.last)
+          mem_op<false, SLOW, V, M_STORE_STD>(PL.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im,
+                                              t & ((1 << PL.n_out) - 1));
         else mem_op<false, SLOW, V, M_STORE>(PL.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
       } else {
         const DevPass& PL = a.passes[a.npass - 1];
@@ -1548,8 +1578,11 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
         if (mem_ph == 0) restore_tma_t<0, V>(a, *bc, P, tid, base_q, unit_base, tb, P.ckpt, rs);
         else restore_tma_t<1, V>(a, *bc, P, tid, base_q, unit_base, tb, P.ckpt, rs);
       }
-      if (CNOTF && P.perm_at[BWD] == 1) load_tma_perm<V>(mem_ph, re, im, tb, P, BWD ? 1 : 0, pco, tid);
-      else load_tma<V>(mem_ph, re, im, tb, P, tid);
+      if (CNOTF && P.perm_at[BWD] == 1) {
+        load_tma_perm<V>(mem_ph, re, im, tb, P, BWD ? 1 : 0, pco, tid);
+      } else {
+        load_tma<V>(mem_ph, re, im, tb, P, tid);
+      }
       __syncthreads();  // every thread has its positions: the landing buffer is free
       if (pf_next && tid == 0) tma_load_tile(&tm0, &tm1, bc->tma_sel, bc->tma_c, tile_s, mbar);
     }
@@ -1561,7 +1594,9 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
       if (pf_next && pf_at < 0) prefetch_next();
       run_fwd_ops(P, P.ops, P.nops, creg, base_q, s_o, unit_base, re, im, pf_next, prefetch_next);
       if (P.ckpt >= 0) mem_op<false, SLOW, V, M_CKPT_STORE>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im, P.ckpt);
-      if (P.last) mem_op<false, SLOW, V, M_STORE_STD>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
+      if (P.last)
+        mem_op<false, SLOW, V, M_STORE_STD>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im,
+                                            t & ((1 << P.n_out) - 1));
       else mem_op<false, SLOW, V, M_STORE>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
     } else {
       if (TMA) {
