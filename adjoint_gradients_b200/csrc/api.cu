@@ -379,7 +379,12 @@ const PassMaps* pass_maps_for(qml_ctx* c, const DevPass& dp, bool backward, int 
   qml_ctx::MapEntry m{};
   m.view = dp, m.backward = backward, m.B = B, m.buf0 = buf0, m.buf1 = buf1;
   if (encode_pass_maps(dp, c->cfg.n_qubits, B, backward, buf0, buf1, &m.maps) != cudaSuccess) return nullptr;
-  if (c->maps.size() >= 64) c->maps.clear();
+  // A plan has a few tile views, and a call rotates through at most three
+  // buffers (the CNOT gather's backward: psi, lambda, scratch), so the
+  // entries in use number at most views x 6 ordered buffer pairs x 2
+  // directions per batch size: well under the cap, which only bounds a
+  // context that sees many different buffers.
+  if (c->maps.size() >= 256) c->maps.clear();
   c->maps.push_back(m);
   return &c->maps.back().maps;
 }
