@@ -720,6 +720,15 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
   const bool timed = span_begin(c, s, &sp, false);
   if (split && !passes[0].tma) {  // one tile holds the state: every pass in one launch
     const DevPass& dp = passes[0];
+    // One sample per batch unit with the amplitude in a lane pair (half the
+    // work per tile of the two-sample form) for the chain from the encoding
+    // to the standard order, CZ entanglers: taken where it gives more tiles
+    // than the two-sample form (a tile of one batch unit, or batches that
+    // fill more than one tile), not for the single tile of a small batch.
+    const long long upt = 1ll << dp.unit_bits;
+    const bool more_tiles = (B + upt - 1) / upt > (a.U + upt - 1) / upt;
+    a.zf = (passes[0].gen && passes[P - 1].last && !c->cnot && !dp.slow && more_tiles) ? 1 : 0;
+    if (a.zf) a.U = B;
     a.npass = P;
     a.passes = at<DevPass>(c, c->lay.passes_split);
     a.coef = cf;

@@ -281,6 +281,7 @@ cudaError_t set_pass_smem_attr(size_t smem_thr, size_t smem_tma) {
   if (e == cudaSuccess) e = pass_fused_attr(smem_thr, smem_tma);
   if (e == cudaSuccess) e = pass_reup_attr(smem_thr, smem_tma);
   if (e == cudaSuccess) e = pass_csplit_attr(smem_thr, smem_tma);
+  if (e == cudaSuccess) e = pass_single_attr(smem_thr, smem_tma);
   return e;
 }
 
@@ -315,6 +316,8 @@ cudaError_t launch_pass(bool backward, const PassArgs& a, const DevPass& p, cons
       if (p.tile_q[b] < 0) form = 2;
   }
   if (form == 3 && p.cnot) form = 4;
+  if (form == 3 && !backward && a.npass > 0 && a.zf) form = 5;
+  if (form == 5) return pass_single_launch(backward, mode, p.variant, form, a, p, maps, grid, smem, coef, s);
   if (form == 4) return pass_csplit_launch(backward, mode, p.variant, form, a, p, maps, grid, smem, coef, s);
   if (form == 3) return pass_split_launch(backward, mode, p.variant, form, a, p, maps, grid, smem, coef, s);
   if (form == 0) return pass_fused_launch(backward, mode, p.variant, form, a, p, maps, grid, smem, coef, s);

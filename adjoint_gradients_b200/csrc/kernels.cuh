@@ -61,6 +61,8 @@ struct PassArgs {
   int npass;                 // passes of the launch (0: one pass, the kernel's parameter)
   const DevPass* passes;     // [npass] device copy, forward order
   const CoefRegion* coef;    // [npass] coefficients of this direction
+  int zf;                    // forward, npass > 0: one sample per batch unit, the amplitude (re, im) in a
+                             // lane pair (form 5; U = B); the chain runs from the encoding to the standard order
   uint32_t cz_nb[kMaxQubits];    // CZ neighbours of each qubit (qubit mask)
   uint32_t cz_nbhi[kMaxQubits];  // CZ neighbours of each qubit above it (qubit mask)
   // Z0 observable, working state in the standard order (at most two qubit
@@ -105,7 +107,8 @@ cudaError_t launch_pass(bool backward, const PassArgs& a, const DevPass& p, cons
 // pass_fused.cu: fused SU(2) form, CZ or CNOT; pass_reup.cu: re-uploading;
 // pass_csplit.cu: split form of the fused CNOT schedule).
 // form: 0 fused SU(2), 1 and 2 re-uploading (2: per register pair), 3 split,
-// 4 split with CNOT permutations.
+// 4 split with CNOT permutations, 5 the split form's one-launch forward with
+// one sample per batch unit (pass_single.cu).
 #define QML_PASS_UNIT_DECL(NAME)                                                                        \
   cudaError_t NAME##_launch(bool backward, int mode, int variant, int form, const PassArgs& a,           \
                             const DevPass& p, const PassMaps& maps, int grid, size_t smem,               \
@@ -115,6 +118,7 @@ QML_PASS_UNIT_DECL(pass_split)
 QML_PASS_UNIT_DECL(pass_fused)
 QML_PASS_UNIT_DECL(pass_reup)
 QML_PASS_UNIT_DECL(pass_csplit)
+QML_PASS_UNIT_DECL(pass_single)
 #undef QML_PASS_UNIT_DECL
 // Full SU(2) coefficients of every pass slot: cf forward, ci backward ([P] regions).
 cudaError_t launch_prep_pass_coef(const DevPass* passes, int n_passes, const float* theta, CoefRegion* cf,

@@ -167,6 +167,36 @@ __device__ __forceinline__ void ry_fwd_k(int k, float2 (&re)[kPos], float2 (&im)
   }
 }
 
+// Complex-lane form (the one-sample forward of single-tile circuits, RE 5):
+// a register pair is one amplitude (re, im).  Ry is real, so the same
+// packed FMAs as ry_pair apply to the pair, one per output amplitude.
+template <int K, bool COT>
+__device__ __forceinline__ void ry1_fwd(float2 (&z)[kPos], float2 p, float2 np) {
+#pragma unroll
+  for (int j = 0; j < kPos; ++j)
+    if (!(j & (1 << K))) {
+      const float2 x = z[j], y = z[j | (1 << K)];
+      if (!COT) {
+        z[j] = __ffma2_rn(np, y, x);
+        z[j | (1 << K)] = __ffma2_rn(p, x, y);
+      } else {
+        z[j] = __ffma2_rn(np, x, y);
+        z[j | (1 << K)] = __ffma2_rn(p, y, x);
+      }
+    }
+}
+
+template <bool COT>
+__device__ __forceinline__ void ry1_fwd_k(int k, float2 (&z)[kPos], float2 p, float2 np) {
+  switch (k) {
+    case 0: ry1_fwd<0, COT>(z, p, np); break;
+    case 1: ry1_fwd<1, COT>(z, p, np); break;
+    case 2: ry1_fwd<2, COT>(z, p, np); break;
+    case 3: ry1_fwd<3, COT>(z, p, np); break;
+    default: ry1_fwd<4, COT>(z, p, np); break;
+  }
+}
+
 // Applier of a register pair's 2x2 gate for rot_bwd_red: the fused SU(2)
 // with per-pair coefficients.
 template <class CF>
@@ -571,9 +601,11 @@ __host__ __device__ constexpr bool exchange8_warp_local() {
   return thr_tbit<X, V>(5) == 10 && thr_tbit<X, V>(6) == 11 && thr_tbit<Y, V>(5) == 10 && thr_tbit<Y, V>(6) == 11;
 }
 
-template <int X, int Y, int V>
+// ONE: the complex-lane form, whose state is the re array alone.
+template <int X, int Y, int V, bool ONE>
 __device__ __forceinline__ void exchange8_t(float2 (&re)[kPos], float2 (&im)[kPos], float2* ex, uint32_t tid) {
-  constexpr bool WL = exchange8_warp_local<X, Y, V>();
+  // (ONE keeps block barriers: its layouts' reads may cross warps)
+  constexpr bool WL = !ONE && exchange8_warp_local<X, Y, V>();
   const uint32_t sx = thr_slot8<X, V>(tid);
   const uint32_t sy = thr_slot8<Y, V>(tid);
   auto sync = []() {
@@ -586,6 +618,7 @@ __device__ __forceinline__ void exchange8_t(float2 (&re)[kPos], float2 (&im)[kPo
   sync();
 #pragma unroll
   for (int j = 0; j < kPos; ++j) re[j] = ex[sy + reg_slot8<Y>(j)];
+  if constexpr (ONE) return;  // the next exchange starts with a barrier
   sync();
 #pragma unroll
   for (int j = 0; j < kPos; ++j) ex[sx + reg_slot8<X>(j)] = im[j];
@@ -594,16 +627,16 @@ __device__ __forceinline__ void exchange8_t(float2 (&re)[kPos], float2 (&im)[kPo
   for (int j = 0; j < kPos; ++j) im[j] = ex[sy + reg_slot8<Y>(j)];
 }
 
-template <int V>
+template <int V, bool ONE = false>
 __device__ __forceinline__ void exchange8(int x, int y, float2 (&re)[kPos], float2 (&im)[kPos], float2* ex,
                                           uint32_t tid) {
   switch (x * 3 + y) {
-    case 1: exchange8_t<0, 1, V>(re, im, ex, tid); break;
-    case 2: exchange8_t<0, 2, V>(re, im, ex, tid); break;
-    case 3: exchange8_t<1, 0, V>(re, im, ex, tid); break;
-    case 5: exchange8_t<1, 2, V>(re, im, ex, tid); break;
-    case 6: exchange8_t<2, 0, V>(re, im, ex, tid); break;
-    default: exchange8_t<2, 1, V>(re, im, ex, tid); break;
+    case 1: exchange8_t<0, 1, V, ONE>(re, im, ex, tid); break;
+    case 2: exchange8_t<0, 2, V, ONE>(re, im, ex, tid); break;
+    case 3: exchange8_t<1, 0, V, ONE>(re, im, ex, tid); break;
+    case 5: exchange8_t<1, 2, V, ONE>(re, im, ex, tid); break;
+    case 6: exchange8_t<2, 0, V, ONE>(re, im, ex, tid); break;
+    default: exchange8_t<2, 1, V, ONE>(re, im, ex, tid); break;
   }
 }
 
@@ -737,8 +770,10 @@ enum MemOp { M_LOAD, M_STORE, M_STORE_STD, M_GEN, M_CKPT_STORE, M_CKPT_RESTORE }
 // (DevPass::tile_abit / out_abit; the identity unless the plan has three or
 // more qubit sets, in which case separate kernels convert it from and to the
 // standard order at the ends of the pass chain).  The encoding and the
-// checkpoint slots use the standard index, i.e. the qubit bits.
-template <bool BWD, bool SLOW, int P, int V, int OP>
+// checkpoint slots use the standard index, i.e. the qubit bits.  ZF: the
+// complex-lane forward (one sample per batch unit, re[j] its amplitude;
+// encoding, checkpoint and standard-order stores only).
+template <bool BWD, bool SLOW, int P, int V, int OP, bool ZF = false>
 __device__ __forceinline__ void mem_t(const PassArgs& a, const BlockCtx& bc, uint32_t tid, uint32_t base_q,
                                       uint32_t base_a, uint32_t unit_base, float2 (&re)[kPos], float2 (&im)[kPos],
                                       int slot, float rs) {
@@ -751,62 +786,117 @@ __device__ __forceinline__ void mem_t(const PassArgs& a, const BlockCtx& bc, uin
   ut += unit_base;
   const RegMaps m = reg_maps<P>(bc);
   const int n = a.n;
+  if constexpr (OP == M_GEN && !SLOW) {
+    // The product state of one batch unit (no unit bit among the register
+    // bits): the factors of the qubits outside the register bits once, then
+    // those of the register bits as a product tree over the positions.
+    const bool ok = ut < (uint32_t)a.U;
+    const float2* e = a.enc + (size_t)(ZF ? ut >> 1 : ut) * n * 2;
+    const bool hi = ZF && (ut & 1u);  // ZF: the sample's lane of the pair table
+    auto fac = [&](int q, uint32_t bit) {
+      const float2 f = __ldg(&e[2 * q + bit]);
+      return ZF ? (hi ? make_float2(f.y, f.y) : make_float2(f.x, f.x)) : f;
+    };
+    uint32_t rq = 0;
 #pragma unroll
-  for (int j = 0; j < kPos; ++j) {
-    const uint32_t i = aq | (std_index ? REG_COMBINE(m.q, j, |=) : REG_COMBINE(m.a, j, |=));
-    const uint32_t u = SLOW ? ut + REG_COMBINE(m.u, j, +=) : ut;
-    const bool ok = u < (uint32_t)a.U;
-    if constexpr (OP == M_LOAD) {
-      if (ok) {
-        re[j] = Planes<BWD>::p0(a, u)[i];
-        im[j] = Planes<BWD>::p1(a, u)[i];
+    for (int k = 0; k < kRegBits; ++k) rq |= m.q[k];
+    float2 v[kPos];
+    v[0] = ok ? make_float2(1.f, 1.f) : make_float2(0.f, 0.f);
+    if (ok)
+      for (int q = 0; q < n; ++q)
+        if (!((rq >> q) & 1u)) v[0] = __fmul2_rn(v[0], fac(q, (aq >> q) & 1u));
+#pragma unroll
+    for (int k = 0; k < kRegBits; ++k) {
+      float2 f0 = make_float2(1.f, 1.f), f1 = f0;
+      if (ok && m.q[k]) {
+        const int q = __ffs(m.q[k]) - 1;
+        f0 = fac(q, 0u);
+        f1 = fac(q, 1u);
+      }
+#pragma unroll
+      for (int j = 0; j < (1 << k); ++j) {
+        v[j | (1 << k)] = __fmul2_rn(v[j], f1);
+        v[j] = __fmul2_rn(v[j], f0);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kPos; ++j) {
+      if (ZF) {
+        re[j] = make_float2(v[j].x, 0.f);
       } else {
-        re[j] = im[j] = make_float2(0.f, 0.f);
+        re[j] = v[j];
+        im[j] = make_float2(0.f, 0.f);
       }
-    } else if constexpr (OP == M_STORE) {
-      if (ok) {
-        Planes<BWD>::p0(a, u)[i] = re[j];
-        Planes<BWD>::p1(a, u)[i] = im[j];
-      }
-    } else if constexpr (OP == M_STORE_STD) {  // forward only
-      if (ok) {
-        a.buf0[(size_t)(2 * u) * a.N + i] = make_float2(re[j].x, im[j].x);
-        if (2 * u + 1 < (uint32_t)a.B) a.buf0[(size_t)(2 * u + 1) * a.N + i] = make_float2(re[j].y, im[j].y);
-      }
-      const float2 pr = __ffma2_rn(re[j], re[j], __fmul2_rn(im[j], im[j]));  // |psi|^2 of both lanes
-      if (i & 1u) ez0 -= pr.x, ez1 -= pr.y;
-      else ez0 += pr.x, ez1 += pr.y;
-    } else if constexpr (OP == M_GEN) {  // forward only: angle-encoded product state
-      float2 v = make_float2(0.f, 0.f);
-      if (ok) {
-        const float2* e = a.enc + (size_t)u * n * 2;
-        v = make_float2(1.f, 1.f);
-        for (int q = 0; q < n; ++q) v = __fmul2_rn(v, __ldg(&e[2 * q + ((i >> q) & 1u)]));
-      }
-      re[j] = v;
-      im[j] = make_float2(0.f, 0.f);
-    } else if constexpr (OP == M_CKPT_STORE) {  // forward only
-      if (ok) {
-        const size_t e0 = ((size_t)slot * a.bmax + 2 * u) * a.N + i;
-        const bool has1 = 2 * u + 1 < (uint32_t)a.B;
-        if (a.storage == 0) {
-          float2* s = reinterpret_cast<float2*>(a.ckpt);
-          s[e0] = make_float2(re[j].x, im[j].x);
-          if (has1) s[e0 + a.N] = make_float2(re[j].y, im[j].y);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < kPos; ++j) {
+      const uint32_t i = aq | (std_index ? REG_COMBINE(m.q, j, |=) : REG_COMBINE(m.a, j, |=));
+      const uint32_t u = SLOW ? ut + REG_COMBINE(m.u, j, +=) : ut;
+      const bool ok = u < (uint32_t)a.U;
+      if constexpr (OP == M_LOAD) {
+        if (ok) {
+          re[j] = Planes<BWD>::p0(a, u)[i];
+          im[j] = Planes<BWD>::p1(a, u)[i];
         } else {
-          __nv_bfloat162* s = reinterpret_cast<__nv_bfloat162*>(a.ckpt);
-          s[e0] = __floats2bfloat162_rn(re[j].x, im[j].x);
-          if (has1) s[e0 + a.N] = __floats2bfloat162_rn(re[j].y, im[j].y);
+          re[j] = im[j] = make_float2(0.f, 0.f);
         }
-      }
-    } else {  // M_CKPT_RESTORE, backward only: psi lanes from the slot
-      if (ok) {
-        const size_t e = ((size_t)slot * a.bmax + u) * a.N + i;
-        float2 v;
-        if (a.storage == 0) v = reinterpret_cast<const float2*>(a.ckpt)[e];
-        else v = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(a.ckpt)[e]);
-        re[j].x = v.x * rs;
-        im[j].x = v.y * rs;
+      } else if constexpr (OP == M_STORE) {
+        if (ok) {
+          Planes<BWD>::p0(a, u)[i] = re[j];
+          Planes<BWD>::p1(a, u)[i] = im[j];
+        }
+      } else if constexpr (OP == M_STORE_STD && ZF) {
+        if (ok) a.buf0[(size_t)u * a.N + i] = re[j];
+        const float pr = fmaf(re[j].x, re[j].x, re[j].y * re[j].y);
+        if (i & 1u) ez0 -= pr;
+        else ez0 += pr;
+      } else if constexpr (OP == M_STORE_STD) {  // forward only
+        if (ok) {
+          a.buf0[(size_t)(2 * u) * a.N + i] = make_float2(re[j].x, im[j].x);
+          if (2 * u + 1 < (uint32_t)a.B) a.buf0[(size_t)(2 * u + 1) * a.N + i] = make_float2(re[j].y, im[j].y);
+        }
+        const float2 pr = __ffma2_rn(re[j], re[j], __fmul2_rn(im[j], im[j]));  // |psi|^2 of both lanes
+        if (i & 1u) ez0 -= pr.x, ez1 -= pr.y;
+        else ez0 += pr.x, ez1 += pr.y;
+      } else if constexpr (OP == M_GEN) {  // forward only, generic addressing: angle-encoded product state
+        float2 v = make_float2(0.f, 0.f);
+        if (ok) {
+          const float2* e = a.enc + (size_t)u * n * 2;
+          v = make_float2(1.f, 1.f);
+          for (int q = 0; q < n; ++q) v = __fmul2_rn(v, __ldg(&e[2 * q + ((i >> q) & 1u)]));
+        }
+        re[j] = v;
+        im[j] = make_float2(0.f, 0.f);
+      } else if constexpr (OP == M_CKPT_STORE && ZF) {
+        if (ok) {
+          const size_t e0 = ((size_t)slot * a.bmax + u) * a.N + i;
+          if (a.storage == 0) reinterpret_cast<float2*>(a.ckpt)[e0] = re[j];
+          else reinterpret_cast<__nv_bfloat162*>(a.ckpt)[e0] = __floats2bfloat162_rn(re[j].x, re[j].y);
+        }
+      } else if constexpr (OP == M_CKPT_STORE) {  // forward only
+        if (ok) {
+          const size_t e0 = ((size_t)slot * a.bmax + 2 * u) * a.N + i;
+          const bool has1 = 2 * u + 1 < (uint32_t)a.B;
+          if (a.storage == 0) {
+            float2* s = reinterpret_cast<float2*>(a.ckpt);
+            s[e0] = make_float2(re[j].x, im[j].x);
+            if (has1) s[e0 + a.N] = make_float2(re[j].y, im[j].y);
+          } else {
+            __nv_bfloat162* s = reinterpret_cast<__nv_bfloat162*>(a.ckpt);
+            s[e0] = __floats2bfloat162_rn(re[j].x, im[j].x);
+            if (has1) s[e0 + a.N] = __floats2bfloat162_rn(re[j].y, im[j].y);
+          }
+        }
+      } else {  // M_CKPT_RESTORE, backward only: psi lanes from the slot
+        if (ok) {
+          const size_t e = ((size_t)slot * a.bmax + u) * a.N + i;
+          float2 v;
+          if (a.storage == 0) v = reinterpret_cast<const float2*>(a.ckpt)[e];
+          else v = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(a.ckpt)[e]);
+          re[j].x = v.x * rs;
+          im[j].x = v.y * rs;
+        }
       }
     }
   }
@@ -827,21 +917,25 @@ __device__ __forceinline__ void mem_t(const PassArgs& a, const BlockCtx& bc, uin
         double s0 = 0.0, s1 = 0.0;
         for (int k = 0; k < kThreads / 32; ++k) s0 += w.ez[k][0], s1 += w.ez[k][1];
         const size_t tps = (size_t)1 << (n > kTileBits ? n - kTileBits : 0);  // tiles per sample
-        a.epart[(size_t)(2 * ut) * tps + (size_t)slot] = s0;
-        if (2 * ut + 1 < (uint32_t)a.B) a.epart[(size_t)(2 * ut + 1) * tps + (size_t)slot] = s1;
+        if (ZF) {
+          a.epart[(size_t)ut * tps + (size_t)slot] = s0;
+        } else {
+          a.epart[(size_t)(2 * ut) * tps + (size_t)slot] = s0;
+          if (2 * ut + 1 < (uint32_t)a.B) a.epart[(size_t)(2 * ut + 1) * tps + (size_t)slot] = s1;
+        }
       }
       __syncthreads();
     }
   }
 }
 
-template <bool BWD, bool SLOW, int V, int OP>
+template <bool BWD, bool SLOW, int V, int OP, bool ZF = false>
 __device__ __forceinline__ void mem_op(int phase, const PassArgs& a, const BlockCtx& bc, uint32_t tid,
                                        uint32_t base_q, uint32_t base_a, uint32_t unit_base, float2 (&re)[kPos],
                                        float2 (&im)[kPos], int slot = 0, float rs = 1.f) {
   // memory ops run in phase 0 or 1 (the planner never picks phase 2)
-  if (phase == 0) mem_t<BWD, SLOW, 0, V, OP>(a, bc, tid, base_q, base_a, unit_base, re, im, slot, rs);
-  else mem_t<BWD, SLOW, 1, V, OP>(a, bc, tid, base_q, base_a, unit_base, re, im, slot, rs);
+  if (phase == 0) mem_t<BWD, SLOW, 0, V, OP, ZF>(a, bc, tid, base_q, base_a, unit_base, re, im, slot, rs);
+  else mem_t<BWD, SLOW, 1, V, OP, ZF>(a, bc, tid, base_q, base_a, unit_base, re, im, slot, rs);
 }
 
 // Prefetch of the block's next tile: each thread copies its own positions of
@@ -1124,7 +1218,7 @@ __device__ __forceinline__ void diag_thread_t(const BlockCtx& bc, const DevPass&
   *w_out = w;
 }
 
-template <int V>
+template <int V, bool ZF = false>
 __device__ __forceinline__ void diag_op(int phase, float2 (&re)[kPos], float2 (&im)[kPos], const BlockCtx& bc,
                                         const DevPass& Pp, const PassArgs& a, const CoefRegion* C, int d, int l,
                                         uint32_t tid, uint32_t base_q, uint32_t s_o) {
@@ -1144,9 +1238,14 @@ __device__ __forceinline__ void diag_op(int phase, float2 (&re)[kPos], float2 (&
     const uint32_t sb = (w << (31 - j)) & 0x80000000u;
     const float gr = __uint_as_float(__float_as_uint(fmaf(-fi, r.y, fr * r.x)) ^ sb);
     const float gi = __uint_as_float(__float_as_uint(fmaf(fr, r.y, fi * r.x)) ^ sb);
-    const float2 xr = re[j], xi = im[j];
-    re[j] = make_float2(fmaf(gr, xr.x, -gi * xi.x), fmaf(gr, xr.y, -gi * xi.y));
-    im[j] = make_float2(fmaf(gi, xr.x, gr * xi.x), fmaf(gi, xr.y, gr * xi.y));
+    if constexpr (ZF) {  // complex-lane form: the pair is one amplitude
+      const float2 z = re[j];
+      re[j] = make_float2(fmaf(gr, z.x, -gi * z.y), fmaf(gi, z.x, gr * z.y));
+    } else {
+      const float2 xr = re[j], xi = im[j];
+      re[j] = make_float2(fmaf(gr, xr.x, -gi * xi.x), fmaf(gr, xr.y, -gi * xi.y));
+      im[j] = make_float2(fmaf(gi, xr.x, gr * xi.x), fmaf(gi, xr.y, gr * xi.y));
+    }
   }
 }
 
@@ -1258,6 +1357,9 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
   // fused CNOT layers (OP_PERM): passes loaded by tensor copies, in the
   // fused SU(2) form (RE 0) or the split form (RE 4)
   constexpr bool CNOTF = TMA && (RE == 0 || RE == 4);
+  // RE 5: the complex-lane forward of single-tile circuits (one sample per
+  // batch unit, its amplitude (re, im) in the re array; im unused)
+  constexpr bool ZF = !BWD && RE == 5;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   float4* tile = reinterpret_cast<float4*>(smem_raw);  // MODE 2: the landing buffer
   float2* ex8 = reinterpret_cast<float2*>(smem_raw + kLandBytes);  // MODE 2: the exchange buffer
@@ -1321,7 +1423,8 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
     for (int oi = 0; oi < nops; ++oi) {
       const DevOp op = OPS[oi];
       if (op.kind == OP_EXCH) {
-        if constexpr (TMA) exchange8<V>(op.a, op.b, re, im, ex8, tid);
+        if constexpr (ZF) exchange8<V, true>(op.a, op.b, re, im, reinterpret_cast<float2*>(tile), tid);
+        else if constexpr (TMA) exchange8<V>(op.a, op.b, re, im, ex8, tid);
         else exchange<V>(op.a, op.b, re, im, tile, tid);
       } else if constexpr (SPLIT) {
         if (op.kind == OP_RY) {
@@ -1333,11 +1436,16 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
               const bool cot = C->rot[slot][1].x != 0.f;
               ++slot;
               const float2 p = make_float2(f0.x, f0.y), np = make_float2(f0.z, f0.w);
-              if (cot) ry_fwd_k<true>(k, re, im, p, np);
-              else ry_fwd_k<false>(k, re, im, p, np);
+              if constexpr (ZF) {
+                if (cot) ry1_fwd_k<true>(k, re, p, np);
+                else ry1_fwd_k<false>(k, re, p, np);
+              } else {
+                if (cot) ry_fwd_k<true>(k, re, im, p, np);
+                else ry_fwd_k<false>(k, re, im, p, np);
+              }
             }
         } else if (op.kind == OP_DIAG) {
-          diag_op<V>(op.a, re, im, *bc, P, a, C, op.d, op.c, tid, base_q, s_o);
+          diag_op<V, ZF>(op.a, re, im, *bc, P, a, C, op.d, op.c, tid, base_q, s_o);
         } else if (op.kind == OP_PERM) {
           if constexpr (CNOTF)
             if (PP.perm_at[0] == 2) exchange8p<V>(op.a, op.b, re, im, ex8, tid, PP, 0, pco);
@@ -1490,7 +1598,27 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
       tile_base(P, t, &base_q, &base_a, &unit_base);
       const uint32_t s_o = bond_parity(base_q, a);
       float2 re[kPos], im[kPos];
-      if (!BWD) {
+      if (ZF) {
+        // the complex-lane form starts from the encoding and ends with the
+        // standard-order state (the host launches it for no other chain)
+        if (!a.passes[0].gen || !a.passes[a.npass - 1].last) {
+          if (tid == 0) atomicOr(a.status, kErrBounds);
+          return;
+        }
+        const DevPass& P0 = a.passes[0];
+        mem_op<false, SLOW, V, M_GEN, ZF>(P0.load_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
+        for (int pi = 0; pi < a.npass; ++pi) {
+          const DevPass& PP = a.passes[pi];
+          stage(pi);
+          run_fwd_ops(PP, stg->ops, stg->nops, &stg->coef, base_q, s_o, unit_base, re, im, false, none);
+          if (PP.ckpt >= 0)
+            mem_op<false, SLOW, V, M_CKPT_STORE, ZF>(PP.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im,
+                                                     PP.ckpt);
+        }
+        const DevPass& PL = a.passes[a.npass - 1];
+        mem_op<false, SLOW, V, M_STORE_STD, ZF>(PL.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im,
+                                                t & ((1 << PL.n_out) - 1));
+      } else if (!BWD) {
         const DevPass& P0 = a.passes[0];
         if (P0.gen) mem_op<false, SLOW, V, M_GEN>(P0.load_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
         else mem_op<false, SLOW, V, M_LOAD>(P0.load_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);

@@ -52,8 +52,10 @@ CASES = [
     (4, 2, 8, 0, "fp32"),
     (5, 7, 4, 3, "bf16"),
     (7, 4, 9, 0, "fp32"),
+    (10, 3, 9, 1, "fp32"),  # one sample per batch unit in the one-launch forward (3 tiles, not 2)
     (11, 3, 6, 1, "fp32"),
     (12, 5, 7, 2, "fp32"),
+    (12, 4, 5, 2, "bf16"),
     (13, 3, 5, 0, "fp32"),
     (14, 4, 3, 2, "fp32"),
     (16, 3, 2, 1, "bf16"),
