@@ -675,6 +675,13 @@ cudaError_t prep_coefficients(qml_ctx* c, const float* theta, cudaStream_t s) {
                            at<float>(c, c->lay.rscale), s);
 }
 
+// Kernel launches of prep_coefficients.
+int prep_launches(const qml_ctx* c) {
+  if (!use_split(c)) return 1;
+  if (c->cnot) return 4;
+  return prep_split_launches(c->cfg.n_layers, c->cfg.n_qubits, (int)c->dpass_split.size());
+}
+
 qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, float2* psi,
                        float* expect, cudaStream_t s) {
   if (c->cnot && !cnot_fused_now(c)) return run_forward_cnot(c, theta, x, B, psi, expect, s);
@@ -715,7 +722,7 @@ qml_status run_forward(qml_ctx* c, const float* theta, const float* x, int B, fl
   // partials, then one fixed-order sum per sample
   const bool epi = expect && fused_z0(c) && passes[P - 1].unit_bits == 0;
   a.epart = epi ? at<double>(c, c->lay.exp_partial) : nullptr;
-  c->launches += split ? 5 : 2;
+  c->launches += prep_launches(c) + 1;  // coefficient prep, encoding table
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, false);
   if (split && !passes[0].tma) {  // one tile holds the state: every pass in one launch
@@ -784,7 +791,7 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
   const bool reuse = c->prep_theta == theta && c->prep_gen == c->gen;
   cudaError_t e = reuse ? cudaSuccess : prep_coefficients(c, theta, s);
   if (e != cudaSuccess) return QML_ERR_CUDA;
-  if (reuse) c->launches -= split ? 4 : 1;
+  if (reuse) c->launches -= prep_launches(c);
   if (c->obs_terms.empty()) {
     e = launch_bwd_init(psi, lam, g, B, n, s);
   } else {
@@ -820,7 +827,7 @@ qml_status run_backward(qml_ctx* c, const float* theta, const float* x, int B, f
   for (int q = 0; q < kMaxQubits; ++q) a.cz_nb[q] = c->cnot ? 0u : c->nb[q], a.cz_nbhi[q] = c->cnot ? 0u : c->nbhi[q];
   a.reupload = c->reupload ? 1 : 0;
   a.dq = split ? at<float2>(c, c->lay.s_dqb) : nullptr;
-  c->launches += split ? 6 : 3;  // coefficient prep, lambda init, gradient reduce
+  c->launches += prep_launches(c) + 2;  // coefficient prep, lambda init, gradient reduce
   qml_ctx::Span sp{};
   const bool timed = span_begin(c, s, &sp, true);
   const bool one_launch = split && !passes[0].tma;  // one tile holds the state: every pass in one launch

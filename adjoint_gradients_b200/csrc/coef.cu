@@ -67,9 +67,7 @@ __global__ void prep_pass_coef_kernel(const DevPass* passes, int n_passes, const
 // it (backward), so that the last pass leaves the exact final state.
 
 template <class T>
-__global__ void split_rot_kernel(const T* theta, int total, SplitRot* out) {
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= total) return;
+__device__ void split_rot_item(const T* theta, int idx, SplitRot* out) {
   double ar, ai, br, bi;
   su2_of(theta + (size_t)idx * 3, &ar, &ai, &br, &bi);
   const double c = sqrt(ar * ar + ai * ai), s = sqrt(br * br + bi * bi);
@@ -85,16 +83,20 @@ __global__ void split_rot_kernel(const T* theta, int total, SplitRot* out) {
   out[idx] = r;
 }
 
+template <class T>
+__global__ void split_rot_kernel(const T* theta, int total, SplitRot* out) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx < total) split_rot_item(theta, idx, out);
+}
+
 // Per layer: the frame of all its rotations, and per rotation the scale of
 // the backward sums.  At the sum of rotation j the backward state is
 // rho * gam * Z^m times the split circuit's (psi, lambda), where rho is the
 // product of k2 over the layer's rotations already un-applied and gam the
 // product of g over those still applied; the sums scale by (rho gam)^2, and
 // their X and Y parts flip sign when j itself is in cotangent form.
-__global__ void split_layer_kernel(const SplitRot* rot, const int* undo, int L, int n, SplitLayer* lay,
-                                   double* gfix) {
-  const int l = blockIdx.x * blockDim.x + threadIdx.x;
-  if (l >= L) return;
+__device__ void split_layer_item(const SplitRot* rot, const int* undo, int l, int n, SplitLayer* lay,
+                                 double* gfix) {
   const SplitRot* r = rot + (size_t)l * n;
   double gam = 1.0, rho = 1.0;
   uint32_t m = 0;
@@ -119,6 +121,12 @@ __global__ void split_layer_kernel(const SplitRot* rot, const int* undo, int L, 
   }
 }
 
+__global__ void split_layer_kernel(const SplitRot* rot, const int* undo, int L, int n, SplitLayer* lay,
+                                   double* gfix) {
+  const int l = blockIdx.x * blockDim.x + threadIdx.x;
+  if (l < L) split_layer_item(rot, undo, l, n, lay, gfix);
+}
+
 // Factor of qubit q's bit b in the diagonal op after layer l (l = -1: before
 // layer 0): Rz(phi1 of layer l + phi2 of layer l + 1), times -1 on b = 1 when
 // q was rotated in cotangent form in layer l; conjugated for the backward.
@@ -133,15 +141,20 @@ __device__ __forceinline__ double2 diag_factor(const SplitRot* rot, const SplitL
   return make_double2(re, im);
 }
 
-__global__ void split_diag_kernel(const SplitRot* rot, const SplitLayer* lay, int L, int n, float2* dq_f,
-                                  float2* dq_b) {
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;  // ((l + 1) * n + q) * 2 + b
-  if (idx >= (L + 1) * n * 2) return;
+__device__ void split_diag_item(const SplitRot* rot, const SplitLayer* lay, int L, int n, int idx, float2* dq_f,
+                                float2* dq_b) {
+  // idx = ((l + 1) * n + q) * 2 + b
   const int b = idx & 1, q = (idx >> 1) % n, l = (idx >> 1) / n - 1;
   const double2 f = diag_factor(rot, lay, L, n, l, q, b, false);
   const double2 g = diag_factor(rot, lay, L, n, l, q, b, true);
   dq_f[idx] = make_float2((float)f.x, (float)f.y);
   dq_b[idx] = make_float2((float)g.x, (float)g.y);
+}
+
+__global__ void split_diag_kernel(const SplitRot* rot, const SplitLayer* lay, int L, int n, float2* dq_f,
+                                  float2* dq_b) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx < (L + 1) * n * 2) split_diag_item(rot, lay, L, n, idx, dq_f, dq_b);
 }
 
 // fp64 mode: the same factors in fp64.
@@ -173,10 +186,8 @@ __global__ void split_rscale64_kernel(const DevPass* passes, int n_passes, const
 // entries, one scale.
 constexpr int kSplitItems = kMaxSlots + kMaxDiag * kPos + 1;
 
-__global__ void split_pass_kernel(const DevPass* passes, int n_passes, const SplitRot* rot, const SplitLayer* lay,
-                                  int L, int n, CoefRegion* cf, CoefRegion* ci, float* rscale) {
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= n_passes * kSplitItems) return;
+__device__ void split_pass_item(const DevPass* passes, int idx, const SplitRot* rot, const SplitLayer* lay, int L,
+                                int n, CoefRegion* cf, CoefRegion* ci, float* rscale) {
   const int p = idx / kSplitItems, it = idx % kSplitItems;
   const DevPass& P = passes[p];
   if (it < kMaxSlots) {
@@ -226,6 +237,29 @@ __global__ void split_pass_kernel(const DevPass* passes, int n_passes, const Spl
   }
   cf[p].diag[d][j] = make_float2((float)fr, (float)fi);
   ci[p].diag[d][j] = make_float2((float)br, (float)bi);
+}
+
+__global__ void split_pass_kernel(const DevPass* passes, int n_passes, const SplitRot* rot, const SplitLayer* lay,
+                                  int L, int n, CoefRegion* cf, CoefRegion* ci, float* rscale) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx < n_passes * kSplitItems) split_pass_item(passes, idx, rot, lay, L, n, cf, ci, rscale);
+}
+
+// Small circuits: the four stages above in one block, a barrier between
+// stages that read what an earlier one wrote, one launch instead of four.
+constexpr int kPrepSmallThreads = 1024;
+constexpr int kPrepSmallItems = 4096;  // largest stage run by the one block
+
+__global__ void __launch_bounds__(kPrepSmallThreads) split_prep_small_kernel(
+    const DevPass* passes, int n_passes, const float* theta, int L, int n, const int* undo, SplitRot* rot,
+    SplitLayer* lay, double* gfix, float2* dq_f, float2* dq_b, CoefRegion* cf, CoefRegion* ci, float* rscale) {
+  const int t = threadIdx.x, T = blockDim.x;
+  for (int i = t; i < L * n; i += T) split_rot_item(theta, i, rot);
+  __syncthreads();
+  for (int l = t; l < L; l += T) split_layer_item(rot, undo, l, n, lay, gfix);
+  __syncthreads();
+  for (int i = t; i < (L + 1) * n * 2; i += T) split_diag_item(rot, lay, L, n, i, dq_f, dq_b);
+  for (int i = t; i < n_passes * kSplitItems; i += T) split_pass_item(passes, i, rot, lay, L, n, cf, ci, rscale);
 }
 
 // ---- split form of the fused CNOT schedule.  A segment (l, s) is the
@@ -365,6 +399,11 @@ cudaError_t launch_prep_split(const DevPass* passes, int n_passes, const float* 
                               const int* undo, SplitRot* rot, SplitLayer* lay, double* gfix, float2* dq_f,
                               float2* dq_b, CoefRegion* cf, CoefRegion* ci, float* rscale, cudaStream_t s) {
   const int nr = L * n;
+  if (nr <= kPrepSmallItems && (L + 1) * n * 2 <= kPrepSmallItems && n_passes * kSplitItems <= kPrepSmallItems) {
+    split_prep_small_kernel<<<1, kPrepSmallThreads, 0, s>>>(passes, n_passes, theta, L, n, undo, rot, lay, gfix, dq_f,
+                                                            dq_b, cf, ci, rscale);
+    return cudaGetLastError();
+  }
   split_rot_kernel<float><<<(nr + 127) / 128, 128, 0, s>>>(theta, nr, rot);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -376,6 +415,12 @@ cudaError_t launch_prep_split(const DevPass* passes, int n_passes, const float* 
   const int np = n_passes * kSplitItems;
   split_pass_kernel<<<(np + 127) / 128, 128, 0, s>>>(passes, n_passes, rot, lay, L, n, cf, ci, rscale);
   return cudaGetLastError();
+}
+
+int prep_split_launches(int L, int n, int n_passes) {
+  const bool small = L * n <= kPrepSmallItems && (L + 1) * n * 2 <= kPrepSmallItems &&
+                     n_passes * kSplitItems <= kPrepSmallItems;
+  return small ? 1 : 4;
 }
 
 cudaError_t launch_prep_split64(const DevPass* passes, int n_passes, const double* theta, int L, int n,

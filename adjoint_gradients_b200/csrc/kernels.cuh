@@ -128,6 +128,9 @@ cudaError_t launch_prep_pass_coef(const DevPass* passes, int n_passes, const flo
 //   dq_f / dq_b [L + 1][n][2] per-qubit diagonal factors, cf / ci [P] regions,
 //   rscale [P] (restore scale of the backward checkpoint passes).
 // undo: [L][n] qubits of each layer in the backward pass's un-apply order.
+// Kernel launches of launch_prep_split for these sizes (1: one block runs
+// every stage, for small circuits; else 4).
+int prep_split_launches(int L, int n, int n_passes);
 cudaError_t launch_prep_split(const DevPass* passes, int n_passes, const float* theta, int L, int n,
                               const int* undo, SplitRot* rot, SplitLayer* lay, double* gfix, float2* dq_f,
                               float2* dq_b, CoefRegion* cf, CoefRegion* ci, float* rscale, cudaStream_t s);
