@@ -1078,7 +1078,9 @@ __device__ __forceinline__ void load_tma_t(float2 (&re)[kPos], float2 (&im)[kPos
 
 // Backward checkpoint restore on the copied tile: replace the psi lanes of
 // this thread's positions (layout P) with the slot's values, before the tile
-// is read into registers (so no state registers are live here).
+// is read into registers (so no state registers are live here).  The 32
+// positions go in four groups of eight (register bits 3 and 4 per group), the
+// eight loads of a group in flight together.
 template <int P, int V>
 __device__ __forceinline__ void restore_tma_t(const PassArgs& a, const BlockCtx& bc, const DevPass& Pp, uint32_t tid,
                                               uint32_t base_q, uint32_t unit_base, float2* buf, int slot, float rs) {
@@ -1091,20 +1093,29 @@ __device__ __forceinline__ void restore_tma_t(const PassArgs& a, const BlockCtx&
 #pragma unroll
   for (int m = 0; m < kThrBits; ++m)
     if ((tid >> m) & 1u) s0 += (uint32_t)Pp.sstride[thr_tbit<P, V>(m)];
-  const RegMaps m = reg_maps<P>(bc);
-  const size_t e0 = ((size_t)slot * a.bmax + ut) * a.N;
-#pragma unroll 4
-  for (int j = 0; j < kPos; ++j) {
-    uint32_t off = s0;
+  uint32_t r[kRegBits];
 #pragma unroll
-    for (int k = 0; k < kRegBits; ++k)
-      if ((j >> k) & 1) off += (uint32_t)Pp.sstride[reg_tbit<P>(k)];
-    const size_t e = e0 + (aq | REG_COMBINE(m.q, j, |=));
-    float2 v;
-    if (a.storage == 0) v = reinterpret_cast<const float2*>(a.ckpt)[e];
-    else v = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(a.ckpt)[e]);
-    buf[off].x = v.x * rs;
-    buf[off + kTilePos].x = v.y * rs;
+  for (int k = 0; k < kRegBits; ++k) r[k] = (uint32_t)Pp.sstride[reg_tbit<P>(k)];
+  const RegMaps m = reg_maps<P>(bc);
+  const size_t e0 = ((size_t)slot * a.bmax + ut) * a.N + aq;
+  const bool f32 = a.storage == 0;
+#pragma unroll 1
+  for (int g = 0; g < 4; ++g) {
+    const uint32_t gq = ((g & 1) ? m.q[3] : 0u) | ((g & 2) ? m.q[4] : 0u);
+    const uint32_t go = s0 + ((g & 1) ? r[3] : 0u) + ((g & 2) ? r[4] : 0u);
+    float2 v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const size_t e = e0 + (gq | REG_COMBINE(m.q, i, |=));
+      if (f32) v[i] = reinterpret_cast<const float2*>(a.ckpt)[e];
+      else v[i] = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(a.ckpt)[e]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t off = go + REG_COMBINE(r, i, +=);
+      buf[off].x = v[i].x * rs;
+      buf[off + kTilePos].x = v[i].y * rs;
+    }
   }
 }
 
