@@ -186,8 +186,8 @@ QML_API qml_status qml_expect_z0(qml_ctx* ctx, const float* psi_dev, int B, floa
 /* Entangler for the following forward and backward calls: every layer ends
  * with CZ(bonds[2e], bonds[2e+1]) for e = 0 .. n_bonds-1 (host array of
  * n_bonds pairs of distinct qubits).  The default after qml_create is the
- * chain CZ(q, q+1), q = 0 .. n-2 ([Deep-dive] sec. 2.1 names CZ entanglers;
- * the chain is this build's reading).  CZ gates are diagonal, so any bond
+ * chain CZ(q, q+1), q = 0 .. n-2 ([Deep-dive] sec. 2.1 names CZ entanglers
+ * without a topology; the open chain is the plain reading).  CZ gates are diagonal, so any bond
  * graph (ring, all-to-all, brick, none: n_bonds = 0) runs through the same
  * fused passes; a bond listed twice cancels (CZ^2 = I).  Returns
  * QML_ERR_INVALID_ARG on a bad pair or count (the previous entangler then
