@@ -133,10 +133,21 @@ __device__ __forceinline__ void rot_fwd_k(int k, float2 (&re)[kPos], float2 (&im
 // The backward pass un-applies a tangent-form rotation with p = -t (the
 // inverse up to the scale 1 + t^2) and a cotangent-form one with the same p
 // (that matrix squares to (1 + u^2) I).
-template <bool COT>
-__device__ __forceinline__ void ry_pair(float2& xr, float2& xi, float2& yr, float2& yi, float2 p, float2 np) {
+// INPLACE (tangent form only): no copy of the old x: x <- x - t y, then
+// y <- t x' + (1 + t^2) y (= y + t x; q = (1 + t^2, 1 + t^2)); one more
+// packed product per output pair, and no register moves.  Measured faster in
+// the tensor-copy passes whose rotations are all in tangent form (the
+// flip-tracked ones), slower where the two forms mix.
+template <bool COT, bool INPLACE = false>
+__device__ __forceinline__ void ry_pair(float2& xr, float2& xi, float2& yr, float2& yi, float2 p, float2 np,
+                                        float2 q) {
   const float2 x0r = xr, x0i = xi;
-  if (!COT) {
+  if (!COT && INPLACE) {
+    xr = __ffma2_rn(np, yr, xr);
+    xi = __ffma2_rn(np, yi, xi);
+    yr = __ffma2_rn(p, xr, __fmul2_rn(q, yr));
+    yi = __ffma2_rn(p, xi, __fmul2_rn(q, yi));
+  } else if (!COT) {
     xr = __ffma2_rn(np, yr, x0r);
     xi = __ffma2_rn(np, yi, x0i);
     yr = __ffma2_rn(p, x0r, yr);
@@ -149,21 +160,22 @@ __device__ __forceinline__ void ry_pair(float2& xr, float2& xi, float2& yr, floa
   }
 }
 
-template <int K, bool COT>
-__device__ __forceinline__ void ry_fwd(float2 (&re)[kPos], float2 (&im)[kPos], float2 p, float2 np) {
+template <int K, bool COT, bool INPLACE>
+__device__ __forceinline__ void ry_fwd(float2 (&re)[kPos], float2 (&im)[kPos], float2 p, float2 np, float2 q) {
 #pragma unroll
   for (int j = 0; j < kPos; ++j)
-    if (!(j & (1 << K))) ry_pair<COT>(re[j], im[j], re[j | (1 << K)], im[j | (1 << K)], p, np);
+    if (!(j & (1 << K))) ry_pair<COT, INPLACE>(re[j], im[j], re[j | (1 << K)], im[j | (1 << K)], p, np, q);
 }
 
-template <bool COT>
+template <bool COT, bool INPLACE = false>
 __device__ __forceinline__ void ry_fwd_k(int k, float2 (&re)[kPos], float2 (&im)[kPos], float2 p, float2 np) {
+  const float2 q = INPLACE ? __ffma2_rn(p, p, make_float2(1.f, 1.f)) : make_float2(0.f, 0.f);
   switch (k) {
-    case 0: ry_fwd<0, COT>(re, im, p, np); break;
-    case 1: ry_fwd<1, COT>(re, im, p, np); break;
-    case 2: ry_fwd<2, COT>(re, im, p, np); break;
-    case 3: ry_fwd<3, COT>(re, im, p, np); break;
-    default: ry_fwd<4, COT>(re, im, p, np); break;
+    case 0: ry_fwd<0, COT, INPLACE>(re, im, p, np, q); break;
+    case 1: ry_fwd<1, COT, INPLACE>(re, im, p, np, q); break;
+    case 2: ry_fwd<2, COT, INPLACE>(re, im, p, np, q); break;
+    case 3: ry_fwd<3, COT, INPLACE>(re, im, p, np, q); break;
+    default: ry_fwd<4, COT, INPLACE>(re, im, p, np, q); break;
   }
 }
 
@@ -601,13 +613,40 @@ __host__ __device__ constexpr bool exchange8_warp_local() {
   return thr_tbit<X, V>(5) == 10 && thr_tbit<X, V>(6) == 11 && thr_tbit<Y, V>(5) == 10 && thr_tbit<Y, V>(6) == 11;
 }
 
-// ONE: the complex-lane form, whose state is the re array alone.
+// Thread-index bit of layout (Y, V) that holds tile bit t (-1: none).
+template <int Y, int V>
+__host__ __device__ constexpr int thr_index_of(int t) {
+  for (int m = 0; m < kThrBits; ++m)
+    if (thr_tbit<Y, V>(m) == t) return m;
+  return -1;
+}
+
+// Pending bit flips of layout X's register bits (fl, bit k: register bit k;
+// see the split-form rotations in pass_kernel) as thread-index bits of
+// layout Y: a register bit of phase 0 or 1 is a thread bit of the other.
+template <int X, int Y, int V>
+__device__ __forceinline__ uint32_t flip_thr(uint32_t fl) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int k = 0; k < kRegBits; ++k) {
+    const int mm = thr_index_of<Y, V>(reg_tbit<X>(k));
+    if (mm >= 0 && ((fl >> k) & 1u)) m |= 1u << mm;
+  }
+  return m;
+}
+
+// ONE: the complex-lane form, whose state is the re array alone.  fl: bit
+// flips pending on X's register bits (register j holds the amplitude of
+// position j ^ fl); the writes go to the registers' own slots, and the reads
+// take the flipped positions, whose flipped bits are thread bits in Y (phases
+// 0 and 1), so only the reading thread's slot base changes.
 template <int X, int Y, int V, bool ONE>
-__device__ __forceinline__ void exchange8_t(float2 (&re)[kPos], float2 (&im)[kPos], float2* ex, uint32_t tid) {
+__device__ __forceinline__ void exchange8_t(float2 (&re)[kPos], float2 (&im)[kPos], float2* ex, uint32_t tid,
+                                            uint32_t fl) {
   // (ONE keeps block barriers: its layouts' reads may cross warps)
   constexpr bool WL = !ONE && exchange8_warp_local<X, Y, V>();
   const uint32_t sx = thr_slot8<X, V>(tid);
-  const uint32_t sy = thr_slot8<Y, V>(tid);
+  const uint32_t sy = thr_slot8<Y, V>(tid ^ flip_thr<X, Y, V>(fl));
   auto sync = []() {
     if constexpr (WL) __syncwarp();
     else __syncthreads();
@@ -629,14 +668,14 @@ __device__ __forceinline__ void exchange8_t(float2 (&re)[kPos], float2 (&im)[kPo
 
 template <int V, bool ONE = false>
 __device__ __forceinline__ void exchange8(int x, int y, float2 (&re)[kPos], float2 (&im)[kPos], float2* ex,
-                                          uint32_t tid) {
+                                          uint32_t tid, uint32_t fl = 0) {
   switch (x * 3 + y) {
-    case 1: exchange8_t<0, 1, V, ONE>(re, im, ex, tid); break;
-    case 2: exchange8_t<0, 2, V, ONE>(re, im, ex, tid); break;
-    case 3: exchange8_t<1, 0, V, ONE>(re, im, ex, tid); break;
-    case 5: exchange8_t<1, 2, V, ONE>(re, im, ex, tid); break;
-    case 6: exchange8_t<2, 0, V, ONE>(re, im, ex, tid); break;
-    default: exchange8_t<2, 1, V, ONE>(re, im, ex, tid); break;
+    case 1: exchange8_t<0, 1, V, ONE>(re, im, ex, tid, fl); break;
+    case 2: exchange8_t<0, 2, V, ONE>(re, im, ex, tid, fl); break;
+    case 3: exchange8_t<1, 0, V, ONE>(re, im, ex, tid, fl); break;
+    case 5: exchange8_t<1, 2, V, ONE>(re, im, ex, tid, fl); break;
+    case 6: exchange8_t<2, 0, V, ONE>(re, im, ex, tid, fl); break;
+    default: exchange8_t<2, 1, V, ONE>(re, im, ex, tid, fl); break;
   }
 }
 
@@ -776,7 +815,7 @@ enum MemOp { M_LOAD, M_STORE, M_STORE_STD, M_GEN, M_CKPT_STORE, M_CKPT_RESTORE }
 template <bool BWD, bool SLOW, int P, int V, int OP, bool ZF = false>
 __device__ __forceinline__ void mem_t(const PassArgs& a, const BlockCtx& bc, uint32_t tid, uint32_t base_q,
                                       uint32_t base_a, uint32_t unit_base, float2 (&re)[kPos], float2 (&im)[kPos],
-                                      int slot, float rs) {
+                                      int slot, float rs, uint32_t fl) {
   uint32_t aq, ut;
   thread_pos<P, V>(bc, tid, &aq, &ut);
   constexpr bool std_index = !(OP == M_LOAD || OP == M_STORE || OP == M_STORE_STD);
@@ -786,6 +825,8 @@ __device__ __forceinline__ void mem_t(const PassArgs& a, const BlockCtx& bc, uin
   ut += unit_base;
   const RegMaps m = reg_maps<P>(bc);
   const int n = a.n;
+  // stores with pending flips fl: register j holds position j ^ fl
+  const uint32_t fx = fl ? (std_index ? REG_COMBINE(m.q, fl, |=) : REG_COMBINE(m.a, fl, |=)) : 0u;
   if constexpr (OP == M_GEN && !SLOW) {
     // The product state of one batch unit (no unit bit among the register
     // bits): the factors of the qubits outside the register bits once, then
@@ -831,7 +872,7 @@ __device__ __forceinline__ void mem_t(const PassArgs& a, const BlockCtx& bc, uin
   } else {
 #pragma unroll
     for (int j = 0; j < kPos; ++j) {
-      const uint32_t i = aq | (std_index ? REG_COMBINE(m.q, j, |=) : REG_COMBINE(m.a, j, |=));
+      const uint32_t i = (aq | (std_index ? REG_COMBINE(m.q, j, |=) : REG_COMBINE(m.a, j, |=))) ^ fx;
       const uint32_t u = SLOW ? ut + REG_COMBINE(m.u, j, +=) : ut;
       const bool ok = u < (uint32_t)a.U;
       if constexpr (OP == M_LOAD) {
@@ -932,10 +973,10 @@ __device__ __forceinline__ void mem_t(const PassArgs& a, const BlockCtx& bc, uin
 template <bool BWD, bool SLOW, int V, int OP, bool ZF = false>
 __device__ __forceinline__ void mem_op(int phase, const PassArgs& a, const BlockCtx& bc, uint32_t tid,
                                        uint32_t base_q, uint32_t base_a, uint32_t unit_base, float2 (&re)[kPos],
-                                       float2 (&im)[kPos], int slot = 0, float rs = 1.f) {
+                                       float2 (&im)[kPos], int slot = 0, float rs = 1.f, uint32_t fl = 0) {
   // memory ops run in phase 0 or 1 (the planner never picks phase 2)
-  if (phase == 0) mem_t<BWD, SLOW, 0, V, OP, ZF>(a, bc, tid, base_q, base_a, unit_base, re, im, slot, rs);
-  else mem_t<BWD, SLOW, 1, V, OP, ZF>(a, bc, tid, base_q, base_a, unit_base, re, im, slot, rs);
+  if (phase == 0) mem_t<BWD, SLOW, 0, V, OP, ZF>(a, bc, tid, base_q, base_a, unit_base, re, im, slot, rs, fl);
+  else mem_t<BWD, SLOW, 1, V, OP, ZF>(a, bc, tid, base_q, base_a, unit_base, re, im, slot, rs, fl);
 }
 
 // Prefetch of the block's next tile: each thread copies its own positions of
@@ -1232,7 +1273,7 @@ __device__ __forceinline__ void diag_thread_t(const BlockCtx& bc, const DevPass&
 template <int V, bool ZF = false>
 __device__ __forceinline__ void diag_op(int phase, float2 (&re)[kPos], float2 (&im)[kPos], const BlockCtx& bc,
                                         const DevPass& Pp, const PassArgs& a, const CoefRegion* C, int d, int l,
-                                        uint32_t tid, uint32_t base_q, uint32_t s_o) {
+                                        uint32_t tid, uint32_t base_q, uint32_t s_o, uint32_t fl = 0) {
   const float2* dq = a.dq + (size_t)(l + 1) * a.n * 2;
   float fr, fi;
   uint32_t w;
@@ -1241,11 +1282,19 @@ __device__ __forceinline__ void diag_op(int phase, float2 (&re)[kPos], float2 (&
     case 1: diag_thread_t<1, V>(bc, Pp, dq, l, tid, base_q, s_o, &fr, &fi, &w); break;
     default: diag_thread_t<2, V>(bc, Pp, dq, l, tid, base_q, s_o, &fr, &fi, &w); break;
   }
+  // pending flips fl: register j holds position j ^ fl, whose factor is
+  // table entry j ^ fl and whose sign is bit j ^ fl of the sign word
+  if (fl) {
+    const uint32_t pat[5] = {0xAAAAAAAAu, 0xCCCCCCCCu, 0xF0F0F0F0u, 0xFF00FF00u, 0xFFFF0000u};
+#pragma unroll
+    for (int k = 0; k < kRegBits; ++k)
+      if ((fl >> k) & 1u) w = ((w & pat[k]) >> (1 << k)) | ((w & ~pat[k]) << (1 << k));
+  }
   // per position: the factor (scalar complex, table entries from the constant
   // bank), its sign, then the product with both lanes
 #pragma unroll
   for (int j = 0; j < kPos; ++j) {
-    const float2 r = C->diag[d][j];
+    const float2 r = C->diag[d][j ^ fl];
     const uint32_t sb = (w << (31 - j)) & 0x80000000u;
     const float gr = __uint_as_float(__float_as_uint(fmaf(-fi, r.y, fr * r.x)) ^ sb);
     const float gi = __uint_as_float(__float_as_uint(fmaf(fr, r.y, fi * r.x)) ^ sb);
@@ -1371,6 +1420,16 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
   // RE 5: the complex-lane forward of single-tile circuits (one sample per
   // batch unit, its amplitude (re, im) in the re array; im unused)
   constexpr bool ZF = !BWD && RE == 5;
+  // split-form tensor-copy passes: a cotangent-form rotation [[-u, 1], [1, u]]
+  // is applied as its tangent-form factor T(-u) = [[1, u], [-u, 1]] followed
+  // by a flip X of the qubit's register bit that is not carried out: register
+  // j then holds the amplitude of position j ^ fl.  A later rotation of a
+  // flipped bit takes the negated coefficient (X T(t) X = T(-t)), its backward
+  // sums the negated y and z parts (X Y X = -Y, X Z X = -Z), a diagonal op
+  // the flipped table index and sign bit, and the next exchange or store the
+  // flipped positions; the exchange and the store end the flips.  One
+  // rotation code per register bit, and no branch on the form.
+  constexpr bool FLIP = SPLIT && TMA && RE == 3;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   float4* tile = reinterpret_cast<float4*>(smem_raw);  // MODE 2: the landing buffer
   float2* ex8 = reinterpret_cast<float2*>(smem_raw + kLandBytes);  // MODE 2: the exchange buffer
@@ -1430,13 +1489,15 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
   // coefficients; the layout is P's, the same for every pass of a launch).
   auto run_fwd_ops = [&](const DevPass& PP, const auto& OPS, int nops, const CoefRegion* C, uint32_t base_q,
                          uint32_t s_o, uint32_t unit_base,
-                         float2 (&re)[kPos], float2 (&im)[kPos], bool pf_next, auto&& prefetch_next) {
+                         float2 (&re)[kPos], float2 (&im)[kPos], bool pf_next, auto&& prefetch_next, uint32_t& fl) {
     for (int oi = 0; oi < nops; ++oi) {
       const DevOp op = OPS[oi];
       if (op.kind == OP_EXCH) {
         if constexpr (ZF) exchange8<V, true>(op.a, op.b, re, im, reinterpret_cast<float2*>(tile), tid);
+        else if constexpr (FLIP) exchange8<V>(op.a, op.b, re, im, ex8, tid, fl);
         else if constexpr (TMA) exchange8<V>(op.a, op.b, re, im, ex8, tid);
         else exchange<V>(op.a, op.b, re, im, tile, tid);
+        fl = 0;
       } else if constexpr (SPLIT) {
         if (op.kind == OP_RY) {
           int slot = op.d;
@@ -1450,13 +1511,18 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
               if constexpr (ZF) {
                 if (cot) ry1_fwd_k<true>(k, re, p, np);
                 else ry1_fwd_k<false>(k, re, p, np);
+              } else if constexpr (FLIP) {
+                // tangent form with t (tangent), -u (cotangent), negated on a flipped bit
+                const bool neg = cot != (((fl >> k) & 1u) != 0u);
+                ry_fwd_k<false, true>(k, re, im, neg ? np : p, neg ? p : np);
+                if (cot) fl ^= 1u << k;
               } else {
                 if (cot) ry_fwd_k<true>(k, re, im, p, np);
                 else ry_fwd_k<false>(k, re, im, p, np);
               }
             }
         } else if (op.kind == OP_DIAG) {
-          diag_op<V, ZF>(op.a, re, im, *bc, P, a, C, op.d, op.c, tid, base_q, s_o);
+          diag_op<V, ZF>(op.a, re, im, *bc, P, a, C, op.d, op.c, tid, base_q, s_o, fl);
         } else if (op.kind == OP_PERM) {
           if constexpr (CNOTF)
             if (PP.perm_at[0] == 2) exchange8p<V>(op.a, op.b, re, im, ex8, tid, PP, 0, pco);
@@ -1497,13 +1563,15 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
   // The ops of one pass in reverse (un-applied), with the gradient sums into acc.
   auto run_bwd_ops = [&](const DevPass& PP, const auto& OPS, int nops, const CoefRegion* C, uint32_t base_q,
                          uint32_t s_o, uint32_t unit_base,
-                         float2 (&re)[kPos], float2 (&im)[kPos], bool pf_next, auto&& prefetch_next) {
+                         float2 (&re)[kPos], float2 (&im)[kPos], bool pf_next, auto&& prefetch_next, uint32_t& fl) {
     const int pacc = PP.nslots * 3;  // row stride of the pass's sums
     for (int oi = nops - 1; oi >= 0; --oi) {
       const DevOp op = OPS[oi];
       if (op.kind == OP_EXCH) {
-        if constexpr (TMA) exchange8<V>(op.b, op.a, re, im, ex8, tid);
+        if constexpr (FLIP) exchange8<V>(op.b, op.a, re, im, ex8, tid, fl);
+        else if constexpr (TMA) exchange8<V>(op.b, op.a, re, im, ex8, tid);
         else exchange<V>(op.b, op.a, re, im, tile, tid);
+        fl = 0;
       } else if constexpr (SPLIT) {
         if (op.kind == OP_RY) {
           // the same sums, then Ry un-applied (tangent or cotangent form)
@@ -1518,8 +1586,16 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
               const bool cot = C->rot[slot][1].x != 0.f;
               const float2 p = make_float2(f0.x, f0.y), np = make_float2(f0.z, f0.w);
               v = rot_bwd_sums_k(k, re, im, pend, lane, &r);
-              if (cot) ry_fwd_k<true>(k, re, im, p, np);
-              else ry_fwd_k<false>(k, re, im, p, np);
+              if constexpr (FLIP) {
+                const bool fk = ((fl >> k) & 1u) != 0u;
+                if (fk) v.y = -v.y, v.z = -v.z;  // sums of the flipped bit's qubit
+                const bool neg = cot != fk;
+                ry_fwd_k<false, true>(k, re, im, neg ? np : p, neg ? p : np);
+                if (cot) fl ^= 1u << k;
+              } else {
+                if (cot) ry_fwd_k<true>(k, re, im, p, np);
+                else ry_fwd_k<false>(k, re, im, p, np);
+              }
               if (pslot >= 0 && (lane & 7) == 0 && lane < 24) acc[warp * pacc + pslot * 3 + (lane >> 3)] += r;
               pend = v;
               pslot = slot++;
@@ -1530,7 +1606,7 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
           }
         } else if (op.kind == OP_DIAG) {
           // the diagonal before layer 0 needs no un-applying: nothing reads the state after it
-          if (op.c >= 0) diag_op<V>(op.a, re, im, *bc, P, a, C, op.d, op.c, tid, base_q, s_o);
+          if (op.c >= 0) diag_op<V>(op.a, re, im, *bc, P, a, C, op.d, op.c, tid, base_q, s_o, fl);
         } else if (op.kind == OP_PERM) {
           if constexpr (CNOTF)
             if (PP.perm_at[1] == 2) exchange8p<V>(op.b, op.a, re, im, ex8, tid, PP, 1, pco);
@@ -1589,6 +1665,7 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
       }
     }
     auto none = []() {};
+    uint32_t nofl = 0;  // (no flips outside the tensor-copy split passes)
     // each pass's ops and coefficients are staged in shared memory before
     // the pass runs (read from global memory they would stall every op)
     MultiStage* stg = multi_stage(smem_raw);
@@ -1621,7 +1698,7 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
         for (int pi = 0; pi < a.npass; ++pi) {
           const DevPass& PP = a.passes[pi];
           stage(pi);
-          run_fwd_ops(PP, stg->ops, stg->nops, &stg->coef, base_q, s_o, unit_base, re, im, false, none);
+          run_fwd_ops(PP, stg->ops, stg->nops, &stg->coef, base_q, s_o, unit_base, re, im, false, none, nofl);
           if (PP.ckpt >= 0)
             mem_op<false, SLOW, V, M_CKPT_STORE, ZF>(PP.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im,
                                                      PP.ckpt);
@@ -1636,7 +1713,7 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
         for (int pi = 0; pi < a.npass; ++pi) {
           const DevPass& PP = a.passes[pi];
           stage(pi);
-          run_fwd_ops(PP, stg->ops, stg->nops, &stg->coef, base_q, s_o, unit_base, re, im, false, none);
+          run_fwd_ops(PP, stg->ops, stg->nops, &stg->coef, base_q, s_o, unit_base, re, im, false, none, nofl);
           if (PP.ckpt >= 0)
             mem_op<false, SLOW, V, M_CKPT_STORE>(PP.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im, PP.ckpt);
         }
@@ -1655,7 +1732,7 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
                                                   PP.ckpt, a.rscale ? __ldg(a.rscale + pi) : 1.f);
           for (int i = tid; i < kWarps * kMaxSlots * 3; i += kThreads) acc[i] = 0.f;
           stage(pi);
-          run_bwd_ops(PP, stg->ops, stg->nops, &stg->coef, base_q, s_o, unit_base, re, im, false, none);
+          run_bwd_ops(PP, stg->ops, stg->nops, &stg->coef, base_q, s_o, unit_base, re, im, false, none, nofl);
           __syncthreads();
           const int pn = PP.nslots * 3;
           float* row = a.partials + PP.partial_off + (size_t)blockIdx.x * pn;
@@ -1731,12 +1808,15 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
       } else if (have_pf) load_prefetched<V>(P.load_phase, re, im, tile, tid);
       else mem_op<false, SLOW, V, M_LOAD>(P.load_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
       if (pf_next && pf_at < 0) prefetch_next();
-      run_fwd_ops(P, P.ops, P.nops, creg, base_q, s_o, unit_base, re, im, pf_next, prefetch_next);
-      if (P.ckpt >= 0) mem_op<false, SLOW, V, M_CKPT_STORE>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im, P.ckpt);
+      uint32_t fl = 0;  // pending flips (FLIP passes)
+      run_fwd_ops(P, P.ops, P.nops, creg, base_q, s_o, unit_base, re, im, pf_next, prefetch_next, fl);
+      if (P.ckpt >= 0)
+        mem_op<false, SLOW, V, M_CKPT_STORE>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im, P.ckpt, 1.f,
+                                             fl);
       if (P.last)
         mem_op<false, SLOW, V, M_STORE_STD>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im,
-                                            t & ((1 << P.n_out) - 1));
-      else mem_op<false, SLOW, V, M_STORE>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
+                                            t & ((1 << P.n_out) - 1), 1.f, fl);
+      else mem_op<false, SLOW, V, M_STORE>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im, 0, 1.f, fl);
     } else {
       if (TMA) {
       } else if (have_pf) load_prefetched<V>(P.store_phase, re, im, tile, tid);
@@ -1744,8 +1824,9 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
       if (!TMA && P.ckpt >= 0)
         mem_op<true, SLOW, V, M_CKPT_RESTORE>(P.store_phase, a, *bc, tid, base_q, base_a, unit_base, re, im, P.ckpt, rs);
       if (pf_next && pf_at < 0) prefetch_next();
-      run_bwd_ops(P, P.ops, P.nops, creg, base_q, s_o, unit_base, re, im, pf_next, prefetch_next);
-      if (!P.gen) mem_op<true, SLOW, V, M_STORE>(P.load_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
+      uint32_t fl = 0;  // pending flips (FLIP passes)
+      run_bwd_ops(P, P.ops, P.nops, creg, base_q, s_o, unit_base, re, im, pf_next, prefetch_next, fl);
+      if (!P.gen) mem_op<true, SLOW, V, M_STORE>(P.load_phase, a, *bc, tid, base_q, base_a, unit_base, re, im, 0, 1.f, fl);
     }
     have_pf = pf_next;
   }
