@@ -704,8 +704,14 @@ __device__ __forceinline__ uint32_t thr_pattern(uint32_t tid) {
 
 template <int X, int Y, int V>
 __device__ __forceinline__ void exchange8p_t(float2 (&re)[kPos], float2 (&im)[kPos], float2* ex, uint32_t tid,
-                                             const DevPass& Pp, int dir, uint32_t co) {
-  const uint32_t sx = perm_slot(thr_pattern<X, V>(tid));
+                                             const DevPass& Pp, int dir, uint32_t co, uint32_t fl) {
+  // pending flips fl of X's register bits: register j holds position j ^ fl,
+  // written at that position's slot (perm_slot is linear: one xor)
+  uint32_t ft = 0;
+#pragma unroll
+  for (int k = 0; k < kRegBits; ++k)
+    if ((fl >> k) & 1u) ft |= 1u << reg_tbit<X>(k);
+  const uint32_t sx = perm_slot(thr_pattern<X, V>(tid)) ^ perm_slot(ft);
   uint32_t cy = co;
 #pragma unroll
   for (int m = 0; m < kThrBits; ++m)
@@ -732,17 +738,17 @@ __device__ __forceinline__ void exchange8p_t(float2 (&re)[kPos], float2 (&im)[kP
 
 template <int V>
 __device__ __forceinline__ void exchange8p(int x, int y, float2 (&re)[kPos], float2 (&im)[kPos], float2* ex,
-                                           uint32_t tid, const DevPass& Pp, int dir, uint32_t co) {
+                                           uint32_t tid, const DevPass& Pp, int dir, uint32_t co, uint32_t fl = 0) {
   switch (x * 3 + y) {
-    case 0: exchange8p_t<0, 0, V>(re, im, ex, tid, Pp, dir, co); break;
-    case 1: exchange8p_t<0, 1, V>(re, im, ex, tid, Pp, dir, co); break;
-    case 2: exchange8p_t<0, 2, V>(re, im, ex, tid, Pp, dir, co); break;
-    case 3: exchange8p_t<1, 0, V>(re, im, ex, tid, Pp, dir, co); break;
-    case 4: exchange8p_t<1, 1, V>(re, im, ex, tid, Pp, dir, co); break;
-    case 5: exchange8p_t<1, 2, V>(re, im, ex, tid, Pp, dir, co); break;
-    case 6: exchange8p_t<2, 0, V>(re, im, ex, tid, Pp, dir, co); break;
-    case 7: exchange8p_t<2, 1, V>(re, im, ex, tid, Pp, dir, co); break;
-    default: exchange8p_t<2, 2, V>(re, im, ex, tid, Pp, dir, co); break;
+    case 0: exchange8p_t<0, 0, V>(re, im, ex, tid, Pp, dir, co, fl); break;
+    case 1: exchange8p_t<0, 1, V>(re, im, ex, tid, Pp, dir, co, fl); break;
+    case 2: exchange8p_t<0, 2, V>(re, im, ex, tid, Pp, dir, co, fl); break;
+    case 3: exchange8p_t<1, 0, V>(re, im, ex, tid, Pp, dir, co, fl); break;
+    case 4: exchange8p_t<1, 1, V>(re, im, ex, tid, Pp, dir, co, fl); break;
+    case 5: exchange8p_t<1, 2, V>(re, im, ex, tid, Pp, dir, co, fl); break;
+    case 6: exchange8p_t<2, 0, V>(re, im, ex, tid, Pp, dir, co, fl); break;
+    case 7: exchange8p_t<2, 1, V>(re, im, ex, tid, Pp, dir, co, fl); break;
+    default: exchange8p_t<2, 2, V>(re, im, ex, tid, Pp, dir, co, fl); break;
   }
 }
 
@@ -1426,10 +1432,11 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
   // j then holds the amplitude of position j ^ fl.  A later rotation of a
   // flipped bit takes the negated coefficient (X T(t) X = T(-t)), its backward
   // sums the negated y and z parts (X Y X = -Y, X Z X = -Z), a diagonal op
-  // the flipped table index and sign bit, and the next exchange or store the
-  // flipped positions; the exchange and the store end the flips.  One
-  // rotation code per register bit, and no branch on the form.
-  constexpr bool FLIP = SPLIT && TMA && RE == 3;
+  // the flipped table index and sign bit, and the next exchange (plain or
+  // permuted, for the CNOT maps) or store the flipped positions, which ends
+  // the flips.  One rotation code per register bit, no branch on the form,
+  // and the tangent form updated in place.
+  constexpr bool FLIP = SPLIT && TMA && (RE == 3 || RE == 4);
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   float4* tile = reinterpret_cast<float4*>(smem_raw);  // MODE 2: the landing buffer
   float2* ex8 = reinterpret_cast<float2*>(smem_raw + kLandBytes);  // MODE 2: the exchange buffer
@@ -1525,7 +1532,10 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
           diag_op<V, ZF>(op.a, re, im, *bc, P, a, C, op.d, op.c, tid, base_q, s_o, fl);
         } else if (op.kind == OP_PERM) {
           if constexpr (CNOTF)
-            if (PP.perm_at[0] == 2) exchange8p<V>(op.a, op.b, re, im, ex8, tid, PP, 0, pco);
+            if (PP.perm_at[0] == 2) {
+              exchange8p<V>(op.a, op.b, re, im, ex8, tid, PP, 0, pco, fl);
+              fl = 0;
+            }
         }
       } else if (op.kind == OP_ROT) {
         int slot = op.d;
@@ -1609,7 +1619,10 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
           if (op.c >= 0) diag_op<V>(op.a, re, im, *bc, P, a, C, op.d, op.c, tid, base_q, s_o, fl);
         } else if (op.kind == OP_PERM) {
           if constexpr (CNOTF)
-            if (PP.perm_at[1] == 2) exchange8p<V>(op.b, op.a, re, im, ex8, tid, PP, 1, pco);
+            if (PP.perm_at[1] == 2) {
+              exchange8p<V>(op.b, op.a, re, im, ex8, tid, PP, 1, pco, fl);
+              fl = 0;
+            }
         }
       } else if (op.kind == OP_ROT) {
         // each rotation finishes the warp sum of the previous one
