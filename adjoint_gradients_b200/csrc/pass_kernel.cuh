@@ -1390,10 +1390,15 @@ __host__ __device__ constexpr size_t pass_buf_bytes(bool tma) {
 // Split passes of single-tile circuits (all passes in one launch): the ops
 // and coefficients of the running pass, staged after the block's context and
 // accumulators (the launch asks for pass_stage_bytes() more shared memory).
+// The backward's gradient rows of every pass of the launch are kept here
+// too (block-private, summed over the block's tiles) when they fit, and
+// written out once at the end.
+constexpr int kMultiRows = 2048;
 struct MultiStage {
   CoefRegion coef;
   DevOp ops[kMaxOps];
   int nops;
+  float rows[kMultiRows];
 };
 __host__ __device__ constexpr size_t multi_stage_offset() {
   return (pass_buf_bytes(false) + sizeof(BlockCtx) + (size_t)(kThreads / 32) * kMaxSlots * 3 * sizeof(float) + 15) &
@@ -1670,7 +1675,16 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
     // each tile, the state kept in registers in between.  The backward's sums
     // go to the block's row of each pass after that pass, so start the rows
     // at zero.
-    if (BWD) {
+    // (a pass's rows start at partial_off = gridDim.x x the rows of the
+    // passes before it, so partial_off / gridDim.x is its offset in the
+    // block's own rows)
+    MultiStage* stg = multi_stage(smem_raw);
+    const DevPass& PLast = a.passes[a.npass - 1];
+    const int nrows = (int)(PLast.partial_off / gridDim.x) + PLast.nslots * 3;
+    const bool srows = BWD && nrows <= kMultiRows;
+    if (srows) {
+      for (int i = tid; i < nrows; i += kThreads) stg->rows[i] = 0.f;
+    } else if (BWD) {
       for (int pi = 0; pi < a.npass; ++pi) {
         const int pn = a.passes[pi].nslots * 3;
         float* row = a.partials + a.passes[pi].partial_off + (size_t)blockIdx.x * pn;
@@ -1681,7 +1695,6 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
     uint32_t nofl = 0;  // (no flips outside the tensor-copy split passes)
     // each pass's ops and coefficients are staged in shared memory before
     // the pass runs (read from global memory they would stall every op)
-    MultiStage* stg = multi_stage(smem_raw);
     auto stage = [&](int pi) {
       __syncthreads();  // the previous pass is done with the stage
       const DevPass& PP = a.passes[pi];
@@ -1748,7 +1761,7 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
           run_bwd_ops(PP, stg->ops, stg->nops, &stg->coef, base_q, s_o, unit_base, re, im, false, none, nofl);
           __syncthreads();
           const int pn = PP.nslots * 3;
-          float* row = a.partials + PP.partial_off + (size_t)blockIdx.x * pn;
+          float* row = srows ? stg->rows + PP.partial_off / gridDim.x : a.partials + PP.partial_off + (size_t)blockIdx.x * pn;
           for (int i = tid; i < pn; i += kThreads) {
             float v = 0.f;
 #pragma unroll
@@ -1759,6 +1772,16 @@ __global__ void __launch_bounds__(kThreads, (RE >= 3 || (RE == 0 && MODE == 2)) 
         }
         // the first pass is the encoding pass: nothing reads the state after it
         if (!a.passes[0].gen) mem_op<true, SLOW, V, M_STORE>(a.passes[0].load_phase, a, *bc, tid, base_q, base_a, unit_base, re, im);
+      }
+    }
+    if (srows) {  // the block's rows, summed over its tiles, written once
+      __syncthreads();
+      for (int pi = 0; pi < a.npass; ++pi) {
+        const DevPass& PP = a.passes[pi];
+        const int pn = PP.nslots * 3;
+        const float* src = stg->rows + PP.partial_off / gridDim.x;
+        float* row = a.partials + PP.partial_off + (size_t)blockIdx.x * pn;
+        for (int i = tid; i < pn; i += kThreads) row[i] = src[i];
       }
     }
     return;
